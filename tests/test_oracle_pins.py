@@ -1,0 +1,308 @@
+"""Pins for the oracle: hand-worked examples from the pages, closed forms,
+invariants, brute force and special cases.  None of these re-types the
+oracle's own formula; each would fail on a dropped term, a wrong sign, a
+wrong index or a transposed operand somewhere in the oracle.
+
+CPU only (no GPU marker)."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from ternary_weight_linear_fwd_b200 import synth
+
+
+def _ints(tok):
+    return np.array([int(t) for t in tok], dtype=np.int64)
+
+
+def _floats(tok):
+    return np.array([float(t) for t in tok], dtype=np.float32)
+
+
+# ---------------------------------------------------------------- worked examples
+
+def test_tl2_worked_example_acc(golden):
+    g = golden("tl2_worked_example.txt")
+    w = _ints(g["weights"][0]).astype(np.int8)
+    q = _ints(g["q"][0]).astype(np.int8)
+    acc = oracle.matmul_i32(q[None, :], w[None, :])
+    assert int(acc[0, 0]) == int(g["acc"][0][0])
+
+
+def test_tl2_lookup_identity(golden):
+    """The 9-entry pair table of the TL2 scheme gives the same dot product as
+    the direct sum, for every pair code and for the page's weight vector."""
+    g = golden("tl2_worked_example.txt")
+    w = _ints(g["weights"][0])
+    idx = [(w[i] + 1) * 3 + (w[i + 1] + 1) for i in range(0, 8, 2)]
+    assert idx == [int(t) for t in g["tl2_pair_index"][0]]
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        a = rng.integers(-127, 128, size=8)
+        lut_sum = 0
+        for i in range(0, 8, 2):
+            a0, a1 = a[i], a[i + 1]
+            lut = [-(a0 + a1), -a0, -a0 + a1, -a1, 0, a1, a0 - a1, a0, a0 + a1]
+            lut_sum += lut[idx[i // 2]]
+        acc = oracle.matmul_i32(a.astype(np.int8)[None, :], w.astype(np.int8)[None, :])
+        assert int(acc[0, 0]) == int(lut_sum)
+
+
+def test_i2s_packed_bytes(golden):
+    g = golden("tl2_worked_example.txt")
+    w = _ints(g["weights"][0]).astype(np.int8)[None, :]
+    expect = np.array([int(t, 16) for t in g["packed_row_hex"][0]], dtype=np.uint8)
+    got = oracle.pack_dense(w)
+    assert got.shape == (1, 16)
+    np.testing.assert_array_equal(got[0], expect)
+    np.testing.assert_array_equal(oracle.unpack_dense(got, 1, 8), w)
+
+
+def test_quant_act_hand(golden):
+    g = golden("quant_act_hand.txt")
+    x = synth.to_bf16_bits(_floats(g["x"][0]))[None, :]
+    for key, qb in (("q_qb127", 127), ("q_qb128", 128)):
+        q, gam, rs = oracle.quant_act(x, qb)
+        np.testing.assert_array_equal(q[0], _ints(g[key][0]))
+        assert float(gam[0]) == float(g["gamma"][0][0])
+        assert int(rs[0]) == int(_ints(g[key][0]).sum())
+
+
+def test_dequant_hand(golden):
+    for acc, alpha, gamma, hexbits in golden("dequant_hand.txt")["case"]:
+        y = oracle.dequant(np.array([[int(acc)]], np.int32), np.array([float(gamma)], np.float32),
+                           np.float32(float(alpha)))
+        assert int(y[0, 0]) == int(hexbits, 16), (acc, alpha, gamma)
+
+
+def test_ternarize_hand(golden):
+    g = golden("ternarize_hand.txt")
+    W = _floats(g["W"][0])[None, :]
+    a = oracle.absmean(W)
+    assert a == np.float32(float(g["alpha"][0][0]))
+    np.testing.assert_array_equal(oracle.ternarize(W, a)[0], _ints(g["Wt"][0]))
+
+
+def test_nm_mask_hand(golden):
+    g = golden("nm_mask_hand.txt")
+    cases = (("w24", "keep24", "meta24", 2, 4), ("w68", "keep68", "meta68", 6, 8),
+             ("w68tie", "keep68tie", "meta68tie", 6, 8))
+    for wk, kk, mk, n, m in cases:
+        W = _floats(g[wk][0])[None, :]
+        mask = oracle.nm_mask(W, n, m)
+        np.testing.assert_array_equal(mask[0], _ints(g[kk][0]))
+        Wt = oracle.ternarize(W, oracle.absmean(W))
+        _, meta = oracle.pack_nm(oracle.apply_mask(Wt, mask), mask, n, m)
+        assert int(meta[0, 0]) == int(g[mk][0][0])
+
+
+# ---------------------------------------------------------------- special cases
+
+def test_ternarize_ties_round_half_to_even():
+    """r = W / RN(alpha + eps) exactly +-0.5 rounds to 0 and +-1.5 to +-2 -> clamp +-1;
+    the next float above 0.5 gives +-1.  d is formed by an independent fp32 add."""
+    alpha = np.float32(0.75) - np.float32(1e-5)
+    d = np.float32(alpha + np.float32(1e-5))
+    half = np.float32(d * np.float32(0.5))  # exact: scaling by a power of two
+    assert np.float32(half / d) == np.float32(0.5)
+    above = np.nextafter(half, np.float32(1))
+    W = np.array([[half, -half, np.float32(3) * half, -np.float32(3) * half, above, -above, 0.0, -0.0]],
+                 dtype=np.float32)
+    got = oracle.ternarize(W, alpha)[0]
+    np.testing.assert_array_equal(got, [0, 0, 1, -1, 1, -1, 0, 0])
+
+
+def test_bf16_rounding_matches_independent_fp32_path():
+    """For values exactly representable in fp32, rounding from fp64 to bf16 must
+    agree with numpy's fp32 -> bf16 bit rounding (an independent implementation)."""
+    rng = np.random.default_rng(1)
+    v = np.concatenate([rng.standard_normal(2000) * 10 ** rng.uniform(-30, 30, 2000),
+                        [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 2 ** -130, 2 ** -133 * 1.5]])
+    v32 = v.astype(np.float32)
+    ref = synth.to_bf16_bits(v32)
+    got = np.array([oracle.bf16_from_f64(float(x)) for x in v32], dtype=np.uint16)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_zero_input_gives_zero():
+    x = np.zeros((3, 64), np.uint16)
+    W = synth.latent_weights(16, 64, seed=7)
+    p = oracle.pack_weights(W)
+    y, acc, q, g, rs = oracle.forward(x, p["Wt"], p["alpha"])
+    assert not q.any() and not acc.any() and not g.any() and not rs.any()
+    assert not y.any()
+
+
+def test_argmax_maps_to_127():
+    x = synth.activations(16, 512, seed=3)
+    q, g, _ = oracle.quant_act(x)
+    xf = synth.bf16_bits_to_f32(x)
+    am = np.abs(xf).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(16), am]) == 127)
+    assert np.all(np.abs(q.astype(np.int32)) <= 127)
+    assert np.all(g == np.abs(xf).max(axis=1))
+
+
+def test_hand_2x8_closed_form():
+    """x = +-c with c >> eps gives q = +-127 exactly (127c/(c+1e-5) > 126.5 for
+    c > 2.54e-3), so acc is 127 times a signed count and y = acc * alpha * c / 127."""
+    c = 0.75
+    signs = np.array([[1, -1, 1, 1, -1, -1, 1, -1], [-1, -1, -1, 1, 1, 1, 1, 1]])
+    x = synth.to_bf16_bits((signs * c).astype(np.float32))
+    Wt = np.array([[1, 0, -1, 1, 0, 0, -1, 1], [0, 0, 0, 0, 0, 0, 0, 0], [1, 1, 1, 1, 1, 1, 1, 1]],
+                  dtype=np.int8)
+    alpha = np.float32(0.5)
+    y, acc, q, g, _ = oracle.forward(x, Wt, alpha)
+    np.testing.assert_array_equal(q, 127 * signs)
+    expect_acc = 127 * (signs @ Wt.T.astype(np.int64))
+    np.testing.assert_array_equal(acc, expect_acc)
+    for i in range(2):
+        for j in range(3):
+            assert y[i, j] == oracle.bf16_from_f64(expect_acc[i, j] * 0.5 * c / 127)
+
+
+def test_qb128_reading_clamps():
+    x = synth.activations(4, 256, seed=11)
+    q, _, _ = oracle.quant_act(x, 128)
+    assert q.min() >= -128 and q.max() <= 127
+    assert (np.abs(q.astype(np.int32)) >= 127).sum() >= 4
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_absmean_constant_magnitude_exact():
+    W = (np.where(synth.uniform(5, 9, 4096) < 0.5, -1.0, 1.0) * 0.037).astype(np.float32).reshape(64, 64)
+    assert oracle.absmean(W) == np.float32(0.037)
+
+
+def test_absmean_and_zero_fraction_closed_form():
+    """For W ~ N(0, s): alpha -> s*sqrt(2/pi) and P(W_t = 0) -> 2*Phi(0.5*sqrt(2/pi)) - 1 = 0.3101."""
+    N, K, s = 512, 256, 0.02
+    W = synth.latent_weights(N, K, seed=0)
+    a = float(oracle.absmean(W))
+    mu = s * math.sqrt(2 / math.pi)
+    se = s * math.sqrt(1 - 2 / math.pi) / math.sqrt(N * K)
+    assert abs(a - mu) < 5 * se
+    Wt = oracle.ternarize(W, a)
+    p0 = (Wt == 0).mean()
+    z = 0.5 * (a + 1e-5) / s
+    expect = math.erf(z / math.sqrt(2))  # = 2*Phi(z) - 1
+    assert abs(expect - 0.3101) < 0.002
+    assert abs(p0 - expect) < 4 * math.sqrt(expect * (1 - expect) / (N * K))
+    assert set(np.unique(Wt).tolist()) <= {-1, 0, 1}
+
+
+def test_pack_recovers_scaled_ternary():
+    """W = c * T (T drawn with P(0) = 0.42) has alpha = c * (1 - p0_emp); every nonzero
+    scales to +-1/(1 - p0) > 1.5 and therefore ternarises back to T exactly."""
+    T = synth.ternary_weights(96, 512, seed=1)
+    c = np.float32(0.03125)
+    W = (T.astype(np.float32) * c)
+    p = oracle.pack_weights(W)
+    np.testing.assert_array_equal(p["Wt"], T)
+    frac_nz = (T != 0).mean()
+    assert abs(float(p["alpha"]) - float(c) * frac_nz) < 1e-7
+    assert abs((T == 0).mean() - 0.42) < 4 * math.sqrt(0.42 * 0.58 / T.size)
+
+
+# ---------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("N,K", [(512, 256), (33, 200), (7, 3)])
+def test_dense_pack_roundtrip_and_codes(N, K):
+    W = synth.latent_weights(N, K, seed=N + K)
+    p = oracle.pack_weights(W)
+    codes = p["codes"]
+    assert codes.shape == (N, 16 * ((K + 63) // 64))
+    np.testing.assert_array_equal(oracle.unpack_dense(codes, N, K), p["Wt"])
+    c = np.stack([(codes >> s) & 3 for s in (0, 2, 4, 6)], axis=-1).reshape(N, -1)
+    assert not (c == 3).any()
+    assert np.all(c[:, K:] == 1)  # padding positions hold the zero code
+    np.testing.assert_array_equal(c[:, :K].astype(np.int8) - 1, p["Wt"])
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (7, 8), (5, 8), (3, 8), (2, 8), (1, 8)])
+def test_nm_mask_is_topn_and_roundtrips(n, m):
+    N, K = 40, 256
+    W = synth.latent_weights(N, K, seed=5)
+    W[3, :16] = 0.01  # tie-heavy blocks
+    W[4, :8] = -0.0
+    mask = oracle.nm_mask(W, n, m)
+    blocks = mask.reshape(N, K // m, m)
+    assert np.all(blocks.sum(-1) == n)
+    # brute force: a stable library sort of -|W| inside each block
+    mag = np.abs(W.reshape(N, K // m, m)).astype(np.float64)
+    order = np.argsort(-mag, axis=-1, kind="stable")
+    ref = np.zeros_like(blocks)
+    np.put_along_axis(ref, order[..., :n], 1, axis=-1)
+    np.testing.assert_array_equal(blocks, ref)
+    p = oracle.pack_weights(W, n, m)
+    assert p["alpha"] == oracle.absmean(W)  # alpha from the dense latent matrix
+    dense_t = oracle.ternarize(W, oracle.absmean(W))
+    np.testing.assert_array_equal(p["Wt"], dense_t * mask)  # quant, then mask
+    back = oracle.unpack_nm(p["values"], p["meta"], N, K, n, m)
+    np.testing.assert_array_equal(back, p["Wt"])
+    assert p["values"].shape[1] == 16 * ((K * n // m + 63) // 64)
+
+
+def test_nm_rejects_bad_pattern():
+    W = synth.latent_weights(4, 64, seed=1)
+    with pytest.raises(ValueError):
+        oracle.pack_nm(np.zeros((4, 64), np.int8), np.ones((4, 64), np.uint8), 3, 4)
+
+
+# ---------------------------------------------------------------- brute force
+
+def test_matmul_matches_float64_library_matmul():
+    x = synth.activations(8, 256, seed=0)
+    W = synth.latent_weights(512, 256, seed=0)
+    p = oracle.pack_weights(W)
+    q, _, _ = oracle.quant_act(x)
+    acc = oracle.matmul_i32(q, p["Wt"])
+    ref = q.astype(np.float64) @ p["Wt"].astype(np.float64).T
+    np.testing.assert_array_equal(acc, ref.astype(np.int64))
+
+
+def test_forward_within_quantisation_error_bound():
+    """|y - x . (alpha W_t)| <= alpha/127 * (|acc| (d - gamma) + d * 0.50001 * sum|W_t|) + |y| 2^-8,
+    d = RN(gamma + eps): the codes are within half a step of 127 x / d, and y is rounded to bf16."""
+    M, K, N = 8, 256, 512
+    x = synth.activations(M, K, seed=0)
+    W = synth.latent_weights(N, K, seed=0)
+    p = oracle.pack_weights(W)
+    y, acc, q, g, _ = oracle.forward(x, p["Wt"], p["alpha"])
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    a = float(p["alpha"])
+    ref = xf @ (a * p["Wt"].astype(np.float64)).T
+    yf = synth.bf16_bits_to_f32(y).astype(np.float64)
+    d = (g.astype(np.float32) + np.float32(1e-5)).astype(np.float64)
+    l1 = np.abs(p["Wt"]).sum(axis=1).astype(np.float64)
+    bound = a / 127 * (np.abs(acc) * (d - g)[:, None] + d[:, None] * 0.50001 * l1[None, :]) \
+        + np.abs(yf) * 2.0 ** -8 + 1e-12
+    assert np.all(np.abs(yf - ref) <= bound)
+    # the bound sits below the signal, and the typical error is far smaller still
+    assert np.median(bound) < np.median(np.abs(ref))
+    assert np.sqrt(np.mean((yf - ref) ** 2)) < 0.05 * np.sqrt(np.mean(ref ** 2))
+
+
+def test_third_restatement_torch_cpu():
+    """The blog's PyTorch BitLinear_b158 formulas (Qb = 127) in torch CPU fp32."""
+    torch = pytest.importorskip("torch")
+    M, K, N = 8, 256, 512
+    x = synth.activations(M, K, seed=0)
+    W = synth.latent_weights(N, K, seed=0)
+    p = oracle.pack_weights(W)
+    wt = torch.from_numpy(W)
+    wq = torch.clamp(torch.round(wt / (torch.tensor(float(p["alpha"]), dtype=torch.float32) + 1e-5)), -1, 1)
+    np.testing.assert_array_equal(wq.numpy().astype(np.int8), p["Wt"])
+    xt = torch.from_numpy(synth.bf16_bits_to_f32(x).copy())
+    gam = xt.abs().max(dim=-1, keepdim=True).values
+    xq = torch.clamp(torch.round(xt * 127 / (gam + 1e-5)), -128, 127)
+    q, g, _ = oracle.quant_act(x)
+    np.testing.assert_array_equal(xq.numpy().astype(np.int8), q)
+    out = torch.nn.functional.linear(xq.double(), wq.double()) * (float(p["alpha"]) * gam.double()) / 127
+    ref = out.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    y, *_ = oracle.forward(x, p["Wt"], p["alpha"])
+    diff = np.abs(y.astype(np.int32) - ref.astype(np.int32))
+    assert diff.max() <= 1
