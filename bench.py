@@ -1,0 +1,508 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 BitLinear forward (ternary weights x int8 activations).
+
+Headline (one JSON line on rank 0): decode weight GB/s of the BitNet b1.58
+2B4T feed-forward BitLinears at M = 1 token -- per step one token passes the
+gate (2560 -> 6912), up (2560 -> 6912) and down (6912 -> 2560) projections of
+every one of the 30 layers of a 2B4T-shaped stack (90 GEMV launches, 398 MB of
+2-bit weights, larger than the 126 MB L2, so every step streams its weights
+from HBM).  Weights are drawn directly in ternary form (P(0) = 0.42,
+P(+-1) = 0.29, alpha ~ U(0.01, 0.05)); x ~ N(0, 1) in bf16.  The step is
+captured once in a CUDA graph with programmatic dependent launch between the
+GEMVs.  Bytes per GEMV = N*K/4 packed codes + 4 (alpha) + 2K (x) + 2N (y).
+
+A second object, "prefill", reports int8 TOPS of the tensor-core path on the
+2B4T prefill shapes (M = 2048 tokens; 2560 -> 6912, 6912 -> 2560,
+2560 -> 2560, 2560 -> 640; latent W ~ N(0, 0.02), x with 1% x10 outliers),
+L2 flushed between iterations, counted as 2*M*N*K ops.
+
+--impl reference times the oracle (plain C, one host core) on the same
+workload and metric.  Multi-GPU (torchrun) runs independent replicas: the
+path has no exchange step, per-GPU work is fixed, the time is the max over
+ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode weight GB/s (% HBM peak); prefill int8 TOPS (% tensor peak)"
+LAYERS = 30
+FFN = (("gate", 2560, 6912), ("up", 2560, 6912), ("down", 6912, 2560))  # (name, K, N)
+PREFILL_SHAPES = ((2560, 6912), (6912, 2560), (2560, 2560), (2560, 640))  # (K, N)
+PREFILL_M = 2048
+DISTINCT_LAYERS = 2  # distinct weight draws, replicated to 30 layers at distinct addresses
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_m1_dense__decode_2b4t_ffn.md")
+GEMV_SOURCES = ("gemv.cuh", "quant_pack.cuh", "ptx.cuh")
+
+
+def decode_bytes_per_gemv(K: int, N: int) -> int:
+    return N * K // 4 + 4 + 2 * K + 2 * N
+
+
+def decode_step_bytes(layers: int = LAYERS) -> int:
+    return layers * sum(decode_bytes_per_gemv(K, N) for _, K, N in FFN)
+
+
+# ------------------------------------------------------------------ multi-rank plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(units_per_rank_step: float, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_rank_step * steps * world / max_seconds
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Polls SM clock, max clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.002, pci_bus_id: str = None):
+        self.index, self.period, self.bus = index, period_s, pci_bus_id
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            if self.bus:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(self.bus.encode())
+            else:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ peaks, profile
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def gemv_source_hash() -> str:
+    h = hashlib.sha256()
+    for n in GEMV_SOURCES:
+        with open(os.path.join(ROOT, "ternary_weight_linear_fwd_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per GEMV launch from the committed ncu summary, if it matches today's kernel source."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    vals = {}
+    with open(PROFILE_SUMMARY) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, _, v = line[2:].partition(":")
+                vals[k.strip()] = v.strip().strip("`")
+    try:
+        if vals.get("source_sha256_16") != gemv_source_hash():
+            return None
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ workloads (ours)
+
+def build_decode(dev, layers: int, seed: int = 1):
+    """Packed weights of `layers` FFN layers (distinct addresses), inputs and outputs."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    distinct = []
+    for d in range(DISTINCT_LAYERS):
+        mats = {}
+        for j, (name, K, N) in enumerate(FFN):
+            s = seed + 100 * d + j
+            T = torch.from_numpy(synth.ternary_weights(N, K, seed=s)).to(dev)
+            mats[name] = bl.pack_ternary(T, float(synth.alpha_uniform(s)))
+            del T
+        distinct.append(mats)
+    layers_w = []
+    for l in range(layers):
+        src = distinct[l % DISTINCT_LAYERS]
+        cp = {}
+        for name, K, N in FFN:
+            w = src[name]
+            cp[name] = bl.PackedWeights(w.N, w.K, 0, 0, w.codes.clone(), None, w.alpha.clone())
+        layers_w.append(cp)
+    del distinct
+    x_in = torch.from_numpy(synth.activations(layers, 2560, seed=seed, outlier_p=0.0).view(np.int16)).to(dev)
+    h_in = torch.from_numpy(synth.activations(layers, 6912, seed=seed + 1, outlier_p=0.0).view(np.int16)).to(dev)
+    x_in = x_in.view(torch.bfloat16)
+    h_in = h_in.view(torch.bfloat16)
+    y_gate = torch.empty((layers, 6912), dtype=torch.bfloat16, device=dev)
+    y_up = torch.empty_like(y_gate)
+    y_down = torch.empty((layers, 2560), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize(dev)
+    return layers_w, x_in, h_in, y_gate, y_up, y_down
+
+
+def decode_step_fn(layers_w, x_in, h_in, y_gate, y_up, y_down, flags):
+    import ternary_weight_linear_fwd_b200 as bl
+
+    def step():
+        for l, w in enumerate(layers_w):
+            xv = x_in[l:l + 1]
+            bl.forward(w["gate"], xv, out=y_gate[l:l + 1], flags=flags)
+            bl.forward(w["up"], xv, out=y_up[l:l + 1], flags=flags)
+            bl.forward(w["down"], h_in[l:l + 1], out=y_down[l:l + 1], flags=flags)
+    return step
+
+
+def time_graph(graph, steps: int, warmup: int, dev, clock_index: int):
+    import torch
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    s = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p = torch.cuda.get_device_properties(dev)
+    bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    with ClockSampler(clock_index, pci_bus_id=bus) as clk:
+        torch.cuda.synchronize(dev)
+        e0.record(s)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(s)
+        e1.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    return e0.elapsed_time(e1) / 1e3, clk.summary()
+
+
+def run_decode(dev, steps, warmup, layers, clock_index):
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+
+    buf = build_decode(dev, layers)
+    layers_w, x_in, h_in, y_gate, y_up, y_down = buf
+    step = decode_step_fn(*buf, flags=bl.FLAG_PDL)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()  # warm the library (attributes, module load) outside capture
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    launches_per_step = 3 * layers
+    secs, clocks = time_graph(g, steps, warmup, dev, clock_index)
+    assert bl.device_status() == 0
+
+    # end to end: pinned host inputs -> device, the captured public-API step, outputs -> host
+    h_x = torch.empty(x_in.shape, dtype=x_in.dtype, pin_memory=True).copy_(x_in.cpu())
+    h_h = torch.empty(h_in.shape, dtype=h_in.dtype, pin_memory=True).copy_(h_in.cpu())
+    o_g = torch.empty(y_gate.shape, dtype=y_gate.dtype, pin_memory=True)
+    o_u = torch.empty_like(o_g, pin_memory=True)
+    o_d = torch.empty(y_down.shape, dtype=y_down.dtype, pin_memory=True)
+    s = torch.cuda.current_stream(dev)
+
+    def e2e_step():
+        x_in.copy_(h_x, non_blocking=True)
+        h_in.copy_(h_h, non_blocking=True)
+        g.replay()
+        o_g.copy_(y_gate, non_blocking=True)
+        o_u.copy_(y_up, non_blocking=True)
+        o_d.copy_(y_down, non_blocking=True)
+
+    for _ in range(max(3, warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, min(steps, 2000))
+    e0.record(s)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(s)
+    e1.synchronize()
+    e2e_secs = e0.elapsed_time(e1) / 1e3
+    barrier(dev)
+    h2d = (x_in.numel() + h_in.numel()) * 2
+    d2h = (y_gate.numel() + y_up.numel() + y_down.numel()) * 2
+    del g
+    return {"secs": secs, "clocks": clocks, "launches_per_step": launches_per_step, "e2e_secs": e2e_secs,
+            "e2e_steps": e_steps, "h2d": h2d, "d2h": d2h}
+
+
+def run_prefill(dev, iters: int, warmup: int):
+    """Per shape: forward at M = 2048 with an L2 flush before each timed call."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    x = torch.from_numpy(synth.activations(PREFILL_M, 6912, seed=3).view(np.int16)).to(dev).view(torch.bfloat16)
+    out = {}
+    tot_ops, tot_sec = 0.0, 0.0
+    s = torch.cuda.current_stream(dev)
+    kernel = None
+    for K, N in PREFILL_SHAPES:
+        W = torch.from_numpy(synth.latent_weights(N, K, seed=3)).to(dev)
+        w = bl.pack_weights(W)
+        del W
+        xk = x[:, :K].contiguous()
+        y = torch.empty((PREFILL_M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(bl.forward_workspace_bytes(PREFILL_M, N, K), dtype=torch.uint8, device=dev)
+        for _ in range(warmup):
+            bl.forward(w, xk, out=y, workspace=ws)
+        kernel = bl.last_kernel()
+        times = []
+        for _ in range(iters):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            bl.forward(w, xk, out=y, workspace=ws)
+            e1.record(s)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1) / 1e3)
+        med = statistics.median(times)
+        ops = 2.0 * PREFILL_M * N * K
+        out[f"{K}x{N}"] = {"ms": med * 1e3, "tops": ops / med / 1e12}
+        tot_ops += ops
+        tot_sec += med
+    assert bl.device_status() == 0
+    return {"shapes": out, "tops": tot_ops / tot_sec / 1e12, "kernel": kernel, "ops": tot_ops, "secs": tot_sec}
+
+
+# ------------------------------------------------------------------ oracle (CPU) legs
+
+def oracle_decode_setup(seed: int = 1):
+    from ternary_weight_linear_fwd_b200 import synth
+    mats = []
+    for j, (name, K, N) in enumerate(FFN):
+        mats.append((synth.ternary_weights(N, K, seed=seed + j), synth.alpha_uniform(seed + j), K, N))
+    x = synth.activations(1, 2560, seed=seed, outlier_p=0.0)
+    h = synth.activations(1, 6912, seed=seed + 1, outlier_p=0.0)
+    return mats, x, h
+
+
+def oracle_decode_pass(setup, frac: float = 1.0):
+    """Oracle forward (quantise, contract, dequantise) of one FFN layer at M = 1, on the first
+    `frac` of each matrix's output rows.  Returns (algorithmic bytes, seconds)."""
+    import oracle
+    mats, x, h = setup
+    nbytes, t0 = 0, time.perf_counter()
+    for T, a, K, N in mats:
+        rows = max(1, int(round(N * frac)))
+        oracle.forward(x if K == 2560 else h, T[:rows], a)
+        nbytes += decode_bytes_per_gemv(K, rows)
+    return nbytes, time.perf_counter() - t0
+
+
+def oracle_decode_sample(seconds: float, seed: int = 1):
+    """Repeats full-layer oracle passes until `seconds` pass; returns (GB/s, passes, seconds)."""
+    setup = oracle_decode_setup(seed)
+    n, tot_b, tot_s = 0, 0, 0.0
+    while tot_s < seconds:
+        b, sec = oracle_decode_pass(setup)
+        n, tot_b, tot_s = n + 1, tot_b + b, tot_s + sec
+    return tot_b / tot_s / 1e9, n, tot_s
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--prefill-iters", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps")
+
+    world, rank, local = dist_env()
+    config = {"workload": f"decode GEMV, BitNet-2B4T FFN (gate/up 2560->6912, down 6912->2560) x {args.layers} "
+                          f"layers, M=1, ternary P(0)=0.42",
+              "M": 1, "layers": args.layers, "gemv_per_step": 3 * args.layers,
+              "bytes_per_step": decode_step_bytes(args.layers), "l2": "weights per step exceed L2 (no reuse)",
+              "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        setup = oracle_decode_setup()
+        full_b, full_s = oracle_decode_pass(setup)
+        # a bounded sample per step: the whole run stays near two minutes of host time
+        frac = min(1.0, (120.0 / (args.steps + args.warmup)) / full_s)
+        for _ in range(args.warmup):
+            oracle_decode_pass(setup, frac)
+        tot_b, tot_s, vals = 0, 0.0, []
+        for _ in range(args.steps):
+            b, sec = oracle_decode_pass(setup, frac)
+            tot_b, tot_s = tot_b + b, tot_s + sec
+            vals.append(b / sec / 1e9)
+        v = tot_b / tot_s / 1e9
+        sample = (f"oracle forward (plain C, 1 thread): per step one FFN layer (gate, up, down at M=1) "
+                  f"restricted to the first {frac:.4f} of each matrix's output rows; GB/s on the same "
+                  f"algorithmic bytes (packed codes + alpha + x + y)")
+        line = {"metric": METRIC, "impl": "reference", "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "int8 x ternary -> int32 (bf16 in/out)", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+                "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    from ternary_weight_linear_fwd_b200 import build as blbuild
+    blbuild.build()
+    import ternary_weight_linear_fwd_b200 as bl
+    bl.lib()
+
+    dec = run_decode(dev, args.steps, args.warmup, args.layers, clock_index=local)
+    max_secs = reduce_max(dec["secs"], dev)
+    max_e2e = reduce_max(dec["e2e_secs"], dev)
+    step_bytes = decode_step_bytes(args.layers)
+    value = aggregate(step_bytes, args.steps, world, max_secs) / 1e9
+    e2e_value = aggregate(step_bytes, dec["e2e_steps"], world, max_e2e) / 1e9
+
+    pre = run_prefill(dev, args.prefill_iters, 3)
+
+    if world > 1:
+        barrier(dev)
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_kind = measured_peaks()
+    per_launch = dec["secs"] / (args.steps * dec["launches_per_step"])
+    launch_bytes = decode_bytes_per_gemv(2560, 6912)
+    achieved = launch_bytes / per_launch / 1e9
+    traffic = profiled_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": "gemv_m1_dense",
+                "peak_source": f"{peak_kind} hbm_gbs"}
+    int8_peak = 2.0 * peaks["bf16_tflops"]
+    prefill = {"metric": "prefill int8 TOPS", "value": pre["tops"], "unit": "TOPS",
+               "workload": f"2B4T prefill M={PREFILL_M}: " + ", ".join(f"{k}->{n}" for k, n in PREFILL_SHAPES),
+               "shapes": pre["shapes"], "kernel": pre["kernel"], "l2": "flushed (256 MB write) before each call",
+               "roofline": {"bound": "tensor", "achieved": pre["tops"], "peak": int8_peak, "unit": "TOPS",
+                            "frac": pre["tops"] / int8_peak,
+                            "peak_source": f"{peak_kind} bf16_tflops x 2 (int8/bf16 nominal ratio)"}}
+    cpu = None
+    if not args.no_cpu_baseline:
+        v, n, el = oracle_decode_sample(args.cpu_seconds)
+        cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"oracle forward (plain C, 1 thread) on one FFN layer (gate, up, down at M=1), "
+                         f"{n} repetitions in {el:.1f} s"}
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8 x ternary -> int32 (bf16 in/out)",
+            "data": "synthetic", "config": config, "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": dec["h2d"],
+                    "d2h_bytes_per_step": dec["d2h"], "steps": dec["e2e_steps"]},
+            "gpu_launches": args.steps * dec["launches_per_step"], "clocks": dec["clocks"],
+            "hbm_frac": value / world / peaks["hbm_gbs"], "prefill": prefill}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

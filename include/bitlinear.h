@@ -1,0 +1,186 @@
+/*
+ * bitlinear.h -- C ABI of the B200 (sm_100a) BitLinear forward library.
+ *
+ * The operation (BitNet b1.58 / Sparse-BitNet BitLinear, forward only):
+ *
+ *   alpha   = mean |W|                       over the whole latent matrix W [N, K]
+ *   W_t     = clamp(round(W / (alpha + 1e-5)), -1, 1)
+ *   gamma_m = max_k |x_mk|                    per token (row of x [M, K])
+ *   q       = clamp(round(127 x / (gamma + 1e-5)), -128, 127)   (int8)
+ *   acc     = q W_t^T                         int32 [M, N]
+ *   y       = acc * alpha * gamma_m / 127     bf16  [M, N]
+ *
+ * Sources, cited by page title and section:
+ *  - "BitNet 1-Bit LLM" blog (youngju.dev), section "BitNet b1.58 / Absmean
+ *    quantization function": weight_quant_ternary, activation_quant and the
+ *    BitLinear_b158 forward (integer matmul, then rescale).
+ *  - "BitNet b1.58 2B4T Technical Report" summary, section 2 Architecture
+ *    (absmean ternary weights, per-token absmax 8-bit activations) and
+ *    section 5.1 GPU Inference (four ternary weights packed per int8, moved
+ *    from HBM to on-chip memory, unpacked, combined with 8-bit activations).
+ *  - "BitNet 1-Bit LLM" blog, section "bitnet.cpp / Architecture overview":
+ *    the I2_S code map -1 -> 00, 0 -> 01, +1 -> 10.
+ *  - "Sparse-BitNet" review, section 3.2 (N:M mask from the latent
+ *    magnitudes, applied after ternarisation) and section 4 (6:8 and 2:4).
+ *
+ * Readings where the pages are silent or disagree: Q_b = 127 in both the
+ * quantisation and the rescale (the blog prints 2**(bits-1) = 128; the
+ * contract here is 127); round-half-to-even everywhere; scale divisions in
+ * IEEE fp32 (RN(x * 127) / RN(gamma + 1e-5)); alpha summed in fp64 and
+ * rounded once to fp32; the rescale as RN(RN(alpha * gamma) / 127) applied
+ * with one fp32 multiply before the bf16 rounding; N:M blocks run along K
+ * inside one output row, ties in |W| go to the lower position.
+ *
+ * Packed layouts (all device memory, caller-owned):
+ *  dense  codes: row n is ld = 16 * ceil(K / 64) bytes; weight k sits in
+ *         byte k / 4, bits 2*(k % 4) .. +1, code = W_t + 1 (00 = -1,
+ *         01 = 0, 10 = +1, 11 unused); tail positions hold code 01.
+ *  N:M    values: per row the n kept codes of every block in increasing k,
+ *         same 2-bit packing, row stride 16 * ceil(K * n / m / 64) bytes.
+ *         meta (2:4): per block a nibble i0 | i1 << 2 (kept positions,
+ *         i0 < i1), block b in byte b / 2, low nibble first.
+ *         meta (n:8): per block one byte, bit j = position j kept.
+ *         meta row stride 16 * ceil(K / 128) bytes.
+ *
+ * Conventions for every call:
+ *  - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *    "host" pointers are ordinary host memory.  The library allocates no
+ *    memory in any call.
+ *  - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously; argument errors are returned before
+ *    anything is enqueued.  A kernel that gives up on an internal wait
+ *    (about one second) writes a code to the device status word instead of
+ *    trapping; read it with bitlinear_device_status().
+ *  - No CPU fallback exists.  Unsupported shapes return BITLINEAR_ERR_SHAPE.
+ *  - bf16 values are passed as their 16-bit patterns (uint16_t).
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bitlinear_status {
+  BITLINEAR_OK = 0,
+  BITLINEAR_ERR_NULL = 1,           /* a required pointer is NULL */
+  BITLINEAR_ERR_SHAPE = 2,          /* M, N or K out of the supported range */
+  BITLINEAR_ERR_ALIGN = 3,          /* a pointer misses its 16-byte alignment */
+  BITLINEAR_ERR_PATTERN = 4,        /* N:M pattern other than dense, 2:4 or n:8 (1 <= n <= 7) */
+  BITLINEAR_ERR_WORKSPACE = 5,      /* workspace NULL or smaller than required */
+  BITLINEAR_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
+  BITLINEAR_ERR_DEVICE = 7,         /* current device is not sm_100 */
+  BITLINEAR_ERR_FLAGS = 8           /* unknown flag, or a path flag the shape cannot take */
+} bitlinear_status;
+
+/* Limits checked by every call. */
+#define BITLINEAR_MAX_K 65536       /* keeps every int32 partial sum exact */
+#define BITLINEAR_MAX_N (1 << 24)
+#define BITLINEAR_MAX_M (1 << 24)
+
+/* Flags of bitlinear_forward / bitlinear_forward_nm. */
+#define BITLINEAR_FLAG_PDL 0x1u       /* launch as a programmatic dependent: the
+                                         kernel may start streaming w->codes /
+                                         w->meta before the preceding kernel on
+                                         the stream finishes.  The caller asserts
+                                         that this preceding kernel does not
+                                         write the weight buffers.  x, y, acc and
+                                         alpha are touched only after it ends. */
+#define BITLINEAR_FLAG_PATH_GEMV 0x2u /* force the M = 1 streaming GEMV (needs M == 1) */
+#define BITLINEAR_FLAG_PATH_TC 0x4u   /* force the tensor-core path at any M */
+
+/* Packed weights.  All pointers device, caller-owned. */
+typedef struct bitlinear_weights {
+  int32_t N;              /* output features (rows of W) */
+  int32_t K;              /* input features */
+  int32_t nm_n;           /* kept per block: 0 for dense */
+  int32_t nm_m;           /* block length: 0 for dense, 4 (with n = 2) or 8 */
+  const uint8_t* codes;   /* dense codes, or the N:M kept values (16-byte aligned) */
+  const uint8_t* meta;    /* N:M metadata (16-byte aligned); NULL for dense */
+  const float* alpha;     /* one fp32: the absmean scale of the dense latent W */
+} bitlinear_weights;
+
+/* Byte sizes of the packed buffers.  ld_codes / ld_meta are row strides in
+ * bytes; meta outputs are 0 for dense.  Any output pointer may be NULL.
+ * Pure host computation.  Errors: SHAPE (N, K out of range or K % m != 0),
+ * PATTERN. */
+bitlinear_status bitlinear_packed_layout(int32_t N, int32_t K, int32_t nm_n, int32_t nm_m,
+                                         int64_t* ld_codes, int64_t* ld_meta,
+                                         size_t* codes_bytes, size_t* meta_bytes);
+
+/* Workspace bytes needed by bitlinear_pack_weights for an N x K matrix. */
+size_t bitlinear_pack_workspace_bytes(int32_t N, int32_t K);
+
+/* Quantises and packs a latent fp32 matrix.
+ * W        device, fp32 [N, K] row-major (read only).
+ * nm_n/m   0,0 dense; 2,4; or n,8 with 1 <= n <= 7 (mask of |W| per block
+ *          of m consecutive k, applied after ternarisation; alpha still comes
+ *          from the dense W).
+ * codes    device, out: codes_bytes (dense) or the kept values (N:M).
+ * meta     device, out: meta_bytes (N:M only; ignored for dense).
+ * alpha    device, out: one fp32.
+ * workspace, workspace_bytes: device scratch of bitlinear_pack_workspace_bytes().
+ * Errors: NULL, SHAPE, PATTERN, ALIGN (codes/meta not 16-byte aligned),
+ *         WORKSPACE, CUDA. */
+bitlinear_status bitlinear_pack_weights(const float* W, int32_t N, int32_t K, int32_t nm_n, int32_t nm_m,
+                                        uint8_t* codes, uint8_t* meta, float* alpha,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Packs an already-ternary matrix (values in {-1, 0, 1}) with a given scale,
+ * for weights drawn directly in ternary form.  Dense layout only.
+ * Wt       device, int8 [N, K] row-major; values outside {-1,0,1} are clamped.
+ * alpha    host value, written to alpha_out (device, one fp32).
+ * Errors: NULL, SHAPE, ALIGN, CUDA. */
+bitlinear_status bitlinear_pack_ternary(const int8_t* Wt, int32_t N, int32_t K, float alpha,
+                                        uint8_t* codes, float* alpha_out, void* stream);
+
+/* Per-token absmax int8 quantisation.
+ * x        device, bf16 bits [M, K] row-major (16-byte aligned).
+ * q        device, out: int8 [M, K] row-major codes in natural k order.
+ * gamma    device, out: fp32 [M] = max_k |x_mk|.
+ * rowsum   device, out (may be NULL): int32 [M] = sum_k q_mk.
+ * Errors: NULL, SHAPE, ALIGN, CUDA. */
+bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* gamma,
+                                     int32_t* rowsum, void* stream);
+
+/* Workspace bytes needed by bitlinear_forward / bitlinear_forward_nm.  0 when
+ * the call takes the M = 1 GEMV path (which quantises in-kernel). */
+size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags);
+
+/* y = BitLinear(x) for dense packed weights.
+ * w        host struct describing device buffers; w->nm_n == w->nm_m == 0.
+ * x        device, bf16 bits [M, K] (16-byte aligned).
+ * y        device, out: bf16 bits [M, N].
+ * acc      device, out (may be NULL): int32 [M, N], the exact accumulator.
+ * workspace, workspace_bytes: device scratch (may be NULL when 0 is needed).
+ * flags    BITLINEAR_FLAG_*.
+ * Path: M == 1 takes the streaming GEMV; M >= 2 the tcgen05 tensor-core GEMM.
+ * Errors: NULL, SHAPE, ALIGN, PATTERN, WORKSPACE, FLAGS, DEVICE, CUDA. */
+bitlinear_status bitlinear_forward(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
+                                   int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                   void* stream);
+
+/* Same as bitlinear_forward for N:M packed weights (w->nm_n/nm_m = 2,4 or n,8). */
+bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
+                                      int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                      void* stream);
+
+/* Synchronises stream and reads the current device's status word into *code
+ * (0 = no kernel gave up on a wait).  If clear != 0 the word is reset. */
+bitlinear_status bitlinear_device_status(void* stream, int32_t* code, int32_t clear);
+
+/* Name of the kernel variant the last successful call on this host thread
+ * enqueued (a static string; "" before the first call). */
+const char* bitlinear_last_kernel(void);
+
+/* Human-readable name of a status code (static string). */
+const char* bitlinear_status_string(bitlinear_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

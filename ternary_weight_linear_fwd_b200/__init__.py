@@ -1,0 +1,202 @@
+"""B200 (sm_100a) BitLinear forward: thin Python binding over ``libbitlinear.so``.
+
+Every step of the forward pass runs in the library's CUDA kernels; this module
+only marshals torch tensors (device memory, the current stream) into the C ABI
+of ``include/bitlinear.h``.  There is no CPU fallback: if the library is not
+built, or the device is not sm_100, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+__all__ = [
+    "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
+    "quant_act", "forward", "forward_nm", "forward_workspace_bytes", "device_status", "last_kernel",
+    "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC",
+]
+
+FLAG_PDL = 0x1
+FLAG_PATH_GEMV = 0x2
+FLAG_PATH_TC = 0x4
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {lib().bitlinear_status_string(status).decode()} (status {status})")
+        self.status = status
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("nm_n", ctypes.c_int32), ("nm_m", ctypes.c_int32),
+        ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build the CUDA library first "
+                "(python -m ternary_weight_linear_fwd_b200.build)")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, i32, i64, u32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_size_t
+        st = ctypes.c_int
+        sig = {
+            "bitlinear_packed_layout": (st, [i32, i32, i32, i32, P, P, P, P]),
+            "bitlinear_pack_workspace_bytes": (sz, [i32, i32]),
+            "bitlinear_pack_weights": (st, [P, i32, i32, i32, i32, P, P, P, P, sz, P]),
+            "bitlinear_pack_ternary": (st, [P, i32, i32, ctypes.c_float, P, P, P]),
+            "bitlinear_quant_act": (st, [P, i32, i32, P, P, P, P]),
+            "bitlinear_forward_workspace_bytes": (sz, [i32, i32, i32, u32]),
+            "bitlinear_forward": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
+            "bitlinear_forward_nm": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
+            "bitlinear_device_status": (st, [P, ctypes.POINTER(i32), i32]),
+            "bitlinear_last_kernel": (ctypes.c_char_p, []),
+            "bitlinear_status_string": (ctypes.c_char_p, [st]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise BitLinearError(status, what)
+
+
+def _stream(stream=None) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def packed_layout(N: int, K: int, n: int = 0, m: int = 0):
+    """(ld_codes, ld_meta, codes_bytes, meta_bytes) of the packed layout."""
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    c, d = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().bitlinear_packed_layout(N, K, n, m, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c),
+                                         ctypes.byref(d)), "packed_layout")
+    return a.value, b.value, c.value, d.value
+
+
+@dataclass
+class PackedWeights:
+    N: int
+    K: int
+    nm_n: int
+    nm_m: int
+    codes: "object"           # torch.uint8 [N, ld_codes] on the device
+    meta: "object"            # torch.uint8 [N, ld_meta] or None
+    alpha: "object"           # torch.float32 [1]
+
+    def c_struct(self) -> _Weights:
+        return _Weights(self.N, self.K, self.nm_n, self.nm_m, _ptr(self.codes), _ptr(self.meta), _ptr(self.alpha))
+
+    @property
+    def nbytes(self) -> int:
+        return self.codes.numel() + (0 if self.meta is None else self.meta.numel())
+
+
+def _alloc_packed(N, K, n, m, device):
+    import torch
+    ldc, ldm, _, _ = packed_layout(N, K, n, m)
+    codes = torch.empty((N, ldc), dtype=torch.uint8, device=device)
+    meta = torch.empty((N, ldm), dtype=torch.uint8, device=device) if m else None
+    alpha = torch.empty(1, dtype=torch.float32, device=device)
+    return codes, meta, alpha
+
+
+def pack_weights(W, n: int = 0, m: int = 0, stream=None) -> PackedWeights:
+    """Absmean-ternarise and pack a latent fp32 [N, K] CUDA matrix (optionally N:M)."""
+    import torch
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
+    N, K = W.shape
+    codes, meta, alpha = _alloc_packed(N, K, n, m, W.device)
+    ws = torch.empty(lib().bitlinear_pack_workspace_bytes(N, K), dtype=torch.uint8, device=W.device)
+    _check(lib().bitlinear_pack_weights(_ptr(W), N, K, n, m, _ptr(codes), _ptr(meta), _ptr(alpha), _ptr(ws),
+                                        ws.numel(), _stream(stream)), "pack_weights")
+    return PackedWeights(N, K, n, m, codes, meta, alpha)
+
+
+def pack_ternary(Wt, alpha: float, stream=None) -> PackedWeights:
+    """Pack an int8 [N, K] CUDA matrix with values in {-1, 0, 1} and a given scale."""
+    import torch
+    assert Wt.is_cuda and Wt.dtype == torch.int8 and Wt.is_contiguous() and Wt.dim() == 2
+    N, K = Wt.shape
+    codes, _, a = _alloc_packed(N, K, 0, 0, Wt.device)
+    _check(lib().bitlinear_pack_ternary(_ptr(Wt), N, K, float(alpha), _ptr(codes), _ptr(a), _stream(stream)),
+           "pack_ternary")
+    return PackedWeights(N, K, 0, 0, codes, None, a)
+
+
+def quant_act(x, rowsum: bool = True, stream=None):
+    """Per-token int8 codes of a bf16 [M, K] CUDA matrix: (q, gamma, rowsum or None)."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    g = torch.empty(M, dtype=torch.float32, device=x.device)
+    rs = torch.empty(M, dtype=torch.int32, device=x.device) if rowsum else None
+    _check(lib().bitlinear_quant_act(_ptr(x), M, K, _ptr(q), _ptr(g), _ptr(rs), _stream(stream)), "quant_act")
+    return q, g, rs
+
+
+def forward_workspace_bytes(M: int, N: int, K: int, flags: int = 0) -> int:
+    return int(lib().bitlinear_forward_workspace_bytes(M, N, K, flags))
+
+
+def _forward(fn, what, w: PackedWeights, x, want_acc, flags, workspace, out, acc_out, stream):
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w.K
+    M = x.shape[0]
+    y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    acc = acc_out if acc_out is not None else (
+        torch.empty((M, w.N), dtype=torch.int32, device=x.device) if want_acc else None)
+    need = forward_workspace_bytes(M, w.N, w.K, flags)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ws = w.c_struct()
+    _check(fn(ctypes.byref(ws), _ptr(x), M, _ptr(y), _ptr(acc), _ptr(workspace), ws_n, flags, _stream(stream)), what)
+    return (y, acc) if want_acc else y
+
+
+def forward(w: PackedWeights, x, want_acc: bool = False, flags: int = 0, workspace=None, out=None, acc_out=None,
+            stream=None):
+    """y = BitLinear(x) (bf16 [M, N]); with want_acc also the int32 accumulator."""
+    return _forward(lib().bitlinear_forward, "forward", w, x, want_acc, flags, workspace, out, acc_out, stream)
+
+
+def forward_nm(w: PackedWeights, x, want_acc: bool = False, flags: int = 0, workspace=None, out=None, acc_out=None,
+               stream=None):
+    """Same as forward for N:M packed weights."""
+    return _forward(lib().bitlinear_forward_nm, "forward_nm", w, x, want_acc, flags, workspace, out, acc_out, stream)
+
+
+def device_status(clear: bool = True, stream=None) -> int:
+    v = ctypes.c_int32()
+    _check(lib().bitlinear_device_status(_stream(stream), ctypes.byref(v), 1 if clear else 0), "device_status")
+    return v.value
+
+
+def last_kernel() -> str:
+    return lib().bitlinear_last_kernel().decode()

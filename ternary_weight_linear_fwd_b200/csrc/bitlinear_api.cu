@@ -1,0 +1,500 @@
+// bitlinear_api.cu -- the C ABI declared in include/bitlinear.h: argument
+// checks, path selection, TMA descriptor encoding and kernel launches.  One
+// translation unit holds every kernel so the device status word is a plain
+// __device__ variable.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/bitlinear.h"
+#include "gemm_tc.cuh"
+
+namespace bl {
+
+__device__ int32_t g_device_status;
+
+namespace {
+
+thread_local const char* t_last_kernel = "";
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  int32_t* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+bitlinear_status current_device(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return BITLINEAR_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    if (d.supported) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+      d.status = static_cast<int32_t*>(p);
+    }
+    d.probed = true;
+  }
+  if (!d.supported) return BITLINEAR_ERR_DEVICE;
+  *out = &d;
+  return BITLINEAR_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor map: inner extent `inner` bytes, `outer` rows of `stride`
+// bytes, box {box_inner, box_outer}; out-of-range elements read as zero.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t stride,
+                 uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {stride};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename Kern, typename... Args>
+bitlinear_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline int64_t dense_ld(int K) { return 16 * ((static_cast<int64_t>(K) + 63) / 64); }
+inline int64_t k16(int K) { return (static_cast<int64_t>(K) + 15) / 16 * 16; }
+
+bool pattern_ok(int n, int m) { return (n == 0 && m == 0) || (n == 2 && m == 4) || (m == 8 && n >= 1 && n <= 7); }
+
+bitlinear_status check_nk(int N, int K) {
+  if (N < 1 || N > BITLINEAR_MAX_N || K < 1 || K > BITLINEAR_MAX_K) return BITLINEAR_ERR_SHAPE;
+  return BITLINEAR_OK;
+}
+
+// ---------------------------------------------------------------- tensor-core path
+int pick_bn(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+
+size_t tc_workspace(int M, int K) { return align256(static_cast<size_t>(M) * k16(K)) + 2 * align256(4 * static_cast<size_t>(M)); }
+
+template <int BN, int NM>
+bitlinear_status launch_tc_bn(const CUtensorMap& mB, const CUtensorMap& mA, const CUtensorMap& mMeta,
+                              const TcArgs& ta, cudaStream_t s) {
+  const size_t smem = tc_smem_bytes(BN, NM, ta.vbox);
+  dim3 grid((ta.N + kTcRows - 1) / kTcRows, (ta.M + BN - 1) / BN);
+  return launch(tc_gemm_kernel<BN, NM>, grid, dim3(kTcThreads), smem, s, true, mB, mA, mMeta, ta);
+}
+
+template <int NM>
+bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA, const CUtensorMap& mMeta,
+                           const TcArgs& ta, cudaStream_t s) {
+  switch (bn) {
+    case 16: return launch_tc_bn<16, NM>(mB, mA, mMeta, ta, s);
+    case 32: return launch_tc_bn<32, NM>(mB, mA, mMeta, ta, s);
+    case 64: return launch_tc_bn<64, NM>(mB, mA, mMeta, ta, s);
+    case 128: return launch_tc_bn<128, NM>(mB, mA, mMeta, ta, s);
+    default: return launch_tc_bn<256, NM>(mB, mA, mMeta, ta, s);
+  }
+}
+
+const char* tc_name(int nm, int bn) {
+  static const char* names[3][5] = {
+      {"tc_gemm_dense_bn16", "tc_gemm_dense_bn32", "tc_gemm_dense_bn64", "tc_gemm_dense_bn128", "tc_gemm_dense_bn256"},
+      {"tc_gemm_nm24_bn16", "tc_gemm_nm24_bn32", "tc_gemm_nm24_bn64", "tc_gemm_nm24_bn128", "tc_gemm_nm24_bn256"},
+      {"tc_gemm_n8_bn16", "tc_gemm_n8_bn32", "tc_gemm_n8_bn64", "tc_gemm_n8_bn128", "tc_gemm_n8_bn256"}};
+  const int i = bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : bn == 128 ? 3 : 4;
+  return names[nm][i];
+}
+
+bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
+                            void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev) {
+  const int N = w->N, K = w->K;
+  if (!ws || ws_bytes < tc_workspace(M, K) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  int8_t* qp = reinterpret_cast<int8_t*>(wsb);
+  float* scale = reinterpret_cast<float*>(wsb + align256(static_cast<size_t>(M) * k16(K)));
+  int32_t* rowsum = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(scale) + align256(4 * static_cast<size_t>(M)));
+
+  bitlinear_status st = launch(quant_act_kernel<true>, dim3(M), dim3(256), 0, s, pdl, x, M, K, static_cast<int>(k16(K)),
+                               qp, static_cast<float*>(nullptr), rowsum, w->alpha, scale);
+  if (st != BITLINEAR_OK) return st;
+
+  const int bn = pick_bn(M);
+  const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? 1 : 2);
+  CUtensorMap mB, mA, mMeta;
+  if (!make_map_u8(&mB, qp, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
+                   kTcBK, static_cast<uint32_t>(bn), true))
+    return BITLINEAR_ERR_CUDA;
+  TcArgs ta;
+  ta.M = M;
+  ta.N = N;
+  ta.K = K;
+  ta.kblocks = (K + kTcBK - 1) / kTcBK;
+  ta.scale = scale;
+  ta.rowsum = rowsum;
+  ta.y = y;
+  ta.acc = acc;
+  ta.nm_n = w->nm_n;
+  ta.vbox = 0;
+  ta.status = dev->status;
+  if (nm == 0) {
+    const int64_t ld = dense_ld(K);
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    mMeta = mA;
+  } else {
+    int64_t ldv = 0, ldm = 0;
+    if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
+      return BITLINEAR_ERR_PATTERN;
+    const uint32_t vbox = nm == 1 ? 16u : static_cast<uint32_t>((4 * w->nm_n + 12 + 15) / 16 * 16);
+    ta.vbox = static_cast<int>(vbox);
+    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+  }
+  if (nm == 0)
+    st = launch_tc<0>(bn, mB, mA, mMeta, ta, s);
+  else if (nm == 1)
+    st = launch_tc<1>(bn, mB, mA, mMeta, ta, s);
+  else
+    st = launch_tc<2>(bn, mB, mA, mMeta, ta, s);
+  if (st == BITLINEAR_OK) t_last_kernel = tc_name(nm, bn);
+  return st;
+}
+
+// ---------------------------------------------------------------- GEMV path
+struct GemvShape {
+  int tpr_log2, cpt, passes;
+};
+
+// Lanes per row and 16-byte chunks per lane: the least idle lanes, then the
+// widest row group; more than 6 * 32 chunks take several passes.
+GemvShape pick_gemv(int C) {
+  GemvShape best{5, 6, (C + 191) / 192};
+  int best_waste = -1;
+  for (int lg = 5; lg >= 0; --lg) {
+    const int tpr = 1 << lg;
+    const int cpt = (C + tpr - 1) / tpr;
+    if (cpt > 6) continue;
+    const int waste = tpr * cpt - C;
+    if (best_waste < 0 || waste < best_waste) {
+      best_waste = waste;
+      best = GemvShape{lg, cpt, 1};
+    }
+  }
+  return best;
+}
+
+constexpr int rmax_for(int cpt) { return cpt == 1 ? 8 : cpt == 2 ? 6 : cpt == 3 ? 4 : cpt == 4 ? 3 : 2; }
+
+template <int CPT>
+bitlinear_status launch_gemv_cpt(GemvArgs ga, int grid, size_t smem, cudaStream_t s, bool pdl) {
+  return launch(gemv_m1_kernel<CPT, rmax_for(CPT)>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, ga);
+}
+
+bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uint16_t* y, int32_t* acc, bool pdl,
+                              cudaStream_t s, DeviceState* dev) {
+  const int N = w->N, K = w->K;
+  GemvArgs ga;
+  std::memset(&ga, 0, sizeof ga);
+  ga.codes = w->codes;
+  ga.meta = w->meta;
+  ga.N = N;
+  ga.K = K;
+  ga.x = x;
+  ga.alpha = w->alpha;
+  ga.y = y;
+  ga.acc = acc;
+  ga.nm_n = w->nm_n;
+  ga.nm_m = w->nm_m;
+  if (w->nm_m == 0) {
+    ga.ld = dense_ld(K);
+    ga.C = static_cast<int>(ga.ld / 16);
+    const GemvShape sh = pick_gemv(ga.C);
+    ga.tpr_log2 = sh.tpr_log2;
+    ga.passes = sh.passes;
+    const int groups = kGemvThreads >> sh.tpr_log2;
+    const int rmax = rmax_for(sh.cpt);
+    int grid = std::min(dev->sm_count, N);
+    if ((N + grid - 1) / grid > groups * rmax) grid = (N + groups * rmax - 1) / (groups * rmax);
+    ga.rows_base = N / grid;
+    ga.rows_rem = N % grid;
+    const size_t smem = static_cast<size_t>(ga.C) * 64;
+    bitlinear_status st;
+    switch (sh.cpt) {
+      case 1: st = launch_gemv_cpt<1>(ga, grid, smem, s, pdl); break;
+      case 2: st = launch_gemv_cpt<2>(ga, grid, smem, s, pdl); break;
+      case 3: st = launch_gemv_cpt<3>(ga, grid, smem, s, pdl); break;
+      case 4: st = launch_gemv_cpt<4>(ga, grid, smem, s, pdl); break;
+      case 5: st = launch_gemv_cpt<5>(ga, grid, smem, s, pdl); break;
+      default: st = launch_gemv_cpt<6>(ga, grid, smem, s, pdl); break;
+    }
+    if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_dense";
+    return st;
+  }
+  int64_t ldv = 0, ldm = 0;
+  if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
+    return BITLINEAR_ERR_PATTERN;
+  ga.ld = ldv;
+  ga.ld_meta = ldm;
+  ga.C = (K + 127) / 128;
+  int lg = 0;
+  while ((1 << lg) < ga.C && lg < 5) ++lg;
+  ga.tpr_log2 = lg;
+  ga.passes = 1;
+  const int groups = kGemvThreads >> lg;
+  int grid = std::min(dev->sm_count * 2, (N + groups - 1) / groups);
+  grid = std::max(grid, 1);
+  ga.rows_base = N / grid;
+  ga.rows_rem = N % grid;
+  const size_t smem = static_cast<size_t>(ga.C) * 128;
+  bitlinear_status st = launch(gemv_nm_m1_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, ga);
+  if (st == BITLINEAR_OK) t_last_kernel = w->nm_m == 4 ? "gemv_m1_nm24" : "gemv_m1_n8";
+  return st;
+}
+
+bitlinear_status forward_common(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y, int32_t* acc,
+                                void* ws, size_t ws_bytes, uint32_t flags, void* stream, bool want_nm) {
+  if (!w || !x || !y || !w->codes || !w->alpha) return BITLINEAR_ERR_NULL;
+  bitlinear_status st = check_nk(w->N, w->K);
+  if (st != BITLINEAR_OK) return st;
+  if (M < 1 || M > BITLINEAR_MAX_M) return BITLINEAR_ERR_SHAPE;
+  if (!pattern_ok(w->nm_n, w->nm_m)) return BITLINEAR_ERR_PATTERN;
+  const bool is_nm = w->nm_m != 0;
+  if (is_nm != want_nm) return BITLINEAR_ERR_PATTERN;
+  if (is_nm && (!w->meta || w->K % w->nm_m != 0)) return is_nm && !w->meta ? BITLINEAR_ERR_NULL : BITLINEAR_ERR_SHAPE;
+  if (!aligned16(w->codes) || !aligned16(x) || (is_nm && !aligned16(w->meta))) return BITLINEAR_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(y) & 1u) || (acc && (reinterpret_cast<uintptr_t>(acc) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(w->alpha) & 3u))
+    return BITLINEAR_ERR_ALIGN;
+  const uint32_t known = BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_GEMV | BITLINEAR_FLAG_PATH_TC;
+  if (flags & ~known) return BITLINEAR_ERR_FLAGS;
+  if ((flags & BITLINEAR_FLAG_PATH_GEMV) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  const bool pdl = (flags & BITLINEAR_FLAG_PDL) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || M > 1;
+  if (tc) return forward_tc(w, x, M, y, acc, ws, ws_bytes, pdl, s, dev);
+  return forward_gemv(w, x, y, acc, pdl, s, dev);
+}
+
+}  // namespace
+}  // namespace bl
+
+using namespace bl;
+
+extern "C" {
+
+bitlinear_status bitlinear_packed_layout(int32_t N, int32_t K, int32_t nm_n, int32_t nm_m, int64_t* ld_codes,
+                                         int64_t* ld_meta, size_t* codes_bytes, size_t* meta_bytes) {
+  bitlinear_status st = check_nk(N, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!pattern_ok(nm_n, nm_m)) return BITLINEAR_ERR_PATTERN;
+  int64_t ldc, ldm = 0;
+  if (nm_m == 0) {
+    ldc = dense_ld(K);
+  } else {
+    if (K % nm_m != 0) return BITLINEAR_ERR_SHAPE;
+    const int64_t kept = static_cast<int64_t>(K) / nm_m * nm_n;
+    ldc = 16 * ((kept + 63) / 64);
+    ldm = 16 * ((static_cast<int64_t>(K) + 127) / 128);
+  }
+  if (ld_codes) *ld_codes = ldc;
+  if (ld_meta) *ld_meta = ldm;
+  if (codes_bytes) *codes_bytes = static_cast<size_t>(ldc) * N;
+  if (meta_bytes) *meta_bytes = static_cast<size_t>(ldm) * N;
+  return BITLINEAR_OK;
+}
+
+size_t bitlinear_pack_workspace_bytes(int32_t N, int32_t K) {
+  (void)N;
+  (void)K;
+  return 1024 * sizeof(double);
+}
+
+bitlinear_status bitlinear_pack_weights(const float* W, int32_t N, int32_t K, int32_t nm_n, int32_t nm_m,
+                                        uint8_t* codes, uint8_t* meta, float* alpha, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (!W || !codes || !alpha) return BITLINEAR_ERR_NULL;
+  int64_t ldc = 0, ldm = 0;
+  bitlinear_status st = bitlinear_packed_layout(N, K, nm_n, nm_m, &ldc, &ldm, nullptr, nullptr);
+  if (st != BITLINEAR_OK) return st;
+  if (nm_m != 0 && !meta) return BITLINEAR_ERR_NULL;
+  if (!aligned16(codes) || (nm_m != 0 && !aligned16(meta)) || (reinterpret_cast<uintptr_t>(W) & 3u) ||
+      (reinterpret_cast<uintptr_t>(alpha) & 3u))
+    return BITLINEAR_ERR_ALIGN;
+  if (!workspace || workspace_bytes < bitlinear_pack_workspace_bytes(N, K) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 7u))
+    return BITLINEAR_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t count = static_cast<int64_t>(N) * K;
+  const int nparts = static_cast<int>(std::min<int64_t>(1024, (count + 255) / 256));
+  double* partial = static_cast<double*>(workspace);
+  st = launch(absmean_partial_kernel, dim3(nparts), dim3(256), 0, s, false, W, count, partial);
+  if (st != BITLINEAR_OK) return st;
+  st = launch(absmean_final_kernel, dim3(1), dim3(256), 0, s, false, static_cast<const double*>(partial), nparts,
+              count, alpha);
+  if (st != BITLINEAR_OK) return st;
+  if (nm_m == 0) {
+    const int64_t units = (ldc / 16) * N;
+    st = launch(pack_dense_kernel<true>, dim3(static_cast<unsigned>((units + 255) / 256)), dim3(256), 0, s, false, W,
+                static_cast<const int8_t*>(nullptr), N, K, ldc, static_cast<const float*>(alpha), codes);
+    if (st == BITLINEAR_OK) t_last_kernel = "pack_dense";
+  } else {
+    const int spans = (K / nm_m + 63) / 64;
+    const int64_t threads = static_cast<int64_t>(spans) * N;
+    st = launch(pack_nm_kernel, dim3(static_cast<unsigned>((threads + 127) / 128)), dim3(128), 0, s, false, W, N, K,
+                nm_n, nm_m, ldc, ldm, static_cast<const float*>(alpha), codes, meta);
+    if (st == BITLINEAR_OK) t_last_kernel = "pack_nm";
+  }
+  return st;
+}
+
+bitlinear_status bitlinear_pack_ternary(const int8_t* Wt, int32_t N, int32_t K, float alpha, uint8_t* codes,
+                                        float* alpha_out, void* stream) {
+  if (!Wt || !codes || !alpha_out) return BITLINEAR_ERR_NULL;
+  bitlinear_status st = check_nk(N, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(alpha_out) & 3u)) return BITLINEAR_ERR_ALIGN;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t ld = dense_ld(K);
+  const int64_t units = (ld / 16) * N;
+  st = launch(write_alpha_kernel, dim3(1), dim3(32), 0, s, false, alpha_out, alpha);
+  if (st != BITLINEAR_OK) return st;
+  st = launch(pack_dense_kernel<false>, dim3(static_cast<unsigned>((units + 255) / 256)), dim3(256), 0, s, false,
+              static_cast<const float*>(nullptr), Wt, N, K, ld, static_cast<const float*>(nullptr), codes);
+  if (st == BITLINEAR_OK) t_last_kernel = "pack_ternary";
+  return st;
+}
+
+bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* gamma,
+                                     int32_t* rowsum, void* stream) {
+  if (!x || !q || !gamma) return BITLINEAR_ERR_NULL;
+  if (M < 1 || M > BITLINEAR_MAX_M || K < 1 || K > BITLINEAR_MAX_K) return BITLINEAR_ERR_SHAPE;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(gamma) & 3u) ||
+      (rowsum && (reinterpret_cast<uintptr_t>(rowsum) & 3u)))
+    return BITLINEAR_ERR_ALIGN;
+  DeviceState* dev = nullptr;
+  bitlinear_status st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  st = launch(quant_act_kernel<false>, dim3(M), dim3(256), 0, static_cast<cudaStream_t>(stream), false, x, M, K, K, q,
+              gamma, rowsum, static_cast<const float*>(nullptr), static_cast<float*>(nullptr));
+  if (st == BITLINEAR_OK) t_last_kernel = "quant_act";
+  return st;
+}
+
+size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {
+  (void)N;
+  if (M < 1 || K < 1) return 0;
+  const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || (M > 1 && !(flags & BITLINEAR_FLAG_PATH_GEMV));
+  return tc ? tc_workspace(M, K) : 0;
+}
+
+bitlinear_status bitlinear_forward(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
+                                   int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                   void* stream) {
+  return forward_common(w, x, M, y, acc, workspace, workspace_bytes, flags, stream, false);
+}
+
+bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
+                                      int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                      void* stream) {
+  return forward_common(w, x, M, y, acc, workspace, workspace_bytes, flags, stream, true);
+}
+
+bitlinear_status bitlinear_device_status(void* stream, int32_t* code, int32_t clear) {
+  if (!code) return BITLINEAR_ERR_NULL;
+  DeviceState* dev = nullptr;
+  bitlinear_status st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, dev->status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  *code = v;
+  if (clear) {
+    const int32_t z = 0;
+    if (cudaMemcpy(dev->status, &z, sizeof z, cudaMemcpyHostToDevice) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  }
+  return BITLINEAR_OK;
+}
+
+const char* bitlinear_last_kernel(void) { return t_last_kernel; }
+
+const char* bitlinear_status_string(bitlinear_status s) {
+  switch (s) {
+    case BITLINEAR_OK: return "ok";
+    case BITLINEAR_ERR_NULL: return "null pointer";
+    case BITLINEAR_ERR_SHAPE: return "unsupported shape";
+    case BITLINEAR_ERR_ALIGN: return "misaligned pointer";
+    case BITLINEAR_ERR_PATTERN: return "unsupported N:M pattern";
+    case BITLINEAR_ERR_WORKSPACE: return "workspace missing or too small";
+    case BITLINEAR_ERR_CUDA: return "CUDA error";
+    case BITLINEAR_ERR_DEVICE: return "device is not sm_100";
+    case BITLINEAR_ERR_FLAGS: return "bad flags";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

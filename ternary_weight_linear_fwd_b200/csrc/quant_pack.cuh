@@ -1,0 +1,282 @@
+// quant_pack.cuh -- per-token activation quantisation and the weight packers.
+//
+// Activation quantisation follows the BitNet b1.58 activation_quant of the
+// "BitNet 1-Bit LLM" blog (section "Absmean quantization function"):
+// gamma = max |x| per token, q = clamp(round(x * 127 / (gamma + 1e-5)), -128, 127),
+// rounded half to even, with the product and the quotient evaluated as IEEE
+// fp32 (x * 127 is exact for bf16 x).
+//
+// Weight quantisation follows weight_quant_ternary on the same page (absmean
+// over the whole matrix, W / (alpha + 1e-5) rounded half to even, clamped to
+// [-1, 1]) and the 2B4T report's section 5.1 (four ternary values per byte);
+// the 2-bit code map is bitnet.cpp's I2_S map (-1 -> 00, 0 -> 01, +1 -> 10).
+// The N:M mask follows the Sparse-BitNet review, section 3.2: the n largest
+// |W| of each block of m consecutive k are kept (ties to the lower k), and the
+// mask is applied after ternarisation.
+#pragma once
+#include "ptx.cuh"
+
+namespace bl {
+
+constexpr float kEps = 1e-5f;
+constexpr float kQb = 127.0f;
+
+// ----------------------------------------------------------------- helpers
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+// Round-half-to-even code of one activation: clamp(rne(RN(v * 127) / d), -128, 127).
+__device__ __forceinline__ int32_t act_code(float v, float d) {
+  const float t = __fmul_rn(v, kQb);
+  int32_t c = __float2int_rn(__fdiv_rn(t, d));
+  return max(-128, min(127, c));
+}
+
+// Ternary value of one latent weight: clamp(rne(w / d), -1, 1).
+__device__ __forceinline__ int32_t ternary_of(float w, float d) {
+  int32_t c = __float2int_rn(__fdiv_rn(w, d));
+  return max(-1, min(1, c));
+}
+
+template <typename T, typename Op>
+__device__ __forceinline__ T block_reduce(T v, Op op, T* red /* >= 32 entries */, T identity) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  const int nw = (blockDim.x + 31) >> 5;
+  v = lane < nw ? red[lane] : identity;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+struct MaxOp {
+  __device__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct AddI {
+  __device__ int32_t operator()(int32_t a, int32_t b) const { return a + b; }
+};
+struct AddD {
+  __device__ double operator()(double a, double b) const { return a + b; }
+};
+
+// Loads 16 consecutive bf16 values of a row starting at k0 (zero past K).
+__device__ __forceinline__ void load16_bf16(const uint16_t* row, int k0, int K, bool vec_ok, float (&v)[16]) {
+  if (vec_ok && k0 + 16 <= K) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + k0);
+    const uint4 b = *reinterpret_cast<const uint4*>(row + k0 + 8);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = (k0 + i < K) ? bf16_bits_to_f32(row[k0 + i]) : 0.0f;
+  }
+}
+
+// Packs the 16 codes of one k-group into the order used by the integer
+// contraction: byte (4j + b) holds the code of k0 + 4b + j.  This matches the
+// order in which a 2-bit weight word unpacks with (w >> 2j) & 0x03030303.
+__device__ __forceinline__ void permute16(const int32_t (&c)[16], uint32_t (&out)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    out[j] = (static_cast<uint32_t>(c[j] & 0xFF)) | (static_cast<uint32_t>(c[4 + j] & 0xFF) << 8) |
+             (static_cast<uint32_t>(c[8 + j] & 0xFF) << 16) | (static_cast<uint32_t>(c[12 + j] & 0xFF) << 24);
+}
+
+// ----------------------------------------------------------------- quant_act
+// One CTA per token row.  kPermute = false writes natural-order codes [M, ldq]
+// (ldq = K); kPermute = true writes the contraction order [M, ldq] with ldq =
+// K rounded up to 16 (zeros past K) and, when alpha is given, the per-token
+// rescale s = RN(RN(alpha * gamma) / 127).
+template <bool kPermute>
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K, int ldq,
+                                                        int8_t* __restrict__ q, float* __restrict__ gamma,
+                                                        int32_t* __restrict__ rowsum, const float* __restrict__ alpha,
+                                                        float* __restrict__ scale) {
+  __shared__ float redf[32];
+  __shared__ int32_t redi[32];
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  const int row = blockIdx.x;
+  if (row >= M) return;
+  const uint16_t* xr = x + static_cast<size_t>(row) * K;
+  const bool vec_ok = (K % 8) == 0;
+
+  float mx = 0.0f;
+  if (vec_ok) {
+    for (int k = threadIdx.x * 8; k < K; k += blockDim.x * 8) {
+      const uint4 a = *reinterpret_cast<const uint4*>(xr + k);
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mx = fmaxf(mx, fabsf(__uint_as_float(w[i] << 16)));
+        mx = fmaxf(mx, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+      }
+    }
+  } else {
+    for (int k = threadIdx.x; k < K; k += blockDim.x) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(xr[k])));
+  }
+  mx = block_reduce(mx, MaxOp(), redf, 0.0f);
+  const float d = __fadd_rn(mx, kEps);
+
+  int32_t sum = 0;
+  const int groups = (K + 15) / 16;
+  int8_t* qr = q + static_cast<size_t>(row) * ldq;
+  const bool qvec = ((reinterpret_cast<uintptr_t>(q) & 15u) == 0) && (ldq % 16) == 0;
+  for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+    const int k0 = g * 16;
+    float v[16];
+    load16_bf16(xr, k0, K, vec_ok, v);
+    int32_t c[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      c[i] = (k0 + i < K) ? act_code(v[i], d) : 0;
+      sum += c[i];
+    }
+    if (kPermute) {
+      uint32_t w[4];
+      permute16(c, w);
+      *reinterpret_cast<uint4*>(qr + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else if (qvec && k0 + 16 <= K) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[j] = (static_cast<uint32_t>(c[4 * j] & 0xFF)) | (static_cast<uint32_t>(c[4 * j + 1] & 0xFF) << 8) |
+               (static_cast<uint32_t>(c[4 * j + 2] & 0xFF) << 16) | (static_cast<uint32_t>(c[4 * j + 3] & 0xFF) << 24);
+      *reinterpret_cast<uint4*>(qr + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      for (int i = 0; i < 16 && k0 + i < K; ++i) qr[k0 + i] = static_cast<int8_t>(c[i]);
+    }
+  }
+  sum = block_reduce(sum, AddI(), redi, 0);
+  if (threadIdx.x == 0) {
+    if (gamma) gamma[row] = mx;
+    if (rowsum) rowsum[row] = sum;
+    if (scale) scale[row] = __fdiv_rn(__fmul_rn(*alpha, mx), kQb);
+  }
+}
+
+// ----------------------------------------------------------------- absmean
+// Stage 1: per-CTA fp64 partial sums of |W| (grid-stride, fixed grid).
+__global__ void __launch_bounds__(256) absmean_partial_kernel(const float* __restrict__ W, int64_t count,
+                                                              double* __restrict__ partial) {
+  __shared__ double red[32];
+  double s = 0.0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride)
+    s += fabs(static_cast<double>(W[i]));
+  s = block_reduce(s, AddD(), red, 0.0);
+  if (threadIdx.x == 0) partial[blockIdx.x] = s;
+}
+
+// Stage 2: one CTA adds the partials in a fixed order; alpha = RN32(sum / count).
+__global__ void __launch_bounds__(256) absmean_final_kernel(const double* __restrict__ partial, int nparts,
+                                                            int64_t count, float* __restrict__ alpha) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += partial[i];
+  s = block_reduce(s, AddD(), red, 0.0);
+  if (threadIdx.x == 0) *alpha = static_cast<float>(s / static_cast<double>(count));
+}
+
+// ----------------------------------------------------------------- dense pack
+// One thread per 16-byte unit (64 weights) of a packed row.  Source is either a
+// latent fp32 matrix (ternarised with alpha) or an int8 ternary matrix.
+template <bool kFromLatent>
+__global__ void __launch_bounds__(256) pack_dense_kernel(const float* __restrict__ W, const int8_t* __restrict__ Wt,
+                                                         int N, int K, int64_t ld, const float* __restrict__ alpha,
+                                                         uint8_t* __restrict__ codes) {
+  const int64_t units_per_row = ld / 16;
+  const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (u >= units_per_row * N) return;
+  const int64_t r = u / units_per_row;
+  const int k0 = static_cast<int>(u % units_per_row) * 64;
+  float d = 0.0f;
+  if (kFromLatent) d = __fadd_rn(*alpha, kEps);
+  uint32_t w[4];
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int k = k0 + wi * 16 + i;
+      int32_t t = 0;
+      if (k < K) {
+        if (kFromLatent)
+          t = ternary_of(W[r * K + k], d);
+        else
+          t = max(-1, min(1, static_cast<int32_t>(Wt[r * K + k])));
+      }
+      acc |= static_cast<uint32_t>(t + 1) << (2 * i);
+    }
+    w[wi] = acc;
+  }
+  *reinterpret_cast<uint4*>(codes + r * ld + (k0 / 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void write_alpha_kernel(float* alpha_out, float a) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) *alpha_out = a;
+}
+
+// ----------------------------------------------------------------- N:M pack
+// One thread per span of 64 blocks of one row.  Writes the span's kept codes
+// (16 * n bytes) and metadata (32 bytes for 2:4, 64 for n:8), clipped to the
+// row strides; positions past the row's last block keep code 01 / meta 0.
+__global__ void __launch_bounds__(128) pack_nm_kernel(const float* __restrict__ W, int N, int K, int n, int m,
+                                                      int64_t ldv, int64_t ldm, const float* __restrict__ alpha,
+                                                      uint8_t* __restrict__ values, uint8_t* __restrict__ meta) {
+  const int blocks_per_row = K / m;
+  const int spans = (blocks_per_row + 63) / 64;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<int64_t>(spans) * N) return;
+  const int64_t r = t / spans;
+  const int s = static_cast<int>(t % spans);
+  const float d = __fadd_rn(*alpha, kEps);
+
+  uint8_t vb[112];  // up to 16 * 7 bytes of kept codes
+  uint8_t mb[64];
+  const int vbytes = 16 * n, mbytes = (m == 4) ? 32 : 64;
+  for (int i = 0; i < vbytes; ++i) vb[i] = 0x55;
+  for (int i = 0; i < mbytes; ++i) mb[i] = 0;
+
+  int out = 0;  // kept-code index inside the span
+  for (int bi = 0; bi < 64; ++bi) {
+    const int b = s * 64 + bi;
+    if (b >= blocks_per_row) break;
+    const float* w = W + r * K + static_cast<int64_t>(b) * m;
+    float a[8];
+    for (int j = 0; j < m; ++j) a[j] = fabsf(w[j]);
+    uint32_t keep = 0;
+    for (int j = 0; j < m; ++j) {
+      int rank = 0;
+      for (int i = 0; i < m; ++i) rank += (a[i] > a[j]) || (a[i] == a[j] && i < j);
+      if (rank < n) keep |= 1u << j;
+    }
+    int kept = 0;
+    uint32_t nib = 0;
+    for (int j = 0; j < m; ++j) {
+      if (!((keep >> j) & 1u)) continue;
+      const uint32_t code = static_cast<uint32_t>(ternary_of(w[j], d) + 1);
+      const int pos = out++;
+      vb[pos >> 2] = static_cast<uint8_t>((vb[pos >> 2] & ~(3u << (2 * (pos & 3)))) | (code << (2 * (pos & 3))));
+      if (m == 4) nib |= static_cast<uint32_t>(j) << (2 * kept);
+      ++kept;
+    }
+    if (m == 4)
+      mb[bi >> 1] |= static_cast<uint8_t>(nib << (4 * (bi & 1)));
+    else
+      mb[bi] = static_cast<uint8_t>(keep);
+  }
+  const int64_t v0 = static_cast<int64_t>(s) * vbytes, m0 = static_cast<int64_t>(s) * mbytes;
+  for (int i = 0; i < vbytes && v0 + i < ldv; ++i) values[r * ldv + v0 + i] = vb[i];
+  for (int i = 0; i < mbytes && m0 + i < ldm; ++i) meta[r * ldm + m0 + i] = mb[i];
+}
+
+}  // namespace bl

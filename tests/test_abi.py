@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every
+entry point declared in include/bitlinear.h, agrees with the oracle on the
+packed layout sizes (two independent implementations of the written format),
+and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from ternary_weight_linear_fwd_b200 import build as blbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    blbuild.build()
+    import ternary_weight_linear_fwd_b200 as bl
+    return bl.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitlinear_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(0, 9):
+        assert L.bitlinear_status_string(code)
+    assert L.bitlinear_status_string(0) == b"ok"
+
+
+@pytest.mark.parametrize("N,K,n,m", [(512, 256, 0, 0), (7, 3, 0, 0), (33, 200, 0, 0), (6912, 2560, 0, 0),
+                                     (11008, 2048, 2, 4), (2048, 11008, 6, 8), (24, 1032, 7, 8),
+                                     (40, 256, 1, 8), (5, 8, 3, 8), (3, 12, 2, 4)])
+def test_layout_matches_oracle(N, K, n, m):
+    import ternary_weight_linear_fwd_b200 as bl
+    ldc, ldm, cb, mb = bl.packed_layout(N, K, n, m)
+    if m == 0:
+        assert ldc == oracle.dense_ld(K) and ldm == 0 and mb == 0
+    else:
+        assert ldc == oracle.nm_values_ld(K, n, m) and ldm == oracle.nm_meta_ld(K)
+        assert mb == N * ldm
+    assert cb == N * ldc
+
+
+@pytest.mark.parametrize("n,m", [(3, 4), (8, 8), (0, 8), (2, 0), (4, 16)])
+def test_layout_rejects_patterns(n, m):
+    import ternary_weight_linear_fwd_b200 as bl
+    with pytest.raises(bl.BitLinearError) as e:
+        bl.packed_layout(64, 256, n, m)
+    assert e.value.status == 4
+
+
+def test_layout_rejects_shapes():
+    import ternary_weight_linear_fwd_b200 as bl
+    for N, K, n, m in [(0, 64, 0, 0), (64, 0, 0, 0), (64, 65537, 0, 0), (64, 100, 6, 8)]:
+        with pytest.raises(bl.BitLinearError) as e:
+            bl.packed_layout(N, K, n, m)
+        assert e.value.status == 2
+
+
+def _w(L, N=64, K=256, n=0, m=0, codes=0x10000, meta=None, alpha=0x20000):
+    import ternary_weight_linear_fwd_b200 as bl
+    return bl._Weights(N, K, n, m, codes, meta, alpha)
+
+
+def test_forward_host_checks(L):
+    """Argument errors come back before any device work (fake, never dereferenced addresses)."""
+    fw = L.bitlinear_forward
+    x, y = 0x30000, 0x40000
+    assert fw(None, x, 1, y, None, None, 0, 0, None) == 1
+    w = _w(L)
+    assert fw(ctypes.byref(w), None, 1, y, None, None, 0, 0, None) == 1
+    assert fw(ctypes.byref(w), x, 0, y, None, None, 0, 0, None) == 2
+    assert fw(ctypes.byref(_w(L, K=70000)), x, 1, y, None, None, 0, 0, None) == 2
+    assert fw(ctypes.byref(_w(L, codes=0x10008)), x, 1, y, None, None, 0, 0, None) == 3
+    assert fw(ctypes.byref(w), x + 4, 1, y, None, None, 0, 0, None) == 3
+    assert fw(ctypes.byref(w), x, 1, y, None, None, 0, 0x80, None) == 8          # unknown flag
+    assert fw(ctypes.byref(w), x, 2, y, None, None, 0, 0x2, None) == 8           # GEMV path needs M == 1
+    assert fw(ctypes.byref(w), x, 1, y, None, None, 0, 0x6, None) == 8           # both path flags
+    nmw = _w(L, n=6, m=8, meta=0x50000)
+    assert fw(ctypes.byref(nmw), x, 1, y, None, None, 0, 0, None) == 4          # dense entry, N:M weights
+    assert L.bitlinear_forward_nm(ctypes.byref(w), x, 1, y, None, None, 0, 0, None) == 4
+    assert L.bitlinear_forward_nm(ctypes.byref(_w(L, n=6, m=8)), x, 1, y, None, None, 0, 0, None) == 1
+    assert L.bitlinear_forward_nm(ctypes.byref(_w(L, n=3, m=4, meta=0x50000)), x, 1, y, None, None, 0, 0,
+                                  None) == 4
+
+
+def test_pack_and_quant_host_checks(L):
+    assert L.bitlinear_pack_weights(None, 64, 256, 0, 0, 0x1000, None, 0x2000, 0x3000, 8192, None) == 1
+    assert L.bitlinear_pack_weights(0x1000, 64, 256, 3, 4, 0x1000, 0x4000, 0x2000, 0x3000, 8192, None) == 4
+    assert L.bitlinear_pack_weights(0x1000, 64, 256, 0, 0, 0x1008, None, 0x2000, 0x3000, 8192, None) == 3
+    assert L.bitlinear_pack_weights(0x1000, 64, 256, 0, 0, 0x1000, None, 0x2000, 0x3000, 16, None) == 5
+    assert L.bitlinear_quant_act(None, 4, 64, 0x1000, 0x2000, None, None) == 1
+    assert L.bitlinear_quant_act(0x1000, 0, 64, 0x1000, 0x2000, None, None) == 2
+    assert L.bitlinear_quant_act(0x1002, 4, 64, 0x1000, 0x2000, None, None) == 3
+    assert L.bitlinear_pack_ternary(None, 4, 64, 0.5, 0x1000, 0x2000, None) == 1
+
+
+def test_workspace_sizes(L):
+    assert L.bitlinear_forward_workspace_bytes(1, 6912, 2560, 0) == 0          # GEMV quantises in-kernel
+    assert L.bitlinear_forward_workspace_bytes(1, 6912, 2560, 0x4) >= 2560     # forced tensor-core path
+    assert L.bitlinear_forward_workspace_bytes(2048, 6912, 2560, 0) >= 2048 * 2560 + 2 * 4 * 2048
+    assert L.bitlinear_pack_workspace_bytes(6912, 2560) >= 8 * 1024

@@ -1,0 +1,249 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle, on seeded inputs.
+
+Integer results (activation codes, gamma, packed bytes, alpha, N:M metadata,
+int32 accumulators) must match bit for bit.  bf16 outputs must lie within one
+bf16 ulp of the oracle's: the oracle rounds acc * alpha * gamma / 127 once
+from fp64, the kernels form RN(RN(alpha * gamma) / 127) and one fp32 multiply
+(relative error below 2 fp32 ulp) before the bf16 rounding, so the two can
+differ only where that product sits next to a bf16 rounding boundary.
+
+Workloads follow the pages' layer shapes (BitNet b1.58 2B4T: 2560 / 6912 /
+640; Qwen2.5-3B MLP: 2048 / 11008).  Small cases are checked in full; the
+full-size prefill cases run the kernel at full size and check sampled tokens
+(every output of those tokens), since the oracle is a plain triple loop.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from ternary_weight_linear_fwd_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import ternary_weight_linear_fwd_b200 as bl  # noqa: E402
+
+DEV = torch.device("cuda:0")
+BF16_ULP_TOL = 1
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from ternary_weight_linear_fwd_b200 import build as b
+    b.build()
+    oracle.build()
+    yield
+    torch.cuda.synchronize()
+    assert bl.device_status() == 0
+
+
+def to_dev_bf16(x_bits):
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).to(DEV).view(torch.bfloat16)
+
+
+def bf16_bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def assert_bf16_close(got_bits, ref_bits):
+    d = np.abs(got_bits.astype(np.int32) - ref_bits.astype(np.int32))
+    # same sign everywhere (acc is exact on both sides), so the bit distance is the ulp distance
+    assert d.max() <= BF16_ULP_TOL, f"max bf16 ulp distance {d.max()} at {np.unravel_index(d.argmax(), d.shape)}"
+    assert (d > 0).mean() < 0.01
+
+
+# ---------------------------------------------------------------- activation quantisation
+
+@pytest.mark.parametrize("M,K", [(8, 256), (5, 200), (3, 203), (1, 6912), (64, 11008), (2048, 2560)])
+def test_quant_act_bit_exact(M, K):
+    x = synth.activations(M, K, seed=M + K)
+    q, g, rs = bl.quant_act(to_dev_bf16(x))
+    qo, go, rso = oracle.quant_act(x)
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(g.cpu().numpy(), go)
+    np.testing.assert_array_equal(rs.cpu().numpy(), rso)
+
+
+def test_quant_act_zero_and_constant_rows():
+    x = synth.activations(4, 320, seed=9)
+    x[1] = 0
+    x[2] = synth.to_bf16_bits(np.full(320, -3.5, np.float32))
+    q, g, rs = bl.quant_act(to_dev_bf16(x))
+    qo, go, rso = oracle.quant_act(x)
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(g.cpu().numpy(), go)
+    assert not qo[1].any() and np.all(qo[2] == -127)
+
+
+# ---------------------------------------------------------------- weight packing
+
+@pytest.mark.parametrize("N,K", [(512, 256), (33, 200), (7, 3), (6912, 2560), (2560, 6912)])
+def test_pack_dense_bit_exact(N, K):
+    W = synth.latent_weights(N, K, seed=3)
+    ref = oracle.pack_weights(W)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV))
+    assert float(w.alpha.cpu()[0]) == float(ref["alpha"])
+    np.testing.assert_array_equal(w.codes.cpu().numpy(), ref["codes"])
+
+
+def test_pack_ternary_bit_exact():
+    T = synth.ternary_weights(6912, 2560, seed=1)
+    a = synth.alpha_uniform(1)
+    w = bl.pack_ternary(torch.from_numpy(T).to(DEV), float(a))
+    np.testing.assert_array_equal(w.codes.cpu().numpy(), oracle.pack_dense(T))
+    assert float(w.alpha.cpu()[0]) == float(a)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (7, 8), (5, 8), (3, 8), (2, 8), (1, 8)])
+@pytest.mark.parametrize("N,K", [(40, 256), (24, 1032), (11008, 2048), (2048, 11008)])
+def test_pack_nm_bit_exact(n, m, N, K):
+    if N * K > 1_000_000 and (n, m) not in ((2, 4), (6, 8)):
+        pytest.skip("full-size shapes only for the 2:4 and 6:8 patterns")
+    if K % m:
+        pytest.skip("K must be a multiple of m")
+    W = synth.latent_weights(N, K, seed=5)
+    W[0, :16] = 0.01  # tie-heavy blocks exercise the lower-position rule
+    ref = oracle.pack_weights(W, n, m)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV), n, m)
+    assert float(w.alpha.cpu()[0]) == float(ref["alpha"])
+    np.testing.assert_array_equal(w.codes.cpu().numpy(), ref["values"])
+    np.testing.assert_array_equal(w.meta.cpu().numpy(), ref["meta"])
+
+
+# ---------------------------------------------------------------- forward helpers
+
+def _dense_case(M, K, N, seed, ternary=False):
+    x = synth.activations(M, K, seed=seed)
+    if ternary:
+        T = synth.ternary_weights(N, K, seed=seed)
+        a = synth.alpha_uniform(seed)
+        w = bl.pack_ternary(torch.from_numpy(T).to(DEV), float(a))
+        return x, T, np.float32(a), w
+    W = synth.latent_weights(N, K, seed=seed)
+    ref = oracle.pack_weights(W)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV))
+    return x, ref["Wt"], ref["alpha"], w
+
+
+def _check_rows(x, Wt, alpha, y, acc, rows):
+    yo, acco, *_ = oracle.forward(x[rows], Wt, alpha)
+    np.testing.assert_array_equal(acc.cpu().numpy()[rows], acco)
+    assert_bf16_close(bf16_bits(y)[rows], yo)
+
+
+# ---------------------------------------------------------------- dense forward
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 512), (1, 2560, 6912), (1, 6912, 2560), (1, 2560, 640),
+                                   (1, 200, 33), (1, 11008, 2048), (1, 20480, 96)])
+def test_forward_gemv_m1(M, K, N):
+    x, Wt, a, w = _dense_case(M, K, N, seed=K + N, ternary=(K, N) in ((2560, 6912), (6912, 2560)))
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+    assert bl.last_kernel() == "gemv_m1_dense"
+    _check_rows(x, Wt, a, y, acc, np.arange(M))
+
+
+@pytest.mark.parametrize("M,K,N", [(8, 256, 512), (2, 256, 512), (16, 2560, 640), (20, 203, 130), (300, 1000, 400),
+                                   (1, 2560, 6912), (130, 384, 256), (64, 128, 128)])
+def test_forward_tc_full(M, K, N):
+    x, Wt, a, w = _dense_case(M, K, N, seed=M * 7 + K)
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, flags=bl.FLAG_PATH_TC)
+    assert bl.last_kernel().startswith("tc_gemm_dense")
+    _check_rows(x, Wt, a, y, acc, np.arange(M))
+
+
+@pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560), (2560, 2560), (2560, 640)])
+def test_forward_tc_prefill_2b4t_sampled(K, N):
+    """Prefill workload (M = 2048 tokens) at full size; 48 sampled tokens checked in full."""
+    M = 2048
+    x, Wt, a, w = _dense_case(M, K, N, seed=3)
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+    rows = np.unique(np.concatenate([[0, 255, 256, M - 1], synth.splitmix64(3, 77, 44) % M])).astype(np.int64)
+    _check_rows(x, Wt, a, y, acc, rows)
+
+
+@pytest.mark.parametrize("M", [16, 256])
+def test_forward_layer_sweep_shapes(M):
+    """The seven 2B4T layer matrices at M = 16 and 256 (sampled tokens)."""
+    for name, (K, N) in synth.B2B4T_LAYER.items():
+        x, Wt, a, w = _dense_case(M, K, N, seed=4)
+        y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+        rows = np.arange(M) if M <= 16 else np.unique(synth.splitmix64(4, 5, 24) % M).astype(np.int64)
+        _check_rows(x, Wt, a, y, acc, rows)
+
+
+def test_forward_zero_and_outlier_rows():
+    M, K, N = 6, 512, 256
+    x = synth.activations(M, K, seed=12)
+    x[2] = 0
+    x[4, 7] = synth.to_bf16_bits(np.array([3.0e4], np.float32))[0]
+    W = synth.latent_weights(N, K, seed=12)
+    ref = oracle.pack_weights(W)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV))
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+    _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
+    assert not bf16_bits(y)[2].any()
+    y1, acc1 = bl.forward(w, to_dev_bf16(x[2:3]), want_acc=True)
+    assert not acc1.cpu().numpy().any() and not bf16_bits(y1).any()
+
+
+def test_forward_pdl_flag_same_result():
+    x, Wt, a, w = _dense_case(33, 640, 300, seed=21)
+    xd = to_dev_bf16(x)
+    y0, acc0 = bl.forward(w, xd, want_acc=True)
+    y1, acc1 = bl.forward(w, xd, want_acc=True, flags=bl.FLAG_PDL)
+    assert torch.equal(acc0, acc1) and torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+    x1 = to_dev_bf16(x[:1])
+    ya = bl.forward(w, x1)
+    yb = bl.forward(w, x1, flags=bl.FLAG_PDL)
+    assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
+
+
+# ---------------------------------------------------------------- N:M forward
+
+def _nm_case(M, K, N, n, m, seed):
+    x = synth.activations(M, K, seed=seed)
+    W = synth.latent_weights(N, K, seed=seed)
+    ref = oracle.pack_weights(W, n, m)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV), n, m)
+    return x, ref["Wt"], ref["alpha"], w
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (7, 8), (3, 8), (1, 8)])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 40), (1, 1032, 24), (1, 2048, 11008), (1, 11008, 2048),
+                                   (5, 1032, 140), (70, 256, 300)])
+def test_forward_nm(n, m, M, K, N):
+    if K % m:
+        pytest.skip("K must be a multiple of m")
+    if N * K > 1_000_000 and (n, m) not in ((2, 4), (6, 8)):
+        pytest.skip("full-size shapes only for the 2:4 and 6:8 patterns")
+    x, Wt, a, w = _nm_case(M, K, N, n, m, seed=5)
+    y, acc = bl.forward_nm(w, to_dev_bf16(x), want_acc=True)
+    _check_rows(x, Wt, a, y, acc, np.arange(M))
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
+@pytest.mark.parametrize("K,N", [(2048, 11008), (11008, 2048)])
+def test_forward_nm_prefill_qwen_sampled(n, m, K, N):
+    """Qwen2.5-3B MLP shapes at M = 4096 tokens; 24 sampled tokens checked in full."""
+    M = 4096
+    x, Wt, a, w = _nm_case(M, K, N, n, m, seed=5)
+    y, acc = bl.forward_nm(w, to_dev_bf16(x), want_acc=True)
+    rows = np.unique(np.concatenate([[0, M - 1], synth.splitmix64(5, 78, 22) % M])).astype(np.int64)
+    _check_rows(x, Wt, a, y, acc, rows)
+
+
+def test_forward_nm_m1_forced_tc_matches_gemv():
+    x, Wt, a, w = _nm_case(1, 2048, 1000, 6, 8, seed=8)
+    xd = to_dev_bf16(x)
+    y0, acc0 = bl.forward_nm(w, xd, want_acc=True)
+    y1, acc1 = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_PATH_TC)
+    assert torch.equal(acc0, acc1)
+    _check_rows(x, Wt, a, y1, acc1, np.arange(1))
+
+
+def test_status_word_clean():
+    torch.cuda.synchronize()
+    assert bl.device_status(clear=False) == 0
