@@ -168,6 +168,39 @@ bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t
                                       int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
                                       void* stream);
 
+/* Largest scratch, in bytes, that bitlinear_forward_noalloc can use. */
+#define BITLINEAR_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* bitlinear_forward / bitlinear_forward_nm (chosen by w->nm_m) for callers
+ * that cannot allocate device memory: the call needs no workspace argument
+ * and performs no allocation of any kind.  The papers have no counterpart to
+ * this entry point; it exists for integration only.
+ *
+ * Who needs it: a host that hands the library only its input and output
+ * buffers and owns no allocator -- for example a plugin inside an inference
+ * server or an embedded deployment whose device memory budget is reserved at
+ * start-up -- and latency-critical callers that may not call cudaMalloc /
+ * cudaFree on their hot path, because those calls can synchronise the whole
+ * device and take unbounded time.
+ *
+ * How: the scratch the tensor-core path needs (quantised activations, per-
+ * token scales and code sums) lives in one fixed device array of
+ * BITLINEAR_NOALLOC_SCRATCH_BYTES inside the library; every GPU that loads
+ * the library holds that array until the process exits.  The first call on
+ * each device looks the array's device address up (with that device
+ * current); make that first call before any stream capture.
+ *
+ * Limits: shapes whose bitlinear_forward_workspace_bytes(M, N, K, flags)
+ * exceeds BITLINEAR_NOALLOC_SCRATCH_BYTES are rejected with
+ * BITLINEAR_ERR_WORKSPACE and nothing is enqueued (for example M = 2048
+ * tokens fits up to K = 4080).  All calls on a device share the one array and
+ * it keeps the previous call's contents, which this call overwrites before
+ * reading; two calls whose work overlaps on the GPU (different streams, no
+ * ordering between them) race on it and may return wrong results.
+ * Arguments, outputs and the other errors are those of bitlinear_forward. */
+bitlinear_status bitlinear_forward_noalloc(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
+                                           int32_t* acc, uint32_t flags, void* stream);
+
 /* Synchronises stream and reads the current device's status word into *code
  * (0 = no kernel gave up on a wait).  If clear != 0 the word is reset. */
 bitlinear_status bitlinear_device_status(void* stream, int32_t* code, int32_t clear);

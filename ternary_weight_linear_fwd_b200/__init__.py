@@ -200,3 +200,31 @@ def device_status(clear: bool = True, stream=None) -> int:
 
 def last_kernel() -> str:
     return lib().bitlinear_last_kernel().decode()
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def forward_noalloc(w: PackedWeights, x, out=None, acc_out=None, want_acc: bool = False, flags: int = 0,
+                    stream=None):
+    """BitLinear forward that allocates nothing inside the library: the scratch
+    of the tensor-core path comes from one fixed array per device, shared by
+    all calls (so calls running concurrently on different streams race).
+    For hosts that can hand over only inputs and outputs.  Raises
+    BitLinearError (status 5) when the shape needs more than
+    NOALLOC_SCRATCH_BYTES of scratch."""
+    import torch
+    L = lib()
+    fn = L.bitlinear_forward_noalloc
+    if fn.argtypes is None:
+        fn.restype = ctypes.c_int
+        fn.argtypes = [ctypes.POINTER(_Weights), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                       ctypes.c_uint32, ctypes.c_void_p]
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w.K
+    M = x.shape[0]
+    y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    acc = acc_out if acc_out is not None else (
+        torch.empty((M, w.N), dtype=torch.int32, device=x.device) if want_acc else None)
+    ws = w.c_struct()
+    _check(fn(ctypes.byref(ws), _ptr(x), M, _ptr(y), _ptr(acc), flags, _stream(stream)), "forward_noalloc")
+    return (y, acc) if (want_acc or acc_out is not None) else y

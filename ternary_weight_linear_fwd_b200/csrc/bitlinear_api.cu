@@ -498,3 +498,54 @@ const char* bitlinear_status_string(bitlinear_status s) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation entry point
+// Scratch for callers that cannot allocate: one fixed array per device,
+// shared by every bitlinear_forward_noalloc call on that device.
+namespace bl {
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[BITLINEAR_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device.  The host-side
+// name is only a stand-in, so the address is looked up once per device, with
+// that device current, and cached.
+bitlinear_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return BITLINEAR_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return BITLINEAR_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BITLINEAR_OK;
+}
+
+}  // namespace
+}  // namespace bl
+
+extern "C" bitlinear_status bitlinear_forward_noalloc(const bitlinear_weights* w, const uint16_t* x, int32_t M,
+                                                      uint16_t* y, int32_t* acc, uint32_t flags, void* stream) {
+  if (!w) return BITLINEAR_ERR_NULL;
+  if (M >= 1 && bitlinear_forward_workspace_bytes(M, w->N, w->K, flags) > BITLINEAR_NOALLOC_SCRATCH_BYTES)
+    return BITLINEAR_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  if (w->N >= 1 && w->K >= 1 && M >= 1) {  // let the shared checks report bad shapes first
+    bitlinear_status st = current_device(&dev);
+    if (st != BITLINEAR_OK) return st;
+  }
+  void* scratch = nullptr;
+  if (dev) {
+    bitlinear_status st = noalloc_scratch(&scratch);
+    if (st != BITLINEAR_OK) return st;
+  }
+  // The quantisation kernel rewrites every scratch byte the GEMM reads, so
+  // nothing has to be cleared between calls.
+  return forward_common(w, x, M, y, acc, scratch, BITLINEAR_NOALLOC_SCRATCH_BYTES, flags, stream, w->nm_m != 0);
+}
