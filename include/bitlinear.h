@@ -24,8 +24,8 @@
  *    magnitudes, applied after ternarisation) and section 4 (6:8 and 2:4).
  *
  * Readings where the pages are silent or disagree: Q_b = 127 in both the
- * quantisation and the rescale (the blog prints 2**(bits-1) = 128; the
- * contract here is 127); round-half-to-even everywhere; scale divisions in
+ * quantisation and the rescale (the blog prints 2**(bits-1) = 128; this
+ * library uses 127 throughout); round-half-to-even everywhere; scale divisions in
  * IEEE fp32 (RN(x * 127) / RN(gamma + 1e-5)); alpha summed in fp64 and
  * rounded once to fp32; the rescale as RN(RN(alpha * gamma) / 127) applied
  * with one fp32 multiply before the bf16 rounding; N:M blocks run along K
@@ -83,12 +83,13 @@ typedef enum bitlinear_status {
 
 /* Flags of bitlinear_forward / bitlinear_forward_nm. */
 #define BITLINEAR_FLAG_PDL 0x1u       /* launch as a programmatic dependent: the
-                                         kernel may start streaming w->codes /
-                                         w->meta before the preceding kernel on
-                                         the stream finishes.  The caller asserts
-                                         that this preceding kernel does not
-                                         write the weight buffers.  x, y, acc and
-                                         alpha are touched only after it ends. */
+                                         kernel may start reading w->codes,
+                                         w->meta and *w->alpha before the
+                                         preceding kernel on the stream finishes.
+                                         The caller asserts that this preceding
+                                         kernel does not write those buffers.
+                                         x, y and acc are touched only after it
+                                         ends. */
 #define BITLINEAR_FLAG_PATH_GEMV 0x2u /* force the M = 1 streaming GEMV (needs M == 1) */
 #define BITLINEAR_FLAG_PATH_TC 0x4u   /* force the tensor-core path at any M */
 

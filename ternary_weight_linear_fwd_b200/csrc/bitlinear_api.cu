@@ -216,33 +216,20 @@ bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M
 }
 
 // ---------------------------------------------------------------- GEMV path
-struct GemvShape {
-  int tpr_log2, cpt, passes;
-};
+// Shared-memory budget for one CTA's weight rows in the decode GEMV: small
+// enough that the next kernel's CTA (launched early under PDL) fits beside it.
+constexpr int64_t kGemvWeightSmem = 96 * 1024;
 
-// Lanes per row and 16-byte chunks per lane: the least idle lanes, then the
-// widest row group; more than 6 * 32 chunks take several passes.
-GemvShape pick_gemv(int C) {
-  GemvShape best{5, 6, (C + 191) / 192};
-  int best_waste = -1;
-  for (int lg = 5; lg >= 0; --lg) {
-    const int tpr = 1 << lg;
-    const int cpt = (C + tpr - 1) / tpr;
-    if (cpt > 6) continue;
-    const int waste = tpr * cpt - C;
-    if (best_waste < 0 || waste < best_waste) {
-      best_waste = waste;
-      best = GemvShape{lg, cpt, 1};
-    }
-  }
-  return best;
-}
-
-constexpr int rmax_for(int cpt) { return cpt == 1 ? 8 : cpt == 2 ? 6 : cpt == 3 ? 4 : cpt == 4 ? 3 : 2; }
-
-template <int CPT>
-bitlinear_status launch_gemv_cpt(GemvArgs ga, int grid, size_t smem, cudaStream_t s, bool pdl) {
-  return launch(gemv_m1_kernel<CPT, rmax_for(CPT)>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, ga);
+// One CTA per SM when its rows fit the shared-memory budget and a TMA box
+// (at most 256 rows), more CTAs (waves) otherwise.
+int gemv_grid(int N, int64_t ld, int C, int sm_count) {
+  int grid = std::min(sm_count, N);
+  auto fits = [&](int g) {
+    const int rows_box = N / g + 1;
+    return rows_box <= 256 && gemv_smem_bytes(rows_box, ld, C) <= static_cast<size_t>(kGemvWeightSmem) + 16 * 1024;
+  };
+  while (!fits(grid) && grid < N) grid = std::min(N, grid * 2);
+  return grid;
 }
 
 bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uint16_t* y, int32_t* acc, bool pdl,
@@ -263,25 +250,19 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
   if (w->nm_m == 0) {
     ga.ld = dense_ld(K);
     ga.C = static_cast<int>(ga.ld / 16);
-    const GemvShape sh = pick_gemv(ga.C);
-    ga.tpr_log2 = sh.tpr_log2;
-    ga.passes = sh.passes;
-    const int groups = kGemvThreads >> sh.tpr_log2;
-    const int rmax = rmax_for(sh.cpt);
-    int grid = std::min(dev->sm_count, N);
-    if ((N + grid - 1) / grid > groups * rmax) grid = (N + groups * rmax - 1) / (groups * rmax);
+    ga.tpr_log2 = 0;
+    ga.passes = 1;
+    const int grid = gemv_grid(N, ga.ld, ga.C, dev->sm_count);
     ga.rows_base = N / grid;
     ga.rows_rem = N % grid;
-    const size_t smem = static_cast<size_t>(ga.C) * 64;
-    bitlinear_status st;
-    switch (sh.cpt) {
-      case 1: st = launch_gemv_cpt<1>(ga, grid, smem, s, pdl); break;
-      case 2: st = launch_gemv_cpt<2>(ga, grid, smem, s, pdl); break;
-      case 3: st = launch_gemv_cpt<3>(ga, grid, smem, s, pdl); break;
-      case 4: st = launch_gemv_cpt<4>(ga, grid, smem, s, pdl); break;
-      case 5: st = launch_gemv_cpt<5>(ga, grid, smem, s, pdl); break;
-      default: st = launch_gemv_cpt<6>(ga, grid, smem, s, pdl); break;
-    }
+    ga.status = dev->status;
+    const int rows_box = ga.rows_base + 1;
+    CUtensorMap wmap;
+    if (!make_map_u8(&wmap, w->codes, static_cast<uint64_t>(ga.ld), static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(ga.ld), 128, static_cast<uint32_t>(rows_box), true))
+      return BITLINEAR_ERR_CUDA;
+    const size_t smem = gemv_smem_bytes(rows_box, ga.ld, ga.C);
+    bitlinear_status st = launch(gemv_m1_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, wmap, ga);
     if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_dense";
     return st;
   }
@@ -295,12 +276,13 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
   while ((1 << lg) < ga.C && lg < 5) ++lg;
   ga.tpr_log2 = lg;
   ga.passes = 1;
+  ga.status = dev->status;
   const int groups = kGemvThreads >> lg;
   int grid = std::min(dev->sm_count * 2, (N + groups - 1) / groups);
   grid = std::max(grid, 1);
   ga.rows_base = N / grid;
   ga.rows_rem = N % grid;
-  const size_t smem = static_cast<size_t>(ga.C) * 128;
+  const size_t smem = static_cast<size_t>(ga.C) * 8 * (16 + 4);
   bitlinear_status st = launch(gemv_nm_m1_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, ga);
   if (st == BITLINEAR_OK) t_last_kernel = w->nm_m == 4 ? "gemv_m1_nm24" : "gemv_m1_n8";
   return st;

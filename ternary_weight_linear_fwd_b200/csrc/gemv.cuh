@@ -4,11 +4,13 @@
 // The 2B4T report (section 5.1, GPU Inference) moves packed ternary weights
 // from HBM on chip, unpacks them and combines them with 8-bit activations;
 // for one token the contraction is bound by those weight bytes.  Here every
-// CTA quantises the single activation row into shared memory (gamma, codes
-// in contraction order, their sum), while the weight loads it issued first
-// are in flight.  A lane owns a fixed set of 64-weight chunks of a row; its
-// activation codes for those chunks stay in registers for every row it
-// visits.  With code = W_t + 1:
+// CTA first hands its contiguous weight rows to the bulk-copy engine
+// (cp.async.bulk into shared memory, before griddepcontrol.wait, so under
+// programmatic dependent launch the copy overlaps the preceding kernel), then
+// quantises the single activation row into shared memory (gamma, codes in
+// contraction order, per-group code sums) while the copy lands.  A lane owns
+// a fixed set of 64-weight chunks of a row; its activation codes for those
+// chunks stay in registers for every row it visits.  With code = W_t + 1:
 //     acc = sum_k q_k * W_t,k = sum_k q_k * code_k - sum_k q_k
 // and sum_k q_k * code_k is formed four bytes at a time with an unsigned x
 // signed dp4a on (word & (3 << 2j) per byte), whose partial sums carry a
@@ -18,7 +20,7 @@
 
 namespace bl {
 
-constexpr int kGemvThreads = 256;
+constexpr int kGemvThreads = 512;
 
 struct GemvArgs {
   const uint8_t* codes;  // dense codes, or N:M kept values
@@ -35,68 +37,140 @@ struct GemvArgs {
   int tpr_log2;          // lanes per row = 1 << tpr_log2
   int passes;            // chunk passes (C > CPT << tpr_log2)
   int rows_base, rows_rem;  // CTA b owns rows_base (+1 if b < rows_rem) consecutive rows
+  int32_t* status;       // device status word
 };
 
-// Exact round-half-to-even of RN(t / d) for |t / d| < 128, given inv = RN(1 / d):
-// y = RN(t * inv) is within 2.3e-5 of RN(t / d); unless y sits within 2^-15 of
-// a half-integer both round to the same integer, otherwise the quotient is
-// formed exactly.
-__device__ __forceinline__ int32_t act_code_fast(float v, float d, float inv) {
-  const float t = __fmul_rn(v, kQb);
-  const float yq = __fmul_rn(t, inv);
-  const float fr = yq - floorf(yq);
-  int32_t c;
-  if (fabsf(fr - 0.5f) < 3.0517578125e-05f)
-    c = __float2int_rn(__fdiv_rn(t, d));
-  else
-    c = __float2int_rn(yq);
-  return max(-128, min(127, c));
+// Exact round-half-to-even of RN(t / d), t = RN(v * 127), for |t / d| < 128,
+// without a division per element.  With c = RN(127 * RN(1 / d)), y = RN(v * c)
+// differs from the true quotient by at most 3 * 2^-24 relative, i.e. by less
+// than 3.1e-5 absolute, and RN(t / d) lies within 7.6e-6 of the true quotient.
+// So unless y sits within 2^-14 of a half-integer, RN(t / d) rounds to the same
+// integer as y; such a group is recomputed with the exact quotient.  The
+// rounding to an integer is done by adding 1.5 * 2^23 (the sum's last place is
+// 1, ties to even), leaving the two's-complement code in the low byte.
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+
+// Codes of 8 consecutive activations (the first or second half of a 16-group).  b[e] holds the code of
+// element e in its low byte.
+__device__ __forceinline__ void codes8(const uint32_t (&raw)[4], float c, float d, uint32_t (&b)[8]) {
+  float emax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float v = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
+    const float yq = __fmul_rn(v, c);
+    const float sm = __fadd_rn(yq, kMagic);
+    emax = fmaxf(emax, fabsf(__fsub_rn(yq, __fsub_rn(sm, kMagic))));
+    b[e] = __float_as_uint(sm);
+  }
+  if (emax > 0.5f - 6.103515625e-05f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float v = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
+      b[e] = 0x4B400000u + static_cast<uint32_t>(__float2int_rn(__fdiv_rn(__fmul_rn(v, kQb), d)));
+    }
+  }
 }
 
-// Quantises the activation row into shared memory (contraction order, 4 * C16
-// entries of 16 codes, zero past K) and returns gamma and sum(q) to every thread.
-__device__ __forceinline__ void gemv_quantise_row(const uint16_t* __restrict__ x, int K, int groups_alloc,
-                                                  uint4* s_act, float* red_f, int32_t* red_i, float& gamma_out,
-                                                  int32_t& qsum_out) {
-  const bool vec_ok = (K % 8) == 0;
-  float mx = 0.0f;
-  if (vec_ok) {
-    for (int k = threadIdx.x * 8; k < K; k += blockDim.x * 8) {
-      const uint4 a = *reinterpret_cast<const uint4*>(x + k);
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mx = fmaxf(mx, fabsf(__uint_as_float(w[i] << 16)));
-        mx = fmaxf(mx, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
-      }
-    }
+// 8 bf16 values of a row from k0 as 4 words (zero past K).
+__device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bool vec_ok, uint32_t (&r)[4]) {
+  if (vec_ok && k0 + 8 <= K) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + k0);
+    r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
   } else {
-    for (int k = threadIdx.x; k < K; k += blockDim.x) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(x[k])));
-  }
-  mx = block_reduce(mx, MaxOp(), red_f, 0.0f);
-  const float d = __fadd_rn(mx, kEps);
-  const float inv = __frcp_rn(d);
-  int32_t sum = 0;
-  const int groups = (K + 15) / 16;
-  for (int g = threadIdx.x; g < groups_alloc; g += blockDim.x) {
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (g < groups) {
-      const int k0 = g * 16;
-      float v[16];
-      load16_bf16(x, k0, K, vec_ok, v);
-      int32_t c[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        c[i] = (k0 + i < K) ? act_code_fast(v[i], d, inv) : 0;
-        sum += c[i];
-      }
-      permute16(c, w);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = (k0 + 2 * i < K) ? row[k0 + 2 * i] : 0u;
+      const uint32_t hi = (k0 + 2 * i + 1 < K) ? row[k0 + 2 * i + 1] : 0u;
+      r[i] = lo | (hi << 16);
     }
-    s_act[g] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  sum = block_reduce(sum, AddI(), red_i, 0);  // also orders the s_act stores before their reads
-  gamma_out = mx;
-  qsum_out = sum;
+}
+
+// Quantises the single activation row into shared memory: s_act[slot(g)]
+// holds the 16 codes of k-group g in contraction order (byte 4j + b <- k =
+// 16g + 4b + j), for g < groups_alloc (zero past K), where
+// slot(g) = (g % 4) * (groups_alloc / 4) + g / 4 puts the four groups of one
+// 64-weight chunk a quarter of the array apart, so lanes reading consecutive
+// chunks hit consecutive 16-byte words; s_csum[ch] is the sum of the 64 codes
+// of chunk ch.  Each thread handles 8-element halves h = tid, tid + nthr, ...:
+// one 16-byte load, 8 codes, four 16-bit stores (bytes 2*(h%2), 2*(h%2)+1 of
+// words 0..3); the 8 halves of a chunk sit in adjacent lanes and add their code
+// sums with three shuffles.  One barrier publishes the per-warp maxima, one the
+// codes.  Returns gamma = max |x|.
+constexpr int kHalvesInRegs = 2;  // halves per thread kept in registers (K <= 8192 at 512 threads)
+
+__device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ x, int K, int groups_alloc,
+                                                   uint4* s_act, int32_t* s_csum, float* s_red) {
+  const bool vec_ok = (K % 8) == 0;
+  const int nthr = blockDim.x;
+  const int halves = (K + 7) / 8;
+  const int halves_alloc = 2 * groups_alloc;
+  const int trips = (halves_alloc + nthr - 1) / nthr;
+  uint32_t v[kHalvesInRegs][4];
+  float mx = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kHalvesInRegs; ++j) {
+    const int h = threadIdx.x + j * nthr;
+    if (h < halves) {
+      load8_raw(x, h * 8, K, vec_ok, v[j]);
+    } else {
+      v[j][0] = v[j][1] = v[j][2] = v[j][3] = 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(v[j][i] << 16)), fabsf(__uint_as_float(v[j][i] & 0xFFFF0000u))));
+  }
+  for (int h = threadIdx.x + kHalvesInRegs * nthr; h < halves; h += nthr) {
+    uint32_t t[4];
+    load8_raw(x, h * 8, K, vec_ok, t);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(t[i] << 16)), fabsf(__uint_as_float(t[i] & 0xFFFF0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = 0.0f;
+  for (int i = 0; i < (nthr >> 5); ++i) mx = fmaxf(mx, s_red[i]);
+  const float d = __fadd_rn(mx, kEps);
+  const float c = __fmul_rn(kQb, __frcp_rn(d));
+  const int quarter = groups_alloc >> 2;
+  // every lane runs the same number of trips, so every lane reaches the shuffle
+  auto emit = [&](const uint32_t (&raw)[4], int h) {
+    uint32_t b[8];
+    codes8(raw, c, d, b);
+    const uint32_t lo = __byte_perm(b[0], b[1], 0x0040), hi = __byte_perm(b[2], b[3], 0x0040);
+    const uint32_t lo2 = __byte_perm(b[4], b[5], 0x0040), hi2 = __byte_perm(b[6], b[7], 0x0040);
+    const uint32_t p0 = __byte_perm(lo, hi, 0x5410), p1 = __byte_perm(lo2, hi2, 0x5410);  // codes 0..3, 4..7
+    int32_t gs = __dp4a(static_cast<int>(p0), 0x01010101, 0);
+    gs = __dp4a(static_cast<int>(p1), 0x01010101, gs);
+    gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+    gs += __shfl_xor_sync(0xffffffffu, gs, 2);
+    gs += __shfl_xor_sync(0xffffffffu, gs, 4);
+    if (h < halves_alloc) {
+      const int g = h >> 1, half = h & 1;
+      const int sl = (g & 3) * quarter + (g >> 2);
+      uint16_t* dst = reinterpret_cast<uint16_t*>(s_act + sl) + half;
+      // word j gets codes j and j + 4 of this half in its bytes 2*half, 2*half + 1
+      dst[0] = static_cast<uint16_t>(__byte_perm(b[0], b[4], 0x0040));
+      dst[2] = static_cast<uint16_t>(__byte_perm(b[1], b[5], 0x0040));
+      dst[4] = static_cast<uint16_t>(__byte_perm(b[2], b[6], 0x0040));
+      dst[6] = static_cast<uint16_t>(__byte_perm(b[3], b[7], 0x0040));
+      if ((h & 7) == 0) s_csum[h >> 3] = gs;
+    }
+  };
+#pragma unroll
+  for (int j = 0; j < kHalvesInRegs; ++j)
+    if (j < trips) emit(v[j], threadIdx.x + j * nthr);
+  for (int j = kHalvesInRegs; j < trips; ++j) {
+    const int h = threadIdx.x + j * nthr;
+    uint32_t raw[4] = {0u, 0u, 0u, 0u};
+    if (h < halves) load8_raw(x, h * 8, K, vec_ok, raw);
+    emit(raw, h);
+  }
+  __syncthreads();
+  return mx;
 }
 
 __device__ __forceinline__ void gemv_store(const GemvArgs& a, int row, int32_t total, float s) {
@@ -120,81 +194,104 @@ __device__ __forceinline__ void dot_word(uint32_t wd, uint32_t a0, uint32_t a1, 
 }
 
 // ------------------------------------------------------------------ dense M = 1
-template <int CPT, int RMAX>
-__global__ void __launch_bounds__(kGemvThreads) gemv_m1_kernel(const GemvArgs a) {
-  extern __shared__ uint4 s_act[];  // 4 * C entries
-  __shared__ float red_f[32];
-  __shared__ int32_t red_i[32];
+// A CTA owns a contiguous range of rows.  One thread issues one TMA tile load
+// per 128-byte stripe of those rows (box {128 bytes, rows}) with the 128-byte
+// swizzle, so chunk ch of row r sits at stripe ch / 8, line r, 16-byte slot
+// (ch % 8) ^ (r % 8): lanes reading one chunk of consecutive rows, or
+// consecutive chunks of one row, never share a bank.  The contraction is a
+// flat list of (chunk, row) units, row fastest, spread evenly over all
+// threads, two units per thread and step; a unit is one 64-weight chunk of
+// one row and adds its partial sum (minus the chunk's share of sum(q)) into
+// the row's shared accumulator.
+
+__host__ __device__ __forceinline__ int gemv_stripes(int64_t ld) { return static_cast<int>((ld + 127) / 128); }
+__host__ __device__ __forceinline__ int gemv_stripe_bytes(int rows_box) { return (rows_box * 128 + 1023) & ~1023; }
+
+__host__ __device__ __forceinline__ size_t gemv_smem_bytes(int rows_box, int64_t ld, int C) {
+  return 1024 /* alignment */ + static_cast<size_t>(gemv_stripes(ld)) * gemv_stripe_bytes(rows_box) +
+         static_cast<size_t>(C) * 4 * 16 + static_cast<size_t>(C) * 4 + static_cast<size_t>(rows_box) * 4;
+}
+
+// Partial sum of one unit: row r, chunk ch, minus the chunk's share of sum(q).
+__device__ __forceinline__ int32_t gemv_unit(const uint8_t* s_w, int stripe_bytes, const uint4* s_act,
+                                             const int32_t* s_csum, int C, int r, int ch) {
+  const uint4 wv = *reinterpret_cast<const uint4*>(s_w + (ch >> 3) * stripe_bytes + r * 128 +
+                                                   (((ch & 7) ^ (r & 7)) << 4));
+  const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
+  int32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+  dot_word(wv.x, q0.x, q0.y, q0.z, q0.w, s0, s1, s2, s3);
+  dot_word(wv.y, q1.x, q1.y, q1.z, q1.w, s0, s1, s2, s3);
+  dot_word(wv.z, q2.x, q2.y, q2.z, q2.w, s0, s1, s2, s3);
+  dot_word(wv.w, q3.x, q3.y, q3.z, q3.w, s0, s1, s2, s3);
+  return s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6) - s_csum[ch];
+}
+
+__global__ void __launch_bounds__(kGemvThreads) gemv_m1_kernel(const __grid_constant__ CUtensorMap wmap,
+                                                               const GemvArgs a) {
+  extern __shared__ uint8_t s_raw[];
+  __shared__ uint64_t s_bar;
+  __shared__ float s_red[32];
   pdl_launch_dependents();
-  const int tpr = 1 << a.tpr_log2;
-  const int sub = threadIdx.x & (tpr - 1);
-  const int grp = threadIdx.x >> a.tpr_log2;
-  const int ngrp = blockDim.x >> a.tpr_log2;
   const int b = blockIdx.x;
   const int r0 = b * a.rows_base + min(b, a.rows_rem);
   const int nrows = a.rows_base + (b < a.rows_rem ? 1 : 0);
+  const int C = a.C;
+  const int rows_box = a.rows_base + 1;
+  const int stripes = gemv_stripes(a.ld);
+  const int stripe_bytes = gemv_stripe_bytes(rows_box);
+  uint8_t* s_w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_raw) + 1023) & ~uintptr_t(1023));
+  uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
+  int32_t* s_csum = reinterpret_cast<int32_t*>(s_act + 4 * C);
+  int32_t* s_acc = s_csum + C;
 
-  // Weight loads of the first pass go out before anything else.
-  uint4 w[RMAX][CPT];
-  auto load_pass = [&](int pass) {
-#pragma unroll
-    for (int r = 0; r < RMAX; ++r) {
-      const int lr = grp + r * ngrp;
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        const int ch = pass * CPT * tpr + sub + c * tpr;
-        if (lr < nrows && ch < a.C)
-          w[r][c] = ldg_stream_v4(a.codes + static_cast<int64_t>(r0 + lr) * a.ld + static_cast<int64_t>(ch) * 16);
-        else
-          w[r][c] = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
-      }
-    }
-  };
-  load_pass(0);
+  // The weights (and alpha, which belongs to them) do not depend on the
+  // preceding kernel: their copies start first.
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&wmap);
+    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box));
+    for (int st = 0; st < stripes; ++st) tma_load_2d(s_w + st * stripe_bytes, &wmap, st * 128, r0, &s_bar);
+  }
+  const float alpha = *a.alpha;
+  for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  __syncthreads();
 
   pdl_wait_primary();  // x may come from the preceding kernel
-  float gamma;
-  int32_t qsum;
-  gemv_quantise_row(a.x, a.K, 4 * a.C, s_act, red_f, red_i, gamma, qsum);
-  const float s = __fdiv_rn(__fmul_rn(*a.alpha, gamma), kQb);
+  const float gamma = quantise_row_smem(a.x, a.K, 4 * C, s_act, s_csum, s_red);
+  const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
+  const bool landed = mbar_wait(&s_bar, 0);
+  if (!landed && threadIdx.x == 0) *a.status = kDevTimeoutProducer;
 
-  int32_t part[RMAX];
-#pragma unroll
-  for (int r = 0; r < RMAX; ++r) part[r] = 0;
-  for (int pass = 0; pass < a.passes; ++pass) {
-    if (pass > 0) load_pass(pass);
-    uint32_t A[CPT][16];
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-      const int ch = pass * CPT * tpr + sub + c * tpr;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = ch < a.C ? s_act[4 * ch + i] : make_uint4(0u, 0u, 0u, 0u);
-        A[c][4 * i + 0] = v.x;
-        A[c][4 * i + 1] = v.y;
-        A[c][4 * i + 2] = v.z;
-        A[c][4 * i + 3] = v.w;
+  if (landed) {
+    const int nthr = blockDim.x;
+    const int total = nrows * C;
+    const int dq = (2 * nthr) / nrows, dr = (2 * nthr) % nrows;
+    int ch = threadIdx.x / nrows, r = threadIdx.x % nrows;                      // unit u
+    int ch2 = (threadIdx.x + nthr) / nrows, r2 = (threadIdx.x + nthr) % nrows;  // unit u + nthr
+    for (int u = threadIdx.x; u < total; u += 2 * nthr) {
+      const bool vb = u + nthr < total;
+      const int32_t pa = gemv_unit(s_w, stripe_bytes, s_act, s_csum, C, r, ch);
+      const int32_t pb = vb ? gemv_unit(s_w, stripe_bytes, s_act, s_csum, C, r2, ch2) : 0;
+      atomicAdd(&s_acc[r], pa);
+      if (vb) atomicAdd(&s_acc[r2], pb);
+      r += dr;
+      ch += dq;
+      if (r >= nrows) {
+        r -= nrows;
+        ++ch;
+      }
+      r2 += dr;
+      ch2 += dq;
+      if (r2 >= nrows) {
+        r2 -= nrows;
+        ++ch2;
       }
     }
-#pragma unroll
-    for (int r = 0; r < RMAX; ++r) {
-      int32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        dot_word(w[r][c].x, A[c][0], A[c][1], A[c][2], A[c][3], s0, s1, s2, s3);
-        dot_word(w[r][c].y, A[c][4], A[c][5], A[c][6], A[c][7], s0, s1, s2, s3);
-        dot_word(w[r][c].z, A[c][8], A[c][9], A[c][10], A[c][11], s0, s1, s2, s3);
-        dot_word(w[r][c].w, A[c][12], A[c][13], A[c][14], A[c][15], s0, s1, s2, s3);
-      }
-      part[r] += s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6);
-    }
   }
-#pragma unroll
-  for (int r = 0; r < RMAX; ++r) {
-    const int v = group_sum(part[r], tpr);
-    const int lr = grp + r * ngrp;
-    if (sub == 0 && lr < nrows) gemv_store(a, r0 + lr, v - qsum, s);
-  }
+  __syncthreads();
+  if (landed)
+    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a, r0 + rr, s_acc[rr], s);
 }
 
 // ------------------------------------------------------------------ N:M M = 1
@@ -241,9 +338,10 @@ __device__ __forceinline__ uint32_t load_bits(const uint8_t* base, int64_t bit, 
 
 // A lane owns 128-weight units (2:4: 32 blocks, n:8: 16 blocks) of a row.
 __global__ void __launch_bounds__(kGemvThreads) gemv_nm_m1_kernel(const GemvArgs a) {
-  extern __shared__ uint4 s_act[];
-  __shared__ float red_f[32];
-  __shared__ int32_t red_i[32];
+  extern __shared__ uint4 s_dyn[];
+  uint4* s_act = s_dyn;                                            // 8 * C entries
+  int32_t* s_csum = reinterpret_cast<int32_t*>(s_dyn + 8 * a.C);   // 2 * C entries
+  __shared__ float s_red[32];
   pdl_launch_dependents();
   const int tpr = 1 << a.tpr_log2;
   const int sub = threadIdx.x & (tpr - 1);
@@ -254,10 +352,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_m1_kernel(const GemvArgs
   const int nrows = a.rows_base + (b < a.rows_rem ? 1 : 0);
 
   pdl_wait_primary();
-  float gamma;
-  int32_t qsum;
-  gemv_quantise_row(a.x, a.K, 8 * a.C, s_act, red_f, red_i, gamma, qsum);
+  const float gamma = quantise_row_smem(a.x, a.K, 8 * a.C, s_act, s_csum, s_red);
   const float s = __fdiv_rn(__fmul_rn(*a.alpha, gamma), kQb);
+  int32_t qsum = 0;  // this lane's share of sum(q): the two 64-weight chunks of each of its units
+  for (int u = sub; u < a.C; u += tpr) qsum += s_csum[2 * u] + s_csum[2 * u + 1];
   const int n = a.nm_n, m = a.nm_m;
   const int blocks_per_row = a.K / m;
 
@@ -301,14 +399,14 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_m1_kernel(const GemvArgs
               dense = n8_dense_block(m0, kv & fmask) | (0x5555u << 16);
             }
           }
-          const uint4 av = s_act[g];
+          const uint4 av = s_act[(g & 3) * (2 * a.C) + (g >> 2)];
           dot_word(dense, av.x, av.y, av.z, av.w, s0, s1, s2, s3);
         }
       }
     }
-    int32_t part = s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6);
+    int32_t part = s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6) - qsum;
     part = group_sum(part, tpr);
-    if (valid && sub == 0) gemv_store(a, r0 + lr, part - qsum, s);
+    if (valid && sub == 0) gemv_store(a, r0 + lr, part, s);
   }
 }
 
