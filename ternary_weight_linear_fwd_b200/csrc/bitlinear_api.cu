@@ -93,26 +93,41 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
 }
 
 template <typename Kern, typename... Args>
-bitlinear_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, Args... args) {
+bitlinear_status launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, int cluster_x,
+                           Args... args) {
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  int n = 0;
   if (pdl) {
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
   }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
       return BITLINEAR_ERR_CUDA;
   }
   return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+template <typename Kern, typename... Args>
+bitlinear_status launch(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, Args... args) {
+  return launch_ex(kern, grid, block, smem, s, pdl, 1, args...);
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -128,36 +143,38 @@ bitlinear_status check_nk(int N, int K) {
 }
 
 // ---------------------------------------------------------------- tensor-core path
-int pick_bn(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+int pick_bn(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 
 size_t tc_workspace(int M, int K) { return align256(static_cast<size_t>(M) * k16(K)) + 2 * align256(4 * static_cast<size_t>(M)); }
 
 template <int BN, int NM>
-bitlinear_status launch_tc_bn(const CUtensorMap& mB, const CUtensorMap& mA, const CUtensorMap& mMeta,
-                              const TcArgs& ta, cudaStream_t s) {
+bitlinear_status launch_tc_bn(const CUtensorMap& mB, const CUtensorMap& mA, const CUtensorMap& mMeta, TcArgs ta,
+                              int sm_count, cudaStream_t s) {
   const size_t smem = tc_smem_bytes(BN, NM, ta.vbox);
-  dim3 grid((ta.N + kTcRows - 1) / kTcRows, (ta.M + BN - 1) / BN);
-  return launch(tc_gemm_kernel<BN, NM>, grid, dim3(kTcThreads), smem, s, true, mB, mA, mMeta, ta);
+  ta.row_tiles = (ta.N + kTcRows - 1) / kTcRows;
+  ta.tok_tiles = (ta.M + BN - 1) / BN;
+  const int tiles = ta.row_tiles * ta.tok_tiles;
+  const int grid = std::min(sm_count, tiles);
+  return launch(tc_gemm_kernel<BN, NM>, dim3(grid), dim3(kTcThreads), smem, s, true, mB, mA, mMeta, ta);
 }
 
 template <int NM>
 bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA, const CUtensorMap& mMeta,
-                           const TcArgs& ta, cudaStream_t s) {
+                           const TcArgs& ta, int sm_count, cudaStream_t s) {
   switch (bn) {
-    case 16: return launch_tc_bn<16, NM>(mB, mA, mMeta, ta, s);
-    case 32: return launch_tc_bn<32, NM>(mB, mA, mMeta, ta, s);
-    case 64: return launch_tc_bn<64, NM>(mB, mA, mMeta, ta, s);
-    case 128: return launch_tc_bn<128, NM>(mB, mA, mMeta, ta, s);
-    default: return launch_tc_bn<256, NM>(mB, mA, mMeta, ta, s);
+    case 16: return launch_tc_bn<16, NM>(mB, mA, mMeta, ta, sm_count, s);
+    case 32: return launch_tc_bn<32, NM>(mB, mA, mMeta, ta, sm_count, s);
+    case 64: return launch_tc_bn<64, NM>(mB, mA, mMeta, ta, sm_count, s);
+    default: return launch_tc_bn<128, NM>(mB, mA, mMeta, ta, sm_count, s);
   }
 }
 
 const char* tc_name(int nm, int bn) {
-  static const char* names[3][5] = {
-      {"tc_gemm_dense_bn16", "tc_gemm_dense_bn32", "tc_gemm_dense_bn64", "tc_gemm_dense_bn128", "tc_gemm_dense_bn256"},
-      {"tc_gemm_nm24_bn16", "tc_gemm_nm24_bn32", "tc_gemm_nm24_bn64", "tc_gemm_nm24_bn128", "tc_gemm_nm24_bn256"},
-      {"tc_gemm_n8_bn16", "tc_gemm_n8_bn32", "tc_gemm_n8_bn64", "tc_gemm_n8_bn128", "tc_gemm_n8_bn256"}};
-  const int i = bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : bn == 128 ? 3 : 4;
+  static const char* names[3][4] = {
+      {"tc_gemm_dense_bn16", "tc_gemm_dense_bn32", "tc_gemm_dense_bn64", "tc_gemm_dense_bn128"},
+      {"tc_gemm_nm24_bn16", "tc_gemm_nm24_bn32", "tc_gemm_nm24_bn64", "tc_gemm_nm24_bn128"},
+      {"tc_gemm_n8_bn16", "tc_gemm_n8_bn32", "tc_gemm_n8_bn64", "tc_gemm_n8_bn128"}};
+  const int i = bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3;
   return names[nm][i];
 }
 
@@ -192,6 +209,8 @@ bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M
   ta.nm_n = w->nm_n;
   ta.vbox = 0;
   ta.status = dev->status;
+  ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
+  ta.row_tiles = ta.tok_tiles = 0;
   if (nm == 0) {
     const int64_t ld = dense_ld(K);
     if (!make_map_u8(&mA, w->codes, ld, N, ld, 32, kTcRows, false)) return BITLINEAR_ERR_CUDA;
@@ -206,11 +225,11 @@ bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M
     if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16, kTcRows, false)) return BITLINEAR_ERR_CUDA;
   }
   if (nm == 0)
-    st = launch_tc<0>(bn, mB, mA, mMeta, ta, s);
+    st = launch_tc<0>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
   else if (nm == 1)
-    st = launch_tc<1>(bn, mB, mA, mMeta, ta, s);
+    st = launch_tc<1>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
   else
-    st = launch_tc<2>(bn, mB, mA, mMeta, ta, s);
+    st = launch_tc<2>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
   if (st == BITLINEAR_OK) t_last_kernel = tc_name(nm, bn);
   return st;
 }

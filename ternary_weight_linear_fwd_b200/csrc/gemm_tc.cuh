@@ -2,7 +2,7 @@
 //
 // The 2B4T report (section 5.1) stages packed ternary weights on chip,
 // unpacks them and multiplies them with 8-bit activations.  On sm_100a that
-// becomes one tcgen05 kind::i8 contraction per CTA tile:
+// becomes a persistent tcgen05 kind::i8 GEMM:
 //
 //   D[128 weight rows, BN tokens] (int32, TMEM) += A * B^T over K, where
 //   A = the weight rows' 2-bit codes (0, 1, 2) expanded to u8 and written
@@ -16,12 +16,16 @@
 // Both operands use the same K order inside each 16-wide group (byte 4j + b
 // holds k = 4b + j), which is the order (w >> 2j) & 0x03030303 produces.
 //
-// Roles (256 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues
-// the MMAs, warp 2 owns the TMEM allocation, warps 4..7 unpack weights and
-// run the epilogue (warp w reaches TMEM lanes 32 * (w % 4) .. + 31).
-// A four-stage mbarrier ring couples them: full (TMA bytes landed), aready
-// (A slot written), empty (MMAs that read the stage completed).  Every wait is
-// bounded; a role that gives up records a status code and unwinds.
+// One CTA per SM walks a static list of (weight-row tile, token tile) pairs.
+// Warp roles (16 warps): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues
+// the MMAs, warp 2 owns the TMEM allocation, warps 4..11 unpack weights (two
+// groups of four, alternating k-blocks), warps 12..15 run the epilogue.  Warp
+// w reaches TMEM lanes 32 * (w % 4) .. + 31.  An 8-stage mbarrier ring couples
+// the producer, unpackers and MMA issuer (full: TMA bytes landed, aready: A
+// slot written, empty: the MMAs that read the stage completed); two TMEM
+// accumulators (accfull / accempty) let the epilogue of one tile overlap the
+// main loop of the next.  Every wait is bounded; a role that gives up records
+// a status code and unwinds.
 //
 // N:M weights (Sparse-BitNet, section 3.2) are expanded from kept values +
 // metadata into the same dense code words before the tcgen05.st, so the MMA
@@ -31,18 +35,25 @@
 
 namespace bl {
 
-constexpr int kTcStages = 4;
+#ifndef BL_TC_STAGES
+#define BL_TC_STAGES 8
+#endif
+constexpr int kTcStages = BL_TC_STAGES;
 constexpr int kTcBK = 128;      // K elements per stage (one 128-byte swizzle row)
-constexpr int kTcRows = 128;    // weight rows per CTA (MMA M)
-constexpr int kTcThreads = 256;
+constexpr int kTcRows = 128;    // weight rows per tile (MMA M)
+constexpr int kTcThreads = 512;
+constexpr int kTcEpiWarp0 = 12;  // first epilogue warp
+constexpr int kTcStageCols = 32;  // TMEM columns of one A slot (128 int8 per lane)
 
 struct TcArgs {
   int M, N, K;
   int kblocks;            // ceil(K / 128)
+  int row_tiles, tok_tiles;
   const float* scale;     // [M] per-token rescale RN(RN(alpha * gamma) / 127)
   const int32_t* rowsum;  // [M] sum of the token's codes
   uint16_t* y;            // [M, N] bf16 bits
   int32_t* acc;           // [M, N] or null
+  int vec_store;          // y / acc rows are 16-byte aligned and N % 8 == 0
   int nm_n;               // kept per 8-block (n:8 mode)
   int vbox;               // n:8: bytes of the values box per row
   int32_t* status;        // device status word
@@ -59,15 +70,21 @@ struct TcStageBytes {
 
 template <int BN>
 struct TcCols {
-  static constexpr int kAcol0 = BN < 32 ? 32 : BN;
-  static constexpr int kNeed = kAcol0 + kTcStages * 32;
-  static constexpr int kAlloc = kNeed <= 128 ? 128 : (kNeed <= 256 ? 256 : 512);
+  static constexpr int kDcols = BN < 32 ? 32 : BN;                 // one accumulator
+  static constexpr int kAcol0 = 2 * kDcols;                        // A slots after both accumulators
+  static constexpr int kNeed = kAcol0 + kTcStages * kTcStageCols;
+  static constexpr int kAlloc = kNeed <= 256 ? 256 : 512;
+  static_assert(kNeed <= 512, "TMEM budget");
 };
 
+__host__ __device__ constexpr int tc_a_stage_bytes(int NM, int vbox) {
+  return ((NM == 0 ? kTcRows * 32 : (NM == 1 ? kTcRows * 16 : kTcRows * vbox)) + (NM == 0 ? 0 : kTcRows * 16) +
+          1023) / 1024 * 1024;
+}
+
 __host__ __device__ constexpr int tc_smem_bytes(int BN, int NM, int vbox) {
-  const int a_bytes = (NM == 0 ? kTcRows * 32 : (NM == 1 ? kTcRows * 16 : kTcRows * vbox)) + (NM == 0 ? 0 : kTcRows * 16);
-  const int a_stage = (a_bytes + 1023) / 1024 * 1024;
-  return 1024 /* alignment slack */ + kTcStages * (BN * 128 + a_stage) + 1024 /* barriers, scales */ + BN * 8;
+  return 1024 /* alignment slack */ + kTcStages * (BN * 128 + tc_a_stage_bytes(NM, vbox)) +
+         4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
 }
 
 // Dense code word of 16 weights for the current stage and group, per mode.
@@ -97,6 +114,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapMeta, const TcArgs a) {
   constexpr int S = kTcStages;
+  constexpr int DCOLS = TcCols<BN>::kDcols;
   constexpr int A_COL0 = TcCols<BN>::kAcol0;
   constexpr int NCOLS = TcCols<BN>::kAlloc;
   constexpr uint32_t IDESC = idesc_i8_u8s8(kTcRows, BN);
@@ -106,24 +124,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int a_val_bytes = TcStageBytes<NM>::a_values(a.vbox);
   const int a_meta_bytes = TcStageBytes<NM>::a_meta();
-  const int a_stage = (a_val_bytes + a_meta_bytes + 1023) / 1024 * 1024;
+  const int a_stage = tc_a_stage_bytes(NM, a.vbox);
   uint8_t* sB = base;
   uint8_t* sA = base + S * B_STAGE;
-  uint8_t* misc = sA + S * a_stage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint32_t* s_stage = reinterpret_cast<uint32_t*>(sA + S * a_stage);   // 4 warps x 32 x 33 words
+  float* s_scale = reinterpret_cast<float*>(s_stage + 4 * 32 * 33);     // [2][BN]
+  int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * BN);     // [2][BN]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_rowsum + 2 * BN);
   uint64_t* empty = full + S;
   uint64_t* aready = empty + S;
-  uint64_t* accfull = aready + S;
-  uint64_t* drain = accfull + 1;
+  uint64_t* accfull = aready + S;   // [2]
+  uint64_t* accempty = accfull + 2; // [2]
+  uint64_t* drain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  float* s_scale = reinterpret_cast<float*>(misc + 256);
-  int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + BN);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = blockIdx.x * kTcRows;
-  const int tok0 = blockIdx.y * BN;
   const int KB = a.kblocks;
+  const int ntiles = a.row_tiles * a.tok_tiles;
+  const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int total_kb = my_tiles * KB;  // k-blocks this CTA streams
   const uint32_t tx_bytes = static_cast<uint32_t>(B_STAGE + a_val_bytes + a_meta_bytes);
+  // tile t of this CTA -> (row tile, token tile), token tile fastest
+  auto tile_of = [&](int t, int& rt, int& tt) {
+    const int g = blockIdx.x + t * gridDim.x;
+    rt = g / a.tok_tiles;
+    tt = g - rt * a.tok_tiles;
+  };
 
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
@@ -132,7 +158,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&empty[s], 1);
       mbar_init(&aready[s], 4);
     }
-    mbar_init(accfull, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
     mbar_init(drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&mapB);
@@ -149,9 +178,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- producer
-      auto load_a = [&](int kb, int s) {
+    if (lane == 0 && total_kb > 0) {
+      // ------------------------------------------------------------ producer
+      auto load_a = [&](int row0, int kb, int s) {
         uint8_t* dst = sA + s * a_stage;
         if (NM == 0) {
           tma_load_2d(dst, &mapA, kb * 32, row0, &full[s]);
@@ -159,86 +188,94 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tma_load_2d(dst, &mapA, kb * 16, row0, &full[s]);
           tma_load_2d(dst + a_val_bytes, &mapMeta, kb * 16, row0, &full[s]);
         } else {
-          const int x0 = (kb * 4 * a.nm_n) & ~15;
-          tma_load_2d(dst, &mapA, x0, row0, &full[s]);
+          tma_load_2d(dst, &mapA, (kb * 4 * a.nm_n) & ~15, row0, &full[s]);
           tma_load_2d(dst + a_val_bytes, &mapMeta, kb * 16, row0, &full[s]);
         }
       };
-      const int pre = KB < S ? KB : S;
+      const int pre = total_kb < S ? total_kb : S;
       // Weights do not depend on the preceding kernel: start them first.
-      for (int kb = 0; kb < pre; ++kb) {
-        mbar_arrive_expect_tx(&full[kb], tx_bytes);
-        load_a(kb, kb);
+      for (int i = 0; i < pre; ++i) {
+        int rt, tt;
+        tile_of(i / KB, rt, tt);
+        mbar_arrive_expect_tx(&full[i], tx_bytes);
+        load_a(rt * kTcRows, i % KB, i);
       }
       pdl_wait_primary();
-      for (int kb = 0; kb < pre; ++kb) tma_load_2d(sB + kb * B_STAGE, &mapB, kb * kTcBK, tok0, &full[kb]);
+      for (int i = 0; i < pre; ++i) {
+        int rt, tt;
+        tile_of(i / KB, rt, tt);
+        tma_load_2d(sB + i * B_STAGE, &mapB, (i % KB) * kTcBK, tt * BN, &full[i]);
+      }
       bool ok = true;
-      int kb = pre;
-      for (; kb < KB; ++kb) {
-        const int s = kb % S, round = kb / S;
-        if (!mbar_wait(&empty[s], (round - 1) & 1)) {
+      int i = pre;
+      for (; i < total_kb; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(&empty[s], ((i / S) - 1) & 1)) {
           *a.status = kDevTimeoutProducer;
           ok = false;
           break;
         }
+        int rt, tt;
+        tile_of(i / KB, rt, tt);
         mbar_arrive_expect_tx(&full[s], tx_bytes);
-        load_a(kb, s);
-        tma_load_2d(sB + s * B_STAGE, &mapB, kb * kTcBK, tok0, &full[s]);
+        load_a(rt * kTcRows, i % KB, s);
+        tma_load_2d(sB + s * B_STAGE, &mapB, (i % KB) * kTcBK, tt * BN, &full[s]);
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
-        for (int j = (kb - S > 0 ? kb - S : 0); j < kb; ++j)
+        for (int j = (i - S > 0 ? i - S : 0); j < i; ++j)
           if (!mbar_wait(&full[j % S], (j / S) & 1)) *a.status = kDevTimeoutDrain;
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && total_kb > 0) {
+      // ------------------------------------------------------------ MMA issuer
       bool issued = false, ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        const uint32_t par = (kb / S) & 1;
-        if (!mbar_wait(&full[s], par) || !mbar_wait(&aready[s], par)) {
+      for (int t = 0; t < my_tiles && ok; ++t) {
+        const int buf = t & 1;
+        if (t >= 2 && !mbar_wait(&accempty[buf], ((t >> 1) - 1) & 1)) {
           *a.status = kDevTimeoutMma;
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE));
+        const uint32_t dcol = tmem + buf * DCOLS;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int i = t * KB + kb;
+          const int s = i % S;
+          const uint32_t par = (i / S) & 1;
+          if (!mbar_wait(&full[s], par) || !mbar_wait(&aready[s], par)) {
+            *a.status = kDevTimeoutMma;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE));
 #pragma unroll
-        for (int kk = 0; kk < kTcBK / 32; ++kk) {
-          tc_mma_i8_ts(tmem, tmem + A_COL0 + s * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), IDESC,
-                       (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kTcBK / 32; ++kk)
+            tc_mma_i8_ts(dcol, tmem + A_COL0 + s * kTcStageCols + kk * 8, bdesc + static_cast<uint64_t>(kk * 2),
+                         IDESC, (kb | kk) != 0 ? 1u : 0u);
+          tc_commit(&empty[s]);
+          issued = true;
         }
-        tc_commit(&empty[s]);
-        issued = true;
+        if (ok) tc_commit(&accfull[buf]);
       }
-      if (ok) {
-        tc_commit(accfull);
-      } else if (issued) {
+      if (!ok && issued) {
         tc_commit(drain);
         if (!mbar_wait(drain, 0)) *a.status = kDevTimeoutDrain;
       }
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ unpack
-    const int q = warp - 4;               // TMEM lane quarter
-    const int r = q * 32 + lane;          // weight row inside the tile
+  } else if (warp >= 4 && warp < kTcEpiWarp0) {
+    // -------------------------------------------------------------- unpack (two groups)
+    const int grp = (warp - 4) >> 2;       // 0: even k-blocks, 1: odd k-blocks
+    const int q = warp & 3;                // TMEM lane quarter
+    const int r = q * 32 + lane;           // weight row inside the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    pdl_wait_primary();
-    for (int t = threadIdx.x - 128; t < BN; t += 128) {
-      const int tok = tok0 + t;
-      s_scale[t] = tok < a.M ? a.scale[tok] : 0.0f;
-      s_rowsum[t] = tok < a.M ? a.rowsum[tok] : 0;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    bool ok = true;
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % S;
-      const uint32_t par = (kb / S) & 1;
-      if (!mbar_wait(&full[s], par)) {
+    for (int i = grp; i < total_kb; i += 2) {
+      const int s = i % S;
+      const int kb = i % KB;
+      if (!mbar_wait(&full[s], (i / S) & 1)) {
         *a.status = kDevTimeoutUnpack;
-        ok = false;
         break;
       }
       const uint8_t* st = sA + s * a_stage;
@@ -253,7 +290,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         arow = st + r * a.vbox;
         rem = (kb * 4 * a.nm_n) & 15;
       }
-      uint32_t outw[32];
       uint32_t dw[8];
       if (NM == 0) {
         const uint4 lo = reinterpret_cast<const uint4*>(arow)[0];
@@ -264,55 +300,106 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int gi = 0; gi < 8; ++gi) dw[gi] = tc_group_word<NM>(arow, mrow, gi, a.nm_n, rem);
       }
+      uint32_t outw[32];
 #pragma unroll
       for (int gi = 0; gi < 8; ++gi) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) outw[4 * gi + j] = (dw[gi] >> (2 * j)) & 0x03030303u;
       }
-      tc_st_32x32b_x32(tmem + lane_base + A_COL0 + s * 32, outw);
+      tc_st_32x32b_x32(tmem + lane_base + A_COL0 + s * kTcStageCols, outw);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&aready[s]);
     }
-    // ------------------------------------------------------------ epilogue
-    if (ok) {
-      if (!mbar_wait(accfull, 0)) {
-        *a.status = kDevTimeoutEpilogue;
-        ok = false;
+  } else if (warp >= kTcEpiWarp0) {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp - kTcEpiWarp0;       // TMEM lane quarter = 32-row block of the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t* stg = s_stage + q * 32 * 33;
+    pdl_wait_primary();
+    for (int t = 0; t < my_tiles; ++t) {
+      const int buf = t & 1;
+      int rt, tt;
+      tile_of(t, rt, tt);
+      const int row0 = rt * kTcRows + q * 32;
+      const int tok0 = tt * BN;
+      float* scl = s_scale + buf * BN;
+      int32_t* rsm = s_rowsum + buf * BN;
+      for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
+        const int tok = tok0 + j;
+        scl[j] = tok < a.M ? a.scale[tok] : 0.0f;
+        rsm[j] = tok < a.M ? a.rowsum[tok] : 0;
       }
-    }
-    tc_fence_after();
-    if (ok) {
-      const int row = row0 + r;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!mbar_wait(&accfull[buf], (t >> 1) & 1)) {
+        *a.status = kDevTimeoutEpilogue;
+        break;
+      }
+      tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
-        tc_ld_32x32b_x32(tmem + lane_base + c0, v);
+        tc_ld_32x32b_x32(tmem + lane_base + buf * DCOLS + c0, v);
         tc_wait_ld();
-        if (row < a.N) {
+        // transpose through shared memory: lane l then owns token c0 + l
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = c0 + j;
-            const int tok = tok0 + t;
-            if (t < BN && tok < a.M) {
-              const int32_t total = static_cast<int32_t>(v[j]) - s_rowsum[t];
-              const size_t o = static_cast<size_t>(tok) * a.N + row;
-              if (a.acc) a.acc[o] = total;
-              const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(total), s_scale[t]));
-              a.y[o] = *reinterpret_cast<const uint16_t*>(&h);
+        for (int j = 0; j < 32; ++j) stg[j * 33 + lane] = v[j];
+        __syncwarp();
+        const int tcol = c0 + lane;
+        const int tok = tok0 + tcol;
+        if (tcol < BN && tok < a.M) {
+          const float sc = scl[tcol];
+          const int32_t rs = rsm[tcol];
+          const size_t o = static_cast<size_t>(tok) * a.N + row0;
+          if (a.vec_store && row0 + 32 <= a.N) {
+            uint32_t hb[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int32_t t0 = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
+              const int32_t t1 = static_cast<int32_t>(stg[lane * 33 + e + 1]) - rs;
+              const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t0), sc));
+              const __nv_bfloat16 h1 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t1), sc));
+              hb[e >> 1] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h0)) |
+                           (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h1)) << 16);
+              if (a.acc) {
+                stg[lane * 33 + e] = static_cast<uint32_t>(t0);
+                stg[lane * 33 + e + 1] = static_cast<uint32_t>(t1);
+              }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.y + o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(hb[4 * e], hb[4 * e + 1], hb[4 * e + 2], hb[4 * e + 3]);
+            if (a.acc) {
+              uint4* da = reinterpret_cast<uint4*>(a.acc + o);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                da[e] = make_uint4(stg[lane * 33 + 4 * e], stg[lane * 33 + 4 * e + 1], stg[lane * 33 + 4 * e + 2],
+                                   stg[lane * 33 + 4 * e + 3]);
+            }
+          } else {
+            for (int e = 0; e < 32 && row0 + e < a.N; ++e) {
+              const int32_t tv = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
+              if (a.acc) a.acc[o + e] = tv;
+              const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), sc));
+              a.y[o + e] = *reinterpret_cast<const uint16_t*>(&h);
             }
           }
         }
+        __syncwarp();
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[buf]);
     }
-    tc_fence_before();
   }
+  tc_fence_before();
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, NCOLS);
   }
 }
+
 
 }  // namespace bl

@@ -82,7 +82,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2-D tiled load (no multicast): box at (x = innermost, y) into smem, completion
+// 2-D tiled load into this CTA: box at (x = innermost, y) into smem, completion
 // counted in bytes on bar.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar) {
@@ -186,6 +186,8 @@ __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[3
       : "r"(taddr)
       : "memory");
 }
+
+
 
 // Shared-memory matrix descriptor for a K-major operand tile written with the
 // 128-byte swizzle (rows of 128 bytes, 8-row atoms of 1024 bytes).  The tile
