@@ -4,12 +4,14 @@
 Headline (one JSON line on rank 0): decode weight GB/s of the BitNet b1.58
 2B4T feed-forward BitLinears at M = 1 token -- per step one token passes the
 gate (2560 -> 6912), up (2560 -> 6912) and down (6912 -> 2560) projections of
-every one of the 30 layers of a 2B4T-shaped stack (90 GEMV launches, 398 MB of
-2-bit weights, larger than the 126 MB L2, so every step streams its weights
-from HBM).  Weights are drawn directly in ternary form (P(0) = 0.42,
+every one of the 30 layers of a 2B4T-shaped stack (398 MB of 2-bit weights,
+larger than the 126 MB L2, so every step streams its weights from HBM).  gate
+and up share their input and run as one grouped GEMV launch, down as another:
+60 launches per step.  Weights are drawn directly in ternary form (P(0) = 0.42,
 P(+-1) = 0.29, alpha ~ U(0.01, 0.05)); x ~ N(0, 1) in bf16.  The step is
 captured once in a CUDA graph with programmatic dependent launch between the
-GEMVs.  Bytes per GEMV = N*K/4 packed codes + 4 (alpha) + 2K (x) + 2N (y).
+GEMVs.  Bytes per step = sum over matrices of N*K/4 packed codes + 4 (alpha)
++ 2N (y), plus 2K per distinct input row (x once for gate and up, h for down).
 
 A second object, "prefill", reports int8 TOPS of the tensor-core path on the
 2B4T prefill shapes (M = 2048 tokens; 2560 -> 6912, 6912 -> 2560,
@@ -51,7 +53,9 @@ def decode_bytes_per_gemv(K: int, N: int) -> int:
 
 
 def decode_step_bytes(layers: int = LAYERS) -> int:
-    return layers * sum(decode_bytes_per_gemv(K, N) for _, K, N in FFN)
+    mats = sum(N * K // 4 + 4 + 2 * N for _, K, N in FFN)
+    inputs = 2 * 2560 + 2 * 6912  # x (read once by the grouped gate/up launch) and h
+    return layers * (mats + inputs)
 
 
 # ------------------------------------------------------------------ multi-rank plumbing
@@ -229,9 +233,7 @@ def decode_step_fn(layers_w, x_in, h_in, y_gate, y_up, y_down, flags):
 
     def step():
         for l, w in enumerate(layers_w):
-            xv = x_in[l:l + 1]
-            bl.forward(w["gate"], xv, out=y_gate[l:l + 1], flags=flags)
-            bl.forward(w["up"], xv, out=y_up[l:l + 1], flags=flags)
+            bl.forward_group([w["gate"], w["up"]], x_in[l:l + 1], outs=[y_gate[l:l + 1], y_up[l:l + 1]], flags=flags)
             bl.forward(w["down"], h_in[l:l + 1], out=y_down[l:l + 1], flags=flags)
     return step
 
@@ -275,7 +277,7 @@ def run_decode(dev, steps, warmup, layers, clock_index):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         step()
-    launches_per_step = 3 * layers
+    launches_per_step = 2 * layers
     secs, clocks = time_graph(g, steps, warmup, dev, clock_index)
     assert bl.device_status() == 0
 
@@ -411,7 +413,8 @@ def main():
     world, rank, local = dist_env()
     config = {"workload": f"decode GEMV, BitNet-2B4T FFN (gate/up 2560->6912, down 6912->2560) x {args.layers} "
                           f"layers, M=1, ternary P(0)=0.42",
-              "M": 1, "layers": args.layers, "gemv_per_step": 3 * args.layers,
+              "M": 1, "layers": args.layers, "matrices_per_step": 3 * args.layers,
+              "gemv_launches_per_step": 2 * args.layers,
               "bytes_per_step": decode_step_bytes(args.layers), "l2": "weights per step exceed L2 (no reuse)",
               "parallelism": f"replicas x{world}"}
 
@@ -473,8 +476,9 @@ def main():
         return
 
     peaks, peak_kind = measured_peaks()
+    # the step holds nothing but GEMV launches: average launch = step time / launches
     per_launch = dec["secs"] / (args.steps * dec["launches_per_step"])
-    launch_bytes = decode_bytes_per_gemv(2560, 6912)
+    launch_bytes = step_bytes / dec["launches_per_step"]
     achieved = launch_bytes / per_launch / 1e9
     traffic = profiled_traffic()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",

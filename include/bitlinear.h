@@ -80,6 +80,7 @@ typedef enum bitlinear_status {
 #define BITLINEAR_MAX_K 65536       /* keeps every int32 partial sum exact */
 #define BITLINEAR_MAX_N (1 << 24)
 #define BITLINEAR_MAX_M (1 << 24)
+#define BITLINEAR_MAX_GROUP 4       /* matrices per bitlinear_forward_group call */
 
 /* Flags of bitlinear_forward / bitlinear_forward_nm. */
 #define BITLINEAR_FLAG_PDL 0x1u       /* launch as a programmatic dependent: the
@@ -168,6 +169,31 @@ bitlinear_status bitlinear_forward(const bitlinear_weights* w, const uint16_t* x
 bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
                                       int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
                                       void* stream);
+
+/* Several BitLinear layers applied to the same input, e.g. the gate and up
+ * projections of one feed-forward block, or q, k and v.  The method defines
+ * each layer on its own ("BitNet b1.58 2B4T Technical Report", section 2
+ * Architecture, BitLinear; the activation quantisation depends on x alone),
+ * so quantising x once for all of them changes no result: every y[i] equals
+ * bitlinear_forward /
+ * bitlinear_forward_nm of w[i] on x, bit for bit.  Only the launches and the
+ * repeated quantisation are saved.
+ * w        host array of count structs (1 <= count <= BITLINEAR_MAX_GROUP),
+ *          dense or N:M, all with the same K.
+ * x        device, bf16 bits [M, K] (16-byte aligned).
+ * y        host array of count device pointers, out: bf16 bits [M, w[i].N].
+ * acc      NULL, or a host array of count device pointers (each may be NULL):
+ *          int32 [M, w[i].N].
+ * workspace, workspace_bytes: bitlinear_forward_workspace_bytes(M, 0, K, flags).
+ * flags    as for bitlinear_forward; PDL applies to the first kernel the call
+ *          launches (the later ones follow kernels of the same call).
+ * Path: M == 1 runs the dense matrices in one GEMV launch (CTAs split among
+ * them by rows) and each N:M matrix in its own; M >= 2 quantises once and
+ * runs one tensor-core GEMM per matrix.
+ * Errors: as bitlinear_forward; SHAPE also for count out of range or unequal K. */
+bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,
+                                         uint16_t* const* y, int32_t* const* acc, void* workspace,
+                                         size_t workspace_bytes, uint32_t flags, void* stream);
 
 /* Largest scratch, in bytes, that bitlinear_forward_noalloc can use. */
 #define BITLINEAR_NOALLOC_SCRATCH_BYTES (8u << 20)

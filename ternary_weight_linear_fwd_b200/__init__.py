@@ -14,11 +14,12 @@ from typing import Optional
 
 __all__ = [
     "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
-    "quant_act", "forward", "forward_nm", "forward_workspace_bytes", "device_status", "last_kernel",
+    "quant_act", "forward", "forward_nm", "forward_group", "forward_workspace_bytes", "device_status", "last_kernel",
     "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC",
 ]
 
 FLAG_PDL = 0x1
+MAX_GROUP = 4
 FLAG_PATH_GEMV = 0x2
 FLAG_PATH_TC = 0x4
 
@@ -62,6 +63,7 @@ def lib() -> ctypes.CDLL:
             "bitlinear_forward_workspace_bytes": (sz, [i32, i32, i32, u32]),
             "bitlinear_forward": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
             "bitlinear_forward_nm": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
+            "bitlinear_forward_group": (st, [ctypes.POINTER(_Weights), i32, P, i32, P, P, P, sz, u32, P]),
             "bitlinear_device_status": (st, [P, ctypes.POINTER(i32), i32]),
             "bitlinear_last_kernel": (ctypes.c_char_p, []),
             "bitlinear_status_string": (ctypes.c_char_p, [st]),
@@ -190,6 +192,29 @@ def forward_nm(w: PackedWeights, x, want_acc: bool = False, flags: int = 0, work
                stream=None):
     """Same as forward for N:M packed weights."""
     return _forward(lib().bitlinear_forward_nm, "forward_nm", w, x, want_acc, flags, workspace, out, acc_out, stream)
+
+
+def forward_group(ws, x, want_acc: bool = False, flags: int = 0, workspace=None, outs=None, stream=None):
+    """BitLinear of several matrices (same K) on one input x: a list of y
+    (with want_acc, a list of (y, acc)), each identical to forward /
+    forward_nm of that matrix."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    count = len(ws)
+    M = x.shape[0]
+    ys = outs if outs is not None else [torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device) for w in ws]
+    accs = [torch.empty((M, w.N), dtype=torch.int32, device=x.device) for w in ws] if want_acc else None
+    K = ws[0].K if count else 0
+    need = forward_workspace_bytes(M, 0, K, flags) if count else 0
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    arr = (_Weights * max(count, 1))(*[w.c_struct() for w in ws])
+    yp = (ctypes.c_void_p * max(count, 1))(*[_ptr(y) for y in ys])
+    ap = (ctypes.c_void_p * max(count, 1))(*[_ptr(a) for a in accs]) if want_acc else None
+    _check(lib().bitlinear_forward_group(arr, count, _ptr(x), M, yp, ap, _ptr(workspace), ws_n, flags,
+                                         _stream(stream)), "forward_group")
+    return list(zip(ys, accs)) if want_acc else ys
 
 
 def device_status(clear: bool = True, stream=None) -> int:

@@ -178,23 +178,36 @@ const char* tc_name(int nm, int bn) {
   return names[nm][i];
 }
 
-bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
-                            void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev) {
-  const int N = w->N, K = w->K;
-  if (!ws || ws_bytes < tc_workspace(M, K) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
+// Token-side scratch of the tensor-core path: the codes in contraction order,
+// gamma and the code sums.  One quantisation serves every matrix that
+// multiplies the same x.
+struct QuantWs {
+  int8_t* q;        // [M, k16(K)]
+  float* gamma;     // [M]
+  int32_t* rowsum;  // [M]
+};
+
+QuantWs tc_ws_layout(void* ws, int M, int K) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  int8_t* qp = reinterpret_cast<int8_t*>(wsb);
-  float* scale = reinterpret_cast<float*>(wsb + align256(static_cast<size_t>(M) * k16(K)));
-  int32_t* rowsum = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(scale) + align256(4 * static_cast<size_t>(M)));
+  QuantWs r;
+  r.q = reinterpret_cast<int8_t*>(wsb);
+  r.gamma = reinterpret_cast<float*>(wsb + align256(static_cast<size_t>(M) * k16(K)));
+  r.rowsum = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(r.gamma) + align256(4 * static_cast<size_t>(M)));
+  return r;
+}
 
-  bitlinear_status st = launch(quant_act_kernel<true>, dim3(M), dim3(256), 0, s, pdl, x, M, K, static_cast<int>(k16(K)),
-                               qp, static_cast<float*>(nullptr), rowsum, w->alpha, scale);
-  if (st != BITLINEAR_OK) return st;
+bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s) {
+  return launch(quant_act_kernel<true>, dim3(M), dim3(256), 0, s, pdl, x, M, K, static_cast<int>(k16(K)), qw.q,
+                qw.gamma, qw.rowsum);
+}
 
+bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
+                         cudaStream_t s, DeviceState* dev) {
+  const int N = w->N, K = w->K;
   const int bn = pick_bn(M);
   const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? 1 : 2);
   CUtensorMap mB, mA, mMeta;
-  if (!make_map_u8(&mB, qp, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
+  if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
                    kTcBK, static_cast<uint32_t>(bn), true))
     return BITLINEAR_ERR_CUDA;
   TcArgs ta;
@@ -202,8 +215,9 @@ bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M
   ta.N = N;
   ta.K = K;
   ta.kblocks = (K + kTcBK - 1) / kTcBK;
-  ta.scale = scale;
-  ta.rowsum = rowsum;
+  ta.gamma = qw.gamma;
+  ta.alpha = w->alpha;
+  ta.rowsum = qw.rowsum;
   ta.y = y;
   ta.acc = acc;
   ta.nm_n = w->nm_n;
@@ -224,6 +238,7 @@ bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M
     if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, false)) return BITLINEAR_ERR_CUDA;
     if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16, kTcRows, false)) return BITLINEAR_ERR_CUDA;
   }
+  bitlinear_status st;
   if (nm == 0)
     st = launch_tc<0>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
   else if (nm == 1)
@@ -234,26 +249,106 @@ bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M
   return st;
 }
 
+bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
+                            void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev) {
+  if (!ws || ws_bytes < tc_workspace(M, w->K) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
+  const QuantWs qw = tc_ws_layout(ws, M, w->K);
+  bitlinear_status st = tc_quant(x, M, w->K, qw, pdl, s);
+  if (st != BITLINEAR_OK) return st;
+  return tc_gemm(w, M, qw, y, acc, s, dev);
+}
+
 // ---------------------------------------------------------------- GEMV path
 // Shared-memory budget for one CTA's weight rows in the decode GEMV: small
 // enough that the next kernel's CTA (launched early under PDL) fits beside it.
 constexpr int64_t kGemvWeightSmem = 96 * 1024;
 
-// One CTA per SM when its rows fit the shared-memory budget and a TMA box
-// (at most 256 rows), more CTAs (waves) otherwise.
-int gemv_grid(int N, int64_t ld, int C, int sm_count) {
-  int grid = std::min(sm_count, N);
-  auto fits = [&](int g) {
-    const int rows_box = N / g + 1;
-    return rows_box <= 256 && gemv_smem_bytes(rows_box, ld, C) <= static_cast<size_t>(kGemvWeightSmem) + 16 * 1024;
+// Splits about one CTA per SM over the matrices of a group in proportion to
+// their rows, then doubles every share until one CTA's rows fit the
+// shared-memory budget and a TMA box (at most 256 rows).  Returns the box
+// height; fills cta_begin, rows_base, rows_rem and the total CTA count.
+int gemv_split(GemvDense& g, const int* N, int count, int sm_count, int* grid) {
+  int64_t R = 0;
+  for (int i = 0; i < count; ++i) R += N[i];
+  int share[kGemvGroup];
+  int used = 0;
+  for (int i = 0; i < count; ++i) {
+    share[i] = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(N[i], sm_count * static_cast<int64_t>(N[i]) / R)));
+    used += share[i];
+  }
+  // hand the CTAs left over to the matrices with the most rows per CTA
+  while (used < sm_count) {
+    int best = -1;
+    for (int i = 0; i < count; ++i)
+      if (share[i] < N[i] && (best < 0 || static_cast<int64_t>(N[i]) * share[best] > static_cast<int64_t>(N[best]) * share[i]))
+        best = i;
+    if (best < 0) break;
+    ++share[best];
+    ++used;
+  }
+  auto box = [&]() {
+    int b = 0;
+    for (int i = 0; i < count; ++i) b = std::max(b, N[i] / share[i] + 1);
+    return b;
   };
-  while (!fits(grid) && grid < N) grid = std::min(N, grid * 2);
-  return grid;
+  auto fits = [&](int rows_box) {
+    return rows_box <= 256 && gemv_smem_bytes(rows_box, g.ld, g.C) <= static_cast<size_t>(kGemvWeightSmem) + 16 * 1024;
+  };
+  for (;;) {
+    if (fits(box())) break;
+    bool grew = false;
+    for (int i = 0; i < count; ++i)
+      if (share[i] < N[i]) {
+        share[i] = std::min(N[i], share[i] * 2);
+        grew = true;
+      }
+    if (!grew) break;
+  }
+  int begin = 0;
+  for (int i = 0; i < count; ++i) {
+    g.mat[i].cta_begin = begin;
+    g.mat[i].rows_base = N[i] / share[i];
+    g.mat[i].rows_rem = N[i] % share[i];
+    begin += share[i];
+  }
+  g.count = count;
+  *grid = begin;
+  return box();
+}
+
+// One launch of the dense decode GEMV over `count` matrices sharing x.
+bitlinear_status gemv_dense_launch(const bitlinear_weights* const* w, uint16_t* const* y, int32_t* const* acc,
+                                   int count, const uint16_t* x, bool pdl, cudaStream_t s, DeviceState* dev) {
+  GemvDense g;
+  std::memset(&g, 0, sizeof g);
+  const int K = w[0]->K;
+  g.ld = dense_ld(K);
+  g.C = static_cast<int>(g.ld / 16);
+  g.K = K;
+  g.x = x;
+  g.status = dev->status;
+  int N[kGemvGroup];
+  for (int i = 0; i < count; ++i) N[i] = w[i]->N;
+  int grid = 0;
+  g.rows_box = gemv_split(g, N, count, dev->sm_count, &grid);
+  for (int i = 0; i < count; ++i) {
+    g.mat[i].alpha = w[i]->alpha;
+    g.mat[i].y = y[i];
+    g.mat[i].acc = acc ? acc[i] : nullptr;
+    if (!make_map_u8(&g.map[i], w[i]->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N[i]),
+                     static_cast<uint64_t>(g.ld), 128, static_cast<uint32_t>(g.rows_box), true))
+      return BITLINEAR_ERR_CUDA;
+  }
+  const size_t smem = gemv_smem_bytes(g.rows_box, g.ld, g.C);
+  bitlinear_status st = launch(gemv_dense_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, g);
+  if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_dense";
+  return st;
 }
 
 bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uint16_t* y, int32_t* acc, bool pdl,
                               cudaStream_t s, DeviceState* dev) {
   const int N = w->N, K = w->K;
+  if (w->nm_m == 0) return gemv_dense_launch(&w, &y, &acc, 1, x, pdl, s, dev);
   GemvArgs ga;
   std::memset(&ga, 0, sizeof ga);
   ga.codes = w->codes;
@@ -266,25 +361,6 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
   ga.acc = acc;
   ga.nm_n = w->nm_n;
   ga.nm_m = w->nm_m;
-  if (w->nm_m == 0) {
-    ga.ld = dense_ld(K);
-    ga.C = static_cast<int>(ga.ld / 16);
-    ga.tpr_log2 = 0;
-    ga.passes = 1;
-    const int grid = gemv_grid(N, ga.ld, ga.C, dev->sm_count);
-    ga.rows_base = N / grid;
-    ga.rows_rem = N % grid;
-    ga.status = dev->status;
-    const int rows_box = ga.rows_base + 1;
-    CUtensorMap wmap;
-    if (!make_map_u8(&wmap, w->codes, static_cast<uint64_t>(ga.ld), static_cast<uint64_t>(N),
-                     static_cast<uint64_t>(ga.ld), 128, static_cast<uint32_t>(rows_box), true))
-      return BITLINEAR_ERR_CUDA;
-    const size_t smem = gemv_smem_bytes(rows_box, ga.ld, ga.C);
-    bitlinear_status st = launch(gemv_m1_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, wmap, ga);
-    if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_dense";
-    return st;
-  }
   int64_t ldv = 0, ldm = 0;
   if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
     return BITLINEAR_ERR_PATTERN;
@@ -307,23 +383,39 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
   return st;
 }
 
-bitlinear_status forward_common(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y, int32_t* acc,
-                                void* ws, size_t ws_bytes, uint32_t flags, void* stream, bool want_nm) {
-  if (!w || !x || !y || !w->codes || !w->alpha) return BITLINEAR_ERR_NULL;
+// Checks one matrix and its outputs (x and the flags are checked by the caller).
+bitlinear_status check_matrix(const bitlinear_weights* w, const uint16_t* y, const int32_t* acc) {
+  if (!w || !y || !w->codes || !w->alpha) return BITLINEAR_ERR_NULL;
   bitlinear_status st = check_nk(w->N, w->K);
   if (st != BITLINEAR_OK) return st;
-  if (M < 1 || M > BITLINEAR_MAX_M) return BITLINEAR_ERR_SHAPE;
   if (!pattern_ok(w->nm_n, w->nm_m)) return BITLINEAR_ERR_PATTERN;
   const bool is_nm = w->nm_m != 0;
-  if (is_nm != want_nm) return BITLINEAR_ERR_PATTERN;
-  if (is_nm && (!w->meta || w->K % w->nm_m != 0)) return is_nm && !w->meta ? BITLINEAR_ERR_NULL : BITLINEAR_ERR_SHAPE;
-  if (!aligned16(w->codes) || !aligned16(x) || (is_nm && !aligned16(w->meta))) return BITLINEAR_ERR_ALIGN;
+  if (is_nm && !w->meta) return BITLINEAR_ERR_NULL;
+  if (is_nm && w->K % w->nm_m != 0) return BITLINEAR_ERR_SHAPE;
+  if (!aligned16(w->codes) || (is_nm && !aligned16(w->meta))) return BITLINEAR_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(y) & 1u) || (acc && (reinterpret_cast<uintptr_t>(acc) & 3u)) ||
       (reinterpret_cast<uintptr_t>(w->alpha) & 3u))
     return BITLINEAR_ERR_ALIGN;
+  return BITLINEAR_OK;
+}
+
+bitlinear_status check_flags(uint32_t flags, int M) {
   const uint32_t known = BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_GEMV | BITLINEAR_FLAG_PATH_TC;
   if (flags & ~known) return BITLINEAR_ERR_FLAGS;
   if ((flags & BITLINEAR_FLAG_PATH_GEMV) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
+  return BITLINEAR_OK;
+}
+
+bitlinear_status forward_common(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y, int32_t* acc,
+                                void* ws, size_t ws_bytes, uint32_t flags, void* stream, bool want_nm) {
+  if (!w || !x || !y) return BITLINEAR_ERR_NULL;
+  bitlinear_status st = check_matrix(w, y, acc);
+  if (st != BITLINEAR_OK) return st;
+  if (M < 1 || M > BITLINEAR_MAX_M) return BITLINEAR_ERR_SHAPE;
+  if ((w->nm_m != 0) != want_nm) return BITLINEAR_ERR_PATTERN;
+  if (!aligned16(x)) return BITLINEAR_ERR_ALIGN;
+  st = check_flags(flags, M);
+  if (st != BITLINEAR_OK) return st;
   DeviceState* dev = nullptr;
   st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
@@ -332,6 +424,58 @@ bitlinear_status forward_common(const bitlinear_weights* w, const uint16_t* x, i
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || M > 1;
   if (tc) return forward_tc(w, x, M, y, acc, ws, ws_bytes, pdl, s, dev);
   return forward_gemv(w, x, y, acc, pdl, s, dev);
+}
+
+bitlinear_status forward_group(const bitlinear_weights* w, int count, const uint16_t* x, int M, uint16_t* const* y,
+                               int32_t* const* acc, void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
+  if (!w || !x || !y) return BITLINEAR_ERR_NULL;
+  if (count < 1 || count > BITLINEAR_MAX_GROUP) return BITLINEAR_ERR_SHAPE;
+  if (M < 1 || M > BITLINEAR_MAX_M) return BITLINEAR_ERR_SHAPE;
+  for (int i = 0; i < count; ++i) {
+    bitlinear_status st = check_matrix(&w[i], y[i], acc ? acc[i] : nullptr);
+    if (st != BITLINEAR_OK) return st;
+    if (w[i].K != w[0].K) return BITLINEAR_ERR_SHAPE;
+  }
+  if (!aligned16(x)) return BITLINEAR_ERR_ALIGN;
+  bitlinear_status st = check_flags(flags, M);
+  if (st != BITLINEAR_OK) return st;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  const bool pdl = (flags & BITLINEAR_FLAG_PDL) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || M > 1;
+  if (tc) {
+    if (!ws || ws_bytes < tc_workspace(M, w[0].K) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
+    const QuantWs qw = tc_ws_layout(ws, M, w[0].K);
+    st = tc_quant(x, M, w[0].K, qw, pdl, s);
+    for (int i = 0; i < count && st == BITLINEAR_OK; ++i) st = tc_gemm(&w[i], M, qw, y[i], acc ? acc[i] : nullptr, s, dev);
+    return st;
+  }
+  // decode: the dense matrices share one launch; each N:M matrix has its own
+  const bitlinear_weights* dw[kGemvGroup];
+  uint16_t* dy[kGemvGroup];
+  int32_t* dacc[kGemvGroup];
+  int nd = 0;
+  for (int i = 0; i < count; ++i)
+    if (w[i].nm_m == 0) {
+      dw[nd] = &w[i];
+      dy[nd] = y[i];
+      dacc[nd] = acc ? acc[i] : nullptr;
+      ++nd;
+    }
+  bool first = true;
+  if (nd) {
+    st = gemv_dense_launch(dw, dy, dacc, nd, x, pdl, s, dev);
+    first = false;
+  }
+  for (int i = 0; i < count && st == BITLINEAR_OK; ++i)
+    if (w[i].nm_m != 0) {
+      // a later kernel of the group may start early: it reads only its weights before waiting
+      st = forward_gemv(&w[i], x, y[i], acc ? acc[i] : nullptr, first ? pdl : true, s, dev);
+      first = false;
+    }
+  return st;
 }
 
 }  // namespace
@@ -440,7 +584,7 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
   st = launch(quant_act_kernel<false>, dim3(M), dim3(256), 0, static_cast<cudaStream_t>(stream), false, x, M, K, K, q,
-              gamma, rowsum, static_cast<const float*>(nullptr), static_cast<float*>(nullptr));
+              gamma, rowsum);
   if (st == BITLINEAR_OK) t_last_kernel = "quant_act";
   return st;
 }
@@ -450,6 +594,12 @@ size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32
   if (M < 1 || K < 1) return 0;
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || (M > 1 && !(flags & BITLINEAR_FLAG_PATH_GEMV));
   return tc ? tc_workspace(M, K) : 0;
+}
+
+bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,
+                                         uint16_t* const* y, int32_t* const* acc, void* workspace,
+                                         size_t workspace_bytes, uint32_t flags, void* stream) {
+  return forward_group(w, count, x, M, y, acc, workspace, workspace_bytes, flags, stream);
 }
 
 bitlinear_status bitlinear_forward(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,

@@ -49,7 +49,8 @@ struct TcArgs {
   int M, N, K;
   int kblocks;            // ceil(K / 128)
   int row_tiles, tok_tiles;
-  const float* scale;     // [M] per-token rescale RN(RN(alpha * gamma) / 127)
+  const float* gamma;     // [M] per-token absmax
+  const float* alpha;     // the matrix's absmean scale (device)
   const int32_t* rowsum;  // [M] sum of the token's codes
   uint16_t* y;            // [M, N] bf16 bits
   int32_t* acc;           // [M, N] or null
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp - kTcEpiWarp0;       // TMEM lane quarter = 32-row block of the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     uint32_t* stg = s_stage + q * 32 * 33;
+    const float alpha = *a.alpha;
     pdl_wait_primary();
     for (int t = 0; t < my_tiles; ++t) {
       const int buf = t & 1;
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int32_t* rsm = s_rowsum + buf * BN;
       for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
         const int tok = tok0 + j;
-        scl[j] = tok < a.M ? a.scale[tok] : 0.0f;
+        scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), kQb) : 0.0f;  // RN(RN(alpha gamma) / 127)
         rsm[j] = tok < a.M ? a.rowsum[tok] : 0;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");

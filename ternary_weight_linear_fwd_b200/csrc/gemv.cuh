@@ -131,8 +131,9 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = mx;
   __syncthreads();
-  mx = 0.0f;
-  for (int i = 0; i < (nthr >> 5); ++i) mx = fmaxf(mx, s_red[i]);
+  mx = (threadIdx.x & 31) < (nthr >> 5) ? s_red[threadIdx.x & 31] : 0.0f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   const float d = __fadd_rn(mx, kEps);
   const float c = __fmul_rn(kQb, __frcp_rn(d));
   const int quarter = groups_alloc >> 2;
@@ -173,10 +174,10 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
   return mx;
 }
 
-__device__ __forceinline__ void gemv_store(const GemvArgs& a, int row, int32_t total, float s) {
-  if (a.acc) a.acc[row] = total;
+__device__ __forceinline__ void gemv_store(uint16_t* y, int32_t* acc, int row, int32_t total, float s) {
+  if (acc) acc[row] = total;
   const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(total), s));
-  a.y[row] = *reinterpret_cast<const uint16_t*>(&h);
+  y[row] = *reinterpret_cast<const uint16_t*>(&h);
 }
 
 __device__ __forceinline__ int32_t group_sum(int32_t v, int tpr) {
@@ -212,32 +213,67 @@ __host__ __device__ __forceinline__ size_t gemv_smem_bytes(int rows_box, int64_t
          static_cast<size_t>(C) * 4 * 16 + static_cast<size_t>(C) * 4 + static_cast<size_t>(rows_box) * 4;
 }
 
-// Partial sum of one unit: row r, chunk ch, minus the chunk's share of sum(q).
-__device__ __forceinline__ int32_t gemv_unit(const uint8_t* s_w, int stripe_bytes, const uint4* s_act,
-                                             const int32_t* s_csum, int C, int r, int ch) {
-  const uint4 wv = *reinterpret_cast<const uint4*>(s_w + (ch >> 3) * stripe_bytes + r * 128 +
-                                                   (((ch & 7) ^ (r & 7)) << 4));
+// Partial sums of one unit: chunk ch of rows r and r2 (r2 < 0: none), each minus
+// the chunk's share of sum(q); the activation words are loaded once for both.
+__device__ __forceinline__ void gemv_unit2(const uint8_t* s_w, int stripe_bytes, const uint4* s_act,
+                                           const int32_t* s_csum, int C, int r, int r2, int ch, int32_t& p1,
+                                           int32_t& p2) {
+  const uint8_t* stripe = s_w + (ch >> 3) * stripe_bytes;
+  const uint4 wa = *reinterpret_cast<const uint4*>(stripe + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+  const uint4 wb = r2 >= 0 ? *reinterpret_cast<const uint4*>(stripe + r2 * 128 + (((ch & 7) ^ (r2 & 7)) << 4))
+                           : make_uint4(0u, 0u, 0u, 0u);
   const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
-  int32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-  dot_word(wv.x, q0.x, q0.y, q0.z, q0.w, s0, s1, s2, s3);
-  dot_word(wv.y, q1.x, q1.y, q1.z, q1.w, s0, s1, s2, s3);
-  dot_word(wv.z, q2.x, q2.y, q2.z, q2.w, s0, s1, s2, s3);
-  dot_word(wv.w, q3.x, q3.y, q3.z, q3.w, s0, s1, s2, s3);
-  return s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6) - s_csum[ch];
+  const int32_t cs = s_csum[ch];
+  int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
+  dot_word(wa.x, q0.x, q0.y, q0.z, q0.w, a0, a1, a2, a3);
+  dot_word(wb.x, q0.x, q0.y, q0.z, q0.w, b0, b1, b2, b3);
+  dot_word(wa.y, q1.x, q1.y, q1.z, q1.w, a0, a1, a2, a3);
+  dot_word(wb.y, q1.x, q1.y, q1.z, q1.w, b0, b1, b2, b3);
+  dot_word(wa.z, q2.x, q2.y, q2.z, q2.w, a0, a1, a2, a3);
+  dot_word(wb.z, q2.x, q2.y, q2.z, q2.w, b0, b1, b2, b3);
+  dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
+  dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
+  p1 = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6) - cs;
+  p2 = b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6) - cs;
 }
 
-__global__ void __launch_bounds__(kGemvThreads) gemv_m1_kernel(const __grid_constant__ CUtensorMap wmap,
-                                                               const GemvArgs a) {
+// Up to kGemvGroup matrices that multiply the same activation row (and have
+// the same K) run in one launch: CTAs [cta_begin, next cta_begin) belong to
+// one matrix.  Each CTA quantises x for itself, so grouping saves the launches
+// and the repeated quantisation, and changes no result.
+constexpr int kGemvGroup = 4;
+
+struct GemvMat {
+  const float* alpha;
+  uint16_t* y;       // [N]
+  int32_t* acc;      // [N] or null
+  int rows_base, rows_rem;  // local CTA b owns rows_base (+1 if b < rows_rem) consecutive rows
+  int cta_begin;
+};
+
+struct __align__(64) GemvDense {
+  CUtensorMap map[kGemvGroup];  // per matrix: uint8 [N, ld], box {128, rows_box}, 128-byte swizzle
+  GemvMat mat[kGemvGroup];
+  const uint16_t* x;  // one bf16 row [K]
+  int32_t* status;
+  int64_t ld;
+  int K, C, rows_box, count;
+};
+
+__global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_constant__ GemvDense g) {
   extern __shared__ uint8_t s_raw[];
   __shared__ uint64_t s_bar;
   __shared__ float s_red[32];
   pdl_launch_dependents();
-  const int b = blockIdx.x;
-  const int r0 = b * a.rows_base + min(b, a.rows_rem);
-  const int nrows = a.rows_base + (b < a.rows_rem ? 1 : 0);
-  const int C = a.C;
-  const int rows_box = a.rows_base + 1;
-  const int stripes = gemv_stripes(a.ld);
+  int mi = 0;
+  while (mi + 1 < g.count && static_cast<int>(blockIdx.x) >= g.mat[mi + 1].cta_begin) ++mi;
+  const GemvMat& mt = g.mat[mi];
+  const int b = blockIdx.x - mt.cta_begin;
+  const int r0 = b * mt.rows_base + min(b, mt.rows_rem);
+  const int nrows = mt.rows_base + (b < mt.rows_rem ? 1 : 0);
+  const int C = g.C;
+  const int rows_box = g.rows_box;
+  const int stripes = gemv_stripes(g.ld);
   const int stripe_bytes = gemv_stripe_bytes(rows_box);
   uint8_t* s_w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_raw) + 1023) & ~uintptr_t(1023));
   uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
@@ -249,49 +285,44 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_m1_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     mbar_init(&s_bar, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&wmap);
+    tma_prefetch_desc(&g.map[mi]);
     mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box));
-    for (int st = 0; st < stripes; ++st) tma_load_2d(s_w + st * stripe_bytes, &wmap, st * 128, r0, &s_bar);
+    for (int st = 0; st < stripes; ++st) tma_load_2d(s_w + st * stripe_bytes, &g.map[mi], st * 128, r0, &s_bar);
   }
-  const float alpha = *a.alpha;
+  const float alpha = *mt.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
   __syncthreads();
 
   pdl_wait_primary();  // x may come from the preceding kernel
-  const float gamma = quantise_row_smem(a.x, a.K, 4 * C, s_act, s_csum, s_red);
+  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_csum, s_red);
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
-  if (!landed && threadIdx.x == 0) *a.status = kDevTimeoutProducer;
+  if (!landed && threadIdx.x == 0) *g.status = kDevTimeoutProducer;
 
   if (landed) {
+    // units: (chunk, row pair), row pair fastest; pair p covers rows p and p + half
     const int nthr = blockDim.x;
-    const int total = nrows * C;
-    const int dq = (2 * nthr) / nrows, dr = (2 * nthr) % nrows;
-    int ch = threadIdx.x / nrows, r = threadIdx.x % nrows;                      // unit u
-    int ch2 = (threadIdx.x + nthr) / nrows, r2 = (threadIdx.x + nthr) % nrows;  // unit u + nthr
-    for (int u = threadIdx.x; u < total; u += 2 * nthr) {
-      const bool vb = u + nthr < total;
-      const int32_t pa = gemv_unit(s_w, stripe_bytes, s_act, s_csum, C, r, ch);
-      const int32_t pb = vb ? gemv_unit(s_w, stripe_bytes, s_act, s_csum, C, r2, ch2) : 0;
-      atomicAdd(&s_acc[r], pa);
-      if (vb) atomicAdd(&s_acc[r2], pb);
-      r += dr;
+    const int half = (nrows + 1) >> 1;
+    const int total = half * C;
+    const int dq = nthr / half, dr = nthr % half;
+    int ch = threadIdx.x / half, p = threadIdx.x % half;
+    for (int u = threadIdx.x; u < total; u += nthr) {
+      const int r2 = p + half < nrows ? p + half : -1;
+      int32_t p1, p2;
+      gemv_unit2(s_w, stripe_bytes, s_act, s_csum, C, p, r2, ch, p1, p2);
+      atomicAdd(&s_acc[p], p1);
+      if (r2 >= 0) atomicAdd(&s_acc[r2], p2);
+      p += dr;
       ch += dq;
-      if (r >= nrows) {
-        r -= nrows;
+      if (p >= half) {
+        p -= half;
         ++ch;
-      }
-      r2 += dr;
-      ch2 += dq;
-      if (r2 >= nrows) {
-        r2 -= nrows;
-        ++ch2;
       }
     }
   }
   __syncthreads();
   if (landed)
-    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a, r0 + rr, s_acc[rr], s);
+    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr], s);
 }
 
 // ------------------------------------------------------------------ N:M M = 1
@@ -406,7 +437,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_m1_kernel(const GemvArgs
     }
     int32_t part = s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6) - qsum;
     part = group_sum(part, tpr);
-    if (valid && sub == 0) gemv_store(a, r0 + lr, part, s);
+    if (valid && sub == 0) gemv_store(a.y, a.acc, r0 + lr, part, s);
   }
 }
 

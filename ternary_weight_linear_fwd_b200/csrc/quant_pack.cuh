@@ -93,13 +93,12 @@ __device__ __forceinline__ void permute16(const int32_t (&c)[16], uint32_t (&out
 // ----------------------------------------------------------------- quant_act
 // One CTA per token row.  kPermute = false writes natural-order codes [M, ldq]
 // (ldq = K); kPermute = true writes the contraction order [M, ldq] with ldq =
-// K rounded up to 16 (zeros past K) and, when alpha is given, the per-token
-// rescale s = RN(RN(alpha * gamma) / 127).
+// K rounded up to 16 (zeros past K).  Both write gamma and, when asked, the
+// sum of the row's codes.
 template <bool kPermute>
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K, int ldq,
                                                         int8_t* __restrict__ q, float* __restrict__ gamma,
-                                                        int32_t* __restrict__ rowsum, const float* __restrict__ alpha,
-                                                        float* __restrict__ scale) {
+                                                        int32_t* __restrict__ rowsum) {
   __shared__ float redf[32];
   __shared__ int32_t redi[32];
   pdl_wait_primary();
@@ -159,7 +158,6 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   if (threadIdx.x == 0) {
     if (gamma) gamma[row] = mx;
     if (rowsum) rowsum[row] = sum;
-    if (scale) scale[row] = __fdiv_rn(__fmul_rn(*alpha, mx), kQb);
   }
 }
 

@@ -114,3 +114,25 @@ def test_workspace_sizes(L):
     assert L.bitlinear_forward_workspace_bytes(1, 6912, 2560, 0x4) >= 2560     # forced tensor-core path
     assert L.bitlinear_forward_workspace_bytes(2048, 6912, 2560, 0) >= 2048 * 2560 + 2 * 4 * 2048
     assert L.bitlinear_pack_workspace_bytes(6912, 2560) >= 8 * 1024
+
+
+def test_forward_group_host_checks(L):
+    """Group-specific argument errors (fake, never dereferenced addresses)."""
+    import ternary_weight_linear_fwd_b200 as bl
+    fg = L.bitlinear_forward_group
+    x = 0x30000
+    ws = (bl._Weights * 5)(*[_w(L) for _ in range(5)])
+    ys = (ctypes.c_void_p * 5)(*[0x40000 + 0x1000 * i for i in range(5)])
+    assert fg(None, 1, x, 1, ys, None, None, 0, 0, None) == 1
+    assert fg(ws, 1, x, 1, None, None, None, 0, 0, None) == 1
+    assert fg(ws, 0, x, 1, ys, None, None, 0, 0, None) == 2                      # empty group
+    assert fg(ws, 5, x, 1, ys, None, None, 0, 0, None) == 2                      # above MAX_GROUP
+    bad_k = (bl._Weights * 2)(_w(L), _w(L, K=512))
+    assert fg(bad_k, 2, x, 1, ys, None, None, 0, 0, None) == 2                   # unequal K
+    bad_a = (bl._Weights * 2)(_w(L), _w(L, codes=0x10008))
+    assert fg(bad_a, 2, x, 1, ys, None, None, 0, 0, None) == 3
+    bad_p = (bl._Weights * 2)(_w(L), _w(L, n=3, m=4, meta=0x50000))
+    assert fg(bad_p, 2, x, 1, ys, None, None, 0, 0, None) == 4
+    nometa = (bl._Weights * 2)(_w(L), _w(L, n=2, m=4))
+    assert fg(nometa, 2, x, 1, ys, None, None, 0, 0, None) == 1
+    assert fg(ws, 2, x, 2, ys, None, None, 0, 0x2, None) == 8                    # GEMV path needs M == 1

@@ -244,6 +244,64 @@ def test_forward_nm_m1_forced_tc_matches_gemv():
     _check_rows(x, Wt, a, y1, acc1, np.arange(1))
 
 
+# ---------------------------------------------------------------- grouped forward
+
+@pytest.mark.parametrize("M", [1, 37])
+@pytest.mark.parametrize("shapes", [((2560, 6912), (2560, 6912)), ((640, 1000), (640, 33), (640, 512), (640, 2048)),
+                                    ((6912, 2560),)])
+def test_forward_group_dense_matches_single_and_oracle(M, shapes):
+    """gate + up of the 2B4T FFN (and a ragged 4-matrix group): each output equals the single-matrix call
+    bit for bit and the oracle within the bf16 tolerance."""
+    K = shapes[0][0]
+    x = synth.activations(M, K, seed=31)
+    xd = to_dev_bf16(x)
+    cases = []
+    for i, (_, N) in enumerate(shapes):
+        T = synth.ternary_weights(N, K, seed=40 + i)
+        a = synth.alpha_uniform(40 + i)
+        cases.append((T, np.float32(a), bl.pack_ternary(torch.from_numpy(T).to(DEV), float(a))))
+    outs = bl.forward_group([c[2] for c in cases], xd, want_acc=True)
+    if M == 1:
+        assert bl.last_kernel() == "gemv_m1_dense"
+    rows = np.arange(M)
+    for (T, a, w), (y, acc) in zip(cases, outs):
+        y1, acc1 = bl.forward(w, xd, want_acc=True)
+        assert torch.equal(acc, acc1) and torch.equal(y.view(torch.int16), y1.view(torch.int16))
+        _check_rows(x, T, a, y, acc, rows)
+
+
+def test_forward_group_mixed_dense_nm():
+    K = 1024
+    x = synth.activations(1, K, seed=33)
+    xd = to_dev_bf16(x)
+    specs = [(300, 0, 0), (200, 2, 4), (130, 6, 8)]
+    ws, refs = [], []
+    for i, (N, n, m) in enumerate(specs):
+        W = synth.latent_weights(N, K, seed=50 + i)
+        refs.append(oracle.pack_weights(W, n, m))
+        ws.append(bl.pack_weights(torch.from_numpy(W).to(DEV), n, m))
+    for flags in (0, bl.FLAG_PDL, bl.FLAG_PATH_TC):
+        outs = bl.forward_group(ws, xd, want_acc=True, flags=flags)
+        for ref, (y, acc) in zip(refs, outs):
+            _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(1))
+
+
+def test_forward_group_prefill_sampled():
+    """gate + up at M = 2048 through one quantisation and two tensor-core GEMMs (sampled tokens)."""
+    M, K, N = 2048, 2560, 6912
+    x = synth.activations(M, K, seed=34)
+    xd = to_dev_bf16(x)
+    cases = []
+    for i in range(2):
+        T = synth.ternary_weights(N, K, seed=60 + i)
+        a = synth.alpha_uniform(60 + i)
+        cases.append((T, np.float32(a), bl.pack_ternary(torch.from_numpy(T).to(DEV), float(a))))
+    outs = bl.forward_group([c[2] for c in cases], xd, want_acc=True)
+    rows = np.unique(np.concatenate([[0, M - 1], synth.splitmix64(34, 9, 14) % M])).astype(np.int64)
+    for (T, a, w), (y, acc) in zip(cases, outs):
+        _check_rows(x, T, a, y, acc, rows)
+
+
 def test_status_word_clean():
     torch.cuda.synchronize()
     assert bl.device_status(clear=False) == 0
