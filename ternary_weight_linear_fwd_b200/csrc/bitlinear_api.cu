@@ -331,16 +331,19 @@ bitlinear_status gemv_dense_launch(const bitlinear_weights* const* w, uint16_t* 
   for (int i = 0; i < count; ++i) N[i] = w[i]->N;
   int grid = 0;
   g.rows_box = gemv_split(g, N, count, dev->sm_count, &grid);
+  CUtensorMap map[kGemvGroup];
   for (int i = 0; i < count; ++i) {
     g.mat[i].alpha = w[i]->alpha;
     g.mat[i].y = y[i];
     g.mat[i].acc = acc ? acc[i] : nullptr;
-    if (!make_map_u8(&g.map[i], w[i]->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N[i]),
+    if (!make_map_u8(&map[i], w[i]->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N[i]),
                      static_cast<uint64_t>(g.ld), 128, static_cast<uint32_t>(g.rows_box), true))
       return BITLINEAR_ERR_CUDA;
   }
+  for (int i = count; i < kGemvGroup; ++i) map[i] = map[0];  // never selected
   const size_t smem = gemv_smem_bytes(g.rows_box, g.ld, g.C);
-  bitlinear_status st = launch(gemv_dense_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, g);
+  bitlinear_status st =
+      launch(gemv_dense_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, map[0], map[1], map[2], map[3], g);
   if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_dense";
   return st;
 }
@@ -377,7 +380,7 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
   grid = std::max(grid, 1);
   ga.rows_base = N / grid;
   ga.rows_rem = N % grid;
-  const size_t smem = static_cast<size_t>(ga.C) * 8 * (16 + 4);
+  const size_t smem = static_cast<size_t>(ga.C) * 8 * (16 + 8);  // codes + half sums
   bitlinear_status st = launch(gemv_nm_m1_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, ga);
   if (st == BITLINEAR_OK) t_last_kernel = w->nm_m == 4 ? "gemv_m1_nm24" : "gemv_m1_n8";
   return st;

@@ -122,7 +122,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int B_STAGE = BN * 128;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // offset arithmetic on the shared array keeps every derived pointer in the shared window
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int a_val_bytes = TcStageBytes<NM>::a_values(a.vbox);
   const int a_meta_bytes = TcStageBytes<NM>::a_meta();
   const int a_stage = tc_a_stage_bytes(NM, a.vbox);

@@ -4,13 +4,13 @@
 // The 2B4T report (section 5.1, GPU Inference) moves packed ternary weights
 // from HBM on chip, unpacks them and combines them with 8-bit activations;
 // for one token the contraction is bound by those weight bytes.  Here every
-// CTA first hands its contiguous weight rows to the bulk-copy engine
-// (cp.async.bulk into shared memory, before griddepcontrol.wait, so under
+// CTA first hands its contiguous weight rows to the tensor-copy engine (TMA
+// tile loads into shared memory, issued before griddepcontrol.wait, so under
 // programmatic dependent launch the copy overlaps the preceding kernel), then
 // quantises the single activation row into shared memory (gamma, codes in
-// contraction order, per-group code sums) while the copy lands.  A lane owns
-// a fixed set of 64-weight chunks of a row; its activation codes for those
-// chunks stay in registers for every row it visits.  With code = W_t + 1:
+// contraction order, per-chunk code sums) while the copy lands, and finally
+// splits the (64-weight chunk, row) products evenly over all its threads.
+// With code = W_t + 1:
 //     acc = sum_k q_k * W_t,k = sum_k q_k * code_k - sum_k q_k
 // and sum_k q_k * code_k is formed four bytes at a time with an unsigned x
 // signed dp4a on (word & (3 << 2j) per byte), whose partial sums carry a
@@ -91,16 +91,15 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 // 16g + 4b + j), for g < groups_alloc (zero past K), where
 // slot(g) = (g % 4) * (groups_alloc / 4) + g / 4 puts the four groups of one
 // 64-weight chunk a quarter of the array apart, so lanes reading consecutive
-// chunks hit consecutive 16-byte words; s_csum[ch] is the sum of the 64 codes
-// of chunk ch.  Each thread handles 8-element halves h = tid, tid + nthr, ...:
-// one 16-byte load, 8 codes, four 16-bit stores (bytes 2*(h%2), 2*(h%2)+1 of
-// words 0..3); the 8 halves of a chunk sit in adjacent lanes and add their code
-// sums with three shuffles.  One barrier publishes the per-warp maxima, one the
-// codes.  Returns gamma = max |x|.
+// chunks hit consecutive 16-byte words; s_hsum[h] is the sum of the 8 codes of
+// half h (chunk_sum adds the eight of a chunk).  Each thread handles 8-element
+// halves h = tid, tid + nthr, ...: one 16-byte load, 8 codes, four 16-bit
+// stores (bytes 2*(h%2), 2*(h%2)+1 of words 0..3) and its code sum.  One
+// barrier publishes the per-warp maxima, one the codes.  Returns gamma = max |x|.
 constexpr int kHalvesInRegs = 2;  // halves per thread kept in registers (K <= 8192 at 512 threads)
 
 __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ x, int K, int groups_alloc,
-                                                   uint4* s_act, int32_t* s_csum, float* s_red) {
+                                                   uint4* s_act, int32_t* s_hsum, float* s_red) {
   const bool vec_ok = (K % 8) == 0;
   const int nthr = blockDim.x;
   const int halves = (K + 7) / 8;
@@ -127,29 +126,23 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
     for (int i = 0; i < 4; ++i)
       mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(t[i] << 16)), fabsf(__uint_as_float(t[i] & 0xFFFF0000u))));
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  // |x| >= 0, whose bit patterns order like the values: one integer warp reduction
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
   if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = mx;
   __syncthreads();
   mx = (threadIdx.x & 31) < (nthr >> 5) ? s_red[threadIdx.x & 31] : 0.0f;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
   const float d = __fadd_rn(mx, kEps);
   const float c = __fmul_rn(kQb, __frcp_rn(d));
   const int quarter = groups_alloc >> 2;
-  // every lane runs the same number of trips, so every lane reaches the shuffle
   auto emit = [&](const uint32_t (&raw)[4], int h) {
     uint32_t b[8];
     codes8(raw, c, d, b);
     const uint32_t lo = __byte_perm(b[0], b[1], 0x0040), hi = __byte_perm(b[2], b[3], 0x0040);
     const uint32_t lo2 = __byte_perm(b[4], b[5], 0x0040), hi2 = __byte_perm(b[6], b[7], 0x0040);
     const uint32_t p0 = __byte_perm(lo, hi, 0x5410), p1 = __byte_perm(lo2, hi2, 0x5410);  // codes 0..3, 4..7
-    int32_t gs = __dp4a(static_cast<int>(p0), 0x01010101, 0);
-    gs = __dp4a(static_cast<int>(p1), 0x01010101, gs);
-    gs += __shfl_xor_sync(0xffffffffu, gs, 1);
-    gs += __shfl_xor_sync(0xffffffffu, gs, 2);
-    gs += __shfl_xor_sync(0xffffffffu, gs, 4);
     if (h < halves_alloc) {
+      s_hsum[h] = __dp4a(static_cast<int>(p1), 0x01010101, __dp4a(static_cast<int>(p0), 0x01010101, 0));
       const int g = h >> 1, half = h & 1;
       const int sl = (g & 3) * quarter + (g >> 2);
       uint16_t* dst = reinterpret_cast<uint16_t*>(s_act + sl) + half;
@@ -158,7 +151,6 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
       dst[2] = static_cast<uint16_t>(__byte_perm(b[1], b[5], 0x0040));
       dst[4] = static_cast<uint16_t>(__byte_perm(b[2], b[6], 0x0040));
       dst[6] = static_cast<uint16_t>(__byte_perm(b[3], b[7], 0x0040));
-      if ((h & 7) == 0) s_csum[h >> 3] = gs;
     }
   };
 #pragma unroll
@@ -180,6 +172,13 @@ __device__ __forceinline__ void gemv_store(uint16_t* y, int32_t* acc, int row, i
   y[row] = *reinterpret_cast<const uint16_t*>(&h);
 }
 
+// Sum of the 64 codes of chunk ch (eight half sums; s_hsum 16-byte aligned).
+__device__ __forceinline__ int32_t chunk_sum(const int32_t* s_hsum, int ch) {
+  const int4 a = reinterpret_cast<const int4*>(s_hsum)[2 * ch];
+  const int4 b = reinterpret_cast<const int4*>(s_hsum)[2 * ch + 1];
+  return (a.x + a.y) + (a.z + a.w) + ((b.x + b.y) + (b.z + b.w));
+}
+
 __device__ __forceinline__ int32_t group_sum(int32_t v, int tpr) {
   for (int o = tpr >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
@@ -198,43 +197,23 @@ __device__ __forceinline__ void dot_word(uint32_t wd, uint32_t a0, uint32_t a1, 
 // A CTA owns a contiguous range of rows.  One thread issues one TMA tile load
 // per 128-byte stripe of those rows (box {128 bytes, rows}) with the 128-byte
 // swizzle, so chunk ch of row r sits at stripe ch / 8, line r, 16-byte slot
-// (ch % 8) ^ (r % 8): lanes reading one chunk of consecutive rows, or
-// consecutive chunks of one row, never share a bank.  The contraction is a
-// flat list of (chunk, row) units, row fastest, spread evenly over all
-// threads, two units per thread and step; a unit is one 64-weight chunk of
-// one row and adds its partial sum (minus the chunk's share of sum(q)) into
-// the row's shared accumulator.
+// (ch % 8) ^ (r % 8): lanes reading one chunk of consecutive rows never share
+// a bank.  The contraction is a flat list of (chunk, row pair) units, row pair
+// fastest, spread evenly over all threads; a unit is one 64-weight chunk of
+// two rows and adds its partial sums (minus the chunk's share of sum(q)) into
+// the rows' shared accumulators.
 
 __host__ __device__ __forceinline__ int gemv_stripes(int64_t ld) { return static_cast<int>((ld + 127) / 128); }
 __host__ __device__ __forceinline__ int gemv_stripe_bytes(int rows_box) { return (rows_box * 128 + 1023) & ~1023; }
 
 __host__ __device__ __forceinline__ size_t gemv_smem_bytes(int rows_box, int64_t ld, int C) {
   return 1024 /* alignment */ + static_cast<size_t>(gemv_stripes(ld)) * gemv_stripe_bytes(rows_box) +
-         static_cast<size_t>(C) * 4 * 16 + static_cast<size_t>(C) * 4 + static_cast<size_t>(rows_box) * 4;
+         static_cast<size_t>(C) * 4 * 16 + static_cast<size_t>(C) * 8 * 4 + static_cast<size_t>(rows_box) * 4;
 }
 
-// Partial sums of one unit: chunk ch of rows r and r2 (r2 < 0: none), each minus
-// the chunk's share of sum(q); the activation words are loaded once for both.
-__device__ __forceinline__ void gemv_unit2(const uint8_t* s_w, int stripe_bytes, const uint4* s_act,
-                                           const int32_t* s_csum, int C, int r, int r2, int ch, int32_t& p1,
-                                           int32_t& p2) {
-  const uint8_t* stripe = s_w + (ch >> 3) * stripe_bytes;
-  const uint4 wa = *reinterpret_cast<const uint4*>(stripe + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
-  const uint4 wb = r2 >= 0 ? *reinterpret_cast<const uint4*>(stripe + r2 * 128 + (((ch & 7) ^ (r2 & 7)) << 4))
-                           : make_uint4(0u, 0u, 0u, 0u);
-  const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
-  const int32_t cs = s_csum[ch];
-  int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
-  dot_word(wa.x, q0.x, q0.y, q0.z, q0.w, a0, a1, a2, a3);
-  dot_word(wb.x, q0.x, q0.y, q0.z, q0.w, b0, b1, b2, b3);
-  dot_word(wa.y, q1.x, q1.y, q1.z, q1.w, a0, a1, a2, a3);
-  dot_word(wb.y, q1.x, q1.y, q1.z, q1.w, b0, b1, b2, b3);
-  dot_word(wa.z, q2.x, q2.y, q2.z, q2.w, a0, a1, a2, a3);
-  dot_word(wb.z, q2.x, q2.y, q2.z, q2.w, b0, b1, b2, b3);
-  dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
-  dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
-  p1 = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6) - cs;
-  p2 = b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6) - cs;
+// Weight chunk ch of local row r in the swizzled stripes.
+__device__ __forceinline__ uint4 gemv_wchunk(const uint8_t* s_w, int stripe_bytes, int r, int ch) {
+  return *reinterpret_cast<const uint4*>(s_w + (ch >> 3) * stripe_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
 }
 
 // Up to kGemvGroup matrices that multiply the same activation row (and have
@@ -251,8 +230,7 @@ struct GemvMat {
   int cta_begin;
 };
 
-struct __align__(64) GemvDense {
-  CUtensorMap map[kGemvGroup];  // per matrix: uint8 [N, ld], box {128, rows_box}, 128-byte swizzle
+struct GemvDense {
   GemvMat mat[kGemvGroup];
   const uint16_t* x;  // one bf16 row [K]
   int32_t* status;
@@ -260,14 +238,26 @@ struct __align__(64) GemvDense {
   int K, C, rows_box, count;
 };
 
-__global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_constant__ GemvDense g) {
+// The tensor maps (per matrix: uint8 [N, ld], box {128, rows_box}, 128-byte
+// swizzle) are separate kernel parameters, and every parameter is read at a
+// fixed offset: the matrix of this CTA is selected into registers.
+__global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_constant__ CUtensorMap map0,
+                                                                  const __grid_constant__ CUtensorMap map1,
+                                                                  const __grid_constant__ CUtensorMap map2,
+                                                                  const __grid_constant__ CUtensorMap map3,
+                                                                  const GemvDense g) {
   extern __shared__ uint8_t s_raw[];
   __shared__ uint64_t s_bar;
   __shared__ float s_red[32];
-  pdl_launch_dependents();
   int mi = 0;
-  while (mi + 1 < g.count && static_cast<int>(blockIdx.x) >= g.mat[mi + 1].cta_begin) ++mi;
-  const GemvMat& mt = g.mat[mi];
+#pragma unroll
+  for (int i = 1; i < kGemvGroup; ++i)
+    if (i < g.count && static_cast<int>(blockIdx.x) >= g.mat[i].cta_begin) mi = i;
+  GemvMat mt = g.mat[0];
+#pragma unroll
+  for (int i = 1; i < kGemvGroup; ++i)
+    if (i == mi) mt = g.mat[i];
+  const CUtensorMap* map = mi == 0 ? &map0 : mi == 1 ? &map1 : mi == 2 ? &map2 : &map3;
   const int b = blockIdx.x - mt.cta_begin;
   const int r0 = b * mt.rows_base + min(b, mt.rows_rem);
   const int nrows = mt.rows_base + (b < mt.rows_rem ? 1 : 0);
@@ -275,43 +265,61 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   const int rows_box = g.rows_box;
   const int stripes = gemv_stripes(g.ld);
   const int stripe_bytes = gemv_stripe_bytes(rows_box);
-  uint8_t* s_w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_raw) + 1023) & ~uintptr_t(1023));
+  // offset arithmetic on the shared array keeps every derived pointer in the shared window
+  uint8_t* s_w = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
   uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
-  int32_t* s_csum = reinterpret_cast<int32_t*>(s_act + 4 * C);
-  int32_t* s_acc = s_csum + C;
+  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_act + 4 * C);  // 8 * C half sums
+  int32_t* s_acc = s_hsum + 8 * C;
 
   // The weights (and alpha, which belongs to them) do not depend on the
   // preceding kernel: their copies start first.
   if (threadIdx.x == 0) {
     mbar_init(&s_bar, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&g.map[mi]);
+    tma_prefetch_desc(map);
     mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box));
-    for (int st = 0; st < stripes; ++st) tma_load_2d(s_w + st * stripe_bytes, &g.map[mi], st * 128, r0, &s_bar);
+    const uint64_t pol = l2_policy_evict_first();
+    for (int st = 0; st < stripes; ++st) tma_load_2d_hint(s_w + st * stripe_bytes, map, st * 128, r0, &s_bar, pol);
   }
   const float alpha = *mt.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
   __syncthreads();
 
   pdl_wait_primary();  // x may come from the preceding kernel
-  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_csum, s_red);
+  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_hsum, s_red);
+  // The next kernel may start now: its weight copies then stream while this
+  // one contracts, and no longer delay this kernel's read of x.
+  pdl_launch_dependents();
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
   if (!landed && threadIdx.x == 0) *g.status = kDevTimeoutProducer;
 
   if (landed) {
-    // units: (chunk, row pair), row pair fastest; pair p covers rows p and p + half
+    // units (chunk, row pair), row pair fastest: the lanes of a warp read one
+    // activation chunk (one shared-memory broadcast) for up to 64 rows
     const int nthr = blockDim.x;
-    const int half = (nrows + 1) >> 1;
+    const int half = (nrows + 1) >> 1;  // pair p covers rows p and p + half
     const int total = half * C;
     const int dq = nthr / half, dr = nthr % half;
     int ch = threadIdx.x / half, p = threadIdx.x % half;
     for (int u = threadIdx.x; u < total; u += nthr) {
-      const int r2 = p + half < nrows ? p + half : -1;
-      int32_t p1, p2;
-      gemv_unit2(s_w, stripe_bytes, s_act, s_csum, C, p, r2, ch, p1, p2);
-      atomicAdd(&s_acc[p], p1);
-      if (r2 >= 0) atomicAdd(&s_acc[r2], p2);
+      const int r2 = p + half < nrows ? p + half : p;  // an odd last pair reads row p twice
+      const uint4 wa = gemv_wchunk(s_w, stripe_bytes, p, ch);
+      const uint4 wb = gemv_wchunk(s_w, stripe_bytes, r2, ch);
+      const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
+      const int32_t cs = chunk_sum(s_hsum, ch);
+      int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
+      dot_word(wa.x, q0.x, q0.y, q0.z, q0.w, a0, a1, a2, a3);
+      dot_word(wb.x, q0.x, q0.y, q0.z, q0.w, b0, b1, b2, b3);
+      dot_word(wa.y, q1.x, q1.y, q1.z, q1.w, a0, a1, a2, a3);
+      dot_word(wb.y, q1.x, q1.y, q1.z, q1.w, b0, b1, b2, b3);
+      dot_word(wa.z, q2.x, q2.y, q2.z, q2.w, a0, a1, a2, a3);
+      dot_word(wb.z, q2.x, q2.y, q2.z, q2.w, b0, b1, b2, b3);
+      dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
+      dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
+      // every partial sum s_j is a multiple of 4^j, so the shifts are exact
+      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6) - cs);
+      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6) - cs);
       p += dr;
       ch += dq;
       if (p >= half) {
@@ -371,7 +379,7 @@ __device__ __forceinline__ uint32_t load_bits(const uint8_t* base, int64_t bit, 
 __global__ void __launch_bounds__(kGemvThreads) gemv_nm_m1_kernel(const GemvArgs a) {
   extern __shared__ uint4 s_dyn[];
   uint4* s_act = s_dyn;                                            // 8 * C entries
-  int32_t* s_csum = reinterpret_cast<int32_t*>(s_dyn + 8 * a.C);   // 2 * C entries
+  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_dyn + 8 * a.C);   // 16 * C half sums
   __shared__ float s_red[32];
   pdl_launch_dependents();
   const int tpr = 1 << a.tpr_log2;
@@ -383,10 +391,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_m1_kernel(const GemvArgs
   const int nrows = a.rows_base + (b < a.rows_rem ? 1 : 0);
 
   pdl_wait_primary();
-  const float gamma = quantise_row_smem(a.x, a.K, 8 * a.C, s_act, s_csum, s_red);
+  const float gamma = quantise_row_smem(a.x, a.K, 8 * a.C, s_act, s_hsum, s_red);
   const float s = __fdiv_rn(__fmul_rn(*a.alpha, gamma), kQb);
   int32_t qsum = 0;  // this lane's share of sum(q): the two 64-weight chunks of each of its units
-  for (int u = sub; u < a.C; u += tpr) qsum += s_csum[2 * u] + s_csum[2 * u + 1];
+  for (int u = sub; u < a.C; u += tpr) qsum += chunk_sum(s_hsum, 2 * u) + chunk_sum(s_hsum, 2 * u + 1);
   const int n = a.nm_n, m = a.nm_m;
   const int blocks_per_row = a.K / m;
 
