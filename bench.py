@@ -44,7 +44,7 @@ FFN = (("gate", 2560, 6912), ("up", 2560, 6912), ("down", 6912, 2560))  # (name,
 PREFILL_SHAPES = ((2560, 6912), (6912, 2560), (2560, 2560), (2560, 640))  # (K, N)
 PREFILL_M = 2048
 DISTINCT_LAYERS = 2  # distinct weight draws, replicated to 30 layers at distinct addresses
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_m1_dense__decode_2b4t_ffn.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_dense__decode_2b4t_ffn.md")
 GEMV_SOURCES = ("gemv.cuh", "quant_pack.cuh", "ptx.cuh")
 
 

@@ -197,8 +197,8 @@ QuantWs tc_ws_layout(void* ws, int M, int K) {
 }
 
 bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s) {
-  return launch(quant_act_kernel<true>, dim3(M), dim3(256), 0, s, pdl, x, M, K, static_cast<int>(k16(K)), qw.q,
-                qw.gamma, qw.rowsum);
+  return launch(quant_act_kernel<true>, dim3((M + kQuantRowsPerCta - 1) / kQuantRowsPerCta),
+                dim3(32 * kQuantRowsPerCta), 0, s, pdl, x, M, K, static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum);
 }
 
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
@@ -586,8 +586,8 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
   DeviceState* dev = nullptr;
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
-  st = launch(quant_act_kernel<false>, dim3(M), dim3(256), 0, static_cast<cudaStream_t>(stream), false, x, M, K, K, q,
-              gamma, rowsum);
+  st = launch(quant_act_kernel<false>, dim3((M + kQuantRowsPerCta - 1) / kQuantRowsPerCta),
+              dim3(32 * kQuantRowsPerCta), 0, static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum);
   if (st == BITLINEAR_OK) t_last_kernel = "quant_act";
   return st;
 }

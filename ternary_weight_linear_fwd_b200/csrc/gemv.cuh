@@ -40,52 +40,6 @@ struct GemvArgs {
   int32_t* status;       // device status word
 };
 
-// Exact round-half-to-even of RN(t / d), t = RN(v * 127), for |t / d| < 128,
-// without a division per element.  With c = RN(127 * RN(1 / d)), y = RN(v * c)
-// differs from the true quotient by at most 3 * 2^-24 relative, i.e. by less
-// than 3.1e-5 absolute, and RN(t / d) lies within 7.6e-6 of the true quotient.
-// So unless y sits within 2^-14 of a half-integer, RN(t / d) rounds to the same
-// integer as y; such a group is recomputed with the exact quotient.  The
-// rounding to an integer is done by adding 1.5 * 2^23 (the sum's last place is
-// 1, ties to even), leaving the two's-complement code in the low byte.
-constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-
-// Codes of 8 consecutive activations (the first or second half of a 16-group).  b[e] holds the code of
-// element e in its low byte.
-__device__ __forceinline__ void codes8(const uint32_t (&raw)[4], float c, float d, uint32_t (&b)[8]) {
-  float emax = 0.0f;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float v = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
-    const float yq = __fmul_rn(v, c);
-    const float sm = __fadd_rn(yq, kMagic);
-    emax = fmaxf(emax, fabsf(__fsub_rn(yq, __fsub_rn(sm, kMagic))));
-    b[e] = __float_as_uint(sm);
-  }
-  if (emax > 0.5f - 6.103515625e-05f) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float v = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
-      b[e] = 0x4B400000u + static_cast<uint32_t>(__float2int_rn(__fdiv_rn(__fmul_rn(v, kQb), d)));
-    }
-  }
-}
-
-// 8 bf16 values of a row from k0 as 4 words (zero past K).
-__device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bool vec_ok, uint32_t (&r)[4]) {
-  if (vec_ok && k0 + 8 <= K) {
-    const uint4 a = *reinterpret_cast<const uint4*>(row + k0);
-    r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = (k0 + 2 * i < K) ? row[k0 + 2 * i] : 0u;
-      const uint32_t hi = (k0 + 2 * i + 1 < K) ? row[k0 + 2 * i + 1] : 0u;
-      r[i] = lo | (hi << 16);
-    }
-  }
-}
-
 // Quantises the single activation row into shared memory: s_act[slot(g)]
 // holds the 16 codes of k-group g in contraction order (byte 4j + b <- k =
 // 16g + 4b + j), for g < groups_alloc (zero past K), where

@@ -25,13 +25,6 @@ constexpr float kQb = 127.0f;
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
-// Round-half-to-even code of one activation: clamp(rne(RN(v * 127) / d), -128, 127).
-__device__ __forceinline__ int32_t act_code(float v, float d) {
-  const float t = __fmul_rn(v, kQb);
-  int32_t c = __float2int_rn(__fdiv_rn(t, d));
-  return max(-128, min(127, c));
-}
-
 // Ternary value of one latent weight: clamp(rne(w / d), -1, 1).
 __device__ __forceinline__ int32_t ternary_of(float w, float d) {
   int32_t c = __float2int_rn(__fdiv_rn(w, d));
@@ -53,109 +46,134 @@ __device__ __forceinline__ T block_reduce(T v, Op op, T* red /* >= 32 entries */
   return v;
 }
 
-struct MaxOp {
-  __device__ float operator()(float a, float b) const { return fmaxf(a, b); }
-};
-struct AddI {
-  __device__ int32_t operator()(int32_t a, int32_t b) const { return a + b; }
-};
 struct AddD {
   __device__ double operator()(double a, double b) const { return a + b; }
 };
 
-// Loads 16 consecutive bf16 values of a row starting at k0 (zero past K).
-__device__ __forceinline__ void load16_bf16(const uint16_t* row, int k0, int K, bool vec_ok, float (&v)[16]) {
-  if (vec_ok && k0 + 16 <= K) {
-    const uint4 a = *reinterpret_cast<const uint4*>(row + k0);
-    const uint4 b = *reinterpret_cast<const uint4*>(row + k0 + 8);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+// Exact round-half-to-even of RN(t / d), t = RN(v * 127), for |t / d| < 128,
+// without a division per element.  With c = RN(127 * RN(1 / d)), y = RN(v * c)
+// differs from the true quotient by at most 3 * 2^-24 relative, i.e. by less
+// than 3.1e-5 absolute, and RN(t / d) lies within 7.6e-6 of the true quotient.
+// So unless y sits within 2^-14 of a half-integer, RN(t / d) rounds to the same
+// integer as y; such a group is recomputed with the exact quotient.  The
+// rounding to an integer is done by adding 1.5 * 2^23 (the sum's last place is
+// 1, ties to even), leaving the two's-complement code in the low byte.
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+
+// Codes of 8 consecutive activations (the first or second half of a 16-group).  b[e] holds the code of
+// element e in its low byte.
+__device__ __forceinline__ void codes8(const uint32_t (&raw)[4], float c, float d, uint32_t (&b)[8]) {
+  float emax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  for (int e = 0; e < 8; ++e) {
+    const float v = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
+    const float yq = __fmul_rn(v, c);
+    const float sm = __fadd_rn(yq, kMagic);
+    emax = fmaxf(emax, fabsf(__fsub_rn(yq, __fsub_rn(sm, kMagic))));
+    b[e] = __float_as_uint(sm);
+  }
+  if (emax > 0.5f - 6.103515625e-05f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float v = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
+      b[e] = 0x4B400000u + static_cast<uint32_t>(__float2int_rn(__fdiv_rn(__fmul_rn(v, kQb), d)));
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = (k0 + i < K) ? bf16_bits_to_f32(row[k0 + i]) : 0.0f;
   }
 }
 
-// Packs the 16 codes of one k-group into the order used by the integer
-// contraction: byte (4j + b) holds the code of k0 + 4b + j.  This matches the
-// order in which a 2-bit weight word unpacks with (w >> 2j) & 0x03030303.
-__device__ __forceinline__ void permute16(const int32_t (&c)[16], uint32_t (&out)[4]) {
+// 8 bf16 values of a row from k0 as 4 words (zero past K).
+__device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bool vec_ok, uint32_t (&r)[4]) {
+  if (vec_ok && k0 + 8 <= K) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + k0);
+    r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
+  } else {
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    out[j] = (static_cast<uint32_t>(c[j] & 0xFF)) | (static_cast<uint32_t>(c[4 + j] & 0xFF) << 8) |
-             (static_cast<uint32_t>(c[8 + j] & 0xFF) << 16) | (static_cast<uint32_t>(c[12 + j] & 0xFF) << 24);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = (k0 + 2 * i < K) ? row[k0 + 2 * i] : 0u;
+      const uint32_t hi = (k0 + 2 * i + 1 < K) ? row[k0 + 2 * i + 1] : 0u;
+      r[i] = lo | (hi << 16);
+    }
+  }
 }
 
 // ----------------------------------------------------------------- quant_act
-// One CTA per token row.  kPermute = false writes natural-order codes [M, ldq]
-// (ldq = K); kPermute = true writes the contraction order [M, ldq] with ldq =
-// K rounded up to 16 (zeros past K).  Both write gamma and, when asked, the
-// sum of the row's codes.
+// One warp per token row (eight rows per 256-thread CTA).  Pass one reads the
+// row for gamma (all loads of a lane in flight together); pass two re-reads it
+// (now from L1/L2) one 16-wide k-group per lane and step: 16 codes by the
+// division-free exact rounding of codes8, one 16-byte store.  kPermute = false
+// writes natural-order codes [M, ldq] (ldq = K); kPermute = true writes the
+// contraction order [M, ldq] with ldq = K rounded up to 16 (zeros past K).
+// Both write gamma and, when asked, the sum of the row's codes.
+constexpr int kQuantRowsPerCta = 8;
+
 template <bool kPermute>
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K, int ldq,
-                                                        int8_t* __restrict__ q, float* __restrict__ gamma,
-                                                        int32_t* __restrict__ rowsum) {
-  __shared__ float redf[32];
-  __shared__ int32_t redi[32];
+__global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                                          int ldq, int8_t* __restrict__ q,
+                                                                          float* __restrict__ gamma,
+                                                                          int32_t* __restrict__ rowsum) {
   pdl_wait_primary();
   pdl_launch_dependents();
-  const int row = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kQuantRowsPerCta + (threadIdx.x >> 5);
   if (row >= M) return;
   const uint16_t* xr = x + static_cast<size_t>(row) * K;
-  const bool vec_ok = (K % 8) == 0;
+  const bool vec_ok = (K % 8) == 0 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
 
   float mx = 0.0f;
+  const int halves = (K + 7) / 8;
   if (vec_ok) {
-    for (int k = threadIdx.x * 8; k < K; k += blockDim.x * 8) {
-      const uint4 a = *reinterpret_cast<const uint4*>(xr + k);
+#pragma unroll 4
+    for (int h = lane; h < halves; h += 32) {
+      const uint4 a = *reinterpret_cast<const uint4*>(xr + 8 * h);
       const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mx = fmaxf(mx, fabsf(__uint_as_float(w[i] << 16)));
-        mx = fmaxf(mx, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
-      }
+      for (int i = 0; i < 4; ++i)
+        mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
     }
   } else {
-    for (int k = threadIdx.x; k < K; k += blockDim.x) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(xr[k])));
+    for (int k = lane; k < K; k += 32) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(xr[k])));
   }
-  mx = block_reduce(mx, MaxOp(), redf, 0.0f);
+  // |x| >= 0, whose bit patterns order like the values: one integer warp reduction
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
   const float d = __fadd_rn(mx, kEps);
+  const float c = __fmul_rn(kQb, __frcp_rn(d));
 
   int32_t sum = 0;
   const int groups = (K + 15) / 16;
   int8_t* qr = q + static_cast<size_t>(row) * ldq;
   const bool qvec = ((reinterpret_cast<uintptr_t>(q) & 15u) == 0) && (ldq % 16) == 0;
-  for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+  for (int g = lane; g < groups; g += 32) {
     const int k0 = g * 16;
-    float v[16];
-    load16_bf16(xr, k0, K, vec_ok, v);
-    int32_t c[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      c[i] = (k0 + i < K) ? act_code(v[i], d) : 0;
-      sum += c[i];
-    }
+    uint32_t r0[4], r1[4], b0[8], b1[8];
+    load8_raw(xr, k0, K, vec_ok, r0);
+    load8_raw(xr, k0 + 8, K, vec_ok, r1);
+    codes8(r0, c, d, b0);  // elements past K are zero and give code 0
+    codes8(r1, c, d, b1);
+    uint32_t w[4];
     if (kPermute) {
-      uint32_t w[4];
-      permute16(c, w);
-      *reinterpret_cast<uint4*>(qr + k0) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else if (qvec && k0 + 16 <= K) {
-      uint32_t w[4];
+      // byte 4j + b <- k0 + 4b + j
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        w[j] = (static_cast<uint32_t>(c[4 * j] & 0xFF)) | (static_cast<uint32_t>(c[4 * j + 1] & 0xFF) << 8) |
-               (static_cast<uint32_t>(c[4 * j + 2] & 0xFF) << 16) | (static_cast<uint32_t>(c[4 * j + 3] & 0xFF) << 24);
+        w[j] = __byte_perm(__byte_perm(b0[j], b0[4 + j], 0x0040), __byte_perm(b1[j], b1[4 + j], 0x0040), 0x5410);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        w[j] = __byte_perm(__byte_perm(b0[4 * j], b0[4 * j + 1], 0x0040), __byte_perm(b0[4 * j + 2], b0[4 * j + 3], 0x0040),
+                           0x5410);
+        w[2 + j] = __byte_perm(__byte_perm(b1[4 * j], b1[4 * j + 1], 0x0040),
+                               __byte_perm(b1[4 * j + 2], b1[4 * j + 3], 0x0040), 0x5410);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sum = __dp4a(static_cast<int>(w[j]), 0x01010101, sum);
+    if (kPermute || (qvec && k0 + 16 <= K)) {
       *reinterpret_cast<uint4*>(qr + k0) = make_uint4(w[0], w[1], w[2], w[3]);
     } else {
-      for (int i = 0; i < 16 && k0 + i < K; ++i) qr[k0 + i] = static_cast<int8_t>(c[i]);
+      for (int i = 0; i < 16 && k0 + i < K; ++i) qr[k0 + i] = static_cast<int8_t>(w[i >> 2] >> (8 * (i & 3)));
     }
   }
-  sum = block_reduce(sum, AddI(), redi, 0);
-  if (threadIdx.x == 0) {
+  sum = __reduce_add_sync(0xffffffffu, sum);
+  if (lane == 0) {
     if (gamma) gamma[row] = mx;
     if (rowsum) rowsum[row] = sum;
   }
