@@ -359,6 +359,123 @@ def run_prefill(dev, iters: int, warmup: int):
     return {"shapes": out, "tops": tot_ops / tot_sec / 1e12, "kernel": kernel, "ops": tot_ops, "secs": tot_sec}
 
 
+def time_chain_graph(dev, calls, warmup: int, reps: int) -> float:
+    """Seconds per replay of a CUDA graph holding `calls` (callables that enqueue
+    library calls on the current stream), after `warmup` replays."""
+    import torch
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for c in calls:
+            c()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    for _ in range(warmup):
+        g.replay()
+    s = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(s)
+    for _ in range(reps):
+        g.replay()
+    e1.record(s)
+    e1.synchronize()
+    del g
+    return e0.elapsed_time(e1) / 1e3 / reps
+
+
+L2_DEFEAT_BYTES = 2 * 126 * 1024 * 1024  # weights rotated over copies until the working set is twice L2
+SWEEP_M = (1, 16, 256, 4096)
+NM_PATTERNS = ((2, 4), (6, 8))
+NM_M = (1, 4096)
+
+
+def _copies(w, nbytes: int):
+    """Distinct device copies of packed weights so that a chain of calls streams > 2 x L2."""
+    import ternary_weight_linear_fwd_b200 as bl
+    n = max(1, min(1024, -(-L2_DEFEAT_BYTES // max(1, nbytes))))
+    return [w] + [bl.PackedWeights(w.N, w.K, w.nm_n, w.nm_m, w.codes.clone(),
+                                   None if w.meta is None else w.meta.clone(), w.alpha.clone()) for _ in range(n - 1)]
+
+
+def run_sweep(dev, min_calls: int = 16, warmup: int = 3, reps: int = 5):
+    """Layer sweep: the seven 2B4T BitLinears at M in SWEEP_M; per matrix a PDL-chained graph that
+    calls each of its weight copies once (> 2 x L2 of weights per replay)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    packed = {}
+    for i, (name, (K, N)) in enumerate(synth.B2B4T_LAYER.items()):
+        T = torch.from_numpy(synth.ternary_weights(N, K, seed=4 + 10 * i)).to(dev)
+        packed[name] = bl.pack_ternary(T, float(synth.alpha_uniform(4 + 10 * i)))
+        del T
+    out = {}
+    for M in SWEEP_M:
+        x = torch.from_numpy(synth.activations(M, 6912, seed=4).view(np.int16)).to(dev).view(torch.bfloat16)
+        ws = torch.empty(max(1, max(bl.forward_workspace_bytes(M, N, K) for K, N in synth.B2B4T_LAYER.values())),
+                         dtype=torch.uint8, device=dev)
+        row, tot_b, tot_ops, tot_s = {}, 0, 0.0, 0.0
+        for name, (K, N) in synth.B2B4T_LAYER.items():
+            xk = x[:, :K].contiguous()
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            wbytes = packed[name].nbytes
+            cps = _copies(packed[name], wbytes)
+            ncall = max(min_calls, len(cps))
+            calls = [(lambda w=cps[i % len(cps)]: bl.forward(w, xk, out=y, workspace=ws, flags=bl.FLAG_PDL))
+                     for i in range(ncall)]
+            sec = time_chain_graph(dev, calls, warmup, reps) / ncall
+            nbytes = N * K // 4 + 4 + 2 * M * K + 2 * M * N
+            ops = 2.0 * M * N * K
+            row[name] = {"us": sec * 1e6, "GBps": nbytes / sec / 1e9, "TOPS": ops / sec / 1e12,
+                         "kernel": bl.last_kernel(), "weight_copies": len(cps)}
+            tot_b, tot_ops, tot_s = tot_b + nbytes, tot_ops + ops, tot_s + sec
+            del cps, calls, y, xk
+        row["layer"] = {"us": tot_s * 1e6, "GBps": tot_b / tot_s / 1e9, "TOPS": tot_ops / tot_s / 1e12}
+        out[f"M={M}"] = row
+        del x, ws
+    assert bl.device_status() == 0
+    return out
+
+
+def run_nm(dev, min_calls: int = 16, warmup: int = 3, reps: int = 5):
+    """Sparse-BitNet N:M on the Qwen2.5-3B MLP shapes at M in NM_M (same chained-graph timing)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    out = {}
+    for n, m in NM_PATTERNS:
+        for name, (K, N) in synth.QWEN25_3B_MLP.items():
+            W = torch.from_numpy(synth.latent_weights(N, K, seed=5)).to(dev)
+            w = bl.pack_weights(W, n, m)
+            del W
+            for M in NM_M:
+                x = torch.from_numpy(synth.activations(M, K, seed=5).view(np.int16)).to(dev).view(torch.bfloat16)
+                ws = torch.empty(max(1, bl.forward_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                cps = _copies(w, w.nbytes) if M == 1 else [w]
+                ncall = max(min_calls, len(cps))
+                calls = [(lambda ww=cps[i % len(cps)]: bl.forward_nm(ww, x, out=y, workspace=ws, flags=bl.FLAG_PDL))
+                         for i in range(ncall)]
+                sec = time_chain_graph(dev, calls, warmup, reps) / ncall
+                nbytes = w.nbytes + 4 + 2 * M * K + 2 * M * N
+                key = f"{n}:{m} {name} {K}->{N} M={M}"
+                out[key] = {"us": sec * 1e6, "GBps": nbytes / sec / 1e9, "TOPS_dense_equiv": 2.0 * M * N * K / sec / 1e12,
+                            "packed_bytes": w.nbytes, "kernel": bl.last_kernel(), "weight_copies": len(cps)}
+                del cps, calls, x, ws, y
+    assert bl.device_status() == 0
+    return out
+
+
 # ------------------------------------------------------------------ oracle (CPU) legs
 
 def oracle_decode_setup(seed: int = 1):
@@ -406,6 +523,7 @@ def main():
     ap.add_argument("--prefill-iters", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the layer sweep and the N:M objects")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps")
@@ -468,6 +586,10 @@ def main():
     e2e_value = aggregate(step_bytes, dec["e2e_steps"], world, max_e2e) / 1e9
 
     pre = run_prefill(dev, args.prefill_iters, 3)
+    sweep = nm = None
+    if not args.no_sweep:
+        sweep = run_sweep(dev)
+        nm = run_nm(dev)
 
     if world > 1:
         barrier(dev)
@@ -505,6 +627,16 @@ def main():
                     "d2h_bytes_per_step": dec["d2h"], "steps": dec["e2e_steps"]},
             "gpu_launches": args.steps * dec["launches_per_step"], "clocks": dec["clocks"],
             "hbm_frac": value / world / peaks["hbm_gbs"], "prefill": prefill}
+    if sweep is not None:
+        line["sweep"] = {"workload": "2B4T layer's 7 BitLinears (q,k,v,o 2560->2560/640, gate/up 2560->6912, "
+                                     "down 6912->2560), ternary P(0)=0.42; per matrix a PDL-chained graph "
+                                     "calling each of its weight copies once (> 2 x L2 of weights); bytes = "
+                                     "N*K/4 + 4 + 2MK + 2MN, ops = 2MNK", "by_M": sweep}
+        line["nm"] = {"workload": "Sparse-BitNet N:M on Qwen2.5-3B MLP (2048->11008, 11008->2048), latent "
+                                  "W ~ N(0,0.02); PDL-chained graph (M=1: each of > 2 x L2 of weight copies once; "
+                                  "M=4096: 16 calls); "
+                                  "bytes = packed values + metadata + 4 + 2MK + 2MN; TOPS counts dense-equivalent "
+                                  "2MNK", "cases": nm}
     print(json.dumps(line), flush=True)
 
 

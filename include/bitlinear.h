@@ -149,7 +149,11 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
                                      int32_t* rowsum, void* stream);
 
 /* Workspace bytes needed by bitlinear_forward / bitlinear_forward_nm.  0 when
- * the call takes the M = 1 GEMV path (which quantises in-kernel). */
+ * the call takes the M = 1 GEMV path (which quantises in-kernel).  The
+ * tensor-core path needs the int8 codes, gamma and code sums of x and, when it
+ * splits K across SMs (few tokens or few weight rows), ksplit int32 [M, N]
+ * partial-sum slabs; the size depends on the current device's SM count.  The
+ * workspace holds no state between calls. */
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags);
 
 /* y = BitLinear(x) for dense packed weights.
@@ -184,7 +188,8 @@ bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t
  * y        host array of count device pointers, out: bf16 bits [M, w[i].N].
  * acc      NULL, or a host array of count device pointers (each may be NULL):
  *          int32 [M, w[i].N].
- * workspace, workspace_bytes: bitlinear_forward_workspace_bytes(M, 0, K, flags).
+ * workspace, workspace_bytes: at least bitlinear_forward_workspace_bytes(M, w[i].N, K,
+ *          flags) for every i.
  * flags    as for bitlinear_forward; PDL applies to the first kernel the call
  *          launches (the later ones follow kernels of the same call).
  * Path: M == 1 runs the dense matrices in one GEMV launch (CTAs split among

@@ -204,8 +204,7 @@ def forward_group(ws, x, want_acc: bool = False, flags: int = 0, workspace=None,
     M = x.shape[0]
     ys = outs if outs is not None else [torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device) for w in ws]
     accs = [torch.empty((M, w.N), dtype=torch.int32, device=x.device) for w in ws] if want_acc else None
-    K = ws[0].K if count else 0
-    need = forward_workspace_bytes(M, 0, K, flags) if count else 0
+    need = max((forward_workspace_bytes(M, w.N, w.K, flags) for w in ws), default=0)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()

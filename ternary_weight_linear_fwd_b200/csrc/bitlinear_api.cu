@@ -145,16 +145,54 @@ bitlinear_status check_nk(int N, int K) {
 // ---------------------------------------------------------------- tensor-core path
 int pick_bn(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 
-size_t tc_workspace(int M, int K) { return align256(static_cast<size_t>(M) * k16(K)) + 2 * align256(4 * static_cast<size_t>(M)); }
+// Tiling of one tensor-core GEMM.  When the (weight-row tile, token tile)
+// pairs leave SMs idle, each tile's K range is cut into ksplit slices (at
+// least two k-blocks each, none empty) so that about one unit runs per SM.
+struct TcPlan {
+  int bn, row_tiles, tok_tiles, kblocks, ksplit, kbs;
+};
+
+TcPlan tc_plan(int M, int N, int K, int sm_count) {
+  TcPlan p;
+  p.bn = pick_bn(M);
+  p.row_tiles = (N + kTcRows - 1) / kTcRows;
+  // narrower token tiles while the tiles would fill fewer than half the SMs
+  while (p.bn > 32 && p.row_tiles * ((M + p.bn - 1) / p.bn) < sm_count / 2) p.bn >>= 1;
+  p.tok_tiles = (M + p.bn - 1) / p.bn;
+  p.kblocks = (K + kTcBK - 1) / kTcBK;
+  const int tiles = p.row_tiles * p.tok_tiles;
+  int ks = 1;
+  if (tiles < sm_count) ks = std::max(1, std::min(std::min(sm_count / tiles, p.kblocks / 2), 16));
+  p.kbs = (p.kblocks + ks - 1) / ks;
+  p.ksplit = (p.kblocks + p.kbs - 1) / p.kbs;
+  return p;
+}
+
+int plan_sm_count() {
+  DeviceState* d = nullptr;
+  return current_device(&d) == BITLINEAR_OK ? d->sm_count : 148;
+}
+
+// Workspace: codes [M, k16(K)] | gamma [M] | code sums [M] | (split only)
+// arrival counters [sm_count] | fp32 sums [M][N].
+size_t tc_base_bytes(int M, int K) {
+  return align256(static_cast<size_t>(M) * k16(K)) + 2 * align256(4 * static_cast<size_t>(M));
+}
+size_t tc_cnt_bytes(int sm_count) { return align256(4 * static_cast<size_t>(sm_count)); }
+
+size_t tc_workspace(int M, int N, int K, int sm_count) {
+  const TcPlan p = tc_plan(M, N, K, sm_count);
+  size_t b = tc_base_bytes(M, K);
+  if (p.ksplit > 1) b += tc_cnt_bytes(sm_count) + align256(static_cast<size_t>(M) * N * 4);
+  return b;
+}
 
 template <int BN, int NM>
 bitlinear_status launch_tc_bn(const CUtensorMap& mB, const CUtensorMap& mA, const CUtensorMap& mMeta, TcArgs ta,
                               int sm_count, cudaStream_t s) {
   const size_t smem = tc_smem_bytes(BN, NM, ta.vbox);
-  ta.row_tiles = (ta.N + kTcRows - 1) / kTcRows;
-  ta.tok_tiles = (ta.M + BN - 1) / BN;
-  const int tiles = ta.row_tiles * ta.tok_tiles;
-  const int grid = std::min(sm_count, tiles);
+  const int units = ta.row_tiles * ta.tok_tiles * ta.ksplit;
+  const int grid = std::min(sm_count, units);
   return launch(tc_gemm_kernel<BN, NM>, dim3(grid), dim3(kTcThreads), smem, s, true, mB, mA, mMeta, ta);
 }
 
@@ -185,26 +223,41 @@ struct QuantWs {
   int8_t* q;        // [M, k16(K)]
   float* gamma;     // [M]
   int32_t* rowsum;  // [M]
+  uint32_t* cnt;    // [ncnt] split-K arrival counters (zeroed by the quantisation kernel)
+  int ncnt;         // 0 when no GEMM of the call splits K
+  float* part;      // split-K fp32 sums [M][max N] (zeroed by the quantisation kernel)
+  size_t part_words;
 };
 
-QuantWs tc_ws_layout(void* ws, int M, int K) {
+QuantWs tc_ws_layout(void* ws, int M, int K, int ncnt, int max_n) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   QuantWs r;
   r.q = reinterpret_cast<int8_t*>(wsb);
   r.gamma = reinterpret_cast<float*>(wsb + align256(static_cast<size_t>(M) * k16(K)));
   r.rowsum = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(r.gamma) + align256(4 * static_cast<size_t>(M)));
+  r.cnt = reinterpret_cast<uint32_t*>(wsb + tc_base_bytes(M, K));
+  r.ncnt = ncnt;
+  r.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(r.cnt) + tc_cnt_bytes(ncnt > 0 ? ncnt : 0));
+  r.part_words = ncnt > 0 ? static_cast<size_t>(M) * max_n : 0;
   return r;
 }
 
 bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s) {
-  return launch(quant_act_kernel<true>, dim3((M + kQuantRowsPerCta - 1) / kQuantRowsPerCta),
-                dim3(32 * kQuantRowsPerCta), 0, s, pdl, x, M, K, static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum);
+  const int qblocks = (M + kQuantRowsPerCta - 1) / kQuantRowsPerCta;
+  // extra CTAs clear the split-K sums, 16 bytes per thread and step, at most four steps each
+  const size_t vec4 = (qw.part_words + 3) / 4;
+  const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * 32 * kQuantRowsPerCta - 1) /
+                                                                   (4 * 32 * kQuantRowsPerCta)));
+  return launch(quant_act_kernel<true>, dim3(qblocks + zblocks), dim3(32 * kQuantRowsPerCta), 0, s, pdl, x, M, K,
+                static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum,
+                qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr), qw.ncnt, qw.part, vec4, qblocks);
 }
 
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
                          cudaStream_t s, DeviceState* dev) {
   const int N = w->N, K = w->K;
-  const int bn = pick_bn(M);
+  const TcPlan plan = tc_plan(M, N, K, dev->sm_count);
+  const int bn = plan.bn;
   const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? 1 : 2);
   CUtensorMap mB, mA, mMeta;
   if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
@@ -214,7 +267,14 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   ta.M = M;
   ta.N = N;
   ta.K = K;
-  ta.kblocks = (K + kTcBK - 1) / kTcBK;
+  ta.kblocks = plan.kblocks;
+  ta.row_tiles = plan.row_tiles;
+  ta.tok_tiles = plan.tok_tiles;
+  ta.ksplit = plan.ksplit;
+  ta.kbs = plan.kbs;
+  ta.part = plan.ksplit > 1 ? qw.part : nullptr;
+  ta.cnt = plan.ksplit > 1 ? qw.cnt : nullptr;
+  if (plan.ksplit > 1 && (qw.ncnt < plan.row_tiles * plan.tok_tiles)) return BITLINEAR_ERR_WORKSPACE;
   ta.gamma = qw.gamma;
   ta.alpha = w->alpha;
   ta.rowsum = qw.rowsum;
@@ -224,7 +284,6 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   ta.vbox = 0;
   ta.status = dev->status;
   ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
-  ta.row_tiles = ta.tok_tiles = 0;
   if (nm == 0) {
     const int64_t ld = dense_ld(K);
     if (!make_map_u8(&mA, w->codes, ld, N, ld, 32, kTcRows, false)) return BITLINEAR_ERR_CUDA;
@@ -251,8 +310,9 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
 
 bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
                             void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev) {
-  if (!ws || ws_bytes < tc_workspace(M, w->K) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
-  const QuantWs qw = tc_ws_layout(ws, M, w->K);
+  if (!ws || ws_bytes < tc_workspace(M, w->N, w->K, dev->sm_count) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
+  const bool split = tc_plan(M, w->N, w->K, dev->sm_count).ksplit > 1;
+  const QuantWs qw = tc_ws_layout(ws, M, w->K, split ? dev->sm_count : 0, w->N);
   bitlinear_status st = tc_quant(x, M, w->K, qw, pdl, s);
   if (st != BITLINEAR_OK) return st;
   return tc_gemm(w, M, qw, y, acc, s, dev);
@@ -352,36 +412,49 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
                               cudaStream_t s, DeviceState* dev) {
   const int N = w->N, K = w->K;
   if (w->nm_m == 0) return gemv_dense_launch(&w, &y, &acc, 1, x, pdl, s, dev);
-  GemvArgs ga;
-  std::memset(&ga, 0, sizeof ga);
-  ga.codes = w->codes;
-  ga.meta = w->meta;
-  ga.N = N;
-  ga.K = K;
-  ga.x = x;
-  ga.alpha = w->alpha;
-  ga.y = y;
-  ga.acc = acc;
-  ga.nm_n = w->nm_n;
-  ga.nm_m = w->nm_m;
   int64_t ldv = 0, ldm = 0;
   if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
     return BITLINEAR_ERR_PATTERN;
-  ga.ld = ldv;
-  ga.ld_meta = ldm;
-  ga.C = (K + 127) / 128;
-  int lg = 0;
-  while ((1 << lg) < ga.C && lg < 5) ++lg;
-  ga.tpr_log2 = lg;
-  ga.passes = 1;
-  ga.status = dev->status;
-  const int groups = kGemvThreads >> lg;
-  int grid = std::min(dev->sm_count * 2, (N + groups - 1) / groups);
-  grid = std::max(grid, 1);
-  ga.rows_base = N / grid;
-  ga.rows_rem = N % grid;
-  const size_t smem = static_cast<size_t>(ga.C) * 8 * (16 + 8);  // codes + half sums
-  bitlinear_status st = launch(gemv_nm_m1_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, ga);
+  GemvNmArgs na;
+  std::memset(&na, 0, sizeof na);
+  na.x = x;
+  na.alpha = w->alpha;
+  na.y = y;
+  na.acc = acc;
+  na.status = dev->status;
+  na.ld_v = ldv;
+  na.ld_m = ldm;
+  na.K = K;
+  na.C = (K + 127) / 128;
+  const bool lut = w->nm_m == 4;
+  // about one CTA per SM; more while a CTA's rows exceed a TMA box or the shared-memory budget
+  int grid = std::min(dev->sm_count, N);
+  auto fits = [&](int g) {
+    const int rows_box = N / g + 1;
+    return rows_box <= 256 && gemv_nm_smem_bytes(rows_box, ldv, ldm, na.C, lut) <= 160 * 1024;
+  };
+  while (!fits(grid) && grid < N) grid = std::min(N, grid * 2);
+  na.rows_base = N / grid;
+  na.rows_rem = N % grid;
+  na.rows_box = na.rows_base + 1;
+  CUtensorMap mv, mm;
+  if (!make_map_u8(&mv, w->codes, static_cast<uint64_t>(ldv), static_cast<uint64_t>(N), static_cast<uint64_t>(ldv), 128,
+                   static_cast<uint32_t>(na.rows_box), true) ||
+      !make_map_u8(&mm, w->meta, static_cast<uint64_t>(ldm), static_cast<uint64_t>(N), static_cast<uint64_t>(ldm), 128,
+                   static_cast<uint32_t>(na.rows_box), true))
+    return BITLINEAR_ERR_CUDA;
+  const size_t smem = gemv_nm_smem_bytes(na.rows_box, ldv, ldm, na.C, lut);
+  bitlinear_status st;
+  switch (w->nm_m == 4 ? 0 : w->nm_n) {
+    case 0: st = launch(gemv_nm_kernel<0>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+    case 1: st = launch(gemv_nm_kernel<1>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+    case 2: st = launch(gemv_nm_kernel<2>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+    case 3: st = launch(gemv_nm_kernel<3>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+    case 4: st = launch(gemv_nm_kernel<4>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+    case 5: st = launch(gemv_nm_kernel<5>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+    case 6: st = launch(gemv_nm_kernel<6>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+    default: st = launch(gemv_nm_kernel<7>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
+  }
   if (st == BITLINEAR_OK) t_last_kernel = w->nm_m == 4 ? "gemv_m1_nm24" : "gemv_m1_n8";
   return st;
 }
@@ -449,8 +522,18 @@ bitlinear_status forward_group(const bitlinear_weights* w, int count, const uint
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || M > 1;
   if (tc) {
-    if (!ws || ws_bytes < tc_workspace(M, w[0].K) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
-    const QuantWs qw = tc_ws_layout(ws, M, w[0].K);
+    size_t need = 0;
+    bool split = false;
+    int max_n = 0;
+    for (int i = 0; i < count; ++i) {
+      need = std::max(need, tc_workspace(M, w[i].N, w[i].K, dev->sm_count));
+      if (tc_plan(M, w[i].N, w[i].K, dev->sm_count).ksplit > 1) {
+        split = true;
+        max_n = std::max(max_n, w[i].N);
+      }
+    }
+    if (!ws || ws_bytes < need || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
+    const QuantWs qw = tc_ws_layout(ws, M, w[0].K, split ? dev->sm_count : 0, max_n);
     st = tc_quant(x, M, w[0].K, qw, pdl, s);
     for (int i = 0; i < count && st == BITLINEAR_OK; ++i) st = tc_gemm(&w[i], M, qw, y[i], acc ? acc[i] : nullptr, s, dev);
     return st;
@@ -587,16 +670,17 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
   st = launch(quant_act_kernel<false>, dim3((M + kQuantRowsPerCta - 1) / kQuantRowsPerCta),
-              dim3(32 * kQuantRowsPerCta), 0, static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum);
+              dim3(32 * kQuantRowsPerCta), 0, static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum,
+              static_cast<uint32_t*>(nullptr), 0, static_cast<float*>(nullptr), static_cast<size_t>(0),
+              (M + kQuantRowsPerCta - 1) / kQuantRowsPerCta);
   if (st == BITLINEAR_OK) t_last_kernel = "quant_act";
   return st;
 }
 
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {
-  (void)N;
-  if (M < 1 || K < 1) return 0;
+  if (M < 1 || K < 1 || N < 1) return 0;
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || (M > 1 && !(flags & BITLINEAR_FLAG_PATH_GEMV));
-  return tc ? tc_workspace(M, K) : 0;
+  return tc ? tc_workspace(M, N, K, plan_sm_count()) : 0;
 }
 
 bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,

@@ -16,7 +16,13 @@
 // Both operands use the same K order inside each 16-wide group (byte 4j + b
 // holds k = 4b + j), which is the order (w >> 2j) & 0x03030303 produces.
 //
-// One CTA per SM walks a static list of (weight-row tile, token tile) pairs.
+// One CTA per SM walks a static list of (weight-row tile, token tile, K slice)
+// units.  When the tiles alone would leave SMs idle (few tokens, or few
+// weight rows), each tile's K range is split into slices; every slice adds its
+// partial sums into one fp32 [M, N] buffer with vector atomic adds, and the
+// slice that arrives last (an atomic counter per tile) reads the sums, runs
+// the epilogue and clears them.  The sums are exact: every partial and total
+// of q * code is an integer of magnitude at most 254 * K <= 254 * 65536 < 2^24.
 // Warp roles (16 warps): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues
 // the MMAs, warp 2 owns the TMEM allocation, warps 4..11 unpack weights (two
 // groups of four, alternating k-blocks), warps 12..15 run the epilogue.  Warp
@@ -49,6 +55,10 @@ struct TcArgs {
   int M, N, K;
   int kblocks;            // ceil(K / 128)
   int row_tiles, tok_tiles;
+  int ksplit;             // K slices per tile (1: no split)
+  int kbs;                // k-blocks per slice, ceil(kblocks / ksplit)
+  float* part;            // ksplit > 1: fp32 [M][N] sums of the slices, zero on entry and left zero
+  uint32_t* cnt;          // ksplit > 1: [row_tiles * tok_tiles] arrival counters, zero on entry and left zero
   const float* gamma;     // [M] per-token absmax
   const float* alpha;     // the matrix's absmean scale (device)
   const int32_t* rowsum;  // [M] sum of the token's codes
@@ -139,18 +149,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* accempty = accfull + 2; // [2]
   uint64_t* drain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* s_last = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KB = a.kblocks;
-  const int ntiles = a.row_tiles * a.tok_tiles;
-  const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int KB = a.kbs;  // k-blocks per unit
+  const int nunits = a.row_tiles * a.tok_tiles * a.ksplit;
+  const int my_tiles = blockIdx.x < nunits ? (nunits - 1 - blockIdx.x) / gridDim.x + 1 : 0;  // units of this CTA
   const int total_kb = my_tiles * KB;  // k-blocks this CTA streams
   const uint32_t tx_bytes = static_cast<uint32_t>(B_STAGE + a_val_bytes + a_meta_bytes);
-  // tile t of this CTA -> (row tile, token tile), token tile fastest
-  auto tile_of = [&](int t, int& rt, int& tt) {
+  // unit t of this CTA -> (row tile, token tile, K slice), slice fastest, then token tile
+  auto unit_of = [&](int t, int& rt, int& tt, int& ks) {
     const int g = blockIdx.x + t * gridDim.x;
-    rt = g / a.tok_tiles;
-    tt = g - rt * a.tok_tiles;
+    const int tile = g / a.ksplit;
+    ks = g - tile * a.ksplit;
+    rt = tile / a.tok_tiles;
+    tt = tile - rt * a.tok_tiles;
+  };
+  // absolute k-block of the i-th k-block this CTA streams (slices past K read zeros)
+  auto kblock_of = [&](int i, int& rt, int& tt) {
+    int ks;
+    unit_of(i / KB, rt, tt, ks);
+    return ks * KB + i % KB;
   };
 
   pdl_launch_dependents();
@@ -198,15 +217,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // Weights do not depend on the preceding kernel: start them first.
       for (int i = 0; i < pre; ++i) {
         int rt, tt;
-        tile_of(i / KB, rt, tt);
+        const int kb = kblock_of(i, rt, tt);
         mbar_arrive_expect_tx(&full[i], tx_bytes);
-        load_a(rt * kTcRows, i % KB, i);
+        load_a(rt * kTcRows, kb, i);
       }
       pdl_wait_primary();
       for (int i = 0; i < pre; ++i) {
         int rt, tt;
-        tile_of(i / KB, rt, tt);
-        tma_load_2d(sB + i * B_STAGE, &mapB, (i % KB) * kTcBK, tt * BN, &full[i]);
+        const int kb = kblock_of(i, rt, tt);
+        tma_load_2d(sB + i * B_STAGE, &mapB, kb * kTcBK, tt * BN, &full[i]);
       }
       bool ok = true;
       int i = pre;
@@ -218,10 +237,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         int rt, tt;
-        tile_of(i / KB, rt, tt);
+        const int kb = kblock_of(i, rt, tt);
         mbar_arrive_expect_tx(&full[s], tx_bytes);
-        load_a(rt * kTcRows, i % KB, s);
-        tma_load_2d(sB + s * B_STAGE, &mapB, (i % KB) * kTcBK, tt * BN, &full[s]);
+        load_a(rt * kTcRows, kb, s);
+        tma_load_2d(sB + s * B_STAGE, &mapB, kb * kTcBK, tt * BN, &full[s]);
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
@@ -275,7 +294,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     for (int i = grp; i < total_kb; i += 2) {
       const int s = i % S;
-      const int kb = i % KB;
+      int rt_u, tt_u;
+      const int kb = kblock_of(i, rt_u, tt_u);
       if (!mbar_wait(&full[s], (i / S) & 1)) {
         *a.status = kDevTimeoutUnpack;
         break;
@@ -323,12 +343,126 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     pdl_wait_primary();
     for (int t = 0; t < my_tiles; ++t) {
       const int buf = t & 1;
-      int rt, tt;
-      tile_of(t, rt, tt);
+      int rt, tt, ks;
+      unit_of(t, rt, tt, ks);
       const int row0 = rt * kTcRows + q * 32;
       const int tok0 = tt * BN;
       float* scl = s_scale + buf * BN;
       int32_t* rsm = s_rowsum + buf * BN;
+      if (a.ksplit > 1) {
+        // ---- K slice: add the partial sums into the tile's fp32 sums; the last slice finishes the tile
+        if (!mbar_wait(&accfull[buf], (t >> 1) & 1)) {
+          *a.status = kDevTimeoutEpilogue;
+          break;
+        }
+        tc_fence_after();
+        const bool vec = (a.N % 4) == 0 && row0 + 32 <= a.N;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tc_ld_32x32b_x32(tmem + lane_base + buf * DCOLS + c0, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[j * 33 + lane] = v[j];
+          __syncwarp();
+          const int tcol = c0 + lane;  // lane l now holds token c0 + l, rows row0 .. row0 + 31
+          const int tok = tok0 + tcol;
+          if (tcol < BN && tok < a.M && row0 < a.N) {
+            float* dst = a.part + static_cast<size_t>(tok) * a.N + row0;
+            const uint32_t* src = stg + lane * 33;
+            if (vec) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                red_add_v4_f32(dst + e, static_cast<float>(static_cast<int32_t>(src[e])),
+                               static_cast<float>(static_cast<int32_t>(src[e + 1])),
+                               static_cast<float>(static_cast<int32_t>(src[e + 2])),
+                               static_cast<float>(static_cast<int32_t>(src[e + 3])));
+            } else {
+              for (int e = 0; e < 32 && row0 + e < a.N; ++e)
+                atomicAdd(dst + e, static_cast<float>(static_cast<int32_t>(src[e])));
+            }
+          }
+          __syncwarp();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[buf]);
+        __threadfence();
+        const int tile = rt * a.tok_tiles + tt;
+        for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
+          const int tok = tok0 + j;
+          scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), kQb) : 0.0f;  // RN(RN(alpha gamma) / 127)
+          rsm[j] = tok < a.M ? a.rowsum[tok] : 0;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == kTcEpiWarp0 * 32)
+          *s_last = (atomicAdd(&a.cnt[tile], 1u) == static_cast<uint32_t>(a.ksplit - 1)) ? 1 : 0;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*s_last) {
+          __threadfence();
+          if (threadIdx.x == kTcEpiWarp0 * 32) a.cnt[tile] = 0u;  // left zero for the next GEMM
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            const int tcol = c0 + lane;
+            const int tok = tok0 + tcol;
+            if (tcol < BN && tok < a.M && row0 < a.N) {
+              float* srcp = a.part + static_cast<size_t>(tok) * a.N + row0;
+              const float sc = scl[tcol];
+              const int32_t rs = rsm[tcol];
+              const size_t o = static_cast<size_t>(tok) * a.N + row0;
+              if (vec) {
+                int32_t tv[32];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                  const float4 f = __ldcg(reinterpret_cast<const float4*>(srcp + e));
+                  tv[e] = __float2int_rn(f.x) - rs;
+                  tv[e + 1] = __float2int_rn(f.y) - rs;
+                  tv[e + 2] = __float2int_rn(f.z) - rs;
+                  tv[e + 3] = __float2int_rn(f.w) - rs;
+                  __stcg(reinterpret_cast<float4*>(srcp + e), make_float4(0.f, 0.f, 0.f, 0.f));
+                }
+                if (a.vec_store) {
+                  uint32_t hb[16];
+#pragma unroll
+                  for (int e = 0; e < 32; e += 2) {
+                    const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv[e]), sc));
+                    const __nv_bfloat16 h1 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv[e + 1]), sc));
+                    hb[e >> 1] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h0)) |
+                                 (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h1)) << 16);
+                  }
+                  uint4* dy = reinterpret_cast<uint4*>(a.y + o);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) dy[e] = make_uint4(hb[4 * e], hb[4 * e + 1], hb[4 * e + 2], hb[4 * e + 3]);
+                  if (a.acc) {
+                    uint4* da = reinterpret_cast<uint4*>(a.acc + o);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                      da[e] = make_uint4(static_cast<uint32_t>(tv[4 * e]), static_cast<uint32_t>(tv[4 * e + 1]),
+                                         static_cast<uint32_t>(tv[4 * e + 2]), static_cast<uint32_t>(tv[4 * e + 3]));
+                  }
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) {
+                    if (a.acc) a.acc[o + e] = tv[e];
+                    const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv[e]), sc));
+                    a.y[o + e] = *reinterpret_cast<const uint16_t*>(&h);
+                  }
+                }
+              } else {
+                for (int e = 0; e < 32 && row0 + e < a.N; ++e) {
+                  const int32_t tv = __float2int_rn(__ldcg(srcp + e)) - rs;
+                  __stcg(srcp + e, 0.0f);
+                  if (a.acc) a.acc[o + e] = tv;
+                  const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), sc));
+                  a.y[o + e] = *reinterpret_cast<const uint16_t*>(&h);
+                }
+              }
+            }
+          }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // s_last and the scales are read before the next unit
+        continue;
+      }
       for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
         const int tok = tok0 + j;
         scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), kQb) : 0.0f;  // RN(RN(alpha gamma) / 127)

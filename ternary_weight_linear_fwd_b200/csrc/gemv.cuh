@@ -22,23 +22,6 @@ namespace bl {
 
 constexpr int kGemvThreads = 512;
 
-struct GemvArgs {
-  const uint8_t* codes;  // dense codes, or N:M kept values
-  const uint8_t* meta;   // N:M metadata (N:M kernel only)
-  int64_t ld;            // row stride of codes/values (bytes)
-  int64_t ld_meta;       // row stride of meta (bytes)
-  int N, K;
-  int C;                 // dense: 16-byte chunks per row; N:M: 128-weight units per row
-  int nm_n, nm_m;
-  const uint16_t* x;     // one bf16 row [K]
-  const float* alpha;
-  uint16_t* y;           // [N]
-  int32_t* acc;          // [N] or null
-  int tpr_log2;          // lanes per row = 1 << tpr_log2
-  int passes;            // chunk passes (C > CPT << tpr_log2)
-  int rows_base, rows_rem;  // CTA b owns rows_base (+1 if b < rows_rem) consecutive rows
-  int32_t* status;       // device status word
-};
 
 // Quantises the single activation row into shared memory: s_act[slot(g)]
 // holds the 16 codes of k-group g in contraction order (byte 4j + b <- k =
@@ -131,11 +114,6 @@ __device__ __forceinline__ int32_t chunk_sum(const int32_t* s_hsum, int ch) {
   const int4 a = reinterpret_cast<const int4*>(s_hsum)[2 * ch];
   const int4 b = reinterpret_cast<const int4*>(s_hsum)[2 * ch + 1];
   return (a.x + a.y) + (a.z + a.w) + ((b.x + b.y) + (b.z + b.w));
-}
-
-__device__ __forceinline__ int32_t group_sum(int32_t v, int tpr) {
-  for (int o = tpr >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
 }
 
 // Dot of one packed 32-bit weight word (16 codes) with its 4 activation words.
@@ -316,91 +294,181 @@ __device__ __forceinline__ uint32_t n8_dense_block(uint32_t mask8, uint32_t kept
   return x & 0xFFFFu;
 }
 
-// nbits (<= 32) bits starting at an even bit offset of a 16-byte aligned row;
-// the following word is read only when the field straddles it.
-__device__ __forceinline__ uint32_t load_bits(const uint8_t* base, int64_t bit, int nbits) {
-  const int64_t wi = bit >> 5;
-  const int sh = static_cast<int>(bit & 31);
-  const uint32_t* p = reinterpret_cast<const uint32_t*>(base);
-  const uint32_t lo = __ldg(p + wi);
-  if (sh == 0) return lo;
-  uint32_t v = lo >> sh;
-  if (sh + nbits > 32) v |= __ldg(p + wi + 1) << (32 - sh);
-  return v;
+// ------------------------------------------------------------------ N:M, M = 1
+// Same structure as the dense kernel: each CTA's rows of kept values and of
+// metadata arrive by TMA tile loads (128-byte swizzle) issued before the
+// dependency wait, x is quantised into shared memory, and a flat list of
+// (128-weight unit, row pair) units is spread over all threads.  A unit
+// rebuilds the dense 2-bit code words of its 128 weights (pruned positions get
+// code 01, weight 0) and runs the dense dot on them, so Σ q * code - Σ q over
+// the unit gives the exact partial sum.
+//   2:4: per block the 4-bit metadata (i0 | i1 << 2) and the block's two kept
+//        codes (4 bits) index a 256-entry table of dense code bytes; each lane
+//        reads its own bank-private copy (entry e of lane l at word e * 32 + l).
+//   n:8: the pruned positions of each 8-block are inserted one by one
+//        (n8_dense_block); the values of a unit are 4n bytes.
+constexpr int kNmLutWords = 256 * 32;
+
+struct GemvNmArgs {
+  const uint16_t* x;   // one bf16 row [K]
+  const float* alpha;
+  uint16_t* y;         // [N]
+  int32_t* acc;        // [N] or null
+  int32_t* status;
+  int64_t ld_v, ld_m;  // row strides of values / metadata (bytes)
+  int K, C;            // C = ceil(K / 128) units per row
+  int rows_base, rows_rem, rows_box;
+};
+
+__host__ __device__ __forceinline__ int nm_unit_value_bytes(int n) { return n == 0 ? 16 : 4 * n; }  // n = 0: 2:4
+
+__host__ __device__ __forceinline__ size_t gemv_nm_smem_bytes(int rows_box, int64_t ld_v, int64_t ld_m, int C, bool lut) {
+  return 1024 + static_cast<size_t>(gemv_stripes(ld_v) + gemv_stripes(ld_m)) * gemv_stripe_bytes(rows_box) +
+         (lut ? static_cast<size_t>(kNmLutWords) * 4 : 0) + static_cast<size_t>(C) * 8 * 16 /* codes */ +
+         static_cast<size_t>(C) * 16 * 4 /* half sums */ + static_cast<size_t>(rows_box) * 4;
 }
 
-// A lane owns 128-weight units (2:4: 32 blocks, n:8: 16 blocks) of a row.
-__global__ void __launch_bounds__(kGemvThreads) gemv_nm_m1_kernel(const GemvArgs a) {
-  extern __shared__ uint4 s_dyn[];
-  uint4* s_act = s_dyn;                                            // 8 * C entries
-  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_dyn + 8 * a.C);   // 16 * C half sums
+// 32-bit word at byte offset off (a multiple of 4) of local row r in swizzled 128-byte stripes.
+__device__ __forceinline__ uint32_t sw_word(const uint8_t* base, int stripe_bytes, int r, int off) {
+  const int w = off & 127;
+  return *reinterpret_cast<const uint32_t*>(base + (off >> 7) * stripe_bytes + r * 128 +
+                                            ((((w >> 4) ^ (r & 7)) << 4) | (w & 15)));
+}
+
+// Dense code word of 16 weights (4 blocks) of a 2:4 row from 16 bits of
+// metadata and 16 bits of kept codes, through the lane's table copy.
+__device__ __forceinline__ uint32_t nm24_word_lut(const uint32_t* lut_lane, uint32_t meta16, uint32_t vals16) {
+  // spread the four nibbles of each into the low nibbles of four bytes
+  uint32_t m = (meta16 | (meta16 << 8)) & 0x00FF00FFu;
+  m = (m | (m << 4)) & 0x0F0F0F0Fu;
+  uint32_t v = (vals16 | (vals16 << 8)) & 0x00FF00FFu;
+  v = (v | (v << 4)) & 0x0F0F0F0Fu;
+  const uint32_t idx = m | (v << 4);  // byte t: block t's table index
+  const uint32_t d0 = lut_lane[(idx & 0xFFu) << 5];
+  const uint32_t d1 = lut_lane[((idx >> 8) & 0xFFu) << 5];
+  const uint32_t d2 = lut_lane[((idx >> 16) & 0xFFu) << 5];
+  const uint32_t d3 = lut_lane[(idx >> 24) << 5];
+  return __byte_perm(__byte_perm(d0, d1, 0x0040), __byte_perm(d2, d3, 0x0040), 0x5410);
+}
+
+// Dense code words of the 8 groups of unit u of local row r.
+template <int NMN>
+__device__ __forceinline__ void nm_unit_words(const uint8_t* s_v, const uint8_t* s_m, int stripe_bytes, int r, int u,
+                                              const uint32_t* lut_lane, uint32_t (&dw)[8]) {
+  uint32_t mw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mw[i] = sw_word(s_m, stripe_bytes, r, 16 * u + 4 * i);
+  if (NMN == 0) {
+    uint32_t vw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vw[i] = sw_word(s_v, stripe_bytes, r, 16 * u + 4 * i);
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      dw[g] = nm24_word_lut(lut_lane, (mw[g >> 1] >> (16 * (g & 1))) & 0xFFFFu, (vw[g >> 1] >> (16 * (g & 1))) & 0xFFFFu);
+  } else {
+    constexpr int n = NMN;
+    uint32_t vw[n + 1];
+#pragma unroll
+    for (int i = 0; i < n; ++i) vw[i] = sw_word(s_v, stripe_bytes, r, 4 * n * u + 4 * i);
+    vw[n] = 0u;
+    constexpr uint32_t fmask = (1u << (2 * n)) - 1u;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const int bit = 4 * n * g;  // two blocks of n kept codes
+      const int wi = bit >> 5, sh = bit & 31;
+      const uint32_t kv = sh == 0 ? vw[wi] : __funnelshift_r(vw[wi], vw[wi + 1], sh);
+      const uint32_t m0 = (mw[g >> 1] >> (16 * (g & 1))) & 0xFFu, m1 = (mw[g >> 1] >> (16 * (g & 1) + 8)) & 0xFFu;
+      dw[g] = n8_dense_block(m0, kv & fmask) | (n8_dense_block(m1, (kv >> (2 * n)) & fmask) << 16);
+    }
+  }
+}
+
+template <int NMN>
+__global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_constant__ CUtensorMap map_v,
+                                                               const __grid_constant__ CUtensorMap map_m,
+                                                               const GemvNmArgs a) {
+  extern __shared__ uint8_t s_raw[];
+  __shared__ uint64_t s_bar;
   __shared__ float s_red[32];
-  pdl_launch_dependents();
-  const int tpr = 1 << a.tpr_log2;
-  const int sub = threadIdx.x & (tpr - 1);
-  const int grp = threadIdx.x >> a.tpr_log2;
-  const int ngrp = blockDim.x >> a.tpr_log2;
   const int b = blockIdx.x;
   const int r0 = b * a.rows_base + min(b, a.rows_rem);
   const int nrows = a.rows_base + (b < a.rows_rem ? 1 : 0);
+  const int C = a.C;
+  const int rows_box = a.rows_box;
+  const int stripes_v = gemv_stripes(a.ld_v), stripes_m = gemv_stripes(a.ld_m);
+  const int stripe_bytes = gemv_stripe_bytes(rows_box);
+  // offset arithmetic on the shared array keeps every derived pointer in the shared window
+  uint8_t* s_v = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
+  uint8_t* s_m = s_v + static_cast<size_t>(stripes_v) * stripe_bytes;
+  uint32_t* s_lut = reinterpret_cast<uint32_t*>(s_m + static_cast<size_t>(stripes_m) * stripe_bytes);
+  uint4* s_act = reinterpret_cast<uint4*>(s_lut + (NMN == 0 ? kNmLutWords : 0));
+  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_act + 8 * C);  // 16 * C half sums
+  int32_t* s_acc = s_hsum + 16 * C;
 
-  pdl_wait_primary();
-  const float gamma = quantise_row_smem(a.x, a.K, 8 * a.C, s_act, s_hsum, s_red);
-  const float s = __fdiv_rn(__fmul_rn(*a.alpha, gamma), kQb);
-  int32_t qsum = 0;  // this lane's share of sum(q): the two 64-weight chunks of each of its units
-  for (int u = sub; u < a.C; u += tpr) qsum += chunk_sum(s_hsum, 2 * u) + chunk_sum(s_hsum, 2 * u + 1);
-  const int n = a.nm_n, m = a.nm_m;
-  const int blocks_per_row = a.K / m;
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&map_v);
+    tma_prefetch_desc(&map_m);
+    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes_v + stripes_m) * 128u * static_cast<uint32_t>(rows_box));
+    const uint64_t pol = l2_policy_evict_first();
+    for (int st = 0; st < stripes_v; ++st) tma_load_2d_hint(s_v + st * stripe_bytes, &map_v, st * 128, r0, &s_bar, pol);
+    for (int st = 0; st < stripes_m; ++st) tma_load_2d_hint(s_m + st * stripe_bytes, &map_m, st * 128, r0, &s_bar, pol);
+  }
+  if (NMN == 0) {
+    // dense code byte of a 2:4 block from (i0 | i1 << 2) | (c0 | c1 << 2) << 4
+    for (int i = threadIdx.x; i < kNmLutWords; i += blockDim.x) {
+      const uint32_t e = static_cast<uint32_t>(i) >> 5;
+      const uint32_t i0 = e & 3u, i1 = (e >> 2) & 3u, c0 = (e >> 4) & 3u, c1 = (e >> 6) & 3u;
+      s_lut[i] = (0x55u ^ ((c0 ^ 1u) << (2 * i0)) ^ ((c1 ^ 1u) << (2 * i1))) & 0xFFu;
+    }
+  }
+  const float alpha = *a.alpha;
+  for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  __syncthreads();
 
-  const int iters = (nrows + ngrp - 1) / ngrp;
-  for (int it = 0; it < iters; ++it) {
-    const int lr = grp + it * ngrp;
-    const bool valid = lr < nrows;
-    int32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-    if (valid) {
-      const int64_t row = r0 + lr;
-      const uint8_t* vrow = a.codes + row * a.ld;
-      const uint8_t* mrow = a.meta + row * a.ld_meta;
-      for (int u = sub; u < a.C; u += tpr) {
-        // 8 groups of 16 dense weights per unit
-        const uint4 mq = *reinterpret_cast<const uint4*>(mrow + static_cast<int64_t>(u) * 16);
-        const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
+  pdl_wait_primary();  // x may come from the preceding kernel
+  const float gamma = quantise_row_smem(a.x, a.K, 8 * C, s_act, s_hsum, s_red);
+  pdl_launch_dependents();
+  const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
+  const bool landed = mbar_wait(&s_bar, 0);
+  if (!landed && threadIdx.x == 0) *a.status = kDevTimeoutProducer;
+
+  if (landed) {
+    const uint32_t* lut_lane = s_lut + (threadIdx.x & 31);
+    const int nthr = blockDim.x;
+    const int half = (nrows + 1) >> 1;
+    const int total = half * C;
+    const int dq = nthr / half, dr = nthr % half;
+    int u = threadIdx.x / half, p = threadIdx.x % half;
+    const int quarter = 2 * C;  // s_act slot stride: group g sits at (g % 4) * 2C + g / 4
+    for (int it = threadIdx.x; it < total; it += nthr) {
+      const int r2 = p + half < nrows ? p + half : p;
+      uint32_t da[8], db[8];
+      nm_unit_words<NMN>(s_v, s_m, stripe_bytes, p, u, lut_lane, da);
+      nm_unit_words<NMN>(s_v, s_m, stripe_bytes, r2, u, lut_lane, db);
+      const int32_t cs = chunk_sum(s_hsum, 2 * u) + chunk_sum(s_hsum, 2 * u + 1);
+      int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
 #pragma unroll
-        for (int gi = 0; gi < 8; ++gi) {
-          const int g = u * 8 + gi;  // 16-weight group index in the row
-          uint32_t dense;
-          if (m == 4) {
-            // group gi: blocks 4gi .. 4gi+3, meta nibbles 4gi.., kept codes 8gi..
-            dense = 0x55555555u;
-            if (g * 4 < blocks_per_row) {  // K is a multiple of 4, so a group is whole or absent
-              const uint32_t meta16 = (mw[gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
-              const uint32_t vals16 = load_bits(vrow, static_cast<int64_t>(g) * 16, 16) & 0xFFFFu;
-              dense = nm24_dense_word(meta16, vals16);
-            }
-          } else {
-            // group gi: blocks 2gi, 2gi+1, meta bytes 2gi, 2gi+1, kept codes n per block
-            const int blk = g * 2;
-            const uint32_t m0 = (mw[gi >> 1] >> (16 * (gi & 1))) & 0xFFu;
-            const uint32_t m1 = (mw[gi >> 1] >> (16 * (gi & 1) + 8)) & 0xFFu;
-            const uint32_t fmask = (1u << (2 * n)) - 1u;
-            dense = 0x55555555u;
-            if (blk + 1 < blocks_per_row) {
-              const uint32_t kv = load_bits(vrow, static_cast<int64_t>(blk) * n * 2, 4 * n);
-              dense = n8_dense_block(m0, kv & fmask) | (n8_dense_block(m1, (kv >> (2 * n)) & fmask) << 16);
-            } else if (blk < blocks_per_row) {
-              const uint32_t kv = load_bits(vrow, static_cast<int64_t>(blk) * n * 2, 2 * n);
-              dense = n8_dense_block(m0, kv & fmask) | (0x5555u << 16);
-            }
-          }
-          const uint4 av = s_act[(g & 3) * (2 * a.C) + (g >> 2)];
-          dot_word(dense, av.x, av.y, av.z, av.w, s0, s1, s2, s3);
-        }
+      for (int gi = 0; gi < 8; ++gi) {
+        const int g = 8 * u + gi;
+        const uint4 q = s_act[(g & 3) * quarter + (g >> 2)];
+        dot_word(da[gi], q.x, q.y, q.z, q.w, a0, a1, a2, a3);
+        dot_word(db[gi], q.x, q.y, q.z, q.w, b0, b1, b2, b3);
+      }
+      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6) - cs);
+      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6) - cs);
+      p += dr;
+      u += dq;
+      if (p >= half) {
+        p -= half;
+        ++u;
       }
     }
-    int32_t part = s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6) - qsum;
-    part = group_sum(part, tpr);
-    if (valid && sub == 0) gemv_store(a.y, a.acc, r0 + lr, part, s);
   }
+  __syncthreads();
+  if (landed)
+    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a.y, a.acc, r0 + rr, s_acc[rr], s);
 }
 
 }  // namespace bl

@@ -103,16 +103,30 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 // division-free exact rounding of codes8, one 16-byte store.  kPermute = false
 // writes natural-order codes [M, ldq] (ldq = K); kPermute = true writes the
 // contraction order [M, ldq] with ldq = K rounded up to 16 (zeros past K).
-// Both write gamma and, when asked, the sum of the row's codes.
+// Both write gamma and, when asked, the sum of the row's codes.  The first CTA
+// also clears the split-K arrival counters, and CTAs past the rows (blockIdx
+// >= qblocks) clear the split-K sums, of the GEMMs that read these codes.
 constexpr int kQuantRowsPerCta = 8;
 
 template <bool kPermute>
 __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                           int ldq, int8_t* __restrict__ q,
                                                                           float* __restrict__ gamma,
-                                                                          int32_t* __restrict__ rowsum) {
+                                                                          int32_t* __restrict__ rowsum,
+                                                                          uint32_t* __restrict__ cnt, int ncnt,
+                                                                          float* __restrict__ zbuf, size_t zvec4,
+                                                                          int qblocks) {
   pdl_wait_primary();
   pdl_launch_dependents();
+  // split-K arrival counters and sums of the GEMMs that follow start from zero
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < ncnt; i += blockDim.x) cnt[i] = 0u;
+  if (static_cast<int>(blockIdx.x) >= qblocks) {
+    const size_t stride = static_cast<size_t>(gridDim.x - qblocks) * blockDim.x;
+    for (size_t i = static_cast<size_t>(blockIdx.x - qblocks) * blockDim.x + threadIdx.x; i < zvec4; i += stride)
+      reinterpret_cast<float4*>(zbuf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kQuantRowsPerCta + (threadIdx.x >> 5);
   if (row >= M) return;

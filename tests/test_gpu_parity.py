@@ -224,6 +224,15 @@ def test_forward_nm(n, m, M, K, N):
     _check_rows(x, Wt, a, y, acc, np.arange(M))
 
 
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 6, 7])
+def test_forward_nm_gemv_every_n8(n):
+    """Decode GEMV for every n:8 pattern on a ragged shape (K not a multiple of the 128-weight unit)."""
+    x, Wt, a, w = _nm_case(1, 1032, 37, n, 8, seed=40 + n)
+    y, acc = bl.forward_nm(w, to_dev_bf16(x), want_acc=True)
+    assert bl.last_kernel() == "gemv_m1_n8"
+    _check_rows(x, Wt, a, y, acc, np.arange(1))
+
+
 @pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
 @pytest.mark.parametrize("K,N", [(2048, 11008), (11008, 2048)])
 def test_forward_nm_prefill_qwen_sampled(n, m, K, N):
