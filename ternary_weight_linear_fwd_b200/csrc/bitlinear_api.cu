@@ -152,14 +152,14 @@ struct TcPlan {
   int bn, row_tiles, tok_tiles, kblocks, ksplit, kbs;
 };
 
-TcPlan tc_plan(int M, int N, int K, int sm_count) {
+TcPlan tc_plan(int M, int N, int K, int nm, int sm_count) {
   TcPlan p;
   p.bn = pick_bn(M);
   p.row_tiles = (N + kTcRows - 1) / kTcRows;
   // narrower token tiles while the tiles would fill fewer than half the SMs
   while (p.bn > 32 && p.row_tiles * ((M + p.bn - 1) / p.bn) < sm_count / 2) p.bn >>= 1;
   p.tok_tiles = (M + p.bn - 1) / p.bn;
-  p.kblocks = (K + kTcBK - 1) / kTcBK;
+  p.kblocks = (K + tc_bk(nm) - 1) / tc_bk(nm);
   const int tiles = p.row_tiles * p.tok_tiles;
   int ks = 1;
   if (tiles < sm_count) ks = std::max(1, std::min(std::min(sm_count / tiles, p.kblocks / 2), 16));
@@ -180,8 +180,8 @@ size_t tc_base_bytes(int M, int K) {
 }
 size_t tc_cnt_bytes(int sm_count) { return align256(4 * static_cast<size_t>(sm_count)); }
 
-size_t tc_workspace(int M, int N, int K, int sm_count) {
-  const TcPlan p = tc_plan(M, N, K, sm_count);
+size_t tc_workspace(int M, int N, int K, int nm, int sm_count) {
+  const TcPlan p = tc_plan(M, N, K, nm, sm_count);
   size_t b = tc_base_bytes(M, K);
   if (p.ksplit > 1) b += tc_cnt_bytes(sm_count) + align256(static_cast<size_t>(M) * N * 4);
   return b;
@@ -256,12 +256,12 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
                          cudaStream_t s, DeviceState* dev) {
   const int N = w->N, K = w->K;
-  const TcPlan plan = tc_plan(M, N, K, dev->sm_count);
-  const int bn = plan.bn;
   const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? 1 : 2);
+  const TcPlan plan = tc_plan(M, N, K, nm, dev->sm_count);
+  const int bn = plan.bn;
   CUtensorMap mB, mA, mMeta;
   if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
-                   kTcBK, static_cast<uint32_t>(bn), true))
+                   kTcSubK, static_cast<uint32_t>(bn), true))
     return BITLINEAR_ERR_CUDA;
   TcArgs ta;
   ta.M = M;
@@ -286,7 +286,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
   if (nm == 0) {
     const int64_t ld = dense_ld(K);
-    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * tc_ksub(0), kTcRows, false)) return BITLINEAR_ERR_CUDA;
     mMeta = mA;
   } else {
     int64_t ldv = 0, ldm = 0;
@@ -310,8 +310,10 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
 
 bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
                             void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev) {
-  if (!ws || ws_bytes < tc_workspace(M, w->N, w->K, dev->sm_count) || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
-  const bool split = tc_plan(M, w->N, w->K, dev->sm_count).ksplit > 1;
+  const int nm = w->nm_m == 0 ? 0 : (w->nm_m == 4 ? 1 : 2);
+  if (!ws || ws_bytes < tc_workspace(M, w->N, w->K, nm, dev->sm_count) || !aligned16(ws))
+    return BITLINEAR_ERR_WORKSPACE;
+  const bool split = tc_plan(M, w->N, w->K, nm, dev->sm_count).ksplit > 1;
   const QuantWs qw = tc_ws_layout(ws, M, w->K, split ? dev->sm_count : 0, w->N);
   bitlinear_status st = tc_quant(x, M, w->K, qw, pdl, s);
   if (st != BITLINEAR_OK) return st;
@@ -526,8 +528,9 @@ bitlinear_status forward_group(const bitlinear_weights* w, int count, const uint
     bool split = false;
     int max_n = 0;
     for (int i = 0; i < count; ++i) {
-      need = std::max(need, tc_workspace(M, w[i].N, w[i].K, dev->sm_count));
-      if (tc_plan(M, w[i].N, w[i].K, dev->sm_count).ksplit > 1) {
+      const int nm = w[i].nm_m == 0 ? 0 : (w[i].nm_m == 4 ? 1 : 2);
+      need = std::max(need, tc_workspace(M, w[i].N, w[i].K, nm, dev->sm_count));
+      if (tc_plan(M, w[i].N, w[i].K, nm, dev->sm_count).ksplit > 1) {
         split = true;
         max_n = std::max(max_n, w[i].N);
       }
@@ -680,7 +683,10 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {
   if (M < 1 || K < 1 || N < 1) return 0;
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || (M > 1 && !(flags & BITLINEAR_FLAG_PATH_GEMV));
-  return tc ? tc_workspace(M, N, K, plan_sm_count()) : 0;
+  if (!tc) return 0;
+  // enough for dense and for N:M weights (their k-blocks differ, and with them the K split)
+  const int sm = plan_sm_count();
+  return std::max(tc_workspace(M, N, K, 0, sm), tc_workspace(M, N, K, 1, sm));
 }
 
 bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,

@@ -26,7 +26,8 @@
 // Warp roles (16 warps): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues
 // the MMAs, warp 2 owns the TMEM allocation, warps 4..11 unpack weights (two
 // groups of four, alternating k-blocks), warps 12..15 run the epilogue.  Warp
-// w reaches TMEM lanes 32 * (w % 4) .. + 31.  An 8-stage mbarrier ring couples
+// w reaches TMEM lanes 32 * (w % 4) .. + 31.  A mbarrier ring (4 to 8 stages of
+// 256 k for dense weights, 128 k for N:M; as many as TMEM has A slots for) couples
 // the producer, unpackers and MMA issuer (full: TMA bytes landed, aready: A
 // slot written, empty: the MMAs that read the stage completed); two TMEM
 // accumulators (accfull / accempty) let the epilogue of one tile overlap the
@@ -41,19 +42,21 @@
 
 namespace bl {
 
-#ifndef BL_TC_STAGES
-#define BL_TC_STAGES 8
-#endif
-constexpr int kTcStages = BL_TC_STAGES;
-constexpr int kTcBK = 128;      // K elements per stage (one 128-byte swizzle row)
+constexpr int kTcMaxStages = 8;
+constexpr int kTcSubK = 128;    // K elements of one 128-byte swizzle row of the activation tile
 constexpr int kTcRows = 128;    // weight rows per tile (MMA M)
 constexpr int kTcThreads = 512;
 constexpr int kTcEpiWarp0 = 12;  // first epilogue warp
-constexpr int kTcStageCols = 32;  // TMEM columns of one A slot (128 int8 per lane)
+
+// K elements per stage: dense weights take two 128-wide sub-tiles (eight MMAs
+// per barrier round trip, which halves the fixed cost of a stage per MAC);
+// N:M weights keep one.
+__host__ __device__ constexpr int tc_ksub(int NM) { return NM == 0 ? 2 : 1; }
+__host__ __device__ constexpr int tc_bk(int NM) { return kTcSubK * tc_ksub(NM); }
 
 struct TcArgs {
   int M, N, K;
-  int kblocks;            // ceil(K / 128)
+  int kblocks;            // ceil(K / tc_bk(NM))
   int row_tiles, tok_tiles;
   int ksplit;             // K slices per tile (1: no split)
   int kbs;                // k-blocks per slice, ceil(kblocks / ksplit)
@@ -74,27 +77,35 @@ template <int NM>
 struct TcStageBytes {
   // packed A bytes per stage (TMA box bytes, rows = 128)
   static __host__ __device__ constexpr int a_values(int vbox) {
-    return NM == 0 ? kTcRows * 32 : (NM == 1 ? kTcRows * 16 : kTcRows * vbox);
+    return NM == 0 ? kTcRows * 32 * tc_ksub(0) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox);
   }
   static __host__ __device__ constexpr int a_meta() { return NM == 0 ? 0 : kTcRows * 16; }
 };
 
-template <int BN>
+__host__ __device__ constexpr int tc_dcols(int BN) { return BN < 32 ? 32 : BN; }  // TMEM columns of one accumulator
+__host__ __device__ constexpr int tc_slot_cols(int NM) { return 32 * tc_ksub(NM); }  // TMEM columns of one A slot
+// Pipeline stages: as many A slots as fit beside the two accumulators, at most 8.
+__host__ __device__ constexpr int tc_stages(int BN, int NM) {
+  return (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM) < kTcMaxStages ? (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM)
+                                                                    : kTcMaxStages;
+}
+
+template <int BN, int NM>
 struct TcCols {
-  static constexpr int kDcols = BN < 32 ? 32 : BN;                 // one accumulator
+  static constexpr int kDcols = tc_dcols(BN);                      // one accumulator
   static constexpr int kAcol0 = 2 * kDcols;                        // A slots after both accumulators
-  static constexpr int kNeed = kAcol0 + kTcStages * kTcStageCols;
+  static constexpr int kNeed = kAcol0 + tc_stages(BN, NM) * tc_slot_cols(NM);
   static constexpr int kAlloc = kNeed <= 256 ? 256 : 512;
   static_assert(kNeed <= 512, "TMEM budget");
 };
 
 __host__ __device__ constexpr int tc_a_stage_bytes(int NM, int vbox) {
-  return ((NM == 0 ? kTcRows * 32 : (NM == 1 ? kTcRows * 16 : kTcRows * vbox)) + (NM == 0 ? 0 : kTcRows * 16) +
-          1023) / 1024 * 1024;
+  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox)) +
+          (NM == 0 ? 0 : kTcRows * 16) + 1023) / 1024 * 1024;
 }
 
 __host__ __device__ constexpr int tc_smem_bytes(int BN, int NM, int vbox) {
-  return 1024 /* alignment slack */ + kTcStages * (BN * 128 + tc_a_stage_bytes(NM, vbox)) +
+  return 1024 /* alignment slack */ + tc_stages(BN, NM) * (BN * 128 * tc_ksub(NM) + tc_a_stage_bytes(NM, vbox)) +
          4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
 }
 
@@ -124,12 +135,15 @@ template <int BN, int NM>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapMeta, const TcArgs a) {
-  constexpr int S = kTcStages;
-  constexpr int DCOLS = TcCols<BN>::kDcols;
-  constexpr int A_COL0 = TcCols<BN>::kAcol0;
-  constexpr int NCOLS = TcCols<BN>::kAlloc;
+  constexpr int S = tc_stages(BN, NM);
+  constexpr int KSUB = tc_ksub(NM);
+  constexpr int SLOT = tc_slot_cols(NM);
+  constexpr int DCOLS = TcCols<BN, NM>::kDcols;
+  constexpr int A_COL0 = TcCols<BN, NM>::kAcol0;
+  constexpr int NCOLS = TcCols<BN, NM>::kAlloc;
   constexpr uint32_t IDESC = idesc_i8_u8s8(kTcRows, BN);
-  constexpr int B_STAGE = BN * 128;
+  constexpr int B_SUB = BN * 128;         // one 128-wide K sub-tile of the activations
+  constexpr int B_STAGE = B_SUB * KSUB;
 
   extern __shared__ uint8_t smem_raw[];
   // offset arithmetic on the shared array keeps every derived pointer in the shared window
@@ -204,7 +218,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       auto load_a = [&](int row0, int kb, int s) {
         uint8_t* dst = sA + s * a_stage;
         if (NM == 0) {
-          tma_load_2d(dst, &mapA, kb * 32, row0, &full[s]);
+          tma_load_2d(dst, &mapA, kb * 32 * KSUB, row0, &full[s]);
         } else if (NM == 1) {
           tma_load_2d(dst, &mapA, kb * 16, row0, &full[s]);
           tma_load_2d(dst + a_val_bytes, &mapMeta, kb * 16, row0, &full[s]);
@@ -225,7 +239,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int i = 0; i < pre; ++i) {
         int rt, tt;
         const int kb = kblock_of(i, rt, tt);
-        tma_load_2d(sB + i * B_STAGE, &mapB, kb * kTcBK, tt * BN, &full[i]);
+        for (int sub = 0; sub < KSUB; ++sub)
+          tma_load_2d(sB + i * B_STAGE + sub * B_SUB, &mapB, (kb * KSUB + sub) * kTcSubK, tt * BN, &full[i]);
       }
       bool ok = true;
       int i = pre;
@@ -240,7 +255,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int kb = kblock_of(i, rt, tt);
         mbar_arrive_expect_tx(&full[s], tx_bytes);
         load_a(rt * kTcRows, kb, s);
-        tma_load_2d(sB + s * B_STAGE, &mapB, kb * kTcBK, tt * BN, &full[s]);
+        for (int sub = 0; sub < KSUB; ++sub)
+          tma_load_2d(sB + s * B_STAGE + sub * B_SUB, &mapB, (kb * KSUB + sub) * kTcSubK, tt * BN, &full[s]);
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
@@ -271,11 +287,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE));
 #pragma unroll
-          for (int kk = 0; kk < kTcBK / 32; ++kk)
-            tc_mma_i8_ts(dcol, tmem + A_COL0 + s * kTcStageCols + kk * 8, bdesc + static_cast<uint64_t>(kk * 2),
-                         IDESC, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4 * KSUB; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE + (kk >> 2) * B_SUB));
+            tc_mma_i8_ts(dcol, tmem + A_COL0 + s * SLOT + kk * 8, bdesc + static_cast<uint64_t>((kk & 3) * 2), IDESC,
+                         (kb | kk) != 0 ? 1u : 0u);
+          }
           tc_commit(&empty[s]);
           issued = true;
         }
@@ -305,30 +322,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint8_t* mrow = st + a_val_bytes + r * 16;
       int rem = 0;
       if (NM == 0)
-        arow = st + r * 32;
+        arow = st + r * 32 * KSUB;
       else if (NM == 1)
         arow = st + r * 16;
       else {
         arow = st + r * a.vbox;
         rem = (kb * 4 * a.nm_n) & 15;
       }
-      uint32_t dw[8];
-      if (NM == 0) {
-        const uint4 lo = reinterpret_cast<const uint4*>(arow)[0];
-        const uint4 hi = reinterpret_cast<const uint4*>(arow)[1];
-        dw[0] = lo.x; dw[1] = lo.y; dw[2] = lo.z; dw[3] = lo.w;
-        dw[4] = hi.x; dw[5] = hi.y; dw[6] = hi.z; dw[7] = hi.w;
-      } else {
 #pragma unroll
-        for (int gi = 0; gi < 8; ++gi) dw[gi] = tc_group_word<NM>(arow, mrow, gi, a.nm_n, rem);
+      for (int sub = 0; sub < KSUB; ++sub) {
+        uint32_t dw[8];
+        if (NM == 0) {
+          const uint4 lo = reinterpret_cast<const uint4*>(arow)[2 * sub];
+          const uint4 hi = reinterpret_cast<const uint4*>(arow)[2 * sub + 1];
+          dw[0] = lo.x; dw[1] = lo.y; dw[2] = lo.z; dw[3] = lo.w;
+          dw[4] = hi.x; dw[5] = hi.y; dw[6] = hi.z; dw[7] = hi.w;
+        } else {
+#pragma unroll
+          for (int gi = 0; gi < 8; ++gi) dw[gi] = tc_group_word<NM>(arow, mrow, gi, a.nm_n, rem);
+        }
+        uint32_t outw[32];
+#pragma unroll
+        for (int gi = 0; gi < 8; ++gi) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) outw[4 * gi + j] = (dw[gi] >> (2 * j)) & 0x03030303u;
+        }
+        tc_st_32x32b_x32(tmem + lane_base + A_COL0 + s * SLOT + sub * 32, outw);
       }
-      uint32_t outw[32];
-#pragma unroll
-      for (int gi = 0; gi < 8; ++gi) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) outw[4 * gi + j] = (dw[gi] >> (2 * j)) & 0x03030303u;
-      }
-      tc_st_32x32b_x32(tmem + lane_base + A_COL0 + s * kTcStageCols, outw);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
