@@ -159,7 +159,7 @@ TcPlan tc_plan(int M, int N, int K, int nm, int sm_count) {
   // narrower token tiles while the tiles would fill fewer than half the SMs
   while (p.bn > 32 && p.row_tiles * ((M + p.bn - 1) / p.bn) < sm_count / 2) p.bn >>= 1;
   p.tok_tiles = (M + p.bn - 1) / p.bn;
-  p.kblocks = (K + tc_bk(nm) - 1) / tc_bk(nm);
+  p.kblocks = (K + tc_bk(nm, p.bn) - 1) / tc_bk(nm, p.bn);
   const int tiles = p.row_tiles * p.tok_tiles;
   int ks = 1;
   if (tiles < sm_count) ks = std::max(1, std::min(std::min(sm_count / tiles, p.kblocks / 2), 16));
@@ -243,14 +243,16 @@ QuantWs tc_ws_layout(void* ws, int M, int K, int ncnt, int max_n) {
 }
 
 bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s) {
-  const int qblocks = (M + kQuantRowsPerCta - 1) / kQuantRowsPerCta;
+  const int wpr = quant_warps_per_row(K);
+  const int rows_per_cta = kQuantWarps / wpr;
+  const int qblocks = (M + rows_per_cta - 1) / rows_per_cta;
   // extra CTAs clear the split-K sums, 16 bytes per thread and step, at most four steps each
   const size_t vec4 = (qw.part_words + 3) / 4;
-  const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * 32 * kQuantRowsPerCta - 1) /
-                                                                   (4 * 32 * kQuantRowsPerCta)));
-  return launch(quant_act_kernel<true>, dim3(qblocks + zblocks), dim3(32 * kQuantRowsPerCta), 0, s, pdl, x, M, K,
+  const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * 32 * kQuantWarps - 1) /
+                                                                   (4 * 32 * kQuantWarps)));
+  return launch(quant_act_kernel<true>, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
                 static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum,
-                qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr), qw.ncnt, qw.part, vec4, qblocks);
+                qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr), qw.ncnt, qw.part, vec4, qblocks, wpr);
 }
 
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
@@ -286,7 +288,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
   if (nm == 0) {
     const int64_t ld = dense_ld(K);
-    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * tc_ksub(0), kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * tc_ksub(0, bn), kTcRows, false)) return BITLINEAR_ERR_CUDA;
     mMeta = mA;
   } else {
     int64_t ldv = 0, ldm = 0;
@@ -672,10 +674,11 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
   DeviceState* dev = nullptr;
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
-  st = launch(quant_act_kernel<false>, dim3((M + kQuantRowsPerCta - 1) / kQuantRowsPerCta),
-              dim3(32 * kQuantRowsPerCta), 0, static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum,
-              static_cast<uint32_t*>(nullptr), 0, static_cast<float*>(nullptr), static_cast<size_t>(0),
-              (M + kQuantRowsPerCta - 1) / kQuantRowsPerCta);
+  const int wpr = quant_warps_per_row(K);
+  const int qblocks = (M + kQuantWarps / wpr - 1) / (kQuantWarps / wpr);
+  st = launch(quant_act_kernel<false>, dim3(qblocks), dim3(32 * kQuantWarps), 0, static_cast<cudaStream_t>(stream), false,
+              x, M, K, K, q, gamma, rowsum, static_cast<uint32_t*>(nullptr), 0, static_cast<float*>(nullptr),
+              static_cast<size_t>(0), qblocks, wpr);
   if (st == BITLINEAR_OK) t_last_kernel = "quant_act";
   return st;
 }

@@ -48,11 +48,11 @@ constexpr int kTcRows = 128;    // weight rows per tile (MMA M)
 constexpr int kTcThreads = 512;
 constexpr int kTcEpiWarp0 = 12;  // first epilogue warp
 
-// K elements per stage: dense weights take two 128-wide sub-tiles (eight MMAs
-// per barrier round trip, which halves the fixed cost of a stage per MAC);
-// N:M weights keep one.
-__host__ __device__ constexpr int tc_ksub(int NM) { return NM == 0 ? 2 : 1; }
-__host__ __device__ constexpr int tc_bk(int NM) { return kTcSubK * tc_ksub(NM); }
+// K elements per stage: dense weights with token tiles up to 128 take two
+// 128-wide sub-tiles (eight MMAs per barrier round trip, which halves the fixed
+// cost of a stage per MAC); wider tiles and N:M weights keep one.
+__host__ __device__ constexpr int tc_ksub(int NM, int BN) { return (NM == 0 && BN <= 128) ? 2 : 1; }
+__host__ __device__ constexpr int tc_bk(int NM, int BN) { return kTcSubK * tc_ksub(NM, BN); }
 
 struct TcArgs {
   int M, N, K;
@@ -73,39 +73,41 @@ struct TcArgs {
   int32_t* status;        // device status word
 };
 
-template <int NM>
+template <int NM, int BN>
 struct TcStageBytes {
   // packed A bytes per stage (TMA box bytes, rows = 128)
   static __host__ __device__ constexpr int a_values(int vbox) {
-    return NM == 0 ? kTcRows * 32 * tc_ksub(0) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox);
+    return NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox);
   }
   static __host__ __device__ constexpr int a_meta() { return NM == 0 ? 0 : kTcRows * 16; }
 };
 
 __host__ __device__ constexpr int tc_dcols(int BN) { return BN < 32 ? 32 : BN; }  // TMEM columns of one accumulator
-__host__ __device__ constexpr int tc_slot_cols(int NM) { return 32 * tc_ksub(NM); }  // TMEM columns of one A slot
+__host__ __device__ constexpr int tc_slot_cols(int NM, int BN) { return 32 * tc_ksub(NM, BN); }  // one A slot
 // Pipeline stages: as many A slots as fit beside the two accumulators, at most 8.
 __host__ __device__ constexpr int tc_stages(int BN, int NM) {
-  return (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM) < kTcMaxStages ? (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM)
-                                                                    : kTcMaxStages;
+  return (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM, BN) < kTcMaxStages
+             ? (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM, BN)
+             : kTcMaxStages;
 }
 
 template <int BN, int NM>
 struct TcCols {
   static constexpr int kDcols = tc_dcols(BN);                      // one accumulator
   static constexpr int kAcol0 = 2 * kDcols;                        // A slots after both accumulators
-  static constexpr int kNeed = kAcol0 + tc_stages(BN, NM) * tc_slot_cols(NM);
+  static constexpr int kNeed = kAcol0 + tc_stages(BN, NM) * tc_slot_cols(NM, BN);
   static constexpr int kAlloc = kNeed <= 256 ? 256 : 512;
   static_assert(kNeed <= 512, "TMEM budget");
 };
 
-__host__ __device__ constexpr int tc_a_stage_bytes(int NM, int vbox) {
-  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox)) +
+__host__ __device__ constexpr int tc_a_stage_bytes(int NM, int BN, int vbox) {
+  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox)) +
           (NM == 0 ? 0 : kTcRows * 16) + 1023) / 1024 * 1024;
 }
 
 __host__ __device__ constexpr int tc_smem_bytes(int BN, int NM, int vbox) {
-  return 1024 /* alignment slack */ + tc_stages(BN, NM) * (BN * 128 * tc_ksub(NM) + tc_a_stage_bytes(NM, vbox)) +
+  return 1024 /* alignment slack */ +
+         tc_stages(BN, NM) * (BN * 128 * tc_ksub(NM, BN) + tc_a_stage_bytes(NM, BN, vbox)) +
          4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
 }
 
@@ -136,8 +138,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapA,
                    const __grid_constant__ CUtensorMap mapMeta, const TcArgs a) {
   constexpr int S = tc_stages(BN, NM);
-  constexpr int KSUB = tc_ksub(NM);
-  constexpr int SLOT = tc_slot_cols(NM);
+  constexpr int KSUB = tc_ksub(NM, BN);
+  constexpr int SLOT = tc_slot_cols(NM, BN);
   constexpr int DCOLS = TcCols<BN, NM>::kDcols;
   constexpr int A_COL0 = TcCols<BN, NM>::kAcol0;
   constexpr int NCOLS = TcCols<BN, NM>::kAlloc;
@@ -148,9 +150,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   // offset arithmetic on the shared array keeps every derived pointer in the shared window
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const int a_val_bytes = TcStageBytes<NM>::a_values(a.vbox);
-  const int a_meta_bytes = TcStageBytes<NM>::a_meta();
-  const int a_stage = tc_a_stage_bytes(NM, a.vbox);
+  const int a_val_bytes = TcStageBytes<NM, BN>::a_values(a.vbox);
+  const int a_meta_bytes = TcStageBytes<NM, BN>::a_meta();
+  const int a_stage = tc_a_stage_bytes(NM, BN, a.vbox);
   uint8_t* sB = base;
   uint8_t* sA = base + S * B_STAGE;
   uint32_t* s_stage = reinterpret_cast<uint32_t*>(sA + S * a_stage);   // 4 warps x 32 x 33 words

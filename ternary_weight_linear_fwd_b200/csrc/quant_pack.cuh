@@ -97,25 +97,72 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 }
 
 // ----------------------------------------------------------------- quant_act
-// One warp per token row (eight rows per 256-thread CTA).  Pass one reads the
-// row for gamma (all loads of a lane in flight together); pass two re-reads it
-// (now from L1/L2) one 16-wide k-group per lane and step: 16 codes by the
-// division-free exact rounding of codes8, one 16-byte store.  kPermute = false
-// writes natural-order codes [M, ldq] (ldq = K); kPermute = true writes the
-// contraction order [M, ldq] with ldq = K rounded up to 16 (zeros past K).
-// Both write gamma and, when asked, the sum of the row's codes.  The first CTA
-// also clears the split-K arrival counters, and CTAs past the rows (blockIdx
-// >= qblocks) clear the split-K sums, of the GEMMs that read these codes.
-constexpr int kQuantRowsPerCta = 8;
+// A token row is handled by wpr warps of a 256-thread CTA (wpr = 1, 2, 4 or 8,
+// chosen by K; 8 / wpr rows per CTA).  A lane owns the 16-wide k-groups
+// g = sub * 32 + lane + j * 32 * wpr of its row; when the row fits (K % 8 == 0,
+// at most kQuantGroupsInRegs groups per lane) every load of the row is issued
+// at once into registers, so each element is read from memory once and all of
+// a CTA's reads are in flight together.  gamma is an integer warp max of the
+// |x| bit patterns (then across the row's warps), and the 16 codes of a group
+// come from the division-free exact rounding of codes8.  Longer or unaligned
+// rows take a two-pass loop (the second pass re-reads from L1/L2).
+// kPermute = false writes natural-order codes [M, ldq] (ldq = K); kPermute =
+// true writes the contraction order [M, ldq] with ldq = K rounded up to 16
+// (zeros past K).  Both write gamma and, when asked, the sum of the row's
+// codes.  The first CTA also clears the split-K arrival counters, and CTAs
+// past the rows (blockIdx >= qblocks) clear the split-K sums, of the GEMMs that
+// read these codes.
+constexpr int kQuantWarps = 8;
+constexpr int kQuantGroupsInRegs = 8;
+
+__host__ __device__ __forceinline__ int quant_warps_per_row(int K) {
+  return K <= 4096 ? 1 : K <= 8192 ? 2 : K <= 16384 ? 4 : 8;
+}
+
+// 16 codes of one k-group (raw: the group's 16 bf16 as 8 words) in the
+// requested order; adds their sum to *sum.
+template <bool kPermute>
+__device__ __forceinline__ uint4 group_codes(const uint32_t (&r0)[4], const uint32_t (&r1)[4], float c, float d,
+                                             int32_t& sum) {
+  uint32_t b0[8], b1[8], w[4];
+  codes8(r0, c, d, b0);  // elements past K are zero and give code 0
+  codes8(r1, c, d, b1);
+  if (kPermute) {
+    // byte 4j + b <- k0 + 4b + j
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = __byte_perm(__byte_perm(b0[j], b0[4 + j], 0x0040), __byte_perm(b1[j], b1[4 + j], 0x0040), 0x5410);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      w[j] = __byte_perm(__byte_perm(b0[4 * j], b0[4 * j + 1], 0x0040), __byte_perm(b0[4 * j + 2], b0[4 * j + 3], 0x0040),
+                         0x5410);
+      w[2 + j] = __byte_perm(__byte_perm(b1[4 * j], b1[4 * j + 1], 0x0040),
+                             __byte_perm(b1[4 * j + 2], b1[4 * j + 3], 0x0040), 0x5410);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) sum = __dp4a(static_cast<int>(w[j]), 0x01010101, sum);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ float absmax8(const uint32_t (&w)[4], float mx) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+  return mx;
+}
 
 template <bool kPermute>
-__global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
-                                                                          int ldq, int8_t* __restrict__ q,
-                                                                          float* __restrict__ gamma,
-                                                                          int32_t* __restrict__ rowsum,
-                                                                          uint32_t* __restrict__ cnt, int ncnt,
-                                                                          float* __restrict__ zbuf, size_t zvec4,
-                                                                          int qblocks) {
+__global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                                     int ldq, int8_t* __restrict__ q,
+                                                                     float* __restrict__ gamma,
+                                                                     int32_t* __restrict__ rowsum,
+                                                                     uint32_t* __restrict__ cnt, int ncnt,
+                                                                     float* __restrict__ zbuf, size_t zvec4,
+                                                                     int qblocks, int wpr) {
+  __shared__ float s_mx[kQuantWarps];
+  __shared__ int32_t s_sum[kQuantWarps];
   pdl_wait_primary();
   pdl_launch_dependents();
   // split-K arrival counters and sums of the GEMMs that follow start from zero
@@ -127,67 +174,92 @@ __global__ void __launch_bounds__(32 * kQuantRowsPerCta) quant_act_kernel(const 
       reinterpret_cast<float4*>(zbuf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kQuantRowsPerCta + (threadIdx.x >> 5);
-  if (row >= M) return;
-  const uint16_t* xr = x + static_cast<size_t>(row) * K;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rloc = warp / wpr, sub = warp - rloc * wpr;
+  const int row = blockIdx.x * (kQuantWarps / wpr) + rloc;
+  const bool active = row < M;  // inactive warps still reach the CTA barriers
+  const uint16_t* xr = x + static_cast<size_t>(active ? row : 0) * K;
   const bool vec_ok = (K % 8) == 0 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
+  const int groups = (K + 15) / 16;
+  const int gstride = 32 * wpr;
+  const int g0 = sub * 32 + lane;
+  const bool in_regs = vec_ok && groups <= kQuantGroupsInRegs * gstride;
 
+  uint32_t v[kQuantGroupsInRegs][8];
   float mx = 0.0f;
-  const int halves = (K + 7) / 8;
-  if (vec_ok) {
-#pragma unroll 4
-    for (int h = lane; h < halves; h += 32) {
-      const uint4 a = *reinterpret_cast<const uint4*>(xr + 8 * h);
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  if (active) {
+    if (in_regs) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+      for (int j = 0; j < kQuantGroupsInRegs; ++j) {
+        const int k0 = 16 * (g0 + j * gstride);
+        uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
+        if (k0 + 8 <= K) a = *reinterpret_cast<const uint4*>(xr + k0);
+        if (k0 + 16 <= K) b = *reinterpret_cast<const uint4*>(xr + k0 + 8);
+        v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
+        v[j][4] = b.x; v[j][5] = b.y; v[j][6] = b.z; v[j][7] = b.w;
+      }
+#pragma unroll
+      for (int j = 0; j < kQuantGroupsInRegs; ++j) {
+        const uint32_t lo[4] = {v[j][0], v[j][1], v[j][2], v[j][3]}, hi[4] = {v[j][4], v[j][5], v[j][6], v[j][7]};
+        mx = absmax8(hi, absmax8(lo, mx));
+      }
+    } else {
+      for (int g = g0; g < groups; g += gstride) {
+        uint32_t r0[4], r1[4];
+        load8_raw(xr, 16 * g, K, vec_ok, r0);
+        load8_raw(xr, 16 * g + 8, K, vec_ok, r1);
+        mx = absmax8(r1, absmax8(r0, mx));
+      }
     }
-  } else {
-    for (int k = lane; k < K; k += 32) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(xr[k])));
   }
-  // |x| >= 0, whose bit patterns order like the values: one integer warp reduction
+  // |x| >= 0, whose bit patterns order like the values: integer maxima
   mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+  if (wpr > 1) {
+    if (lane == 0) s_mx[warp] = mx;
+    __syncthreads();
+    for (int i = 0; i < wpr; ++i) mx = fmaxf(mx, s_mx[rloc * wpr + i]);
+  }
   const float d = __fadd_rn(mx, kEps);
   const float c = __fmul_rn(kQb, __frcp_rn(d));
 
   int32_t sum = 0;
-  const int groups = (K + 15) / 16;
-  int8_t* qr = q + static_cast<size_t>(row) * ldq;
-  const bool qvec = ((reinterpret_cast<uintptr_t>(q) & 15u) == 0) && (ldq % 16) == 0;
-  for (int g = lane; g < groups; g += 32) {
-    const int k0 = g * 16;
-    uint32_t r0[4], r1[4], b0[8], b1[8];
-    load8_raw(xr, k0, K, vec_ok, r0);
-    load8_raw(xr, k0 + 8, K, vec_ok, r1);
-    codes8(r0, c, d, b0);  // elements past K are zero and give code 0
-    codes8(r1, c, d, b1);
-    uint32_t w[4];
-    if (kPermute) {
-      // byte 4j + b <- k0 + 4b + j
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        w[j] = __byte_perm(__byte_perm(b0[j], b0[4 + j], 0x0040), __byte_perm(b1[j], b1[4 + j], 0x0040), 0x5410);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        w[j] = __byte_perm(__byte_perm(b0[4 * j], b0[4 * j + 1], 0x0040), __byte_perm(b0[4 * j + 2], b0[4 * j + 3], 0x0040),
-                           0x5410);
-        w[2 + j] = __byte_perm(__byte_perm(b1[4 * j], b1[4 * j + 1], 0x0040),
-                               __byte_perm(b1[4 * j + 2], b1[4 * j + 3], 0x0040), 0x5410);
+  if (active) {
+    int8_t* qr = q + static_cast<size_t>(row) * ldq;
+    const bool qvec = ((reinterpret_cast<uintptr_t>(q) & 15u) == 0) && (ldq % 16) == 0;
+    auto put = [&](int k0, const uint4& w) {
+      if (kPermute || (qvec && k0 + 16 <= K)) {
+        *reinterpret_cast<uint4*>(qr + k0) = w;
+      } else {
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int i = 0; i < 16 && k0 + i < K; ++i) qr[k0 + i] = static_cast<int8_t>(ww[i >> 2] >> (8 * (i & 3)));
       }
-    }
+    };
+    if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) sum = __dp4a(static_cast<int>(w[j]), 0x01010101, sum);
-    if (kPermute || (qvec && k0 + 16 <= K)) {
-      *reinterpret_cast<uint4*>(qr + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int j = 0; j < kQuantGroupsInRegs; ++j) {
+        const int g = g0 + j * gstride;
+        if (g < groups) {
+          const uint32_t lo[4] = {v[j][0], v[j][1], v[j][2], v[j][3]}, hi[4] = {v[j][4], v[j][5], v[j][6], v[j][7]};
+          put(16 * g, group_codes<kPermute>(lo, hi, c, d, sum));
+        }
+      }
     } else {
-      for (int i = 0; i < 16 && k0 + i < K; ++i) qr[k0 + i] = static_cast<int8_t>(w[i >> 2] >> (8 * (i & 3)));
+      for (int g = g0; g < groups; g += gstride) {
+        uint32_t r0[4], r1[4];
+        load8_raw(xr, 16 * g, K, vec_ok, r0);
+        load8_raw(xr, 16 * g + 8, K, vec_ok, r1);
+        put(16 * g, group_codes<kPermute>(r0, r1, c, d, sum));
+      }
     }
   }
   sum = __reduce_add_sync(0xffffffffu, sum);
-  if (lane == 0) {
+  if (wpr > 1) {
+    if (lane == 0) s_sum[warp] = sum;
+    __syncthreads();
+    sum = 0;
+    for (int i = 0; i < wpr; ++i) sum += s_sum[rloc * wpr + i];
+  }
+  if (active && sub == 0 && lane == 0) {
     if (gamma) gamma[row] = mx;
     if (rowsum) rowsum[row] = sum;
   }
