@@ -108,6 +108,7 @@ __host__ __device__ constexpr int tc_a_stage_bytes(int NM, int BN, int vbox) {
 __host__ __device__ constexpr int tc_smem_bytes(int BN, int NM, int vbox) {
   return 1024 /* alignment slack */ +
          tc_stages(BN, NM) * (BN * 128 * tc_ksub(NM, BN) + tc_a_stage_bytes(NM, BN, vbox)) +
+         (NM == 1 ? kNmLutWords * 4 : 0) /* 2:4 expansion table, one copy per lane */ +
          4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
 }
 
@@ -155,7 +156,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int a_stage = tc_a_stage_bytes(NM, BN, a.vbox);
   uint8_t* sB = base;
   uint8_t* sA = base + S * B_STAGE;
-  uint32_t* s_stage = reinterpret_cast<uint32_t*>(sA + S * a_stage);   // 4 warps x 32 x 33 words
+  uint32_t* s_lut = reinterpret_cast<uint32_t*>(sA + S * a_stage);     // 2:4 only: [256][32] dense code bytes
+  uint32_t* s_stage = s_lut + (NM == 1 ? kNmLutWords : 0);               // 4 warps x 32 x 33 words
   float* s_scale = reinterpret_cast<float*>(s_stage + 4 * 32 * 33);     // [2][BN]
   int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * BN);     // [2][BN]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_rowsum + 2 * BN);
@@ -209,6 +211,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(tmem_slot, NCOLS);
     tmem_relinquish();
   }
+  if (NM == 1) nm24_fill_lut(s_lut);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -339,6 +342,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint4 hi = reinterpret_cast<const uint4*>(arow)[2 * sub + 1];
           dw[0] = lo.x; dw[1] = lo.y; dw[2] = lo.z; dw[3] = lo.w;
           dw[4] = hi.x; dw[5] = hi.y; dw[6] = hi.z; dw[7] = hi.w;
+        } else if (NM == 1) {
+          // 16 bytes of kept codes and 16 of metadata per row: 8 groups of 16 weights
+          const uint4 vv = *reinterpret_cast<const uint4*>(arow);
+          const uint4 mm = *reinterpret_cast<const uint4*>(mrow);
+          const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w}, mw[4] = {mm.x, mm.y, mm.z, mm.w};
+          const uint32_t* lut_lane = s_lut + lane;
+#pragma unroll
+          for (int gi = 0; gi < 8; ++gi)
+            dw[gi] = nm24_word_lut(lut_lane, (mw[gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu,
+                                   (vw[gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu);
         } else {
 #pragma unroll
           for (int gi = 0; gi < 8; ++gi) dw[gi] = tc_group_word<NM>(arow, mrow, gi, a.nm_n, rem);

@@ -335,6 +335,17 @@ __device__ __forceinline__ uint32_t sw_word(const uint8_t* base, int stripe_byte
                                             ((((w >> 4) ^ (r & 7)) << 4) | (w & 15)));
 }
 
+// Fills the 2:4 table (all threads of the CTA): entry e = (i0 | i1 << 2) |
+// (c0 | c1 << 2) << 4 holds the dense code byte of a block, lane l's copy at
+// word e * 32 + l.
+__device__ __forceinline__ void nm24_fill_lut(uint32_t* s_lut) {
+  for (int i = threadIdx.x; i < kNmLutWords; i += blockDim.x) {
+    const uint32_t e = static_cast<uint32_t>(i) >> 5;
+    const uint32_t i0 = e & 3u, i1 = (e >> 2) & 3u, c0 = (e >> 4) & 3u, c1 = (e >> 6) & 3u;
+    s_lut[i] = (0x55u ^ ((c0 ^ 1u) << (2 * i0)) ^ ((c1 ^ 1u) << (2 * i1))) & 0xFFu;
+  }
+}
+
 // Dense code word of 16 weights (4 blocks) of a 2:4 row from 16 bits of
 // metadata and 16 bits of kept codes, through the lane's table copy.
 __device__ __forceinline__ uint32_t nm24_word_lut(const uint32_t* lut_lane, uint32_t meta16, uint32_t vals16) {
@@ -415,14 +426,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
     for (int st = 0; st < stripes_v; ++st) tma_load_2d_hint(s_v + st * stripe_bytes, &map_v, st * 128, r0, &s_bar, pol);
     for (int st = 0; st < stripes_m; ++st) tma_load_2d_hint(s_m + st * stripe_bytes, &map_m, st * 128, r0, &s_bar, pol);
   }
-  if (NMN == 0) {
-    // dense code byte of a 2:4 block from (i0 | i1 << 2) | (c0 | c1 << 2) << 4
-    for (int i = threadIdx.x; i < kNmLutWords; i += blockDim.x) {
-      const uint32_t e = static_cast<uint32_t>(i) >> 5;
-      const uint32_t i0 = e & 3u, i1 = (e >> 2) & 3u, c0 = (e >> 4) & 3u, c1 = (e >> 6) & 3u;
-      s_lut[i] = (0x55u ^ ((c0 ^ 1u) << (2 * i0)) ^ ((c1 ^ 1u) << (2 * i1))) & 0xFFu;
-    }
-  }
+  if (NMN == 0) nm24_fill_lut(s_lut);
   const float alpha = *a.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
   __syncthreads();
