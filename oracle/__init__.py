@@ -59,6 +59,8 @@ def _load():
             "orc_pack_nm": (i32, [P, P, i32, i32, i32, i32, P, P]),
             "orc_unpack_nm": (i32, [P, P, i32, i32, i32, i32, P]),
             "orc_quant_act": (None, [P, i32, i32, i32, P, P, P]),
+            "orc_rmsnorm": (None, [P, P, i32, i32, f32, P]),
+            "orc_quant_act_f32": (None, [P, i32, i32, i32, P, P, P]),
             "orc_matmul_i32": (i32, [P, P, i32, i32, i32, P]),
             "orc_dequant": (None, [P, P, f32, i32, i32, i32, P]),
             "orc_bf16_from_f64": (ctypes.c_uint16, [ctypes.c_double]),
@@ -168,6 +170,37 @@ def quant_act(x_bf16: np.ndarray, Qb: int = QB):
     rs = np.empty(M, dtype=np.int32)
     _load().orc_quant_act(_ptr(x), M, K, Qb, _ptr(q), _ptr(g), _ptr(rs))
     return q, g, rs
+
+
+def rmsnorm(x_bf16: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """fp32 [M,K]: RN(RN(x * r) * g), r = RN32(1 / sqrt(RN32(mean x^2) + eps)) in fp64."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    assert g.shape == (K,)
+    xn = np.empty((M, K), dtype=np.float32)
+    _load().orc_rmsnorm(_ptr(x), _ptr(g), M, K, eps, _ptr(xn))
+    return xn
+
+
+def quant_act_f32(xn: np.ndarray, Qb: int = QB):
+    """(q int8 [M,K], gamma fp32 [M], rowsum int32 [M]) from fp32 rows."""
+    xn = np.ascontiguousarray(xn, dtype=np.float32)
+    M, K = xn.shape
+    q = np.empty((M, K), dtype=np.int8)
+    gm = np.empty(M, dtype=np.float32)
+    rs = np.empty(M, dtype=np.int32)
+    _load().orc_quant_act_f32(_ptr(xn), M, K, Qb, _ptr(q), _ptr(gm), _ptr(rs))
+    return q, gm, rs
+
+
+def forward_norm(x_bf16: np.ndarray, g: np.ndarray, eps: float, Wt: np.ndarray, alpha, Qb: int = QB):
+    """BitLinear with RMSNorm first: (y bf16 bits, acc int32, q, gamma, rowsum)."""
+    xn = rmsnorm(x_bf16, g, eps)
+    q, gm, rs = quant_act_f32(xn, Qb)
+    acc = matmul_i32(q, Wt)
+    y = dequant(acc, gm, alpha, Qb)
+    return y, acc, q, gm, rs
 
 
 def matmul_i32(q: np.ndarray, Wt: np.ndarray) -> np.ndarray:

@@ -37,6 +37,13 @@
  *  - N:M blocks are M consecutive positions along K inside one output row;
  *    ties in |W| go to the lower position; the mask is applied after
  *    ternarisation; alpha comes from the dense latent matrix.
+ *  - RMSNorm before the activation quantisation ([b158] BitLinear_b158.forward
+ *    normalises x first; nn.RMSNorm with a per-feature weight g): the mean of
+ *    x^2 is summed in fp64 and rounded once to fp32 (ms); the reciprocal root
+ *    r = 1 / sqrt(ms + eps) is evaluated in fp64 and rounded once to fp32;
+ *    xn = RN(RN(x * r) * g) in fp32 and is not rounded to bf16 before the
+ *    quantisation.  eps is a parameter (the page's nn.RMSNorm leaves it to
+ *    the dtype's default).
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math
  */
@@ -274,6 +281,59 @@ void orc_quant_act(const uint16_t* x, int M, int K, int Qb, int8_t* q, float* ga
         int64_t s = 0;
         for (int k = 0; k < K; ++k) {
             volatile float t = orc_bf16_to_f32(xr[k]) * (float)Qb;
+            volatile float v = t / d;
+            float c = nearbyintf(v);
+            if (c > 127.0f) c = 127.0f;
+            if (c < -128.0f) c = -128.0f;
+            q[(int64_t)r * K + k] = (int8_t)c;
+            s += (int64_t)c;
+        }
+        if (rowsum) rowsum[r] = (int32_t)s;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* RMSNorm, then activation quantisation ([b158] BitLinear_b158.forward:      */
+/* x = self.norm(x) before activation_quant)                                  */
+/* ------------------------------------------------------------------------ */
+
+/* xn[m][k] = RN(RN(x[m][k] * r_m) * g[k]) with r_m = RN32(1 / sqrt(ms_m + eps))
+ * (fp64), ms_m = RN32(sum_k x[m][k]^2 / K) (fp64 sum in index order). */
+void orc_rmsnorm(const uint16_t* x, const float* g, int M, int K, float eps, float* xn) {
+    fesetround(FE_TONEAREST);
+    for (int r = 0; r < M; ++r) {
+        const uint16_t* xr = x + (int64_t)r * K;
+        double ss = 0.0;
+        for (int k = 0; k < K; ++k) {
+            const double v = (double)orc_bf16_to_f32(xr[k]);
+            ss += v * v;
+        }
+        const float ms = (float)(ss / (double)K);
+        const float rr = (float)(1.0 / sqrt((double)ms + (double)eps));
+        for (int k = 0; k < K; ++k) {
+            volatile float a = orc_bf16_to_f32(xr[k]) * rr;
+            volatile float b = a * g[k];
+            xn[(int64_t)r * K + k] = b;
+        }
+    }
+}
+
+/* Activation quantisation of fp32 rows: gamma = max |xn|,
+ * q = clamp(rne(RN(xn * Qb) / RN(gamma + eps)), -128, 127). */
+void orc_quant_act_f32(const float* xn, int M, int K, int Qb, int8_t* q, float* gamma, int32_t* rowsum) {
+    fesetround(FE_TONEAREST);
+    for (int r = 0; r < M; ++r) {
+        const float* xr = xn + (int64_t)r * K;
+        float g = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(xr[k]);
+            if (a > g) g = a;
+        }
+        gamma[r] = g;
+        volatile float d = g + ORC_EPS;
+        int64_t s = 0;
+        for (int k = 0; k < K; ++k) {
+            volatile float t = xr[k] * (float)Qb;
             volatile float v = t / d;
             float c = nearbyintf(v);
             if (c > 127.0f) c = 127.0f;

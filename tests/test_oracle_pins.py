@@ -306,3 +306,81 @@ def test_third_restatement_torch_cpu():
     y, *_ = oracle.forward(x, p["Wt"], p["alpha"])
     diff = np.abs(y.astype(np.int32) - ref.astype(np.int32))
     assert diff.max() <= 1
+
+
+# ---------------------------------------------------------------- RMSNorm before the activation quantisation
+# [b158] BitLinear_b158.forward normalises x with nn.RMSNorm (per-feature weight g) before activation_quant.
+
+def _bf16(vals):
+    return synth.to_bf16_bits(np.asarray(vals, np.float32))
+
+
+def test_rmsnorm_hand_worked():
+    """x = (3, 4): ms = 12.5, xn = (3, 4) / sqrt(12.5); gamma = 4 r; codes 127 * (3/4) = 95.25 -> 95 and 127.
+    With g = (2, 0.5): xn = (6 r, 2 r), codes 127 and 127/3 = 42.33 -> 42."""
+    x = _bf16([[3.0, 4.0]])
+    r = np.float32(1.0 / np.sqrt(12.5))
+    xn = oracle.rmsnorm(x, np.array([1.0, 1.0], np.float32), 0.0)
+    assert xn[0, 0] == np.float32(np.float32(3.0) * r) and xn[0, 1] == np.float32(np.float32(4.0) * r)
+    q, g, rs = oracle.quant_act_f32(xn)
+    assert list(q[0]) == [95, 127] and rs[0] == 222 and g[0] == xn[0, 1]
+    xn2 = oracle.rmsnorm(x, np.array([2.0, 0.5], np.float32), 0.0)
+    q2, g2, _ = oracle.quant_act_f32(xn2)
+    assert list(q2[0]) == [127, 42] and g2[0] == xn2[0, 0]
+
+
+def test_rmsnorm_unit_mean_square():
+    """g = 1, eps = 0: mean(xn^2) = 1 up to fp32 rounding, for any row."""
+    x = synth.activations(6, 1000, seed=21)
+    xn = oracle.rmsnorm(x, np.ones(1000, np.float32), 0.0).astype(np.float64)
+    np.testing.assert_allclose((xn ** 2).mean(axis=1), 1.0, rtol=1e-6)
+
+
+def test_rmsnorm_scale_invariance():
+    """eps = 0: scaling x by a power of two leaves xn unchanged bit for bit; doubling g doubles xn and leaves
+    the codes and code sums unchanged."""
+    x = synth.activations(4, 300, seed=22)
+    xf = synth.bf16_bits_to_f32(x)
+    x4 = synth.to_bf16_bits(xf * np.float32(4.0))
+    g = (1.0 + 0.25 * synth.uniform(22, 9, 300)).astype(np.float32)
+    a = oracle.rmsnorm(x, g, 0.0)
+    np.testing.assert_array_equal(oracle.rmsnorm(x4, g, 0.0), a)
+    b = oracle.rmsnorm(x, g * np.float32(2.0), 0.0)
+    np.testing.assert_array_equal(b, a * np.float32(2.0))
+    qa, ga, ra = oracle.quant_act_f32(a)
+    qb, gb, rb = oracle.quant_act_f32(b)
+    np.testing.assert_array_equal(qa, qb)
+    np.testing.assert_array_equal(ra, rb)
+    np.testing.assert_array_equal(gb, ga * np.float32(2.0))
+
+
+def test_rmsnorm_constant_and_zero_rows():
+    """A constant row of a power of two normalises to +-1 exactly with eps = 0 (codes +-127, gamma 1); with
+    eps > 0 a zero row gives zeros (with eps = 0 it is 0 / 0, left undefined)."""
+    x = _bf16([[0.5] * 8, [-2.0] * 8])
+    xn = oracle.rmsnorm(x, np.ones(8, np.float32), 0.0)
+    assert (xn[0] == 1.0).all() and (xn[1] == -1.0).all()
+    q, g, rs = oracle.quant_act_f32(xn)
+    assert (q[0] == 127).all() and (q[1] == -127).all()
+    assert list(g) == [1.0, 1.0] and list(rs) == [1016, -1016]
+    xe = oracle.rmsnorm(_bf16([[0.0] * 8]), np.ones(8, np.float32), 1e-6)
+    assert not xe.any()
+    qe, ge, re_ = oracle.quant_act_f32(xe)
+    assert not qe.any() and ge[0] == 0.0 and re_[0] == 0
+
+
+def test_rmsnorm_eps_lowers_scale():
+    """eps > 0 can only shrink xn: |xn(eps)| <= |xn(0)| elementwise."""
+    x = synth.activations(3, 64, seed=23)
+    g = np.ones(64, np.float32)
+    assert (np.abs(oracle.rmsnorm(x, g, 1e-2)) <= np.abs(oracle.rmsnorm(x, g, 0.0))).all()
+
+
+def test_quant_act_f32_matches_bf16_path_on_bf16_values():
+    """On rows whose values are bf16 numbers, the fp32-input quantisation is the bf16 one."""
+    x = synth.activations(5, 200, seed=24)
+    q1, g1, r1 = oracle.quant_act(x)
+    q2, g2, r2 = oracle.quant_act_f32(synth.bf16_bits_to_f32(x))
+    np.testing.assert_array_equal(q1, q2)
+    np.testing.assert_array_equal(g1, g2)
+    np.testing.assert_array_equal(r1, r2)
