@@ -476,6 +476,43 @@ def run_nm(dev, min_calls: int = 16, warmup: int = 3, reps: int = 5):
     return out
 
 
+def run_norm(dev, warmup: int = 3, reps: int = 5, calls: int = 16):
+    """RMSNorm fused into the activation quantisation: the fused kernel alone (GB/s) and
+    forward_norm against forward on the 2B4T gate shape (2560 -> 6912), PDL-chained graphs."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    K, N = 2560, 6912
+    T = torch.from_numpy(synth.ternary_weights(N, K, seed=6)).to(dev)
+    w = bl.pack_ternary(T, float(synth.alpha_uniform(6)))
+    del T
+    g = torch.from_numpy((0.5 + synth.uniform(6, 11, K)).astype(np.float32)).to(dev)
+    out = {}
+    for M in (16, 2048):
+        x = torch.from_numpy(synth.activations(M, K, seed=6).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(bl.forward_workspace_bytes(M, N, K, bl.FLAG_PATH_TC), dtype=torch.uint8, device=dev)
+        q = torch.empty((M, K), dtype=torch.int8, device=dev)
+        gm = torch.empty(M, dtype=torch.float32, device=dev)
+        lib = bl.lib()
+        qcall = (lambda: lib.bitlinear_rmsnorm_quant_act(x.data_ptr(), M, K, g.data_ptr(), 1e-5, q.data_ptr(),
+                                                         gm.data_ptr(), None, torch.cuda.current_stream(dev).cuda_stream))
+        t_q = time_chain_graph(dev, [qcall] * calls, warmup, reps) / calls
+        t_fn = time_chain_graph(dev, [lambda: bl.forward_norm(w, x, g, 1e-5, out=y, workspace=ws,
+                                                              flags=bl.FLAG_PDL)] * calls, warmup, reps) / calls
+        t_f = time_chain_graph(dev, [lambda: bl.forward(w, x, out=y, workspace=ws, flags=bl.FLAG_PDL | bl.FLAG_PATH_TC)]
+                               * calls, warmup, reps) / calls
+        out[f"M={M}"] = {"rmsnorm_quant_act_us": t_q * 1e6,
+                         "rmsnorm_quant_act_GBps": (2 * M * K + M * K + 4 * K + 8 * M) / t_q / 1e9,
+                         "forward_norm_us": t_fn * 1e6, "forward_us": t_f * 1e6,
+                         "forward_norm_TOPS": 2.0 * M * N * K / t_fn / 1e12}
+    assert bl.device_status() == 0
+    return out
+
+
 # ------------------------------------------------------------------ oracle (CPU) legs
 
 def oracle_decode_setup(seed: int = 1):
@@ -586,10 +623,11 @@ def main():
     e2e_value = aggregate(step_bytes, dec["e2e_steps"], world, max_e2e) / 1e9
 
     pre = run_prefill(dev, args.prefill_iters, 3)
-    sweep = nm = None
+    sweep = nm = norm = None
     if not args.no_sweep:
         sweep = run_sweep(dev)
         nm = run_nm(dev)
+        norm = run_norm(dev)
 
     if world > 1:
         barrier(dev)
@@ -639,6 +677,10 @@ def main():
                                   "M=4096: 16 calls); "
                                   "bytes = packed values + metadata + 4 + 2MK + 2MN; TOPS counts dense-equivalent "
                                   "2MNK", "cases": nm}
+        line["norm"] = {"workload": "RMSNorm (fp32 weight, eps 1e-5) fused into the activation quantisation, "
+                                    "2B4T gate 2560->6912, ternary P(0)=0.42; PDL-chained graphs of 16 calls; "
+                                    "rmsnorm_quant_act bytes = 2MK (x) + MK (q) + 4K (g) + 8M; forward_norm vs "
+                                    "forward on the tensor-core path", "by_M": norm}
     print(json.dumps(line), flush=True)
 
 

@@ -148,6 +148,36 @@ bitlinear_status bitlinear_pack_ternary(const int8_t* Wt, int32_t N, int32_t K, 
 bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* gamma,
                                      int32_t* rowsum, void* stream);
 
+/* RMSNorm followed by the per-token absmax int8 quantisation, in one kernel.
+ * The page's BitLinear normalises its input with an RMSNorm (per-feature
+ * weight g) before the activation quantisation ("BitNet 1-Bit LLM" blog,
+ * section "BitNet b1.58: Absmean quantization function", BitLinear_b158.forward).
+ * Per row: ms = RN32(sum_k x_k^2 / K) and r = RN32(1 / sqrt(ms + eps)), the sum,
+ * root and quotient in fp64; xn_k = RN32(RN32(x_k * r) * g_k) (not rounded to
+ * bf16); then gamma = max |xn| and q = clamp(rne(RN32(xn * 127) / RN32(gamma +
+ * 1e-5)), -128, 127) as in bitlinear_quant_act.
+ * x        device, bf16 bits [M, K] (16-byte aligned).
+ * g        device, fp32 [K] (4-byte aligned).
+ * eps      0 <= eps <= 1 (with eps = 0 an all-zero row is undefined).
+ * q, gamma, rowsum: as bitlinear_quant_act (natural k order; rowsum may be NULL).
+ * Errors: NULL, SHAPE (also eps out of range), ALIGN, DEVICE, CUDA. */
+bitlinear_status bitlinear_rmsnorm_quant_act(const uint16_t* x, int32_t M, int32_t K, const float* g, float eps,
+                                             int8_t* q, float* gamma, int32_t* rowsum, void* stream);
+
+/* y = BitLinear(RMSNorm(x)) as the page's BitLinear_b158.forward computes it
+ * (see bitlinear_rmsnorm_quant_act for the normalisation): the normalisation
+ * is fused into the activation quantisation kernel, which writes the codes
+ * into the workspace, and the tensor-core GEMM follows for every M.
+ * w        dense or N:M weights.
+ * g, eps   as bitlinear_rmsnorm_quant_act.
+ * workspace, workspace_bytes: bitlinear_forward_workspace_bytes(M, N, K,
+ *          BITLINEAR_FLAG_PATH_TC).
+ * flags    BITLINEAR_FLAG_PDL and/or BITLINEAR_FLAG_PATH_TC (implied).
+ * Errors: as bitlinear_forward; SHAPE also for eps out of range. */
+bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16_t* x, int32_t M, const float* g,
+                                        float eps, uint16_t* y, int32_t* acc, void* workspace, size_t workspace_bytes,
+                                        uint32_t flags, void* stream);
+
 /* Workspace bytes needed by bitlinear_forward / bitlinear_forward_nm.  0 when
  * the call takes the M = 1 GEMV path (which quantises in-kernel).  The
  * tensor-core path needs the int8 codes, gamma and code sums of x and, when it

@@ -14,7 +14,8 @@ from typing import Optional
 
 __all__ = [
     "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
-    "quant_act", "forward", "forward_nm", "forward_group", "forward_workspace_bytes", "device_status", "last_kernel",
+    "quant_act", "rmsnorm_quant_act", "forward", "forward_nm", "forward_group", "forward_norm",
+    "forward_workspace_bytes", "device_status", "last_kernel",
     "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC",
 ]
 
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
             "bitlinear_forward": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
             "bitlinear_forward_nm": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
             "bitlinear_forward_group": (st, [ctypes.POINTER(_Weights), i32, P, i32, P, P, P, sz, u32, P]),
+            "bitlinear_rmsnorm_quant_act": (st, [P, i32, i32, P, ctypes.c_float, P, P, P, P]),
+            "bitlinear_forward_norm": (st, [ctypes.POINTER(_Weights), P, i32, P, ctypes.c_float, P, P, P, sz, u32, P]),
             "bitlinear_device_status": (st, [P, ctypes.POINTER(i32), i32]),
             "bitlinear_last_kernel": (ctypes.c_char_p, []),
             "bitlinear_status_string": (ctypes.c_char_p, [st]),
@@ -162,6 +165,21 @@ def quant_act(x, rowsum: bool = True, stream=None):
     return q, g, rs
 
 
+def rmsnorm_quant_act(x, g, eps: float, rowsum: bool = True, stream=None):
+    """RMSNorm (weight g, fp32 [K]) then per-token int8 codes of a bf16 [M, K] CUDA matrix:
+    (q, gamma, rowsum or None)."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    assert g.is_cuda and g.dtype == torch.float32 and g.is_contiguous() and g.numel() == x.shape[1]
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    gm = torch.empty(M, dtype=torch.float32, device=x.device)
+    rs = torch.empty(M, dtype=torch.int32, device=x.device) if rowsum else None
+    _check(lib().bitlinear_rmsnorm_quant_act(_ptr(x), M, K, _ptr(g), float(eps), _ptr(q), _ptr(gm), _ptr(rs),
+                                             _stream(stream)), "rmsnorm_quant_act")
+    return q, gm, rs
+
+
 def forward_workspace_bytes(M: int, N: int, K: int, flags: int = 0) -> int:
     return int(lib().bitlinear_forward_workspace_bytes(M, N, K, flags))
 
@@ -214,6 +232,26 @@ def forward_group(ws, x, want_acc: bool = False, flags: int = 0, workspace=None,
     _check(lib().bitlinear_forward_group(arr, count, _ptr(x), M, yp, ap, _ptr(workspace), ws_n, flags,
                                          _stream(stream)), "forward_group")
     return list(zip(ys, accs)) if want_acc else ys
+
+
+def forward_norm(w: PackedWeights, x, g, eps: float, want_acc: bool = False, flags: int = 0, workspace=None,
+                 out=None, acc_out=None, stream=None):
+    """y = BitLinear(RMSNorm(x)) with the normalisation fused into the activation quantisation."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w.K
+    assert g.is_cuda and g.dtype == torch.float32 and g.is_contiguous() and g.numel() == w.K
+    M = x.shape[0]
+    y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    acc = acc_out if acc_out is not None else (
+        torch.empty((M, w.N), dtype=torch.int32, device=x.device) if want_acc else None)
+    need = forward_workspace_bytes(M, w.N, w.K, FLAG_PATH_TC)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_n = workspace.numel() * workspace.element_size()
+    ws = w.c_struct()
+    _check(lib().bitlinear_forward_norm(ctypes.byref(ws), _ptr(x), M, _ptr(g), float(eps), _ptr(y), _ptr(acc),
+                                        _ptr(workspace), ws_n, flags, _stream(stream)), "forward_norm")
+    return (y, acc) if want_acc else y
 
 
 def device_status(clear: bool = True, stream=None) -> int:

@@ -242,7 +242,8 @@ QuantWs tc_ws_layout(void* ws, int M, int K, int ncnt, int max_n) {
   return r;
 }
 
-bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s) {
+bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s,
+                          const float* gnorm = nullptr, float eps = 0.0f) {
   const int wpr = quant_warps_per_row(K);
   const int rows_per_cta = kQuantWarps / wpr;
   const int qblocks = (M + rows_per_cta - 1) / rows_per_cta;
@@ -250,9 +251,14 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
   const size_t vec4 = (qw.part_words + 3) / 4;
   const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * 32 * kQuantWarps - 1) /
                                                                    (4 * 32 * kQuantWarps)));
-  return launch(quant_act_kernel<true>, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
-                static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum,
-                qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr), qw.ncnt, qw.part, vec4, qblocks, wpr);
+  uint32_t* cnt = qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr);
+  if (gnorm)
+    return launch(quant_act_kernel<true, true>, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
+                  static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr, gnorm,
+                  eps);
+  return launch(quant_act_kernel<true, false>, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
+                static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr,
+                static_cast<const float*>(nullptr), 0.0f);
 }
 
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
@@ -311,13 +317,14 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
 }
 
 bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
-                            void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev) {
+                            void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev,
+                            const float* gnorm = nullptr, float eps = 0.0f) {
   const int nm = w->nm_m == 0 ? 0 : (w->nm_m == 4 ? 1 : 2);
   if (!ws || ws_bytes < tc_workspace(M, w->N, w->K, nm, dev->sm_count) || !aligned16(ws))
     return BITLINEAR_ERR_WORKSPACE;
   const bool split = tc_plan(M, w->N, w->K, nm, dev->sm_count).ksplit > 1;
   const QuantWs qw = tc_ws_layout(ws, M, w->K, split ? dev->sm_count : 0, w->N);
-  bitlinear_status st = tc_quant(x, M, w->K, qw, pdl, s);
+  bitlinear_status st = tc_quant(x, M, w->K, qw, pdl, s, gnorm, eps);
   if (st != BITLINEAR_OK) return st;
   return tc_gemm(w, M, qw, y, acc, s, dev);
 }
@@ -676,11 +683,49 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
   if (st != BITLINEAR_OK) return st;
   const int wpr = quant_warps_per_row(K);
   const int qblocks = (M + kQuantWarps / wpr - 1) / (kQuantWarps / wpr);
-  st = launch(quant_act_kernel<false>, dim3(qblocks), dim3(32 * kQuantWarps), 0, static_cast<cudaStream_t>(stream), false,
-              x, M, K, K, q, gamma, rowsum, static_cast<uint32_t*>(nullptr), 0, static_cast<float*>(nullptr),
-              static_cast<size_t>(0), qblocks, wpr);
+  st = launch(quant_act_kernel<false, false>, dim3(qblocks), dim3(32 * kQuantWarps), 0,
+              static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum, static_cast<uint32_t*>(nullptr), 0,
+              static_cast<float*>(nullptr), static_cast<size_t>(0), qblocks, wpr, static_cast<const float*>(nullptr),
+              0.0f);
   if (st == BITLINEAR_OK) t_last_kernel = "quant_act";
   return st;
+}
+
+bitlinear_status bitlinear_rmsnorm_quant_act(const uint16_t* x, int32_t M, int32_t K, const float* g, float eps,
+                                             int8_t* q, float* gamma, int32_t* rowsum, void* stream) {
+  if (!x || !g || !q || !gamma) return BITLINEAR_ERR_NULL;
+  if (M < 1 || M > BITLINEAR_MAX_M || K < 1 || K > BITLINEAR_MAX_K) return BITLINEAR_ERR_SHAPE;
+  if (!(eps >= 0.0f) || eps > 1.0f) return BITLINEAR_ERR_SHAPE;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(g) & 3u) || (reinterpret_cast<uintptr_t>(gamma) & 3u) ||
+      (rowsum && (reinterpret_cast<uintptr_t>(rowsum) & 3u)))
+    return BITLINEAR_ERR_ALIGN;
+  DeviceState* dev = nullptr;
+  bitlinear_status st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  const int wpr = quant_warps_per_row(K);
+  const int qblocks = (M + kQuantWarps / wpr - 1) / (kQuantWarps / wpr);
+  st = launch(quant_act_kernel<false, true>, dim3(qblocks), dim3(32 * kQuantWarps), 0,
+              static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum, static_cast<uint32_t*>(nullptr), 0,
+              static_cast<float*>(nullptr), static_cast<size_t>(0), qblocks, wpr, g, eps);
+  if (st == BITLINEAR_OK) t_last_kernel = "rmsnorm_quant_act";
+  return st;
+}
+
+bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16_t* x, int32_t M, const float* g,
+                                        float eps, uint16_t* y, int32_t* acc, void* workspace, size_t workspace_bytes,
+                                        uint32_t flags, void* stream) {
+  if (!w || !x || !y || !g) return BITLINEAR_ERR_NULL;
+  bitlinear_status st = check_matrix(w, y, acc);
+  if (st != BITLINEAR_OK) return st;
+  if (M < 1 || M > BITLINEAR_MAX_M) return BITLINEAR_ERR_SHAPE;
+  if (!(eps >= 0.0f) || eps > 1.0f) return BITLINEAR_ERR_SHAPE;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(g) & 3u)) return BITLINEAR_ERR_ALIGN;
+  if (flags & ~static_cast<uint32_t>(BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_TC)) return BITLINEAR_ERR_FLAGS;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, (flags & BITLINEAR_FLAG_PDL) != 0,
+                    static_cast<cudaStream_t>(stream), dev, g, eps);
 }
 
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {

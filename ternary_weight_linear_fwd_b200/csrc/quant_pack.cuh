@@ -81,6 +81,25 @@ __device__ __forceinline__ void codes8(const uint32_t (&raw)[4], float c, float 
   }
 }
 
+// codes8 for fp32 values (RMSNorm outputs): the same rounding argument holds
+// with t = RN(v * 127) no longer exact, since |y - RN(t / d)| stays below
+// 5 * 2^-24 * 127 < 2^-14; the fallback recomputes RN(RN(v * 127) / d).
+__device__ __forceinline__ void codes8f(const float* v, float c, float d, uint32_t (&b)[8]) {
+  float emax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float yq = __fmul_rn(v[e], c);
+    const float sm = __fadd_rn(yq, kMagic);
+    emax = fmaxf(emax, fabsf(__fsub_rn(yq, __fsub_rn(sm, kMagic))));
+    b[e] = __float_as_uint(sm);
+  }
+  if (emax > 0.5f - 6.103515625e-05f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      b[e] = 0x4B400000u + static_cast<uint32_t>(__float2int_rn(__fdiv_rn(__fmul_rn(v[e], kQb), d)));
+  }
+}
+
 // 8 bf16 values of a row from k0 as 4 words (zero past K).
 __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bool vec_ok, uint32_t (&r)[4]) {
   if (vec_ok && k0 + 8 <= K) {
@@ -108,7 +127,10 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 // rows take a two-pass loop (the second pass re-reads from L1/L2).
 // kPermute = false writes natural-order codes [M, ldq] (ldq = K); kPermute =
 // true writes the contraction order [M, ldq] with ldq = K rounded up to 16
-// (zeros past K).  Both write gamma and, when asked, the sum of the row's
+// (zeros past K).  kNorm = true first applies RMSNorm with weight gnorm
+// ([b158] BitLinear_b158.forward normalises x before activation_quant):
+// r = RN32(1 / sqrt(RN32(sum x^2 / K) + eps)) with the sum, the root and the
+// quotient in fp64, xn = RN(RN(x * r) * g) in fp32, and quantises xn.  Both write gamma and, when asked, the sum of the row's
 // codes.  The first CTA also clears the split-K arrival counters, and CTAs
 // past the rows (blockIdx >= qblocks) clear the split-K sums, of the GEMMs that
 // read these codes.
@@ -122,11 +144,8 @@ __host__ __device__ __forceinline__ int quant_warps_per_row(int K) {
 // 16 codes of one k-group (raw: the group's 16 bf16 as 8 words) in the
 // requested order; adds their sum to *sum.
 template <bool kPermute>
-__device__ __forceinline__ uint4 group_codes(const uint32_t (&r0)[4], const uint32_t (&r1)[4], float c, float d,
-                                             int32_t& sum) {
-  uint32_t b0[8], b1[8], w[4];
-  codes8(r0, c, d, b0);  // elements past K are zero and give code 0
-  codes8(r1, c, d, b1);
+__device__ __forceinline__ uint4 pack_group(const uint32_t (&b0)[8], const uint32_t (&b1)[8], int32_t& sum) {
+  uint32_t w[4];
   if (kPermute) {
     // byte 4j + b <- k0 + 4b + j
 #pragma unroll
@@ -146,6 +165,48 @@ __device__ __forceinline__ uint4 group_codes(const uint32_t (&r0)[4], const uint
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+template <bool kPermute>
+__device__ __forceinline__ uint4 group_codes(const uint32_t (&r0)[4], const uint32_t (&r1)[4], float c, float d,
+                                             int32_t& sum) {
+  uint32_t b0[8], b1[8];
+  codes8(r0, c, d, b0);  // elements past K are zero and give code 0
+  codes8(r1, c, d, b1);
+  return pack_group<kPermute>(b0, b1, sum);
+}
+
+// 16 normalised values of a group: xn = RN(RN(x * r) * g) (zero past K, where g is not read).
+__device__ __forceinline__ void norm16(const uint32_t (&r0)[4], const uint32_t (&r1)[4], const float* __restrict__ g,
+                                       int k0, int K, float r, float (&xn)[16]) {
+  float gv[16];
+  if (k0 + 16 <= K && (reinterpret_cast<uintptr_t>(g + k0) & 15u) == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 t = reinterpret_cast<const float4*>(g + k0)[i];
+      gv[4 * i] = t.x; gv[4 * i + 1] = t.y; gv[4 * i + 2] = t.z; gv[4 * i + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) gv[i] = k0 + i < K ? g[k0 + i] : 0.0f;
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const uint32_t w = e < 8 ? r0[e >> 1] : r1[(e - 8) >> 1];
+    const float xv = __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
+    xn[e] = __fmul_rn(__fmul_rn(xv, r), gv[e]);
+  }
+}
+
+__device__ __forceinline__ double sumsq8(const uint32_t (&w)[4], double acc) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double lo = static_cast<double>(__uint_as_float(w[i] << 16));
+    const double hi = static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
+    acc = __fma_rn(lo, lo, acc);
+    acc = __fma_rn(hi, hi, acc);
+  }
+  return acc;
+}
+
 __device__ __forceinline__ float absmax8(const uint32_t (&w)[4], float mx) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -153,16 +214,18 @@ __device__ __forceinline__ float absmax8(const uint32_t (&w)[4], float mx) {
   return mx;
 }
 
-template <bool kPermute>
+template <bool kPermute, bool kNorm>
 __global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                      int ldq, int8_t* __restrict__ q,
                                                                      float* __restrict__ gamma,
                                                                      int32_t* __restrict__ rowsum,
                                                                      uint32_t* __restrict__ cnt, int ncnt,
                                                                      float* __restrict__ zbuf, size_t zvec4,
-                                                                     int qblocks, int wpr) {
+                                                                     int qblocks, int wpr,
+                                                                     const float* __restrict__ gnorm, float eps) {
   __shared__ float s_mx[kQuantWarps];
   __shared__ int32_t s_sum[kQuantWarps];
+  __shared__ double s_ss[kQuantWarps];
   pdl_wait_primary();
   pdl_launch_dependents();
   // split-K arrival counters and sums of the GEMMs that follow start from zero
@@ -185,33 +248,74 @@ __global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint1
   const int g0 = sub * 32 + lane;
   const bool in_regs = vec_ok && groups <= kQuantGroupsInRegs * gstride;
 
+  // Calls f(g, r0, r1) for each of this lane's groups with the group's raw
+  // bf16 words: from registers (unrolled, static indices) or loaded again.
   uint32_t v[kQuantGroupsInRegs][8];
-  float mx = 0.0f;
-  if (active) {
+  auto for_groups = [&](auto&& f) {
     if (in_regs) {
 #pragma unroll
       for (int j = 0; j < kQuantGroupsInRegs; ++j) {
-        const int k0 = 16 * (g0 + j * gstride);
-        uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
-        if (k0 + 8 <= K) a = *reinterpret_cast<const uint4*>(xr + k0);
-        if (k0 + 16 <= K) b = *reinterpret_cast<const uint4*>(xr + k0 + 8);
-        v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
-        v[j][4] = b.x; v[j][5] = b.y; v[j][6] = b.z; v[j][7] = b.w;
-      }
+        const int g = g0 + j * gstride;
+        if (g < groups) {
+          uint32_t r0[4], r1[4];
 #pragma unroll
-      for (int j = 0; j < kQuantGroupsInRegs; ++j) {
-        const uint32_t lo[4] = {v[j][0], v[j][1], v[j][2], v[j][3]}, hi[4] = {v[j][4], v[j][5], v[j][6], v[j][7]};
-        mx = absmax8(hi, absmax8(lo, mx));
+          for (int i = 0; i < 4; ++i) {
+            r0[i] = v[j][i];
+            r1[i] = v[j][4 + i];
+          }
+          f(g, r0, r1);
+        }
       }
     } else {
       for (int g = g0; g < groups; g += gstride) {
         uint32_t r0[4], r1[4];
         load8_raw(xr, 16 * g, K, vec_ok, r0);
         load8_raw(xr, 16 * g + 8, K, vec_ok, r1);
-        mx = absmax8(r1, absmax8(r0, mx));
+        f(g, r0, r1);
       }
     }
+  };
+  if (active && in_regs) {
+#pragma unroll
+    for (int j = 0; j < kQuantGroupsInRegs; ++j) {
+      const int k0 = 16 * (g0 + j * gstride);
+      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
+      if (k0 + 8 <= K) a = *reinterpret_cast<const uint4*>(xr + k0);
+      if (k0 + 16 <= K) b = *reinterpret_cast<const uint4*>(xr + k0 + 8);
+      v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
+      v[j][4] = b.x; v[j][5] = b.y; v[j][6] = b.z; v[j][7] = b.w;
+    }
   }
+
+  // RMSNorm: r = RN32(1 / sqrt(RN32(sum x^2 / K) + eps)), sums in fp64
+  float rn = 1.0f;
+  if (kNorm) {
+    double ss = 0.0;
+    if (active) for_groups([&](int, const uint32_t (&r0)[4], const uint32_t (&r1)[4]) { ss = sumsq8(r1, sumsq8(r0, ss)); });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (wpr > 1) {
+      if (lane == 0) s_ss[warp] = ss;
+      __syncthreads();
+      ss = 0.0;
+      for (int i = 0; i < wpr; ++i) ss += s_ss[rloc * wpr + i];
+    }
+    const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
+    rn = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(static_cast<double>(ms), static_cast<double>(eps)))));
+  }
+
+  float mx = 0.0f;
+  if (active)
+    for_groups([&](int g, const uint32_t (&r0)[4], const uint32_t (&r1)[4]) {
+      if (kNorm) {
+        float xn[16];
+        norm16(r0, r1, gnorm, 16 * g, K, rn, xn);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(xn[e]));
+      } else {
+        mx = absmax8(r1, absmax8(r0, mx));
+      }
+    });
   // |x| >= 0, whose bit patterns order like the values: integer maxima
   mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
   if (wpr > 1) {
@@ -226,31 +330,26 @@ __global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint1
   if (active) {
     int8_t* qr = q + static_cast<size_t>(row) * ldq;
     const bool qvec = ((reinterpret_cast<uintptr_t>(q) & 15u) == 0) && (ldq % 16) == 0;
-    auto put = [&](int k0, const uint4& w) {
+    for_groups([&](int g, const uint32_t (&r0)[4], const uint32_t (&r1)[4]) {
+      const int k0 = 16 * g;
+      uint4 w;
+      if (kNorm) {
+        float xn[16];
+        norm16(r0, r1, gnorm, k0, K, rn, xn);
+        uint32_t b0[8], b1[8];
+        codes8f(xn, c, d, b0);
+        codes8f(xn + 8, c, d, b1);
+        w = pack_group<kPermute>(b0, b1, sum);
+      } else {
+        w = group_codes<kPermute>(r0, r1, c, d, sum);
+      }
       if (kPermute || (qvec && k0 + 16 <= K)) {
         *reinterpret_cast<uint4*>(qr + k0) = w;
       } else {
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
         for (int i = 0; i < 16 && k0 + i < K; ++i) qr[k0 + i] = static_cast<int8_t>(ww[i >> 2] >> (8 * (i & 3)));
       }
-    };
-    if (in_regs) {
-#pragma unroll
-      for (int j = 0; j < kQuantGroupsInRegs; ++j) {
-        const int g = g0 + j * gstride;
-        if (g < groups) {
-          const uint32_t lo[4] = {v[j][0], v[j][1], v[j][2], v[j][3]}, hi[4] = {v[j][4], v[j][5], v[j][6], v[j][7]};
-          put(16 * g, group_codes<kPermute>(lo, hi, c, d, sum));
-        }
-      }
-    } else {
-      for (int g = g0; g < groups; g += gstride) {
-        uint32_t r0[4], r1[4];
-        load8_raw(xr, 16 * g, K, vec_ok, r0);
-        load8_raw(xr, 16 * g + 8, K, vec_ok, r1);
-        put(16 * g, group_codes<kPermute>(r0, r1, c, d, sum));
-      }
-    }
+    });
   }
   sum = __reduce_add_sync(0xffffffffu, sum);
   if (wpr > 1) {

@@ -136,3 +136,23 @@ def test_forward_group_host_checks(L):
     nometa = (bl._Weights * 2)(_w(L), _w(L, n=2, m=4))
     assert fg(nometa, 2, x, 1, ys, None, None, 0, 0, None) == 1
     assert fg(ws, 2, x, 2, ys, None, None, 0, 0x2, None) == 8                    # GEMV path needs M == 1
+
+
+def test_rmsnorm_entry_points_host_checks(L):
+    """RMSNorm entry points reject bad arguments before any device work (fake addresses)."""
+    x, g, q, gm = 0x30000, 0x40000, 0x50000, 0x60000
+    f = L.bitlinear_rmsnorm_quant_act
+    assert f(None, 4, 64, g, 1e-6, q, gm, None, None) == 1
+    assert f(x, 4, 64, None, 1e-6, q, gm, None, None) == 1
+    assert f(x, 0, 64, g, 1e-6, q, gm, None, None) == 2
+    assert f(x, 4, 64, g, -1.0, q, gm, None, None) == 2           # eps out of range
+    assert f(x, 4, 64, g, float("nan"), q, gm, None, None) == 2
+    assert f(x + 2, 4, 64, g, 1e-6, q, gm, None, None) == 3
+    assert f(x, 4, 64, g + 2, 1e-6, q, gm, None, None) == 3
+    fn = L.bitlinear_forward_norm
+    w = _w(L)
+    y = 0x70000
+    assert fn(ctypes.byref(w), x, 1, None, 1e-6, y, None, None, 0, 0, None) == 1
+    assert fn(ctypes.byref(w), x, 1, g, 2.0, y, None, None, 0, 0, None) == 2
+    assert fn(ctypes.byref(w), x, 1, g, 1e-6, y, None, None, 0, 0x2, None) == 8   # the GEMV path is not offered
+    assert fn(ctypes.byref(_w(L, codes=0x10008)), x, 1, g, 1e-6, y, None, None, 0, 0, None) == 3

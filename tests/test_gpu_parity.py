@@ -57,7 +57,7 @@ def assert_bf16_close(got_bits, ref_bits):
 
 # ---------------------------------------------------------------- activation quantisation
 
-@pytest.mark.parametrize("M,K", [(8, 256), (5, 200), (3, 203), (1, 6912), (64, 11008), (2048, 2560)])
+@pytest.mark.parametrize("M,K", [(8, 256), (5, 200), (3, 203), (1, 6912), (64, 11008), (2048, 2560), (2, 40000)])
 def test_quant_act_bit_exact(M, K):
     x = synth.activations(M, K, seed=M + K)
     q, g, rs = bl.quant_act(to_dev_bf16(x))
@@ -309,6 +309,40 @@ def test_forward_group_prefill_sampled():
     rows = np.unique(np.concatenate([[0, M - 1], synth.splitmix64(34, 9, 14) % M])).astype(np.int64)
     for (T, a, w), (y, acc) in zip(cases, outs):
         _check_rows(x, T, a, y, acc, rows)
+
+
+# ---------------------------------------------------------------- RMSNorm before the quantisation
+
+def _norm_weight(K, seed):
+    return (0.5 + synth.uniform(seed, 11, K)).astype(np.float32)
+
+
+@pytest.mark.parametrize("M,K", [(8, 256), (5, 200), (3, 203), (1, 6912), (64, 11008), (2048, 2560), (2, 20480),
+                                 (1, 40000)])
+def test_rmsnorm_quant_act_bit_exact(M, K):
+    x = synth.activations(M, K, seed=M + K)
+    g = _norm_weight(K, K)
+    q, gm, rs = bl.rmsnorm_quant_act(to_dev_bf16(x), torch.from_numpy(g).to(DEV), 1e-6)
+    xn = oracle.rmsnorm(x, g, 1e-6)
+    qo, go, ro = oracle.quant_act_f32(xn)
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(gm.cpu().numpy(), go)
+    np.testing.assert_array_equal(rs.cpu().numpy(), ro)
+    assert bl.last_kernel() == "rmsnorm_quant_act"
+
+
+@pytest.mark.parametrize("n,m", [(0, 0), (2, 4), (6, 8)])
+@pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (16, 1024, 300), (300, 512, 1000)])
+def test_forward_norm(n, m, M, K, N):
+    x = synth.activations(M, K, seed=7 + M)
+    W = synth.latent_weights(N, K, seed=7 + N)
+    ref = oracle.pack_weights(W, n, m)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV), n, m)
+    g = _norm_weight(K, 3)
+    y, acc = bl.forward_norm(w, to_dev_bf16(x), torch.from_numpy(g).to(DEV), 1e-5, want_acc=True)
+    yo, acco, *_ = oracle.forward_norm(x, g, 1e-5, ref["Wt"], ref["alpha"])
+    np.testing.assert_array_equal(acc.cpu().numpy(), acco)
+    assert_bf16_close(bf16_bits(y), yo)
 
 
 def test_status_word_clean():
