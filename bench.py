@@ -491,7 +491,7 @@ def run_norm(dev, warmup: int = 3, reps: int = 5, calls: int = 16):
     del T
     g = torch.from_numpy((0.5 + synth.uniform(6, 11, K)).astype(np.float32)).to(dev)
     out = {}
-    for M in (16, 2048):
+    for M in (1, 16, 2048):
         x = torch.from_numpy(synth.activations(M, K, seed=6).view(np.int16)).to(dev).view(torch.bfloat16)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ws = torch.empty(bl.forward_workspace_bytes(M, N, K, bl.FLAG_PATH_TC), dtype=torch.uint8, device=dev)
@@ -503,7 +503,7 @@ def run_norm(dev, warmup: int = 3, reps: int = 5, calls: int = 16):
         t_q = time_chain_graph(dev, [qcall] * calls, warmup, reps) / calls
         t_fn = time_chain_graph(dev, [lambda: bl.forward_norm(w, x, g, 1e-5, out=y, workspace=ws,
                                                               flags=bl.FLAG_PDL)] * calls, warmup, reps) / calls
-        t_f = time_chain_graph(dev, [lambda: bl.forward(w, x, out=y, workspace=ws, flags=bl.FLAG_PDL | bl.FLAG_PATH_TC)]
+        t_f = time_chain_graph(dev, [lambda: bl.forward(w, x, out=y, workspace=ws, flags=bl.FLAG_PDL)]
                                * calls, warmup, reps) / calls
         out[f"M={M}"] = {"rmsnorm_quant_act_us": t_q * 1e6,
                          "rmsnorm_quant_act_GBps": (2 * M * K + M * K + 4 * K + 8 * M) / t_q / 1e9,
@@ -680,7 +680,8 @@ def main():
         line["norm"] = {"workload": "RMSNorm (fp32 weight, eps 1e-5) fused into the activation quantisation, "
                                     "2B4T gate 2560->6912, ternary P(0)=0.42; PDL-chained graphs of 16 calls; "
                                     "rmsnorm_quant_act bytes = 2MK (x) + MK (q) + 4K (g) + 8M; forward_norm vs "
-                                    "forward on the tensor-core path", "by_M": norm}
+                                    "forward (M=1: normalising quantisation + GEMV on the codes vs the GEMV "
+                                    "quantising in-kernel; M>1: tensor-core path)", "by_M": norm}
     print(json.dumps(line), flush=True)
 
 

@@ -165,14 +165,17 @@ bitlinear_status bitlinear_rmsnorm_quant_act(const uint16_t* x, int32_t M, int32
                                              int8_t* q, float* gamma, int32_t* rowsum, void* stream);
 
 /* y = BitLinear(RMSNorm(x)) as the page's BitLinear_b158.forward computes it
- * (see bitlinear_rmsnorm_quant_act for the normalisation): the normalisation
- * is fused into the activation quantisation kernel, which writes the codes
- * into the workspace, and the tensor-core GEMM follows for every M.
+ * (see bitlinear_rmsnorm_quant_act for the normalisation).  For M == 1 and
+ * dense weights every CTA of the decode GEMV normalises and quantises the
+ * token itself (no workspace is used); otherwise the normalisation is fused
+ * into the activation quantisation kernel, which writes the codes into the
+ * workspace, and the tensor-core GEMM follows.
  * w        dense or N:M weights.
  * g, eps   as bitlinear_rmsnorm_quant_act.
  * workspace, workspace_bytes: bitlinear_forward_workspace_bytes(M, N, K,
  *          BITLINEAR_FLAG_PATH_TC).
- * flags    BITLINEAR_FLAG_PDL and/or BITLINEAR_FLAG_PATH_TC (implied).
+ * flags    BITLINEAR_FLAG_PDL; BITLINEAR_FLAG_PATH_TC forces the tensor-core
+ *          GEMM at M == 1 (BITLINEAR_FLAG_PATH_GEMV is not accepted).
  * Errors: as bitlinear_forward; SHAPE also for eps out of range. */
 bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16_t* x, int32_t M, const float* g,
                                         float eps, uint16_t* y, int32_t* acc, void* workspace, size_t workspace_bytes,

@@ -389,9 +389,12 @@ int gemv_split(GemvDense& g, const int* N, int count, int sm_count, int* grid) {
 
 // One launch of the dense decode GEMV over `count` matrices sharing x.
 bitlinear_status gemv_dense_launch(const bitlinear_weights* const* w, uint16_t* const* y, int32_t* const* acc,
-                                   int count, const uint16_t* x, bool pdl, cudaStream_t s, DeviceState* dev) {
+                                   int count, const uint16_t* x, bool pdl, cudaStream_t s, DeviceState* dev,
+                                   const float* gnorm = nullptr, float eps = 0.0f) {
   GemvDense g;
   std::memset(&g, 0, sizeof g);
+  g.gnorm = gnorm;
+  g.eps = eps;
   const int K = w[0]->K;
   g.ld = dense_ld(K);
   g.C = static_cast<int>(g.ld / 16);
@@ -412,9 +415,16 @@ bitlinear_status gemv_dense_launch(const bitlinear_weights* const* w, uint16_t* 
       return BITLINEAR_ERR_CUDA;
   }
   for (int i = count; i < kGemvGroup; ++i) map[i] = map[0];  // never selected
-  const size_t smem = gemv_smem_bytes(g.rows_box, g.ld, g.C);
-  bitlinear_status st =
-      launch(gemv_dense_kernel, dim3(grid), dim3(kGemvThreads), smem, s, pdl, map[0], map[1], map[2], map[3], g);
+  bitlinear_status st;
+  if (gnorm) {
+    const size_t smem = gemv_smem_bytes(g.rows_box, g.ld, g.C) + 4 * static_cast<size_t>(K);
+    st = launch(gemv_dense_kernel<true>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, map[0], map[1], map[2], map[3],
+                g);
+  } else {
+    const size_t smem = gemv_smem_bytes(g.rows_box, g.ld, g.C);
+    st = launch(gemv_dense_kernel<false>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, map[0], map[1], map[2], map[3],
+                g);
+  }
   if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_dense";
   return st;
 }
@@ -724,8 +734,13 @@ bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16
   DeviceState* dev = nullptr;
   st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
-  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, (flags & BITLINEAR_FLAG_PDL) != 0,
-                    static_cast<cudaStream_t>(stream), dev, g, eps);
+  const bool pdl = (flags & BITLINEAR_FLAG_PDL) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 1 && w->nm_m == 0 && !(flags & BITLINEAR_FLAG_PATH_TC)) {
+    // decode: every GEMV CTA normalises and quantises the token itself
+    return gemv_dense_launch(&w, &y, &acc, 1, x, pdl, s, dev, g, eps);
+  }
+  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, pdl, s, dev, g, eps);
 }
 
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {

@@ -103,6 +103,111 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
   return mx;
 }
 
+// quantise_row_smem with RMSNorm first (weight s_g[K] already in shared
+// memory): r = RN32(1 / sqrt(RN32(sum x^2 / K) + eps)) with the sum (one
+// fixed-order reduction over the CTA), the root and the quotient in fp64;
+// the codes are those of xn = RN(RN(x * r) * g), which is never stored.
+__device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restrict__ x, int K, int groups_alloc,
+                                                        uint4* s_act, int32_t* s_hsum, float* s_red, double* s_redd,
+                                                        const float* s_g, float eps) {
+  const bool vec_ok = (K % 8) == 0;
+  const int nthr = blockDim.x;
+  const int halves = (K + 7) / 8;
+  const int halves_alloc = 2 * groups_alloc;
+  const int trips = (halves_alloc + nthr - 1) / nthr;
+  uint32_t v[kHalvesInRegs][4];
+  double ss = 0.0;
+#pragma unroll
+  for (int j = 0; j < kHalvesInRegs; ++j) {
+    const int h = threadIdx.x + j * nthr;
+    if (h < halves) {
+      load8_raw(x, h * 8, K, vec_ok, v[j]);
+    } else {
+      v[j][0] = v[j][1] = v[j][2] = v[j][3] = 0u;
+    }
+    ss = sumsq8(v[j], ss);
+  }
+  for (int h = threadIdx.x + kHalvesInRegs * nthr; h < halves; h += nthr) {
+    uint32_t t[4];
+    load8_raw(x, h * 8, K, vec_ok, t);
+    ss = sumsq8(t, ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) s_redd[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  ss = 0.0;
+  for (int w = 0; w < (nthr >> 5); ++w) ss += s_redd[w];
+  const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
+  const float rn = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(static_cast<double>(ms), static_cast<double>(eps)))));
+  // xn of half h (zero past K)
+  auto norm8 = [&](const uint32_t (&raw)[4], int h, float (&xn)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = 8 * h + e;
+      const float xv = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
+      xn[e] = k < K ? __fmul_rn(__fmul_rn(xv, rn), s_g[k]) : 0.0f;
+    }
+  };
+  float mx = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kHalvesInRegs; ++j) {
+    const int h = threadIdx.x + j * nthr;
+    if (h < halves) {
+      float xn[8];
+      norm8(v[j], h, xn);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(xn[e]));
+    }
+  }
+  for (int h = threadIdx.x + kHalvesInRegs * nthr; h < halves; h += nthr) {
+    uint32_t t[4];
+    load8_raw(x, h * 8, K, vec_ok, t);
+    float xn[8];
+    norm8(t, h, xn);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(xn[e]));
+  }
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = (threadIdx.x & 31) < (nthr >> 5) ? s_red[threadIdx.x & 31] : 0.0f;
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+  const float d = __fadd_rn(mx, kEps);
+  const float c = __fmul_rn(kQb, __frcp_rn(d));
+  const int quarter = groups_alloc >> 2;
+  auto emit = [&](const uint32_t (&raw)[4], int h) {
+    float xn[8];
+    norm8(raw, h, xn);
+    uint32_t b[8];
+    codes8f(xn, c, d, b);
+    const uint32_t lo = __byte_perm(b[0], b[1], 0x0040), hi = __byte_perm(b[2], b[3], 0x0040);
+    const uint32_t lo2 = __byte_perm(b[4], b[5], 0x0040), hi2 = __byte_perm(b[6], b[7], 0x0040);
+    const uint32_t p0 = __byte_perm(lo, hi, 0x5410), p1 = __byte_perm(lo2, hi2, 0x5410);
+    if (h < halves_alloc) {
+      s_hsum[h] = __dp4a(static_cast<int>(p1), 0x01010101, __dp4a(static_cast<int>(p0), 0x01010101, 0));
+      const int g = h >> 1, half = h & 1;
+      const int sl = (g & 3) * quarter + (g >> 2);
+      uint16_t* dst = reinterpret_cast<uint16_t*>(s_act + sl) + half;
+      dst[0] = static_cast<uint16_t>(__byte_perm(b[0], b[4], 0x0040));
+      dst[2] = static_cast<uint16_t>(__byte_perm(b[1], b[5], 0x0040));
+      dst[4] = static_cast<uint16_t>(__byte_perm(b[2], b[6], 0x0040));
+      dst[6] = static_cast<uint16_t>(__byte_perm(b[3], b[7], 0x0040));
+    }
+  };
+#pragma unroll
+  for (int j = 0; j < kHalvesInRegs; ++j)
+    if (j < trips) emit(v[j], threadIdx.x + j * nthr);
+  for (int j = kHalvesInRegs; j < trips; ++j) {
+    const int h = threadIdx.x + j * nthr;
+    uint32_t raw[4] = {0u, 0u, 0u, 0u};
+    if (h < halves) load8_raw(x, h * 8, K, vec_ok, raw);
+    emit(raw, h);
+  }
+  __syncthreads();
+  return mx;
+}
+
 __device__ __forceinline__ void gemv_store(uint16_t* y, int32_t* acc, int row, int32_t total, float s) {
   if (acc) acc[row] = total;
   const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(total), s));
@@ -164,7 +269,9 @@ struct GemvMat {
 
 struct GemvDense {
   GemvMat mat[kGemvGroup];
-  const uint16_t* x;  // one bf16 row [K]
+  const uint16_t* x;      // one bf16 row [K]
+  const float* gnorm;     // RMSNorm weight [K] (norm kernel variant only)
+  float eps;
   int32_t* status;
   int64_t ld;
   int K, C, rows_box, count;
@@ -173,6 +280,7 @@ struct GemvDense {
 // The tensor maps (per matrix: uint8 [N, ld], box {128, rows_box}, 128-byte
 // swizzle) are separate kernel parameters, and every parameter is read at a
 // fixed offset: the matrix of this CTA is selected into registers.
+template <bool kNorm>
 __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_constant__ CUtensorMap map0,
                                                                   const __grid_constant__ CUtensorMap map1,
                                                                   const __grid_constant__ CUtensorMap map2,
@@ -202,6 +310,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
   int32_t* s_hsum = reinterpret_cast<int32_t*>(s_act + 4 * C);  // 8 * C half sums
   int32_t* s_acc = s_hsum + 8 * C;
+  float* s_g = reinterpret_cast<float*>(s_acc + rows_box);        // norm variant: RMSNorm weight [K]
+  __shared__ double s_redd[32];
 
   // The weights (and alpha, which belongs to them) do not depend on the
   // preceding kernel: their copies start first.
@@ -215,10 +325,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   }
   const float alpha = *mt.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  if (kNorm)  // the norm weight, like the matrix, does not depend on the preceding kernel
+    for (int k = threadIdx.x; k < g.K; k += blockDim.x) s_g[k] = g.gnorm[k];
   __syncthreads();
 
   pdl_wait_primary();  // x may come from the preceding kernel
-  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_hsum, s_red);
+  float gamma;
+  if (kNorm)
+    gamma = quantise_row_smem_norm(g.x, g.K, 4 * C, s_act, s_hsum, s_red, s_redd, s_g, g.eps);
+  else
+    gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_hsum, s_red);
   // The next kernel may start now: its weight copies then stream while this
   // one contracts, and no longer delay this kernel's read of x.
   pdl_launch_dependents();

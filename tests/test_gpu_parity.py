@@ -340,9 +340,15 @@ def test_forward_norm(n, m, M, K, N):
     w = bl.pack_weights(torch.from_numpy(W).to(DEV), n, m)
     g = _norm_weight(K, 3)
     y, acc = bl.forward_norm(w, to_dev_bf16(x), torch.from_numpy(g).to(DEV), 1e-5, want_acc=True)
+    if M == 1 and m == 0:
+        assert bl.last_kernel() == "gemv_m1_dense"  # the decode GEMV on the normalised codes
     yo, acco, *_ = oracle.forward_norm(x, g, 1e-5, ref["Wt"], ref["alpha"])
     np.testing.assert_array_equal(acc.cpu().numpy(), acco)
     assert_bf16_close(bf16_bits(y), yo)
+    if M == 1:
+        y2, acc2 = bl.forward_norm(w, to_dev_bf16(x), torch.from_numpy(g).to(DEV), 1e-5, want_acc=True,
+                                   flags=bl.FLAG_PATH_TC)
+        assert torch.equal(acc2, acc) and torch.equal(y2.view(torch.int16), y.view(torch.int16))
 
 
 def test_status_word_clean():
