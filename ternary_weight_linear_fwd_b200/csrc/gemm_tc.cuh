@@ -112,26 +112,18 @@ __host__ __device__ constexpr int tc_smem_bytes(int BN, int NM, int vbox) {
          4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
 }
 
-// Dense code word of 16 weights for the current stage and group, per mode.
-template <int NM>
-__device__ __forceinline__ uint32_t tc_group_word(const uint8_t* arow, const uint8_t* mrow, int gi, int n,
-                                                  int rem) {
-  if (NM == 0) {
-    return reinterpret_cast<const uint32_t*>(arow)[gi];
-  } else if (NM == 1) {
-    const uint32_t meta16 = reinterpret_cast<const uint16_t*>(mrow)[gi];
-    const uint32_t vals16 = reinterpret_cast<const uint16_t*>(arow)[gi];
-    return nm24_dense_word(meta16, vals16);
-  } else {
-    const uint32_t m0 = mrow[2 * gi], m1 = mrow[2 * gi + 1];
-    const int bit = rem * 8 + gi * 4 * n;  // two blocks of n kept codes
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(arow);
-    const int wi = bit >> 5, sh = bit & 31;
-    uint32_t kv = p[wi] >> sh;
-    if (sh != 0 && sh + 4 * n > 32) kv |= p[wi + 1] << (32 - sh);
-    const uint32_t fmask = (1u << (2 * n)) - 1u;
-    return n8_dense_block(m0, kv & fmask) | (n8_dense_block(m1, (kv >> (2 * n)) & fmask) << 16);
-  }
+// Dense code word of 16 weights (group gi of the stage) of an n:8 row: two
+// blocks of n kept codes starting at bit rem * 8 + gi * 4n of the values.
+__device__ __forceinline__ uint32_t tc_n8_group_word(const uint8_t* arow, const uint8_t* mrow, int gi, int n,
+                                                     int rem) {
+  const uint32_t m0 = mrow[2 * gi], m1 = mrow[2 * gi + 1];
+  const int bit = rem * 8 + gi * 4 * n;
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(arow);
+  const int wi = bit >> 5, sh = bit & 31;
+  uint32_t kv = p[wi] >> sh;
+  if (sh != 0 && sh + 4 * n > 32) kv |= p[wi + 1] << (32 - sh);
+  const uint32_t fmask = (1u << (2 * n)) - 1u;
+  return n8_dense_block(m0, kv & fmask) | (n8_dense_block(m1, (kv >> (2 * n)) & fmask) << 16);
 }
 
 template <int BN, int NM>
@@ -354,7 +346,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                    (vw[gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu);
         } else {
 #pragma unroll
-          for (int gi = 0; gi < 8; ++gi) dw[gi] = tc_group_word<NM>(arow, mrow, gi, a.nm_n, rem);
+          for (int gi = 0; gi < 8; ++gi) dw[gi] = tc_n8_group_word(arow, mrow, gi, a.nm_n, rem);
         }
         uint32_t outw[32];
 #pragma unroll

@@ -381,21 +381,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr], s);
 }
 
-// ------------------------------------------------------------------ N:M M = 1
-// Expands kept codes + metadata of 16 dense weights into one dense 2-bit code
-// word (pruned positions get code 01, the zero weight).
-__device__ __forceinline__ uint32_t nm24_dense_word(uint32_t meta16, uint32_t vals16) {
-  uint32_t dense = 0x55555555u;
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {  // four 2:4 blocks
-    const uint32_t nib = (meta16 >> (4 * t)) & 0xFu;
-    const uint32_t i0 = nib & 3u, i1 = nib >> 2;
-    const uint32_t c0 = (vals16 >> (4 * t)) & 3u, c1 = (vals16 >> (4 * t + 2)) & 3u;
-    dense ^= ((c0 ^ 1u) << (8 * t + 2 * i0)) ^ ((c1 ^ 1u) << (8 * t + 2 * i1));
-  }
-  return dense;
-}
-
+// ------------------------------------------------------------------ N:M helpers
 // One n:8 block: inserts code 01 at every pruned position, in increasing order.
 __device__ __forceinline__ uint32_t n8_dense_block(uint32_t mask8, uint32_t kept) {
   uint32_t x = kept;
