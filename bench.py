@@ -163,11 +163,35 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+# Definitions the dense decode GEMV is compiled from (kernel, device helpers, PTX wrappers).
+GEMV_DEFS = ("gemv_dense_kernel", "quantise_row_smem", "quantise_row_smem_norm", "gemv_wchunk", "chunk_sum",
+             "dot_word", "gemv_store", "gemv_stripes", "gemv_stripe_bytes", "gemv_smem_bytes", "codes8", "codes8f",
+             "load8_raw", "sumsq8", "mbar_init", "mbar_arrive_expect_tx", "mbar_try_wait", "mbar_wait",
+             "fence_mbar_init", "tma_prefetch_desc", "tma_load_2d_hint", "l2_policy_evict_first", "dp4a_us",
+             "pdl_wait_primary", "pdl_launch_dependents", "smem_u32", "globaltimer_ns", "struct GemvDense",
+             "struct GemvMat")
+
+
 def gemv_source_hash() -> str:
+    """Fingerprint of the text of the definitions in GEMV_DEFS: a top-level definition runs from
+    its first line to the next line that is a lone closing brace."""
+    import re
     h = hashlib.sha256()
     for n in GEMV_SOURCES:
-        with open(os.path.join(ROOT, "ternary_weight_linear_fwd_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "ternary_weight_linear_fwd_b200", "csrc", n)) as f:
+            lines = f.read().split("\n")
+        i = 0
+        while i < len(lines):
+            line = lines[i]
+            hit = any(re.search(r"(^|\W)" + re.escape(d) + r"\s*(\(|\{|$)", line) for d in GEMV_DEFS)
+            if hit and not line.startswith((" ", "/", "#")):
+                j = i
+                while j < len(lines) and lines[j] not in ("}", "};"):
+                    j += 1
+                h.update("\n".join(lines[i:j + 1]).encode())
+                i = j + 1
+            else:
+                i += 1
     return h.hexdigest()[:16]
 
 
