@@ -500,6 +500,35 @@ def run_nm(dev, min_calls: int = 16, warmup: int = 3, reps: int = 5):
     return out
 
 
+def run_lut(dev, warmup: int = 3, reps: int = 5):
+    """Decode GEMV with dp4a against the TL2-style lookup-table variant, gate and down at M = 1
+    (PDL-chained graphs calling each of > 2 x L2 of weight copies once)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    out = {}
+    for name, K, N in (("gate", 2560, 6912), ("down", 6912, 2560)):
+        T = torch.from_numpy(synth.ternary_weights(N, K, seed=8)).to(dev)
+        w = bl.pack_ternary(T, float(synth.alpha_uniform(8)))
+        del T
+        cps = _copies(w, w.nbytes)
+        x = torch.from_numpy(synth.activations(1, K, seed=8).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        nbytes = N * K // 4 + 4 + 2 * K + 2 * N
+        row = {}
+        for label, fl in (("dp4a", bl.FLAG_PDL), ("lut", bl.FLAG_PDL | bl.FLAG_DECODE_LUT)):
+            calls = [(lambda ww=c, f=fl: bl.forward(ww, x, out=y, flags=f)) for c in cps]
+            sec = time_chain_graph(dev, calls, warmup, reps) / len(calls)
+            row[label] = {"us": sec * 1e6, "GBps": nbytes / sec / 1e9}
+        out[f"{name} {K}->{N}"] = row
+        del cps
+    assert bl.device_status() == 0
+    return out
+
+
 def run_norm(dev, warmup: int = 3, reps: int = 5, calls: int = 16):
     """RMSNorm fused into the activation quantisation: the fused kernel alone (GB/s) and
     forward_norm against forward on the 2B4T gate shape (2560 -> 6912), PDL-chained graphs."""
@@ -647,11 +676,12 @@ def main():
     e2e_value = aggregate(step_bytes, dec["e2e_steps"], world, max_e2e) / 1e9
 
     pre = run_prefill(dev, args.prefill_iters, 3)
-    sweep = nm = norm = None
+    sweep = nm = norm = lut = None
     if not args.no_sweep:
         sweep = run_sweep(dev)
         nm = run_nm(dev)
         norm = run_norm(dev)
+        lut = run_lut(dev)
 
     if world > 1:
         barrier(dev)
@@ -706,6 +736,9 @@ def main():
                                     "rmsnorm_quant_act bytes = 2MK (x) + MK (q) + 4K (g) + 8M; forward_norm vs "
                                     "forward (M=1: normalising quantisation + GEMV on the codes vs the GEMV "
                                     "quantising in-kernel; M>1: tensor-core path)", "by_M": norm}
+        line["decode_lut"] = {"workload": "decode GEMV at M=1, dp4a against per-pair lookup tables (TL2 idea), "
+                                          "ternary P(0)=0.42; PDL-chained graphs over > 2 x L2 of weight copies",
+                              "cases": lut}
     print(json.dumps(line), flush=True)
 
 

@@ -93,6 +93,11 @@ typedef enum bitlinear_status {
                                          ends. */
 #define BITLINEAR_FLAG_PATH_GEMV 0x2u /* force the M = 1 streaming GEMV (needs M == 1) */
 #define BITLINEAR_FLAG_PATH_TC 0x4u   /* force the tensor-core path at any M */
+#define BITLINEAR_FLAG_DECODE_LUT 0x8u /* M = 1, dense weights: run the decode GEMV with
+                                        * per-pair lookup tables (the TL2 idea of the
+                                        * "BitNet 1-Bit LLM" blog, section "I2_S kernel
+                                        * internals") instead of dp4a; same results.  A
+                                        * comparison path, not the default. */
 
 /* Packed weights.  All pointers device, caller-owned. */
 typedef struct bitlinear_weights {

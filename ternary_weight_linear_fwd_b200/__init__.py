@@ -16,13 +16,14 @@ __all__ = [
     "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
     "quant_act", "rmsnorm_quant_act", "forward", "forward_nm", "forward_group", "forward_norm",
     "forward_workspace_bytes", "device_status", "last_kernel",
-    "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC",
+    "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT",
 ]
 
 FLAG_PDL = 0x1
 MAX_GROUP = 4
 FLAG_PATH_GEMV = 0x2
 FLAG_PATH_TC = 0x4
+FLAG_DECODE_LUT = 0x8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libbitlinear.so")

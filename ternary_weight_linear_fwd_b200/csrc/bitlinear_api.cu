@@ -429,9 +429,45 @@ bitlinear_status gemv_dense_launch(const bitlinear_weights* const* w, uint16_t* 
   return st;
 }
 
-bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uint16_t* y, int32_t* acc, bool pdl,
-                              cudaStream_t s, DeviceState* dev) {
+// The lookup-table variant of the dense decode GEMV (one matrix).
+bitlinear_status gemv_lut_launch(const bitlinear_weights* w, uint16_t* y, int32_t* acc, const uint16_t* x, bool pdl,
+                                 cudaStream_t s, DeviceState* dev) {
+  GemvDense g;
+  std::memset(&g, 0, sizeof g);
   const int N = w->N, K = w->K;
+  g.ld = dense_ld(K);
+  g.C = static_cast<int>(g.ld / 16);
+  g.K = K;
+  g.x = x;
+  g.status = dev->status;
+  g.count = 1;
+  int grid = std::min(dev->sm_count, N);
+  auto fits = [&](int gr) {
+    const int rows_box = N / gr + 1;
+    return rows_box <= 256 && gemv_lut_smem_bytes(rows_box, g.ld, g.C) <= 200 * 1024;
+  };
+  while (!fits(grid) && grid < N) grid = std::min(N, grid * 2);
+  if (!fits(grid)) return BITLINEAR_ERR_SHAPE;
+  g.mat[0].alpha = w->alpha;
+  g.mat[0].y = y;
+  g.mat[0].acc = acc;
+  g.mat[0].rows_base = N / grid;
+  g.mat[0].rows_rem = N % grid;
+  g.rows_box = g.mat[0].rows_base + 1;
+  CUtensorMap map;
+  if (!make_map_u8(&map, w->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N), static_cast<uint64_t>(g.ld),
+                   128, static_cast<uint32_t>(g.rows_box), true))
+    return BITLINEAR_ERR_CUDA;
+  bitlinear_status st = launch(gemv_lut_kernel, dim3(grid), dim3(kGemvThreads),
+                               gemv_lut_smem_bytes(g.rows_box, g.ld, g.C), s, pdl, map, g);
+  if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_dense_lut";
+  return st;
+}
+
+bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uint16_t* y, int32_t* acc, bool pdl,
+                              cudaStream_t s, DeviceState* dev, bool lut = false) {
+  const int N = w->N, K = w->K;
+  if (w->nm_m == 0 && lut) return gemv_lut_launch(w, y, acc, x, pdl, s, dev);
   if (w->nm_m == 0) return gemv_dense_launch(&w, &y, &acc, 1, x, pdl, s, dev);
   int64_t ldv = 0, ldm = 0;
   if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
@@ -447,12 +483,12 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
   na.ld_m = ldm;
   na.K = K;
   na.C = (K + 127) / 128;
-  const bool lut = w->nm_m == 4;
+  const bool nm_lut = w->nm_m == 4;
   // about one CTA per SM; more while a CTA's rows exceed a TMA box or the shared-memory budget
   int grid = std::min(dev->sm_count, N);
   auto fits = [&](int g) {
     const int rows_box = N / g + 1;
-    return rows_box <= 256 && gemv_nm_smem_bytes(rows_box, ldv, ldm, na.C, lut) <= 160 * 1024;
+    return rows_box <= 256 && gemv_nm_smem_bytes(rows_box, ldv, ldm, na.C, nm_lut) <= 160 * 1024;
   };
   while (!fits(grid) && grid < N) grid = std::min(N, grid * 2);
   na.rows_base = N / grid;
@@ -464,7 +500,7 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
       !make_map_u8(&mm, w->meta, static_cast<uint64_t>(ldm), static_cast<uint64_t>(N), static_cast<uint64_t>(ldm), 128,
                    static_cast<uint32_t>(na.rows_box), true))
     return BITLINEAR_ERR_CUDA;
-  const size_t smem = gemv_nm_smem_bytes(na.rows_box, ldv, ldm, na.C, lut);
+  const size_t smem = gemv_nm_smem_bytes(na.rows_box, ldv, ldm, na.C, nm_lut);
   bitlinear_status st;
   switch (w->nm_m == 4 ? 0 : w->nm_n) {
     case 0: st = launch(gemv_nm_kernel<0>, dim3(grid), dim3(kGemvThreads), smem, s, pdl, mv, mm, na); break;
@@ -497,9 +533,11 @@ bitlinear_status check_matrix(const bitlinear_weights* w, const uint16_t* y, con
 }
 
 bitlinear_status check_flags(uint32_t flags, int M) {
-  const uint32_t known = BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_GEMV | BITLINEAR_FLAG_PATH_TC;
+  const uint32_t known = BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_GEMV | BITLINEAR_FLAG_PATH_TC |
+                         BITLINEAR_FLAG_DECODE_LUT;
   if (flags & ~known) return BITLINEAR_ERR_FLAGS;
   if ((flags & BITLINEAR_FLAG_PATH_GEMV) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
+  if ((flags & BITLINEAR_FLAG_DECODE_LUT) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
   return BITLINEAR_OK;
 }
 
@@ -520,7 +558,8 @@ bitlinear_status forward_common(const bitlinear_weights* w, const uint16_t* x, i
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || M > 1;
   if (tc) return forward_tc(w, x, M, y, acc, ws, ws_bytes, pdl, s, dev);
-  return forward_gemv(w, x, y, acc, pdl, s, dev);
+  if ((flags & BITLINEAR_FLAG_DECODE_LUT) && want_nm) return BITLINEAR_ERR_FLAGS;
+  return forward_gemv(w, x, y, acc, pdl, s, dev, (flags & BITLINEAR_FLAG_DECODE_LUT) != 0);
 }
 
 bitlinear_status forward_group(const bitlinear_weights* w, int count, const uint16_t* x, int M, uint16_t* const* y,

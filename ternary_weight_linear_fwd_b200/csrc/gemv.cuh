@@ -381,6 +381,94 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr], s);
 }
 
+// ------------------------------------------------------------------ dense M = 1, lookup tables
+// The TL2 lookup idea of bitnet.cpp ("BitNet 1-Bit LLM" blog, section "I2_S
+// kernel internals"): two consecutive ternary weights index a table of the
+// nine sums +-a0 +-a1 of their two activations.  Here the index is the pair's
+// 4-bit nibble of I2_S codes (c0 | c1 << 2, 9 of 16 entries used), the table
+// entry is (c0 - 1) q0 + (c1 - 1) q1 (int16) for the pair's int8 codes, and
+// one table of 16 entries per pair is built in shared memory after the
+// quantisation.  A unit (64-weight chunk, row) then costs 32 lookups and adds
+// instead of 16 masked dp4a: this kernel exists to measure that trade against
+// gemv_dense_kernel (same weights, same staging, same results).
+__host__ __device__ __forceinline__ size_t gemv_lut_smem_bytes(int rows_box, int64_t ld, int C) {
+  return gemv_smem_bytes(rows_box, ld, C) + static_cast<size_t>(C) * 32 * 16 * 2 + 16;
+}
+
+__global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_constant__ CUtensorMap map0,
+                                                                const GemvDense g) {
+  extern __shared__ uint8_t s_raw[];
+  __shared__ uint64_t s_bar;
+  __shared__ float s_red[32];
+  const GemvMat mt = g.mat[0];
+  const int b = blockIdx.x;
+  const int r0 = b * mt.rows_base + min(b, mt.rows_rem);
+  const int nrows = mt.rows_base + (b < mt.rows_rem ? 1 : 0);
+  const int C = g.C;
+  const int rows_box = g.rows_box;
+  const int stripes = gemv_stripes(g.ld);
+  const int stripe_bytes = gemv_stripe_bytes(rows_box);
+  uint8_t* s_w = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
+  uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
+  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_act + 4 * C);
+  int32_t* s_acc = s_hsum + 8 * C;
+  int16_t* s_lut = reinterpret_cast<int16_t*>(s_acc + rows_box + 3 - ((rows_box + 3) & 3));  // [pairs][16]
+
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&map0);
+    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box));
+    const uint64_t pol = l2_policy_evict_first();
+    for (int st = 0; st < stripes; ++st) tma_load_2d_hint(s_w + st * stripe_bytes, &map0, st * 128, r0, &s_bar, pol);
+  }
+  const float alpha = *mt.alpha;
+  for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  __syncthreads();
+
+  pdl_wait_primary();
+  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_hsum, s_red);
+  pdl_launch_dependents();
+  // tables: pair p covers k = 2p, 2p + 1; code of k sits in group k / 16, word k % 4, byte (k % 16) / 4
+  const int pairs = 32 * C;  // 64-weight chunks of 32 pairs (codes past K are 0)
+  const int quarter = C;     // s_act slot stride (groups_alloc / 4)
+  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+    int32_t qv[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int k = 2 * p + t, gi = k >> 4;
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(s_act + (gi & 3) * quarter + (gi >> 2));
+      qv[t] = static_cast<int8_t>(w[k & 3] >> (8 * ((k & 15) >> 2)));
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      s_lut[16 * p + n] = static_cast<int16_t>(((n & 3) - 1) * qv[0] + ((n >> 2) - 1) * qv[1]);
+  }
+  __syncthreads();
+  const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
+  const bool landed = mbar_wait(&s_bar, 0);
+  if (!landed && threadIdx.x == 0) *g.status = kDevTimeoutProducer;
+
+  if (landed) {
+    const int total = nrows * C;  // units (chunk, row), row fastest
+    for (int u = threadIdx.x; u < total; u += blockDim.x) {
+      const int ch = u / nrows, r = u - ch * nrows;
+      const uint4 wv = gemv_wchunk(s_w, stripe_bytes, r, ch);
+      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+      const int16_t* lut = s_lut + 16 * 32 * ch;
+      int32_t acc = 0;
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc += lut[16 * (8 * wi + i) + ((ww[wi] >> (4 * i)) & 0xFu)];
+      atomicAdd(&s_acc[r], acc);
+    }
+  }
+  __syncthreads();
+  if (landed)
+    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr], s);
+}
+
 // ------------------------------------------------------------------ N:M helpers
 // One n:8 block: inserts code 01 at every pruned position, in increasing order.
 __device__ __forceinline__ uint32_t n8_dense_block(uint32_t mask8, uint32_t kept) {

@@ -90,6 +90,8 @@ def test_forward_host_checks(L):
     assert fw(ctypes.byref(w), x, 1, y, None, None, 0, 0x80, None) == 8          # unknown flag
     assert fw(ctypes.byref(w), x, 2, y, None, None, 0, 0x2, None) == 8           # GEMV path needs M == 1
     assert fw(ctypes.byref(w), x, 1, y, None, None, 0, 0x6, None) == 8           # both path flags
+    assert fw(ctypes.byref(w), x, 2, y, None, None, 0, 0x8, None) == 8           # lookup-table decode needs M == 1
+    assert fw(ctypes.byref(w), x, 1, y, None, None, 0, 0xC, None) == 8           # ... and the GEMV path
     nmw = _w(L, n=6, m=8, meta=0x50000)
     assert fw(ctypes.byref(nmw), x, 1, y, None, None, 0, 0, None) == 4          # dense entry, N:M weights
     assert L.bitlinear_forward_nm(ctypes.byref(w), x, 1, y, None, None, 0, 0, None) == 4

@@ -311,6 +311,20 @@ def test_forward_group_prefill_sampled():
         _check_rows(x, T, a, y, acc, rows)
 
 
+# ---------------------------------------------------------------- lookup-table decode (comparison path)
+
+@pytest.mark.parametrize("K,N", [(256, 512), (2560, 6912), (6912, 2560), (200, 33), (1032, 300)])
+def test_forward_decode_lut_matches(K, N):
+    """The TL2-style lookup-table GEMV gives the dp4a GEMV's results bit for bit, and the oracle's."""
+    x, Wt, a, w = _dense_case(1, K, N, seed=K + 3 * N, ternary=True)
+    xd = to_dev_bf16(x)
+    y, acc = bl.forward(w, xd, want_acc=True, flags=bl.FLAG_DECODE_LUT)
+    assert bl.last_kernel() == "gemv_m1_dense_lut"
+    y0, acc0 = bl.forward(w, xd, want_acc=True)
+    assert torch.equal(acc, acc0) and torch.equal(y.view(torch.int16), y0.view(torch.int16))
+    _check_rows(x, Wt, a, y, acc, np.arange(1))
+
+
 # ---------------------------------------------------------------- RMSNorm before the quantisation
 
 def _norm_weight(K, seed):
