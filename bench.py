@@ -164,7 +164,7 @@ def measured_peaks():
 
 
 # Definitions the dense decode GEMV is compiled from (kernel, device helpers, PTX wrappers).
-GEMV_DEFS = ("gemv_dense_kernel", "quantise_row_smem", "quantise_row_smem_norm", "gemv_wchunk", "chunk_sum",
+GEMV_DEFS = ("gemv_dense_kernel", "quantise_row_smem", "quantise_row_smem_norm", "gemv_wchunk",
              "dot_word", "gemv_store", "gemv_stripes", "gemv_stripe_bytes", "gemv_smem_bytes", "codes8", "codes8f",
              "load8_raw", "sumsq8", "mbar_init", "mbar_arrive_expect_tx", "mbar_try_wait", "mbar_wait",
              "fence_mbar_init", "tma_prefetch_desc", "tma_load_2d_hint", "l2_policy_evict_first", "dp4a_us",

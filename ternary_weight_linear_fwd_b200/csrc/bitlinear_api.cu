@@ -242,9 +242,17 @@ QuantWs tc_ws_layout(void* ws, int M, int K, int ncnt, int max_n) {
   return r;
 }
 
+// The quant_act_kernel instantiation for G k-groups per lane in registers.
+template <bool kPermute, bool kNorm>
+auto quant_kernel(int G) {
+  return G == 2 ? quant_act_kernel<kPermute, kNorm, 2>
+                : G == 3 ? quant_act_kernel<kPermute, kNorm, 3> : quant_act_kernel<kPermute, kNorm, 8>;
+}
+
 bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s,
                           const float* gnorm = nullptr, float eps = 0.0f) {
-  const int wpr = quant_warps_per_row(K);
+  const QuantShape qs = quant_shape(K);
+  const int wpr = qs.wpr;
   const int rows_per_cta = kQuantWarps / wpr;
   const int qblocks = (M + rows_per_cta - 1) / rows_per_cta;
   // extra CTAs clear the split-K sums, 16 bytes per thread and step, at most four steps each
@@ -253,10 +261,10 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
                                                                    (4 * 32 * kQuantWarps)));
   uint32_t* cnt = qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr);
   if (gnorm)
-    return launch(quant_act_kernel<true, true>, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
+    return launch(quant_kernel<true, true>(qs.G), dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
                   static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr, gnorm,
                   eps);
-  return launch(quant_act_kernel<true, false>, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
+  return launch(quant_kernel<true, false>(qs.G), dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
                 static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr,
                 static_cast<const float*>(nullptr), 0.0f);
 }
@@ -730,9 +738,10 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
   DeviceState* dev = nullptr;
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
-  const int wpr = quant_warps_per_row(K);
+  const QuantShape qs = quant_shape(K);
+  const int wpr = qs.wpr;
   const int qblocks = (M + kQuantWarps / wpr - 1) / (kQuantWarps / wpr);
-  st = launch(quant_act_kernel<false, false>, dim3(qblocks), dim3(32 * kQuantWarps), 0,
+  st = launch(quant_kernel<false, false>(qs.G), dim3(qblocks), dim3(32 * kQuantWarps), 0,
               static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum, static_cast<uint32_t*>(nullptr), 0,
               static_cast<float*>(nullptr), static_cast<size_t>(0), qblocks, wpr, static_cast<const float*>(nullptr),
               0.0f);
@@ -751,9 +760,10 @@ bitlinear_status bitlinear_rmsnorm_quant_act(const uint16_t* x, int32_t M, int32
   DeviceState* dev = nullptr;
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
-  const int wpr = quant_warps_per_row(K);
+  const QuantShape qs = quant_shape(K);
+  const int wpr = qs.wpr;
   const int qblocks = (M + kQuantWarps / wpr - 1) / (kQuantWarps / wpr);
-  st = launch(quant_act_kernel<false, true>, dim3(qblocks), dim3(32 * kQuantWarps), 0,
+  st = launch(quant_kernel<false, true>(qs.G), dim3(qblocks), dim3(32 * kQuantWarps), 0,
               static_cast<cudaStream_t>(stream), false, x, M, K, K, q, gamma, rowsum, static_cast<uint32_t*>(nullptr), 0,
               static_cast<float*>(nullptr), static_cast<size_t>(0), qblocks, wpr, g, eps);
   if (st == BITLINEAR_OK) t_last_kernel = "rmsnorm_quant_act";

@@ -12,6 +12,7 @@
 // splits the (64-weight chunk, row) products evenly over all its threads.
 // With code = W_t + 1:
 //     acc = sum_k q_k * W_t,k = sum_k q_k * code_k - sum_k q_k
+// where sum_k q_k is the same for every row (formed once, with the codes),
 // and sum_k q_k * code_k is formed four bytes at a time with an unsigned x
 // signed dp4a on (word & (3 << 2j) per byte), whose partial sums carry a
 // factor 4^j that is removed exactly at the end (every term is a multiple).
@@ -28,15 +29,16 @@ constexpr int kGemvThreads = 512;
 // 16g + 4b + j), for g < groups_alloc (zero past K), where
 // slot(g) = (g % 4) * (groups_alloc / 4) + g / 4 puts the four groups of one
 // 64-weight chunk a quarter of the array apart, so lanes reading consecutive
-// chunks hit consecutive 16-byte words; s_hsum[h] is the sum of the 8 codes of
-// half h (chunk_sum adds the eight of a chunk).  Each thread handles 8-element
-// halves h = tid, tid + nthr, ...: one 16-byte load, 8 codes, four 16-bit
-// stores (bytes 2*(h%2), 2*(h%2)+1 of words 0..3) and its code sum.  One
-// barrier publishes the per-warp maxima, one the codes.  Returns gamma = max |x|.
+// chunks hit consecutive 16-byte words.  *s_qsum (zeroed by the caller before
+// a barrier that precedes this call) receives the sum of all codes.  Each
+// thread handles 8-element halves h = tid, tid + nthr, ...: one 16-byte load,
+// 8 codes and four 16-bit stores (bytes 2*(h%2), 2*(h%2)+1 of words 0..3).
+// One barrier publishes the per-warp maxima, one the codes and their sum.
+// Returns gamma = max |x|.
 constexpr int kHalvesInRegs = 2;  // halves per thread kept in registers (K <= 8192 at 512 threads)
 
 __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ x, int K, int groups_alloc,
-                                                   uint4* s_act, int32_t* s_hsum, float* s_red) {
+                                                   uint4* s_act, int32_t* s_qsum, float* s_red) {
   const bool vec_ok = (K % 8) == 0;
   const int nthr = blockDim.x;
   const int halves = (K + 7) / 8;
@@ -72,6 +74,7 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
   const float d = __fadd_rn(mx, kEps);
   const float c = __fmul_rn(kQb, __frcp_rn(d));
   const int quarter = groups_alloc >> 2;
+  int32_t qsum = 0;
   auto emit = [&](const uint32_t (&raw)[4], int h) {
     uint32_t b[8];
     codes8(raw, c, d, b);
@@ -79,7 +82,7 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
     const uint32_t lo2 = __byte_perm(b[4], b[5], 0x0040), hi2 = __byte_perm(b[6], b[7], 0x0040);
     const uint32_t p0 = __byte_perm(lo, hi, 0x5410), p1 = __byte_perm(lo2, hi2, 0x5410);  // codes 0..3, 4..7
     if (h < halves_alloc) {
-      s_hsum[h] = __dp4a(static_cast<int>(p1), 0x01010101, __dp4a(static_cast<int>(p0), 0x01010101, 0));
+      qsum = __dp4a(static_cast<int>(p1), 0x01010101, __dp4a(static_cast<int>(p0), 0x01010101, qsum));
       const int g = h >> 1, half = h & 1;
       const int sl = (g & 3) * quarter + (g >> 2);
       uint16_t* dst = reinterpret_cast<uint16_t*>(s_act + sl) + half;
@@ -99,6 +102,8 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
     if (h < halves) load8_raw(x, h * 8, K, vec_ok, raw);
     emit(raw, h);
   }
+  qsum = __reduce_add_sync(0xffffffffu, qsum);
+  if ((threadIdx.x & 31) == 0) atomicAdd(s_qsum, qsum);
   __syncthreads();
   return mx;
 }
@@ -108,7 +113,7 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
 // fixed-order reduction over the CTA), the root and the quotient in fp64;
 // the codes are those of xn = RN(RN(x * r) * g), which is never stored.
 __device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restrict__ x, int K, int groups_alloc,
-                                                        uint4* s_act, int32_t* s_hsum, float* s_red, double* s_redd,
+                                                        uint4* s_act, int32_t* s_qsum, float* s_red, double* s_redd,
                                                         const float* s_g, float eps) {
   const bool vec_ok = (K % 8) == 0;
   const int nthr = blockDim.x;
@@ -176,6 +181,7 @@ __device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restri
   const float d = __fadd_rn(mx, kEps);
   const float c = __fmul_rn(kQb, __frcp_rn(d));
   const int quarter = groups_alloc >> 2;
+  int32_t qsum = 0;
   auto emit = [&](const uint32_t (&raw)[4], int h) {
     float xn[8];
     norm8(raw, h, xn);
@@ -185,7 +191,7 @@ __device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restri
     const uint32_t lo2 = __byte_perm(b[4], b[5], 0x0040), hi2 = __byte_perm(b[6], b[7], 0x0040);
     const uint32_t p0 = __byte_perm(lo, hi, 0x5410), p1 = __byte_perm(lo2, hi2, 0x5410);
     if (h < halves_alloc) {
-      s_hsum[h] = __dp4a(static_cast<int>(p1), 0x01010101, __dp4a(static_cast<int>(p0), 0x01010101, 0));
+      qsum = __dp4a(static_cast<int>(p1), 0x01010101, __dp4a(static_cast<int>(p0), 0x01010101, qsum));
       const int g = h >> 1, half = h & 1;
       const int sl = (g & 3) * quarter + (g >> 2);
       uint16_t* dst = reinterpret_cast<uint16_t*>(s_act + sl) + half;
@@ -204,6 +210,8 @@ __device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restri
     if (h < halves) load8_raw(x, h * 8, K, vec_ok, raw);
     emit(raw, h);
   }
+  qsum = __reduce_add_sync(0xffffffffu, qsum);
+  if ((threadIdx.x & 31) == 0) atomicAdd(s_qsum, qsum);
   __syncthreads();
   return mx;
 }
@@ -212,13 +220,6 @@ __device__ __forceinline__ void gemv_store(uint16_t* y, int32_t* acc, int row, i
   if (acc) acc[row] = total;
   const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(total), s));
   y[row] = *reinterpret_cast<const uint16_t*>(&h);
-}
-
-// Sum of the 64 codes of chunk ch (eight half sums; s_hsum 16-byte aligned).
-__device__ __forceinline__ int32_t chunk_sum(const int32_t* s_hsum, int ch) {
-  const int4 a = reinterpret_cast<const int4*>(s_hsum)[2 * ch];
-  const int4 b = reinterpret_cast<const int4*>(s_hsum)[2 * ch + 1];
-  return (a.x + a.y) + (a.z + a.w) + ((b.x + b.y) + (b.z + b.w));
 }
 
 // Dot of one packed 32-bit weight word (16 codes) with its 4 activation words.
@@ -245,7 +246,7 @@ __host__ __device__ __forceinline__ int gemv_stripe_bytes(int rows_box) { return
 
 __host__ __device__ __forceinline__ size_t gemv_smem_bytes(int rows_box, int64_t ld, int C) {
   return 1024 /* alignment */ + static_cast<size_t>(gemv_stripes(ld)) * gemv_stripe_bytes(rows_box) +
-         static_cast<size_t>(C) * 4 * 16 + static_cast<size_t>(C) * 8 * 4 + static_cast<size_t>(rows_box) * 4;
+         static_cast<size_t>(C) * 4 * 16 + 16 /* code sum */ + static_cast<size_t>(rows_box) * 4;
 }
 
 // Weight chunk ch of local row r in the swizzled stripes.
@@ -308,8 +309,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   // offset arithmetic on the shared array keeps every derived pointer in the shared window
   uint8_t* s_w = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
   uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
-  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_act + 4 * C);  // 8 * C half sums
-  int32_t* s_acc = s_hsum + 8 * C;
+  int32_t* s_qsum = reinterpret_cast<int32_t*>(s_act + 4 * C);  // sum of the codes (one 16-byte slot)
+  int32_t* s_acc = s_qsum + 4;
   float* s_g = reinterpret_cast<float*>(s_acc + rows_box);        // norm variant: RMSNorm weight [K]
   __shared__ double s_redd[32];
 
@@ -325,6 +326,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   }
   const float alpha = *mt.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  if (threadIdx.x == 0) *s_qsum = 0;
   if (kNorm)  // the norm weight, like the matrix, does not depend on the preceding kernel
     for (int k = threadIdx.x; k < g.K; k += blockDim.x) s_g[k] = g.gnorm[k];
   __syncthreads();
@@ -332,9 +334,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   pdl_wait_primary();  // x may come from the preceding kernel
   float gamma;
   if (kNorm)
-    gamma = quantise_row_smem_norm(g.x, g.K, 4 * C, s_act, s_hsum, s_red, s_redd, s_g, g.eps);
+    gamma = quantise_row_smem_norm(g.x, g.K, 4 * C, s_act, s_qsum, s_red, s_redd, s_g, g.eps);
   else
-    gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_hsum, s_red);
+    gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qsum, s_red);
   // The next kernel may start now: its weight copies then stream while this
   // one contracts, and no longer delay this kernel's read of x.
   pdl_launch_dependents();
@@ -355,7 +357,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
       const uint4 wa = gemv_wchunk(s_w, stripe_bytes, p, ch);
       const uint4 wb = gemv_wchunk(s_w, stripe_bytes, r2, ch);
       const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
-      const int32_t cs = chunk_sum(s_hsum, ch);
       int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
       dot_word(wa.x, q0.x, q0.y, q0.z, q0.w, a0, a1, a2, a3);
       dot_word(wb.x, q0.x, q0.y, q0.z, q0.w, b0, b1, b2, b3);
@@ -366,8 +367,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
       dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
       dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
       // every partial sum s_j is a multiple of 4^j, so the shifts are exact
-      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6) - cs);
-      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6) - cs);
+      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6));
+      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6));
       p += dr;
       ch += dq;
       if (p >= half) {
@@ -377,8 +378,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     }
   }
   __syncthreads();
-  if (landed)
-    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr], s);
+  if (landed) {
+    const int32_t qsum = *s_qsum;
+    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr] - qsum, s);
+  }
 }
 
 // ------------------------------------------------------------------ dense M = 1, lookup tables
@@ -410,8 +413,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_con
   const int stripe_bytes = gemv_stripe_bytes(rows_box);
   uint8_t* s_w = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
   uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
-  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_act + 4 * C);
-  int32_t* s_acc = s_hsum + 8 * C;
+  int32_t* s_qsum = reinterpret_cast<int32_t*>(s_act + 4 * C);  // filled, not needed: the tables carry W_t
+  int32_t* s_acc = s_qsum + 4;
   int16_t* s_lut = reinterpret_cast<int16_t*>(s_acc + rows_box + 3 - ((rows_box + 3) & 3));  // [pairs][16]
 
   if (threadIdx.x == 0) {
@@ -424,10 +427,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_con
   }
   const float alpha = *mt.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  if (threadIdx.x == 0) *s_qsum = 0;
   __syncthreads();
 
   pdl_wait_primary();
-  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_hsum, s_red);
+  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qsum, s_red);
   pdl_launch_dependents();
   // tables: pair p covers k = 2p, 2p + 1; code of k sits in group k / 16, word k % 4, byte (k % 16) / 4
   const int pairs = 32 * C;  // 64-weight chunks of 32 pairs (codes past K are 0)
@@ -515,7 +519,7 @@ __host__ __device__ __forceinline__ int nm_unit_value_bytes(int n) { return n ==
 __host__ __device__ __forceinline__ size_t gemv_nm_smem_bytes(int rows_box, int64_t ld_v, int64_t ld_m, int C, bool lut) {
   return 1024 + static_cast<size_t>(gemv_stripes(ld_v) + gemv_stripes(ld_m)) * gemv_stripe_bytes(rows_box) +
          (lut ? static_cast<size_t>(kNmLutWords) * 4 : 0) + static_cast<size_t>(C) * 8 * 16 /* codes */ +
-         static_cast<size_t>(C) * 16 * 4 /* half sums */ + static_cast<size_t>(rows_box) * 4;
+         16 /* code sum */ + static_cast<size_t>(rows_box) * 4;
 }
 
 // 32-bit word at byte offset off (a multiple of 4) of local row r in swizzled 128-byte stripes.
@@ -603,8 +607,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
   uint8_t* s_m = s_v + static_cast<size_t>(stripes_v) * stripe_bytes;
   uint32_t* s_lut = reinterpret_cast<uint32_t*>(s_m + static_cast<size_t>(stripes_m) * stripe_bytes);
   uint4* s_act = reinterpret_cast<uint4*>(s_lut + (NMN == 0 ? kNmLutWords : 0));
-  int32_t* s_hsum = reinterpret_cast<int32_t*>(s_act + 8 * C);  // 16 * C half sums
-  int32_t* s_acc = s_hsum + 16 * C;
+  int32_t* s_qsum = reinterpret_cast<int32_t*>(s_act + 8 * C);  // sum of the codes (one 16-byte slot)
+  int32_t* s_acc = s_qsum + 4;
 
   if (threadIdx.x == 0) {
     mbar_init(&s_bar, 1);
@@ -619,10 +623,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
   if (NMN == 0) nm24_fill_lut(s_lut);
   const float alpha = *a.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  if (threadIdx.x == 0) *s_qsum = 0;
   __syncthreads();
 
   pdl_wait_primary();  // x may come from the preceding kernel
-  const float gamma = quantise_row_smem(a.x, a.K, 8 * C, s_act, s_hsum, s_red);
+  const float gamma = quantise_row_smem(a.x, a.K, 8 * C, s_act, s_qsum, s_red);
   pdl_launch_dependents();
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
@@ -641,7 +646,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
       uint32_t da[8], db[8];
       nm_unit_words<NMN>(s_v, s_m, stripe_bytes, p, u, lut_lane, da);
       nm_unit_words<NMN>(s_v, s_m, stripe_bytes, r2, u, lut_lane, db);
-      const int32_t cs = chunk_sum(s_hsum, 2 * u) + chunk_sum(s_hsum, 2 * u + 1);
       int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
 #pragma unroll
       for (int gi = 0; gi < 8; ++gi) {
@@ -650,8 +654,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
         dot_word(da[gi], q.x, q.y, q.z, q.w, a0, a1, a2, a3);
         dot_word(db[gi], q.x, q.y, q.z, q.w, b0, b1, b2, b3);
       }
-      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6) - cs);
-      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6) - cs);
+      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6));
+      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6));
       p += dr;
       u += dq;
       if (p >= half) {
@@ -661,8 +665,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
     }
   }
   __syncthreads();
-  if (landed)
-    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a.y, a.acc, r0 + rr, s_acc[rr], s);
+  if (landed) {
+    const int32_t qsum = *s_qsum;
+    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a.y, a.acc, r0 + rr, s_acc[rr] - qsum, s);
+  }
 }
 
 }  // namespace bl

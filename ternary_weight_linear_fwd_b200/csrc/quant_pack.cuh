@@ -51,13 +51,15 @@ struct AddD {
 };
 
 // Exact round-half-to-even of RN(t / d), t = RN(v * 127), for |t / d| < 128,
-// without a division per element.  With c = RN(127 * RN(1 / d)), y = RN(v * c)
-// differs from the true quotient by at most 3 * 2^-24 relative, i.e. by less
-// than 3.1e-5 absolute, and RN(t / d) lies within 7.6e-6 of the true quotient.
-// So unless y sits within 2^-14 of a half-integer, RN(t / d) rounds to the same
-// integer as y; such a group is recomputed with the exact quotient.  The
-// rounding to an integer is done by adding 1.5 * 2^23 (the sum's last place is
-// 1, ties to even), leaving the two's-complement code in the low byte.
+// without a division per element.  With c = RN(127 * RN(1 / d)), the exact
+// product v * c differs from t / d by at most 2 * 2^-24 relative (bf16 v: t is
+// exact), i.e. by less than 1.6e-5 absolute, and RN(t / d) lies within 7.6e-6
+// of t / d.  One fused multiply-add, r' = RN(v * c + 1.5 * 2^23), rounds the
+// exact product to the nearest integer r (the sum's last place is 1, ties to
+// even) and leaves the two's-complement code in the low byte; a second,
+// e = RN(v * c - r), gives the distance to it within 2^-25.  Unless some |e| of
+// a group exceeds 1/2 - 2^-14, RN(t / d) is nearer than 1/2 to r and rounds to
+// it; such a group is recomputed with the exact quotient.
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
 
 // Codes of 8 consecutive activations (the first or second half of a 16-group).  b[e] holds the code of
@@ -67,9 +69,8 @@ __device__ __forceinline__ void codes8(const uint32_t (&raw)[4], float c, float 
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const float v = __uint_as_float((e & 1) ? (raw[e >> 1] & 0xFFFF0000u) : (raw[e >> 1] << 16));
-    const float yq = __fmul_rn(v, c);
-    const float sm = __fadd_rn(yq, kMagic);
-    emax = fmaxf(emax, fabsf(__fsub_rn(yq, __fsub_rn(sm, kMagic))));
+    const float sm = __fmaf_rn(v, c, kMagic);
+    emax = fmaxf(emax, fabsf(__fmaf_rn(v, c, -__fsub_rn(sm, kMagic))));
     b[e] = __float_as_uint(sm);
   }
   if (emax > 0.5f - 6.103515625e-05f) {
@@ -82,15 +83,14 @@ __device__ __forceinline__ void codes8(const uint32_t (&raw)[4], float c, float 
 }
 
 // codes8 for fp32 values (RMSNorm outputs): the same rounding argument holds
-// with t = RN(v * 127) no longer exact, since |y - RN(t / d)| stays below
-// 5 * 2^-24 * 127 < 2^-14; the fallback recomputes RN(RN(v * 127) / d).
+// with t = RN(v * 127) no longer exact, since |v * c - RN(t / d)| stays below
+// 4 * 2^-24 * 127 < 2^-14; the fallback recomputes RN(RN(v * 127) / d).
 __device__ __forceinline__ void codes8f(const float* v, float c, float d, uint32_t (&b)[8]) {
   float emax = 0.0f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    const float yq = __fmul_rn(v[e], c);
-    const float sm = __fadd_rn(yq, kMagic);
-    emax = fmaxf(emax, fabsf(__fsub_rn(yq, __fsub_rn(sm, kMagic))));
+    const float sm = __fmaf_rn(v[e], c, kMagic);
+    emax = fmaxf(emax, fabsf(__fmaf_rn(v[e], c, -__fsub_rn(sm, kMagic))));
     b[e] = __float_as_uint(sm);
   }
   if (emax > 0.5f - 6.103515625e-05f) {
@@ -117,11 +117,14 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 
 // ----------------------------------------------------------------- quant_act
 // A token row is handled by wpr warps of a 256-thread CTA (wpr = 1, 2, 4 or 8,
-// chosen by K; 8 / wpr rows per CTA).  A lane owns the 16-wide k-groups
+// 8 / wpr rows per CTA).  A lane owns the 16-wide k-groups
 // g = sub * 32 + lane + j * 32 * wpr of its row; when the row fits (K % 8 == 0,
-// at most kQuantGroupsInRegs groups per lane) every load of the row is issued
-// at once into registers, so each element is read from memory once and all of
-// a CTA's reads are in flight together.  gamma is an integer warp max of the
+// at most G groups per lane) every load of the row is issued at once into
+// registers, so each element is read from memory once and all of a CTA's
+// reads are in flight together.  quant_shape picks the smallest wpr that
+// leaves at most three groups per lane (short per-warp chains, many warps in
+// flight; the kernel is bound by latency, not by issue) and G, a compile-time
+// register count of 2, 3 or 8.  gamma is an integer warp max of the
 // |x| bit patterns (then across the row's warps), and the 16 codes of a group
 // come from the division-free exact rounding of codes8.  Longer or unaligned
 // rows take a two-pass loop (the second pass re-reads from L1/L2).
@@ -135,10 +138,18 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 // past the rows (blockIdx >= qblocks) clear the split-K sums, of the GEMMs that
 // read these codes.
 constexpr int kQuantWarps = 8;
-constexpr int kQuantGroupsInRegs = 8;
 
-__host__ __device__ __forceinline__ int quant_warps_per_row(int K) {
-  return K <= 4096 ? 1 : K <= 8192 ? 2 : K <= 16384 ? 4 : 8;
+struct QuantShape {
+  int wpr;  // warps per token row
+  int G;    // k-groups per lane held in registers (template argument: 2, 3 or 8)
+};
+
+__host__ __device__ __forceinline__ QuantShape quant_shape(int K) {
+  const int groups = (K + 15) / 16;
+  int wpr = 1;
+  while (wpr < kQuantWarps && groups > 3 * 32 * wpr) wpr *= 2;
+  const int need = (groups + 32 * wpr - 1) / (32 * wpr);
+  return {wpr, need <= 2 ? 2 : need <= 3 ? 3 : 8};
 }
 
 // 16 codes of one k-group (raw: the group's 16 bf16 as 8 words) in the
@@ -214,7 +225,7 @@ __device__ __forceinline__ float absmax8(const uint32_t (&w)[4], float mx) {
   return mx;
 }
 
-template <bool kPermute, bool kNorm>
+template <bool kPermute, bool kNorm, int G>
 __global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                      int ldq, int8_t* __restrict__ q,
                                                                      float* __restrict__ gamma,
@@ -246,15 +257,15 @@ __global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint1
   const int groups = (K + 15) / 16;
   const int gstride = 32 * wpr;
   const int g0 = sub * 32 + lane;
-  const bool in_regs = vec_ok && groups <= kQuantGroupsInRegs * gstride;
+  const bool in_regs = vec_ok && groups <= G * gstride;
 
   // Calls f(g, r0, r1) for each of this lane's groups with the group's raw
   // bf16 words: from registers (unrolled, static indices) or loaded again.
-  uint32_t v[kQuantGroupsInRegs][8];
+  uint32_t v[G][8];
   auto for_groups = [&](auto&& f) {
     if (in_regs) {
 #pragma unroll
-      for (int j = 0; j < kQuantGroupsInRegs; ++j) {
+      for (int j = 0; j < G; ++j) {
         const int g = g0 + j * gstride;
         if (g < groups) {
           uint32_t r0[4], r1[4];
@@ -277,7 +288,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint1
   };
   if (active && in_regs) {
 #pragma unroll
-    for (int j = 0; j < kQuantGroupsInRegs; ++j) {
+    for (int j = 0; j < G; ++j) {
       const int k0 = 16 * (g0 + j * gstride);
       uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
       if (k0 + 8 <= K) a = *reinterpret_cast<const uint4*>(xr + k0);

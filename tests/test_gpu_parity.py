@@ -345,6 +345,35 @@ def test_rmsnorm_quant_act_bit_exact(M, K):
     assert bl.last_kernel() == "rmsnorm_quant_act"
 
 
+# Every launch shape of the quantisation kernel (warps per token row, k-groups
+# per lane held in registers): K = 1536 (1 warp, 3 groups), 1544 (2, 2, a
+# half-filled last group), 2048 (2, 2), 4096 (4, 2), 16384 (8, 8 in registers),
+# 40008 (8, the streaming loop), each in natural order, with RMSNorm, and in
+# contraction order through the tensor-core forward with and without the norm.
+@pytest.mark.parametrize("K", [1536, 1544, 2048, 4096, 16384, 40008])
+def test_quant_every_launch_shape(K):
+    M, N = 3, 40
+    x, Wt, a, w = _dense_case(M, K, N, seed=K)
+    q, gm, rs = bl.quant_act(to_dev_bf16(x))
+    qo, go, ro = oracle.quant_act(x)
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(gm.cpu().numpy(), go)
+    np.testing.assert_array_equal(rs.cpu().numpy(), ro)
+    g = _norm_weight(K, K + 1)
+    gd = torch.from_numpy(g).to(DEV)
+    q, gm, rs = bl.rmsnorm_quant_act(to_dev_bf16(x), gd, 1e-6)
+    qo, go, ro = oracle.quant_act_f32(oracle.rmsnorm(x, g, 1e-6))
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(gm.cpu().numpy(), go)
+    np.testing.assert_array_equal(rs.cpu().numpy(), ro)
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, flags=bl.FLAG_PATH_TC)
+    _check_rows(x, Wt, a, y, acc, np.arange(M))
+    y, acc = bl.forward_norm(w, to_dev_bf16(x), gd, 1e-6, want_acc=True)
+    yo, acco, *_ = oracle.forward_norm(x, g, 1e-6, Wt, a)
+    np.testing.assert_array_equal(acc.cpu().numpy(), acco)
+    assert_bf16_close(bf16_bits(y), yo)
+
+
 @pytest.mark.parametrize("n,m", [(0, 0), (2, 4), (6, 8)])
 @pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (16, 1024, 300), (300, 512, 1000)])
 def test_forward_norm(n, m, M, K, N):
