@@ -529,6 +529,43 @@ def run_lut(dev, warmup: int = 3, reps: int = 5):
     return out
 
 
+def run_isolated(dev, iters: int = 30, warmup: int = 3):
+    """Latency of one isolated forward call at M = 1 (gate 2560 -> 6912, down 6912 -> 2560): per
+    iteration a 256 MB L2-flushing write, then one eager call without PDL between two CUDA events
+    on the launching stream; median over `iters` (launch latency included, no graph)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream(dev)
+    out = {}
+    for name, K, N in (("gate", 2560, 6912), ("down", 6912, 2560)):
+        T = torch.from_numpy(synth.ternary_weights(N, K, seed=9)).to(dev)
+        w = bl.pack_ternary(T, float(synth.alpha_uniform(9)))
+        del T
+        x = torch.from_numpy(synth.activations(1, K, seed=9).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(warmup):
+            bl.forward(w, x, out=y, flags=0)
+        ts = []
+        for _ in range(iters):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            bl.forward(w, x, out=y, flags=0)
+            e1.record(s)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        sec = statistics.median(ts)
+        nbytes = N * K // 4 + 4 + 2 * K + 2 * N
+        out[f"{name} {K}->{N}"] = {"us": sec * 1e6, "GBps": nbytes / sec / 1e9, "kernel": bl.last_kernel()}
+    assert bl.device_status() == 0
+    return out
+
+
 def run_norm(dev, warmup: int = 3, reps: int = 5, calls: int = 16):
     """RMSNorm fused into the activation quantisation: the fused kernel alone (GB/s) and
     forward_norm against forward on the 2B4T gate shape (2560 -> 6912), PDL-chained graphs."""
@@ -676,6 +713,7 @@ def main():
     e2e_value = aggregate(step_bytes, dec["e2e_steps"], world, max_e2e) / 1e9
 
     pre = run_prefill(dev, args.prefill_iters, 3)
+    iso = run_isolated(dev)
     sweep = nm = norm = lut = None
     if not args.no_sweep:
         sweep = run_sweep(dev)
@@ -720,7 +758,10 @@ def main():
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": dec["h2d"],
                     "d2h_bytes_per_step": dec["d2h"], "steps": dec["e2e_steps"]},
             "gpu_launches": args.steps * dec["launches_per_step"], "clocks": dec["clocks"],
-            "hbm_frac": value / world / peaks["hbm_gbs"], "prefill": prefill}
+            "hbm_frac": value / world / peaks["hbm_gbs"], "prefill": prefill,
+            "isolated": {"workload": "one forward call at M=1 on a cold L2 (256 MB write before it), eager, "
+                                     "no PDL, CUDA events around the call (launch latency included); median of "
+                                     "30; bytes = N*K/4 + 4 + 2K + 2N", "cases": iso}}
     if sweep is not None:
         line["sweep"] = {"workload": "2B4T layer's 7 BitLinears (q,k,v,o 2560->2560/640, gate/up 2560->6912, "
                                      "down 6912->2560), ternary P(0)=0.42; per matrix a PDL-chained graph "

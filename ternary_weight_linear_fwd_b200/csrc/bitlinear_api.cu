@@ -251,7 +251,7 @@ auto quant_kernel(int G) {
 
 bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s,
                           const float* gnorm = nullptr, float eps = 0.0f) {
-  const QuantShape qs = quant_shape(K);
+  const QuantShape qs = quant_shape(M, K, gnorm != nullptr, plan_sm_count());
   const int wpr = qs.wpr;
   const int rows_per_cta = kQuantWarps / wpr;
   const int qblocks = (M + rows_per_cta - 1) / rows_per_cta;
@@ -738,7 +738,7 @@ bitlinear_status bitlinear_quant_act(const uint16_t* x, int32_t M, int32_t K, in
   DeviceState* dev = nullptr;
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
-  const QuantShape qs = quant_shape(K);
+  const QuantShape qs = quant_shape(M, K, false, plan_sm_count());
   const int wpr = qs.wpr;
   const int qblocks = (M + kQuantWarps / wpr - 1) / (kQuantWarps / wpr);
   st = launch(quant_kernel<false, false>(qs.G), dim3(qblocks), dim3(32 * kQuantWarps), 0,
@@ -760,7 +760,7 @@ bitlinear_status bitlinear_rmsnorm_quant_act(const uint16_t* x, int32_t M, int32
   DeviceState* dev = nullptr;
   bitlinear_status st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
-  const QuantShape qs = quant_shape(K);
+  const QuantShape qs = quant_shape(M, K, true, plan_sm_count());
   const int wpr = qs.wpr;
   const int qblocks = (M + kQuantWarps / wpr - 1) / (kQuantWarps / wpr);
   st = launch(quant_kernel<false, true>(qs.G), dim3(qblocks), dim3(32 * kQuantWarps), 0,

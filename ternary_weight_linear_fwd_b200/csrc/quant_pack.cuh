@@ -124,7 +124,11 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 // reads are in flight together.  quant_shape picks the smallest wpr that
 // leaves at most three groups per lane (short per-warp chains, many warps in
 // flight; the kernel is bound by latency, not by issue) and G, a compile-time
-// register count of 2, 3 or 8.  gamma is an integer warp max of the
+// register count of 2, 3 or 8.  With RMSNorm and enough rows to give every SM
+// a CTA of eight (M >= 8 * SMs), a row of up to 256 groups stays in one warp:
+// at M = 2048, K = 2560 that measured faster than two warps joined by the
+// barriers of the fp64 sum, the maximum and the code sum, while for a few rows
+// the shorter per-warp chains of the split win.  gamma is an integer warp max of the
 // |x| bit patterns (then across the row's warps), and the 16 codes of a group
 // come from the division-free exact rounding of codes8.  Longer or unaligned
 // rows take a two-pass loop (the second pass re-reads from L1/L2).
@@ -144,10 +148,11 @@ struct QuantShape {
   int G;    // k-groups per lane held in registers (template argument: 2, 3 or 8)
 };
 
-__host__ __device__ __forceinline__ QuantShape quant_shape(int K) {
+__host__ __device__ __forceinline__ QuantShape quant_shape(int M, int K, bool norm, int sm_count) {
   const int groups = (K + 15) / 16;
   int wpr = 1;
-  while (wpr < kQuantWarps && groups > 3 * 32 * wpr) wpr *= 2;
+  if (!(norm && groups <= 8 * 32 && M >= kQuantWarps * sm_count))
+    while (wpr < kQuantWarps && groups > 3 * 32 * wpr) wpr *= 2;
   const int need = (groups + 32 * wpr - 1) / (32 * wpr);
   return {wpr, need <= 2 ? 2 : need <= 3 ? 3 : 8};
 }
@@ -225,8 +230,10 @@ __device__ __forceinline__ float absmax8(const uint32_t (&w)[4], float mx) {
   return mx;
 }
 
+// Four CTAs per SM for G <= 3 (at most 64 registers a thread), so that one
+// wave holds 2048 tokens split over two warps each; two for G = 8.
 template <bool kPermute, bool kNorm, int G>
-__global__ void __launch_bounds__(32 * kQuantWarps) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
+__global__ void __launch_bounds__(32 * kQuantWarps, G <= 3 ? 4 : 2) quant_act_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                      int ldq, int8_t* __restrict__ q,
                                                                      float* __restrict__ gamma,
                                                                      int32_t* __restrict__ rowsum,

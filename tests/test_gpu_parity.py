@@ -350,6 +350,9 @@ def test_rmsnorm_quant_act_bit_exact(M, K):
 # half-filled last group), 2048 (2, 2), 4096 (4, 2), 16384 (8, 8 in registers),
 # 40008 (8, the streaming loop), each in natural order, with RMSNorm, and in
 # contraction order through the tensor-core forward with and without the norm.
+# (With the norm and at least eight rows per SM, rows of up to 256 groups stay
+# in one warp: test_rmsnorm_quant_act_bit_exact and test_forward_norm at
+# M = 2048 run that shape.)
 @pytest.mark.parametrize("K", [1536, 1544, 2048, 4096, 16384, 40008])
 def test_quant_every_launch_shape(K):
     M, N = 3, 40
@@ -375,7 +378,7 @@ def test_quant_every_launch_shape(K):
 
 
 @pytest.mark.parametrize("n,m", [(0, 0), (2, 4), (6, 8)])
-@pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (16, 1024, 300), (300, 512, 1000)])
+@pytest.mark.parametrize("M,K,N", [(1, 2560, 640), (16, 1024, 300), (300, 512, 1000), (2048, 2560, 96)])
 def test_forward_norm(n, m, M, K, N):
     x = synth.activations(M, K, seed=7 + M)
     W = synth.latent_weights(N, K, seed=7 + N)
