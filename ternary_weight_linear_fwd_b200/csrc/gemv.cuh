@@ -8,8 +8,8 @@
 // tile loads into shared memory, issued before griddepcontrol.wait, so under
 // programmatic dependent launch the copy overlaps the preceding kernel), then
 // quantises the single activation row into shared memory (gamma, codes in
-// contraction order, per-chunk code sums) while the copy lands, and finally
-// splits the (64-weight chunk, row) products evenly over all its threads.
+// contraction order, their sum) while the copy lands, and finally splits the
+// (64-weight chunk, row) products evenly over all its threads.
 // With code = W_t + 1:
 //     acc = sum_k q_k * W_t,k = sum_k q_k * code_k - sum_k q_k
 // where sum_k q_k is the same for every row (formed once, with the codes),
@@ -238,8 +238,8 @@ __device__ __forceinline__ void dot_word(uint32_t wd, uint32_t a0, uint32_t a1, 
 // (ch % 8) ^ (r % 8): lanes reading one chunk of consecutive rows never share
 // a bank.  The contraction is a flat list of (chunk, row pair) units, row pair
 // fastest, spread evenly over all threads; a unit is one 64-weight chunk of
-// two rows and adds its partial sums (minus the chunk's share of sum(q)) into
-// the rows' shared accumulators.
+// two rows and adds its partial sums of q * code into the rows' shared
+// accumulators, from which the store subtracts sum(q) once.
 
 __host__ __device__ __forceinline__ int gemv_stripes(int64_t ld) { return static_cast<int>((ld + 127) / 128); }
 __host__ __device__ __forceinline__ int gemv_stripe_bytes(int rows_box) { return (rows_box * 128 + 1023) & ~1023; }
