@@ -145,6 +145,29 @@ def test_forward_gemv_m1(M, K, N):
     _check_rows(x, Wt, a, y, acc, np.arange(M))
 
 
+# Decode GEMV row splits and chunk counts: 47 rows per CTA with an odd number
+# of 64-weight chunks (K = 2624), 64 rows with a ragged last chunk (K = 2600),
+# 64- and 65-row CTAs in one launch, 32 rows with a single chunk (K = 64), 94
+# rows (the grouped gate+up shape), and the RMSNorm variant on 2560 -> 6912.
+@pytest.mark.parametrize("K,N", [(2624, 6956), (2600, 9472), (2600, 9477), (64, 4736), (1024, 13912)])
+def test_forward_gemv_row_splits(K, N):
+    x, Wt, a, w = _dense_case(1, K, N, seed=K + 3 * N)
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+    assert bl.last_kernel() == "gemv_m1_dense"
+    _check_rows(x, Wt, a, y, acc, np.arange(1))
+
+
+def test_forward_norm_gemv_gate_shape():
+    K, N = 2560, 6912
+    x, Wt, a, w = _dense_case(1, K, N, seed=41)
+    g = _norm_weight(K, 5)
+    y, acc = bl.forward_norm(w, to_dev_bf16(x), torch.from_numpy(g).to(DEV), 1e-5, want_acc=True)
+    assert bl.last_kernel() == "gemv_m1_dense"
+    yo, acco, *_ = oracle.forward_norm(x, g, 1e-5, Wt, a)
+    np.testing.assert_array_equal(acc.cpu().numpy(), acco)
+    assert_bf16_close(bf16_bits(y), yo)
+
+
 @pytest.mark.parametrize("M,K,N", [(8, 256, 512), (2, 256, 512), (16, 2560, 640), (20, 203, 130), (300, 1000, 400),
                                    (1, 2560, 6912), (130, 384, 256), (64, 128, 128)])
 def test_forward_tc_full(M, K, N):
