@@ -18,6 +18,13 @@ A second object, "prefill", reports int8 TOPS of the tensor-core path on the
 2560 -> 2560, 2560 -> 640; latent W ~ N(0, 0.02), x with 1% x10 outliers),
 L2 flushed between iterations, counted as 2*M*N*K ops.
 
+Further objects on the same line (skipped with --no-sweep, except the
+last): "sweep" (the 7 BitLinears of a 2B4T layer at M = 1, 16, 256, 4096),
+"nm" (Sparse-BitNet 2:4 and 6:8 on the Qwen2.5-3B MLP shapes at M = 1 and
+4096), "norm" (RMSNorm fused into the activation quantisation), "decode_lut"
+(the lookup-table decode GEMV against the dp4a one) and "isolated" (one
+eager forward call at M = 1 on a cold L2, launch latency included).
+
 --impl reference times the oracle (plain C, one host core) on the same
 workload and metric.  Multi-GPU (torchrun) runs independent replicas: the
 path has no exchange step, per-GPU work is fixed, the time is the max over
