@@ -384,3 +384,55 @@ def test_quant_act_f32_matches_bf16_path_on_bf16_values():
     np.testing.assert_array_equal(q1, q2)
     np.testing.assert_array_equal(g1, g2)
     np.testing.assert_array_equal(r1, r2)
+
+
+# ---------------------------------------------------------------- N:M packed bytes, worked by hand
+
+def test_nm_packed_bytes_hand():
+    """Sparse-BitNet review, section 3.2 (top-n |W| per block of m along k, quant then mask), with the
+    I2_S 2-bit codes of the 2B4T report (section 5.1) and the layout: kept codes in increasing k,
+    LSB first, tail code 01; 2:4 meta a nibble i0 | i1 << 2 per block, low nibble first; n:8 meta
+    one bitmask byte per block.
+
+    2:4, W = (0.9, 0.1, 0.05, -0.8 | 0.02, 0.7, -0.6, 0.01): alpha = 3.18 / 8 = 0.3975, W / alpha
+    rounds to (1, 0, 0, -1 | 0, 1, -1, 0) (-0.6 / 0.3975 = -1.51 -> -2 -> -1).  Kept k = 0, 3 | 5, 6:
+    meta = 12 | 9 << 4 = 0x9C; codes (2, 0, 2, 0) -> 0x22.
+    3:8, W = (0.1, -0.5, 0.05, 0.3, -0.35, 0.2, 0.01, 0.45): alpha = 1.96 / 8 = 0.245, W_t =
+    (0, -1, 0, 1, -1, 1, 0, 1); kept k = 1, 4, 7 (|W| 0.5, 0.35, 0.45): meta 0b10010010 = 0x92;
+    codes (0, 0, 2) and one tail code 01 -> 0x60; the masked matrix drops W_t = 1 at k = 3 and 5."""
+    cases = (
+        ([0.9, 0.1, 0.05, -0.8, 0.02, 0.7, -0.6, 0.01], 2, 4, 0.3975, [1, 0, 0, -1, 0, 1, -1, 0], 0x22, 0x9C,
+         [1, 0, 0, -1, 0, 1, -1, 0]),
+        ([0.1, -0.5, 0.05, 0.3, -0.35, 0.2, 0.01, 0.45], 3, 8, 0.245, [0, -1, 0, 1, -1, 1, 0, 1], 0x60, 0x92,
+         [0, -1, 0, 0, -1, 0, 0, 1]),
+    )
+    for w, n, m, alpha, wt, vbyte, mbyte, weff in cases:
+        W = np.array([w], np.float32)
+        p = oracle.pack_weights(W, n, m)
+        assert p["alpha"] == np.float32(alpha)
+        np.testing.assert_array_equal(oracle.ternarize(W, p["alpha"])[0], wt)
+        np.testing.assert_array_equal(p["Wt"][0], weff)
+        assert p["values"].shape == (1, 16) and p["meta"].shape == (1, 16)
+        assert int(p["values"][0, 0]) == vbyte and int(p["meta"][0, 0]) == mbyte
+        assert (p["values"][0, 1:] == 0x55).all()  # tail codes 01
+
+
+# ---------------------------------------------------------------- RMSNorm composed with the forward
+
+def test_forward_norm_reduces_to_forward_on_unit_rows():
+    """Rows of +-1 have mean square 1, so with g = 1 and eps = 0 the normalised row is the row itself
+    and forward_norm equals forward bit for bit; with g = 2 every xn doubles, the codes stay and gamma
+    doubles, so y doubles exactly (a rescale that used gamma of x instead of xn would not)."""
+    M, K, N = 4, 128, 96
+    signs = np.where(synth.uniform(31, 3, M * K) < 0.5, -1.0, 1.0).reshape(M, K).astype(np.float32)
+    x = synth.to_bf16_bits(signs)
+    W = synth.latent_weights(N, K, seed=31)
+    p = oracle.pack_weights(W)
+    y0, acc0, *_ = oracle.forward(x, p["Wt"], p["alpha"])
+    y1, acc1, *_ = oracle.forward_norm(x, np.ones(K, np.float32), 0.0, p["Wt"], p["alpha"])
+    np.testing.assert_array_equal(acc1, acc0)
+    np.testing.assert_array_equal(y1, y0)
+    y2, acc2, *_ = oracle.forward_norm(x, np.full(K, 2.0, np.float32), 0.0, p["Wt"], p["alpha"])
+    np.testing.assert_array_equal(acc2, acc0)
+    np.testing.assert_array_equal(synth.bf16_bits_to_f32(y2), 2.0 * synth.bf16_bits_to_f32(y0))
+    assert np.abs(acc0).max() > 0
