@@ -95,6 +95,22 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _check_out(t, shape, dtype, device, what: str):
+    """A caller-supplied output must be a contiguous tensor of exactly the shape, dtype and device the
+    kernels write: they take only its address, so anything smaller would be overrun."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{what}: expected a contiguous {dtype} tensor of shape {tuple(shape)} on {device}, "
+                         f"got {tuple(t.shape)} {t.dtype} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _check_workspace(t, device):
+    if t is not None and (t.device != device or not t.is_contiguous()):
+        raise ValueError(f"workspace: expected a contiguous tensor on {device}, got one on {t.device}")
+
+
 def packed_layout(N: int, K: int, n: int = 0, m: int = 0):
     """(ld_codes, ld_meta, codes_bytes, meta_bytes) of the packed layout."""
     a, b = ctypes.c_int64(), ctypes.c_int64()
@@ -189,6 +205,9 @@ def _forward(fn, what, w: PackedWeights, x, want_acc, flags, workspace, out, acc
     import torch
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w.K
     M = x.shape[0]
+    _check_out(out, (M, w.N), torch.bfloat16, x.device, "out")
+    _check_out(acc_out, (M, w.N), torch.int32, x.device, "acc_out")
+    _check_workspace(workspace, x.device)
     y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
     acc = acc_out if acc_out is not None else (
         torch.empty((M, w.N), dtype=torch.int32, device=x.device) if want_acc else None)
@@ -221,6 +240,12 @@ def forward_group(ws, x, want_acc: bool = False, flags: int = 0, workspace=None,
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
     count = len(ws)
     M = x.shape[0]
+    if outs is not None:
+        if len(outs) != count:
+            raise ValueError(f"forward_group: {count} matrices but {len(outs)} outputs")
+        for i, (o, w) in enumerate(zip(outs, ws)):
+            _check_out(o, (M, w.N), torch.bfloat16, x.device, f"outs[{i}]")
+    _check_workspace(workspace, x.device)
     ys = outs if outs is not None else [torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device) for w in ws]
     accs = [torch.empty((M, w.N), dtype=torch.int32, device=x.device) for w in ws] if want_acc else None
     need = max((forward_workspace_bytes(M, w.N, w.K, flags) for w in ws), default=0)
@@ -242,6 +267,9 @@ def forward_norm(w: PackedWeights, x, g, eps: float, want_acc: bool = False, fla
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w.K
     assert g.is_cuda and g.dtype == torch.float32 and g.is_contiguous() and g.numel() == w.K
     M = x.shape[0]
+    _check_out(out, (M, w.N), torch.bfloat16, x.device, "out")
+    _check_out(acc_out, (M, w.N), torch.int32, x.device, "acc_out")
+    _check_workspace(workspace, x.device)
     y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
     acc = acc_out if acc_out is not None else (
         torch.empty((M, w.N), dtype=torch.int32, device=x.device) if want_acc else None)
@@ -285,6 +313,8 @@ def forward_noalloc(w: PackedWeights, x, out=None, acc_out=None, want_acc: bool 
                        ctypes.c_uint32, ctypes.c_void_p]
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w.K
     M = x.shape[0]
+    _check_out(out, (M, w.N), torch.bfloat16, x.device, "out")
+    _check_out(acc_out, (M, w.N), torch.int32, x.device, "acc_out")
     y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
     acc = acc_out if acc_out is not None else (
         torch.empty((M, w.N), dtype=torch.int32, device=x.device) if want_acc else None)

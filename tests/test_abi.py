@@ -158,3 +158,27 @@ def test_rmsnorm_entry_points_host_checks(L):
     assert fn(ctypes.byref(w), x, 1, g, 2.0, y, None, None, 0, 0, None) == 2
     assert fn(ctypes.byref(w), x, 1, g, 1e-6, y, None, None, 0, 0x2, None) == 8   # the GEMV path is not offered
     assert fn(ctypes.byref(_w(L, codes=0x10008)), x, 1, g, 1e-6, y, None, None, 0, 0, None) == 3
+
+
+def test_binding_rejects_bad_outputs():
+    """Caller-supplied outputs must have exactly the shape, dtype and device the kernels write (they
+    receive only an address); the checks run before any library call, so CPU tensors exercise them."""
+    torch = pytest.importorskip("torch")
+    import ternary_weight_linear_fwd_b200 as bl
+    dev = torch.device("cpu")
+    good = torch.empty((3, 5), dtype=torch.bfloat16)
+    bl._check_out(good, (3, 5), torch.bfloat16, dev, "out")
+    bl._check_out(None, (3, 5), torch.bfloat16, dev, "out")
+    bad = [torch.empty((3, 4), dtype=torch.bfloat16),            # too narrow: would be overrun
+           torch.empty((2, 5), dtype=torch.bfloat16),            # too few rows
+           torch.empty((3, 5), dtype=torch.float32),             # wrong dtype
+           torch.empty((5, 3), dtype=torch.bfloat16).t(),        # right shape, not contiguous
+           torch.empty((3, 10), dtype=torch.bfloat16)[:, ::2]]   # strided view
+    for t in bad:
+        with pytest.raises(ValueError):
+            bl._check_out(t, (3, 5), torch.bfloat16, dev, "out")
+    with pytest.raises(ValueError):
+        bl._check_out(good, (3, 5), torch.bfloat16, torch.device("meta"), "out")
+    bl._check_workspace(torch.empty(64, dtype=torch.uint8), dev)
+    with pytest.raises(ValueError):
+        bl._check_workspace(torch.empty((8, 16), dtype=torch.uint8)[:, ::2], dev)
