@@ -77,6 +77,7 @@ typedef enum bitlinear_status {
 } bitlinear_status;
 
 /* Limits checked by every call. */
+#define BITLINEAR_LAYOUT_VERSION 1
 #define BITLINEAR_MAX_K 65536       /* keeps every int32 partial sum exact */
 #define BITLINEAR_MAX_N (1 << 24)
 #define BITLINEAR_MAX_M (1 << 24)
@@ -276,8 +277,16 @@ bitlinear_status bitlinear_forward_noalloc(const bitlinear_weights* w, const uin
 bitlinear_status bitlinear_device_status(void* stream, int32_t* code, int32_t clear);
 
 /* Name of the kernel variant the last successful call on this host thread
- * enqueued (a static string; "" before the first call). */
+ * enqueued (a static string; "" before the first call).  With the environment
+ * variable BITLINEAR_LOG set to a non-empty value other than "0" when the
+ * library is first used, every such call also writes "bitlinear: <name>" on
+ * a line of stderr. */
 const char* bitlinear_last_kernel(void);
+
+/* BITLINEAR_LAYOUT_VERSION of the compiled library: the version of the packed
+ * layouts described at the top of this header.  Buffers packed under another
+ * version must be packed again from the latent (or ternary) weights. */
+int32_t bitlinear_layout_version(void);
 
 /* Human-readable name of a status code (static string). */
 const char* bitlinear_status_string(bitlinear_status s);

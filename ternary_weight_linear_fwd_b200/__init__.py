@@ -15,7 +15,7 @@ from typing import Optional
 __all__ = [
     "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
     "quant_act", "rmsnorm_quant_act", "forward", "forward_nm", "forward_group", "forward_norm",
-    "forward_workspace_bytes", "device_status", "last_kernel",
+    "forward_workspace_bytes", "device_status", "last_kernel", "layout_version",
     "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT",
 ]
 
@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "bitlinear_forward_norm": (st, [ctypes.POINTER(_Weights), P, i32, P, ctypes.c_float, P, P, P, sz, u32, P]),
             "bitlinear_device_status": (st, [P, ctypes.POINTER(i32), i32]),
             "bitlinear_last_kernel": (ctypes.c_char_p, []),
+            "bitlinear_layout_version": (i32, []),
             "bitlinear_status_string": (ctypes.c_char_p, [st]),
         }
         for name, (res, args) in sig.items():
@@ -291,6 +292,11 @@ def device_status(clear: bool = True, stream=None) -> int:
 
 def last_kernel() -> str:
     return lib().bitlinear_last_kernel().decode()
+
+
+def layout_version() -> int:
+    """Version of the packed weight layouts the library reads and writes."""
+    return int(lib().bitlinear_layout_version())
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

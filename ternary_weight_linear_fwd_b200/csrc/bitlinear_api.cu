@@ -8,6 +8,8 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -20,7 +22,26 @@ __device__ int32_t g_device_status;
 
 namespace {
 
-thread_local const char* t_last_kernel = "";
+// The kernel variant of the last successful call on this thread; assigning it
+// also logs the name to stderr when BITLINEAR_LOG is set (read once).
+bool log_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("BITLINEAR_LOG");
+    return v != nullptr && v[0] != '\0' && std::strcmp(v, "0") != 0;
+  }();
+  return on;
+}
+
+struct LastKernel {
+  const char* name = "";
+  LastKernel& operator=(const char* n) {
+    name = n;
+    if (log_enabled()) std::fprintf(stderr, "bitlinear: %s\n", n);
+    return *this;
+  }
+};
+
+thread_local LastKernel t_last_kernel;
 
 constexpr int kMaxDevices = 64;
 
@@ -836,7 +857,9 @@ bitlinear_status bitlinear_device_status(void* stream, int32_t* code, int32_t cl
   return BITLINEAR_OK;
 }
 
-const char* bitlinear_last_kernel(void) { return t_last_kernel; }
+const char* bitlinear_last_kernel(void) { return t_last_kernel.name; }
+
+int32_t bitlinear_layout_version(void) { return BITLINEAR_LAYOUT_VERSION; }
 
 const char* bitlinear_status_string(bitlinear_status s) {
   switch (s) {

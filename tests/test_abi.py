@@ -182,3 +182,12 @@ def test_binding_rejects_bad_outputs():
     bl._check_workspace(torch.empty(64, dtype=torch.uint8), dev)
     with pytest.raises(ValueError):
         bl._check_workspace(torch.empty((8, 16), dtype=torch.uint8)[:, ::2], dev)
+
+
+def test_layout_version_matches_header(L):
+    m = re.search(r"#define BITLINEAR_LAYOUT_VERSION (\d+)", open(HEADER).read())
+    assert m is not None
+    L.bitlinear_layout_version.restype = ctypes.c_int32
+    assert L.bitlinear_layout_version() == int(m.group(1))
+    import ternary_weight_linear_fwd_b200 as bl
+    assert bl.layout_version() == int(m.group(1))
