@@ -64,6 +64,10 @@ def _load():
             "orc_matmul_i32": (i32, [P, P, i32, i32, i32, P]),
             "orc_dequant": (None, [P, P, f32, i32, i32, i32, P]),
             "orc_bf16_from_f64": (ctypes.c_uint16, [ctypes.c_double]),
+            "orc_hadamard_block": (i32, [i32]),
+            "orc_hadamard_rows": (None, [P, i32, i32, i32, P]),
+            "orc_quant_act4": (None, [P, i32, i32, P, P, P]),
+            "orc_forward_hbit": (i32, [P, i32, i32, P, i32, f32, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -249,3 +253,51 @@ def pack_weights(W: np.ndarray, n: int = 0, m: int = 0):
     Weff = apply_mask(Wt, mask)
     vals, meta = pack_nm(Weff, mask, n, m)
     return {"alpha": alpha, "Wt": Weff, "values": vals, "meta": meta, "mask": mask}
+
+
+# ---------------------------------------------------------------- H-BitLinear (BitNet v2 section of the blog)
+
+def hadamard_block(K: int) -> int:
+    """Size of the Hadamard blocks along K: the largest power of two dividing K."""
+    return int(_load().orc_hadamard_block(int(K)))
+
+
+def hadamard(x_bf16: np.ndarray, B: int = None) -> np.ndarray:
+    """fp32 [M, K]: each B-block of each bf16 row times the orthonormal Sylvester
+    Hadamard matrix (fast butterflies in fp32, then one multiply by RN32(1/sqrt(B)))."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    if B is None:
+        B = hadamard_block(K)
+    assert B >= 1 and (B & (B - 1)) == 0 and K % B == 0
+    xh = np.empty((M, K), dtype=np.float32)
+    _load().orc_hadamard_rows(_ptr(x), M, K, int(B), _ptr(xh))
+    return xh
+
+
+def quant_act4(xh: np.ndarray):
+    """(q int8 in [-8, 7], gamma fp32 [M], rowsum int32 [M]) of fp32 rows, Q_b = 7."""
+    xh = np.ascontiguousarray(xh, dtype=np.float32)
+    M, K = xh.shape
+    q = np.empty((M, K), dtype=np.int8)
+    g = np.empty(M, dtype=np.float32)
+    rs = np.empty(M, dtype=np.int32)
+    _load().orc_quant_act4(_ptr(xh), M, K, _ptr(q), _ptr(g), _ptr(rs))
+    return q, g, rs
+
+
+def forward_hbit(x_bf16: np.ndarray, Wt: np.ndarray, alpha):
+    """H-BitLinear: Hadamard transform, 4-bit codes, ternary contraction, y = acc * alpha * gamma / 7.
+    Returns (y bf16 bits, acc, q, gamma)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    Wt = np.ascontiguousarray(Wt, dtype=np.int8)
+    M, K = x.shape
+    N = Wt.shape[0]
+    y = np.empty((M, N), dtype=np.uint16)
+    q = np.empty((M, K), dtype=np.int8)
+    acc = np.empty((M, N), dtype=np.int32)
+    g = np.empty(M, dtype=np.float32)
+    if _load().orc_forward_hbit(_ptr(x), M, K, _ptr(Wt), N, float(np.float32(alpha)), _ptr(y), _ptr(q), _ptr(acc),
+                                _ptr(g)) != 0:
+        raise OverflowError("accumulator left int32")
+    return y, acc, q, g

@@ -45,6 +45,20 @@
  *    quantisation.  eps is a parameter (the page's nn.RMSNorm leaves it to
  *    the dtype's default).
  *
+ *  - H-BitLinear ("BitNet 1-Bit LLM" blog, section on BitNet v2: an online
+ *    Hadamard transform of the activations, then 4-bit activation
+ *    quantisation, then the ternary linear map).  The pages give neither the
+ *    transform's size, normalisation or evaluation order nor the 4-bit
+ *    quantiser, so: the Sylvester-order Walsh-Hadamard matrix of size B = the
+ *    largest power of two dividing K, applied to each of the K / B blocks of
+ *    a row; evaluated in fp32 by the in-place fast transform (stages
+ *    h = 1, 2, 4, ..., B/2, each pair (j, j + h) with bit h of j clear becomes
+ *    (a + b, a - b), one fp32 rounding per sum), then scaled by one fp32
+ *    multiply with RN32(1 / sqrt(B)) so the transform is orthonormal; 4-bit
+ *    codes by the absmax formula with Q_b = 7 clamped to [-8, 7]; the weights
+ *    are the ternary matrix of the rotated-basis latent weights (the
+ *    transform is not applied to them at run time).
+ *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math
  */
 #include <fenv.h>
@@ -386,6 +400,95 @@ int orc_forward(const uint16_t* x, int M, int K, const int8_t* Wt, int N, float 
         rc = orc_matmul_i32(q, Wt, M, N, K, acc);
         orc_dequant(acc, g, alpha, M, N, Qb, y);
     }
+    if (!q_out) free(q);
+    if (!acc_out) free(acc);
+    if (!gamma_out) free(g);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* H-BitLinear: online Hadamard transform, 4-bit activations ("BitNet 1-Bit  */
+/* LLM" blog, BitNet v2 section)                                             */
+/* ------------------------------------------------------------------------ */
+
+/* Largest power of two that divides K (1 for odd K). */
+int orc_hadamard_block(int K) {
+    int b = 1;
+    while (K % (2 * b) == 0) b *= 2;
+    return b;
+}
+
+/* xh = RN32(1 / sqrt(B)) * H_B x on every B-block of every bf16 row, with the
+ * unnormalised transform formed by the in-place fast Walsh-Hadamard butterflies
+ * in fp32 (stage h = 1, 2, ..., B/2: (a, b) -> (a + b, a - b) for j with
+ * bit h clear and its partner j + h). */
+void orc_hadamard_rows(const uint16_t* x, int M, int K, int B, float* xh) {
+    fesetround(FE_TONEAREST);
+    const float scale = (float)(1.0 / sqrt((double)B));
+    for (int r = 0; r < M; ++r) {
+        float* row = xh + (int64_t)r * K;
+        for (int k = 0; k < K; ++k) row[k] = orc_bf16_to_f32(x[(int64_t)r * K + k]);
+        for (int b0 = 0; b0 < K; b0 += B) {
+            float* v = row + b0;
+            for (int h = 1; h < B; h *= 2)
+                for (int j = 0; j < B; ++j)
+                    if ((j & h) == 0) {
+                        volatile float a = v[j], b = v[j + h];
+                        volatile float s = a + b, d = a - b;
+                        v[j] = s;
+                        v[j + h] = d;
+                    }
+            for (int j = 0; j < B; ++j) {
+                volatile float t = v[j] * scale;
+                v[j] = t;
+            }
+        }
+    }
+}
+
+/* 4-bit activation codes of fp32 rows: gamma = max |xh|,
+ * q = clamp(rne(RN(xh * 7) / RN(gamma + eps)), -8, 7). */
+void orc_quant_act4(const float* xh, int M, int K, int8_t* q, float* gamma, int32_t* rowsum) {
+    fesetround(FE_TONEAREST);
+    for (int r = 0; r < M; ++r) {
+        const float* xr = xh + (int64_t)r * K;
+        float g = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(xr[k]);
+            if (a > g) g = a;
+        }
+        gamma[r] = g;
+        volatile float d = g + ORC_EPS;
+        int64_t s = 0;
+        for (int k = 0; k < K; ++k) {
+            volatile float t = xr[k] * 7.0f;
+            volatile float v = t / d;
+            float c = nearbyintf(v);
+            if (c > 7.0f) c = 7.0f;
+            if (c < -8.0f) c = -8.0f;
+            q[(int64_t)r * K + k] = (int8_t)c;
+            s += (int64_t)c;
+        }
+        if (rowsum) rowsum[r] = (int32_t)s;
+    }
+}
+
+/* H-BitLinear forward: transform, 4-bit codes, contraction with the ternary
+ * matrix, y = acc * alpha * gamma / 7 in fp64 rounded once to bf16. */
+int orc_forward_hbit(const uint16_t* x, int M, int K, const int8_t* Wt, int N, float alpha, uint16_t* y,
+                     int8_t* q_out, int32_t* acc_out, float* gamma_out) {
+    float* xh = (float*)malloc((size_t)M * (size_t)K * sizeof(float));
+    int8_t* q = q_out ? q_out : (int8_t*)malloc((size_t)M * (size_t)K);
+    int32_t* acc = acc_out ? acc_out : (int32_t*)malloc((size_t)M * (size_t)N * sizeof(int32_t));
+    float* g = gamma_out ? gamma_out : (float*)malloc((size_t)M * sizeof(float));
+    int rc = -1;
+    if (xh && q && acc && g) {
+        orc_hadamard_rows(x, M, K, orc_hadamard_block(K), xh);
+        orc_quant_act4(xh, M, K, q, g, NULL);
+        rc = orc_matmul_i32(q, Wt, M, N, K, acc);
+        orc_dequant(acc, g, alpha, M, N, 7, y);
+    }
+    free(xh);
     if (!q_out) free(q);
     if (!acc_out) free(acc);
     if (!gamma_out) free(g);
