@@ -51,7 +51,7 @@ FFN = (("gate", 2560, 6912), ("up", 2560, 6912), ("down", 6912, 2560))  # (name,
 PREFILL_SHAPES = ((2560, 6912), (6912, 2560), (2560, 2560), (2560, 640))  # (K, N)
 PREFILL_M = 2048
 DISTINCT_LAYERS = 2  # distinct weight draws, replicated to 30 layers at distinct addresses
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_dense__decode_2b4t_ffn.md")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "gemv_dense__decode_2b4t_ffn.json")
 GEMV_SOURCES = ("gemv.cuh", "quant_pack.cuh", "ptx.cuh")
 
 
@@ -203,20 +203,17 @@ def gemv_source_hash() -> str:
 
 
 def profiled_traffic():
-    """DRAM bytes per GEMV launch from the committed ncu summary, if it matches today's kernel source."""
-    if not os.path.exists(PROFILE_SUMMARY):
+    """DRAM bytes per GEMV launch from the committed ncu figures (profiles/*.json), if they were taken on
+    today's kernel source (same fingerprint of the definitions in GEMV_DEFS)."""
+    if not os.path.exists(PROFILE_TRAFFIC):
         return None
-    vals = {}
-    with open(PROFILE_SUMMARY) as f:
-        for line in f:
-            if ":" in line and line.startswith("- "):
-                k, _, v = line[2:].partition(":")
-                vals[k.strip()] = v.strip().strip("`")
+    with open(PROFILE_TRAFFIC) as f:
+        d = json.load(f)
+    if d.get("source_sha256_16") != gemv_source_hash():
+        return None
     try:
-        if vals.get("source_sha256_16") != gemv_source_hash():
-            return None
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return float(d["dram_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -344,8 +341,32 @@ def run_decode(dev, steps, warmup, layers, clock_index):
     h2d = (x_in.numel() + h_in.numel()) * 2
     d2h = (y_gate.numel() + y_up.numel() + y_down.numel()) * 2
     del g
+
+    # the same, issued call by call (no graph): the per-call host path of the binding and the C ABI
+    def e2e_eager_step():
+        x_in.copy_(h_x, non_blocking=True)
+        h_in.copy_(h_h, non_blocking=True)
+        step()
+        o_g.copy_(y_gate, non_blocking=True)
+        o_u.copy_(y_up, non_blocking=True)
+        o_d.copy_(y_down, non_blocking=True)
+
+    for _ in range(max(3, warmup)):
+        e2e_eager_step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    eager_steps = max(1, min(steps, 200))
+    e0.record(s)
+    for _ in range(eager_steps):
+        e2e_eager_step()
+    e1.record(s)
+    e1.synchronize()
+    eager_secs = e0.elapsed_time(e1) / 1e3
+    barrier(dev)
     return {"secs": secs, "clocks": clocks, "launches_per_step": launches_per_step, "e2e_secs": e2e_secs,
-            "e2e_steps": e_steps, "h2d": h2d, "d2h": d2h}
+            "e2e_steps": e_steps, "h2d": h2d, "d2h": d2h, "e2e_eager_steps": eager_steps,
+            "e2e_eager_ms": eager_secs / eager_steps * 1e3,
+            "e2e_eager_gbps": decode_step_bytes(layers) * eager_steps / eager_secs / 1e9}
 
 
 def run_prefill(dev, iters: int, warmup: int):
@@ -612,6 +633,25 @@ def run_norm(dev, warmup: int = 3, reps: int = 5, calls: int = 16):
 
 # ------------------------------------------------------------------ oracle (CPU) legs
 
+def host_cpu():
+    """CPU model, threads the system reports online, and threads this process may run on."""
+    import oracle
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count() or 1
+    return {"model": model, "online_cpus": oracle.online_cpus(), "usable_threads": usable}
+
+
 def oracle_decode_setup(seed: int = 1):
     from ternary_weight_linear_fwd_b200 import synth
     mats = []
@@ -622,7 +662,7 @@ def oracle_decode_setup(seed: int = 1):
     return mats, x, h
 
 
-def oracle_decode_pass(setup, frac: float = 1.0):
+def oracle_decode_pass(setup, frac: float = 1.0, threads: int = 1):
     """Oracle forward (quantise, contract, dequantise) of one FFN layer at M = 1, on the first
     `frac` of each matrix's output rows.  Returns (algorithmic bytes, seconds)."""
     import oracle
@@ -630,19 +670,102 @@ def oracle_decode_pass(setup, frac: float = 1.0):
     nbytes, t0 = 0, time.perf_counter()
     for T, a, K, N in mats:
         rows = max(1, int(round(N * frac)))
-        oracle.forward(x if K == 2560 else h, T[:rows], a)
+        oracle.forward(x if K == 2560 else h, T[:rows], a, threads=threads)
         nbytes += decode_bytes_per_gemv(K, rows)
     return nbytes, time.perf_counter() - t0
 
 
-def oracle_decode_sample(seconds: float, seed: int = 1):
+def oracle_decode_sample(seconds: float, threads: int, setup=None, seed: int = 1):
     """Repeats full-layer oracle passes until `seconds` pass; returns (GB/s, passes, seconds)."""
-    setup = oracle_decode_setup(seed)
+    setup = setup or oracle_decode_setup(seed)
     n, tot_b, tot_s = 0, 0, 0.0
     while tot_s < seconds:
-        b, sec = oracle_decode_pass(setup)
+        b, sec = oracle_decode_pass(setup, threads=threads)
         n, tot_b, tot_s = n + 1, tot_b + b, tot_s + sec
     return tot_b / tot_s / 1e9, n, tot_s
+
+
+ORACLE_SLICE = 64  # tokens the oracle runs for the many-token workloads (time scaled linearly in M)
+
+
+def _oracle_tokens(x_bits, Wt, alpha, threads):
+    """Seconds of one oracle forward (quantise, contract, dequantise) of the given tokens."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward(x_bits, Wt, alpha, threads=threads)
+    return time.perf_counter() - t0
+
+
+def run_cpu_baselines(decode_seconds: float, threads: int, with_sweep: bool):
+    """The oracle, as it stands, on the host: the decode workload on one core and on `threads` cores, the
+    prefill shapes, and (with_sweep) the layer sweep and the N:M shapes.  Many-token workloads run a
+    slice of ORACLE_SLICE tokens and scale the time linearly to the full M (stated in each object)."""
+    import numpy as np
+
+    import oracle
+    from ternary_weight_linear_fwd_b200 import synth
+    cpu = host_cpu()
+    setup = oracle_decode_setup()
+    v1, n1, s1 = oracle_decode_sample(decode_seconds / 2, 1, setup)
+    vt, nt, st = oracle_decode_sample(decode_seconds / 2, threads, setup)
+    out = {"host": cpu, "decode": {
+        "single_core": {"value": v1, "unit": "GB/s", "cores": 1, "passes": n1, "seconds": s1},
+        "all_cores": {"value": vt, "unit": "GB/s", "cores": threads, "passes": nt, "seconds": st}}}
+
+    def many_tokens(mats, M, seed):
+        """mats: (key, K, N, Wt, alpha).  Per matrix the scaled oracle time of M tokens."""
+        res, ops_tot, sec_tot = {}, 0.0, 0.0
+        for key, K, N, Wt, alpha in mats:
+            rows = min(M, ORACLE_SLICE)
+            x = synth.activations(rows, K, seed=seed)
+            sec = _oracle_tokens(x, Wt, alpha, threads) * M / rows
+            ops = 2.0 * M * N * K
+            res[key] = {"ms_scaled": sec * 1e3, "TOPS": ops / sec / 1e12,
+                        "GBps": (N * K // 4 + 4 + 2 * M * K + 2 * M * N) / sec / 1e9}
+            ops_tot, sec_tot = ops_tot + ops, sec_tot + sec
+        return res, ops_tot, sec_tot
+
+    mats = []
+    for K, N in PREFILL_SHAPES:
+        r = oracle.pack_weights(synth.latent_weights(N, K, seed=3))
+        mats.append((f"{K}x{N}", K, N, r["Wt"], r["alpha"]))
+    res, ops, sec = many_tokens(mats, PREFILL_M, 3)
+    del mats
+    out["prefill"] = {"value": ops / sec / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                      "shapes": res,
+                      "sample": f"oracle forward of {ORACLE_SLICE} of the {PREFILL_M} tokens per shape on "
+                                f"{threads} threads, time scaled linearly to {PREFILL_M} tokens"}
+    if with_sweep:
+        layer = []
+        for i, (name, (K, N)) in enumerate(synth.B2B4T_LAYER.items()):
+            layer.append((name, K, N, synth.ternary_weights(N, K, seed=4 + 10 * i),
+                          np.float32(synth.alpha_uniform(4 + 10 * i))))
+        sweep = {}
+        for M in SWEEP_M:
+            res, ops, sec = many_tokens(layer, M, 4)
+            nbytes = sum(N * K // 4 + 4 + 2 * M * K + 2 * M * N for _, K, N, _, _ in layer)
+            sweep[f"M={M}"] = {"layer_us_scaled": sec * 1e6, "GBps": nbytes / sec / 1e9, "TOPS": ops / sec / 1e12,
+                               "tokens_run": min(M, ORACLE_SLICE), "matrices": res}
+        del layer
+        out["sweep"] = {"cores": threads, "kind": "oracle", "by_M": sweep,
+                        "sample": f"oracle forward of min(M, {ORACLE_SLICE}) tokens through the 7 matrices on "
+                                  f"{threads} threads, time scaled linearly to M"}
+        nm = {}
+        for n, m in NM_PATTERNS:
+            for name, (K, N) in synth.QWEN25_3B_MLP.items():
+                r = oracle.pack_weights(synth.latent_weights(N, K, seed=5), n, m)
+                nbytes_w = r["values"].size + r["meta"].size
+                for M in NM_M:
+                    rows = min(M, ORACLE_SLICE)
+                    x = synth.activations(rows, K, seed=5)
+                    sec = _oracle_tokens(x, r["Wt"], r["alpha"], threads) * M / rows
+                    nm[f"{n}:{m} {name} {K}->{N} M={M}"] = {
+                        "us_scaled": sec * 1e6, "GBps": (nbytes_w + 4 + 2 * M * K + 2 * M * N) / sec / 1e9,
+                        "TOPS_dense_equiv": 2.0 * M * N * K / sec / 1e12, "tokens_run": rows}
+        out["nm"] = {"cores": threads, "kind": "oracle", "cases": nm,
+                     "sample": f"oracle forward (the masked ternary matrix, dense loop) of min(M, {ORACLE_SLICE}) "
+                               f"tokens on {threads} threads, time scaled linearly to M"}
+    return out
 
 
 # ------------------------------------------------------------------ main
@@ -673,26 +796,30 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
+        threads = host_cpu()["usable_threads"]
         setup = oracle_decode_setup()
-        full_b, full_s = oracle_decode_pass(setup)
+        full_b, full_s = oracle_decode_pass(setup, threads=threads)
         # a bounded sample per step: the whole run stays near two minutes of host time
         frac = min(1.0, (120.0 / (args.steps + args.warmup)) / full_s)
         for _ in range(args.warmup):
-            oracle_decode_pass(setup, frac)
+            oracle_decode_pass(setup, frac, threads)
         tot_b, tot_s, vals = 0, 0.0, []
         for _ in range(args.steps):
-            b, sec = oracle_decode_pass(setup, frac)
+            b, sec = oracle_decode_pass(setup, frac, threads)
             tot_b, tot_s = tot_b + b, tot_s + sec
             vals.append(b / sec / 1e9)
         v = tot_b / tot_s / 1e9
-        sample = (f"oracle forward (plain C, 1 thread): per step one FFN layer (gate, up, down at M=1) "
-                  f"restricted to the first {frac:.4f} of each matrix's output rows; GB/s on the same "
-                  f"algorithmic bytes (packed codes + alpha + x + y)")
+        cpu = host_cpu()
+        sample = (f"oracle forward (plain C; contraction over {threads} threads): per step one FFN layer (gate, "
+                  f"up, down at M=1) restricted to the first {frac:.4f} of each matrix's output rows; GB/s on "
+                  f"the same algorithmic bytes (packed codes + alpha + x + y); host {cpu['model']}, "
+                  f"{cpu['online_cpus']} threads online")
         line = {"metric": METRIC, "impl": "reference", "value": v, "unit": "GB/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "int8 x ternary -> int32 (bf16 in/out)", "data": "synthetic", "config": config,
-                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample,
+                                 "host": cpu},
                 "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -752,18 +879,32 @@ def main():
                "roofline": {"bound": "tensor", "achieved": pre["tops"], "peak": int8_peak, "unit": "TOPS",
                             "frac": pre["tops"] / int8_peak,
                             "peak_source": f"{peak_kind} bf16_tflops x 2 (int8/bf16 nominal ratio)"}}
-    cpu = None
+    cpu = cpu_all = None
     if not args.no_cpu_baseline:
-        v, n, el = oracle_decode_sample(args.cpu_seconds)
-        cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"oracle forward (plain C, 1 thread) on one FFN layer (gate, up, down at M=1), "
-                         f"{n} repetitions in {el:.1f} s"}
+        threads = host_cpu()["usable_threads"]
+        cpu_all = run_cpu_baselines(args.cpu_seconds, threads, sweep is not None)
+        d = cpu_all["decode"]
+        h = cpu_all["host"]
+        cpu = {"value": d["all_cores"]["value"], "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"oracle forward (plain C; contraction over {threads} threads, quantisation and rescale "
+                         f"on one) on one FFN layer (gate, up, down at M=1), {d['all_cores']['passes']} passes "
+                         f"in {d['all_cores']['seconds']:.1f} s; host {h['model']}, {h['online_cpus']} threads "
+                         f"online",
+               "single_core": d["single_core"], "host": h}
+        prefill["cpu_baseline"] = cpu_all["prefill"]
+    e2e = {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": dec["h2d"],
+           "d2h_bytes_per_step": dec["d2h"], "steps": dec["e2e_steps"],
+           "how": "each step: pinned-host copies of every layer's inputs, the captured decode step (CUDA graph "
+                  "of the public-API calls), copies of every output back",
+           "eager": {"value": dec["e2e_eager_gbps"], "unit": "GB/s", "steps": dec["e2e_eager_steps"],
+                     "ms_per_step": dec["e2e_eager_ms"],
+                     "how": "the same step issued call by call through the Python binding and the C ABI "
+                            "(argument checks, cached tensor maps, 60 launches), no graph"}}
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_secs / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8 x ternary -> int32 (bf16 in/out)",
             "data": "synthetic", "config": config, "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": dec["h2d"],
-                    "d2h_bytes_per_step": dec["d2h"], "steps": dec["e2e_steps"]},
+            "e2e": e2e,
             "gpu_launches": args.steps * dec["launches_per_step"], "clocks": dec["clocks"],
             "hbm_frac": value / world / peaks["hbm_gbs"], "prefill": prefill,
             "isolated": {"workload": "one forward call at M=1 on a cold L2 (256 MB write before it), eager, "
@@ -787,6 +928,9 @@ def main():
         line["decode_lut"] = {"workload": "decode GEMV at M=1, dp4a against per-pair lookup tables (TL2 idea), "
                                           "ternary P(0)=0.42; PDL-chained graphs over > 2 x L2 of weight copies",
                               "cases": lut}
+        if cpu_all is not None:
+            line["sweep"]["cpu_baseline"] = cpu_all["sweep"]
+            line["nm"]["cpu_baseline"] = cpu_all["nm"]
     print(json.dumps(line), flush=True)
 
 

@@ -261,10 +261,12 @@ bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t cou
  * each device looks the array's device address up (with that device
  * current); make that first call before any stream capture.
  *
- * Limits: shapes whose bitlinear_forward_workspace_bytes(M, N, K, flags)
- * exceeds BITLINEAR_NOALLOC_SCRATCH_BYTES are rejected with
- * BITLINEAR_ERR_WORKSPACE and nothing is enqueued (for example M = 2048
- * tokens fits up to K = 4080).  All calls on a device share the one array and
+ * Limits: the one test is bitlinear_forward_workspace_bytes(M, N, K, flags)
+ * <= BITLINEAR_NOALLOC_SCRATCH_BYTES; larger shapes are rejected with
+ * BITLINEAR_ERR_WORKSPACE and nothing is enqueued.  For example M = 2048
+ * tokens fits up to K = 4080 when the tensor-core plan does not split K
+ * (enough weight rows, e.g. N >= 2048); with few weight rows the K split adds
+ * M * N fp32 partial sums, so the same M and K may not fit.  All calls on a device share the one array and
  * it keeps the previous call's contents, which this call overwrites before
  * reading; two calls whose work overlaps on the GPU (different streams, no
  * ordering between them) race on it and may return wrong results.

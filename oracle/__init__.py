@@ -29,7 +29,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+            ["gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
              "-fno-fast-math", "-fno-builtin", "-o", tmp, _SRC, "-lm"]
         )
         os.replace(tmp, _LIB)
@@ -62,6 +62,8 @@ def _load():
             "orc_rmsnorm": (None, [P, P, i32, i32, f32, P]),
             "orc_quant_act_f32": (None, [P, i32, i32, i32, P, P, P]),
             "orc_matmul_i32": (i32, [P, P, i32, i32, i32, P]),
+            "orc_matmul_i32_threads": (i32, [P, P, i32, i32, i32, P, i32]),
+            "orc_online_cpus": (i32, []),
             "orc_dequant": (None, [P, P, f32, i32, i32, i32, P]),
             "orc_bf16_from_f64": (ctypes.c_uint16, [ctypes.c_double]),
             "orc_hadamard_block": (i32, [i32]),
@@ -220,6 +222,24 @@ def matmul_i32(q: np.ndarray, Wt: np.ndarray) -> np.ndarray:
     return acc
 
 
+def matmul_i32_threads(q: np.ndarray, Wt: np.ndarray, threads: int) -> np.ndarray:
+    """matmul_i32 with the output columns split over `threads` POSIX threads (same loop per element)."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    Wt = np.ascontiguousarray(Wt, dtype=np.int8)
+    M, K = q.shape
+    N, K2 = Wt.shape
+    assert K == K2
+    acc = np.empty((M, N), dtype=np.int32)
+    if _load().orc_matmul_i32_threads(_ptr(q), _ptr(Wt), M, N, K, _ptr(acc), int(threads)) != 0:
+        raise OverflowError("accumulator left int32 (or a thread could not start)")
+    return acc
+
+
+def online_cpus() -> int:
+    """Host threads the system reports online."""
+    return int(_load().orc_online_cpus())
+
+
 def dequant(acc: np.ndarray, gamma: np.ndarray, alpha, Qb: int = QB) -> np.ndarray:
     """bf16 bits of acc * alpha * gamma / Qb (fp64, one rounding)."""
     acc = np.ascontiguousarray(acc, dtype=np.int32)
@@ -234,10 +254,11 @@ def bf16_from_f64(v: float) -> int:
     return int(_load().orc_bf16_from_f64(float(v)))
 
 
-def forward(x_bf16: np.ndarray, Wt: np.ndarray, alpha, Qb: int = QB):
-    """Full forward on a dense ternary matrix: returns (y bf16 bits, acc, q, gamma, rowsum)."""
+def forward(x_bf16: np.ndarray, Wt: np.ndarray, alpha, Qb: int = QB, threads: int = 1):
+    """Full forward on a dense ternary matrix: returns (y bf16 bits, acc, q, gamma, rowsum).
+    threads > 1 runs the contraction on that many host threads (same result)."""
     q, g, rs = quant_act(x_bf16, Qb)
-    acc = matmul_i32(q, Wt)
+    acc = matmul_i32(q, Wt) if threads <= 1 else matmul_i32_threads(q, Wt, threads)
     y = dequant(acc, g, alpha, Qb)
     return y, acc, q, g, rs
 
@@ -255,7 +276,8 @@ def pack_weights(W: np.ndarray, n: int = 0, m: int = 0):
     return {"alpha": alpha, "Wt": Weff, "values": vals, "meta": meta, "mask": mask}
 
 
-# ---------------------------------------------------------------- H-BitLinear (BitNet v2 section of the blog)
+# ---------------------------------------------------------------- H-BitLinear ("BitNet v2" page, brain.hanbit.co.kr:
+# the H-BitLinear module and native 4-bit activation paragraphs)
 
 def hadamard_block(K: int) -> int:
     """Size of the Hadamard blocks along K: the largest power of two dividing K."""

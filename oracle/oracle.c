@@ -45,7 +45,8 @@
  *    quantisation.  eps is a parameter (the page's nn.RMSNorm leaves it to
  *    the dtype's default).
  *
- *  - H-BitLinear ("BitNet 1-Bit LLM" blog, section on BitNet v2: an online
+ *  - H-BitLinear ("BitNet v2" page of brain.hanbit.co.kr, the paragraphs on
+ *    the H-BitLinear module and on native 4-bit activations: an online
  *    Hadamard transform of the activations, then 4-bit activation
  *    quantisation, then the ternary linear map).  The pages give neither the
  *    transform's size, normalisation or evaluation order nor the 4-bit
@@ -59,10 +60,12 @@
  *    are the ternary matrix of the rotated-basis latent weights (the
  *    transform is not applied to them at run time).
  *
- * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math
+ * Build: gcc -O2 -std=gnu11 -fPIC -shared -pthread -ffp-contract=off -fno-fast-math
  */
 #include <fenv.h>
 #include <math.h>
+#include <pthread.h>
+#include <unistd.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -378,6 +381,65 @@ int orc_matmul_i32(const int8_t* q, const int8_t* Wt, int M, int N, int K, int32
     return bad ? -1 : 0;
 }
 
+/* The same contraction spread over nthreads POSIX threads, each running the
+ * loop above on its own band of output columns j (no other change: the
+ * timed all-cores baseline of the benchmark, not a second definition).
+ * Returns -1 if a sum leaves int32 or a thread cannot be started. */
+typedef struct {
+    const int8_t* q;
+    const int8_t* Wt;
+    int M, N, K, j0, j1, bad;
+    int32_t* acc;
+} orc_band;
+
+static void* orc_band_run(void* arg) {
+    orc_band* b = (orc_band*)arg;
+    for (int i = 0; i < b->M; ++i)
+        for (int j = b->j0; j < b->j1; ++j) {
+            int64_t s = 0;
+            const int8_t* a = b->q + (int64_t)i * b->K;
+            const int8_t* w = b->Wt + (int64_t)j * b->K;
+            for (int k = 0; k < b->K; ++k) s += (int64_t)a[k] * (int64_t)w[k];
+            if (s > INT32_MAX || s < INT32_MIN) b->bad = 1;
+            b->acc[(int64_t)i * b->N + j] = (int32_t)s;
+        }
+    return NULL;
+}
+
+int orc_matmul_i32_threads(const int8_t* q, const int8_t* Wt, int M, int N, int K, int32_t* acc, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > N) nthreads = N;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    orc_band* bands = (orc_band*)malloc(sizeof(orc_band) * (size_t)nthreads);
+    if (!th || !bands) {
+        free(th);
+        free(bands);
+        return -1;
+    }
+    int started = 0, bad = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        orc_band* b = &bands[t];
+        b->q = q; b->Wt = Wt; b->M = M; b->N = N; b->K = K; b->acc = acc; b->bad = 0;
+        b->j0 = (int)((int64_t)N * t / nthreads);
+        b->j1 = (int)((int64_t)N * (t + 1) / nthreads);
+        if (pthread_create(&th[t], NULL, orc_band_run, b) != 0) {
+            bad = 1;
+            break;
+        }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) {
+        pthread_join(th[t], NULL);
+        bad |= bands[t].bad;
+    }
+    free(th);
+    free(bands);
+    return bad ? -1 : 0;
+}
+
+/* Number of host threads the system reports online. */
+int orc_online_cpus(void) { return (int)sysconf(_SC_NPROCESSORS_ONLN); }
+
 /* y = acc * alpha * gamma_m / Qb in fp64, rounded once to bf16. */
 void orc_dequant(const int32_t* acc, const float* gamma, float alpha, int M, int N, int Qb, uint16_t* y) {
     for (int i = 0; i < M; ++i)
@@ -407,8 +469,8 @@ int orc_forward(const uint16_t* x, int M, int K, const int8_t* Wt, int N, float 
 }
 
 /* ------------------------------------------------------------------------ */
-/* H-BitLinear: online Hadamard transform, 4-bit activations ("BitNet 1-Bit  */
-/* LLM" blog, BitNet v2 section)                                             */
+/* H-BitLinear: online Hadamard transform, 4-bit activations ("BitNet v2"   */
+/* page, brain.hanbit.co.kr: the H-BitLinear and native 4-bit paragraphs)   */
 /* ------------------------------------------------------------------------ */
 
 /* Largest power of two that divides K (1 for odd K). */

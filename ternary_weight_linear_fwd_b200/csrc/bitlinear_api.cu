@@ -97,10 +97,40 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// A tensor map depends only on the address, extents, stride, box and swizzle
+// it was encoded from, so encoded maps are kept per host thread (a small
+// round-robin table) and reused by later calls with the same key: repeated
+// calls on the same weights and buffers skip the driver's encoding.
+struct MapKey {
+  const void* base;
+  uint64_t inner, outer, stride;
+  uint32_t box_inner, box_outer, swizzle;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && inner == o.inner && outer == o.outer && stride == o.stride &&
+           box_inner == o.box_inner && box_outer == o.box_outer && swizzle == o.swizzle;
+  }
+};
+
+constexpr int kMapCache = 256;
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  bool used[kMapCache] = {};
+  int next = 0;
+};
+thread_local MapCache t_maps;
+
 // 2-D uint8 tensor map: inner extent `inner` bytes, `outer` rows of `stride`
 // bytes, box {box_inner, box_outer}; out-of-range elements read as zero.
 bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t stride,
                  uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  const MapKey k{base, inner, outer, stride, box_inner, box_outer, swizzle128 ? 1u : 0u};
+  MapCache& c = t_maps;
+  for (int i = 0; i < kMapCache; ++i)
+    if (c.used[i] && c.key[i] == k) {
+      *map = c.map[i];
+      return true;
+    }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -110,7 +140,41 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  c.key[c.next] = k;
+  c.map[c.next] = *map;
+  c.used[c.next] = true;
+  c.next = (c.next + 1) % kMapCache;
+  return true;
+}
+
+// Largest dynamic shared memory already granted to a kernel on a device
+// (per host thread): the attribute is set only when a launch needs more.
+struct SmemGrant {
+  int dev;
+  const void* fn;
+  size_t bytes;
+};
+constexpr int kSmemGrants = 128;
+thread_local SmemGrant t_grants[kSmemGrants];
+thread_local int t_ngrants = 0;
+
+bool ensure_smem(const void* fn, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  for (int i = 0; i < t_ngrants; ++i)
+    if (t_grants[i].dev == dev && t_grants[i].fn == fn) {
+      if (t_grants[i].bytes >= smem) return true;
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess)
+        return false;
+      t_grants[i].bytes = smem;
+      return true;
+    }
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return false;
+  if (t_ngrants < kSmemGrants) t_grants[t_ngrants++] = SmemGrant{dev, fn, smem};
+  return true;
 }
 
 template <typename Kern, typename... Args>
@@ -138,11 +202,7 @@ bitlinear_status launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaSt
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-        cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-  }
+  if (smem > 48 * 1024 && !ensure_smem(reinterpret_cast<const void*>(kern), smem)) return BITLINEAR_ERR_CUDA;
   return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
@@ -928,3 +988,19 @@ extern "C" bitlinear_status bitlinear_forward_noalloc(const bitlinear_weights* w
   // nothing has to be cleared between calls.
   return forward_common(w, x, M, y, acc, scratch, BITLINEAR_NOALLOC_SCRATCH_BYTES, flags, stream, w->nm_m != 0);
 }
+
+#ifdef BITLINEAR_TEST_HOOKS
+// ---------------------------------------------------------------- test builds only
+#include "../../include/bitlinear_test_hooks.h"
+
+extern "C" bitlinear_status bitlinear_test_set_wait_fault(uint64_t wait_limit_ns, uint32_t extra_tx_bytes) {
+  DeviceState* dev = nullptr;
+  bitlinear_status st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_test_wait_limit_ns, &wait_limit_ns, sizeof wait_limit_ns) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_test_extra_tx, &extra_tx_bytes, sizeof extra_tx_bytes) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+#endif

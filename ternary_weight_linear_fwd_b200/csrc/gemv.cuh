@@ -216,6 +216,20 @@ __device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restri
   return mx;
 }
 
+// CTA-wide barrier that also settles a timed-out wait for the weight copies
+// (one barrier, phase 0).  Returns true when some thread of the CTA gave up:
+// then thread 0 records kDevTimeoutProducer and waits once more (bounded) for
+// the copies still in flight, so that the CTA's shared memory is not released
+// under them, and the CTA writes no output.
+__device__ __forceinline__ bool gemv_gave_up(bool landed, uint64_t* bar, int32_t* status) {
+  if (!__syncthreads_or(!landed)) return false;
+  if (threadIdx.x == 0) {
+    *status = kDevTimeoutProducer;
+    if (!mbar_wait(bar, 0)) *status = kDevTimeoutDrain;
+  }
+  return true;
+}
+
 __device__ __forceinline__ void gemv_store(uint16_t* y, int32_t* acc, int row, int32_t total, float s) {
   if (acc) acc[row] = total;
   const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(total), s));
@@ -320,7 +334,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     mbar_init(&s_bar, 1);
     fence_mbar_init();
     tma_prefetch_desc(map);
-    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box));
+    mbar_arrive_expect_tx(&s_bar,
+                          static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box) + test_extra_tx());
     const uint64_t pol = l2_policy_evict_first();
     for (int st = 0; st < stripes; ++st) tma_load_2d_hint(s_w + st * stripe_bytes, map, st * 128, r0, &s_bar, pol);
   }
@@ -342,7 +357,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   pdl_launch_dependents();
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
-  if (!landed && threadIdx.x == 0) *g.status = kDevTimeoutProducer;
 
   if (landed) {
     // units (chunk, row pair), row pair fastest: the lanes of a warp read one
@@ -377,11 +391,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
       }
     }
   }
-  __syncthreads();
-  if (landed) {
-    const int32_t qsum = *s_qsum;
-    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr] - qsum, s);
-  }
+  if (gemv_gave_up(landed, &s_bar, g.status)) return;
+  const int32_t qsum = *s_qsum;
+  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr] - qsum, s);
 }
 
 // ------------------------------------------------------------------ dense M = 1, lookup tables
@@ -421,7 +433,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_con
     mbar_init(&s_bar, 1);
     fence_mbar_init();
     tma_prefetch_desc(&map0);
-    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box));
+    mbar_arrive_expect_tx(&s_bar,
+                          static_cast<uint32_t>(stripes) * 128u * static_cast<uint32_t>(rows_box) + test_extra_tx());
     const uint64_t pol = l2_policy_evict_first();
     for (int st = 0; st < stripes; ++st) tma_load_2d_hint(s_w + st * stripe_bytes, &map0, st * 128, r0, &s_bar, pol);
   }
@@ -451,7 +464,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_con
   __syncthreads();
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
-  if (!landed && threadIdx.x == 0) *g.status = kDevTimeoutProducer;
 
   if (landed) {
     const int total = nrows * C;  // units (chunk, row), row fastest
@@ -468,9 +480,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_con
       atomicAdd(&s_acc[r], acc);
     }
   }
-  __syncthreads();
-  if (landed)
-    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr], s);
+  if (gemv_gave_up(landed, &s_bar, g.status)) return;
+  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr], s);
 }
 
 // ------------------------------------------------------------------ N:M helpers
@@ -615,7 +626,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
     fence_mbar_init();
     tma_prefetch_desc(&map_v);
     tma_prefetch_desc(&map_m);
-    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes_v + stripes_m) * 128u * static_cast<uint32_t>(rows_box));
+    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(stripes_v + stripes_m) * 128u * static_cast<uint32_t>(rows_box) +
+                                      test_extra_tx());
     const uint64_t pol = l2_policy_evict_first();
     for (int st = 0; st < stripes_v; ++st) tma_load_2d_hint(s_v + st * stripe_bytes, &map_v, st * 128, r0, &s_bar, pol);
     for (int st = 0; st < stripes_m; ++st) tma_load_2d_hint(s_m + st * stripe_bytes, &map_m, st * 128, r0, &s_bar, pol);
@@ -631,7 +643,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
   pdl_launch_dependents();
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
-  if (!landed && threadIdx.x == 0) *a.status = kDevTimeoutProducer;
 
   if (landed) {
     const uint32_t* lut_lane = s_lut + (threadIdx.x & 31);
@@ -664,11 +675,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
       }
     }
   }
-  __syncthreads();
-  if (landed) {
-    const int32_t qsum = *s_qsum;
-    for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a.y, a.acc, r0 + rr, s_acc[rr] - qsum, s);
-  }
+  if (gemv_gave_up(landed, &s_bar, a.status)) return;
+  const int32_t qsum = *s_qsum;
+  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a.y, a.acc, r0 + rr, s_acc[rr] - qsum, s);
 }
 
 }  // namespace bl

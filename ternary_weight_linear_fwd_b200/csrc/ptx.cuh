@@ -24,6 +24,20 @@ enum : int32_t {
 // Wait limit for every spin: about one second of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 
+#ifdef BITLINEAR_TEST_HOOKS
+// Test builds only (a separate library): the wait limit and a number of bytes
+// added to the decode GEMV's expected copy count, both settable from the host,
+// so that a test can make a bounded wait run out without any fault: every copy
+// that is issued still lands, the barrier just never completes.
+__device__ uint64_t g_test_wait_limit_ns = kWaitLimitNs;
+__device__ uint32_t g_test_extra_tx = 0;
+__device__ __forceinline__ uint64_t wait_limit_ns() { return *const_cast<volatile uint64_t*>(&g_test_wait_limit_ns); }
+__device__ __forceinline__ uint32_t test_extra_tx() { return *const_cast<volatile uint32_t*>(&g_test_extra_tx); }
+#else
+__device__ __forceinline__ uint64_t wait_limit_ns() { return kWaitLimitNs; }
+__device__ __forceinline__ uint32_t test_extra_tx() { return 0u; }
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -66,13 +80,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs and returns false (the caller records a status and unwinds).
+// wait_limit_ns() (kWaitLimitNs) and returns false (the caller records a
+// status and unwinds).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if ((++spins & 255u) == 0u && globaltimer_ns() - t0 > limit) return false;
   }
   return true;
 }

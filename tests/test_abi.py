@@ -22,8 +22,11 @@ def L():
     return bl.lib()
 
 
-def _declared():
-    src = open(HEADER).read()
+HOOKS_HEADER = os.path.join(ROOT, "include", "bitlinear_test_hooks.h")
+
+
+def _declared(header=HEADER):
+    src = open(header).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(bitlinear_[a-z_0-9]+)\s*\(", src)))
 
@@ -33,6 +36,22 @@ def test_exports_every_declared_symbol(L):
     assert len(names) >= 10
     for n in names:
         assert hasattr(L, n), n
+
+
+def test_headers_cover_every_header_file():
+    """include/ holds the product header and the test-hook header, nothing else."""
+    assert sorted(os.listdir(os.path.join(ROOT, "include"))) == ["bitlinear.h", "bitlinear_test_hooks.h"]
+
+
+def test_test_hooks_only_in_the_test_build(L):
+    """The test build exports the product ABI plus the hooks; the product library has no hook."""
+    hooks = _declared(HOOKS_HEADER)
+    assert hooks == ["bitlinear_test_set_wait_fault"]
+    T = ctypes.CDLL(blbuild.build_test_hooks())
+    for n in _declared() + hooks:
+        assert hasattr(T, n), n
+    for n in hooks:
+        assert not hasattr(L, n), n
 
 
 def test_status_strings(L):

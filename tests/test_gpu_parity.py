@@ -197,6 +197,73 @@ def test_forward_layer_sweep_shapes(M):
         _check_rows(x, Wt, a, y, acc, rows)
 
 
+def test_forward_layer_sweep_m4096_sampled():
+    """The seven 2B4T layer matrices at M = 4096 tokens through bitlinear_forward's default path (the
+    largest configuration of the layer sweep): the kernels run at full size, 20 sampled tokens (the
+    first, the last, the edges of the 128-token tiles around the middle and 15 drawn at random) are
+    checked against the oracle on every output."""
+    M = 4096
+    rows = np.unique(np.concatenate([[0, 127, 128, 2047, 2048, M - 1], synth.splitmix64(4096, 6, 15) % M]))
+    rows = rows.astype(np.int64)
+    for name, (K, N) in synth.B2B4T_LAYER.items():
+        x, Wt, a, w = _dense_case(M, K, N, seed=4)
+        y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+        assert bl.last_kernel().startswith("tc_gemm_dense"), (name, bl.last_kernel())
+        _check_rows(x, Wt, a, y, acc, rows)
+
+
+def test_forward_stale_workspace():
+    """A caller workspace full of 0xFF bytes gives the same results as a fresh one: every byte the GEMM
+    reads is written (codes, scales, code sums) or cleared (split-K sums and counters) by the call itself.
+    Shapes: a K-split GEMM (few row tiles), then a tile-parallel one, then the split one again."""
+    cases = [(16, 2560, 640), (300, 1000, 2048), (16, 2560, 640)]
+    ws = torch.full((max(bl.forward_workspace_bytes(M, N, K) for M, K, N in cases),), 0xFF, dtype=torch.uint8,
+                    device=DEV)
+    for M, K, N in cases:
+        x, Wt, a, w = _dense_case(M, K, N, seed=M + N)
+        y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, workspace=ws)
+        _check_rows(x, Wt, a, y, acc, np.arange(M))
+        ws.fill_(0xFF)
+
+
+def test_pack_dense_exact_ties():
+    """Latent weights at exactly +-0.5 * d and +-1.5 * d, d = RN(alpha + 1e-5), ternarise to 0 and to +-1
+    (round half to even, then the clamp), and the next float above 0.5 * d to +-1, on the GPU as in the
+    oracle.  alpha depends on the tie entries themselves, so they are placed by a fixed-point iteration:
+    alpha of the final matrix is the alpha the ties were computed from (the sums of fp32 magnitudes are
+    exact in fp64 here, so the kernel's summation order cannot change it)."""
+    N, K = 96, 520
+    W = synth.latent_weights(N, K, seed=44)
+    rows = [0, 1, 47, 95]
+    for _ in range(50):
+        a = oracle.absmean(W)
+        d = np.float32(a + np.float32(1e-5))
+        h = np.float32(d * np.float32(0.5))
+        t = np.float32(np.float32(3) * h)
+        above = np.nextafter(h, np.float32(1))
+        vals = [h, -h, above, -above]
+        if np.float64(t) == 3.0 * np.float64(h):  # 1.5 d is representable: include that tie as well
+            vals += [t, -t]
+        for r in rows:
+            W[r, 3:3 + len(vals)] = vals
+        if oracle.absmean(W) == a:
+            break
+    else:
+        pytest.fail("no fixed point for alpha")
+    expect = [0, 0, 1, -1] + ([1, -1] if len(vals) == 6 else [])
+    ref = oracle.pack_weights(W)
+    for r in rows:
+        np.testing.assert_array_equal(ref["Wt"][r, 3:3 + len(vals)], expect)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV))
+    assert float(w.alpha.cpu()[0]) == float(ref["alpha"])
+    np.testing.assert_array_equal(w.codes.cpu().numpy(), ref["codes"])
+    for n, m in ((2, 4), (6, 8)):
+        refn = oracle.pack_weights(W, n, m)
+        wn = bl.pack_weights(torch.from_numpy(W).to(DEV), n, m)
+        np.testing.assert_array_equal(wn.codes.cpu().numpy(), refn["values"])
+        np.testing.assert_array_equal(wn.meta.cpu().numpy(), refn["meta"])
+
+
 def test_forward_zero_and_outlier_rows():
     M, K, N = 6, 512, 256
     x = synth.activations(M, K, seed=12)

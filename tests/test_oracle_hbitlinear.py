@@ -1,5 +1,6 @@
-"""Pins for the H-BitLinear oracle ("BitNet 1-Bit LLM" blog, BitNet v2 section: an online Hadamard
-transform of the activations, 4-bit activation quantisation, then the ternary linear map).  Closed
+"""Pins for the H-BitLinear oracle ("BitNet v2" page of brain.hanbit.co.kr, the paragraphs on the
+H-BitLinear module and on native 4-bit activations: an online Hadamard transform of the activations,
+4-bit activation quantisation, then the ternary linear map).  Closed
 forms of the Sylvester Hadamard matrix, its orthogonality, hand-worked codes, the reduction to the
 plain 4-bit BitLinear for odd K, and the quantisation error bound against a float64 reference.
 

@@ -436,3 +436,15 @@ def test_forward_norm_reduces_to_forward_on_unit_rows():
     np.testing.assert_array_equal(acc2, acc0)
     np.testing.assert_array_equal(synth.bf16_bits_to_f32(y2), 2.0 * synth.bf16_bits_to_f32(y0))
     assert np.abs(acc0).max() > 0
+
+
+def test_threaded_contraction_equals_plain_loop():
+    """The benchmark's all-cores leg splits the output columns over threads; every element is the same
+    loop, so the accumulators must equal the single-threaded ones (and the float64 library matmul)."""
+    T = synth.ternary_weights(301, 777, seed=12)
+    x = synth.activations(5, 777, seed=13)
+    q, _, _ = oracle.quant_act(x)
+    a1 = oracle.matmul_i32(q, T)
+    for th in (2, 3, 8, 400):
+        np.testing.assert_array_equal(oracle.matmul_i32_threads(q, T, th), a1)
+    np.testing.assert_array_equal(a1, (q.astype(np.float64) @ T.astype(np.float64).T).astype(np.int64))

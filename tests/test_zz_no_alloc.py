@@ -5,12 +5,16 @@ array inside the library, so its results must equal those of
 bitlinear_forward with a caller-provided workspace -- on consecutive calls too,
 since each call reuses the array the previous one left behind.
 
-This file is collected last on purpose (see the file name)."""
+The file name sorts after every other test file, so pytest collects it last:
+a run that stops at the first failure has then already run every other test,
+and the test also runs after the others have left the library's state (the
+scratch array's contents) behind, as well as alone in a fresh process."""
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle
 from ternary_weight_linear_fwd_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -42,9 +46,10 @@ def _bits(t):
 def _case(M, K, N, seed, n=0, m=0):
     x = synth.activations(M, K, seed=seed)
     W = synth.latent_weights(N, K, seed=seed)
+    ref = oracle.pack_weights(W, n, m)
     w = bl.pack_weights(torch.from_numpy(W).to(DEV), n, m)
     xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
-    return w, xd
+    return w, xd, x, ref
 
 
 def _noalloc(L, w, xd):
@@ -58,25 +63,36 @@ def _noalloc(L, w, xd):
     return y, acc
 
 
+def _check(L, fwd, M, K, N, seed, n, m):
+    """The no-allocation call equals the workspace call bit for bit (same kernels, same inputs) and the
+    oracle within the parity tolerance (accumulators exact, outputs within one bf16 ulp)."""
+    w, xd, x, ref = _case(M, K, N, seed, n, m)
+    y_ref, acc_ref = fwd(w, xd, want_acc=True)
+    y, acc = _noalloc(L, w, xd)
+    torch.cuda.synchronize()
+    assert torch.equal(acc, acc_ref)
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    yo, acco, *_ = oracle.forward(x, ref["Wt"], ref["alpha"])
+    np.testing.assert_array_equal(acc.cpu().numpy(), acco)
+    d = np.abs(_bits(y).astype(np.int32) - yo.astype(np.int32))
+    assert d.max() <= 1  # one bf16 ulp, the tolerance of every forward parity test
+
+
+# Two or three calls in a row with different inputs and shapes, each reusing the scratch the previous
+# call left behind: a K-split tensor-core GEMM (few weight-row tiles), a tile-parallel one with a
+# different M x N, and the M = 1 decode GEMV, which uses no scratch.
 @pytest.mark.parametrize("n,m", [(0, 0), (6, 8)])
 def test_noalloc_matches_workspace_forward_twice(n, m):
     L = _lib()
     fwd = bl.forward_nm if m else bl.forward
-    # two calls in a row with different inputs and shapes: the second reuses the scratch the first left behind
-    for (M, K, N, seed) in ((300, 1000, 400, 1), (64, 2560, 640, 2)):
-        w, xd = _case(M, K, N, seed, n, m)
-        y_ref, acc_ref = fwd(w, xd, want_acc=True)
-        y, acc = _noalloc(L, w, xd)
-        torch.cuda.synchronize()
-        np.testing.assert_array_equal(acc.cpu().numpy(), acc_ref.cpu().numpy())
-        d = np.abs(_bits(y).astype(np.int32) - _bits(y_ref).astype(np.int32))
-        assert d.max() <= 1  # the tolerance the parity tests use (one bf16 ulp)
+    for (M, K, N, seed) in ((64, 2560, 640, 2), (300, 512, 2048, 1), (64, 2560, 640, 3), (1, 2560, 1000, 4)):
+        _check(L, fwd, M, K, N, seed, n, m)
     assert bl.device_status() == 0
 
 
 def test_noalloc_rejects_oversized_scratch():
     L = _lib()
-    w, xd = _case(2, 4096, 64, 3)
+    w, xd, _, _ = _case(2, 4096, 64, 3)
     big_m = 2048  # 2048 x 4096 int8 codes + scales exceed the fixed 8 MiB array
     assert bl.forward_workspace_bytes(big_m, 64, 4096) > bl.NOALLOC_SCRATCH_BYTES
     ws = w.c_struct()
