@@ -490,6 +490,9 @@ def run_sweep(dev, min_calls: int = 16, warmup: int = 3, reps: int = 5):
             tot_b, tot_ops, tot_s = tot_b + nbytes, tot_ops + ops, tot_s + sec
             del cps, calls, y, xk
         row["layer"] = {"us": tot_s * 1e6, "GBps": tot_b / tot_s / 1e9, "TOPS": tot_ops / tot_s / 1e12}
+        peaks, _ = measured_peaks()
+        row["layer"]["hbm_frac"] = row["layer"]["GBps"] / peaks["hbm_gbs"]
+        row["layer"]["int8_frac"] = row["layer"]["TOPS"] / (2.0 * peaks["bf16_tflops"])
         out[f"M={M}"] = row
         del x, ws
     assert bl.device_status() == 0
@@ -590,6 +593,50 @@ def run_isolated(dev, iters: int = 30, warmup: int = 3):
         sec = statistics.median(ts)
         nbytes = N * K // 4 + 4 + 2 * K + 2 * N
         out[f"{name} {K}->{N}"] = {"us": sec * 1e6, "GBps": nbytes / sec / 1e9, "kernel": bl.last_kernel()}
+    assert bl.device_status() == 0
+    return out
+
+
+def run_hbit(dev, warmup: int = 3, reps: int = 5, calls: int = 16):
+    """H-BitLinear (Hadamard transform + 4-bit codes + the tensor-core GEMM) on the 2B4T FFN shapes at
+    M = 1 (chained over > 2 x L2 of weight copies) and M = 2048, against the 8-bit forward of the same
+    call; and the transform-and-quantise kernel alone (GB/s on 2MK read + MK written + 8M)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+
+    out = {}
+    for name, K, N in (("gate", 2560, 6912), ("down", 6912, 2560)):
+        T = torch.from_numpy(synth.ternary_weights(N, K, seed=14)).to(dev)
+        w = bl.pack_ternary(T, float(synth.alpha_uniform(14)))
+        del T
+        for M in (1, 2048):
+            x = torch.from_numpy(synth.activations(M, K, seed=14).view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bl.forward_workspace_bytes(M, N, K, bl.FLAG_PATH_TC), dtype=torch.uint8, device=dev)
+            cps = _copies(w, w.nbytes) if M == 1 else [w]
+            n = max(calls, len(cps))
+            t_h = time_chain_graph(dev, [(lambda ww=cps[i % len(cps)]: bl.forward_hbit(ww, x, out=y, workspace=ws,
+                                                                                        flags=bl.FLAG_PDL))
+                                         for i in range(n)], warmup, reps) / n
+            kern = bl.last_kernel()
+            t_8 = time_chain_graph(dev, [(lambda ww=cps[i % len(cps)]: bl.forward(ww, x, out=y, workspace=ws,
+                                                                                   flags=bl.FLAG_PDL))
+                                         for i in range(n)], warmup, reps) / n
+            lib = bl.lib()
+            q = torch.empty((M, K), dtype=torch.int8, device=dev)
+            gm = torch.empty(M, dtype=torch.float32, device=dev)
+            qcall = (lambda: lib.bitlinear_hadamard_quant_act4(x.data_ptr(), M, K, q.data_ptr(), gm.data_ptr(), None,
+                                                               torch.cuda.current_stream(dev).cuda_stream))
+            t_q = time_chain_graph(dev, [qcall] * calls, warmup, reps) / calls
+            out[f"{name} {K}->{N} M={M}"] = {
+                "forward_hbit_us": t_h * 1e6, "forward_hbit_TOPS": 2.0 * M * N * K / t_h / 1e12,
+                "forward_hbit_GBps": (w.nbytes + 4 + 2 * M * K + 2 * M * N) / t_h / 1e9, "kernel": kern,
+                "forward_8bit_us": t_8 * 1e6, "hadamard_quant_act4_us": t_q * 1e6,
+                "hadamard_quant_act4_GBps": (3 * M * K + 8 * M) / t_q / 1e9, "weight_copies": len(cps)}
+            del cps, x, y, ws, q, gm
     assert bl.device_status() == 0
     return out
 
@@ -848,12 +895,13 @@ def main():
 
     pre = run_prefill(dev, args.prefill_iters, 3)
     iso = run_isolated(dev)
-    sweep = nm = norm = lut = None
+    sweep = nm = norm = lut = hbit = None
     if not args.no_sweep:
         sweep = run_sweep(dev)
         nm = run_nm(dev)
         norm = run_norm(dev)
         lut = run_lut(dev)
+        hbit = run_hbit(dev)
 
     if world > 1:
         barrier(dev)
@@ -928,6 +976,10 @@ def main():
         line["decode_lut"] = {"workload": "decode GEMV at M=1, dp4a against per-pair lookup tables (TL2 idea), "
                                           "ternary P(0)=0.42; PDL-chained graphs over > 2 x L2 of weight copies",
                               "cases": lut}
+        line["hbit"] = {"workload": "H-BitLinear (Hadamard transform of each token row, 4-bit codes, tcgen05 "
+                                    "GEMM, rescale by alpha*gamma/7) on 2B4T gate/down, ternary P(0)=0.42; "
+                                    "PDL-chained graphs (M=1: > 2 x L2 of weight copies); the 8-bit forward of "
+                                    "the same call beside it", "cases": hbit}
         if cpu_all is not None:
             line["sweep"]["cpu_baseline"] = cpu_all["sweep"]
             line["nm"]["cpu_baseline"] = cpu_all["nm"]

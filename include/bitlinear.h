@@ -94,6 +94,9 @@ typedef enum bitlinear_status {
                                          ends. */
 #define BITLINEAR_FLAG_PATH_GEMV 0x2u /* force the M = 1 streaming GEMV (needs M == 1) */
 #define BITLINEAR_FLAG_PATH_TC 0x4u   /* force the tensor-core path at any M */
+#define BITLINEAR_FLAG_PATH_PERSISTENT 0x10u /* tensor-core path: take the persistent GEMM (separate
+                                        * quantisation launch, K split through a workspace) even
+                                        * where the fused few-token kernel applies; same results */
 #define BITLINEAR_FLAG_DECODE_LUT 0x8u /* M = 1, dense weights: run the decode GEMV with
                                         * per-pair lookup tables (the TL2 idea of the
                                         * "BitNet 1-Bit LLM" blog, section "I2_S kernel
@@ -187,6 +190,41 @@ bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16
                                         float eps, uint16_t* y, int32_t* acc, void* workspace, size_t workspace_bytes,
                                         uint32_t flags, void* stream);
 
+/* H-BitLinear ("BitNet v2" page, brain.hanbit.co.kr: the paragraphs on the
+ * H-BitLinear module and on native 4-bit activations): an online Hadamard
+ * transform of the activations, then 4-bit quantisation, then the ternary
+ * linear map.  The page fixes neither the transform's size, normalisation and
+ * evaluation order nor the 4-bit quantiser; this library takes, per token row:
+ *   B  = the largest power of two dividing K (2560 -> 512, 6912 -> 256,
+ *        odd K -> 1, no transform);
+ *   xh = each B-block times the Sylvester-order Walsh-Hadamard matrix, by the
+ *        fast butterflies in fp32 (stage h = 1, 2, ..., B/2: every pair
+ *        (j, j + h) with bit h of j clear becomes (a + b, a - b), one rounding
+ *        each), then one fp32 multiply by RN32(1 / sqrt(B));
+ *   gamma = max_k |xh_k|, q = clamp(rne(RN32(xh * 7) / RN32(gamma + 1e-5)),
+ *        -8, 7) (held in int8), and y = acc * alpha * gamma / 7 with the
+ *        rescale s = RN(RN(alpha * gamma) / 7).
+ * The weights are the ternary matrix as given (no transform at run time). */
+#define BITLINEAR_HBIT_MAX_K 16384  /* the row is transformed in shared memory */
+
+/* Hadamard transform and 4-bit codes of each token row (natural k order).
+ * x device, bf16 bits [M, K] (2-byte aligned); q device out int8 [M, K] in
+ * [-8, 7]; gamma device out fp32 [M] = max |xh|; rowsum device out (may be
+ * NULL) int32 [M] = sum of the row's codes.  Errors: NULL, SHAPE (K above
+ * BITLINEAR_HBIT_MAX_K), ALIGN, DEVICE, CUDA. */
+bitlinear_status bitlinear_hadamard_quant_act4(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* gamma,
+                                               int32_t* rowsum, void* stream);
+
+/* y = H-BitLinear(x): the transform and 4-bit codes above, then the
+ * tensor-core GEMM with dense or N:M weights (every M, M = 1 included).
+ * Arguments as bitlinear_forward; workspace_bytes at least
+ * bitlinear_forward_workspace_bytes(M, N, K, BITLINEAR_FLAG_PATH_TC).
+ * flags: BITLINEAR_FLAG_PDL (BITLINEAR_FLAG_PATH_TC is accepted, and implied).
+ * Errors: as bitlinear_forward; SHAPE also for K above BITLINEAR_HBIT_MAX_K. */
+bitlinear_status bitlinear_forward_hbit(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
+                                        int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                        void* stream);
+
 /* Workspace bytes needed by bitlinear_forward / bitlinear_forward_nm.  0 when
  * the call takes the M = 1 GEMV path (which quantises in-kernel).  The
  * tensor-core path needs the int8 codes, gamma and code sums of x and, when it
@@ -202,7 +240,14 @@ size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32
  * acc      device, out (may be NULL): int32 [M, N], the exact accumulator.
  * workspace, workspace_bytes: device scratch (may be NULL when 0 is needed).
  * flags    BITLINEAR_FLAG_*.
- * Path: M == 1 takes the streaming GEMV; M >= 2 the tcgen05 tensor-core GEMM.
+ * Path: M == 1 takes the streaming GEMV.  2 <= M <= 64 (or M == 1 with
+ * BITLINEAR_FLAG_PATH_TC) takes the fused few-token tensor-core kernel: one
+ * launch that quantises, contracts on tcgen05 with K split over the CTAs of a
+ * thread-block cluster and reduced through distributed shared memory, and
+ * rescales; it needs no workspace (and reads none it is given) when K fits
+ * eight slices of resident weights (K <= 8 * 24 * 128 for up to 32 tokens).
+ * Larger M, longer K, or BITLINEAR_FLAG_PATH_PERSISTENT take the persistent
+ * tcgen05 GEMM after a quantisation launch.  Every path gives the same bits.
  * Errors: NULL, SHAPE, ALIGN, PATTERN, WORKSPACE, FLAGS, DEVICE, CUDA. */
 bitlinear_status bitlinear_forward(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
                                    int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,

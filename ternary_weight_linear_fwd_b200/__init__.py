@@ -15,8 +15,9 @@ from typing import Optional
 __all__ = [
     "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
     "quant_act", "rmsnorm_quant_act", "forward", "forward_nm", "forward_group", "forward_norm",
-    "forward_workspace_bytes", "device_status", "last_kernel", "layout_version",
-    "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT",
+    "forward_workspace_bytes", "device_status", "last_kernel", "layout_version", "hadamard_quant_act4",
+    "forward_hbit", "HBIT_MAX_K",
+    "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT", "FLAG_PATH_PERSISTENT",
 ]
 
 FLAG_PDL = 0x1
@@ -24,6 +25,7 @@ MAX_GROUP = 4
 FLAG_PATH_GEMV = 0x2
 FLAG_PATH_TC = 0x4
 FLAG_DECODE_LUT = 0x8
+FLAG_PATH_PERSISTENT = 0x10
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
@@ -68,6 +70,8 @@ def lib() -> ctypes.CDLL:
             "bitlinear_forward_group": (st, [ctypes.POINTER(_Weights), i32, P, i32, P, P, P, sz, u32, P]),
             "bitlinear_rmsnorm_quant_act": (st, [P, i32, i32, P, ctypes.c_float, P, P, P, P]),
             "bitlinear_forward_norm": (st, [ctypes.POINTER(_Weights), P, i32, P, ctypes.c_float, P, P, P, sz, u32, P]),
+            "bitlinear_hadamard_quant_act4": (st, [P, i32, i32, P, P, P, P]),
+            "bitlinear_forward_hbit": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
             "bitlinear_device_status": (st, [P, ctypes.POINTER(i32), i32]),
             "bitlinear_last_kernel": (ctypes.c_char_p, []),
             "bitlinear_layout_version": (i32, []),
@@ -196,6 +200,46 @@ def rmsnorm_quant_act(x, g, eps: float, rowsum: bool = True, stream=None):
     _check(lib().bitlinear_rmsnorm_quant_act(_ptr(x), M, K, _ptr(g), float(eps), _ptr(q), _ptr(gm), _ptr(rs),
                                              _stream(stream)), "rmsnorm_quant_act")
     return q, gm, rs
+
+
+HBIT_MAX_K = 16384
+
+
+def hadamard_quant_act4(x, rowsum: bool = True, stream=None):
+    """H-BitLinear activations of a bf16 [M, K] CUDA matrix: the per-row Hadamard transform and 4-bit
+    codes (natural k order): (q int8 in [-8, 7], gamma, rowsum or None)."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    g = torch.empty(M, dtype=torch.float32, device=x.device)
+    rs = torch.empty(M, dtype=torch.int32, device=x.device) if rowsum else None
+    _check(lib().bitlinear_hadamard_quant_act4(_ptr(x), M, K, _ptr(q), _ptr(g), _ptr(rs), _stream(stream)),
+           "hadamard_quant_act4")
+    return q, g, rs
+
+
+def forward_hbit(w: PackedWeights, x, want_acc: bool = False, flags: int = 0, workspace=None, out=None,
+                 acc_out=None, stream=None):
+    """y = H-BitLinear(x): Hadamard transform, 4-bit codes, ternary contraction on the tensor cores,
+    rescale by alpha * gamma / 7."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w.K
+    M = x.shape[0]
+    _check_out(out, (M, w.N), torch.bfloat16, x.device, "out")
+    _check_out(acc_out, (M, w.N), torch.int32, x.device, "acc_out")
+    _check_workspace(workspace, x.device)
+    y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    acc = acc_out if acc_out is not None else (
+        torch.empty((M, w.N), dtype=torch.int32, device=x.device) if want_acc else None)
+    if workspace is None:
+        workspace = torch.empty(forward_workspace_bytes(M, w.N, w.K, FLAG_PATH_TC), dtype=torch.uint8,
+                                device=x.device)
+    ws = w.c_struct()
+    _check(lib().bitlinear_forward_hbit(ctypes.byref(ws), _ptr(x), M, _ptr(y), _ptr(acc), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), flags, _stream(stream)),
+           "forward_hbit")
+    return (y, acc) if want_acc else y
 
 
 def forward_workspace_bytes(M: int, N: int, K: int, flags: int = 0) -> int:

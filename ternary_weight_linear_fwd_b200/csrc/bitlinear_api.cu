@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -14,7 +15,7 @@
 #include <mutex>
 
 #include "../../include/bitlinear.h"
-#include "gemm_tc.cuh"
+#include "gemm_skinny.cuh"
 
 namespace bl {
 
@@ -50,6 +51,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int32_t* status = nullptr;
+  int sk_clusters[kSkMaxCluster + 1] = {};  // clusters of each size the few-token kernel fits at once (0: not asked)
 };
 
 std::mutex g_mu;
@@ -297,6 +299,104 @@ const char* tc_name(int nm, int bn) {
   return names[nm][i];
 }
 
+// ---------------------------------------------------------------- few-token path
+// Plan of the fused few-token kernel (gemm_skinny.cuh): token tile BN, K
+// slices per cluster and chunks per slice.  Not eligible (ok = false) for more
+// than 64 tokens or a K too long for eight resident slices.
+struct SkPlan {
+  bool ok;
+  int bn, cs, per, row_tiles, kchunks;
+  size_t smem;
+};
+
+// Clusters of cs CTAs of the few-token kernel resident at once on the device
+// (one CTA per SM), asked once per device and size.
+int sk_active_clusters(DeviceState* dev, int cs, size_t smem) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (dev->sk_clusters[cs] == 0) {
+    int n = -1;
+    if (ensure_smem(reinterpret_cast<const void*>(skinny_kernel<16>), smem)) {
+      cudaLaunchConfig_t cfg;
+      std::memset(&cfg, 0, sizeof cfg);
+      cfg.gridDim = dim3(cs * 64);
+      cfg.blockDim = dim3(kSkThreads);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = static_cast<unsigned>(cs);
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, skinny_kernel<16>, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = -1;
+      }
+    }
+    dev->sk_clusters[cs] = n;
+  }
+  return dev->sk_clusters[cs];
+}
+
+SkPlan sk_plan(int M, int N, int K, DeviceState* dev) {
+  SkPlan p;
+  std::memset(&p, 0, sizeof p);
+  if (M < 1 || M > 64) return p;
+  p.bn = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+  p.row_tiles = (N + kTcRows - 1) / kTcRows;
+  p.kchunks = (K + 127) / 128;
+  const size_t budget = 227 * 1024;
+  const int maxch = static_cast<int>(std::min<size_t>(kSkMaxChunks, (budget - sk_fixed_bytes(p.bn)) /
+                                                                        sk_chunk_bytes(p.bn)));
+  const int cs_min = (p.kchunks + maxch - 1) / maxch;
+  if (cs_min > kSkMaxCluster) return p;
+  // as many K slices as keep the whole grid in one wave of clusters (one CTA per SM)
+  int cs = std::max(1, std::min(std::min(dev->sm_count / p.row_tiles, kSkMaxCluster), p.kchunks));
+  cs = std::max(cs, cs_min);
+  for (; cs > cs_min; --cs) {
+    const int per = (p.kchunks + cs - 1) / cs;
+    const int n = sk_active_clusters(dev, cs, std::max(sk_smem_bytes(p.bn, per), kSkMinSmem));
+    if (n >= p.row_tiles) break;
+  }
+  p.per = (p.kchunks + cs - 1) / cs;
+  p.cs = (p.kchunks + p.per - 1) / p.per;  // no empty slice
+  p.smem = std::max(sk_smem_bytes(p.bn, p.per), kSkMinSmem);
+  if (sk_active_clusters(dev, p.cs, p.smem) <= 0) return p;  // this cluster size cannot be launched here
+  p.ok = true;
+  return p;
+}
+
+bitlinear_status skinny_launch(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
+                               bool pdl, cudaStream_t s, DeviceState* dev, const SkPlan& p) {
+  const int N = w->N, K = w->K;
+  const int64_t ld = dense_ld(K);
+  CUtensorMap mW;
+  if (!make_map_u8(&mW, w->codes, static_cast<uint64_t>(ld), static_cast<uint64_t>(N), static_cast<uint64_t>(ld), 32,
+                   kTcRows, false))
+    return BITLINEAR_ERR_CUDA;
+  SkArgs sa;
+  sa.x = x;
+  sa.M = M;
+  sa.N = N;
+  sa.K = K;
+  sa.kchunks = p.kchunks;
+  sa.per = p.per;
+  sa.cs = p.cs;
+  sa.alpha = w->alpha;
+  sa.y = y;
+  sa.acc = acc;
+  sa.status = dev->status;
+  const dim3 grid(static_cast<unsigned>(p.row_tiles * p.cs));
+  bitlinear_status st;
+  switch (p.bn) {
+    case 16: st = launch_ex(skinny_kernel<16>, grid, dim3(kSkThreads), p.smem, s, pdl, p.cs, mW, sa); break;
+    case 32: st = launch_ex(skinny_kernel<32>, grid, dim3(kSkThreads), p.smem, s, pdl, p.cs, mW, sa); break;
+    default: st = launch_ex(skinny_kernel<64>, grid, dim3(kSkThreads), p.smem, s, pdl, p.cs, mW, sa); break;
+  }
+  if (st == BITLINEAR_OK) t_last_kernel = p.bn == 16 ? "tc_skinny_bn16" : p.bn == 32 ? "tc_skinny_bn32" : "tc_skinny_bn64";
+  return st;
+}
+
 // Token-side scratch of the tensor-core path: the codes in contraction order,
 // gamma and the code sums.  One quantisation serves every matrix that
 // multiplies the same x.
@@ -351,7 +451,7 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
 }
 
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
-                         cudaStream_t s, DeviceState* dev) {
+                         cudaStream_t s, DeviceState* dev, float qb = kQb) {
   const int N = w->N, K = w->K;
   const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? 1 : 2);
   const TcPlan plan = tc_plan(M, N, K, nm, dev->sm_count);
@@ -379,6 +479,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   ta.acc = acc;
   ta.nm_n = w->nm_n;
   ta.vbox = 0;
+  ta.qb = qb;
   ta.status = dev->status;
   ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
   if (nm == 0) {
@@ -405,15 +506,42 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   return st;
 }
 
+// H-BitLinear activations for the tensor-core GEMM: Hadamard transform and
+// 4-bit codes in contraction order (plus the split-K clearing of tc_quant).
+bitlinear_status hbit_quant(const uint16_t* x, int M, int K, int8_t* q, int ldq, bool permute, float* gamma,
+                            int32_t* rowsum, uint32_t* cnt, int ncnt, float* part, size_t part_words, bool pdl,
+                            cudaStream_t s) {
+  const int B = hbit_block(K);
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(B)));
+  const size_t vec4 = (part_words + 3) / 4;
+  const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * kHbitThreads - 1) / (4 * kHbitThreads)));
+  const size_t smem = static_cast<size_t>(K) * 4;
+  if (permute)
+    return launch(hbit_quant_kernel<true>, dim3(M + zblocks), dim3(kHbitThreads), smem, s, pdl, x, M, K, B, scale,
+                  ldq, q, gamma, rowsum, cnt, ncnt, part, vec4);
+  return launch(hbit_quant_kernel<false>, dim3(M + zblocks), dim3(kHbitThreads), smem, s, pdl, x, M, K, B, scale, ldq,
+                q, gamma, rowsum, cnt, ncnt, part, vec4);
+}
+
+// Activation quantisation feeding the tensor-core GEMM.
+enum class ActKind { kInt8, kInt8Norm, kHbit4 };
+
 bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
                             void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev,
-                            const float* gnorm = nullptr, float eps = 0.0f) {
+                            const float* gnorm = nullptr, float eps = 0.0f, ActKind act = ActKind::kInt8) {
   const int nm = w->nm_m == 0 ? 0 : (w->nm_m == 4 ? 1 : 2);
   if (!ws || ws_bytes < tc_workspace(M, w->N, w->K, nm, dev->sm_count) || !aligned16(ws))
     return BITLINEAR_ERR_WORKSPACE;
   const bool split = tc_plan(M, w->N, w->K, nm, dev->sm_count).ksplit > 1;
   const QuantWs qw = tc_ws_layout(ws, M, w->K, split ? dev->sm_count : 0, w->N);
-  bitlinear_status st = tc_quant(x, M, w->K, qw, pdl, s, gnorm, eps);
+  bitlinear_status st;
+  if (act == ActKind::kHbit4) {
+    st = hbit_quant(x, M, w->K, qw.q, static_cast<int>(k16(w->K)), true, qw.gamma, qw.rowsum,
+                    qw.ncnt > 0 ? qw.cnt : nullptr, qw.ncnt, qw.part, qw.part_words, pdl, s);
+    if (st != BITLINEAR_OK) return st;
+    return tc_gemm(w, M, qw, y, acc, s, dev, kQb4);
+  }
+  st = tc_quant(x, M, w->K, qw, pdl, s, act == ActKind::kInt8Norm ? gnorm : nullptr, eps);
   if (st != BITLINEAR_OK) return st;
   return tc_gemm(w, M, qw, y, acc, s, dev);
 }
@@ -623,10 +751,12 @@ bitlinear_status check_matrix(const bitlinear_weights* w, const uint16_t* y, con
 
 bitlinear_status check_flags(uint32_t flags, int M) {
   const uint32_t known = BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_GEMV | BITLINEAR_FLAG_PATH_TC |
-                         BITLINEAR_FLAG_DECODE_LUT;
+                         BITLINEAR_FLAG_DECODE_LUT | BITLINEAR_FLAG_PATH_PERSISTENT;
   if (flags & ~known) return BITLINEAR_ERR_FLAGS;
   if ((flags & BITLINEAR_FLAG_PATH_GEMV) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
   if ((flags & BITLINEAR_FLAG_DECODE_LUT) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
+  if ((flags & BITLINEAR_FLAG_PATH_PERSISTENT) && (flags & (BITLINEAR_FLAG_PATH_GEMV | BITLINEAR_FLAG_DECODE_LUT)))
+    return BITLINEAR_ERR_FLAGS;
   return BITLINEAR_OK;
 }
 
@@ -646,6 +776,10 @@ bitlinear_status forward_common(const bitlinear_weights* w, const uint16_t* x, i
   const bool pdl = (flags & BITLINEAR_FLAG_PDL) != 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || M > 1;
+  if (tc && w->nm_m == 0 && !(flags & BITLINEAR_FLAG_PATH_PERSISTENT)) {
+    const SkPlan p = sk_plan(M, w->N, w->K, dev);
+    if (p.ok) return skinny_launch(w, x, M, y, acc, pdl, s, dev, p);
+  }
   if (tc) return forward_tc(w, x, M, y, acc, ws, ws_bytes, pdl, s, dev);
   if ((flags & BITLINEAR_FLAG_DECODE_LUT) && want_nm) return BITLINEAR_ERR_FLAGS;
   return forward_gemv(w, x, y, acc, pdl, s, dev, (flags & BITLINEAR_FLAG_DECODE_LUT) != 0);
@@ -870,7 +1004,39 @@ bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16
     // decode: every GEMV CTA normalises and quantises the token itself
     return gemv_dense_launch(&w, &y, &acc, 1, x, pdl, s, dev, g, eps);
   }
-  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, pdl, s, dev, g, eps);
+  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, pdl, s, dev, g, eps, ActKind::kInt8Norm);
+}
+
+bitlinear_status bitlinear_hadamard_quant_act4(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* gamma,
+                                               int32_t* rowsum, void* stream) {
+  if (!x || !q || !gamma) return BITLINEAR_ERR_NULL;
+  if (M < 1 || M > BITLINEAR_MAX_M || K < 1 || K > BITLINEAR_HBIT_MAX_K) return BITLINEAR_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (reinterpret_cast<uintptr_t>(gamma) & 3u) ||
+      (rowsum && (reinterpret_cast<uintptr_t>(rowsum) & 3u)))
+    return BITLINEAR_ERR_ALIGN;
+  DeviceState* dev = nullptr;
+  bitlinear_status st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  st = hbit_quant(x, M, K, q, K, false, gamma, rowsum, nullptr, 0, nullptr, 0, false,
+                  static_cast<cudaStream_t>(stream));
+  if (st == BITLINEAR_OK) t_last_kernel = "hadamard_quant_act4";
+  return st;
+}
+
+bitlinear_status bitlinear_forward_hbit(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
+                                        int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                        void* stream) {
+  if (!w || !x || !y) return BITLINEAR_ERR_NULL;
+  bitlinear_status st = check_matrix(w, y, acc);
+  if (st != BITLINEAR_OK) return st;
+  if (M < 1 || M > BITLINEAR_MAX_M || w->K > BITLINEAR_HBIT_MAX_K) return BITLINEAR_ERR_SHAPE;
+  if (!aligned16(x)) return BITLINEAR_ERR_ALIGN;
+  if (flags & ~static_cast<uint32_t>(BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_TC)) return BITLINEAR_ERR_FLAGS;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, (flags & BITLINEAR_FLAG_PDL) != 0,
+                    static_cast<cudaStream_t>(stream), dev, nullptr, 0.0f, ActKind::kHbit4);
 }
 
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {

@@ -39,6 +39,7 @@
 // is the dense one.
 #pragma once
 #include "gemv.cuh"
+#include "hbit.cuh"
 
 namespace bl {
 
@@ -70,6 +71,7 @@ struct TcArgs {
   int vec_store;          // y / acc rows are 16-byte aligned and N % 8 == 0
   int nm_n;               // kept per 8-block (n:8 mode)
   int vbox;               // n:8: bytes of the values box per row
+  float qb;               // Q_b of the activation codes: 127 (8-bit), 7 (H-BitLinear 4-bit)
   int32_t* status;        // device status word
 };
 
@@ -418,7 +420,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int tile = rt * a.tok_tiles + tt;
         for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
           const int tok = tok0 + j;
-          scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), kQb) : 0.0f;  // RN(RN(alpha gamma) / 127)
+          scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), a.qb) : 0.0f;  // RN(RN(alpha gamma) / Q_b)
           rsm[j] = tok < a.M ? a.rowsum[tok] : 0;
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -492,7 +494,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
         const int tok = tok0 + j;
-        scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), kQb) : 0.0f;  // RN(RN(alpha gamma) / 127)
+        scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), a.qb) : 0.0f;  // RN(RN(alpha gamma) / Q_b)
         rsm[j] = tok < a.M ? a.rowsum[tok] : 0;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");

@@ -210,3 +210,18 @@ def test_layout_version_matches_header(L):
     assert L.bitlinear_layout_version() == int(m.group(1))
     import ternary_weight_linear_fwd_b200 as bl
     assert bl.layout_version() == int(m.group(1))
+
+
+def test_hbit_host_checks(L):
+    """H-BitLinear argument errors come back before any device work (fake addresses)."""
+    fh = L.bitlinear_forward_hbit
+    x, y = 0x30000, 0x40000
+    assert fh(None, x, 1, y, None, None, 0, 0, None) == 1
+    assert fh(ctypes.byref(_w(L, K=16385)), x, 1, y, None, None, 0, 0, None) == 2   # above the transform limit
+    assert fh(ctypes.byref(_w(L)), x, 0, y, None, None, 0, 0, None) == 2
+    assert fh(ctypes.byref(_w(L)), x + 4, 1, y, None, None, 0, 0, None) == 3
+    assert fh(ctypes.byref(_w(L)), x, 1, y, None, None, 0, 0x2, None) == 8          # no GEMV path
+    hq = L.bitlinear_hadamard_quant_act4
+    assert hq(None, 4, 64, 0x1000, 0x2000, None, None) == 1
+    assert hq(0x1000, 4, 16385, 0x1000, 0x2000, None, None) == 2
+    assert hq(0x1001, 4, 64, 0x1000, 0x2000, None, None) == 3

@@ -173,8 +173,46 @@ def test_forward_norm_gemv_gate_shape():
 def test_forward_tc_full(M, K, N):
     x, Wt, a, w = _dense_case(M, K, N, seed=M * 7 + K)
     y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, flags=bl.FLAG_PATH_TC)
-    assert bl.last_kernel().startswith("tc_gemm") and "dense" in bl.last_kernel()
+    assert bl.last_kernel().startswith(("tc_gemm_dense", "tc_skinny"))
     _check_rows(x, Wt, a, y, acc, np.arange(M))
+    y2, acc2 = bl.forward(w, to_dev_bf16(x), want_acc=True, flags=bl.FLAG_PATH_TC | bl.FLAG_PATH_PERSISTENT)
+    assert bl.last_kernel().startswith("tc_gemm_dense")
+    assert torch.equal(acc, acc2) and torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+# The fused few-token kernel: token tiles of 16, 32 and 64; one to eight K slices per cluster (2560 -> 6912:
+# two; 6912 -> 2560: seven or fewer; 11008 -> 2048: eight); a ragged K (203: a partial 16-group and chunk)
+# and N (130, 1, 33); the forced tensor-core path at M = 1.  Every output is checked against the oracle and
+# against the persistent GEMM bit for bit.
+@pytest.mark.parametrize("M,K,N", [(2, 256, 512), (16, 2560, 6912), (16, 6912, 2560), (16, 2560, 640),
+                                   (32, 2560, 2560), (64, 2560, 6912), (33, 203, 130), (5, 11008, 2048),
+                                   (64, 2048, 11008), (9, 1000, 1), (17, 384, 33), (1, 2560, 6912)])
+def test_forward_skinny(M, K, N):
+    x, Wt, a, w = _dense_case(M, K, N, seed=M * 11 + K + N, ternary=(K, N) in ((2560, 6912), (6912, 2560)))
+    xd = to_dev_bf16(x)
+    y, acc = bl.forward(w, xd, want_acc=True, flags=bl.FLAG_PATH_TC if M == 1 else 0)
+    assert bl.last_kernel().startswith("tc_skinny"), bl.last_kernel()
+    _check_rows(x, Wt, a, y, acc, np.arange(M))
+    y2, acc2 = bl.forward(w, xd, want_acc=True, flags=bl.FLAG_PATH_TC | bl.FLAG_PATH_PERSISTENT)
+    assert torch.equal(acc, acc2) and torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    y3 = bl.forward(w, xd, flags=bl.FLAG_PDL | (bl.FLAG_PATH_TC if M == 1 else 0))  # no acc, programmatic launch
+    assert torch.equal(y.view(torch.int16), y3.view(torch.int16))
+
+
+def test_forward_skinny_zero_and_outlier_tokens():
+    """A zero token, a single huge outlier and a constant token in one few-token call."""
+    M, K, N = 12, 2560, 640
+    x = synth.activations(M, K, seed=13)
+    x[3] = 0
+    x[5, 1234] = synth.to_bf16_bits(np.array([3.0e4], np.float32))[0]
+    x[7] = synth.to_bf16_bits(np.full(K, -0.75, np.float32))
+    W = synth.latent_weights(N, K, seed=13)
+    ref = oracle.pack_weights(W)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV))
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+    assert bl.last_kernel().startswith("tc_skinny")
+    _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
+    assert not bf16_bits(y)[3].any()
 
 
 @pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560), (2560, 2560), (2560, 640)])
@@ -221,7 +259,8 @@ def test_forward_stale_workspace():
                     device=DEV)
     for M, K, N in cases:
         x, Wt, a, w = _dense_case(M, K, N, seed=M + N)
-        y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, workspace=ws)
+        y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, workspace=ws, flags=bl.FLAG_PATH_PERSISTENT)
+        assert bl.last_kernel().startswith("tc_gemm_dense")
         _check_rows(x, Wt, a, y, acc, np.arange(M))
         ws.fill_(0xFF)
 

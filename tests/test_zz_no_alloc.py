@@ -52,23 +52,23 @@ def _case(M, K, N, seed, n=0, m=0):
     return w, xd, x, ref
 
 
-def _noalloc(L, w, xd):
+def _noalloc(L, w, xd, flags=0):
     M = xd.shape[0]
     y = torch.empty((M, w.N), dtype=torch.bfloat16, device=DEV)
     acc = torch.empty((M, w.N), dtype=torch.int32, device=DEV)
     ws = w.c_struct()
-    st = L.bitlinear_forward_noalloc(ctypes.byref(ws), xd.data_ptr(), M, y.data_ptr(), acc.data_ptr(), 0,
+    st = L.bitlinear_forward_noalloc(ctypes.byref(ws), xd.data_ptr(), M, y.data_ptr(), acc.data_ptr(), flags,
                                      torch.cuda.current_stream().cuda_stream)
     assert st == 0, L.bitlinear_status_string(st)
     return y, acc
 
 
-def _check(L, fwd, M, K, N, seed, n, m):
+def _check(L, fwd, M, K, N, seed, n, m, flags):
     """The no-allocation call equals the workspace call bit for bit (same kernels, same inputs) and the
     oracle within the parity tolerance (accumulators exact, outputs within one bf16 ulp)."""
     w, xd, x, ref = _case(M, K, N, seed, n, m)
-    y_ref, acc_ref = fwd(w, xd, want_acc=True)
-    y, acc = _noalloc(L, w, xd)
+    y_ref, acc_ref = fwd(w, xd, want_acc=True, flags=flags)
+    y, acc = _noalloc(L, w, xd, flags)
     torch.cuda.synchronize()
     assert torch.equal(acc, acc_ref)
     assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
@@ -78,15 +78,20 @@ def _check(L, fwd, M, K, N, seed, n, m):
     assert d.max() <= 1  # one bf16 ulp, the tolerance of every forward parity test
 
 
-# Two or three calls in a row with different inputs and shapes, each reusing the scratch the previous
-# call left behind: a K-split tensor-core GEMM (few weight-row tiles), a tile-parallel one with a
-# different M x N, and the M = 1 decode GEMV, which uses no scratch.
+# Calls in a row with different inputs and shapes, each reusing the scratch the previous call left
+# behind: a K-split persistent tensor-core GEMM (few weight-row tiles), a tile-parallel one with a
+# different M x N, the K-split one again, the fused few-token kernel and the M = 1 decode GEMV (these
+# two use no scratch).
+P = bl.FLAG_PATH_PERSISTENT
+
+
 @pytest.mark.parametrize("n,m", [(0, 0), (6, 8)])
 def test_noalloc_matches_workspace_forward_twice(n, m):
     L = _lib()
     fwd = bl.forward_nm if m else bl.forward
-    for (M, K, N, seed) in ((64, 2560, 640, 2), (300, 512, 2048, 1), (64, 2560, 640, 3), (1, 2560, 1000, 4)):
-        _check(L, fwd, M, K, N, seed, n, m)
+    for (M, K, N, seed, flags) in ((64, 2560, 640, 2, P), (300, 512, 2048, 1, P), (64, 2560, 640, 3, P),
+                                   (16, 2560, 640, 5, 0), (1, 2560, 1000, 4, 0)):
+        _check(L, fwd, M, K, N, seed, n, m, flags)
     assert bl.device_status() == 0
 
 
