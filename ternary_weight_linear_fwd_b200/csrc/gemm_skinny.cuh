@@ -27,7 +27,9 @@
 // exact integer contraction, the same rescale.  No global workspace, atomic
 // or second launch is involved.  Every mbarrier wait is bounded; every thread
 // passes every cluster barrier (roles that give up skip work, never the
-// barriers), so a timeout cannot leave a CTA of the cluster waiting forever.
+// barriers), so a timeout cannot leave a CTA of the cluster waiting forever;
+// a CTA whose role gave up raises a flag that every CTA of the cluster reads
+// before storing, so no partial result is written.
 #pragma once
 #include "gemm_tc.cuh"
 
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   uint64_t* afree = aready + SA;                                          // [SA]
   uint64_t* accfull = afree + SA;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+  uint32_t* s_fail = tmem_slot + 1;  // nonzero: a role of this CTA gave up on a wait
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -107,6 +110,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       mbar_init(&afree[i], 1);
     }
     mbar_init(accfull, 1);
+    *s_fail = 0u;
     fence_mbar_init();
     tma_prefetch_desc(&mapW);
     // the weights do not depend on the preceding kernel: every chunk of the slice now
@@ -125,6 +129,9 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The first access to another CTA's shared memory must follow a cluster barrier
+  // (every CTA of the cluster running); its wait comes just before that access.
+  cluster_arrive_relaxed();
 
   // ------------------------------------------------ quantisation of this CTA's K slice
   pdl_wait_primary();  // x may come from the preceding kernel
@@ -145,6 +152,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   uint32_t mb = __float_as_uint(mx);  // |x| >= 0: bit patterns order like the values
 #pragma unroll
   for (int o = TPT / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+  cluster_wait();
   if (sub == 0) {
     const uint32_t local = smem_u32(&sPmax[rank * BN + t]);
     for (int p = 0; p < a.cs; ++p) st_cluster_u32(mapa_shared(local, static_cast<uint32_t>(p)), mb);
@@ -187,6 +195,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
         const int sl = c % SA;
         if (!mbar_wait(&aready[sl], (c / SA) & 1)) {
           *a.status = kDevTimeoutMma;
+          *s_fail = 1u;
           break;
         }
         tc_fence_after();
@@ -212,6 +221,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       const int sl = c % SA;
       if ((c >= SA && !mbar_wait(&afree[sl], ((c / SA) - 1) & 1)) || !mbar_wait(&full[c], 0)) {
         *a.status = kDevTimeoutUnpack;
+        *s_fail = 1u;
         break;
       }
       const uint4 lo = *reinterpret_cast<const uint4*>(sW + c * kSkChunkBytes + r * 32);
@@ -230,7 +240,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
     }
     if (warp < 8) {
       // epilogue part 1: this CTA's partial tile minus its slice's code sums
-      if (!mbar_wait(accfull, 0)) *a.status = kDevTimeoutEpilogue;
+      if (!mbar_wait(accfull, 0)) {
+        *a.status = kDevTimeoutEpilogue;
+        *s_fail = 1u;
+      }
       tc_fence_after();
 #pragma unroll
       for (int cb = 0; cb < (BN + 31) / 32; ++cb) {
@@ -250,7 +263,9 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   const int band = ((kTcRows + a.cs - 1) / a.cs + 3) & ~3;  // rows per CTA, a multiple of 4
   const int rb = static_cast<int>(rank) * band;
   const int re = min(kTcRows, rb + band);
-  const int quads = re > rb ? (re - rb) / 4 : 0;
+  int quads = re > rb ? (re - rb) / 4 : 0;
+  for (int p = 0; p < a.cs; ++p)  // a partial tile of a CTA that gave up is not a result: store nothing
+    if (ld_cluster_u32(mapa_shared(smem_u32(s_fail), static_cast<uint32_t>(p))) != 0u) quads = 0;
   for (int it = threadIdx.x; it < BN * quads; it += kSkThreads) {
     const int tok = it / quads;
     const int rq = rb + 4 * (it - tok * quads);

@@ -77,12 +77,12 @@ def _pack(L, W, n, m):
 
 
 def _call(L, w, xd, flags=0):
-    N = w.N
-    y = torch.full((1, N), -1, dtype=torch.int16, device=DEV)  # 0xFFFF: a NaN pattern no output has
-    acc = torch.full((1, N), -(2 ** 31), dtype=torch.int32, device=DEV)
+    M, N = xd.shape[0], w.N
+    y = torch.full((M, N), -1, dtype=torch.int16, device=DEV)  # 0xFFFF: a NaN pattern no output has
+    acc = torch.full((M, N), -(2 ** 31), dtype=torch.int32, device=DEV)
     ws = w.c_struct()
     fn = L.bitlinear_forward_nm if w.nm_m else L.bitlinear_forward
-    assert fn(ctypes.byref(ws), xd.data_ptr(), 1, y.data_ptr(), acc.data_ptr(), None, 0, flags, _stream()) == 0
+    assert fn(ctypes.byref(ws), xd.data_ptr(), M, y.data_ptr(), acc.data_ptr(), None, 0, flags, _stream()) == 0
     torch.cuda.synchronize()
     return y.cpu().numpy().view(np.uint16), acc.cpu().numpy()
 
@@ -106,6 +106,33 @@ def test_gemv_gives_up_records_status_and_recovers(T, n, m, flags):
 
     assert T.bitlinear_test_set_wait_fault(PRODUCT_WAIT_NS, 0) == 0
     y, acc = _call(T, w, xd, flags)
+    assert _status(T) == 0
+    np.testing.assert_array_equal(acc, acc_ref)
+    d = np.abs(y.astype(np.int32) - y_ref.astype(np.int32))
+    assert d.max() <= 1
+
+
+def test_few_token_kernel_gives_up_records_status_and_recovers(T):
+    """The fused few-token tensor-core kernel (K split over a cluster): its weight chunks are told to
+    expect more bytes than arrive, the unpack warps and the MMA issuer give up, every CTA still passes
+    the cluster barriers, and since some CTA of each cluster gave up none stores a result."""
+    M, K, N = 8, 2560, 700
+    x = synth.activations(M, K, seed=77)
+    W = synth.latent_weights(N, K, seed=78)
+    ref = oracle.pack_weights(W)
+    y_ref, acc_ref, *_ = oracle.forward(x, ref["Wt"], ref["alpha"])
+    w = _pack(T, W, 0, 0)
+    xd = torch.from_numpy(x.view(np.int16)).to(DEV).view(torch.bfloat16)
+    assert _status(T) == 0
+
+    assert T.bitlinear_test_set_wait_fault(SHORT_WAIT_NS, 16) == 0
+    y, acc = _call(T, w, xd)
+    code = _status(T)
+    assert code in (2, 3, 4, 5), code
+    assert np.all(y == 0xFFFF) and np.all(acc == -(2 ** 31))
+
+    assert T.bitlinear_test_set_wait_fault(PRODUCT_WAIT_NS, 0) == 0
+    y, acc = _call(T, w, xd)
     assert _status(T) == 0
     np.testing.assert_array_equal(acc, acc_ref)
     d = np.abs(y.astype(np.int32) - y_ref.astype(np.int32))
