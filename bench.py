@@ -403,8 +403,19 @@ def run_prefill(dev, iters: int, warmup: int):
             t_flush = time_chain_graph(dev, [lambda: flush.fill_(1)] * 10, 1, 3)
             times.append((t_both - t_flush) / 10)
         med = statistics.median(times)
+        # the activation quantisation alone (public bitlinear_quant_act: same kernel, natural k order), cold L2
+        q = torch.empty((PREFILL_M, K), dtype=torch.int8, device=dev)
+        gq = torch.empty(PREFILL_M, dtype=torch.float32, device=dev)
+        lib = bl.lib()
+        qcall = (lambda: lib.bitlinear_quant_act(xk.data_ptr(), PREFILL_M, K, q.data_ptr(), gq.data_ptr(), None,
+                                                 torch.cuda.current_stream(dev).cuda_stream))
+        t_qb = time_chain_graph(dev, [lambda: flush.fill_(1), qcall] * 10, 1, 3)
+        t_qf = time_chain_graph(dev, [lambda: flush.fill_(1)] * 10, 1, 3)
+        quant_us = (t_qb - t_qf) / 10 * 1e6
         ops = 2.0 * PREFILL_M * N * K
-        out[f"{K}x{N}"] = {"ms": med * 1e3, "tops": ops / med / 1e12}
+        out[f"{K}x{N}"] = {"ms": med * 1e3, "tops": ops / med / 1e12, "quant_alone_us": quant_us,
+                           "quant_alone_GBps": (3 * PREFILL_M * K + 8 * PREFILL_M) / (quant_us * 1e-6) / 1e9}
+        del q, gq
         tot_ops += ops
         tot_sec += med
     assert bl.device_status() == 0

@@ -490,10 +490,12 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
     int64_t ldv = 0, ldm = 0;
     if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
       return BITLINEAR_ERR_PATTERN;
-    const uint32_t vbox = nm == 1 ? 16u : static_cast<uint32_t>((4 * w->nm_n + 12 + 15) / 16 * 16);
+    const uint32_t vbox = nm == 1 ? static_cast<uint32_t>(16 * tc_ksub(1, bn))
+                                  : static_cast<uint32_t>((4 * w->nm_n + 12 + 15) / 16 * 16);
     ta.vbox = static_cast<int>(vbox);
     if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, false)) return BITLINEAR_ERR_CUDA;
-    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, static_cast<uint32_t>(16 * tc_ksub(nm, bn)), kTcRows, false))
+      return BITLINEAR_ERR_CUDA;
   }
   bitlinear_status st;
   if (nm == 0)

@@ -49,10 +49,10 @@ constexpr int kTcRows = 128;    // weight rows per tile (MMA M)
 constexpr int kTcThreads = 512;
 constexpr int kTcEpiWarp0 = 12;  // first epilogue warp
 
-// K elements per stage: dense weights with token tiles up to 128 take two
-// 128-wide sub-tiles (eight MMAs per barrier round trip, which halves the fixed
-// cost of a stage per MAC); wider tiles and N:M weights keep one.
-__host__ __device__ constexpr int tc_ksub(int NM, int BN) { return (NM == 0 && BN <= 128) ? 2 : 1; }
+// K elements per stage: dense and 2:4 weights with token tiles up to 128 take
+// two 128-wide sub-tiles (eight MMAs per barrier round trip, which halves the
+// fixed cost of a stage per MAC); wider tiles and n:8 weights keep one.
+__host__ __device__ constexpr int tc_ksub(int NM, int BN) { return (NM <= 1 && BN <= 128) ? 2 : 1; }
 __host__ __device__ constexpr int tc_bk(int NM, int BN) { return kTcSubK * tc_ksub(NM, BN); }
 
 struct TcArgs {
@@ -79,9 +79,9 @@ template <int NM, int BN>
 struct TcStageBytes {
   // packed A bytes per stage (TMA box bytes, rows = 128)
   static __host__ __device__ constexpr int a_values(int vbox) {
-    return NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox);
+    return NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 * tc_ksub(1, BN) : kTcRows * vbox);
   }
-  static __host__ __device__ constexpr int a_meta() { return NM == 0 ? 0 : kTcRows * 16; }
+  static __host__ __device__ constexpr int a_meta() { return NM == 0 ? 0 : kTcRows * 16 * tc_ksub(NM, BN); }
 };
 
 __host__ __device__ constexpr int tc_dcols(int BN) { return BN < 32 ? 32 : BN; }  // TMEM columns of one accumulator
@@ -103,8 +103,8 @@ struct TcCols {
 };
 
 __host__ __device__ constexpr int tc_a_stage_bytes(int NM, int BN, int vbox) {
-  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 : kTcRows * vbox)) +
-          (NM == 0 ? 0 : kTcRows * 16) + 1023) / 1024 * 1024;
+  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 * tc_ksub(1, BN) : kTcRows * vbox)) +
+          (NM == 0 ? 0 : kTcRows * 16 * tc_ksub(NM, BN)) + 1023) / 1024 * 1024;
 }
 
 __host__ __device__ constexpr int tc_smem_bytes(int BN, int NM, int vbox) {
@@ -219,8 +219,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (NM == 0) {
           tma_load_2d(dst, &mapA, kb * 32 * KSUB, row0, &full[s]);
         } else if (NM == 1) {
-          tma_load_2d(dst, &mapA, kb * 16, row0, &full[s]);
-          tma_load_2d(dst + a_val_bytes, &mapMeta, kb * 16, row0, &full[s]);
+          tma_load_2d(dst, &mapA, kb * 16 * KSUB, row0, &full[s]);
+          tma_load_2d(dst + a_val_bytes, &mapMeta, kb * 16 * KSUB, row0, &full[s]);
         } else {
           tma_load_2d(dst, &mapA, (kb * 4 * a.nm_n) & ~15, row0, &full[s]);
           tma_load_2d(dst + a_val_bytes, &mapMeta, kb * 16, row0, &full[s]);
@@ -318,12 +318,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const uint8_t* st = sA + s * a_stage;
       const uint8_t* arow;
-      const uint8_t* mrow = st + a_val_bytes + r * 16;
+      const uint8_t* mrow = st + a_val_bytes + r * 16 * KSUB;
       int rem = 0;
       if (NM == 0)
         arow = st + r * 32 * KSUB;
       else if (NM == 1)
-        arow = st + r * 16;
+        arow = st + r * 16 * KSUB;
       else {
         arow = st + r * a.vbox;
         rem = (kb * 4 * a.nm_n) & 15;
@@ -337,9 +337,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           dw[0] = lo.x; dw[1] = lo.y; dw[2] = lo.z; dw[3] = lo.w;
           dw[4] = hi.x; dw[5] = hi.y; dw[6] = hi.z; dw[7] = hi.w;
         } else if (NM == 1) {
-          // 16 bytes of kept codes and 16 of metadata per row: 8 groups of 16 weights
-          const uint4 vv = *reinterpret_cast<const uint4*>(arow);
-          const uint4 mm = *reinterpret_cast<const uint4*>(mrow);
+          // 16 bytes of kept codes and 16 of metadata per row and sub-tile: 8 groups of 16 weights
+          const uint4 vv = reinterpret_cast<const uint4*>(arow)[sub];
+          const uint4 mm = reinterpret_cast<const uint4*>(mrow)[sub];
           const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w}, mw[4] = {mm.x, mm.y, mm.z, mm.w};
           const uint32_t* lut_lane = s_lut + lane;
 #pragma unroll

@@ -359,35 +359,35 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   const bool landed = mbar_wait(&s_bar, 0);
 
   if (landed) {
-    // units (chunk, row pair), row pair fastest: the lanes of a warp read one
-    // activation chunk (one shared-memory broadcast) for up to 64 rows
-    const int nthr = blockDim.x;
-    const int half = (nrows + 1) >> 1;  // pair p covers rows p and p + half
-    const int total = half * C;
-    const int dq = nthr / half, dr = nthr % half;
-    int ch = threadIdx.x / half, p = threadIdx.x % half;
-    for (int u = threadIdx.x; u < total; u += nthr) {
+    // Thread (seg, p) takes row pair p (rows p and p + half) over the chunks of
+    // segment seg and keeps the partial sums in registers; consecutive threads
+    // take consecutive pairs of one segment, so a warp's lanes read one
+    // activation chunk (a shared-memory broadcast) and conflict-free weight
+    // slots.  Each partial sum s_j carries the factor 4^j of its bit plane and
+    // stays below 2 * 64 * 127 * K / 4 < 2^31, so the final shifts are exact.
+    const int half = (nrows + 1) >> 1;  // rows_box <= 256: at most 128 pairs, at least 4 segments
+    const int nseg = blockDim.x / half;
+    const int seg = threadIdx.x / half, p = threadIdx.x - seg * half;
+    if (seg < nseg) {
+      const int c_beg = seg * C / nseg, c_end = (seg + 1) * C / nseg;
       const int r2 = p + half < nrows ? p + half : p;  // an odd last pair reads row p twice
-      const uint4 wa = gemv_wchunk(s_w, stripe_bytes, p, ch);
-      const uint4 wb = gemv_wchunk(s_w, stripe_bytes, r2, ch);
-      const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
       int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
-      dot_word(wa.x, q0.x, q0.y, q0.z, q0.w, a0, a1, a2, a3);
-      dot_word(wb.x, q0.x, q0.y, q0.z, q0.w, b0, b1, b2, b3);
-      dot_word(wa.y, q1.x, q1.y, q1.z, q1.w, a0, a1, a2, a3);
-      dot_word(wb.y, q1.x, q1.y, q1.z, q1.w, b0, b1, b2, b3);
-      dot_word(wa.z, q2.x, q2.y, q2.z, q2.w, a0, a1, a2, a3);
-      dot_word(wb.z, q2.x, q2.y, q2.z, q2.w, b0, b1, b2, b3);
-      dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
-      dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
-      // every partial sum s_j is a multiple of 4^j, so the shifts are exact
-      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6));
-      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6));
-      p += dr;
-      ch += dq;
-      if (p >= half) {
-        p -= half;
-        ++ch;
+      for (int ch = c_beg; ch < c_end; ++ch) {
+        const uint4 wa = gemv_wchunk(s_w, stripe_bytes, p, ch);
+        const uint4 wb = gemv_wchunk(s_w, stripe_bytes, r2, ch);
+        const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
+        dot_word(wa.x, q0.x, q0.y, q0.z, q0.w, a0, a1, a2, a3);
+        dot_word(wb.x, q0.x, q0.y, q0.z, q0.w, b0, b1, b2, b3);
+        dot_word(wa.y, q1.x, q1.y, q1.z, q1.w, a0, a1, a2, a3);
+        dot_word(wb.y, q1.x, q1.y, q1.z, q1.w, b0, b1, b2, b3);
+        dot_word(wa.z, q2.x, q2.y, q2.z, q2.w, a0, a1, a2, a3);
+        dot_word(wb.z, q2.x, q2.y, q2.z, q2.w, b0, b1, b2, b3);
+        dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
+        dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
+      }
+      if (c_end > c_beg) {
+        atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6));
+        if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6));
       }
     }
   }
