@@ -360,6 +360,7 @@ SkPlan sk_plan(int M, int N, int K, DeviceState* dev) {
   }
   p.per = (p.kchunks + cs - 1) / cs;
   p.cs = (p.kchunks + p.per - 1) / p.per;  // no empty slice
+  if (sk_band_rows(p.cs, p.cs - 1) <= 0) return p;  // every CTA owns some rows of the tile
   p.smem = std::max(sk_smem_bytes(p.bn, p.per), kSkMinSmem);
   if (sk_active_clusters(dev, p.cs, p.smem) <= 0) return p;  // this cluster size cannot be launched here
   p.ok = true;
@@ -518,11 +519,20 @@ bitlinear_status hbit_quant(const uint16_t* x, int M, int K, int8_t* q, int ldq,
   const size_t vec4 = (part_words + 3) / 4;
   const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * kHbitThreads - 1) / (4 * kHbitThreads)));
   const size_t smem = static_cast<size_t>(K) * 4;
-  if (permute)
-    return launch(hbit_quant_kernel<true>, dim3(M + zblocks), dim3(kHbitThreads), smem, s, pdl, x, M, K, B, scale,
-                  ldq, q, gamma, rowsum, cnt, ncnt, part, vec4);
-  return launch(hbit_quant_kernel<false>, dim3(M + zblocks), dim3(kHbitThreads), smem, s, pdl, x, M, K, B, scale, ldq,
-                q, gamma, rowsum, cnt, ncnt, part, vec4);
+  const dim3 grid(static_cast<unsigned>(M + zblocks)), block(kHbitThreads);
+  auto go = [&](auto kern) {
+    return launch(kern, grid, block, smem, s, pdl, x, M, K, B, scale, ldq, q, gamma, rowsum, cnt, ncnt, part, vec4);
+  };
+  switch (hbit_vals_per_lane(B)) {
+    case 1: return permute ? go(hbit_quant_kernel<true, 1>) : go(hbit_quant_kernel<false, 1>);
+    case 2: return permute ? go(hbit_quant_kernel<true, 2>) : go(hbit_quant_kernel<false, 2>);
+    case 4: return permute ? go(hbit_quant_kernel<true, 4>) : go(hbit_quant_kernel<false, 4>);
+    case 8: return permute ? go(hbit_quant_kernel<true, 8>) : go(hbit_quant_kernel<false, 8>);
+    case 16: return permute ? go(hbit_quant_kernel<true, 16>) : go(hbit_quant_kernel<false, 16>);
+    case 32: return permute ? go(hbit_quant_kernel<true, 32>) : go(hbit_quant_kernel<false, 32>);
+    case 64: return permute ? go(hbit_quant_kernel<true, 64>) : go(hbit_quant_kernel<false, 64>);
+    default: return permute ? go(hbit_quant_kernel<true, 0>) : go(hbit_quant_kernel<false, 0>);
+  }
 }
 
 // Activation quantisation feeding the tensor-core GEMM.

@@ -8,28 +8,28 @@
 // and one slice of K, and
 //   1. hands all of its packed weight chunks (128 rows x 128 k, 4 KB each) to
 //      the tensor-copy engine at once, before waiting on the preceding kernel;
-//   2. quantises its K slice of every token: the per-token maximum of the
-//      slice goes to every CTA of the cluster (st.shared::cluster), one
-//      cluster barrier, gamma = the maximum over the cluster, and the codes go
+//   2. quantises its K slice of every token: the slice's per-token maximum is
+//      stored into every CTA of the cluster (st.shared::cluster) followed by a
+//      remote mbarrier arrive with release semantics; each CTA waits on its own
+//      barrier, takes gamma = the maximum over the cluster and writes the codes
 //      straight into the 128-byte-swizzled K-major B operand in shared memory
 //      (contraction order inside each 16-group, as the A unpack produces);
 //   3. expands each weight chunk to u8 codes in tensor memory (three groups of
-//      four unpack warps, one chunk each in turn; seven A slots ring) and
-//      issues the chunk's four tcgen05.mma kind::i8 (M = 128 weight rows,
-//      N = BN tokens, K = 32) into one int32 accumulator;
-//   4. writes its partial accumulator tile minus its slice's code sums to
-//      shared memory; after a cluster barrier every CTA reduces a band of the
-//      tile's rows over all CTAs of the cluster (ld.shared::cluster), rescales
-//      by RN(RN(alpha * gamma) / 127) and stores bf16 (and int32 on request);
-//      a last cluster barrier keeps every CTA's shared memory alive until all
-//      the others have read it.
-// The result equals the persistent GEMM's bit for bit: the same codes, an
-// exact integer contraction, the same rescale.  No global workspace, atomic
-// or second launch is involved.  Every mbarrier wait is bounded; every thread
-// passes every cluster barrier (roles that give up skip work, never the
-// barriers), so a timeout cannot leave a CTA of the cluster waiting forever;
-// a CTA whose role gave up raises a flag that every CTA of the cluster reads
-// before storing, so no partial result is written.
+//      four unpack warps, one chunk each in turn; a ring of A slots) and issues
+//      the chunk's four tcgen05.mma kind::i8 (M = 128 weight rows, N = BN
+//      tokens, K = 32) into one int32 accumulator;
+//   4. reads its accumulator (tcgen05.ld), subtracts its slice's code sums and
+//      stores each row into the CTA that owns the row's band (rows are split
+//      in bands, one per CTA), then arrives remotely on that CTA's barrier;
+//      each CTA waits for its band from every CTA of the cluster, sums the
+//      slices in its own shared memory, rescales by RN(RN(alpha gamma) / 127)
+//      and stores bf16 (and int32 on request).
+// Only point-to-point signals cross CTAs (no cluster-wide barrier after the
+// start), every wait is a bounded mbarrier wait, and no CTA reads another's
+// shared memory, so a CTA may leave once its own band is done.  A CTA whose
+// role gave up on a wait sends a flag with its rows; a band that received one
+// is not stored.  The result equals the persistent GEMM's bit for bit: the
+// same codes, an exact integer contraction, the same rescale.
 #pragma once
 #include "gemm_tc.cuh"
 
@@ -47,10 +47,16 @@ constexpr size_t kSkMinSmem = 116 * 1024;
 
 __host__ __device__ constexpr int sk_dcols(int BN) { return BN <= 32 ? 32 : 64; }  // accumulator columns
 __host__ __device__ constexpr int sk_aslots(int BN) { return (kSkTmemCols - sk_dcols(BN)) / 32; }
+// Rows of the tile each CTA of a cluster of cs reduces and stores (a multiple of 4).
+__host__ __device__ constexpr int sk_band(int cs) { return ((kTcRows + cs - 1) / cs + 3) & ~3; }
+__host__ __device__ constexpr int sk_band_rows(int cs, int rank) {
+  return rank * sk_band(cs) >= kTcRows ? 0
+         : (kTcRows - rank * sk_band(cs) < sk_band(cs) ? kTcRows - rank * sk_band(cs) : sk_band(cs));
+}
 
 __host__ __device__ constexpr size_t sk_fixed_bytes(int BN) {
-  return 1024 /* alignment */ + static_cast<size_t>(BN) * kTcRows * 4 /* partial tile */ +
-         kSkMaxCluster * BN * 4 /* partial maxima */ + BN * 8 /* code sums, scales */ + 512 /* barriers */;
+  return 1024 /* alignment */ + static_cast<size_t>(160) * BN * 4 /* band staging: cs * band <= 160 rows */ +
+         kSkMaxCluster * BN * 4 /* partial maxima */ + BN * 8 /* code sums, scales */ + 768 /* flags, barriers */;
 }
 __host__ __device__ constexpr size_t sk_chunk_bytes(int BN) { return kSkChunkBytes + static_cast<size_t>(BN) * 128; }
 __host__ __device__ constexpr size_t sk_smem_bytes(int BN, int per) {
@@ -84,24 +90,30 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   // offset arithmetic on the shared array keeps every derived pointer in the shared window
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int per = a.per;
+  const int cs = a.cs;
+  const int band = sk_band(cs);
   uint8_t* sB = base;                                                     // [per][B_CHUNK]
   uint8_t* sW = sB + static_cast<size_t>(per) * B_CHUNK;                  // [per][128 rows x 32 B]
-  int32_t* sP = reinterpret_cast<int32_t*>(sW + static_cast<size_t>(per) * kSkChunkBytes);  // [BN][128]
-  uint32_t* sPmax = reinterpret_cast<uint32_t*>(sP + BN * kTcRows);      // [kSkMaxCluster][BN]
+  int32_t* sStage = reinterpret_cast<int32_t*>(sW + static_cast<size_t>(per) * kSkChunkBytes);  // [cs][band][BN]
+  uint32_t* sPmax = reinterpret_cast<uint32_t*>(sStage + 160 * BN);     // [kSkMaxCluster][BN]
   int32_t* sQsum = reinterpret_cast<int32_t*>(sPmax + kSkMaxCluster * BN);  // [BN]
   float* sScale = reinterpret_cast<float*>(sQsum + BN);                   // [BN]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sScale + BN);              // [kSkMaxChunks]
+  uint32_t* sFailIn = reinterpret_cast<uint32_t*>(sScale + BN);           // [kSkMaxCluster]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sFailIn + kSkMaxCluster);  // [kSkMaxChunks]
   uint64_t* aready = full + kSkMaxChunks;                                 // [SA]
   uint64_t* afree = aready + SA;                                          // [SA]
   uint64_t* accfull = afree + SA;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
-  uint32_t* s_fail = tmem_slot + 1;  // nonzero: a role of this CTA gave up on a wait
+  uint64_t* maxbar = accfull + 1;  // every CTA's per-token maxima have arrived
+  uint64_t* redbar = maxbar + 1;   // every CTA's rows of this CTA's band have arrived
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + 1);
+  uint32_t* s_fail = tmem_slot + 1;  // nonzero: a wait of this CTA gave up
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int row0 = static_cast<int>(blockIdx.x / a.cs) * kTcRows;
+  const int row0 = static_cast<int>(blockIdx.x / cs) * kTcRows;
   const int c0 = static_cast<int>(rank) * per;
   const int nch = max(0, min(per, a.kchunks - c0));
+  const int my_rows = sk_band_rows(cs, static_cast<int>(rank));
 
   if (threadIdx.x == 0) {
     for (int c = 0; c < nch; ++c) mbar_init(&full[c], 1);
@@ -110,6 +122,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       mbar_init(&afree[i], 1);
     }
     mbar_init(accfull, 1);
+    mbar_init(maxbar, static_cast<uint32_t>(cs * BN));
+    mbar_init(redbar, static_cast<uint32_t>(cs * (my_rows > 0 ? my_rows : 1)));
     *s_fail = 0u;
     fence_mbar_init();
     tma_prefetch_desc(&mapW);
@@ -129,8 +143,9 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // The first access to another CTA's shared memory must follow a cluster barrier
-  // (every CTA of the cluster running); its wait comes just before that access.
+  // The first access to another CTA's shared memory must follow a cluster
+  // barrier (every CTA of the cluster running, its barriers initialised); its
+  // wait comes just before that access.
   cluster_arrive_relaxed();
 
   // ------------------------------------------------ quantisation of this CTA's K slice
@@ -154,12 +169,15 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   for (int o = TPT / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
   cluster_wait();
   if (sub == 0) {
-    const uint32_t local = smem_u32(&sPmax[rank * BN + t]);
-    for (int p = 0; p < a.cs; ++p) st_cluster_u32(mapa_shared(local, static_cast<uint32_t>(p)), mb);
+    const uint32_t lmax = smem_u32(&sPmax[rank * BN + t]), lbar = smem_u32(maxbar);
+    for (int p = 0; p < cs; ++p) {
+      st_cluster_u32(mapa_shared(lmax, static_cast<uint32_t>(p)), mb);
+      mbar_arrive_remote(mapa_shared(lbar, static_cast<uint32_t>(p)));
+    }
   }
-  cluster_sync_all();  // 1: every CTA holds the partial maxima of the whole cluster
+  if (!mbar_wait_cluster(maxbar, 0)) *s_fail = 1u;
   uint32_t gb = 0u;
-  for (int p = 0; p < a.cs; ++p) gb = max(gb, sPmax[p * BN + t]);
+  for (int p = 0; p < cs; ++p) gb = max(gb, sPmax[p * BN + t]);
   const float gamma = __uint_as_float(gb);
   const float d = __fadd_rn(gamma, kEps);
   const float cq = __fmul_rn(kQb, __frcp_rn(d));
@@ -190,7 +208,6 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   if (warp == 1) {
     if (lane == 0) {
       // MMA issuer
-      bool issued = false;
       for (int c = 0; c < nch; ++c) {
         const int sl = c % SA;
         if (!mbar_wait(&aready[sl], (c / SA) & 1)) {
@@ -205,11 +222,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
           tc_mma_i8_ts(tmem, tmem + DC + sl * 32 + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), IDESC,
                        (c | kk) != 0 ? 1u : 0u);
         tc_commit(&afree[sl]);
-        issued = true;
       }
-      // completes once every MMA issued above has (also on the give-up path)
-      tc_commit(accfull);
-      (void)issued;
+      tc_commit(accfull);  // completes once every MMA issued above has (also after a give-up)
     }
   } else if (warp >= 4) {
     // unpack: group grp expands chunks grp, grp + 3, ... for the 32 rows of its lane quarter
@@ -239,58 +253,51 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       if (lane == 0) mbar_arrive(&aready[sl]);
     }
     if (warp < 8) {
-      // epilogue part 1: this CTA's partial tile minus its slice's code sums
+      // epilogue part 1: row r of this CTA's partial tile, minus the slice's code
+      // sums, goes to the CTA whose band holds the row
       if (!mbar_wait(accfull, 0)) {
         *a.status = kDevTimeoutEpilogue;
         *s_fail = 1u;
       }
       tc_fence_after();
+      const int p = r / band;
+      const uint32_t dst = mapa_shared(smem_u32(sStage + (static_cast<int>(rank) * band + (r - p * band)) * BN),
+                                       static_cast<uint32_t>(p));
 #pragma unroll
       for (int cb = 0; cb < (BN + 31) / 32; ++cb) {
         uint32_t v[32];
         tc_ld_32x32b_x32(tmem + lane_base + cb * 32, v);
         tc_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (cb * 32 + j < BN) sP[(cb * 32 + j) * kTcRows + r] = static_cast<int32_t>(v[j]) - sQsum[cb * 32 + j];
+        for (int j = 0; j < 32 && cb * 32 + j < BN; j += 4)
+          st_cluster_v4(dst + (cb * 32 + j) * 4, v[j] - sQsum[cb * 32 + j], v[j + 1] - sQsum[cb * 32 + j + 1],
+                        v[j + 2] - sQsum[cb * 32 + j + 2], v[j + 3] - sQsum[cb * 32 + j + 3]);
       }
+      st_cluster_u32(mapa_shared(smem_u32(&sFailIn[rank]), static_cast<uint32_t>(p)), *s_fail);
+      mbar_arrive_remote(mapa_shared(smem_u32(redbar), static_cast<uint32_t>(p)));
+    }
+  }
+
+  // ------------------------------------------------ this CTA's band: sum the slices, rescale, store
+  bool ok = my_rows > 0 && mbar_wait_cluster(redbar, 0);
+  if (!ok && my_rows > 0) *a.status = kDevTimeoutEpilogue;
+  for (int p = 0; p < cs && ok; ++p) ok = sFailIn[p] == 0u;
+  if (ok) {
+    const int rb = static_cast<int>(rank) * band;
+    for (int it = threadIdx.x; it < my_rows * a.M; it += kSkThreads) {
+      const int lr = it / a.M, tok = it - lr * a.M;
+      int32_t acc = 0;
+      for (int p = 0; p < cs; ++p) acc += sStage[(p * band + lr) * BN + tok];
+      const int n = row0 + rb + lr;
+      if (n >= a.N) continue;
+      const size_t o = static_cast<size_t>(tok) * a.N + n;
+      if (a.acc) a.acc[o] = acc;
+      const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(acc), sScale[tok]));
+      a.y[o] = *reinterpret_cast<const uint16_t*>(&h);
     }
   }
   tc_fence_before();
-  cluster_sync_all();  // 2: every partial tile of the cluster is written
-
-  // ------------------------------------------------ reduction over the cluster, rescale, store
-  const int band = ((kTcRows + a.cs - 1) / a.cs + 3) & ~3;  // rows per CTA, a multiple of 4
-  const int rb = static_cast<int>(rank) * band;
-  const int re = min(kTcRows, rb + band);
-  int quads = re > rb ? (re - rb) / 4 : 0;
-  for (int p = 0; p < a.cs; ++p)  // a partial tile of a CTA that gave up is not a result: store nothing
-    if (ld_cluster_u32(mapa_shared(smem_u32(s_fail), static_cast<uint32_t>(p))) != 0u) quads = 0;
-  for (int it = threadIdx.x; it < BN * quads; it += kSkThreads) {
-    const int tok = it / quads;
-    const int rq = rb + 4 * (it - tok * quads);
-    if (tok >= a.M) continue;
-    const uint32_t local = smem_u32(&sP[tok * kTcRows + rq]);
-    int32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-    for (int p = 0; p < a.cs; ++p) {
-      const uint4 v = ld_cluster_v4(mapa_shared(local, static_cast<uint32_t>(p)));
-      s0 += static_cast<int32_t>(v.x);
-      s1 += static_cast<int32_t>(v.y);
-      s2 += static_cast<int32_t>(v.z);
-      s3 += static_cast<int32_t>(v.w);
-    }
-    const int32_t sv[4] = {s0, s1, s2, s3};
-    const float sc = sScale[tok];
-    const size_t o = static_cast<size_t>(tok) * a.N + row0 + rq;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (row0 + rq + e >= a.N) break;
-      if (a.acc) a.acc[o + e] = sv[e];
-      const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(sv[e]), sc));
-      a.y[o + e] = *reinterpret_cast<const uint16_t*>(&h);
-    }
-  }
-  cluster_sync_all();  // 3: no CTA leaves while another still reads its shared memory
+  __syncthreads();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, kSkTmemCols);
