@@ -277,8 +277,10 @@ bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t
  * flags    as for bitlinear_forward; PDL applies to the first kernel the call
  *          launches (the later ones follow kernels of the same call).
  * Path: M == 1 runs the dense matrices in one GEMV launch (CTAs split among
- * them by rows) and each N:M matrix in its own; M >= 2 quantises once and
- * runs one tensor-core GEMM per matrix.
+ * them by rows) and each N:M matrix in its own; 2 <= M <= 64 with dense
+ * weights runs the fused few-token kernel once per matrix (see
+ * bitlinear_forward); otherwise the call quantises once and runs one
+ * persistent tensor-core GEMM per matrix.
  * Errors: as bitlinear_forward; SHAPE also for count out of range or unequal K. */
 bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,
                                          uint16_t* const* y, int32_t* const* acc, void* workspace,

@@ -816,6 +816,23 @@ bitlinear_status forward_group(const bitlinear_weights* w, int count, const uint
   const bool pdl = (flags & BITLINEAR_FLAG_PDL) != 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || M > 1;
+  if (tc && !(flags & BITLINEAR_FLAG_PATH_PERSISTENT)) {
+    // few tokens, dense weights: one fused launch per matrix (each quantises its own K slices)
+    SkPlan plans[BITLINEAR_MAX_GROUP];
+    bool all = true;
+    for (int i = 0; i < count && all; ++i) {
+      all = w[i].nm_m == 0;
+      if (all) {
+        plans[i] = sk_plan(M, w[i].N, w[i].K, dev);
+        all = plans[i].ok;
+      }
+    }
+    if (all) {
+      for (int i = 0; i < count && st == BITLINEAR_OK; ++i)
+        st = skinny_launch(&w[i], x, M, y[i], acc ? acc[i] : nullptr, i == 0 ? pdl : true, s, dev, plans[i]);
+      return st;
+    }
+  }
   if (tc) {
     size_t need = 0;
     bool split = false;

@@ -398,14 +398,18 @@ def test_forward_group_dense_matches_single_and_oracle(M, shapes):
         T = synth.ternary_weights(N, K, seed=40 + i)
         a = synth.alpha_uniform(40 + i)
         cases.append((T, np.float32(a), bl.pack_ternary(torch.from_numpy(T).to(DEV), float(a))))
-    outs = bl.forward_group([c[2] for c in cases], xd, want_acc=True)
-    if M == 1:
-        assert bl.last_kernel() == "gemv_m1_dense"
     rows = np.arange(M)
-    for (T, a, w), (y, acc) in zip(cases, outs):
-        y1, acc1 = bl.forward(w, xd, want_acc=True)
-        assert torch.equal(acc, acc1) and torch.equal(y.view(torch.int16), y1.view(torch.int16))
-        _check_rows(x, T, a, y, acc, rows)
+    # at M = 37 both the fused few-token launches and the quantise-once persistent path
+    for flags in ((0,) if M == 1 else (0, bl.FLAG_PATH_PERSISTENT)):
+        outs = bl.forward_group([c[2] for c in cases], xd, want_acc=True, flags=flags)
+        if M == 1:
+            assert bl.last_kernel() == "gemv_m1_dense"
+        else:
+            assert bl.last_kernel().startswith("tc_gemm_dense" if flags else "tc_skinny"), bl.last_kernel()
+        for (T, a, w), (y, acc) in zip(cases, outs):
+            y1, acc1 = bl.forward(w, xd, want_acc=True)
+            assert torch.equal(acc, acc1) and torch.equal(y.view(torch.int16), y1.view(torch.int16))
+            _check_rows(x, T, a, y, acc, rows)
 
 
 def test_forward_group_mixed_dense_nm():
