@@ -204,7 +204,8 @@ bitlinear_status launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaSt
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  if (smem > 48 * 1024 && !ensure_smem(reinterpret_cast<const void*>(kern), smem)) return BITLINEAR_ERR_CUDA;
+  // the 48 KB default covers static and dynamic shared memory together: opt in well below it
+  if (smem > 32 * 1024 && !ensure_smem(reinterpret_cast<const void*>(kern), smem)) return BITLINEAR_ERR_CUDA;
   return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 

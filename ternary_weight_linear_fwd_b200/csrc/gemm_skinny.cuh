@@ -9,8 +9,8 @@
 //   1. hands all of its packed weight chunks (128 rows x 128 k, 4 KB each) to
 //      the tensor-copy engine at once, before waiting on the preceding kernel;
 //   2. quantises its K slice of every token: the slice's per-token maximum is
-//      stored into every CTA of the cluster (st.shared::cluster) followed by a
-//      remote mbarrier arrive with release semantics; each CTA waits on its own
+//      stored into every CTA of the cluster (st.shared::cluster), then, after
+//      one cluster-scope fence, a remote mbarrier arrive; each CTA waits on its own
 //      barrier, takes gamma = the maximum over the cluster and writes the codes
 //      straight into the 128-byte-swizzled K-major B operand in shared memory
 //      (contraction order inside each 16-group, as the A unpack produces);
@@ -169,11 +169,12 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   for (int o = TPT / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
   cluster_wait();
   if (sub == 0) {
+    // all stores, one cluster-scope fence, then the arrives (each arrive with its
+    // own release would wait for the stores once per destination)
     const uint32_t lmax = smem_u32(&sPmax[rank * BN + t]), lbar = smem_u32(maxbar);
-    for (int p = 0; p < cs; ++p) {
-      st_cluster_u32(mapa_shared(lmax, static_cast<uint32_t>(p)), mb);
-      mbar_arrive_remote(mapa_shared(lbar, static_cast<uint32_t>(p)));
-    }
+    for (int p = 0; p < cs; ++p) st_cluster_u32(mapa_shared(lmax, static_cast<uint32_t>(p)), mb);
+    fence_cluster();
+    for (int p = 0; p < cs; ++p) mbar_arrive_remote_relaxed(mapa_shared(lbar, static_cast<uint32_t>(p)));
   }
   if (!mbar_wait_cluster(maxbar, 0)) *s_fail = 1u;
   uint32_t gb = 0u;

@@ -220,6 +220,13 @@ __global__ void __launch_bounds__(kHbitThreads) hbit_quant_kernel(const uint16_t
       w.z = cb[2] | (cb[6] << 8) | (cb[10] << 16) | (cb[14] << 24);
       w.w = cb[3] | (cb[7] << 8) | (cb[11] << 16) | (cb[15] << 24);
       *reinterpret_cast<uint4*>(qr + 16 * gi) = w;
+    } else if (16 * gi + 16 <= K && ((reinterpret_cast<uintptr_t>(qr) | (16u * gi)) & 15u) == 0) {
+      uint4 w;
+      w.x = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
+      w.y = cb[4] | (cb[5] << 8) | (cb[6] << 16) | (cb[7] << 24);
+      w.z = cb[8] | (cb[9] << 8) | (cb[10] << 16) | (cb[11] << 24);
+      w.w = cb[12] | (cb[13] << 8) | (cb[14] << 16) | (cb[15] << 24);
+      *reinterpret_cast<uint4*>(qr + 16 * gi) = w;
     } else {
       for (int i = 0; i < 16 && 16 * gi + i < K; ++i) qr[16 * gi + i] = static_cast<int8_t>(cb[i]);
     }
