@@ -176,7 +176,8 @@ GEMV_DEFS = ("gemv_dense_kernel", "quantise_row_smem", "quantise_row_smem_norm",
              "load8_raw", "sumsq8", "mbar_init", "mbar_arrive_expect_tx", "mbar_try_wait", "mbar_wait",
              "fence_mbar_init", "tma_prefetch_desc", "tma_load_2d_hint", "l2_policy_evict_first", "dp4a_us",
              "pdl_wait_primary", "pdl_launch_dependents", "smem_u32", "globaltimer_ns", "struct GemvDense",
-             "struct GemvMat", "row_code_sum", "gemv_gave_up", "wait_limit_ns", "test_extra_tx")
+             "struct GemvMat", "row_code_sum", "gemv_gave_up", "wait_limit_ns", "test_extra_tx",
+             "gemv_row_totals")
 
 
 def gemv_source_hash() -> str:

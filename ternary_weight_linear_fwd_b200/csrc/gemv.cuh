@@ -109,6 +109,21 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
   return mx;
 }
 
+// Row totals of the contraction from s_part[seg][row] (nseg segments of nrows
+// rows): warp w takes rows w, w + 16, ...; its lanes add the segments lane,
+// lane + 32, ... and a warp reduction finishes the row, so no row is summed by
+// one thread alone.  Calls store(row, total) on lane 0.
+template <typename Store>
+__device__ __forceinline__ void gemv_row_totals(const int32_t* s_part, int nseg, int nrows, Store&& store) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int r = warp; r < nrows; r += nw) {
+    int32_t t = 0;
+    for (int sg = lane; sg < nseg; sg += 32) t += s_part[sg * nrows + r];
+    t = __reduce_add_sync(0xffffffffu, t);
+    if (lane == 0) store(r, t);
+  }
+}
+
 // Sum of the per-warp code sums of quantise_row_smem.
 __device__ __forceinline__ int32_t row_code_sum(const int32_t* s_qparts) {
   int32_t t = 0;
@@ -402,12 +417,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     }
   }
   if (gemv_gave_up(landed, &s_bar, g.status)) return;
-  const int nseg_all = blockDim.x / ((nrows + 1) >> 1);
-  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) {
-    int32_t t = -row_code_sum(s_qparts);
-    for (int sg = 0; sg < nseg_all; ++sg) t += s_part[sg * nrows + rr];
-    gemv_store(mt.y, mt.acc, r0 + rr, t, s);
-  }
+  const int32_t qsum = row_code_sum(s_qparts);
+  gemv_row_totals(s_part, blockDim.x / ((nrows + 1) >> 1), nrows,
+                  [&](int rr, int32_t t) { gemv_store(mt.y, mt.acc, r0 + rr, t - qsum, s); });
 }
 
 // ------------------------------------------------------------------ dense M = 1, lookup tables
@@ -685,12 +697,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
     }
   }
   if (gemv_gave_up(landed, &s_bar, a.status)) return;
-  const int nseg_all = blockDim.x / ((nrows + 1) >> 1);
-  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) {
-    int32_t t = -row_code_sum(s_qparts);
-    for (int sg = 0; sg < nseg_all; ++sg) t += s_part[sg * nrows + rr];
-    gemv_store(a.y, a.acc, r0 + rr, t, s);
-  }
+  const int32_t qsum = row_code_sum(s_qparts);
+  gemv_row_totals(s_part, blockDim.x / ((nrows + 1) >> 1), nrows,
+                  [&](int rr, int32_t t) { gemv_store(a.y, a.acc, r0 + rr, t - qsum, s); });
 }
 
 }  // namespace bl
