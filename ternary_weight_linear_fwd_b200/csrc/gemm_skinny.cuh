@@ -8,18 +8,16 @@
 // and one slice of K, and
 //   1. hands all of its packed weight chunks (128 rows x 128 k, 4 KB each) to
 //      the tensor-copy engine at once, before waiting on the preceding kernel;
-//   2. quantises (warps 0..3) its K slice of every token: the slice's per-token maximum is
+//   2. quantises its K slice of every token: the slice's per-token maximum is
 //      stored into every CTA of the cluster (st.shared::cluster), then, after
 //      one cluster-scope fence, a remote mbarrier arrive; each CTA waits on its own
 //      barrier, takes gamma = the maximum over the cluster and writes the codes
 //      straight into the 128-byte-swizzled K-major B operand in shared memory
 //      (contraction order inside each 16-group, as the A unpack produces);
-//   3. meanwhile (warps 4..15, from the start: the weights do not depend on
-//      the preceding kernel) expands each weight chunk to u8 codes in tensor
-//      memory as it lands (three groups of four warps, one chunk each in turn;
-//      a ring of A slots); once the codes are written, one thread issues each
-//      chunk's four tcgen05.mma kind::i8 (M = 128 weight rows, N = BN tokens,
-//      K = 32) into one int32 accumulator;
+//   3. expands each weight chunk to u8 codes in tensor memory (three groups of
+//      four unpack warps, one chunk each in turn; a ring of A slots) and issues
+//      the chunk's four tcgen05.mma kind::i8 (M = 128 weight rows, N = BN
+//      tokens, K = 32) into one int32 accumulator;
 //   4. reads its accumulator (tcgen05.ld), subtracts its slice's code sums and
 //      stores each row into the CTA that owns the row's band (rows are split
 //      in bands, one per CTA), then arrives remotely on that CTA's barrier;
@@ -43,7 +41,6 @@ constexpr int kSkMaxChunks = 24;             // weight chunks per CTA, all resid
 constexpr int kSkMaxCluster = 8;             // portable cluster size
 constexpr int kSkGroups = 3;                 // unpack groups of four warps (warps 4 .. 15)
 constexpr int kSkTmemCols = 256;
-constexpr int kSkQuantThreads = 128;  // warps 0..3 quantise while warps 4..15 unpack the weights
 // Dynamic shared memory of at least this many bytes keeps one CTA per SM, so
 // the 256 TMEM columns a CTA allocates are always available to it.
 constexpr size_t kSkMinSmem = 116 * 1024;
@@ -84,7 +81,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   constexpr int DC = sk_dcols(BN);
   constexpr int SA = sk_aslots(BN);
   constexpr uint32_t IDESC = idesc_i8_u8s8(kTcRows, BN);
-  constexpr int TPT = kSkQuantThreads / BN;  // threads per token in the quantisation (8, 4 or 2 lanes)
+  constexpr int TPT = kSkThreads / BN;  // threads per token in the quantisation (32, 16 or 8 lanes)
   constexpr int B_CHUNK = BN * 128;     // one chunk of the B operand (BN rows x 128 bytes)
   static_assert(DC + SA * 32 <= kSkTmemCols, "TMEM budget");
   static_assert(B_CHUNK % 1024 == 0, "B chunks keep the 1024-byte swizzle alignment");
@@ -108,8 +105,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   uint64_t* accfull = afree + SA;
   uint64_t* maxbar = accfull + 1;  // every CTA's per-token maxima have arrived
   uint64_t* redbar = maxbar + 1;   // every CTA's rows of this CTA's band have arrived
-  uint64_t* qready = redbar + 1;   // the B tile, code sums and scales of this CTA are written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qready + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + 1);
   uint32_t* s_fail = tmem_slot + 1;  // nonzero: a wait of this CTA gave up
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,7 +124,6 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
     mbar_init(accfull, 1);
     mbar_init(maxbar, static_cast<uint32_t>(cs * BN));
     mbar_init(redbar, static_cast<uint32_t>(cs * (my_rows > 0 ? my_rows : 1)));
-    mbar_init(qready, 1);
     *s_fail = 0u;
     fence_mbar_init();
     tma_prefetch_desc(&mapW);
@@ -153,66 +148,66 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   // wait comes just before that access.
   cluster_arrive_relaxed();
 
-  if (warp < kSkQuantThreads / 32) {
-    // ---------------------------------------------- warps 0..3: quantisation of this CTA's K slice
-    pdl_wait_primary();  // x may come from the preceding kernel
-    const int t = threadIdx.x / TPT, sub = threadIdx.x % TPT;
-    const bool active = t < a.M;
-    const uint16_t* xr = a.x + static_cast<size_t>(active ? t : 0) * a.K;
-    const bool vec_ok = (a.K % 8) == 0;
-    const int gbeg = c0 * 8;                                    // first 16-group of the slice
-    const int gend = min((a.K + 15) / 16, (c0 + nch) * 8);      // groups holding some k < K
-    float mx = 0.0f;
-    if (active)
-      for (int g = gbeg + sub; g < gend; g += TPT) {
-        uint32_t r0[4], r1[4];
-        load8_raw(xr, 16 * g, a.K, vec_ok, r0);
-        load8_raw(xr, 16 * g + 8, a.K, vec_ok, r1);
-        mx = absmax8(r1, absmax8(r0, mx));
-      }
-    uint32_t mb = __float_as_uint(mx);  // |x| >= 0: bit patterns order like the values
+  // ------------------------------------------------ quantisation of this CTA's K slice
+  pdl_wait_primary();  // x may come from the preceding kernel
+  const int t = threadIdx.x / TPT, sub = threadIdx.x % TPT;
+  const bool active = t < a.M;
+  const uint16_t* xr = a.x + static_cast<size_t>(active ? t : 0) * a.K;
+  const bool vec_ok = (a.K % 8) == 0;
+  const int gbeg = c0 * 8;                                    // first 16-group of the slice
+  const int gend = min((a.K + 15) / 16, (c0 + nch) * 8);      // groups holding some k < K
+  float mx = 0.0f;
+  if (active)
+    for (int g = gbeg + sub; g < gend; g += TPT) {
+      uint32_t r0[4], r1[4];
+      load8_raw(xr, 16 * g, a.K, vec_ok, r0);
+      load8_raw(xr, 16 * g + 8, a.K, vec_ok, r1);
+      mx = absmax8(r1, absmax8(r0, mx));
+    }
+  uint32_t mb = __float_as_uint(mx);  // |x| >= 0: bit patterns order like the values
 #pragma unroll
-    for (int o = TPT / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-    cluster_wait();
-    if (sub == 0) {
-      // all stores, one cluster-scope fence, then the arrives (each arrive with its
-      // own release would wait for the stores once per destination)
-      const uint32_t lmax = smem_u32(&sPmax[rank * BN + t]), lbar = smem_u32(maxbar);
-      for (int p = 0; p < cs; ++p) st_cluster_u32(mapa_shared(lmax, static_cast<uint32_t>(p)), mb);
-      fence_cluster();
-      for (int p = 0; p < cs; ++p) mbar_arrive_remote_relaxed(mapa_shared(lbar, static_cast<uint32_t>(p)));
+  for (int o = TPT / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+  cluster_wait();
+  if (sub == 0) {
+    // all stores, one cluster-scope fence, then the arrives (each arrive with its
+    // own release would wait for the stores once per destination)
+    const uint32_t lmax = smem_u32(&sPmax[rank * BN + t]), lbar = smem_u32(maxbar);
+    for (int p = 0; p < cs; ++p) st_cluster_u32(mapa_shared(lmax, static_cast<uint32_t>(p)), mb);
+    fence_cluster();
+    for (int p = 0; p < cs; ++p) mbar_arrive_remote_relaxed(mapa_shared(lbar, static_cast<uint32_t>(p)));
+  }
+  if (!mbar_wait_cluster(maxbar, 0)) *s_fail = 1u;
+  uint32_t gb = 0u;
+  for (int p = 0; p < cs; ++p) gb = max(gb, sPmax[p * BN + t]);
+  const float gamma = __uint_as_float(gb);
+  const float d = __fadd_rn(gamma, kEps);
+  const float cq = __fmul_rn(kQb, __frcp_rn(d));
+  int32_t qs = 0;
+  for (int g = gbeg + sub; g < gbeg + nch * 8; g += TPT) {
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);  // past K and for absent tokens: code 0
+    if (active && g < gend) {
+      uint32_t r0[4], r1[4];
+      load8_raw(xr, 16 * g, a.K, vec_ok, r0);
+      load8_raw(xr, 16 * g + 8, a.K, vec_ok, r1);
+      w = group_codes<true>(r0, r1, cq, d, qs);
     }
-    if (!mbar_wait_cluster(maxbar, 0)) *s_fail = 1u;
-    uint32_t gb = 0u;
-    for (int p = 0; p < cs; ++p) gb = max(gb, sPmax[p * BN + t]);
-    const float gamma = __uint_as_float(gb);
-    const float d = __fadd_rn(gamma, kEps);
-    const float cq = __fmul_rn(kQb, __frcp_rn(d));
-    int32_t qs = 0;
-    for (int g = gbeg + sub; g < gbeg + nch * 8; g += TPT) {
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);  // past K and for absent tokens: code 0
-      if (active && g < gend) {
-        uint32_t r0[4], r1[4];
-        load8_raw(xr, 16 * g, a.K, vec_ok, r0);
-        load8_raw(xr, 16 * g + 8, a.K, vec_ok, r1);
-        w = group_codes<true>(r0, r1, cq, d, qs);
-      }
-      const int gl = g - gbeg;
-      const int ch = gl >> 3, j16 = gl & 7;  // chunk, 16-byte column of the token's 128-byte row
-      *reinterpret_cast<uint4*>(sB + ch * B_CHUNK + (t >> 3) * 1024 + (t & 7) * 128 + ((j16 ^ (t & 7)) << 4)) = w;
-    }
+    const int gl = g - gbeg;
+    const int ch = gl >> 3, j16 = gl & 7;  // chunk, 16-byte column of the token's 128-byte row
+    *reinterpret_cast<uint4*>(sB + ch * B_CHUNK + (t >> 3) * 1024 + (t & 7) * 128 + ((j16 ^ (t & 7)) << 4)) = w;
+  }
 #pragma unroll
-    for (int o = TPT / 2; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
-    if (sub == 0) {
-      sQsum[t] = qs;  // this slice's share of the token's code sum
-      sScale[t] = active ? __fdiv_rn(__fmul_rn(alpha, gamma), kQb) : 0.0f;  // RN(RN(alpha gamma) / 127)
-    }
-    fence_proxy_async_smem();  // the B tile is read by the tensor cores
-    asm volatile("bar.sync 1, %0;" ::"n"(kSkQuantThreads) : "memory");
-    if (threadIdx.x == 0) mbar_arrive(qready);  // publishes the codes, sums and scales to the other warps
-    pdl_launch_dependents();
+  for (int o = TPT / 2; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+  if (sub == 0) {
+    sQsum[t] = qs;  // this slice's share of the token's code sum
+    sScale[t] = active ? __fdiv_rn(__fmul_rn(alpha, gamma), kQb) : 0.0f;  // RN(RN(alpha gamma) / 127)
+  }
+  fence_proxy_async_smem();  // the B tile is read by the tensor cores
+  __syncthreads();
+  pdl_launch_dependents();
 
-    if (warp == 1 && lane == 0) {
+  // ------------------------------------------------ roles
+  if (warp == 1) {
+    if (lane == 0) {
       // MMA issuer
       for (int c = 0; c < nch; ++c) {
         const int sl = c % SA;
@@ -231,10 +226,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       }
       tc_commit(accfull);  // completes once every MMA issued above has (also after a give-up)
     }
-  } else {
-    // ---------------------------------------------- warps 4..15: expand the weights as they land
-    // (they do not depend on the preceding kernel), group grp taking chunks grp, grp + 3, ...
-    // for the 32 rows of its lane quarter
+  } else if (warp >= 4) {
+    // unpack: group grp expands chunks grp, grp + 3, ... for the 32 rows of its lane quarter
     const int grp = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
@@ -260,11 +253,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&aready[sl]);
     }
-    cluster_wait();  // before this warp's first access to another CTA's shared memory
     if (warp < 8) {
       // epilogue part 1: row r of this CTA's partial tile, minus the slice's code
       // sums, goes to the CTA whose band holds the row
-      if (!mbar_wait(accfull, 0) || !mbar_wait(qready, 0)) {
+      if (!mbar_wait(accfull, 0)) {
         *a.status = kDevTimeoutEpilogue;
         *s_fail = 1u;
       }
@@ -288,7 +280,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   }
 
   // ------------------------------------------------ this CTA's band: sum the slices, rescale, store
-  bool ok = my_rows > 0 && mbar_wait(qready, 0) && mbar_wait_cluster(redbar, 0);
+  bool ok = my_rows > 0 && mbar_wait_cluster(redbar, 0);
   if (!ok && my_rows > 0) *a.status = kDevTimeoutEpilogue;
   for (int p = 0; p < cs && ok; ++p) ok = sFailIn[p] == 0u;
   if (ok) {

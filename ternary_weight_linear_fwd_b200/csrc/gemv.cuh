@@ -29,9 +29,8 @@ constexpr int kGemvThreads = 512;
 // 16g + 4b + j), for g < groups_alloc (zero past K), where
 // slot(g) = (g % 4) * (groups_alloc / 4) + g / 4 puts the four groups of one
 // 64-weight chunk a quarter of the array apart, so lanes reading consecutive
-// chunks hit consecutive 16-byte words.  s_qparts[w] receives the sum of the
-// codes warp w formed (the row's code sum is the sum over the block's warps,
-// visible after the barrier that ends this function).  Each
+// chunks hit consecutive 16-byte words.  *s_qsum (zeroed by the caller before
+// a barrier that precedes this call) receives the sum of all codes.  Each
 // thread handles 8-element halves h = tid, tid + nthr, ...: one 16-byte load,
 // 8 codes and four 16-bit stores (bytes 2*(h%2), 2*(h%2)+1 of words 0..3).
 // One barrier publishes the per-warp maxima, one the codes and their sum.
@@ -39,7 +38,7 @@ constexpr int kGemvThreads = 512;
 constexpr int kHalvesInRegs = 2;  // halves per thread kept in registers (K <= 8192 at 512 threads)
 
 __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ x, int K, int groups_alloc,
-                                                   uint4* s_act, int32_t* s_qparts, float* s_red) {
+                                                   uint4* s_act, int32_t* s_qsum, float* s_red) {
   const bool vec_ok = (K % 8) == 0;
   const int nthr = blockDim.x;
   const int halves = (K + 7) / 8;
@@ -104,31 +103,9 @@ __device__ __forceinline__ float quantise_row_smem(const uint16_t* __restrict__ 
     emit(raw, h);
   }
   qsum = __reduce_add_sync(0xffffffffu, qsum);
-  if ((threadIdx.x & 31) == 0) s_qparts[threadIdx.x >> 5] = qsum;
+  if ((threadIdx.x & 31) == 0) atomicAdd(s_qsum, qsum);
   __syncthreads();
   return mx;
-}
-
-// Row totals of the contraction from s_part[seg][row] (nseg segments of nrows
-// rows): warp w takes rows w, w + 16, ...; its lanes add the segments lane,
-// lane + 32, ... and a warp reduction finishes the row, so no row is summed by
-// one thread alone.  Calls store(row, total) on lane 0.
-template <typename Store>
-__device__ __forceinline__ void gemv_row_totals(const int32_t* s_part, int nseg, int nrows, Store&& store) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int r = warp; r < nrows; r += nw) {
-    int32_t t = 0;
-    for (int sg = lane; sg < nseg; sg += 32) t += s_part[sg * nrows + r];
-    t = __reduce_add_sync(0xffffffffu, t);
-    if (lane == 0) store(r, t);
-  }
-}
-
-// Sum of the per-warp code sums of quantise_row_smem.
-__device__ __forceinline__ int32_t row_code_sum(const int32_t* s_qparts) {
-  int32_t t = 0;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += s_qparts[w];
-  return t;
 }
 
 // quantise_row_smem with RMSNorm first (weight s_g[K] already in shared
@@ -136,7 +113,7 @@ __device__ __forceinline__ int32_t row_code_sum(const int32_t* s_qparts) {
 // fixed-order reduction over the CTA), the root and the quotient in fp64;
 // the codes are those of xn = RN(RN(x * r) * g), which is never stored.
 __device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restrict__ x, int K, int groups_alloc,
-                                                        uint4* s_act, int32_t* s_qparts, float* s_red, double* s_redd,
+                                                        uint4* s_act, int32_t* s_qsum, float* s_red, double* s_redd,
                                                         const float* s_g, float eps) {
   const bool vec_ok = (K % 8) == 0;
   const int nthr = blockDim.x;
@@ -234,7 +211,7 @@ __device__ __forceinline__ float quantise_row_smem_norm(const uint16_t* __restri
     emit(raw, h);
   }
   qsum = __reduce_add_sync(0xffffffffu, qsum);
-  if ((threadIdx.x & 31) == 0) s_qparts[threadIdx.x >> 5] = qsum;
+  if ((threadIdx.x & 31) == 0) atomicAdd(s_qsum, qsum);
   __syncthreads();
   return mx;
 }
@@ -281,13 +258,9 @@ __device__ __forceinline__ void dot_word(uint32_t wd, uint32_t a0, uint32_t a1, 
 __host__ __device__ __forceinline__ int gemv_stripes(int64_t ld) { return static_cast<int>((ld + 127) / 128); }
 __host__ __device__ __forceinline__ int gemv_stripe_bytes(int rows_box) { return (rows_box * 128 + 1023) & ~1023; }
 
-// Per-thread partial sums of the contraction, [segments][rows]: at most
-// (512 / half) * 2 * half = 1024 entries for half = ceil(rows / 2) pairs.
-constexpr int kGemvPartWords = 1024;
-
 __host__ __device__ __forceinline__ size_t gemv_smem_bytes(int rows_box, int64_t ld, int C) {
   return 1024 /* alignment */ + static_cast<size_t>(gemv_stripes(ld)) * gemv_stripe_bytes(rows_box) +
-         static_cast<size_t>(C) * 4 * 16 + 32 * 4 /* per-warp code sums */ + kGemvPartWords * 4;
+         static_cast<size_t>(C) * 4 * 16 + 16 /* code sum */ + static_cast<size_t>(rows_box) * 4;
 }
 
 // Weight chunk ch of local row r in the swizzled stripes.
@@ -350,9 +323,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   // offset arithmetic on the shared array keeps every derived pointer in the shared window
   uint8_t* s_w = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
   uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
-  int32_t* s_qparts = reinterpret_cast<int32_t*>(s_act + 4 * C);  // per-warp code sums [32]
-  int32_t* s_part = s_qparts + 32;                                  // contraction partial sums [kGemvPartWords]
-  float* s_g = reinterpret_cast<float*>(s_part + kGemvPartWords);   // norm variant: RMSNorm weight [K]
+  int32_t* s_qsum = reinterpret_cast<int32_t*>(s_act + 4 * C);  // sum of the codes (one 16-byte slot)
+  int32_t* s_acc = s_qsum + 4;
+  float* s_g = reinterpret_cast<float*>(s_acc + rows_box);        // norm variant: RMSNorm weight [K]
   __shared__ double s_redd[32];
 
   // The weights (and alpha, which belongs to them) do not depend on the
@@ -367,6 +340,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     for (int st = 0; st < stripes; ++st) tma_load_2d_hint(s_w + st * stripe_bytes, map, st * 128, r0, &s_bar, pol);
   }
   const float alpha = *mt.alpha;
+  for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  if (threadIdx.x == 0) *s_qsum = 0;
   if (kNorm)  // the norm weight, like the matrix, does not depend on the preceding kernel
     for (int k = threadIdx.x; k < g.K; k += blockDim.x) s_g[k] = g.gnorm[k];
   __syncthreads();
@@ -374,9 +349,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   pdl_wait_primary();  // x may come from the preceding kernel
   float gamma;
   if (kNorm)
-    gamma = quantise_row_smem_norm(g.x, g.K, 4 * C, s_act, s_qparts, s_red, s_redd, s_g, g.eps);
+    gamma = quantise_row_smem_norm(g.x, g.K, 4 * C, s_act, s_qsum, s_red, s_redd, s_g, g.eps);
   else
-    gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qparts, s_red);
+    gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qsum, s_red);
   // The next kernel may start now: its weight copies then stream while this
   // one contracts, and no longer delay this kernel's read of x.
   pdl_launch_dependents();
@@ -390,8 +365,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     // activation chunk (a shared-memory broadcast) and conflict-free weight
     // slots.  Each partial sum s_j carries the factor 4^j of its bit plane and
     // stays below 2 * 64 * 127 * K / 4 < 2^31, so the final shifts are exact.
-    // The thread's two row totals go to s_part[seg][row] (no atomics: the
-    // segments of a row are summed by one thread after the barrier).
     const int half = (nrows + 1) >> 1;  // rows_box <= 256: at most 128 pairs, at least 4 segments
     const int nseg = blockDim.x / half;
     const int seg = threadIdx.x / half, p = threadIdx.x - seg * half;
@@ -412,14 +385,15 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
         dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
         dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
       }
-      s_part[seg * nrows + p] = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
-      if (p + half < nrows) s_part[seg * nrows + p + half] = b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6);
+      if (c_end > c_beg) {
+        atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6));
+        if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6));
+      }
     }
   }
   if (gemv_gave_up(landed, &s_bar, g.status)) return;
-  const int32_t qsum = row_code_sum(s_qparts);
-  gemv_row_totals(s_part, blockDim.x / ((nrows + 1) >> 1), nrows,
-                  [&](int rr, int32_t t) { gemv_store(mt.y, mt.acc, r0 + rr, t - qsum, s); });
+  const int32_t qsum = *s_qsum;
+  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr] - qsum, s);
 }
 
 // ------------------------------------------------------------------ dense M = 1, lookup tables
@@ -451,8 +425,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_con
   const int stripe_bytes = gemv_stripe_bytes(rows_box);
   uint8_t* s_w = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
   uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
-  int32_t* s_qparts = reinterpret_cast<int32_t*>(s_act + 4 * C);  // filled, not needed: the tables carry W_t
-  int32_t* s_acc = s_qparts + 32;
+  int32_t* s_qsum = reinterpret_cast<int32_t*>(s_act + 4 * C);  // filled, not needed: the tables carry W_t
+  int32_t* s_acc = s_qsum + 4;
   int16_t* s_lut = reinterpret_cast<int16_t*>(s_acc + rows_box + 3 - ((rows_box + 3) & 3));  // [pairs][16]
 
   if (threadIdx.x == 0) {
@@ -466,10 +440,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_lut_kernel(const __grid_con
   }
   const float alpha = *mt.alpha;
   for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  if (threadIdx.x == 0) *s_qsum = 0;
   __syncthreads();
 
   pdl_wait_primary();
-  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qparts, s_red);
+  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qsum, s_red);
   pdl_launch_dependents();
   // tables: pair p covers k = 2p, 2p + 1; code of k sits in group k / 16, word k % 4, byte (k % 16) / 4
   const int pairs = 32 * C;  // 64-weight chunks of 32 pairs (codes past K are 0)
@@ -555,7 +530,7 @@ __host__ __device__ __forceinline__ int nm_unit_value_bytes(int n) { return n ==
 __host__ __device__ __forceinline__ size_t gemv_nm_smem_bytes(int rows_box, int64_t ld_v, int64_t ld_m, int C, bool lut) {
   return 1024 + static_cast<size_t>(gemv_stripes(ld_v) + gemv_stripes(ld_m)) * gemv_stripe_bytes(rows_box) +
          (lut ? static_cast<size_t>(kNmLutWords) * 4 : 0) + static_cast<size_t>(C) * 8 * 16 /* codes */ +
-         32 * 4 /* per-warp code sums */ + kGemvPartWords * 4;
+         16 /* code sum */ + static_cast<size_t>(rows_box) * 4;
 }
 
 // 32-bit word at byte offset off (a multiple of 4) of local row r in swizzled 128-byte stripes.
@@ -643,8 +618,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
   uint8_t* s_m = s_v + static_cast<size_t>(stripes_v) * stripe_bytes;
   uint32_t* s_lut = reinterpret_cast<uint32_t*>(s_m + static_cast<size_t>(stripes_m) * stripe_bytes);
   uint4* s_act = reinterpret_cast<uint4*>(s_lut + (NMN == 0 ? kNmLutWords : 0));
-  int32_t* s_qparts = reinterpret_cast<int32_t*>(s_act + 8 * C);  // per-warp code sums [32]
-  int32_t* s_part = s_qparts + 32;                                  // contraction partial sums [kGemvPartWords]
+  int32_t* s_qsum = reinterpret_cast<int32_t*>(s_act + 8 * C);  // sum of the codes (one 16-byte slot)
+  int32_t* s_acc = s_qsum + 4;
 
   if (threadIdx.x == 0) {
     mbar_init(&s_bar, 1);
@@ -659,47 +634,50 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nm_kernel(const __grid_cons
   }
   if (NMN == 0) nm24_fill_lut(s_lut);
   const float alpha = *a.alpha;
+  for (int r = threadIdx.x; r < nrows; r += blockDim.x) s_acc[r] = 0;
+  if (threadIdx.x == 0) *s_qsum = 0;
   __syncthreads();
 
   pdl_wait_primary();  // x may come from the preceding kernel
-  const float gamma = quantise_row_smem(a.x, a.K, 8 * C, s_act, s_qparts, s_red);
+  const float gamma = quantise_row_smem(a.x, a.K, 8 * C, s_act, s_qsum, s_red);
   pdl_launch_dependents();
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
 
   if (landed) {
-    // the dense kernel's mapping: thread (seg, p) takes row pair p over the
-    // 128-weight units of segment seg, partial sums in registers, totals to
-    // s_part[seg][row]
     const uint32_t* lut_lane = s_lut + (threadIdx.x & 31);
+    const int nthr = blockDim.x;
     const int half = (nrows + 1) >> 1;
-    const int nseg = blockDim.x / half;
-    const int seg = threadIdx.x / half, p = threadIdx.x - seg * half;
+    const int total = half * C;
+    const int dq = nthr / half, dr = nthr % half;
+    int u = threadIdx.x / half, p = threadIdx.x % half;
     const int quarter = 2 * C;  // s_act slot stride: group g sits at (g % 4) * 2C + g / 4
-    if (seg < nseg) {
-      const int u_beg = seg * C / nseg, u_end = (seg + 1) * C / nseg;
+    for (int it = threadIdx.x; it < total; it += nthr) {
       const int r2 = p + half < nrows ? p + half : p;
+      uint32_t da[8], db[8];
+      nm_unit_words<NMN>(s_v, s_m, stripe_bytes, p, u, lut_lane, da);
+      nm_unit_words<NMN>(s_v, s_m, stripe_bytes, r2, u, lut_lane, db);
       int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
-      for (int u = u_beg; u < u_end; ++u) {
-        uint32_t da[8], db[8];
-        nm_unit_words<NMN>(s_v, s_m, stripe_bytes, p, u, lut_lane, da);
-        nm_unit_words<NMN>(s_v, s_m, stripe_bytes, r2, u, lut_lane, db);
 #pragma unroll
-        for (int gi = 0; gi < 8; ++gi) {
-          const int g = 8 * u + gi;
-          const uint4 q = s_act[(g & 3) * quarter + (g >> 2)];
-          dot_word(da[gi], q.x, q.y, q.z, q.w, a0, a1, a2, a3);
-          dot_word(db[gi], q.x, q.y, q.z, q.w, b0, b1, b2, b3);
-        }
+      for (int gi = 0; gi < 8; ++gi) {
+        const int g = 8 * u + gi;
+        const uint4 q = s_act[(g & 3) * quarter + (g >> 2)];
+        dot_word(da[gi], q.x, q.y, q.z, q.w, a0, a1, a2, a3);
+        dot_word(db[gi], q.x, q.y, q.z, q.w, b0, b1, b2, b3);
       }
-      s_part[seg * nrows + p] = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
-      if (p + half < nrows) s_part[seg * nrows + p + half] = b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6);
+      atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6));
+      if (p + half < nrows) atomicAdd(&s_acc[p + half], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6));
+      p += dr;
+      u += dq;
+      if (p >= half) {
+        p -= half;
+        ++u;
+      }
     }
   }
   if (gemv_gave_up(landed, &s_bar, a.status)) return;
-  const int32_t qsum = row_code_sum(s_qparts);
-  gemv_row_totals(s_part, blockDim.x / ((nrows + 1) >> 1), nrows,
-                  [&](int rr, int32_t t) { gemv_store(a.y, a.acc, r0 + rr, t - qsum, s); });
+  const int32_t qsum = *s_qsum;
+  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(a.y, a.acc, r0 + rr, s_acc[rr] - qsum, s);
 }
 
 }  // namespace bl
