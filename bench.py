@@ -827,6 +827,50 @@ def run_cpu_baselines(decode_seconds: float, threads: int, with_sweep: bool):
     return out
 
 
+# ------------------------------------------------------------------ profiling cases
+
+def _case_few_token(dev):
+    """bitlinear_forward at M = 16 on a 2560 x 2560 ternary matrix: the fused few-token kernel."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+    w = bl.pack_ternary(torch.from_numpy(synth.ternary_weights(2560, 2560, seed=1)).to(dev), 0.03)
+    x = torch.from_numpy(synth.activations(16, 2560, seed=2).view(np.int16)).to(dev).view(torch.bfloat16)
+    for _ in range(3):
+        bl.forward(w, x)
+
+
+def _case_hbit_m1(dev):
+    """bitlinear_hadamard_quant_act4 on one 2560-wide token."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+    x = torch.from_numpy(synth.activations(1, 2560, seed=4).view(np.int16)).to(dev).view(torch.bfloat16)
+    for _ in range(3):
+        bl.hadamard_quant_act4(x)
+
+
+PROFILE_CASES = {"few_token_m16": _case_few_token, "hbit_m1": _case_hbit_m1}
+
+
+def run_profile_case(name: str):
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import build as blbuild
+    blbuild.build()
+    dev = torch.device("cuda", 0)
+    PROFILE_CASES[name](dev)
+    torch.cuda.synchronize(dev)
+    if bl.device_status() != 0:
+        raise SystemExit(f"{name}: device status word set")
+    print(f"{name}: ok, last kernel {bl.last_kernel()}")
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -840,7 +884,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the layer sweep and the N:M objects")
+    ap.add_argument("--case", choices=sorted(PROFILE_CASES),
+                    help="run one small profiling case (three calls of one kernel) and exit: the target of the "
+                         "ncu captures summarised under profiles/")
     args = ap.parse_args()
+    if args.case:
+        run_profile_case(args.case)
+        return
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps")
 
