@@ -97,6 +97,11 @@ typedef enum bitlinear_status {
 #define BITLINEAR_FLAG_PATH_PERSISTENT 0x10u /* tensor-core path: take the persistent GEMM (separate
                                         * quantisation launch, K split through a workspace) even
                                         * where the fused few-token kernel applies; same results */
+#define BITLINEAR_FLAG_NM24_EXPAND 0x20u /* tensor-core path, 2:4 weights: expand the kept values
+                                        * to dense codes and run the dense MMA instead of the
+                                        * structured-sparse tcgen05.mma.sp (the Sparse-BitNet
+                                        * review, section 4: 2:4 on sparse tensor cores); same
+                                        * results.  A comparison path, not the default. */
 #define BITLINEAR_FLAG_DECODE_LUT 0x8u /* M = 1, dense weights: run the decode GEMV with
                                         * per-pair lookup tables (the TL2 idea of the
                                         * "BitNet 1-Bit LLM" blog, section "I2_S kernel
@@ -253,7 +258,15 @@ bitlinear_status bitlinear_forward(const bitlinear_weights* w, const uint16_t* x
                                    int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
                                    void* stream);
 
-/* Same as bitlinear_forward for N:M packed weights (w->nm_n/nm_m = 2,4 or n,8). */
+/* Same as bitlinear_forward for N:M packed weights (w->nm_n/nm_m = 2,4 or n,8).
+ * Path: M == 1 takes the N:M streaming GEMV; otherwise (or with
+ * BITLINEAR_FLAG_PATH_TC) a quantisation launch and the persistent tcgen05
+ * GEMM.  There 2:4 weights run on the structured-sparse MMA
+ * (tcgen05.mma.sp kind::i8: the kept values as signed int8, the packed
+ * metadata unchanged, activation codes in natural K order), the Sparse-BitNet
+ * review's sparse tensor-core path (section 4); n:8 weights, and 2:4 with
+ * BITLINEAR_FLAG_NM24_EXPAND, are expanded to dense codes for the dense MMA.
+ * Every path gives the same bits. */
 bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t* x, int32_t M, uint16_t* y,
                                       int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
                                       void* stream);
@@ -280,7 +293,8 @@ bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t
  * them by rows) and each N:M matrix in its own; 2 <= M <= 64 with dense
  * weights runs the fused few-token kernel once per matrix (see
  * bitlinear_forward); otherwise the call quantises once and runs one
- * persistent tensor-core GEMM per matrix.
+ * persistent tensor-core GEMM per matrix (the structured-sparse MMA when
+ * every matrix is 2:4, since the codes' K order is shared).
  * Errors: as bitlinear_forward; SHAPE also for count out of range or unequal K. */
 bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,
                                          uint16_t* const* y, int32_t* const* acc, void* workspace,

@@ -17,7 +17,7 @@ __all__ = [
     "quant_act", "rmsnorm_quant_act", "forward", "forward_nm", "forward_group", "forward_norm",
     "forward_workspace_bytes", "device_status", "last_kernel", "layout_version", "hadamard_quant_act4",
     "forward_hbit", "HBIT_MAX_K",
-    "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT", "FLAG_PATH_PERSISTENT",
+    "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT", "FLAG_PATH_PERSISTENT", "FLAG_NM24_EXPAND",
 ]
 
 FLAG_PDL = 0x1
@@ -26,6 +26,7 @@ FLAG_PATH_GEMV = 0x2
 FLAG_PATH_TC = 0x4
 FLAG_DECODE_LUT = 0x8
 FLAG_PATH_PERSISTENT = 0x10
+FLAG_NM24_EXPAND = 0x20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libbitlinear.so")

@@ -292,10 +292,11 @@ bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA,
 }
 
 const char* tc_name(int nm, int bn) {
-  static const char* names[3][4] = {
+  static const char* names[4][4] = {
       {"tc_gemm_dense_bn16", "tc_gemm_dense_bn32", "tc_gemm_dense_bn64", "tc_gemm_dense_bn128"},
       {"tc_gemm_nm24_bn16", "tc_gemm_nm24_bn32", "tc_gemm_nm24_bn64", "tc_gemm_nm24_bn128"},
-      {"tc_gemm_n8_bn16", "tc_gemm_n8_bn32", "tc_gemm_n8_bn64", "tc_gemm_n8_bn128"}};
+      {"tc_gemm_n8_bn16", "tc_gemm_n8_bn32", "tc_gemm_n8_bn64", "tc_gemm_n8_bn128"},
+      {"tc_gemm_sp24_bn16", "tc_gemm_sp24_bn32", "tc_gemm_sp24_bn64", "tc_gemm_sp24_bn128"}};
   const int i = bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3;
   return names[nm][i];
 }
@@ -433,7 +434,7 @@ auto quant_kernel(int G) {
 }
 
 bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s,
-                          const float* gnorm = nullptr, float eps = 0.0f) {
+                          const float* gnorm = nullptr, float eps = 0.0f, bool natural = false) {
   const QuantShape qs = quant_shape(M, K, gnorm != nullptr, plan_sm_count());
   const int wpr = qs.wpr;
   const int rows_per_cta = kQuantWarps / wpr;
@@ -443,19 +444,24 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
   const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * 32 * kQuantWarps - 1) /
                                                                    (4 * 32 * kQuantWarps)));
   uint32_t* cnt = qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr);
-  if (gnorm)
-    return launch(quant_kernel<true, true>(qs.G), dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
-                  static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr, gnorm,
-                  eps);
-  return launch(quant_kernel<true, false>(qs.G), dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K,
-                static_cast<int>(k16(K)), qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr,
-                static_cast<const float*>(nullptr), 0.0f);
+  // contraction order for the dense and expanded MMAs; natural K order (zero-padded to 16) for the
+  // structured-sparse MMA, whose metadata names positions inside runs of four consecutive k
+  auto go = [&](auto kern, const float* g, float e) {
+    return launch(kern, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K, static_cast<int>(k16(K)),
+                  qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr, g, e);
+  };
+  if (gnorm) return natural ? go(quant_kernel<false, true>(qs.G), gnorm, eps) : go(quant_kernel<true, true>(qs.G), gnorm, eps);
+  return natural ? go(quant_kernel<false, false>(qs.G), static_cast<const float*>(nullptr), 0.0f)
+                 : go(quant_kernel<true, false>(qs.G), static_cast<const float*>(nullptr), 0.0f);
 }
 
+// natural: the codes in qw are in natural K order (tc_quant(..., natural = true)),
+// which sends 2:4 weights to the structured-sparse MMA.
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
-                         cudaStream_t s, DeviceState* dev, float qb = kQb) {
+                         cudaStream_t s, DeviceState* dev, float qb = kQb, bool natural = false) {
   const int N = w->N, K = w->K;
-  const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? 1 : 2);
+  const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? (natural ? 3 : 1) : 2);
+  if (natural && nm != 3) return BITLINEAR_ERR_PATTERN;
   const TcPlan plan = tc_plan(M, N, K, nm, dev->sm_count);
   const int bn = plan.bn;
   CUtensorMap mB, mA, mMeta;
@@ -476,7 +482,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   if (plan.ksplit > 1 && (qw.ncnt < plan.row_tiles * plan.tok_tiles)) return BITLINEAR_ERR_WORKSPACE;
   ta.gamma = qw.gamma;
   ta.alpha = w->alpha;
-  ta.rowsum = qw.rowsum;
+  ta.rowsum = nm == 3 ? nullptr : qw.rowsum;  // signed kept weights: no code-sum correction
   ta.y = y;
   ta.acc = acc;
   ta.nm_n = w->nm_n;
@@ -492,7 +498,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
     int64_t ldv = 0, ldm = 0;
     if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
       return BITLINEAR_ERR_PATTERN;
-    const uint32_t vbox = nm == 1 ? static_cast<uint32_t>(16 * tc_ksub(1, bn))
+    const uint32_t vbox = nm != 2 ? static_cast<uint32_t>(16 * tc_ksub(nm, bn))
                                   : static_cast<uint32_t>((4 * w->nm_n + 12 + 15) / 16 * 16);
     ta.vbox = static_cast<int>(vbox);
     if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, false)) return BITLINEAR_ERR_CUDA;
@@ -504,6 +510,8 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
     st = launch_tc<0>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
   else if (nm == 1)
     st = launch_tc<1>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
+  else if (nm == 3)
+    st = launch_tc<3>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
   else
     st = launch_tc<2>(bn, mB, mA, mMeta, ta, dev->sm_count, s);
   if (st == BITLINEAR_OK) t_last_kernel = tc_name(nm, bn);
@@ -541,22 +549,24 @@ enum class ActKind { kInt8, kInt8Norm, kHbit4 };
 
 bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M, uint16_t* y, int32_t* acc,
                             void* ws, size_t ws_bytes, bool pdl, cudaStream_t s, DeviceState* dev,
-                            const float* gnorm = nullptr, float eps = 0.0f, ActKind act = ActKind::kInt8) {
+                            const float* gnorm = nullptr, float eps = 0.0f, ActKind act = ActKind::kInt8,
+                            bool nm24_expand = false) {
   const int nm = w->nm_m == 0 ? 0 : (w->nm_m == 4 ? 1 : 2);
+  const bool natural = nm == 1 && !nm24_expand;  // 2:4 on the structured-sparse MMA
   if (!ws || ws_bytes < tc_workspace(M, w->N, w->K, nm, dev->sm_count) || !aligned16(ws))
     return BITLINEAR_ERR_WORKSPACE;
   const bool split = tc_plan(M, w->N, w->K, nm, dev->sm_count).ksplit > 1;
   const QuantWs qw = tc_ws_layout(ws, M, w->K, split ? dev->sm_count : 0, w->N);
   bitlinear_status st;
   if (act == ActKind::kHbit4) {
-    st = hbit_quant(x, M, w->K, qw.q, static_cast<int>(k16(w->K)), true, qw.gamma, qw.rowsum,
+    st = hbit_quant(x, M, w->K, qw.q, static_cast<int>(k16(w->K)), !natural, qw.gamma, qw.rowsum,
                     qw.ncnt > 0 ? qw.cnt : nullptr, qw.ncnt, qw.part, qw.part_words, pdl, s);
     if (st != BITLINEAR_OK) return st;
-    return tc_gemm(w, M, qw, y, acc, s, dev, kQb4);
+    return tc_gemm(w, M, qw, y, acc, s, dev, kQb4, natural);
   }
-  st = tc_quant(x, M, w->K, qw, pdl, s, act == ActKind::kInt8Norm ? gnorm : nullptr, eps);
+  st = tc_quant(x, M, w->K, qw, pdl, s, act == ActKind::kInt8Norm ? gnorm : nullptr, eps, natural);
   if (st != BITLINEAR_OK) return st;
-  return tc_gemm(w, M, qw, y, acc, s, dev);
+  return tc_gemm(w, M, qw, y, acc, s, dev, kQb, natural);
 }
 
 // ---------------------------------------------------------------- GEMV path
@@ -764,7 +774,7 @@ bitlinear_status check_matrix(const bitlinear_weights* w, const uint16_t* y, con
 
 bitlinear_status check_flags(uint32_t flags, int M) {
   const uint32_t known = BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_GEMV | BITLINEAR_FLAG_PATH_TC |
-                         BITLINEAR_FLAG_DECODE_LUT | BITLINEAR_FLAG_PATH_PERSISTENT;
+                         BITLINEAR_FLAG_DECODE_LUT | BITLINEAR_FLAG_PATH_PERSISTENT | BITLINEAR_FLAG_NM24_EXPAND;
   if (flags & ~known) return BITLINEAR_ERR_FLAGS;
   if ((flags & BITLINEAR_FLAG_PATH_GEMV) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
   if ((flags & BITLINEAR_FLAG_DECODE_LUT) && ((flags & BITLINEAR_FLAG_PATH_TC) || M != 1)) return BITLINEAR_ERR_FLAGS;
@@ -793,7 +803,9 @@ bitlinear_status forward_common(const bitlinear_weights* w, const uint16_t* x, i
     const SkPlan p = sk_plan(M, w->N, w->K, dev);
     if (p.ok) return skinny_launch(w, x, M, y, acc, pdl, s, dev, p);
   }
-  if (tc) return forward_tc(w, x, M, y, acc, ws, ws_bytes, pdl, s, dev);
+  if (tc)
+    return forward_tc(w, x, M, y, acc, ws, ws_bytes, pdl, s, dev, nullptr, 0.0f, ActKind::kInt8,
+                      (flags & BITLINEAR_FLAG_NM24_EXPAND) != 0);
   if ((flags & BITLINEAR_FLAG_DECODE_LUT) && want_nm) return BITLINEAR_ERR_FLAGS;
   return forward_gemv(w, x, y, acc, pdl, s, dev, (flags & BITLINEAR_FLAG_DECODE_LUT) != 0);
 }
@@ -848,8 +860,12 @@ bitlinear_status forward_group(const bitlinear_weights* w, int count, const uint
     }
     if (!ws || ws_bytes < need || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
     const QuantWs qw = tc_ws_layout(ws, M, w[0].K, split ? dev->sm_count : 0, max_n);
-    st = tc_quant(x, M, w[0].K, qw, pdl, s);
-    for (int i = 0; i < count && st == BITLINEAR_OK; ++i) st = tc_gemm(&w[i], M, qw, y[i], acc ? acc[i] : nullptr, s, dev);
+    // one quantisation serves every matrix: natural K order (structured-sparse MMA) only when all are 2:4
+    bool natural = !(flags & BITLINEAR_FLAG_NM24_EXPAND);
+    for (int i = 0; i < count; ++i) natural = natural && w[i].nm_m == 4;
+    st = tc_quant(x, M, w[0].K, qw, pdl, s, nullptr, 0.0f, natural);
+    for (int i = 0; i < count && st == BITLINEAR_OK; ++i)
+      st = tc_gemm(&w[i], M, qw, y[i], acc ? acc[i] : nullptr, s, dev, kQb, natural);
     return st;
   }
   // decode: the dense matrices share one launch; each N:M matrix has its own
@@ -1024,7 +1040,8 @@ bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16
   if (M < 1 || M > BITLINEAR_MAX_M) return BITLINEAR_ERR_SHAPE;
   if (!(eps >= 0.0f) || eps > 1.0f) return BITLINEAR_ERR_SHAPE;
   if (!aligned16(x) || (reinterpret_cast<uintptr_t>(g) & 3u)) return BITLINEAR_ERR_ALIGN;
-  if (flags & ~static_cast<uint32_t>(BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_TC)) return BITLINEAR_ERR_FLAGS;
+  if (flags & ~static_cast<uint32_t>(BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_TC | BITLINEAR_FLAG_NM24_EXPAND))
+    return BITLINEAR_ERR_FLAGS;
   DeviceState* dev = nullptr;
   st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
@@ -1034,7 +1051,8 @@ bitlinear_status bitlinear_forward_norm(const bitlinear_weights* w, const uint16
     // decode: every GEMV CTA normalises and quantises the token itself
     return gemv_dense_launch(&w, &y, &acc, 1, x, pdl, s, dev, g, eps);
   }
-  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, pdl, s, dev, g, eps, ActKind::kInt8Norm);
+  return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, pdl, s, dev, g, eps, ActKind::kInt8Norm,
+                    (flags & BITLINEAR_FLAG_NM24_EXPAND) != 0);
 }
 
 bitlinear_status bitlinear_hadamard_quant_act4(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* gamma,
@@ -1061,12 +1079,14 @@ bitlinear_status bitlinear_forward_hbit(const bitlinear_weights* w, const uint16
   if (st != BITLINEAR_OK) return st;
   if (M < 1 || M > BITLINEAR_MAX_M || w->K > BITLINEAR_HBIT_MAX_K) return BITLINEAR_ERR_SHAPE;
   if (!aligned16(x)) return BITLINEAR_ERR_ALIGN;
-  if (flags & ~static_cast<uint32_t>(BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_TC)) return BITLINEAR_ERR_FLAGS;
+  if (flags & ~static_cast<uint32_t>(BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_TC | BITLINEAR_FLAG_NM24_EXPAND))
+    return BITLINEAR_ERR_FLAGS;
   DeviceState* dev = nullptr;
   st = current_device(&dev);
   if (st != BITLINEAR_OK) return st;
   return forward_tc(w, x, M, y, acc, workspace, workspace_bytes, (flags & BITLINEAR_FLAG_PDL) != 0,
-                    static_cast<cudaStream_t>(stream), dev, nullptr, 0.0f, ActKind::kHbit4);
+                    static_cast<cudaStream_t>(stream), dev, nullptr, 0.0f, ActKind::kHbit4,
+                    (flags & BITLINEAR_FLAG_NM24_EXPAND) != 0);
 }
 
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {

@@ -25,7 +25,7 @@
 // of q * code is an integer of magnitude at most 254 * K <= 254 * 65536 < 2^24.
 // Warp roles (16 warps): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues
 // the MMAs, warp 2 owns the TMEM allocation, warps 4..11 unpack weights (two
-// groups of four, alternating k-blocks), warps 12..15 run the epilogue.  Warp
+// groups of four, for the even and the odd stages), warps 12..15 run the epilogue.  Warp
 // w reaches TMEM lanes 32 * (w % 4) .. + 31.  A mbarrier ring (4 to 8 stages of
 // 256 k for dense weights, 128 k for N:M; as many as TMEM has A slots for) couples
 // the producer, unpackers and MMA issuer (full: TMA bytes landed, aready: A
@@ -34,9 +34,17 @@
 // main loop of the next.  Every wait is bounded; a role that gives up records
 // a status code and unwinds.
 //
-// N:M weights (Sparse-BitNet, section 3.2) are expanded from kept values +
-// metadata into the same dense code words before the tcgen05.st, so the MMA
-// is the dense one.
+// N:M weights (Sparse-BitNet, section 3.2): n:8 rows, and 2:4 rows on request,
+// are expanded from kept values + metadata into the same dense code words
+// before the tcgen05.st, so the MMA is the dense one.  By default 2:4 rows
+// run on the structured-sparse MMA (NM = 3, the sparse tensor-core path of
+// the Sparse-BitNet review, section 4): the unpack warps turn the kept codes
+// into signed int8 weights (W_t itself, so no code-sum correction) in the
+// 128-byte-swizzled K-major layout of a shared-memory A operand holding only
+// the kept values, copy the packed metadata unchanged into TMEM (its nibble
+// i0 | i1 << 2 per block of four is the instruction's metadata format), and
+// tcgen05.mma.sp kind::i8 multiplies them with activation codes in natural K
+// order: 64 K per instruction, half the instructions of the dense MMA.
 #pragma once
 #include "gemv.cuh"
 #include "hbit.cuh"
@@ -52,7 +60,7 @@ constexpr int kTcEpiWarp0 = 12;  // first epilogue warp
 // K elements per stage: dense and 2:4 weights with token tiles up to 128 take
 // two 128-wide sub-tiles (eight MMAs per barrier round trip, which halves the
 // fixed cost of a stage per MAC); wider tiles and n:8 weights keep one.
-__host__ __device__ constexpr int tc_ksub(int NM, int BN) { return (NM <= 1 && BN <= 128) ? 2 : 1; }
+__host__ __device__ constexpr int tc_ksub(int NM, int BN) { return (NM != 2 && BN <= 128) ? 2 : 1; }
 __host__ __device__ constexpr int tc_bk(int NM, int BN) { return kTcSubK * tc_ksub(NM, BN); }
 
 struct TcArgs {
@@ -79,18 +87,36 @@ template <int NM, int BN>
 struct TcStageBytes {
   // packed A bytes per stage (TMA box bytes, rows = 128)
   static __host__ __device__ constexpr int a_values(int vbox) {
-    return NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 * tc_ksub(1, BN) : kTcRows * vbox);
+    return NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM != 2 ? kTcRows * 16 * tc_ksub(NM, BN) : kTcRows * vbox);
   }
   static __host__ __device__ constexpr int a_meta() { return NM == 0 ? 0 : kTcRows * 16 * tc_ksub(NM, BN); }
 };
 
 __host__ __device__ constexpr int tc_dcols(int BN) { return BN < 32 ? 32 : BN; }  // TMEM columns of one accumulator
-__host__ __device__ constexpr int tc_slot_cols(int NM, int BN) { return 32 * tc_ksub(NM, BN); }  // one A slot
-// Pipeline stages: as many A slots as fit beside the two accumulators, at most 8.
+// TMEM columns of one stage: the expanded A codes (32 per 128 k), or for the
+// sparse MMA the metadata (4 bits per 4 k: 4 columns per 128 k)
+__host__ __device__ constexpr int tc_slot_cols(int NM, int BN) { return (NM == 3 ? 4 : 32) * tc_ksub(NM, BN); }
+constexpr int kTcSmemMax = 232448;  // dynamic shared memory a CTA may opt into
+// Compressed int8 A of one sparse-MMA stage: 128 rows x (stage K / 2) bytes.
+__host__ __device__ constexpr int tc_sp_a_bytes(int BN) { return kTcRows * 64 * tc_ksub(3, BN); }
+__host__ __device__ constexpr int tc_a_stage_bytes(int NM, int BN, int vbox) {
+  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM != 2 ? kTcRows * 16 * tc_ksub(NM, BN) : kTcRows * vbox)) +
+          (NM == 0 ? 0 : kTcRows * 16 * tc_ksub(NM, BN)) + 1023) / 1024 * 1024;
+}
+__host__ __device__ constexpr int tc_fixed_smem(int BN, int NM) {
+  return 1024 /* alignment slack */ + (NM == 1 ? kNmLutWords * 4 : 0) /* 2:4 expansion table, one copy per lane */ +
+         4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
+}
+// Shared memory of one pipeline stage (the sparse MMA's operand only for 2:4 rows, vbox fixed).
+__host__ __device__ constexpr int tc_stage_smem(int BN, int NM, int vbox) {
+  return BN * 128 * tc_ksub(NM, BN) + tc_a_stage_bytes(NM, BN, vbox) + (NM == 3 ? tc_sp_a_bytes(BN) : 0);
+}
+__host__ __device__ constexpr int tc_min3(int a, int b, int c) { return a < b ? (a < c ? a : c) : (b < c ? b : c); }
+// Pipeline stages: as many as TMEM has slots for beside the two accumulators,
+// at most 8; the sparse MMA's stages are bounded by shared memory instead.
 __host__ __device__ constexpr int tc_stages(int BN, int NM) {
-  return (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM, BN) < kTcMaxStages
-             ? (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM, BN)
-             : kTcMaxStages;
+  return tc_min3(kTcMaxStages, (512 - 2 * tc_dcols(BN)) / tc_slot_cols(NM, BN),
+                 NM == 3 ? (kTcSmemMax - tc_fixed_smem(BN, 3)) / tc_stage_smem(BN, 3, 0) : kTcMaxStages);
 }
 
 template <int BN, int NM>
@@ -102,16 +128,8 @@ struct TcCols {
   static_assert(kNeed <= 512, "TMEM budget");
 };
 
-__host__ __device__ constexpr int tc_a_stage_bytes(int NM, int BN, int vbox) {
-  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM == 1 ? kTcRows * 16 * tc_ksub(1, BN) : kTcRows * vbox)) +
-          (NM == 0 ? 0 : kTcRows * 16 * tc_ksub(NM, BN)) + 1023) / 1024 * 1024;
-}
-
 __host__ __device__ constexpr int tc_smem_bytes(int BN, int NM, int vbox) {
-  return 1024 /* alignment slack */ +
-         tc_stages(BN, NM) * (BN * 128 * tc_ksub(NM, BN) + tc_a_stage_bytes(NM, BN, vbox)) +
-         (NM == 1 ? kNmLutWords * 4 : 0) /* 2:4 expansion table, one copy per lane */ +
-         4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
+  return tc_fixed_smem(BN, NM) + tc_stages(BN, NM) * tc_stage_smem(BN, NM, vbox);
 }
 
 // Dense code word of 16 weights (group gi of the stage) of an n:8 row: two
@@ -138,7 +156,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int DCOLS = TcCols<BN, NM>::kDcols;
   constexpr int A_COL0 = TcCols<BN, NM>::kAcol0;
   constexpr int NCOLS = TcCols<BN, NM>::kAlloc;
-  constexpr uint32_t IDESC = idesc_i8_u8s8(kTcRows, BN);
+  constexpr bool SP = NM == 3;  // 2:4 rows on the structured-sparse MMA
+  static_assert(!SP || KSUB == 2, "the sparse stage is one 128-byte swizzle row of kept values");
+  constexpr uint32_t IDESC = SP ? idesc_i8_sp_s8s8(kTcRows, BN) : idesc_i8_u8s8(kTcRows, BN);
+  constexpr int SPA = SP ? tc_sp_a_bytes(BN) : 0;  // compressed A of one stage
   constexpr int B_SUB = BN * 128;         // one 128-wide K sub-tile of the activations
   constexpr int B_STAGE = B_SUB * KSUB;
 
@@ -150,7 +171,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int a_stage = tc_a_stage_bytes(NM, BN, a.vbox);
   uint8_t* sB = base;
   uint8_t* sA = base + S * B_STAGE;
-  uint32_t* s_lut = reinterpret_cast<uint32_t*>(sA + S * a_stage);     // 2:4 only: [256][32] dense code bytes
+  uint8_t* sAs = sA + S * a_stage;                                       // sparse MMA: [S][128 rows][128 B]
+  uint32_t* s_lut = reinterpret_cast<uint32_t*>(sAs + S * SPA);         // expanded 2:4 only: [256][32] code bytes
   uint32_t* s_stage = s_lut + (NM == 1 ? kNmLutWords : 0);               // 4 warps x 32 x 33 words
   float* s_scale = reinterpret_cast<float*>(s_stage + 4 * 32 * 33);     // [2][BN]
   int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * BN);     // [2][BN]
@@ -218,7 +240,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint8_t* dst = sA + s * a_stage;
         if (NM == 0) {
           tma_load_2d(dst, &mapA, kb * 32 * KSUB, row0, &full[s]);
-        } else if (NM == 1) {
+        } else if (NM == 1 || NM == 3) {
           tma_load_2d(dst, &mapA, kb * 16 * KSUB, row0, &full[s]);
           tma_load_2d(dst + a_val_bytes, &mapMeta, kb * 16 * KSUB, row0, &full[s]);
         } else {
@@ -286,11 +308,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           tc_fence_after();
+          if (SP) {
+            // four instructions of 64 k: 32 bytes of kept values, two metadata columns, 64 bytes of B each
+            const uint64_t adesc = smem_desc_sw128_kmajor(smem_u32(sAs + s * SPA));
 #pragma unroll
-          for (int kk = 0; kk < 4 * KSUB; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE + (kk >> 2) * B_SUB));
-            tc_mma_i8_ts(dcol, tmem + A_COL0 + s * SLOT + kk * 8, bdesc + static_cast<uint64_t>((kk & 3) * 2), IDESC,
-                         (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 2 * KSUB; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE + (kk >> 1) * B_SUB));
+              tc_mma_sp_i8_ss(dcol, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>((kk & 1) * 4),
+                              tmem + A_COL0 + s * SLOT + kk * 2, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4 * KSUB; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE + (kk >> 2) * B_SUB));
+              tc_mma_i8_ts(dcol, tmem + A_COL0 + s * SLOT + kk * 8, bdesc + static_cast<uint64_t>((kk & 3) * 2),
+                           IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           tc_commit(&empty[s]);
           issued = true;
@@ -304,12 +337,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp >= 4 && warp < kTcEpiWarp0) {
     // -------------------------------------------------------------- unpack (two groups)
-    const int grp = (warp - 4) >> 2;       // 0: even k-blocks, 1: odd k-blocks
+    // A group takes every use of the stages of its parity, so its parity waits on a
+    // stage never skip a phase.  (Alternating k-blocks would, with an odd stage
+    // count, hand each stage to the two groups in turn, and a group could pass
+    // the wait on a phase that completed two uses earlier.)
+    const int grp = (warp - 4) >> 2;       // 0: even stages, 1: odd stages
     const int q = warp & 3;                // TMEM lane quarter
     const int r = q * 32 + lane;           // weight row inside the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    for (int i = grp; i < total_kb; i += 2) {
+    for (int i = 0; i < total_kb; ++i) {
       const int s = i % S;
+      if ((s & 1) != grp) continue;
       int rt_u, tt_u;
       const int kb = kblock_of(i, rt_u, tt_u);
       if (!mbar_wait(&full[s], (i / S) & 1)) {
@@ -317,6 +355,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       const uint8_t* st = sA + s * a_stage;
+      if (SP) {
+        // 32 bytes of kept codes (128 kept values, 256 k) and 32 of metadata for this row
+        const uint4* vp = reinterpret_cast<const uint4*>(st + r * 32);
+        const uint4* mp = reinterpret_cast<const uint4*>(st + a_val_bytes + r * 32);
+        const uint4 v0 = vp[0], v1 = vp[1], m0 = mp[0], m1 = mp[1];
+        const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint32_t mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        uint8_t* arow_s = sAs + s * SPA + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          // 16 kept codes (32 k) -> 16 int8 weights W_t = code - 1 in kept order: the 16-byte chunk c
+          // of the row's 128-byte swizzle row
+          uint32_t sj[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)  // byte b of sj[j]: kept value 4b + j, as 0x80 + code - 1
+            sj[j] = (((vw[c] >> (2 * j)) & 0x03030303u) | 0x80808080u) - 0x01010101u;
+          const uint32_t t0 = __byte_perm(sj[0], sj[1], 0x5140), t1 = __byte_perm(sj[0], sj[1], 0x7362);
+          const uint32_t t2 = __byte_perm(sj[2], sj[3], 0x5140), t3 = __byte_perm(sj[2], sj[3], 0x7362);
+          const uint4 o = make_uint4(__byte_perm(t0, t2, 0x5410) ^ 0x80808080u, __byte_perm(t0, t2, 0x7632) ^ 0x80808080u,
+                                     __byte_perm(t1, t3, 0x5410) ^ 0x80808080u, __byte_perm(t1, t3, 0x7632) ^ 0x80808080u);
+          *reinterpret_cast<uint4*>(arow_s + ((c ^ (r & 7)) << 4)) = o;
+        }
+        tc_st_32x32b_x8(tmem + lane_base + A_COL0 + s * SLOT, mw);
+        fence_proxy_async_smem();  // the compressed A is read by the tensor cores
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&aready[s]);
+        continue;
+      }
       const uint8_t* arow;
       const uint8_t* mrow = st + a_val_bytes + r * 16 * KSUB;
       int rem = 0;
@@ -421,7 +489,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
           const int tok = tok0 + j;
           scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), a.qb) : 0.0f;  // RN(RN(alpha gamma) / Q_b)
-          rsm[j] = tok < a.M ? a.rowsum[tok] : 0;
+          rsm[j] = (tok < a.M && a.rowsum) ? a.rowsum[tok] : 0;
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == kTcEpiWarp0 * 32)
@@ -495,7 +563,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
         const int tok = tok0 + j;
         scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), a.qb) : 0.0f;  // RN(RN(alpha gamma) / Q_b)
-        rsm[j] = tok < a.M ? a.rowsum[tok] : 0;
+        rsm[j] = (tok < a.M && a.rowsum) ? a.rowsum[tok] : 0;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (!mbar_wait(&accfull[buf], (t >> 1) & 1)) {

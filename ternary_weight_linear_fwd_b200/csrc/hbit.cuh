@@ -90,7 +90,8 @@ __device__ __forceinline__ void hadamard_tile(float (&v)[V], int B, int lane) {
 // One CTA (kHbitThreads) per token row; blocks past M clear the split-K sums
 // and blockIdx 0 the arrival counters of the GEMMs that follow, as
 // quant_act_kernel does.  kPermute: codes in contraction order [M, ldq],
-// ldq = K rounded up to 16 (zeros past K); otherwise natural order, ldq = K.
+// ldq = K rounded up to 16 (zeros past K); otherwise natural order, ldq = K
+// or K rounded up to 16 (then zeros past K as well).
 // V > 0: the transform runs in registers, warps taking the row's tiles of
 // 32 * V elements in turn; V = 0 (blocks of more than 2048): stage by stage
 // over the row in shared memory, with a CTA barrier between stages.  Either
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kHbitThreads) hbit_quant_kernel(const uint16_t
       w.z = cb[2] | (cb[6] << 8) | (cb[10] << 16) | (cb[14] << 24);
       w.w = cb[3] | (cb[7] << 8) | (cb[11] << 16) | (cb[15] << 24);
       *reinterpret_cast<uint4*>(qr + 16 * gi) = w;
-    } else if (16 * gi + 16 <= K && ((reinterpret_cast<uintptr_t>(qr) | (16u * gi)) & 15u) == 0) {
+    } else if (16 * gi + 16 <= ldq && ((reinterpret_cast<uintptr_t>(qr) | (16u * gi)) & 15u) == 0) {
       uint4 w;
       w.x = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
       w.y = cb[4] | (cb[5] << 8) | (cb[6] << 16) | (cb[7] << 24);

@@ -290,6 +290,21 @@ __device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc, 2:4 compressed] * B[smem desc]^T, kind::i8, one
+// CTA, structured-sparse.  A holds the two kept values of every group of four
+// consecutive K (32 bytes per row for the instruction's K = 64); the
+// metadata sits in TMEM at e_tmem: lane = row of A, 4 bits per group of four
+// (kept positions i0 | i1 << 2, i0 < i1), groups in K order from bit 0 of the
+// first of the instruction's two 32-bit columns.
+__device__ __forceinline__ void tc_mma_sp_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on bar when all prior tcgen05 async operations of this thread complete.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -309,6 +324,13 @@ __device__ __forceinline__ void tc_st_32x32b_x32(uint32_t taddr, const uint32_t 
       "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+// Store 8 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tc_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 // Load 32 consecutive 32-bit columns of this thread's TMEM lane.
@@ -344,6 +366,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_kmajor(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t idesc_i8_u8s8(int m, int n) {
   return (2u << 4)                                   // D format: s32
          | (0u << 7)                                 // A: unsigned 8-bit
+         | (1u << 10)                                // B: signed 8-bit
+         | (static_cast<uint32_t>(n >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor for kind::i8 with 2:4 structured sparsity on A:
+// D s32, A and B signed 8-bit, both K-major, sparse flag set (metadata
+// selector 0).
+__host__ __device__ constexpr uint32_t idesc_i8_sp_s8s8(int m, int n) {
+  return (1u << 2)                                   // sparse A
+         | (2u << 4)                                 // D format: s32
+         | (1u << 7)                                 // A: signed 8-bit
          | (1u << 10)                                // B: signed 8-bit
          | (static_cast<uint32_t>(n >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24);    // M / 16

@@ -128,13 +128,17 @@ __device__ __forceinline__ void load8_raw(const uint16_t* row, int k0, int K, bo
 // a CTA of eight (M >= 8 * SMs), a row of up to 256 groups stays in one warp:
 // at M = 2048, K = 2560 that measured faster than two warps joined by the
 // barriers of the fp64 sum, the maximum and the code sum, while for a few rows
-// the shorter per-warp chains of the split win.  gamma is an integer warp max of the
+// the shorter per-warp chains of the split win.  With fewer rows than about
+// 24 warps per SM would take, each row is split further (up to eight warps):
+// at M = 256 and M = 16, K = 2560, eight warps a row took 2.9 and 2.5 us
+// against 4.0 and 3.3 us for two, while at M = 2048 two stayed fastest.  gamma is an integer warp max of the
 // |x| bit patterns (then across the row's warps), and the 16 codes of a group
 // come from the division-free exact rounding of codes8.  Longer or unaligned
 // rows take a two-pass loop (the second pass re-reads from L1/L2).
-// kPermute = false writes natural-order codes [M, ldq] (ldq = K); kPermute =
-// true writes the contraction order [M, ldq] with ldq = K rounded up to 16
-// (zeros past K).  kNorm = true first applies RMSNorm with weight gnorm
+// kPermute = false writes natural-order codes [M, ldq] (ldq = K, or K rounded
+// up to 16 with zeros past K, as the structured-sparse MMA reads them);
+// kPermute = true writes the contraction order [M, ldq] with ldq = K rounded
+// up to 16 (zeros past K).  kNorm = true first applies RMSNorm with weight gnorm
 // ([b158] BitLinear_b158.forward normalises x before activation_quant):
 // r = RN32(1 / sqrt(RN32(sum x^2 / K) + eps)) with the sum, the root and the
 // quotient in fp64, xn = RN(RN(x * r) * g) in fp32, and quantises xn.  Both write gamma and, when asked, the sum of the row's
@@ -153,6 +157,8 @@ __host__ __device__ __forceinline__ QuantShape quant_shape(int M, int K, bool no
   int wpr = 1;
   if (!(norm && groups <= 8 * 32 && M >= kQuantWarps * sm_count))
     while (wpr < kQuantWarps && groups > 3 * 32 * wpr) wpr *= 2;
+  // few rows: split them over more warps until about 24 warps per SM are in flight
+  while (wpr < kQuantWarps && M * wpr < 24 * sm_count && !(norm && M >= kQuantWarps * sm_count)) wpr *= 2;
   const int need = (groups + 32 * wpr - 1) / (32 * wpr);
   return {wpr, need <= 2 ? 2 : need <= 3 ? 3 : 8};
 }
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps, G <= 3 ? 4 : 2) quant_act_ke
       } else {
         w = group_codes<kPermute>(r0, r1, c, d, sum);
       }
-      if (kPermute || (qvec && k0 + 16 <= K)) {
+      if (kPermute || (qvec && k0 + 16 <= ldq)) {
         *reinterpret_cast<uint4*>(qr + k0) = w;
       } else {
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};

@@ -225,3 +225,14 @@ def test_hbit_host_checks(L):
     assert hq(None, 4, 64, 0x1000, 0x2000, None, None) == 1
     assert hq(0x1000, 4, 16385, 0x1000, 0x2000, None, None) == 2
     assert hq(0x1001, 4, 64, 0x1000, 0x2000, None, None) == 3
+
+
+def test_flag_values_match_header():
+    """Every BITLINEAR_FLAG_* of the header has the same value in the binding, and no two flags share a bit."""
+    import ternary_weight_linear_fwd_b200 as bl
+    flags = dict(re.findall(r"#define BITLINEAR_(FLAG_\w+) (0x[0-9a-fA-F]+)u", open(HEADER).read()))
+    assert "FLAG_NM24_EXPAND" in flags and len(flags) >= 6
+    for name, val in flags.items():
+        assert getattr(bl, name) == int(val, 16), name
+    vals = [int(v, 16) for v in flags.values()]
+    assert all(v and (v & (v - 1)) == 0 for v in vals) and len(set(vals)) == len(vals)

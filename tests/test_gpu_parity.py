@@ -382,6 +382,73 @@ def test_forward_nm_m1_forced_tc_matches_gemv():
     _check_rows(x, Wt, a, y1, acc1, np.arange(1))
 
 
+# ---------------------------------------------------------------- 2:4 on the structured-sparse MMA
+
+@pytest.mark.parametrize("M,K,N", [(2, 256, 128), (37, 1032, 300), (300, 2048, 520), (128, 4100, 257),
+                                   (1, 768, 130), (2048, 2048, 1100)])
+def test_forward_nm24_sparse_mma_matches_expanded_and_oracle(M, K, N):
+    """2:4 weights on tcgen05.mma.sp (kept values as int8, packed metadata in TMEM, natural-order codes)
+    against the expanded dense MMA of the same call (bit for bit) and the oracle (every token)."""
+    x, Wt, a, w = _nm_case(M, K, N, 2, 4, seed=K + N)
+    xd = to_dev_bf16(x)
+    y, acc = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_PATH_TC if M == 1 else 0)
+    assert bl.last_kernel().startswith("tc_gemm_sp24"), bl.last_kernel()
+    ye, acce = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_NM24_EXPAND | (bl.FLAG_PATH_TC if M == 1 else 0))
+    assert bl.last_kernel().startswith("tc_gemm_nm24"), bl.last_kernel()
+    assert torch.equal(acc, acce) and torch.equal(y.view(torch.int16), ye.view(torch.int16))
+    _check_rows(x, Wt, a, y, acc, np.arange(M))
+
+
+def test_forward_nm24_sparse_mma_tie_decides_kept_pair():
+    """Blocks whose latent magnitudes tie (all four equal, or three equal largest): the mask rule decides which
+    two positions are kept, the pack must keep the same pair as the oracle, and the sparse MMA must then
+    contract exactly those positions (acc bit-exact against the oracle on every token)."""
+    M, K, N = 96, 512, 160
+    W = synth.latent_weights(N, K, seed=91)
+    base = np.float32(3 * np.abs(W).mean())
+    for r in range(0, N, 3):
+        for b in range(r % 7, K // 4, 5):
+            k0 = 4 * b
+            if (r + b) % 2:
+                W[r, k0:k0 + 4] = np.array([1, -1, 1, -1], np.float32) * base          # all four tie
+            else:
+                W[r, k0:k0 + 4] = np.array([0.5, 1, -1, 1], np.float32) * base         # three tie for two places
+    ref = oracle.pack_weights(W, 2, 4)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV), 2, 4)
+    np.testing.assert_array_equal(w.codes.cpu().numpy(), ref["values"])
+    np.testing.assert_array_equal(w.meta.cpu().numpy(), ref["meta"])
+    x = synth.activations(M, K, seed=92)
+    y, acc = bl.forward_nm(w, to_dev_bf16(x), want_acc=True)
+    assert bl.last_kernel().startswith("tc_gemm_sp24")
+    _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
+
+
+def test_forward_group_all_nm24_uses_sparse_mma():
+    """A group of 2:4 matrices quantises once in natural order and runs each on the sparse MMA; a group
+    mixing dense and 2:4 keeps the contraction order and the expanded MMA.  Both match single calls."""
+    M, K = 40, 1024
+    x = synth.activations(M, K, seed=93)
+    xd = to_dev_bf16(x)
+    specs = [(300, 2, 4), (200, 2, 4)]
+    ws, refs = [], []
+    for i, (N, n, m) in enumerate(specs):
+        W = synth.latent_weights(N, K, seed=94 + i)
+        refs.append(oracle.pack_weights(W, n, m))
+        ws.append(bl.pack_weights(torch.from_numpy(W).to(DEV), n, m))
+    outs = bl.forward_group(ws, xd, want_acc=True)
+    assert bl.last_kernel().startswith("tc_gemm_sp24")
+    for w, ref, (y, acc) in zip(ws, refs, outs):
+        y1, acc1 = bl.forward_nm(w, xd, want_acc=True)
+        assert torch.equal(acc, acc1) and torch.equal(y.view(torch.int16), y1.view(torch.int16))
+        _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
+    Wd = synth.latent_weights(130, K, seed=97)
+    refd = oracle.pack_weights(Wd)
+    wd = bl.pack_weights(torch.from_numpy(Wd).to(DEV))
+    outs = bl.forward_group([ws[0], wd], xd, want_acc=True, flags=bl.FLAG_PATH_PERSISTENT)
+    for ref, (y, acc) in zip([refs[0], refd], outs):
+        _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
+
+
 # ---------------------------------------------------------------- grouped forward
 
 @pytest.mark.parametrize("M", [1, 37])
