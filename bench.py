@@ -867,7 +867,23 @@ def _case_hbit_m1(dev):
         bl.hadamard_quant_act4(x)
 
 
-PROFILE_CASES = {"few_token_m16": _case_few_token, "hbit_m1": _case_hbit_m1}
+def _case_sparse24_m2048(dev):
+    """bitlinear_forward_nm at M = 2048 on the Qwen2.5-3B up projection (2048 -> 11008) pruned 2:4:
+    quantisation in natural K order, then the structured-sparse tensor-core GEMM."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+    W = torch.from_numpy(synth.latent_weights(11008, 2048, seed=5)).to(dev)
+    w = bl.pack_weights(W, 2, 4)
+    del W
+    x = torch.from_numpy(synth.activations(2048, 2048, seed=5).view(np.int16)).to(dev).view(torch.bfloat16)
+    for _ in range(3):
+        bl.forward_nm(w, x)
+
+
+PROFILE_CASES = {"few_token_m16": _case_few_token, "hbit_m1": _case_hbit_m1, "sparse24_m2048": _case_sparse24_m2048}
 
 
 def run_profile_case(name: str):

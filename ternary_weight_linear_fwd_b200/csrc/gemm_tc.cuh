@@ -99,17 +99,21 @@ __host__ __device__ constexpr int tc_slot_cols(int NM, int BN) { return (NM == 3
 constexpr int kTcSmemMax = 232448;  // dynamic shared memory a CTA may opt into
 // Compressed int8 A of one sparse-MMA stage: 128 rows x (stage K / 2) bytes.
 __host__ __device__ constexpr int tc_sp_a_bytes(int BN) { return kTcRows * 64 * tc_ksub(3, BN); }
+// Shared memory of one stage's A: the TMA box(es) of packed weights; for the
+// sparse MMA the compressed operand, which the packed values and metadata
+// (half its size) land in and are unpacked over.
 __host__ __device__ constexpr int tc_a_stage_bytes(int NM, int BN, int vbox) {
-  return ((NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM != 2 ? kTcRows * 16 * tc_ksub(NM, BN) : kTcRows * vbox)) +
-          (NM == 0 ? 0 : kTcRows * 16 * tc_ksub(NM, BN)) + 1023) / 1024 * 1024;
+  return NM == 3 ? tc_sp_a_bytes(BN)
+                 : ((NM == 0 ? kTcRows * 32 * tc_ksub(0, BN) : (NM != 2 ? kTcRows * 16 * tc_ksub(NM, BN) : kTcRows * vbox)) +
+                    (NM == 0 ? 0 : kTcRows * 16 * tc_ksub(NM, BN)) + 1023) / 1024 * 1024;
 }
 __host__ __device__ constexpr int tc_fixed_smem(int BN, int NM) {
   return 1024 /* alignment slack */ + (NM == 1 ? kNmLutWords * 4 : 0) /* 2:4 expansion table, one copy per lane */ +
          4 * 32 * 33 * 4 /* epilogue staging */ + 2 * BN * 8 /* scales, code sums */ + 256 /* barriers */;
 }
-// Shared memory of one pipeline stage (the sparse MMA's operand only for 2:4 rows, vbox fixed).
+// Shared memory of one pipeline stage.
 __host__ __device__ constexpr int tc_stage_smem(int BN, int NM, int vbox) {
-  return BN * 128 * tc_ksub(NM, BN) + tc_a_stage_bytes(NM, BN, vbox) + (NM == 3 ? tc_sp_a_bytes(BN) : 0);
+  return BN * 128 * tc_ksub(NM, BN) + tc_a_stage_bytes(NM, BN, vbox);
 }
 __host__ __device__ constexpr int tc_min3(int a, int b, int c) { return a < b ? (a < c ? a : c) : (b < c ? b : c); }
 // Pipeline stages: as many as TMEM has slots for beside the two accumulators,
@@ -159,7 +163,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr bool SP = NM == 3;  // 2:4 rows on the structured-sparse MMA
   static_assert(!SP || KSUB == 2, "the sparse stage is one 128-byte swizzle row of kept values");
   constexpr uint32_t IDESC = SP ? idesc_i8_sp_s8s8(kTcRows, BN) : idesc_i8_u8s8(kTcRows, BN);
-  constexpr int SPA = SP ? tc_sp_a_bytes(BN) : 0;  // compressed A of one stage
+
   constexpr int B_SUB = BN * 128;         // one 128-wide K sub-tile of the activations
   constexpr int B_STAGE = B_SUB * KSUB;
 
@@ -171,8 +175,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int a_stage = tc_a_stage_bytes(NM, BN, a.vbox);
   uint8_t* sB = base;
   uint8_t* sA = base + S * B_STAGE;
-  uint8_t* sAs = sA + S * a_stage;                                       // sparse MMA: [S][128 rows][128 B]
-  uint32_t* s_lut = reinterpret_cast<uint32_t*>(sAs + S * SPA);         // expanded 2:4 only: [256][32] code bytes
+  // sparse MMA: stage s of sA is the compressed operand [128 rows][128 B] once unpacked
+  uint32_t* s_lut = reinterpret_cast<uint32_t*>(sA + S * a_stage);     // expanded 2:4 only: [256][32] code bytes
   uint32_t* s_stage = s_lut + (NM == 1 ? kNmLutWords : 0);               // 4 warps x 32 x 33 words
   float* s_scale = reinterpret_cast<float*>(s_stage + 4 * 32 * 33);     // [2][BN]
   int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * BN);     // [2][BN]
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_after();
           if (SP) {
             // four instructions of 64 k: 32 bytes of kept values, two metadata columns, 64 bytes of B each
-            const uint64_t adesc = smem_desc_sw128_kmajor(smem_u32(sAs + s * SPA));
+            const uint64_t adesc = smem_desc_sw128_kmajor(smem_u32(sA + s * a_stage));
 #pragma unroll
             for (int kk = 0; kk < 2 * KSUB; ++kk) {
               const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * B_STAGE + (kk >> 1) * B_SUB));
@@ -350,19 +354,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if ((s & 1) != grp) continue;
       int rt_u, tt_u;
       const int kb = kblock_of(i, rt_u, tt_u);
-      if (!mbar_wait(&full[s], (i / S) & 1)) {
+      bool landed = mbar_wait(&full[s], (i / S) & 1);
+      // sparse MMA: the group's four warps unpack over a shared buffer, so they give up together
+      if (SP) landed = bar_red_and(landed, 2 + grp, 128);
+      if (!landed) {
         *a.status = kDevTimeoutUnpack;
         break;
       }
-      const uint8_t* st = sA + s * a_stage;
+      uint8_t* st = sA + s * a_stage;
       if (SP) {
-        // 32 bytes of kept codes (128 kept values, 256 k) and 32 of metadata for this row
+        // 32 bytes of kept codes (128 kept values, 256 k) and 32 of metadata for this row; every
+        // row of the group is read before any is overwritten by the compressed operand
         const uint4* vp = reinterpret_cast<const uint4*>(st + r * 32);
         const uint4* mp = reinterpret_cast<const uint4*>(st + a_val_bytes + r * 32);
         const uint4 v0 = vp[0], v1 = vp[1], m0 = mp[0], m1 = mp[1];
         const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         const uint32_t mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-        uint8_t* arow_s = sAs + s * SPA + (r >> 3) * 1024 + (r & 7) * 128;
+        bar_sync_n(2 + grp, 128);
+        uint8_t* arow_s = st + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           // 16 kept codes (32 k) -> 16 int8 weights W_t = code - 1 in kept order: the 16-byte chunk c
