@@ -16,6 +16,7 @@
 
 #include "../../include/bitlinear.h"
 #include "gemm_skinny.cuh"
+#include "gemm_tc2.cuh"
 
 namespace bl {
 
@@ -52,6 +53,7 @@ struct DeviceState {
   int sm_count = 0;
   int32_t* status = nullptr;
   int sk_clusters[kSkMaxCluster + 1] = {};  // clusters of each size the few-token kernel fits at once (0: not asked)
+  int t2_pairs[2] = {};                     // CTA pairs of the pair GEMM (dense, 2:4) resident at once (0: not asked)
 };
 
 std::mutex g_mu;
@@ -291,6 +293,36 @@ bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA,
   }
 }
 
+// CTA pairs of the pair GEMM resident at once (one CTA per SM), asked once per device.
+template <int NM>
+int t2_active_pairs(DeviceState* dev) {
+  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1];
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (slot == 0) {
+    int n = -1;
+    if (ensure_smem(reinterpret_cast<const void*>(tc2_gemm_kernel<NM>), T2<NM>::SMEM)) {
+      cudaLaunchConfig_t cfg;
+      std::memset(&cfg, 0, sizeof cfg);
+      cfg.gridDim = dim3(2 * 64);
+      cfg.blockDim = dim3(kTcThreads);
+      cfg.dynamicSmemBytes = T2<NM>::SMEM;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, tc2_gemm_kernel<NM>, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = -1;
+      }
+    }
+    slot = n;
+  }
+  return slot;
+}
+
 const char* tc_name(int nm, int bn) {
   static const char* names[4][4] = {
       {"tc_gemm_dense_bn16", "tc_gemm_dense_bn32", "tc_gemm_dense_bn64", "tc_gemm_dense_bn128"},
@@ -455,6 +487,54 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
                  : go(quant_kernel<true, false>(qs.G), static_cast<const float*>(nullptr), 0.0f);
 }
 
+// The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
+template <int NM>
+bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
+                          cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
+  const int pairs_max = t2_active_pairs<NM>(dev);
+  if (pairs_max < 1) return BITLINEAR_ERR_DEVICE;
+  const int N = w->N, K = w->K;
+  CUtensorMap mB, mA, mMeta;
+  if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
+                   kTcSubK, static_cast<uint32_t>(kT2Half), true))
+    return BITLINEAR_ERR_CUDA;
+  if (NM == 0) {
+    const int64_t ld = dense_ld(K);
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * T2<0>::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    mMeta = mA;
+  } else {
+    int64_t ldv = 0, ldm = 0;
+    if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
+      return BITLINEAR_ERR_PATTERN;
+    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, 16 * T2<3>::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16 * T2<3>::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+  }
+  TcArgs ta;
+  std::memset(&ta, 0, sizeof ta);
+  ta.M = M;
+  ta.N = N;
+  ta.K = K;
+  ta.kblocks = plan.kblocks;
+  ta.row_tiles = (N + kT2Rows - 1) / kT2Rows;
+  ta.tok_tiles = (M + kT2Tok - 1) / kT2Tok;
+  ta.ksplit = 1;
+  ta.kbs = plan.kblocks;
+  ta.gamma = qw.gamma;
+  ta.alpha = w->alpha;
+  ta.rowsum = NM == 3 ? nullptr : qw.rowsum;
+  ta.y = y;
+  ta.acc = acc;
+  ta.qb = qb;
+  ta.status = dev->status;
+  ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
+  const int units = ta.row_tiles * ta.tok_tiles;
+  const int pairs = std::min(pairs_max, units);
+  const bitlinear_status st =
+      launch_ex(tc2_gemm_kernel<NM>, dim3(2 * pairs), dim3(kTcThreads), T2<NM>::SMEM, s, true, 2, mB, mA, mMeta, ta);
+  if (st == BITLINEAR_OK) t_last_kernel = NM == 0 ? "tc2_gemm_dense" : "tc2_gemm_sp24";
+  return st;
+}
+
 // natural: the codes in qw are in natural K order (tc_quant(..., natural = true)),
 // which sends 2:4 weights to the structured-sparse MMA.
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
@@ -463,6 +543,11 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? (natural ? 3 : 1) : 2);
   if (natural && nm != 3) return BITLINEAR_ERR_PATTERN;
   const TcPlan plan = tc_plan(M, N, K, nm, dev->sm_count);
+  if ((nm == 0 || nm == 3) && plan.bn == 128 && plan.ksplit == 1) {
+    const bitlinear_status st = nm == 0 ? tc2_gemm<0>(w, M, qw, y, acc, s, dev, qb, plan)
+                                        : tc2_gemm<3>(w, M, qw, y, acc, s, dev, qb, plan);
+    if (st != BITLINEAR_ERR_DEVICE) return st;  // DEVICE: no pair fits at once, take the one-CTA kernel
+  }
   const int bn = plan.bn;
   CUtensorMap mB, mA, mMeta;
   if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),

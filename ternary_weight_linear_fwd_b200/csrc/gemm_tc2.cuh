@@ -1,0 +1,378 @@
+// gemm_tc2.cuh -- many-token BitLinear on pairs of SMs (tcgen05 cta_group::2).
+//
+// The persistent GEMM of gemm_tc.cuh reads, for every 128-row weight tile, the
+// whole activation tile of its tokens from L2: at 128 x 128 tiles the
+// activations are four fifths of the bytes a stage moves, and a copy of the
+// kernel that skipped both the MMAs and the unpacking still took four fifths
+// of the full kernel's time (2048 -> 11008 at M = 4096).  Here two CTAs of a
+// cluster share one MMA of M = 256 weight rows: each CTA holds its own 128
+// weight rows (expanded codes in its TMEM for dense weights, the compressed
+// kept values in its shared memory for 2:4 weights) and HALF of the 128
+// tokens' activation tile, so the activation bytes per MAC halve.
+//
+//   D[256 rows, 128 tokens] += A[256 rows, K] * B[128 tokens, K]^T
+//   CTA r of the pair: rows 128 r .. 128 r + 127 of A and D (its own TMEM),
+//                      tokens 64 r .. 64 r + 63 of B (its own shared memory).
+//
+// Every copy is an ordinary one-CTA TMA load signalling the CTA's own
+// barrier.  The unpack warps of both CTAs wait for their CTA's stage (weights
+// and activations landed), unpack, and arrive on the MMA barrier of the pair's
+// rank-0 CTA (release at cluster scope); rank 0's MMA thread waits there
+// (acquire), issues the pair MMAs and commits them to the stage's "empty"
+// barrier of both CTAs at once (multicast commit), which frees the stage for
+// both producers.  The accumulators work the same way: the commit of a tile
+// reaches both CTAs' epilogues, and both epilogues arrive on rank 0's
+// "accumulator free" barrier.  Each CTA's epilogue stores its own 128 rows.
+// Every wait is bounded; a role that gives up records a status and unwinds,
+// and neither CTA leaves before the other (final cluster barrier), so no
+// remote arrive or multicast commit reaches an exited CTA.
+#pragma once
+#include "gemm_tc.cuh"
+
+namespace bl {
+
+constexpr int kT2Tok = 128;      // tokens of a pair tile (the MMA's N)
+constexpr int kT2Half = 64;      // tokens per CTA
+constexpr int kT2Rows = 256;     // weight rows of a pair tile (the MMA's M)
+
+// 256-k stages; dense: as many as TMEM holds A slots for beside two 128-column
+// accumulators (4); 2:4: as many as shared memory holds (TMEM keeps 8 metadata
+// columns per stage).
+template <int NM>
+struct T2 {
+  static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
+  static constexpr bool SP = NM == 3;
+  static constexpr int KSUB = 2;
+  static constexpr int B_SUB = kT2Half * 128;
+  static constexpr int B_STAGE = B_SUB * KSUB;
+  static constexpr int A_STAGE = SP ? kTcRows * 128 : kTcRows * 64;  // compressed operand / packed codes
+  static constexpr int A_VAL = SP ? kTcRows * 32 : kTcRows * 64;     // TMA bytes of values ...
+  static constexpr int A_META = SP ? kTcRows * 32 : 0;               // ... and metadata per stage
+  static constexpr int SLOT = SP ? 8 : 64;                           // TMEM columns per stage
+  static constexpr int DCOLS = kT2Tok;
+  static constexpr int FIXED = 1024 + 4 * 32 * 33 * 4 + 2 * kT2Tok * 8 + 256;
+  static constexpr int S_SMEM = (kTcSmemMax - FIXED) / (B_STAGE + A_STAGE);
+  static constexpr int S_TMEM = (512 - 2 * DCOLS) / SLOT;
+  static constexpr int S = tc_min3(kTcMaxStages, S_SMEM, S_TMEM) & ~1;  // even: one unpack group per stage parity
+  static constexpr int SMEM = FIXED + S * (B_STAGE + A_STAGE);
+  static constexpr int A_COL0 = 2 * DCOLS;
+  static constexpr uint32_t IDESC = SP ? idesc_i8_sp_s8s8(kT2Rows, kT2Tok) : idesc_i8_u8s8(kT2Rows, kT2Tok);
+};
+
+// Launched in clusters of two CTAs (an even grid); a.row_tiles counts 256-row
+// pair tiles here; no K split (a.ksplit == 1).
+template <int NM>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc2_gemm_kernel(const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapA,
+                    const __grid_constant__ CUtensorMap mapMeta, const TcArgs a) {
+  using C = T2<NM>;
+  constexpr int S = C::S;
+  constexpr bool SP = C::SP;
+  constexpr int KSUB = C::KSUB;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sB = base;
+  uint8_t* sA = base + S * C::B_STAGE;
+  uint32_t* s_stage = reinterpret_cast<uint32_t*>(sA + S * C::A_STAGE);  // 4 warps x 32 x 33 words
+  float* s_scale = reinterpret_cast<float*>(s_stage + 4 * 32 * 33);     // [2][128]
+  int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * kT2Tok);  // [2][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_rowsum + 2 * kT2Tok);
+  uint64_t* empty = full + S;
+  uint64_t* aready = empty + S;     // rank 0's: both CTAs' unpack warps
+  uint64_t* accfull = aready + S;   // [2]
+  uint64_t* accempty = accfull + 2; // [2] rank 0's: both CTAs' epilogue warps
+  uint64_t* drain = accempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int KB = a.kbs;
+  const int nunits = a.row_tiles * a.tok_tiles;
+  const int my_tiles = pair < nunits ? (nunits - 1 - pair) / npairs + 1 : 0;
+  const int total_kb = my_tiles * KB;
+  const uint32_t tx_bytes = static_cast<uint32_t>(C::B_STAGE + C::A_VAL + C::A_META);
+  auto unit_of = [&](int t, int& rt, int& tt) {  // token tile fastest: neighbouring pairs share weight rows
+    const int g = pair + t * npairs;
+    rt = g / a.tok_tiles;
+    tt = g - rt * a.tok_tiles;
+  };
+
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&aready[s], 8);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 8);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&mapB);
+    tma_prefetch_desc(&mapA);
+    if (SP) tma_prefetch_desc(&mapMeta);
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrive or multicast commit
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t aready0 = mapa_shared(smem_u32(aready), 0);
+  const uint32_t accempty0 = mapa_shared(smem_u32(accempty), 0);
+
+  if (warp == 0) {
+    if (lane == 0 && total_kb > 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      auto load_a = [&](int rt, int kb, int s) {
+        uint8_t* dst = sA + s * C::A_STAGE;
+        const int row0 = rt * kT2Rows + static_cast<int>(rank) * kTcRows;
+        if (SP) {
+          tma_load_2d(dst, &mapA, kb * 16 * KSUB, row0, &full[s]);
+          tma_load_2d(dst + C::A_VAL, &mapMeta, kb * 16 * KSUB, row0, &full[s]);
+        } else {
+          tma_load_2d(dst, &mapA, kb * 32 * KSUB, row0, &full[s]);
+        }
+      };
+      auto load_b = [&](int tt, int kb, int s) {
+        const int tok0 = tt * kT2Tok + static_cast<int>(rank) * kT2Half;
+        for (int sub = 0; sub < KSUB; ++sub)
+          tma_load_2d(sB + s * C::B_STAGE + sub * C::B_SUB, &mapB, (kb * KSUB + sub) * kTcSubK, tok0, &full[s]);
+      };
+      const int pre = total_kb < S ? total_kb : S;
+      for (int i = 0; i < pre; ++i) {  // weights do not depend on the preceding kernel
+        int rt, tt;
+        unit_of(i / KB, rt, tt);
+        mbar_arrive_expect_tx(&full[i], tx_bytes);
+        load_a(rt, i % KB, i);
+      }
+      pdl_wait_primary();
+      for (int i = 0; i < pre; ++i) {
+        int rt, tt;
+        unit_of(i / KB, rt, tt);
+        load_b(tt, i % KB, i);
+      }
+      bool ok = true;
+      int i = pre;
+      for (; i < total_kb; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(&empty[s], ((i / S) - 1) & 1)) {
+          *a.status = kDevTimeoutProducer;
+          ok = false;
+          break;
+        }
+        int rt, tt;
+        unit_of(i / KB, rt, tt);
+        mbar_arrive_expect_tx(&full[s], tx_bytes);
+        load_a(rt, i % KB, s);
+        load_b(tt, i % KB, s);
+      }
+      if (!ok) {
+        for (int j = (i - S > 0 ? i - S : 0); j < i; ++j)
+          if (!mbar_wait(&full[j % S], (j / S) & 1)) *a.status = kDevTimeoutDrain;
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0 && total_kb > 0) {
+      // ------------------------------------------------------------ MMA issuer (rank 0 only)
+      bool issued = false, ok = true;
+      for (int t = 0; t < my_tiles && ok; ++t) {
+        const int buf = t & 1;
+        if (t >= 2 && !mbar_wait_cluster(&accempty[buf], ((t >> 1) - 1) & 1)) {
+          *a.status = kDevTimeoutMma;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem + buf * C::DCOLS;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int i = t * KB + kb;
+          const int s = i % S;
+          // both CTAs' unpack warps arrived: both stages landed and both A operands are written
+          if (!mbar_wait_cluster(&aready[s], (i / S) & 1)) {
+            *a.status = kDevTimeoutMma;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (SP) {
+            const uint64_t adesc = smem_desc_sw128_kmajor(smem_u32(sA + s * C::A_STAGE));
+#pragma unroll
+            for (int kk = 0; kk < 2 * KSUB; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * C::B_STAGE + (kk >> 1) * C::B_SUB));
+              tc_mma_sp_i8_ss_pair(dcol, adesc + static_cast<uint64_t>(kk * 2),
+                                   bdesc + static_cast<uint64_t>((kk & 1) * 4), tmem + C::A_COL0 + s * C::SLOT + kk * 2,
+                                   C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4 * KSUB; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * C::B_STAGE + (kk >> 2) * C::B_SUB));
+              tc_mma_i8_ts_pair(dcol, tmem + C::A_COL0 + s * C::SLOT + kk * 8,
+                                bdesc + static_cast<uint64_t>((kk & 3) * 2), C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
+          }
+          tc_commit_pair_mc(&empty[s], 0x3);
+          issued = true;
+        }
+        if (ok) tc_commit_pair_mc(&accfull[buf], 0x3);
+      }
+      if (!ok && issued) {
+        tc_commit_pair(drain);
+        if (!mbar_wait(drain, 0)) *a.status = kDevTimeoutDrain;
+      }
+    }
+  } else if (warp >= 4 && warp < kTcEpiWarp0) {
+    // -------------------------------------------------------------- unpack (both CTAs)
+    const int grp = (warp - 4) >> 2;  // 0: even stages, 1: odd stages (S is even)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    for (int i = grp; i < total_kb; i += 2) {
+      const int s = i % S;
+      bool landed = mbar_wait(&full[s], (i / S) & 1);
+      if (SP) landed = bar_red_and(landed, 2 + grp, 128);
+      if (!landed) {
+        *a.status = kDevTimeoutUnpack;
+        break;
+      }
+      uint8_t* st = sA + s * C::A_STAGE;
+      if (SP) {
+        const uint4* vp = reinterpret_cast<const uint4*>(st + r * 32);
+        const uint4* mp = reinterpret_cast<const uint4*>(st + C::A_VAL + r * 32);
+        const uint4 v0 = vp[0], v1 = vp[1], m0 = mp[0], m1 = mp[1];
+        const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint32_t mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        bar_sync_n(2 + grp, 128);  // every row read before any is overwritten
+        uint8_t* arow_s = st + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t sj[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sj[j] = (((vw[c] >> (2 * j)) & 0x03030303u) | 0x80808080u) - 0x01010101u;
+          const uint32_t t0 = __byte_perm(sj[0], sj[1], 0x5140), t1 = __byte_perm(sj[0], sj[1], 0x7362);
+          const uint32_t t2 = __byte_perm(sj[2], sj[3], 0x5140), t3 = __byte_perm(sj[2], sj[3], 0x7362);
+          const uint4 o = make_uint4(__byte_perm(t0, t2, 0x5410) ^ 0x80808080u, __byte_perm(t0, t2, 0x7632) ^ 0x80808080u,
+                                     __byte_perm(t1, t3, 0x5410) ^ 0x80808080u, __byte_perm(t1, t3, 0x7632) ^ 0x80808080u);
+          *reinterpret_cast<uint4*>(arow_s + ((c ^ (r & 7)) << 4)) = o;
+        }
+        tc_st_32x32b_x8(tmem + lane_base + C::A_COL0 + s * C::SLOT, mw);
+        fence_proxy_async_smem();
+      } else {
+        const uint8_t* arow = st + r * 64;
+#pragma unroll
+        for (int sub = 0; sub < KSUB; ++sub) {
+          const uint4 lo = reinterpret_cast<const uint4*>(arow)[2 * sub];
+          const uint4 hi = reinterpret_cast<const uint4*>(arow)[2 * sub + 1];
+          const uint32_t dw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          uint32_t outw[32];
+#pragma unroll
+          for (int gi = 0; gi < 8; ++gi) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) outw[4 * gi + j] = (dw[gi] >> (2 * j)) & 0x03030303u;
+          }
+          tc_st_32x32b_x32(tmem + lane_base + C::A_COL0 + s * C::SLOT + sub * 32, outw);
+        }
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(aready0 + static_cast<uint32_t>(s * 8));
+    }
+  } else if (warp >= kTcEpiWarp0) {
+    // -------------------------------------------------------------- epilogue (both CTAs, own rows)
+    const int q = warp - kTcEpiWarp0;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t* stg = s_stage + q * 32 * 33;
+    const float alpha = *a.alpha;
+    pdl_wait_primary();
+    for (int t = 0; t < my_tiles; ++t) {
+      const int buf = t & 1;
+      int rt, tt;
+      unit_of(t, rt, tt);
+      const int row0 = rt * kT2Rows + static_cast<int>(rank) * kTcRows + q * 32;
+      const int tok0 = tt * kT2Tok;
+      float* scl = s_scale + buf * kT2Tok;
+      int32_t* rsm = s_rowsum + buf * kT2Tok;
+      for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < kT2Tok; j += 128) {
+        const int tok = tok0 + j;
+        scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), a.qb) : 0.0f;  // RN(RN(alpha gamma) / Q_b)
+        rsm[j] = (tok < a.M && a.rowsum) ? a.rowsum[tok] : 0;
+      }
+      bar_sync_n(1, 128);
+      if (!mbar_wait(&accfull[buf], (t >> 1) & 1)) {
+        *a.status = kDevTimeoutEpilogue;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < kT2Tok; c0 += 32) {
+        uint32_t v[32];
+        tc_ld_32x32b_x32(tmem + lane_base + buf * C::DCOLS + c0, v);
+        tc_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stg[j * 33 + lane] = v[j];
+        __syncwarp();
+        const int tcol = c0 + lane;
+        const int tok = tok0 + tcol;
+        if (tok < a.M) {
+          const float sc = scl[tcol];
+          const int32_t rs = rsm[tcol];
+          const size_t o = static_cast<size_t>(tok) * a.N + row0;
+          if (a.vec_store && row0 + 32 <= a.N) {
+            uint32_t hb[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int32_t t0 = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
+              const int32_t t1 = static_cast<int32_t>(stg[lane * 33 + e + 1]) - rs;
+              const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t0), sc));
+              const __nv_bfloat16 h1 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t1), sc));
+              hb[e >> 1] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h0)) |
+                           (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h1)) << 16);
+              if (a.acc) {
+                stg[lane * 33 + e] = static_cast<uint32_t>(t0);
+                stg[lane * 33 + e + 1] = static_cast<uint32_t>(t1);
+              }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.y + o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(hb[4 * e], hb[4 * e + 1], hb[4 * e + 2], hb[4 * e + 3]);
+            if (a.acc) {
+              uint4* da = reinterpret_cast<uint4*>(a.acc + o);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                da[e] = make_uint4(stg[lane * 33 + 4 * e], stg[lane * 33 + 4 * e + 1], stg[lane * 33 + 4 * e + 2],
+                                   stg[lane * 33 + 4 * e + 3]);
+            }
+          } else {
+            for (int e = 0; e < 32 && row0 + e < a.N; ++e) {
+              const int32_t tv = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
+              if (a.acc) a.acc[o + e] = tv;
+              const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), sc));
+              a.y[o + e] = *reinterpret_cast<const uint16_t*>(&h);
+            }
+          }
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(accempty0 + static_cast<uint32_t>(buf * 8));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no remote arrive or multicast commit is left in flight towards either CTA
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+}  // namespace bl

@@ -176,7 +176,7 @@ def test_forward_tc_full(M, K, N):
     assert bl.last_kernel().startswith(("tc_gemm_dense", "tc_skinny"))
     _check_rows(x, Wt, a, y, acc, np.arange(M))
     y2, acc2 = bl.forward(w, to_dev_bf16(x), want_acc=True, flags=bl.FLAG_PATH_TC | bl.FLAG_PATH_PERSISTENT)
-    assert bl.last_kernel().startswith("tc_gemm_dense")
+    assert bl.last_kernel().startswith(("tc_gemm_dense", "tc2_gemm_dense"))
     assert torch.equal(acc, acc2) and torch.equal(y.view(torch.int16), y2.view(torch.int16))
 
 
@@ -246,7 +246,7 @@ def test_forward_layer_sweep_m4096_sampled():
     for name, (K, N) in synth.B2B4T_LAYER.items():
         x, Wt, a, w = _dense_case(M, K, N, seed=4)
         y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
-        assert bl.last_kernel().startswith("tc_gemm_dense"), (name, bl.last_kernel())
+        assert bl.last_kernel().startswith(("tc_gemm_dense", "tc2_gemm_dense")), (name, bl.last_kernel())
         _check_rows(x, Wt, a, y, acc, rows)
 
 
@@ -260,7 +260,7 @@ def test_forward_stale_workspace():
     for M, K, N in cases:
         x, Wt, a, w = _dense_case(M, K, N, seed=M + N)
         y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, workspace=ws, flags=bl.FLAG_PATH_PERSISTENT)
-        assert bl.last_kernel().startswith("tc_gemm_dense")
+        assert bl.last_kernel().startswith(("tc_gemm_dense", "tc2_gemm_dense"))
         _check_rows(x, Wt, a, y, acc, np.arange(M))
         ws.fill_(0xFF)
 
@@ -392,7 +392,7 @@ def test_forward_nm24_sparse_mma_matches_expanded_and_oracle(M, K, N):
     x, Wt, a, w = _nm_case(M, K, N, 2, 4, seed=K + N)
     xd = to_dev_bf16(x)
     y, acc = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_PATH_TC if M == 1 else 0)
-    assert bl.last_kernel().startswith("tc_gemm_sp24"), bl.last_kernel()
+    assert bl.last_kernel().startswith(("tc_gemm_sp24", "tc2_gemm_sp24")), bl.last_kernel()
     ye, acce = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_NM24_EXPAND | (bl.FLAG_PATH_TC if M == 1 else 0))
     assert bl.last_kernel().startswith("tc_gemm_nm24"), bl.last_kernel()
     assert torch.equal(acc, acce) and torch.equal(y.view(torch.int16), ye.view(torch.int16))
@@ -419,7 +419,7 @@ def test_forward_nm24_sparse_mma_tie_decides_kept_pair():
     np.testing.assert_array_equal(w.meta.cpu().numpy(), ref["meta"])
     x = synth.activations(M, K, seed=92)
     y, acc = bl.forward_nm(w, to_dev_bf16(x), want_acc=True)
-    assert bl.last_kernel().startswith("tc_gemm_sp24")
+    assert bl.last_kernel().startswith(("tc_gemm_sp24", "tc2_gemm_sp24"))
     _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
 
 
@@ -436,7 +436,7 @@ def test_forward_group_all_nm24_uses_sparse_mma():
         refs.append(oracle.pack_weights(W, n, m))
         ws.append(bl.pack_weights(torch.from_numpy(W).to(DEV), n, m))
     outs = bl.forward_group(ws, xd, want_acc=True)
-    assert bl.last_kernel().startswith("tc_gemm_sp24")
+    assert bl.last_kernel().startswith(("tc_gemm_sp24", "tc2_gemm_sp24"))
     for w, ref, (y, acc) in zip(ws, refs, outs):
         y1, acc1 = bl.forward_nm(w, xd, want_acc=True)
         assert torch.equal(acc, acc1) and torch.equal(y.view(torch.int16), y1.view(torch.int16))
@@ -447,6 +447,35 @@ def test_forward_group_all_nm24_uses_sparse_mma():
     outs = bl.forward_group([ws[0], wd], xd, want_acc=True, flags=bl.FLAG_PATH_PERSISTENT)
     for ref, (y, acc) in zip([refs[0], refd], outs):
         _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
+
+
+# ---------------------------------------------------------------- pairs of SMs (cta_group::2)
+
+# Shapes whose plan is 128-token tiles without a K split (at least 75 tiles of 128 x 128), so the GEMM
+# runs on CTA pairs sharing one M = 256 MMA: ragged M (a last tile of 1 or 44 tokens), ragged N (the
+# last pair tile's second CTA partly or wholly past N), K not a multiple of the 256-k stage.
+@pytest.mark.parametrize("M,K,N", [(1000, 2560, 2000), (4096, 1032, 640), (300, 2048, 11008), (129, 6912, 9000)])
+def test_forward_pair_gemm_dense(M, K, N):
+    x, Wt, a, w = _dense_case(M, K, N, seed=M + K + N)
+    y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
+    assert bl.last_kernel() == "tc2_gemm_dense", bl.last_kernel()
+    rows = np.arange(M) if M * N <= 3_000_000 else np.unique(np.concatenate(
+        [[0, 63, 64, 127, 128, M - 1], synth.splitmix64(M, 7, 18) % M])).astype(np.int64)
+    _check_rows(x, Wt, a, y, acc, rows)
+
+
+@pytest.mark.parametrize("M,K,N", [(1000, 2048, 2000), (129, 4096, 9000), (2048, 11008, 2048)])
+def test_forward_pair_gemm_sparse24(M, K, N):
+    """2:4 weights on the pair's structured-sparse MMA, against the expanded one-CTA kernel (bit for bit)
+    and the oracle (sampled tokens)."""
+    x, Wt, a, w = _nm_case(M, K, N, 2, 4, seed=M + K)
+    xd = to_dev_bf16(x)
+    y, acc = bl.forward_nm(w, xd, want_acc=True)
+    assert bl.last_kernel() == "tc2_gemm_sp24", bl.last_kernel()
+    ye, acce = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_NM24_EXPAND)
+    assert torch.equal(acc, acce) and torch.equal(y.view(torch.int16), ye.view(torch.int16))
+    rows = np.unique(np.concatenate([[0, 63, 64, M - 1], synth.splitmix64(M, 8, 12) % M])).astype(np.int64)
+    _check_rows(x, Wt, a, y, acc, rows)
 
 
 # ---------------------------------------------------------------- grouped forward
