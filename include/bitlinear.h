@@ -336,7 +336,12 @@ bitlinear_status bitlinear_forward_noalloc(const bitlinear_weights* w, const uin
                                            int32_t* acc, uint32_t flags, void* stream);
 
 /* Synchronises stream and reads the current device's status word into *code
- * (0 = no kernel gave up on a wait).  If clear != 0 the word is reset. */
+ * (0 = no kernel gave up on a wait).  If clear != 0 the word is reset.
+ * Codes: 1 weight/activation copies, 2 weight unpacking, 3 MMA issue, 4
+ * epilogue (the role whose wait ran out); 5 the wait for copies or MMAs
+ * already issued ran out as well; 6 a kernel found its dynamic shared memory
+ * misaligned and did nothing.  Outputs of a call that set a code are
+ * undefined. */
 bitlinear_status bitlinear_device_status(void* stream, int32_t* code, int32_t clear);
 
 /* Name of the kernel variant the last successful call on this host thread

@@ -150,6 +150,46 @@ __device__ __forceinline__ uint32_t tc_n8_group_word(const uint8_t* arow, const 
   return n8_dense_block(m0, kv & fmask) | (n8_dense_block(m1, (kv >> (2 * n)) & fmask) << 16);
 }
 
+// Rescales and stores the first ntok (<= 32) tokens of one warp's 32
+// accumulator rows, as read from TMEM (v[j] = D[row][tokb + j], lane = row),
+// tokens past M skipped: for each token the 32 lanes
+// write its 32 consecutive outputs, 64 contiguous bytes of y (128 of acc)
+// per store, straight from the lane layout.  scl / rsm: the tokens' scales and
+// code sums (broadcast reads from shared memory).
+__device__ __forceinline__ void tc_store_token_rows(const uint32_t (&v)[32], const float* scl, const int32_t* rsm,
+                                                    int row, int tokb, int ntok, const TcArgs& a) {
+  if (row >= a.N) return;
+  if (ntok > a.M - tokb) ntok = a.M - tokb;
+  uint16_t* yr = a.y + static_cast<size_t>(tokb) * a.N + row;
+  int32_t* ar = a.acc ? a.acc + static_cast<size_t>(tokb) * a.N + row : nullptr;
+  if (ntok == 32) {
+    // a full chunk: scales and sums as 16-byte broadcast reads, then 32 independent stores
+    float sc[32];
+    int32_t rs[32];
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(scl + j);
+      const int4 r = *reinterpret_cast<const int4*>(rsm + j);
+      sc[j] = f.x; sc[j + 1] = f.y; sc[j + 2] = f.z; sc[j + 3] = f.w;
+      rs[j] = r.x; rs[j + 1] = r.y; rs[j + 2] = r.z; rs[j + 3] = r.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int32_t tv = static_cast<int32_t>(v[j]) - rs[j];
+      const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), sc[j]));
+      yr[static_cast<size_t>(j) * a.N] = *reinterpret_cast<const uint16_t*>(&h);
+      if (ar) ar[static_cast<size_t>(j) * a.N] = tv;
+    }
+    return;
+  }
+  for (int j = 0; j < ntok; ++j) {
+    const int32_t tv = static_cast<int32_t>(v[j]) - rsm[j];
+    const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), scl[j]));
+    yr[static_cast<size_t>(j) * a.N] = *reinterpret_cast<const uint16_t*>(&h);
+    if (ar) ar[static_cast<size_t>(j) * a.N] = tv;
+  }
+}
+
 template <int BN, int NM>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapA,
@@ -585,51 +625,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t v[32];
         tc_ld_32x32b_x32(tmem + lane_base + buf * DCOLS + c0, v);
         tc_wait_ld();
-        // transpose through shared memory: lane l then owns token c0 + l
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stg[j * 33 + lane] = v[j];
-        __syncwarp();
-        const int tcol = c0 + lane;
-        const int tok = tok0 + tcol;
-        if (tcol < BN && tok < a.M) {
-          const float sc = scl[tcol];
-          const int32_t rs = rsm[tcol];
-          const size_t o = static_cast<size_t>(tok) * a.N + row0;
-          if (a.vec_store && row0 + 32 <= a.N) {
-            uint32_t hb[16];
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int32_t t0 = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
-              const int32_t t1 = static_cast<int32_t>(stg[lane * 33 + e + 1]) - rs;
-              const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t0), sc));
-              const __nv_bfloat16 h1 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t1), sc));
-              hb[e >> 1] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h0)) |
-                           (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h1)) << 16);
-              if (a.acc) {
-                stg[lane * 33 + e] = static_cast<uint32_t>(t0);
-                stg[lane * 33 + e + 1] = static_cast<uint32_t>(t1);
-              }
-            }
-            uint4* dst = reinterpret_cast<uint4*>(a.y + o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(hb[4 * e], hb[4 * e + 1], hb[4 * e + 2], hb[4 * e + 3]);
-            if (a.acc) {
-              uint4* da = reinterpret_cast<uint4*>(a.acc + o);
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                da[e] = make_uint4(stg[lane * 33 + 4 * e], stg[lane * 33 + 4 * e + 1], stg[lane * 33 + 4 * e + 2],
-                                   stg[lane * 33 + 4 * e + 3]);
-            }
-          } else {
-            for (int e = 0; e < 32 && row0 + e < a.N; ++e) {
-              const int32_t tv = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
-              if (a.acc) a.acc[o + e] = tv;
-              const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), sc));
-              a.y[o + e] = *reinterpret_cast<const uint16_t*>(&h);
-            }
-          }
-        }
-        __syncwarp();
+        tc_store_token_rows(v, scl + c0, rsm + c0, row0 + lane, tok0 + c0, BN - c0 < 32 ? BN - c0 : 32, a);
       }
       tc_fence_before();
       __syncwarp();

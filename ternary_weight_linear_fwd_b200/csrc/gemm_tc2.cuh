@@ -14,11 +14,21 @@
 //   CTA r of the pair: rows 128 r .. 128 r + 127 of A and D (its own TMEM),
 //                      tokens 64 r .. 64 r + 63 of B (its own shared memory).
 //
+// Two rings: S copy stages in shared memory (the CTA's half of the activation
+// tile and its packed weights) and R operand slots (expanded codes in TMEM, or
+// compressed kept values in shared memory plus metadata in TMEM).  A copy
+// stage is freed when the MMAs that read its activations complete, an operand
+// slot likewise; S > R lets the copies run further ahead of the MMAs than the
+// operand slots alone would allow: the copies' latency from L2 (about 2 us
+// per round trip under this load) needs about eight stages in flight.
+//
 // Every copy is an ordinary one-CTA TMA load signalling the CTA's own
 // barrier.  The unpack warps of both CTAs wait for their CTA's stage (weights
 // and activations landed), unpack, and arrive on the MMA barrier of the pair's
-// rank-0 CTA (release at cluster scope); rank 0's MMA thread waits there
-// (acquire), issues the pair MMAs and commits them to the stage's "empty"
+// rank-0 CTA (tcgen05 / async-proxy fences first, then a CTA-scope release
+// arrive: a cluster-scope release cost about 1500 cycles per arrive and made
+// the unpacking the bottleneck); rank 0's MMA thread waits there (acquire at
+// cluster scope), issues the pair MMAs and commits them to the stage's "empty"
 // barrier of both CTAs at once (multicast commit), which frees the stage for
 // both producers.  The accumulators work the same way: the commit of a tile
 // reaches both CTAs' epilogues, and both epilogues arrive on rank 0's
@@ -35,9 +45,9 @@ constexpr int kT2Tok = 128;      // tokens of a pair tile (the MMA's N)
 constexpr int kT2Half = 64;      // tokens per CTA
 constexpr int kT2Rows = 256;     // weight rows of a pair tile (the MMA's M)
 
-// 256-k stages; dense: as many as TMEM holds A slots for beside two 128-column
-// accumulators (4); 2:4: as many as shared memory holds (TMEM keeps 8 metadata
-// columns per stage).
+// 256-k stages.  Dense: 8 copy stages of 24 KB, 4 operand slots of 64 TMEM
+// columns beside two 128-column accumulators.  2:4: 6 copy stages of 24 KB and
+// 4 slots of 16 KB compressed operand (+ 8 metadata columns each).
 template <int NM>
 struct T2 {
   static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
@@ -45,17 +55,20 @@ struct T2 {
   static constexpr int KSUB = 2;
   static constexpr int B_SUB = kT2Half * 128;
   static constexpr int B_STAGE = B_SUB * KSUB;
-  static constexpr int A_STAGE = SP ? kTcRows * 128 : kTcRows * 64;  // compressed operand / packed codes
   static constexpr int A_VAL = SP ? kTcRows * 32 : kTcRows * 64;     // TMA bytes of values ...
   static constexpr int A_META = SP ? kTcRows * 32 : 0;               // ... and metadata per stage
-  static constexpr int SLOT = SP ? 8 : 64;                           // TMEM columns per stage
+  static constexpr int STAGE = B_STAGE + A_VAL + A_META;             // one copy stage
+  static constexpr int OPA = SP ? kTcRows * 128 : 0;                 // compressed operand in shared memory
+  static constexpr int SLOT = SP ? 8 : 64;                           // TMEM columns per operand slot
   static constexpr int DCOLS = kT2Tok;
-  static constexpr int FIXED = 1024 + 4 * 32 * 33 * 4 + 2 * kT2Tok * 8 + 256;
-  static constexpr int S_SMEM = (kTcSmemMax - FIXED) / (B_STAGE + A_STAGE);
-  static constexpr int S_TMEM = (512 - 2 * DCOLS) / SLOT;
-  static constexpr int S = tc_min3(kTcMaxStages, S_SMEM, S_TMEM) & ~1;  // even: one unpack group per stage parity
-  static constexpr int SMEM = FIXED + S * (B_STAGE + A_STAGE);
+  static constexpr int R = 4;                                        // operand slots
+  // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
+  static constexpr int FIXED = 2 * kT2Tok * 8 + 256;
+  static constexpr int S = tc_min3(kTcMaxStages, (kTcSmemMax - FIXED - R * OPA) / STAGE, 64) & ~1;  // even
+  static constexpr int SMEM = FIXED + S * STAGE + R * OPA;
   static constexpr int A_COL0 = 2 * DCOLS;
+  static_assert(A_COL0 + R * SLOT <= 512, "TMEM budget");
+  static_assert(S >= R, "copy ring at least as deep as the operand ring");
   static constexpr uint32_t IDESC = SP ? idesc_i8_sp_s8s8(kT2Rows, kT2Tok) : idesc_i8_u8s8(kT2Rows, kT2Tok);
 };
 
@@ -70,17 +83,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr bool SP = C::SP;
   constexpr int KSUB = C::KSUB;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sB = base;
-  uint8_t* sA = base + S * C::B_STAGE;
-  uint32_t* s_stage = reinterpret_cast<uint32_t*>(sA + S * C::A_STAGE);  // 4 warps x 32 x 33 words
-  float* s_scale = reinterpret_cast<float*>(s_stage + 4 * 32 * 33);     // [2][128]
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // both CTAs see the same offset, so both leave here together (before any cluster barrier)
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0) *a.status = kDevBadSmemAlign;
+    return;
+  }
+  uint8_t* base = smem_raw;
+  constexpr int R = C::R;
+  uint8_t* sStage = base;                        // [S][B half | packed values | metadata]
+  uint8_t* sOp = base + S * C::STAGE;            // 2:4: [R][128 rows][128 B] compressed operand
+  float* s_scale = reinterpret_cast<float*>(sOp + R * C::OPA);           // [2][128]
   int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * kT2Tok);  // [2][128]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_rowsum + 2 * kT2Tok);
   uint64_t* empty = full + S;
-  uint64_t* aready = empty + S;     // rank 0's: both CTAs' unpack warps
-  uint64_t* accfull = aready + S;   // [2]
+  uint64_t* aready = empty + S;     // [R] rank 0's: both CTAs' unpack warps
+  uint64_t* afree = aready + R;     // [R] operand slot read by the MMAs (multicast commit)
+  uint64_t* accfull = afree + R;    // [2]
   uint64_t* accempty = accfull + 2; // [2] rank 0's: both CTAs' epilogue warps
   uint64_t* drain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -104,7 +123,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&aready[s], 8);
+    }
+    for (int j = 0; j < R; ++j) {
+      mbar_init(&aready[j], 8);
+      mbar_init(&afree[j], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
@@ -131,7 +153,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0 && total_kb > 0) {
       // ------------------------------------------------------------ producer (both CTAs)
       auto load_a = [&](int rt, int kb, int s) {
-        uint8_t* dst = sA + s * C::A_STAGE;
+        uint8_t* dst = sStage + s * C::STAGE + C::B_STAGE;
         const int row0 = rt * kT2Rows + static_cast<int>(rank) * kTcRows;
         if (SP) {
           tma_load_2d(dst, &mapA, kb * 16 * KSUB, row0, &full[s]);
@@ -143,7 +165,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       auto load_b = [&](int tt, int kb, int s) {
         const int tok0 = tt * kT2Tok + static_cast<int>(rank) * kT2Half;
         for (int sub = 0; sub < KSUB; ++sub)
-          tma_load_2d(sB + s * C::B_STAGE + sub * C::B_SUB, &mapB, (kb * KSUB + sub) * kTcSubK, tok0, &full[s]);
+          tma_load_2d(sStage + s * C::STAGE + sub * C::B_SUB, &mapB, (kb * KSUB + sub) * kTcSubK, tok0, &full[s]);
       };
       const int pre = total_kb < S ? total_kb : S;
       for (int i = 0; i < pre; ++i) {  // weights do not depend on the preceding kernel
@@ -193,32 +215,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t dcol = tmem + buf * C::DCOLS;
         for (int kb = 0; kb < KB; ++kb) {
           const int i = t * KB + kb;
-          const int s = i % S;
-          // both CTAs' unpack warps arrived: both stages landed and both A operands are written
-          if (!mbar_wait_cluster(&aready[s], (i / S) & 1)) {
+          const int s = i % S, j = i % R;
+          // both CTAs' unpack warps arrived: both stages landed and both operands are written
+          if (!mbar_wait_cluster(&aready[j], (i / R) & 1)) {
             *a.status = kDevTimeoutMma;
             ok = false;
             break;
           }
           tc_fence_after();
+          const uint8_t* sB = sStage + s * C::STAGE;
           if (SP) {
-            const uint64_t adesc = smem_desc_sw128_kmajor(smem_u32(sA + s * C::A_STAGE));
+            const uint64_t adesc = smem_desc_sw128_kmajor(smem_u32(sOp + j * C::OPA));
 #pragma unroll
             for (int kk = 0; kk < 2 * KSUB; ++kk) {
-              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * C::B_STAGE + (kk >> 1) * C::B_SUB));
+              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + (kk >> 1) * C::B_SUB));
               tc_mma_sp_i8_ss_pair(dcol, adesc + static_cast<uint64_t>(kk * 2),
-                                   bdesc + static_cast<uint64_t>((kk & 1) * 4), tmem + C::A_COL0 + s * C::SLOT + kk * 2,
+                                   bdesc + static_cast<uint64_t>((kk & 1) * 4), tmem + C::A_COL0 + j * C::SLOT + kk * 2,
                                    C::IDESC, (kb | kk) != 0 ? 1u : 0u);
             }
           } else {
 #pragma unroll
             for (int kk = 0; kk < 4 * KSUB; ++kk) {
-              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + s * C::B_STAGE + (kk >> 2) * C::B_SUB));
-              tc_mma_i8_ts_pair(dcol, tmem + C::A_COL0 + s * C::SLOT + kk * 8,
+              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + (kk >> 2) * C::B_SUB));
+              tc_mma_i8_ts_pair(dcol, tmem + C::A_COL0 + j * C::SLOT + kk * 8,
                                 bdesc + static_cast<uint64_t>((kk & 3) * 2), C::IDESC, (kb | kk) != 0 ? 1u : 0u);
             }
           }
           tc_commit_pair_mc(&empty[s], 0x3);
+          tc_commit_pair_mc(&afree[j], 0x3);
           issued = true;
         }
         if (ok) tc_commit_pair_mc(&accfull[buf], 0x3);
@@ -230,27 +254,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp >= 4 && warp < kTcEpiWarp0) {
     // -------------------------------------------------------------- unpack (both CTAs)
-    const int grp = (warp - 4) >> 2;  // 0: even stages, 1: odd stages (S is even)
+    // group g takes the k-blocks of parity g: with S and R even, every use of
+    // its copy stages and operand slots, so no parity wait skips a phase
+    const int grp = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     for (int i = grp; i < total_kb; i += 2) {
-      const int s = i % S;
-      bool landed = mbar_wait(&full[s], (i / S) & 1);
-      if (SP) landed = bar_red_and(landed, 2 + grp, 128);
-      if (!landed) {
+      const int s = i % S, j = i % R;
+      if (!mbar_wait(&full[s], (i / S) & 1) || (i >= R && !mbar_wait(&afree[j], ((i / R) - 1) & 1))) {
         *a.status = kDevTimeoutUnpack;
         break;
       }
-      uint8_t* st = sA + s * C::A_STAGE;
+      const uint8_t* st = sStage + s * C::STAGE + C::B_STAGE;
       if (SP) {
         const uint4* vp = reinterpret_cast<const uint4*>(st + r * 32);
         const uint4* mp = reinterpret_cast<const uint4*>(st + C::A_VAL + r * 32);
         const uint4 v0 = vp[0], v1 = vp[1], m0 = mp[0], m1 = mp[1];
         const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         const uint32_t mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-        bar_sync_n(2 + grp, 128);  // every row read before any is overwritten
-        uint8_t* arow_s = st + (r >> 3) * 1024 + (r & 7) * 128;
+        uint8_t* arow_s = sOp + j * C::OPA + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t sj[4];
@@ -262,7 +285,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                      __byte_perm(t1, t3, 0x5410) ^ 0x80808080u, __byte_perm(t1, t3, 0x7632) ^ 0x80808080u);
           *reinterpret_cast<uint4*>(arow_s + ((c ^ (r & 7)) << 4)) = o;
         }
-        tc_st_32x32b_x8(tmem + lane_base + C::A_COL0 + s * C::SLOT, mw);
+        tc_st_32x32b_x8(tmem + lane_base + C::A_COL0 + j * C::SLOT, mw);
         fence_proxy_async_smem();
       } else {
         const uint8_t* arow = st + r * 64;
@@ -277,19 +300,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) outw[4 * gi + j] = (dw[gi] >> (2 * j)) & 0x03030303u;
           }
-          tc_st_32x32b_x32(tmem + lane_base + C::A_COL0 + s * C::SLOT + sub * 32, outw);
+          tc_st_32x32b_x32(tmem + lane_base + C::A_COL0 + j * C::SLOT + sub * 32, outw);
         }
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(aready0 + static_cast<uint32_t>(s * 8));
+      if (lane == 0) mbar_arrive_remote_cta(aready0 + static_cast<uint32_t>(j * 8));
     }
   } else if (warp >= kTcEpiWarp0) {
     // -------------------------------------------------------------- epilogue (both CTAs, own rows)
     const int q = warp - kTcEpiWarp0;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t* stg = s_stage + q * 32 * 33;
     const float alpha = *a.alpha;
     pdl_wait_primary();
     for (int t = 0; t < my_tiles; ++t) {
@@ -316,54 +338,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t v[32];
         tc_ld_32x32b_x32(tmem + lane_base + buf * C::DCOLS + c0, v);
         tc_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stg[j * 33 + lane] = v[j];
-        __syncwarp();
-        const int tcol = c0 + lane;
-        const int tok = tok0 + tcol;
-        if (tok < a.M) {
-          const float sc = scl[tcol];
-          const int32_t rs = rsm[tcol];
-          const size_t o = static_cast<size_t>(tok) * a.N + row0;
-          if (a.vec_store && row0 + 32 <= a.N) {
-            uint32_t hb[16];
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int32_t t0 = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
-              const int32_t t1 = static_cast<int32_t>(stg[lane * 33 + e + 1]) - rs;
-              const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t0), sc));
-              const __nv_bfloat16 h1 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(t1), sc));
-              hb[e >> 1] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h0)) |
-                           (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h1)) << 16);
-              if (a.acc) {
-                stg[lane * 33 + e] = static_cast<uint32_t>(t0);
-                stg[lane * 33 + e + 1] = static_cast<uint32_t>(t1);
-              }
-            }
-            uint4* dst = reinterpret_cast<uint4*>(a.y + o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(hb[4 * e], hb[4 * e + 1], hb[4 * e + 2], hb[4 * e + 3]);
-            if (a.acc) {
-              uint4* da = reinterpret_cast<uint4*>(a.acc + o);
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                da[e] = make_uint4(stg[lane * 33 + 4 * e], stg[lane * 33 + 4 * e + 1], stg[lane * 33 + 4 * e + 2],
-                                   stg[lane * 33 + 4 * e + 3]);
-            }
-          } else {
-            for (int e = 0; e < 32 && row0 + e < a.N; ++e) {
-              const int32_t tv = static_cast<int32_t>(stg[lane * 33 + e]) - rs;
-              if (a.acc) a.acc[o + e] = tv;
-              const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), sc));
-              a.y[o + e] = *reinterpret_cast<const uint16_t*>(&h);
-            }
-          }
-        }
-        __syncwarp();
+        tc_store_token_rows(v, scl + c0, rsm + c0, row0 + lane, tok0 + c0, 32, a);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(accempty0 + static_cast<uint32_t>(buf * 8));
+      if (lane == 0) mbar_arrive_remote_cta(accempty0 + static_cast<uint32_t>(buf * 8));
     }
   }
   tc_fence_before();

@@ -19,6 +19,7 @@ enum : int32_t {
   kDevTimeoutMma = 3,
   kDevTimeoutEpilogue = 4,
   kDevTimeoutDrain = 5,
+  kDevBadSmemAlign = 6,  // dynamic shared memory not at the alignment a kernel declares (nothing done)
 };
 
 // Wait limit for every spin: about one second of %globaltimer.
@@ -181,6 +182,16 @@ __device__ __forceinline__ void cluster_sync_all() {
 // waiter that observes the phase also observes them.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Remote arrive with the default semantics (release at CTA scope), as used
+// to hand tensor-memory and tensor-core work between the two CTAs of a pair:
+// the data it signals is ordered by the tcgen05 fences (and, for shared
+// memory the tensor cores read, the async-proxy fence) around it; the
+// cluster-scope release of mbar_arrive_remote measured about 1500 cycles
+// per arrive there.
+__device__ __forceinline__ void mbar_arrive_remote_cta(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // The same arrive without ordering of its own: the caller orders its prior

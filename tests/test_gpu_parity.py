@@ -169,7 +169,7 @@ def test_forward_norm_gemv_gate_shape():
 
 
 @pytest.mark.parametrize("M,K,N", [(8, 256, 512), (2, 256, 512), (16, 2560, 640), (20, 203, 130), (300, 1000, 400),
-                                   (1, 2560, 6912), (130, 384, 256), (64, 128, 128)])
+                                   (1, 2560, 6912), (130, 384, 256), (64, 128, 128), (13, 256, 9600)])
 def test_forward_tc_full(M, K, N):
     x, Wt, a, w = _dense_case(M, K, N, seed=M * 7 + K)
     y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True, flags=bl.FLAG_PATH_TC)
