@@ -551,6 +551,22 @@ def run_nm(dev, min_calls: int = 16, warmup: int = 3, reps: int = 5):
                 key = f"{n}:{m} {name} {K}->{N} M={M}"
                 out[key] = {"us": sec * 1e6, "GBps": nbytes / sec / 1e9, "TOPS_dense_equiv": 2.0 * M * N * K / sec / 1e12,
                             "packed_bytes": w.nbytes, "kernel": bl.last_kernel(), "weight_copies": len(cps)}
+                if (n, m) == (2, 4) and M > 1:
+                    # the same call with the kept values expanded for the dense MMA, and the dense (unpruned)
+                    # matrix of the same shape: what the structured-sparse MMA is measured against
+                    ce = [(lambda: bl.forward_nm(w, x, out=y, workspace=ws, flags=bl.FLAG_PDL | bl.FLAG_NM24_EXPAND))]
+                    se = time_chain_graph(dev, ce * ncall, warmup, reps) / ncall
+                    out[key]["expanded_dense_mma"] = {"us": se * 1e6, "TOPS_dense_equiv": 2.0 * M * N * K / se / 1e12,
+                                                      "kernel": bl.last_kernel()}
+                    Wd = torch.from_numpy(synth.latent_weights(N, K, seed=5)).to(dev)
+                    wd = bl.pack_weights(Wd)
+                    del Wd
+                    cd = [(lambda: bl.forward(wd, x, out=y, workspace=ws, flags=bl.FLAG_PDL))]
+                    sd = time_chain_graph(dev, cd * ncall, warmup, reps) / ncall
+                    out[key]["dense_same_shape"] = {"us": sd * 1e6, "TOPS": 2.0 * M * N * K / sd / 1e12,
+                                                    "kernel": bl.last_kernel()}
+                    out[key]["speedup_vs_dense"] = sd / sec
+                    del wd, ce, cd
                 del cps, calls, x, ws, y
     assert bl.device_status() == 0
     return out

@@ -182,7 +182,9 @@ __device__ __forceinline__ void tc_store_token_rows(const uint32_t (&v)[32], con
     }
     return;
   }
-  for (int j = 0; j < ntok; ++j) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {  // static indices keep v in registers
+    if (j >= ntok) break;
     const int32_t tv = static_cast<int32_t>(v[j]) - rsm[j];
     const __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(static_cast<float>(tv), scl[j]));
     yr[static_cast<size_t>(j) * a.N] = *reinterpret_cast<const uint16_t*>(&h);
