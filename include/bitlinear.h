@@ -230,6 +230,33 @@ bitlinear_status bitlinear_forward_hbit(const bitlinear_weights* w, const uint16
                                         int32_t* acc, void* workspace, size_t workspace_bytes, uint32_t flags,
                                         void* stream);
 
+/* y = BitLinear for activations already quantised: the int8 codes, gamma and
+ * code sums of x as bitlinear_quant_act writes them ("BitNet b1.58 2B4T
+ * Technical Report", section 2 Architecture, BitLinear: activation_quant then
+ * the ternary contraction and the rescale by alpha * gamma / Q_b), so that a
+ * producer that quantises once (for example bitlinear_rmsnorm_quant_act)
+ * feeds several matrices, and so that the contraction can be timed on its
+ * own.  Dense or N:M weights; always the tensor-core GEMM (any M >= 1); the
+ * same bits as bitlinear_forward / bitlinear_forward_nm on the x the codes came
+ * from.
+ * q        device, int8 [M, ldq]: codes in natural K order; ldq >= K and a
+ *          multiple of 16 (bitlinear_quant_act writes ldq = K, so K % 16 == 0
+ *          there, or copy into a padded buffer); bytes K .. ldq - 1 of every
+ *          row zero; 16-byte aligned.
+ * gamma    device, fp32 [M];  rowsum  device, int32 [M] (sum of each row's codes).
+ * y, acc   as bitlinear_forward.
+ * workspace, workspace_bytes: device scratch of at least
+ *          bitlinear_forward_q8_workspace_bytes(M, N, K) (0 when the GEMM does
+ *          not split K; then NULL is accepted).
+ * flags    BITLINEAR_FLAG_PDL (the GEMM is always launched as a programmatic
+ *          dependent), BITLINEAR_FLAG_PATH_TC (accepted), BITLINEAR_FLAG_NM24_EXPAND.
+ * Errors: NULL, SHAPE (also ldq < K or not a multiple of 16), ALIGN, PATTERN,
+ *         WORKSPACE, FLAGS, DEVICE, CUDA. */
+bitlinear_status bitlinear_forward_q8(const bitlinear_weights* w, const int8_t* q, int32_t ldq, const float* gamma,
+                                      const int32_t* rowsum, int32_t M, uint16_t* y, int32_t* acc, void* workspace,
+                                      size_t workspace_bytes, uint32_t flags, void* stream);
+size_t bitlinear_forward_q8_workspace_bytes(int32_t M, int32_t N, int32_t K);
+
 /* Workspace bytes needed by bitlinear_forward / bitlinear_forward_nm.  0 when
  * the call takes the M = 1 GEMV path (which quantises in-kernel).  The
  * tensor-core path needs the int8 codes, gamma and code sums of x and, when it
@@ -293,8 +320,7 @@ bitlinear_status bitlinear_forward_nm(const bitlinear_weights* w, const uint16_t
  * them by rows) and each N:M matrix in its own; 2 <= M <= 64 with dense
  * weights runs the fused few-token kernel once per matrix (see
  * bitlinear_forward); otherwise the call quantises once and runs one
- * persistent tensor-core GEMM per matrix (the structured-sparse MMA when
- * every matrix is 2:4, since the codes' K order is shared).
+ * persistent tensor-core GEMM per matrix.
  * Errors: as bitlinear_forward; SHAPE also for count out of range or unequal K. */
 bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,
                                          uint16_t* const* y, int32_t* const* acc, void* workspace,

@@ -16,7 +16,7 @@ __all__ = [
     "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
     "quant_act", "rmsnorm_quant_act", "forward", "forward_nm", "forward_group", "forward_norm",
     "forward_workspace_bytes", "device_status", "last_kernel", "layout_version", "hadamard_quant_act4",
-    "forward_hbit", "HBIT_MAX_K",
+    "forward_hbit", "HBIT_MAX_K", "forward_q8", "forward_q8_workspace_bytes",
     "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT", "FLAG_PATH_PERSISTENT", "FLAG_NM24_EXPAND",
 ]
 
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
             "bitlinear_forward_norm": (st, [ctypes.POINTER(_Weights), P, i32, P, ctypes.c_float, P, P, P, sz, u32, P]),
             "bitlinear_hadamard_quant_act4": (st, [P, i32, i32, P, P, P, P]),
             "bitlinear_forward_hbit": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
+            "bitlinear_forward_q8": (st, [ctypes.POINTER(_Weights), P, i32, P, P, i32, P, P, P, sz, u32, P]),
+            "bitlinear_forward_q8_workspace_bytes": (sz, [i32, i32, i32]),
             "bitlinear_device_status": (st, [P, ctypes.POINTER(i32), i32]),
             "bitlinear_last_kernel": (ctypes.c_char_p, []),
             "bitlinear_layout_version": (i32, []),
@@ -240,6 +242,36 @@ def forward_hbit(w: PackedWeights, x, want_acc: bool = False, flags: int = 0, wo
     _check(lib().bitlinear_forward_hbit(ctypes.byref(ws), _ptr(x), M, _ptr(y), _ptr(acc), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(), flags, _stream(stream)),
            "forward_hbit")
+    return (y, acc) if want_acc else y
+
+
+def forward_q8_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bitlinear_forward_q8_workspace_bytes(M, N, K))
+
+
+def forward_q8(w: PackedWeights, q, gamma, rowsum, want_acc: bool = False, flags: int = 0, workspace=None, out=None,
+               acc_out=None, stream=None):
+    """y = BitLinear from activations already quantised (q int8 [M, ldq] natural k order with ldq >= K a
+    multiple of 16 and zeros past K, gamma fp32 [M], rowsum int32 [M], e.g. from quant_act): the
+    tensor-core GEMM alone, dense or N:M weights."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.int8 and q.dim() == 2 and q.stride(1) == 1 and q.shape[1] >= w.K
+    M = q.shape[0]
+    assert gamma.dtype == torch.float32 and gamma.numel() == M and gamma.is_contiguous()
+    assert rowsum.dtype == torch.int32 and rowsum.numel() == M and rowsum.is_contiguous()
+    _check_out(out, (M, w.N), torch.bfloat16, q.device, "out")
+    _check_out(acc_out, (M, w.N), torch.int32, q.device, "acc_out")
+    _check_workspace(workspace, q.device)
+    y = out if out is not None else torch.empty((M, w.N), dtype=torch.bfloat16, device=q.device)
+    acc = acc_out if acc_out is not None else (
+        torch.empty((M, w.N), dtype=torch.int32, device=q.device) if want_acc else None)
+    need = forward_q8_workspace_bytes(M, w.N, w.K)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ws = w.c_struct()
+    _check(lib().bitlinear_forward_q8(ctypes.byref(ws), _ptr(q), q.stride(0), _ptr(gamma), _ptr(rowsum), M, _ptr(y),
+                                      _ptr(acc), _ptr(workspace), ws_n, flags, _stream(stream)), "forward_q8")
     return (y, acc) if want_acc else y
 
 

@@ -266,6 +266,16 @@ size_t tc_base_bytes(int M, int K) {
 }
 size_t tc_cnt_bytes(int sm_count) { return align256(4 * static_cast<size_t>(sm_count)); }
 
+// Workspace of bitlinear_forward_q8: only the split-K counters and sums (none without a split).
+size_t tc_workspace_q8(int M, int N, int K, int nm, int sm_count) {
+  const TcPlan p = tc_plan(M, N, K, nm, sm_count);
+  return p.ksplit > 1 ? tc_cnt_bytes(sm_count) + align256(static_cast<size_t>(M) * N * 4) : 0;
+}
+bool workspace_ok_q8(const void* ws, size_t bytes, int M, int N, int K, int nm, int sm_count) {
+  const size_t need = tc_workspace_q8(M, N, K, nm, sm_count);
+  return need == 0 || (ws && bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 15u) == 0);
+}
+
 size_t tc_workspace(int M, int N, int K, int nm, int sm_count) {
   const TcPlan p = tc_plan(M, N, K, nm, sm_count);
   size_t b = tc_base_bytes(M, K);
@@ -436,7 +446,8 @@ bitlinear_status skinny_launch(const bitlinear_weights* w, const uint16_t* x, in
 // gamma and the code sums.  One quantisation serves every matrix that
 // multiplies the same x.
 struct QuantWs {
-  int8_t* q;        // [M, k16(K)]
+  int8_t* q;        // [M, ldq] natural K order
+  int ldq;          // row stride of q in bytes (k16(K) in the workspace)
   float* gamma;     // [M]
   int32_t* rowsum;  // [M]
   uint32_t* cnt;    // [ncnt] split-K arrival counters (zeroed by the quantisation kernel)
@@ -449,6 +460,7 @@ QuantWs tc_ws_layout(void* ws, int M, int K, int ncnt, int max_n) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   QuantWs r;
   r.q = reinterpret_cast<int8_t*>(wsb);
+  r.ldq = static_cast<int>(k16(K));
   r.gamma = reinterpret_cast<float*>(wsb + align256(static_cast<size_t>(M) * k16(K)));
   r.rowsum = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(r.gamma) + align256(4 * static_cast<size_t>(M)));
   r.cnt = reinterpret_cast<uint32_t*>(wsb + tc_base_bytes(M, K));
@@ -466,7 +478,7 @@ auto quant_kernel(int G) {
 }
 
 bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bool pdl, cudaStream_t s,
-                          const float* gnorm = nullptr, float eps = 0.0f, bool natural = false) {
+                          const float* gnorm = nullptr, float eps = 0.0f) {
   const QuantShape qs = quant_shape(M, K, gnorm != nullptr, plan_sm_count());
   const int wpr = qs.wpr;
   const int rows_per_cta = kQuantWarps / wpr;
@@ -476,15 +488,14 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
   const int zblocks = static_cast<int>(std::min<size_t>(1024, (vec4 + 4 * 32 * kQuantWarps - 1) /
                                                                    (4 * 32 * kQuantWarps)));
   uint32_t* cnt = qw.ncnt > 0 ? qw.cnt : static_cast<uint32_t*>(nullptr);
-  // contraction order for the dense and expanded MMAs; natural K order (zero-padded to 16) for the
-  // structured-sparse MMA, whose metadata names positions inside runs of four consecutive k
+  // natural K order, rows zero-padded to a multiple of 16 (the order every tensor-core GEMM reads;
+  // the structured-sparse MMA's metadata names positions inside runs of four consecutive k)
   auto go = [&](auto kern, const float* g, float e) {
     return launch(kern, dim3(qblocks + zblocks), dim3(32 * kQuantWarps), 0, s, pdl, x, M, K, static_cast<int>(k16(K)),
                   qw.q, qw.gamma, qw.rowsum, cnt, qw.ncnt, qw.part, vec4, qblocks, wpr, g, e);
   };
-  if (gnorm) return natural ? go(quant_kernel<false, true>(qs.G), gnorm, eps) : go(quant_kernel<true, true>(qs.G), gnorm, eps);
-  return natural ? go(quant_kernel<false, false>(qs.G), static_cast<const float*>(nullptr), 0.0f)
-                 : go(quant_kernel<true, false>(qs.G), static_cast<const float*>(nullptr), 0.0f);
+  if (gnorm) return go(quant_kernel<false, true>(qs.G), gnorm, eps);
+  return go(quant_kernel<false, false>(qs.G), static_cast<const float*>(nullptr), 0.0f);
 }
 
 // The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
@@ -495,7 +506,7 @@ bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, 
   if (pairs_max < 1) return BITLINEAR_ERR_DEVICE;
   const int N = w->N, K = w->K;
   CUtensorMap mB, mA, mMeta;
-  if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
+  if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(qw.ldq),
                    kTcSubK, static_cast<uint32_t>(kT2Half), true))
     return BITLINEAR_ERR_CUDA;
   if (NM == 0) {
@@ -535,13 +546,11 @@ bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, 
   return st;
 }
 
-// natural: the codes in qw are in natural K order (tc_quant(..., natural = true)),
-// which sends 2:4 weights to the structured-sparse MMA.
+// sparse24: 2:4 weights on the structured-sparse MMA (otherwise expanded for the dense one).
 bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
-                         cudaStream_t s, DeviceState* dev, float qb = kQb, bool natural = false) {
+                         cudaStream_t s, DeviceState* dev, float qb = kQb, bool sparse24 = true) {
   const int N = w->N, K = w->K;
-  const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? (natural ? 3 : 1) : 2);
-  if (natural && nm != 3) return BITLINEAR_ERR_PATTERN;
+  const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? (sparse24 ? 3 : 1) : 2);
   const TcPlan plan = tc_plan(M, N, K, nm, dev->sm_count);
   if ((nm == 0 || nm == 3) && plan.bn == 128 && plan.ksplit == 1) {
     const bitlinear_status st = nm == 0 ? tc2_gemm<0>(w, M, qw, y, acc, s, dev, qb, plan)
@@ -550,7 +559,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   }
   const int bn = plan.bn;
   CUtensorMap mB, mA, mMeta;
-  if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(k16(K)),
+  if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(qw.ldq),
                    kTcSubK, static_cast<uint32_t>(bn), true))
     return BITLINEAR_ERR_CUDA;
   TcArgs ta;
@@ -637,21 +646,21 @@ bitlinear_status forward_tc(const bitlinear_weights* w, const uint16_t* x, int M
                             const float* gnorm = nullptr, float eps = 0.0f, ActKind act = ActKind::kInt8,
                             bool nm24_expand = false) {
   const int nm = w->nm_m == 0 ? 0 : (w->nm_m == 4 ? 1 : 2);
-  const bool natural = nm == 1 && !nm24_expand;  // 2:4 on the structured-sparse MMA
+  const bool sparse24 = !nm24_expand;  // 2:4 weights on the structured-sparse MMA
   if (!ws || ws_bytes < tc_workspace(M, w->N, w->K, nm, dev->sm_count) || !aligned16(ws))
     return BITLINEAR_ERR_WORKSPACE;
   const bool split = tc_plan(M, w->N, w->K, nm, dev->sm_count).ksplit > 1;
   const QuantWs qw = tc_ws_layout(ws, M, w->K, split ? dev->sm_count : 0, w->N);
   bitlinear_status st;
   if (act == ActKind::kHbit4) {
-    st = hbit_quant(x, M, w->K, qw.q, static_cast<int>(k16(w->K)), !natural, qw.gamma, qw.rowsum,
+    st = hbit_quant(x, M, w->K, qw.q, static_cast<int>(k16(w->K)), false, qw.gamma, qw.rowsum,
                     qw.ncnt > 0 ? qw.cnt : nullptr, qw.ncnt, qw.part, qw.part_words, pdl, s);
     if (st != BITLINEAR_OK) return st;
-    return tc_gemm(w, M, qw, y, acc, s, dev, kQb4, natural);
+    return tc_gemm(w, M, qw, y, acc, s, dev, kQb4, sparse24);
   }
-  st = tc_quant(x, M, w->K, qw, pdl, s, act == ActKind::kInt8Norm ? gnorm : nullptr, eps, natural);
+  st = tc_quant(x, M, w->K, qw, pdl, s, act == ActKind::kInt8Norm ? gnorm : nullptr, eps);
   if (st != BITLINEAR_OK) return st;
-  return tc_gemm(w, M, qw, y, acc, s, dev, kQb, natural);
+  return tc_gemm(w, M, qw, y, acc, s, dev, kQb, sparse24);
 }
 
 // ---------------------------------------------------------------- GEMV path
@@ -945,12 +954,11 @@ bitlinear_status forward_group(const bitlinear_weights* w, int count, const uint
     }
     if (!ws || ws_bytes < need || !aligned16(ws)) return BITLINEAR_ERR_WORKSPACE;
     const QuantWs qw = tc_ws_layout(ws, M, w[0].K, split ? dev->sm_count : 0, max_n);
-    // one quantisation serves every matrix: natural K order (structured-sparse MMA) only when all are 2:4
-    bool natural = !(flags & BITLINEAR_FLAG_NM24_EXPAND);
-    for (int i = 0; i < count; ++i) natural = natural && w[i].nm_m == 4;
-    st = tc_quant(x, M, w[0].K, qw, pdl, s, nullptr, 0.0f, natural);
+    // one quantisation serves every matrix
+    const bool sparse24 = !(flags & BITLINEAR_FLAG_NM24_EXPAND);
+    st = tc_quant(x, M, w[0].K, qw, pdl, s);
     for (int i = 0; i < count && st == BITLINEAR_OK; ++i)
-      st = tc_gemm(&w[i], M, qw, y[i], acc ? acc[i] : nullptr, s, dev, kQb, natural);
+      st = tc_gemm(&w[i], M, qw, y[i], acc ? acc[i] : nullptr, s, dev, kQb, sparse24);
     return st;
   }
   // decode: the dense matrices share one launch; each N:M matrix has its own
@@ -1174,13 +1182,56 @@ bitlinear_status bitlinear_forward_hbit(const bitlinear_weights* w, const uint16
                     (flags & BITLINEAR_FLAG_NM24_EXPAND) != 0);
 }
 
+bitlinear_status bitlinear_forward_q8(const bitlinear_weights* w, const int8_t* q, int32_t ldq, const float* gamma,
+                                      const int32_t* rowsum, int32_t M, uint16_t* y, int32_t* acc, void* workspace,
+                                      size_t workspace_bytes, uint32_t flags, void* stream) {
+  if (!w || !q || !gamma || !rowsum || !y) return BITLINEAR_ERR_NULL;
+  bitlinear_status st = check_matrix(w, y, acc);
+  if (st != BITLINEAR_OK) return st;
+  if (M < 1 || M > BITLINEAR_MAX_M || ldq < w->K || (ldq % 16) != 0) return BITLINEAR_ERR_SHAPE;
+  if (!aligned16(q) || (reinterpret_cast<uintptr_t>(gamma) & 3u) || (reinterpret_cast<uintptr_t>(rowsum) & 3u))
+    return BITLINEAR_ERR_ALIGN;
+  if (flags & ~static_cast<uint32_t>(BITLINEAR_FLAG_PDL | BITLINEAR_FLAG_PATH_TC | BITLINEAR_FLAG_NM24_EXPAND))
+    return BITLINEAR_ERR_FLAGS;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nm = w->nm_m == 0 ? 0 : (w->nm_m == 4 ? 1 : 2);
+  if (!workspace_ok_q8(workspace, workspace_bytes, M, w->N, w->K, nm, dev->sm_count)) return BITLINEAR_ERR_WORKSPACE;
+  const bool split = tc_plan(M, w->N, w->K, nm, dev->sm_count).ksplit > 1;
+  QuantWs qw;
+  std::memset(&qw, 0, sizeof qw);
+  qw.q = const_cast<int8_t*>(q);
+  qw.ldq = ldq;
+  qw.gamma = const_cast<float*>(gamma);
+  qw.rowsum = const_cast<int32_t*>(rowsum);
+  if (split) {
+    // the K slices' sums and arrival counters start from zero (the quantisation launch clears them otherwise)
+    qw.cnt = static_cast<uint32_t*>(workspace);
+    qw.ncnt = dev->sm_count;
+    qw.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + tc_cnt_bytes(dev->sm_count));
+    qw.part_words = static_cast<size_t>(M) * w->N;
+    if (cudaMemsetAsync(workspace, 0, tc_cnt_bytes(dev->sm_count) + 4 * qw.part_words, s) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+  }
+  (void)(flags & BITLINEAR_FLAG_PDL);  // the GEMM always launches as a programmatic dependent
+  return tc_gemm(w, M, qw, y, acc, s, dev, kQb, (flags & BITLINEAR_FLAG_NM24_EXPAND) == 0);
+}
+
 size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {
   if (M < 1 || K < 1 || N < 1) return 0;
   const bool tc = (flags & BITLINEAR_FLAG_PATH_TC) || (M > 1 && !(flags & BITLINEAR_FLAG_PATH_GEMV));
   if (!tc) return 0;
   // enough for dense and for N:M weights (their k-blocks differ, and with them the K split)
   const int sm = plan_sm_count();
-  return std::max(tc_workspace(M, N, K, 0, sm), tc_workspace(M, N, K, 1, sm));
+  return std::max({tc_workspace(M, N, K, 0, sm), tc_workspace(M, N, K, 1, sm), tc_workspace(M, N, K, 2, sm)});
+}
+
+size_t bitlinear_forward_q8_workspace_bytes(int32_t M, int32_t N, int32_t K) {
+  if (M < 1 || K < 1 || N < 1) return 0;
+  const int sm = plan_sm_count();
+  return std::max({tc_workspace_q8(M, N, K, 0, sm), tc_workspace_q8(M, N, K, 1, sm), tc_workspace_q8(M, N, K, 2, sm)});
 }
 
 bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t count, const uint16_t* x, int32_t M,

@@ -13,8 +13,9 @@
 //
 // With code = W_t + 1 the contraction gives sum q * code, and the epilogue
 // subtracts the token's sum of codes: acc = D - rowsum (exact in int32).
-// Both operands use the same K order inside each 16-wide group (byte 4j + b
-// holds k = 4b + j), which is the order (w >> 2j) & 0x03030303 produces.
+// Both operands are in natural K order: the activation codes as the
+// quantisation writes them, the weights after a 4 x 4 byte transpose of the
+// masked 2-bit fields (codes_word_natural).
 //
 // One CTA per SM walks a static list of (weight-row tile, token tile, K slice)
 // units.  When the tiles alone would leave SMs idle (few tokens, or few
@@ -190,6 +191,21 @@ __device__ __forceinline__ void tc_store_token_rows(const uint32_t (&v)[32], con
     yr[static_cast<size_t>(j) * a.N] = *reinterpret_cast<const uint16_t*>(&h);
     if (ar) ar[static_cast<size_t>(j) * a.N] = tv;
   }
+}
+
+// The 16 codes of one dense code word (weight k of the 16-group at bits
+// 2k .. 2k + 1) as bytes in natural k order: o[m] byte b = code of weight
+// 4m + b.  (w >> 2j) & 0x03030303 gives byte b = code of weight 4b + j; the
+// byte permutes transpose that 4 x 4 arrangement.
+__device__ __forceinline__ void codes_word_natural(uint32_t w, uint32_t* o) {
+  const uint32_t s0 = w & 0x03030303u, s1 = (w >> 2) & 0x03030303u;
+  const uint32_t s2 = (w >> 4) & 0x03030303u, s3 = (w >> 6) & 0x03030303u;
+  const uint32_t t0 = __byte_perm(s0, s1, 0x5140), t1 = __byte_perm(s0, s1, 0x7362);
+  const uint32_t t2 = __byte_perm(s2, s3, 0x5140), t3 = __byte_perm(s2, s3, 0x7362);
+  o[0] = __byte_perm(t0, t2, 0x5410);
+  o[1] = __byte_perm(t0, t2, 0x7632);
+  o[2] = __byte_perm(t1, t3, 0x5410);
+  o[3] = __byte_perm(t1, t3, 0x7632);
 }
 
 template <int BN, int NM>
@@ -471,10 +487,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         uint32_t outw[32];
 #pragma unroll
-        for (int gi = 0; gi < 8; ++gi) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) outw[4 * gi + j] = (dw[gi] >> (2 * j)) & 0x03030303u;
-        }
+        for (int gi = 0; gi < 8; ++gi) codes_word_natural(dw[gi], outw + 4 * gi);
         tc_st_32x32b_x32(tmem + lane_base + A_COL0 + s * SLOT + sub * 32, outw);
       }
       tc_wait_st();

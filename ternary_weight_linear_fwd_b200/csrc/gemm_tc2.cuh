@@ -296,10 +296,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t dw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
           uint32_t outw[32];
 #pragma unroll
-          for (int gi = 0; gi < 8; ++gi) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) outw[4 * gi + j] = (dw[gi] >> (2 * j)) & 0x03030303u;
-          }
+          for (int gi = 0; gi < 8; ++gi) codes_word_natural(dw[gi], outw + 4 * gi);
           tc_st_32x32b_x32(tmem + lane_base + C::A_COL0 + j * C::SLOT + sub * 32, outw);
         }
       }

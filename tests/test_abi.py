@@ -236,3 +236,21 @@ def test_flag_values_match_header():
         assert getattr(bl, name) == int(val, 16), name
     vals = [int(v, 16) for v in flags.values()]
     assert all(v and (v & (v - 1)) == 0 for v in vals) and len(set(vals)) == len(vals)
+
+
+def test_forward_q8_host_checks(L):
+    """Codes-in entry: argument errors before any device work (fake addresses)."""
+    import ternary_weight_linear_fwd_b200 as bl
+    f = L.bitlinear_forward_q8
+    f.restype = ctypes.c_int
+    P, i32 = ctypes.c_void_p, ctypes.c_int32
+    f.argtypes = [ctypes.POINTER(bl._Weights), P, i32, P, P, i32, P, P, P, ctypes.c_size_t, ctypes.c_uint32, P]
+    q, g, rs, y = 0x10000, 0x20000, 0x30000, 0x40000
+    w = _w(L)
+    assert f(None, q, 256, g, rs, 4, y, None, None, 0, 0, None) == 1
+    assert f(ctypes.byref(w), None, 256, g, rs, 4, y, None, None, 0, 0, None) == 1
+    assert f(ctypes.byref(w), q, 256, g, None, 4, y, None, None, 0, 0, None) == 1
+    assert f(ctypes.byref(w), q, 250, g, rs, 4, y, None, None, 0, 0, None) == 2   # ldq < K
+    assert f(ctypes.byref(w), q, 264, g, rs, 0, y, None, None, 0, 0, None) == 2   # M = 0
+    assert f(ctypes.byref(w), q + 8, 256, g, rs, 4, y, None, None, 0, 0, None) == 3
+    assert f(ctypes.byref(w), q, 256, g, rs, 4, y, None, None, 0, 0x2, None) == 8  # no GEMV path

@@ -478,6 +478,41 @@ def test_forward_pair_gemm_sparse24(M, K, N):
     _check_rows(x, Wt, a, y, acc, rows)
 
 
+# ---------------------------------------------------------------- codes-in entry (the GEMM alone)
+
+@pytest.mark.parametrize("n,m", [(0, 0), (2, 4), (6, 8)])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 300), (37, 1024, 640), (300, 2048, 1100), (2048, 2560, 2560)])
+def test_forward_q8_matches_forward(n, m, M, K, N):
+    """bitlinear_forward_q8 on the codes, gamma and code sums of bitlinear_quant_act gives the bits of
+    bitlinear_forward / bitlinear_forward_nm on x (same plan, same kernels after the quantisation)."""
+    x = synth.activations(M, K, seed=M + N)
+    W = synth.latent_weights(N, K, seed=K + N)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV), n, m)
+    ref = oracle.pack_weights(W, n, m)
+    xd = to_dev_bf16(x)
+    q, g, rs = bl.quant_act(xd)
+    y, acc = bl.forward_q8(w, q, g, rs, want_acc=True)
+    fn = bl.forward_nm if m else bl.forward
+    y1, acc1 = fn(w, xd, want_acc=True, flags=bl.FLAG_PATH_TC)
+    assert torch.equal(acc, acc1) and torch.equal(y.view(torch.int16), y1.view(torch.int16))
+    rows = np.arange(M) if M <= 300 else np.unique(np.concatenate([[0, M - 1], synth.splitmix64(M, 3, 10) % M]))
+    _check_rows(x, ref["Wt"], ref["alpha"], y, acc, rows.astype(np.int64))
+
+
+def test_forward_q8_padded_rows():
+    """Codes in a row stride above K (K = 1000 padded to 1008, zeros past K)."""
+    M, K, N = 96, 1000, 512
+    x = synth.activations(M, K, seed=61)
+    W = synth.latent_weights(N, K, seed=62)
+    w = bl.pack_weights(torch.from_numpy(W).to(DEV))
+    ref = oracle.pack_weights(W)
+    q, g, rs = bl.quant_act(to_dev_bf16(x))
+    qp = torch.zeros((M, 1008), dtype=torch.int8, device=DEV)
+    qp[:, :K] = q
+    y, acc = bl.forward_q8(w, qp, g, rs, want_acc=True)
+    _check_rows(x, ref["Wt"], ref["alpha"], y, acc, np.arange(M))
+
+
 # ---------------------------------------------------------------- grouped forward
 
 @pytest.mark.parametrize("M", [1, 37])
