@@ -910,7 +910,25 @@ def _case_sparse24_m2048(dev):
         bl.forward_nm(w, x)
 
 
-PROFILE_CASES = {"few_token_m16": _case_few_token, "hbit_m1": _case_hbit_m1, "sparse24_m2048": _case_sparse24_m2048}
+def _case_pair_gemm_m2048(dev):
+    """bitlinear_forward_q8 (the GEMM alone, codes quantised first) at M = 2048 on the 2B4T gate projection
+    2560 -> 6912: the pair GEMM (tcgen05 cta_group::2)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+    W = torch.from_numpy(synth.latent_weights(6912, 2560, seed=3)).to(dev)
+    w = bl.pack_weights(W)
+    del W
+    x = torch.from_numpy(synth.activations(2048, 2560, seed=3).view(np.int16)).to(dev).view(torch.bfloat16)
+    q, g, rs = bl.quant_act(x)
+    for _ in range(3):
+        bl.forward_q8(w, q, g, rs)
+
+
+PROFILE_CASES = {"few_token_m16": _case_few_token, "hbit_m1": _case_hbit_m1, "sparse24_m2048": _case_sparse24_m2048,
+                 "pair_gemm_m2048": _case_pair_gemm_m2048}
 
 
 def run_profile_case(name: str):

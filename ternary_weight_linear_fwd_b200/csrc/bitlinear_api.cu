@@ -53,7 +53,7 @@ struct DeviceState {
   int sm_count = 0;
   int32_t* status = nullptr;
   int sk_clusters[kSkMaxCluster + 1] = {};  // clusters of each size the few-token kernel fits at once (0: not asked)
-  int t2_pairs[2] = {};                     // CTA pairs of the pair GEMM (dense, 2:4) resident at once (0: not asked)
+  int t2_pairs[2][3] = {};                  // CTA pairs of the pair GEMM (dense, 2:4; 64, 96, 128 tokens) resident at once
 };
 
 std::mutex g_mu;
@@ -303,19 +303,19 @@ bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA,
   }
 }
 
-// CTA pairs of the pair GEMM resident at once (one CTA per SM), asked once per device.
-template <int NM>
+// CTA pairs of the pair GEMM resident at once (one CTA per SM), asked once per device and variant.
+template <int NM, int BN>
 int t2_active_pairs(DeviceState* dev) {
-  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1];
+  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1][BN == 64 ? 0 : BN == 96 ? 1 : 2];
   std::lock_guard<std::mutex> lk(g_mu);
   if (slot == 0) {
     int n = -1;
-    if (ensure_smem(reinterpret_cast<const void*>(tc2_gemm_kernel<NM>), T2<NM>::SMEM)) {
+    if (ensure_smem(reinterpret_cast<const void*>(tc2_gemm_kernel<NM, BN>), T2<NM, BN>::SMEM)) {
       cudaLaunchConfig_t cfg;
       std::memset(&cfg, 0, sizeof cfg);
       cfg.gridDim = dim3(2 * 64);
       cfg.blockDim = dim3(kTcThreads);
-      cfg.dynamicSmemBytes = T2<NM>::SMEM;
+      cfg.dynamicSmemBytes = T2<NM, BN>::SMEM;
       cudaLaunchAttribute attr;
       attr.id = cudaLaunchAttributeClusterDimension;
       attr.val.clusterDim.x = 2;
@@ -323,7 +323,7 @@ int t2_active_pairs(DeviceState* dev) {
       attr.val.clusterDim.z = 1;
       cfg.attrs = &attr;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, tc2_gemm_kernel<NM>, &cfg) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveClusters(&n, tc2_gemm_kernel<NM, BN>, &cfg) != cudaSuccess) {
         (void)cudaGetLastError();
         n = -1;
       }
@@ -498,27 +498,25 @@ bitlinear_status tc_quant(const uint16_t* x, int M, int K, const QuantWs& qw, bo
   return go(quant_kernel<false, false>(qs.G), static_cast<const float*>(nullptr), 0.0f);
 }
 
-// The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
-template <int NM>
-bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
-                          cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
-  const int pairs_max = t2_active_pairs<NM>(dev);
-  if (pairs_max < 1) return BITLINEAR_ERR_DEVICE;
+template <int NM, int BN>
+bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
+                            cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan, int pairs) {
+  using C = T2<NM, BN>;
   const int N = w->N, K = w->K;
   CUtensorMap mB, mA, mMeta;
   if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(qw.ldq),
-                   kTcSubK, static_cast<uint32_t>(kT2Half), true))
+                   kTcSubK, static_cast<uint32_t>(C::HALF), true))
     return BITLINEAR_ERR_CUDA;
   if (NM == 0) {
     const int64_t ld = dense_ld(K);
-    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * T2<0>::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * C::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
     mMeta = mA;
   } else {
     int64_t ldv = 0, ldm = 0;
     if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
       return BITLINEAR_ERR_PATTERN;
-    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, 16 * T2<3>::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
-    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16 * T2<3>::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, 16 * C::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16 * C::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
   }
   TcArgs ta;
   std::memset(&ta, 0, sizeof ta);
@@ -527,7 +525,7 @@ bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, 
   ta.K = K;
   ta.kblocks = plan.kblocks;
   ta.row_tiles = (N + kT2Rows - 1) / kT2Rows;
-  ta.tok_tiles = (M + kT2Tok - 1) / kT2Tok;
+  ta.tok_tiles = (M + BN - 1) / BN;
   ta.ksplit = 1;
   ta.kbs = plan.kblocks;
   ta.gamma = qw.gamma;
@@ -538,12 +536,40 @@ bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, 
   ta.qb = qb;
   ta.status = dev->status;
   ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
-  const int units = ta.row_tiles * ta.tok_tiles;
-  const int pairs = std::min(pairs_max, units);
+  pairs = std::min(pairs, ta.row_tiles * ta.tok_tiles);
   const bitlinear_status st =
-      launch_ex(tc2_gemm_kernel<NM>, dim3(2 * pairs), dim3(kTcThreads), T2<NM>::SMEM, s, true, 2, mB, mA, mMeta, ta);
+      launch_ex(tc2_gemm_kernel<NM, BN>, dim3(2 * pairs), dim3(kTcThreads), C::SMEM, s, true, 2, mB, mA, mMeta, ta);
   if (st == BITLINEAR_OK) t_last_kernel = NM == 0 ? "tc2_gemm_dense" : "tc2_gemm_sp24";
   return st;
+}
+
+// The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
+// The token tile (128, 96 or 64 tokens) is the one whose tiles fill the
+// resident pairs' waves best (ties to the wider tile).  DEVICE: no pair fits.
+template <int NM>
+bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
+                          cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
+  const int bns[3] = {128, 96, 64};
+  const int pmax[3] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 96>(dev), t2_active_pairs<NM, 64>(dev)};
+  const int rows = (w->N + kT2Rows - 1) / kT2Rows;
+  int best = -1;
+  double best_eff = 0.0;
+  for (int i = 0; i < 3; ++i) {
+    if (pmax[i] < 1) continue;
+    const int units = rows * ((M + bns[i] - 1) / bns[i]);
+    const int waves = (units + pmax[i] - 1) / pmax[i];
+    const double eff = static_cast<double>(units) / (static_cast<double>(waves) * pmax[i]);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = i;
+    }
+  }
+  if (best < 0) return BITLINEAR_ERR_DEVICE;
+  switch (bns[best]) {
+    case 128: return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pmax[best]);
+    case 96: return tc2_launch<NM, 96>(w, M, qw, y, acc, s, dev, qb, plan, pmax[best]);
+    default: return tc2_launch<NM, 64>(w, M, qw, y, acc, s, dev, qb, plan, pmax[best]);
+  }
 }
 
 // sparse24: 2:4 weights on the structured-sparse MMA (otherwise expanded for the dense one).

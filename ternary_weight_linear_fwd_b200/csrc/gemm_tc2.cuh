@@ -7,12 +7,15 @@
 // of the full kernel's time (2048 -> 11008 at M = 4096).  Here two CTAs of a
 // cluster share one MMA of M = 256 weight rows: each CTA holds its own 128
 // weight rows (expanded codes in its TMEM for dense weights, the compressed
-// kept values in its shared memory for 2:4 weights) and HALF of the 128
+// kept values in its shared memory for 2:4 weights) and HALF of the BN
 // tokens' activation tile, so the activation bytes per MAC halve.
 //
-//   D[256 rows, 128 tokens] += A[256 rows, K] * B[128 tokens, K]^T
+//   D[256 rows, BN tokens] += A[256 rows, K] * B[BN tokens, K]^T
 //   CTA r of the pair: rows 128 r .. 128 r + 127 of A and D (its own TMEM),
-//                      tokens 64 r .. 64 r + 63 of B (its own shared memory).
+//                      tokens BN/2 r .. BN/2 r + BN/2 - 1 of B (its own shared memory).
+// BN (64, 96 or 128) is chosen per shape so that the tiles fill whole waves of
+// the resident pairs (2560 -> 2560 at M = 2048: 160 tiles of 128 tokens leave
+// a third wave 16% full on 74 pairs, 220 tiles of 96 tokens fill three).
 //
 // Two rings: S copy stages in shared memory (the CTA's half of the activation
 // tile and its packed weights) and R operand slots (expanded codes in TMEM, or
@@ -41,44 +44,45 @@
 
 namespace bl {
 
-constexpr int kT2Tok = 128;      // tokens of a pair tile (the MMA's N)
-constexpr int kT2Half = 64;      // tokens per CTA
 constexpr int kT2Rows = 256;     // weight rows of a pair tile (the MMA's M)
 
 // 256-k stages.  Dense: 8 copy stages of 24 KB, 4 operand slots of 64 TMEM
 // columns beside two 128-column accumulators.  2:4: 6 copy stages of 24 KB and
 // 4 slots of 16 KB compressed operand (+ 8 metadata columns each).
-template <int NM>
+// BN: tokens of a pair tile (the MMA's N: 64, 96 or 128), BN / 2 per CTA.
+template <int NM, int BN>
 struct T2 {
   static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
+  static_assert(BN == 64 || BN == 96 || BN == 128, "pair token tile");
   static constexpr bool SP = NM == 3;
   static constexpr int KSUB = 2;
-  static constexpr int B_SUB = kT2Half * 128;
+  static constexpr int HALF = BN / 2;
+  static constexpr int B_SUB = HALF * 128;  // a whole number of 8-row swizzle atoms
   static constexpr int B_STAGE = B_SUB * KSUB;
   static constexpr int A_VAL = SP ? kTcRows * 32 : kTcRows * 64;     // TMA bytes of values ...
   static constexpr int A_META = SP ? kTcRows * 32 : 0;               // ... and metadata per stage
   static constexpr int STAGE = B_STAGE + A_VAL + A_META;             // one copy stage
   static constexpr int OPA = SP ? kTcRows * 128 : 0;                 // compressed operand in shared memory
   static constexpr int SLOT = SP ? 8 : 64;                           // TMEM columns per operand slot
-  static constexpr int DCOLS = kT2Tok;
+  static constexpr int DCOLS = BN;
   static constexpr int R = 4;                                        // operand slots
   // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
-  static constexpr int FIXED = 2 * kT2Tok * 8 + 256;
+  static constexpr int FIXED = 2 * BN * 8 + 256;
   static constexpr int S = tc_min3(kTcMaxStages, (kTcSmemMax - FIXED - R * OPA) / STAGE, 64) & ~1;  // even
   static constexpr int SMEM = FIXED + S * STAGE + R * OPA;
   static constexpr int A_COL0 = 2 * DCOLS;
   static_assert(A_COL0 + R * SLOT <= 512, "TMEM budget");
   static_assert(S >= R, "copy ring at least as deep as the operand ring");
-  static constexpr uint32_t IDESC = SP ? idesc_i8_sp_s8s8(kT2Rows, kT2Tok) : idesc_i8_u8s8(kT2Rows, kT2Tok);
+  static constexpr uint32_t IDESC = SP ? idesc_i8_sp_s8s8(kT2Rows, BN) : idesc_i8_u8s8(kT2Rows, BN);
 };
 
 // Launched in clusters of two CTAs (an even grid); a.row_tiles counts 256-row
 // pair tiles here; no K split (a.ksplit == 1).
-template <int NM>
+template <int NM, int BN>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc2_gemm_kernel(const __grid_constant__ CUtensorMap mapB, const __grid_constant__ CUtensorMap mapA,
                     const __grid_constant__ CUtensorMap mapMeta, const TcArgs a) {
-  using C = T2<NM>;
+  using C = T2<NM, BN>;
   constexpr int S = C::S;
   constexpr bool SP = C::SP;
   constexpr int KSUB = C::KSUB;
@@ -93,9 +97,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int R = C::R;
   uint8_t* sStage = base;                        // [S][B half | packed values | metadata]
   uint8_t* sOp = base + S * C::STAGE;            // 2:4: [R][128 rows][128 B] compressed operand
-  float* s_scale = reinterpret_cast<float*>(sOp + R * C::OPA);           // [2][128]
-  int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * kT2Tok);  // [2][128]
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_rowsum + 2 * kT2Tok);
+  float* s_scale = reinterpret_cast<float*>(sOp + R * C::OPA);  // [2][BN]
+  int32_t* s_rowsum = reinterpret_cast<int32_t*>(s_scale + 2 * BN);  // [2][BN]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_rowsum + 2 * BN);
   uint64_t* empty = full + S;
   uint64_t* aready = empty + S;     // [R] rank 0's: both CTAs' unpack warps
   uint64_t* afree = aready + R;     // [R] operand slot read by the MMAs (multicast commit)
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       };
       auto load_b = [&](int tt, int kb, int s) {
-        const int tok0 = tt * kT2Tok + static_cast<int>(rank) * kT2Half;
+        const int tok0 = tt * BN + static_cast<int>(rank) * C::HALF;
         for (int sub = 0; sub < KSUB; ++sub)
           tma_load_2d(sStage + s * C::STAGE + sub * C::B_SUB, &mapB, (kb * KSUB + sub) * kTcSubK, tok0, &full[s]);
       };
@@ -316,10 +320,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int rt, tt;
       unit_of(t, rt, tt);
       const int row0 = rt * kT2Rows + static_cast<int>(rank) * kTcRows + q * 32;
-      const int tok0 = tt * kT2Tok;
-      float* scl = s_scale + buf * kT2Tok;
-      int32_t* rsm = s_rowsum + buf * kT2Tok;
-      for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < kT2Tok; j += 128) {
+      const int tok0 = tt * BN;
+      float* scl = s_scale + buf * BN;
+      int32_t* rsm = s_rowsum + buf * BN;
+      for (int j = threadIdx.x - kTcEpiWarp0 * 32; j < BN; j += 128) {
         const int tok = tok0 + j;
         scl[j] = tok < a.M ? __fdiv_rn(__fmul_rn(alpha, a.gamma[tok]), a.qb) : 0.0f;  // RN(RN(alpha gamma) / Q_b)
         rsm[j] = (tok < a.M && a.rowsum) ? a.rowsum[tok] : 0;
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < kT2Tok; c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
         tc_ld_32x32b_x32(tmem + lane_base + buf * C::DCOLS + c0, v);
         tc_wait_ld();

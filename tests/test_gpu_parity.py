@@ -454,7 +454,9 @@ def test_forward_group_all_nm24_uses_sparse_mma():
 # Shapes whose plan is 128-token tiles without a K split (at least 75 tiles of 128 x 128), so the GEMM
 # runs on CTA pairs sharing one M = 256 MMA: ragged M (a last tile of 1 or 44 tokens), ragged N (the
 # last pair tile's second CTA partly or wholly past N), K not a multiple of the 256-k stage.
-@pytest.mark.parametrize("M,K,N", [(1000, 2560, 2000), (4096, 1032, 640), (300, 2048, 11008), (129, 6912, 9000)])
+# (4736, 512, 256): 74 tiles of 64 tokens fill the pairs exactly, so the 64-token pair tile is chosen.
+@pytest.mark.parametrize("M,K,N", [(1000, 2560, 2000), (4096, 1032, 640), (300, 2048, 11008), (129, 6912, 9000),
+                                   (4736, 512, 256), (2048, 2560, 2560)])
 def test_forward_pair_gemm_dense(M, K, N):
     x, Wt, a, w = _dense_case(M, K, N, seed=M + K + N)
     y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
@@ -464,7 +466,7 @@ def test_forward_pair_gemm_dense(M, K, N):
     _check_rows(x, Wt, a, y, acc, rows)
 
 
-@pytest.mark.parametrize("M,K,N", [(1000, 2048, 2000), (129, 4096, 9000), (2048, 11008, 2048)])
+@pytest.mark.parametrize("M,K,N", [(1000, 2048, 2000), (129, 4096, 9000), (2048, 11008, 2048), (4736, 512, 256)])
 def test_forward_pair_gemm_sparse24(M, K, N):
     """2:4 weights on the pair's structured-sparse MMA, against the expanded one-CTA kernel (bit for bit)
     and the oracle (sampled tokens)."""
