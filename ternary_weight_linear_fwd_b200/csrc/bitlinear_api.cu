@@ -53,7 +53,7 @@ struct DeviceState {
   int sm_count = 0;
   int32_t* status = nullptr;
   int sk_clusters[kSkMaxCluster + 1] = {};  // clusters of each size the few-token kernel fits at once (0: not asked)
-  int t2_pairs[2][3] = {};                  // CTA pairs of the pair GEMM (dense, 2:4; 64, 96, 128 tokens) resident at once
+  int t2_pairs[2] = {};                     // CTA pairs of the pair GEMM (dense, 2:4) resident at once (0: not asked)
 };
 
 std::mutex g_mu;
@@ -306,7 +306,7 @@ bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA,
 // CTA pairs of the pair GEMM resident at once (one CTA per SM), asked once per device and variant.
 template <int NM, int BN>
 int t2_active_pairs(DeviceState* dev) {
-  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1][BN == 64 ? 0 : BN == 96 ? 1 : 2];
+  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1];
   std::lock_guard<std::mutex> lk(g_mu);
   if (slot == 0) {
     int n = -1;
@@ -544,32 +544,16 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
 }
 
 // The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
-// The token tile (128, 96 or 64 tokens) is the one whose tiles fill the
-// resident pairs' waves best (ties to the wider tile).  DEVICE: no pair fits.
+// DEVICE: no pair fits at once.  (Token tiles of 96 and 64 were measured too:
+// a k-block's cost is mostly per instruction and per hand-off, so a narrower
+// tile did less work in nearly the same time, and more tiles never means
+// fewer rounds of the pairs.)
 template <int NM>
 bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
                           cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
-  const int bns[3] = {128, 96, 64};
-  const int pmax[3] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 96>(dev), t2_active_pairs<NM, 64>(dev)};
-  const int rows = (w->N + kT2Rows - 1) / kT2Rows;
-  int best = -1;
-  double best_eff = 0.0;
-  for (int i = 0; i < 3; ++i) {
-    if (pmax[i] < 1) continue;
-    const int units = rows * ((M + bns[i] - 1) / bns[i]);
-    const int waves = (units + pmax[i] - 1) / pmax[i];
-    const double eff = static_cast<double>(units) / (static_cast<double>(waves) * pmax[i]);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = i;
-    }
-  }
-  if (best < 0) return BITLINEAR_ERR_DEVICE;
-  switch (bns[best]) {
-    case 128: return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pmax[best]);
-    case 96: return tc2_launch<NM, 96>(w, M, qw, y, acc, s, dev, qb, plan, pmax[best]);
-    default: return tc2_launch<NM, 64>(w, M, qw, y, acc, s, dev, qb, plan, pmax[best]);
-  }
+  const int pairs = t2_active_pairs<NM, 128>(dev);
+  if (pairs < 1) return BITLINEAR_ERR_DEVICE;
+  return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs);
 }
 
 // sparse24: 2:4 weights on the structured-sparse MMA (otherwise expanded for the dense one).

@@ -13,17 +13,16 @@
 //   D[256 rows, BN tokens] += A[256 rows, K] * B[BN tokens, K]^T
 //   CTA r of the pair: rows 128 r .. 128 r + 127 of A and D (its own TMEM),
 //                      tokens BN/2 r .. BN/2 r + BN/2 - 1 of B (its own shared memory).
-// BN (64, 96 or 128) is chosen per shape so that the tiles fill whole waves of
-// the resident pairs (2560 -> 2560 at M = 2048: 160 tiles of 128 tokens leave
-// a third wave 16% full on 74 pairs, 220 tiles of 96 tokens fill three).
+// The library runs BN = 128 (narrower tiles did less work per k-block in
+// nearly the same time: the k-block's cost is mostly per MMA instruction and
+// per hand-off).
 //
 // Two rings: S copy stages in shared memory (the CTA's half of the activation
 // tile and its packed weights) and R operand slots (expanded codes in TMEM, or
 // compressed kept values in shared memory plus metadata in TMEM).  A copy
 // stage is freed when the MMAs that read its activations complete, an operand
-// slot likewise; S > R lets the copies run further ahead of the MMAs than the
-// operand slots alone would allow: the copies' latency from L2 (about 2 us
-// per round trip under this load) needs about eight stages in flight.
+// slot likewise (one commit per k-block serves both); S > R lets the copies
+// run further ahead of the MMAs than the operand slots alone would allow.
 //
 // Every copy is an ordinary one-CTA TMA load signalling the CTA's own
 // barrier.  The unpack warps of both CTAs wait for their CTA's stage (weights
@@ -49,11 +48,11 @@ constexpr int kT2Rows = 256;     // weight rows of a pair tile (the MMA's M)
 // 256-k stages.  Dense: 8 copy stages of 24 KB, 4 operand slots of 64 TMEM
 // columns beside two 128-column accumulators.  2:4: 6 copy stages of 24 KB and
 // 4 slots of 16 KB compressed operand (+ 8 metadata columns each).
-// BN: tokens of a pair tile (the MMA's N: 64, 96 or 128), BN / 2 per CTA.
+// BN: tokens of a pair tile (the MMA's N, a multiple of 32 up to 128), BN / 2 per CTA.
 template <int NM, int BN>
 struct T2 {
   static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
-  static_assert(BN == 64 || BN == 96 || BN == 128, "pair token tile");
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "pair token tile");
   static constexpr bool SP = NM == 3;
   static constexpr int KSUB = 2;
   static constexpr int HALF = BN / 2;
@@ -102,8 +101,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(s_rowsum + 2 * BN);
   uint64_t* empty = full + S;
   uint64_t* aready = empty + S;     // [R] rank 0's: both CTAs' unpack warps
-  uint64_t* afree = aready + R;     // [R] operand slot read by the MMAs (multicast commit)
-  uint64_t* accfull = afree + R;    // [2]
+  uint64_t* accfull = aready + R;   // [2]
   uint64_t* accempty = accfull + 2; // [2] rank 0's: both CTAs' epilogue warps
   uint64_t* drain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -128,10 +126,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int j = 0; j < R; ++j) {
-      mbar_init(&aready[j], 8);
-      mbar_init(&afree[j], 1);
-    }
+    for (int j = 0; j < R; ++j) mbar_init(&aready[j], 8);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 8);
@@ -245,8 +240,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                 bdesc + static_cast<uint64_t>((kk & 3) * 2), C::IDESC, (kb | kk) != 0 ? 1u : 0u);
             }
           }
-          tc_commit_pair_mc(&empty[s], 0x3);
-          tc_commit_pair_mc(&afree[j], 0x3);
+          tc_commit_pair_mc(&empty[s], 0x3);  // frees copy stage s, and operand slot j for k-block i + R
           issued = true;
         }
         if (ok) tc_commit_pair_mc(&accfull[buf], 0x3);
@@ -259,14 +253,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp >= 4 && warp < kTcEpiWarp0) {
     // -------------------------------------------------------------- unpack (both CTAs)
     // group g takes the k-blocks of parity g: with S and R even, every use of
-    // its copy stages and operand slots, so no parity wait skips a phase
+    // its copy stages and operand slots, so no parity wait skips a phase.  The
+    // operand slot of k-block i is free once the MMAs of k-block i - R have
+    // completed: the commit that frees copy stage (i - R) % S says so.
     const int grp = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     for (int i = grp; i < total_kb; i += 2) {
       const int s = i % S, j = i % R;
-      if (!mbar_wait(&full[s], (i / S) & 1) || (i >= R && !mbar_wait(&afree[j], ((i / R) - 1) & 1))) {
+      if (!mbar_wait(&full[s], (i / S) & 1) || (i >= R && !mbar_wait(&empty[(i - R) % S], ((i - R) / S) & 1))) {
         *a.status = kDevTimeoutUnpack;
         break;
       }

@@ -454,7 +454,6 @@ def test_forward_group_all_nm24_uses_sparse_mma():
 # Shapes whose plan is 128-token tiles without a K split (at least 75 tiles of 128 x 128), so the GEMM
 # runs on CTA pairs sharing one M = 256 MMA: ragged M (a last tile of 1 or 44 tokens), ragged N (the
 # last pair tile's second CTA partly or wholly past N), K not a multiple of the 256-k stage.
-# (4736, 512, 256): 74 tiles of 64 tokens fill the pairs exactly, so the 64-token pair tile is chosen.
 @pytest.mark.parametrize("M,K,N", [(1000, 2560, 2000), (4096, 1032, 640), (300, 2048, 11008), (129, 6912, 9000),
                                    (4736, 512, 256), (2048, 2560, 2560)])
 def test_forward_pair_gemm_dense(M, K, N):
