@@ -523,11 +523,11 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
   ta.M = M;
   ta.N = N;
   ta.K = K;
-  ta.kblocks = plan.kblocks;
+  ta.kblocks = (K + kTcSubK * C::KSUB - 1) / (kTcSubK * C::KSUB);  // the pair GEMM's own k-block
   ta.row_tiles = (N + kT2Rows - 1) / kT2Rows;
   ta.tok_tiles = (M + BN - 1) / BN;
   ta.ksplit = 1;
-  ta.kbs = plan.kblocks;
+  ta.kbs = ta.kblocks;
   ta.gamma = qw.gamma;
   ta.alpha = w->alpha;
   ta.rowsum = NM == 3 ? nullptr : qw.rowsum;

@@ -54,17 +54,17 @@ struct T2 {
   static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "pair token tile");
   static constexpr bool SP = NM == 3;
-  static constexpr int KSUB = 2;
+  static constexpr int KSUB = SP ? 2 : 4;  // k-block: 512 k dense (16 MMAs per hand-off), 256 k for 2:4
   static constexpr int HALF = BN / 2;
   static constexpr int B_SUB = HALF * 128;  // a whole number of 8-row swizzle atoms
   static constexpr int B_STAGE = B_SUB * KSUB;
-  static constexpr int A_VAL = SP ? kTcRows * 32 : kTcRows * 64;     // TMA bytes of values ...
-  static constexpr int A_META = SP ? kTcRows * 32 : 0;               // ... and metadata per stage
+  static constexpr int A_VAL = kTcRows * (SP ? 16 : 32) * KSUB;      // TMA bytes of values ...
+  static constexpr int A_META = SP ? kTcRows * 16 * KSUB : 0;        // ... and metadata per stage
   static constexpr int STAGE = B_STAGE + A_VAL + A_META;             // one copy stage
   static constexpr int OPA = SP ? kTcRows * 128 : 0;                 // compressed operand in shared memory
-  static constexpr int SLOT = SP ? 8 : 64;                           // TMEM columns per operand slot
+  static constexpr int SLOT = (SP ? 4 : 32) * KSUB;                  // TMEM columns per operand slot
   static constexpr int DCOLS = BN;
-  static constexpr int R = 4;                                        // operand slots
+  static constexpr int R = SP ? 4 : (512 - 2 * BN) / SLOT;           // operand slots (dense: as TMEM holds)
   // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
   static constexpr int FIXED = 2 * BN * 8 + 256;
   static constexpr int S = tc_min3(kTcMaxStages, (kTcSmemMax - FIXED - R * OPA) / STAGE, 64) & ~1;  // even
@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_st_32x32b_x8(tmem + lane_base + C::A_COL0 + j * C::SLOT, mw);
         fence_proxy_async_smem();
       } else {
-        const uint8_t* arow = st + r * 64;
+        const uint8_t* arow = st + r * 32 * KSUB;
 #pragma unroll
         for (int sub = 0; sub < KSUB; ++sub) {
           const uint4 lo = reinterpret_cast<const uint4*>(arow)[2 * sub];
