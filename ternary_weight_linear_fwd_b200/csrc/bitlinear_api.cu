@@ -509,7 +509,7 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
     return BITLINEAR_ERR_CUDA;
   if (NM == 0) {
     const int64_t ld = dense_ld(K);
-    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * C::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * C::KSUB, kTcRows, true)) return BITLINEAR_ERR_CUDA;  // swizzled rows
     mMeta = mA;
   } else {
     int64_t ldv = 0, ldm = 0;

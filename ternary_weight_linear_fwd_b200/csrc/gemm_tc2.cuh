@@ -288,11 +288,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_st_32x32b_x8(tmem + lane_base + C::A_COL0 + j * C::SLOT, mw);
         fence_proxy_async_smem();
       } else {
-        const uint8_t* arow = st + r * 32 * KSUB;
+        // the packed row (128 bytes) landed 128-byte-swizzled: its 16-byte chunk c sits at chunk c ^ (r % 8),
+        // so the 8 rows a quarter-warp reads at once fall in 8 different bank groups
+        static_assert(SP || 32 * KSUB == 128, "one swizzle row of packed codes per weight row");
+        const uint8_t* arow = st + r * 128;
 #pragma unroll
         for (int sub = 0; sub < KSUB; ++sub) {
-          const uint4 lo = reinterpret_cast<const uint4*>(arow)[2 * sub];
-          const uint4 hi = reinterpret_cast<const uint4*>(arow)[2 * sub + 1];
+          const uint4 lo = *reinterpret_cast<const uint4*>(arow + (((2 * sub) ^ (r & 7)) << 4));
+          const uint4 hi = *reinterpret_cast<const uint4*>(arow + (((2 * sub + 1) ^ (r & 7)) << 4));
           const uint32_t dw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
           uint32_t outw[32];
 #pragma unroll
