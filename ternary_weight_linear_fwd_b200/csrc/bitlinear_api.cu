@@ -126,9 +126,10 @@ thread_local MapCache t_maps;
 
 // 2-D uint8 tensor map: inner extent `inner` bytes, `outer` rows of `stride`
 // bytes, box {box_inner, box_outer}; out-of-range elements read as zero.
+// swizzle: 0 (none), 32, 64 or 128 (the shared-memory swizzle of the landed box, in bytes).
 bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t stride,
-                 uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
-  const MapKey k{base, inner, outer, stride, box_inner, box_outer, swizzle128 ? 1u : 0u};
+                 uint32_t box_inner, uint32_t box_outer, int swizzle) {
+  const MapKey k{base, inner, outer, stride, box_inner, box_outer, static_cast<uint32_t>(swizzle)};
   MapCache& c = t_maps;
   for (int i = 0; i < kMapCache; ++i)
     if (c.used[i] && c.key[i] == k) {
@@ -142,7 +143,11 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                  : swizzle == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                  : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
   c.key[c.next] = k;
@@ -417,7 +422,7 @@ bitlinear_status skinny_launch(const bitlinear_weights* w, const uint16_t* x, in
   const int64_t ld = dense_ld(K);
   CUtensorMap mW;
   if (!make_map_u8(&mW, w->codes, static_cast<uint64_t>(ld), static_cast<uint64_t>(N), static_cast<uint64_t>(ld), 32,
-                   kTcRows, false))
+                   kTcRows, 0))
     return BITLINEAR_ERR_CUDA;
   SkArgs sa;
   sa.x = x;
@@ -505,18 +510,18 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
   const int N = w->N, K = w->K;
   CUtensorMap mB, mA, mMeta;
   if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(qw.ldq),
-                   kTcSubK, static_cast<uint32_t>(C::HALF), true))
+                   kTcSubK, static_cast<uint32_t>(C::HALF), 128))
     return BITLINEAR_ERR_CUDA;
   if (NM == 0) {
     const int64_t ld = dense_ld(K);
-    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * C::KSUB, kTcRows, true)) return BITLINEAR_ERR_CUDA;  // swizzled rows
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * C::KSUB, kTcRows, 128)) return BITLINEAR_ERR_CUDA;  // swizzled rows
     mMeta = mA;
   } else {
     int64_t ldv = 0, ldm = 0;
     if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
       return BITLINEAR_ERR_PATTERN;
-    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, 16 * C::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
-    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16 * C::KSUB, kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, 16 * C::KSUB, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16 * C::KSUB, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
   }
   TcArgs ta;
   std::memset(&ta, 0, sizeof ta);
@@ -570,7 +575,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   const int bn = plan.bn;
   CUtensorMap mB, mA, mMeta;
   if (!make_map_u8(&mB, qw.q, static_cast<uint64_t>(k16(K)), static_cast<uint64_t>(M), static_cast<uint64_t>(qw.ldq),
-                   kTcSubK, static_cast<uint32_t>(bn), true))
+                   kTcSubK, static_cast<uint32_t>(bn), 128))
     return BITLINEAR_ERR_CUDA;
   TcArgs ta;
   ta.M = M;
@@ -596,7 +601,7 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   ta.vec_store = aligned16(y) && (!acc || aligned16(acc)) && (N % 8) == 0;
   if (nm == 0) {
     const int64_t ld = dense_ld(K);
-    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * tc_ksub(0, bn), kTcRows, false)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * tc_ksub(0, bn), kTcRows, 0)) return BITLINEAR_ERR_CUDA;
     mMeta = mA;
   } else {
     int64_t ldv = 0, ldm = 0;
@@ -605,8 +610,8 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
     const uint32_t vbox = nm != 2 ? static_cast<uint32_t>(16 * tc_ksub(nm, bn))
                                   : static_cast<uint32_t>((4 * w->nm_n + 12 + 15) / 16 * 16);
     ta.vbox = static_cast<int>(vbox);
-    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, false)) return BITLINEAR_ERR_CUDA;
-    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, static_cast<uint32_t>(16 * tc_ksub(nm, bn)), kTcRows, false))
+    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, static_cast<uint32_t>(16 * tc_ksub(nm, bn)), kTcRows, 0))
       return BITLINEAR_ERR_CUDA;
   }
   bitlinear_status st;
@@ -755,7 +760,7 @@ bitlinear_status gemv_dense_launch(const bitlinear_weights* const* w, uint16_t* 
     g.mat[i].y = y[i];
     g.mat[i].acc = acc ? acc[i] : nullptr;
     if (!make_map_u8(&map[i], w[i]->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N[i]),
-                     static_cast<uint64_t>(g.ld), 128, static_cast<uint32_t>(g.rows_box), true))
+                     static_cast<uint64_t>(g.ld), 128, static_cast<uint32_t>(g.rows_box), 128))
       return BITLINEAR_ERR_CUDA;
   }
   for (int i = count; i < kGemvGroup; ++i) map[i] = map[0];  // never selected
@@ -800,7 +805,7 @@ bitlinear_status gemv_lut_launch(const bitlinear_weights* w, uint16_t* y, int32_
   g.rows_box = g.mat[0].rows_base + 1;
   CUtensorMap map;
   if (!make_map_u8(&map, w->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N), static_cast<uint64_t>(g.ld),
-                   128, static_cast<uint32_t>(g.rows_box), true))
+                   128, static_cast<uint32_t>(g.rows_box), 128))
     return BITLINEAR_ERR_CUDA;
   bitlinear_status st = launch(gemv_lut_kernel, dim3(grid), dim3(kGemvThreads),
                                gemv_lut_smem_bytes(g.rows_box, g.ld, g.C), s, pdl, map, g);
@@ -840,9 +845,9 @@ bitlinear_status forward_gemv(const bitlinear_weights* w, const uint16_t* x, uin
   na.rows_box = na.rows_base + 1;
   CUtensorMap mv, mm;
   if (!make_map_u8(&mv, w->codes, static_cast<uint64_t>(ldv), static_cast<uint64_t>(N), static_cast<uint64_t>(ldv), 128,
-                   static_cast<uint32_t>(na.rows_box), true) ||
+                   static_cast<uint32_t>(na.rows_box), 128) ||
       !make_map_u8(&mm, w->meta, static_cast<uint64_t>(ldm), static_cast<uint64_t>(N), static_cast<uint64_t>(ldm), 128,
-                   static_cast<uint32_t>(na.rows_box), true))
+                   static_cast<uint32_t>(na.rows_box), 128))
     return BITLINEAR_ERR_CUDA;
   const size_t smem = gemv_nm_smem_bytes(na.rows_box, ldv, ldm, na.C, nm_lut);
   bitlinear_status st;
