@@ -53,7 +53,7 @@ struct DeviceState {
   int sm_count = 0;
   int32_t* status = nullptr;
   int sk_clusters[kSkMaxCluster + 1] = {};  // clusters of each size the few-token kernel fits at once (0: not asked)
-  int t2_pairs[2] = {};                     // CTA pairs of the pair GEMM (dense, 2:4) resident at once (0: not asked)
+  int t2_pairs[4] = {};  // CTA pairs of the pair GEMM resident at once (dense; 2:4 at BN 128, 192, 224; 0: not asked)
 };
 
 std::mutex g_mu;
@@ -311,7 +311,7 @@ bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA,
 // CTA pairs of the pair GEMM resident at once (one CTA per SM), asked once per device and variant.
 template <int NM, int BN>
 int t2_active_pairs(DeviceState* dev) {
-  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1];
+  int& slot = dev->t2_pairs[NM == 0 ? 0 : BN == 128 ? 1 : BN == 192 ? 2 : 3];
   std::lock_guard<std::mutex> lk(g_mu);
   if (slot == 0) {
     int n = -1;
@@ -544,21 +544,55 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
   pairs = std::min(pairs, ta.row_tiles * ta.tok_tiles);
   const bitlinear_status st =
       launch_ex(tc2_gemm_kernel<NM, BN>, dim3(2 * pairs), dim3(kTcThreads), C::SMEM, s, true, 2, mB, mA, mMeta, ta);
-  if (st == BITLINEAR_OK) t_last_kernel = NM == 0 ? "tc2_gemm_dense" : "tc2_gemm_sp24";
+  if (st == BITLINEAR_OK)
+    t_last_kernel = NM == 0      ? "tc2_gemm_dense"
+                    : BN == 128 ? "tc2_gemm_sp24_bn128"
+                    : BN == 192 ? "tc2_gemm_sp24_bn192"
+                                : "tc2_gemm_sp24_bn224";
   return st;
 }
 
+// Token tile of the 2:4 pair GEMM: the fewest (rounds of the pairs) x (time of
+// one k-block), the k-block's time taken as 272 + BN in units of 1.25 ns
+// (fitted to the measured k-block times of 2048 -> 11008 at M = 4096: about
+// 500, 590 and 620 ns at BN = 128, 192 and 224).  A wider tile does more work
+// per k-block but may leave the last round of pairs half idle.
+int t2_sparse_bn(int row_tiles, int M, const int pairs[3]) {
+  static const int bns[3] = {128, 192, 224};
+  int best = 128;
+  int64_t best_cost = -1;
+  for (int v = 0; v < 3; ++v) {
+    if (pairs[v] < 1) continue;
+    const int64_t units = static_cast<int64_t>(row_tiles) * ((M + bns[v] - 1) / bns[v]);
+    const int64_t cost = (units + pairs[v] - 1) / pairs[v] * (272 + bns[v]);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bns[v];
+    }
+  }
+  return best_cost < 0 ? 0 : best;
+}
+
 // The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
-// DEVICE: no pair fits at once.  (Token tiles of 96 and 64 were measured too:
-// a k-block's cost is mostly per instruction and per hand-off, so a narrower
-// tile did less work in nearly the same time, and more tiles never means
-// fewer rounds of the pairs.)
+// DEVICE: no pair fits at once.  (Dense token tiles of 96 and 64 were measured
+// too: a k-block's cost is mostly per instruction and per hand-off, so a
+// narrower tile did less work in nearly the same time.)
 template <int NM>
 bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
                           cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
-  const int pairs = t2_active_pairs<NM, 128>(dev);
-  if (pairs < 1) return BITLINEAR_ERR_DEVICE;
-  return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs);
+  if constexpr (NM == 0) {
+    const int pairs = t2_active_pairs<0, 128>(dev);
+    if (pairs < 1) return BITLINEAR_ERR_DEVICE;
+    return tc2_launch<0, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs);
+  } else {
+    const int pairs[3] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 192>(dev), t2_active_pairs<NM, 224>(dev)};
+    switch (t2_sparse_bn((w->N + kT2Rows - 1) / kT2Rows, M, pairs)) {
+      case 128: return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs[0]);
+      case 192: return tc2_launch<NM, 192>(w, M, qw, y, acc, s, dev, qb, plan, pairs[1]);
+      case 224: return tc2_launch<NM, 224>(w, M, qw, y, acc, s, dev, qb, plan, pairs[2]);
+      default: return BITLINEAR_ERR_DEVICE;
+    }
+  }
 }
 
 // sparse24: 2:4 weights on the structured-sparse MMA (otherwise expanded for the dense one).

@@ -13,9 +13,13 @@
 //   D[256 rows, BN tokens] += A[256 rows, K] * B[BN tokens, K]^T
 //   CTA r of the pair: rows 128 r .. 128 r + 127 of A and D (its own TMEM),
 //                      tokens BN/2 r .. BN/2 r + BN/2 - 1 of B (its own shared memory).
-// The library runs BN = 128 (narrower tiles did less work per k-block in
+// Dense weights run BN = 128 (narrower tiles did less work per k-block in
 // nearly the same time: the k-block's cost is mostly per MMA instruction and
-// per hand-off).
+// per hand-off; wider ones leave TMEM too few operand slots).  2:4 weights
+// read their operand from shared memory, where every MMA reads the 128 rows'
+// kept values again: a wider token tile spreads that read over more tokens,
+// so the host picks BN = 128, 192 or 224 by how many rounds of pairs a shape
+// takes.
 //
 // Two rings: S copy stages in shared memory (the CTA's half of the activation
 // tile and its packed weights) and R operand slots (expanded codes in TMEM, or
@@ -45,14 +49,14 @@ namespace bl {
 
 constexpr int kT2Rows = 256;     // weight rows of a pair tile (the MMA's M)
 
-// 256-k stages.  Dense: 8 copy stages of 24 KB, 4 operand slots of 64 TMEM
-// columns beside two 128-column accumulators.  2:4: 6 copy stages of 24 KB and
-// 4 slots of 16 KB compressed operand (+ 8 metadata columns each).
-// BN: tokens of a pair tile (the MMA's N, a multiple of 32 up to 128), BN / 2 per CTA.
+// Dense: 512-k stages, 4 copy stages of 48 KB, 2 operand slots of 128 TMEM
+// columns beside two 128-column accumulators.  2:4: 256-k stages, 4 to 6 copy
+// stages (by BN) and 4 slots of 16 KB compressed operand (+ 8 metadata columns each).
+// BN: tokens of a pair tile (the MMA's N, a multiple of 32), BN / 2 per CTA.
 template <int NM, int BN>
 struct T2 {
   static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
-  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "pair token tile");
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 224, "pair token tile");
   static constexpr bool SP = NM == 3;
   static constexpr int KSUB = SP ? 2 : 4;  // k-block: 512 k dense (16 MMAs per hand-off), 256 k for 2:4
   static constexpr int HALF = BN / 2;
@@ -63,13 +67,13 @@ struct T2 {
   static constexpr int STAGE = B_STAGE + A_VAL + A_META;             // one copy stage
   static constexpr int OPA = SP ? kTcRows * 128 : 0;                 // compressed operand in shared memory
   static constexpr int SLOT = (SP ? 4 : 32) * KSUB;                  // TMEM columns per operand slot
-  static constexpr int DCOLS = BN;
+  static constexpr int DCOLS = BN > 128 ? 256 : BN;  // accumulator 1's first column (256 for wide tiles)
   static constexpr int R = SP ? 4 : (512 - 2 * BN) / SLOT;           // operand slots (dense: as TMEM holds)
   // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
   static constexpr int FIXED = 2 * BN * 8 + 256;
   static constexpr int S = tc_min3(kTcMaxStages, (kTcSmemMax - FIXED - R * OPA) / STAGE, 64) & ~1;  // even
   static constexpr int SMEM = FIXED + S * STAGE + R * OPA;
-  static constexpr int A_COL0 = 2 * DCOLS;
+  static constexpr int A_COL0 = DCOLS + BN;         // operand slots after accumulator 1
   static_assert(A_COL0 + R * SLOT <= 512, "TMEM budget");
   static_assert(S >= R, "copy ring at least as deep as the operand ring");
   static constexpr uint32_t IDESC = SP ? idesc_i8_sp_s8s8(kT2Rows, BN) : idesc_i8_u8s8(kT2Rows, BN);

@@ -465,17 +465,25 @@ def test_forward_pair_gemm_dense(M, K, N):
     _check_rows(x, Wt, a, y, acc, rows)
 
 
-@pytest.mark.parametrize("M,K,N", [(1000, 2048, 2000), (129, 4096, 9000), (2048, 11008, 2048), (4736, 512, 256)])
-def test_forward_pair_gemm_sparse24(M, K, N):
+# The token tile (128, 192 or 224 tokens a pair) follows the rounds of pairs a shape takes on 148 SMs;
+# the wide tiles run here with a ragged last token tile, ragged N and K off the 256-k stage.
+@pytest.mark.parametrize("M,K,N,bn", [(1000, 2048, 2000, 128), (129, 4096, 9000, 128), (2048, 11008, 2048, 128),
+                                      (4736, 512, 256, 128), (3001, 1544, 2050, 192), (4000, 1032, 11000, 224),
+                                      (4096, 2048, 11008, 224)])
+def test_forward_pair_gemm_sparse24(M, K, N, bn):
     """2:4 weights on the pair's structured-sparse MMA, against the expanded one-CTA kernel (bit for bit)
     and the oracle (sampled tokens)."""
     x, Wt, a, w = _nm_case(M, K, N, 2, 4, seed=M + K)
     xd = to_dev_bf16(x)
     y, acc = bl.forward_nm(w, xd, want_acc=True)
-    assert bl.last_kernel() == "tc2_gemm_sp24", bl.last_kernel()
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert bl.last_kernel() == f"tc2_gemm_sp24_bn{bn}", bl.last_kernel()
+    else:
+        assert bl.last_kernel().startswith("tc2_gemm_sp24"), bl.last_kernel()
     ye, acce = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_NM24_EXPAND)
     assert torch.equal(acc, acce) and torch.equal(y.view(torch.int16), ye.view(torch.int16))
-    rows = np.unique(np.concatenate([[0, 63, 64, M - 1], synth.splitmix64(M, 8, 12) % M])).astype(np.int64)
+    edges = [t for t in (0, bn // 2 - 1, bn // 2, bn - 1, bn, M - 1) if t < M]  # each CTA's token half
+    rows = np.unique(np.concatenate([edges, synth.splitmix64(M, 8, 12) % M])).astype(np.int64)
     _check_rows(x, Wt, a, y, acc, rows)
 
 
