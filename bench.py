@@ -1082,7 +1082,8 @@ def main():
                      "call instead, device time of (flush, forward) graph replays minus flush-only replays",
                "flushed_tops": pre["flushed_tops"],
                "roofline": {"bound": "tensor", "achieved": pre["gemm_tops"], "peak": int8_peak, "unit": "TOPS",
-                            "frac": pre["gemm_tops"] / int8_peak, "kernel": "tc2_gemm_dense / tc_gemm_dense",
+                            "frac": pre["gemm_tops"] / int8_peak,
+                            "kernel": " / ".join(sorted({v["gemm_kernel"] for v in pre["shapes"].values()})),
                             "forward_frac": pre["tops"] / int8_peak,
                             "peak_source": f"{peak_kind} bf16_tflops x 2 (int8/bf16 nominal ratio)"}}
     cpu = cpu_all = None

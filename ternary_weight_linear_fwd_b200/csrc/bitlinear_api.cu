@@ -53,7 +53,7 @@ struct DeviceState {
   int sm_count = 0;
   int32_t* status = nullptr;
   int sk_clusters[kSkMaxCluster + 1] = {};  // clusters of each size the few-token kernel fits at once (0: not asked)
-  int t2_pairs[4] = {};  // CTA pairs of the pair GEMM resident at once (dense; 2:4 at BN 128, 192, 224; 0: not asked)
+  int t2_pairs[2][4] = {};  // CTA pairs of the pair GEMM resident at once ([dense, 2:4][BN 128 .. 224]; 0: not asked)
 };
 
 std::mutex g_mu;
@@ -311,7 +311,7 @@ bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA,
 // CTA pairs of the pair GEMM resident at once (one CTA per SM), asked once per device and variant.
 template <int NM, int BN>
 int t2_active_pairs(DeviceState* dev) {
-  int& slot = dev->t2_pairs[NM == 0 ? 0 : BN == 128 ? 1 : BN == 192 ? 2 : 3];
+  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1][(BN - 128) / 32];
   std::lock_guard<std::mutex> lk(g_mu);
   if (slot == 0) {
     int n = -1;
@@ -514,7 +514,8 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
     return BITLINEAR_ERR_CUDA;
   if (NM == 0) {
     const int64_t ld = dense_ld(K);
-    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * C::KSUB, kTcRows, 128)) return BITLINEAR_ERR_CUDA;  // swizzled rows
+    // packed rows land swizzled (128-byte rows at 512 k a stage, 64-byte rows at 256 k)
+    if (!make_map_u8(&mA, w->codes, ld, N, ld, 32 * C::KSUB, kTcRows, 32 * C::KSUB)) return BITLINEAR_ERR_CUDA;
     mMeta = mA;
   } else {
     int64_t ldv = 0, ldm = 0;
@@ -544,33 +545,37 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
   pairs = std::min(pairs, ta.row_tiles * ta.tok_tiles);
   const bitlinear_status st =
       launch_ex(tc2_gemm_kernel<NM, BN>, dim3(2 * pairs), dim3(kTcThreads), C::SMEM, s, true, 2, mB, mA, mMeta, ta);
-  if (st == BITLINEAR_OK)
-    t_last_kernel = NM == 0      ? "tc2_gemm_dense"
-                    : BN == 128 ? "tc2_gemm_sp24_bn128"
-                    : BN == 192 ? "tc2_gemm_sp24_bn192"
-                                : "tc2_gemm_sp24_bn224";
+  static const char* names[2][4] = {
+      {"tc2_gemm_dense_bn128", "tc2_gemm_dense_bn160", "tc2_gemm_dense_bn192", "tc2_gemm_dense_bn224"},
+      {"tc2_gemm_sp24_bn128", "tc2_gemm_sp24_bn160", "tc2_gemm_sp24_bn192", "tc2_gemm_sp24_bn224"}};
+  if (st == BITLINEAR_OK) t_last_kernel = names[NM == 0 ? 0 : 1][(BN - 128) / 32];
   return st;
 }
 
-// Token tile of the 2:4 pair GEMM: the fewest (rounds of the pairs) x (time of
-// one k-block), the k-block's time taken as 272 + BN in units of 1.25 ns
-// (fitted to the measured k-block times of 2048 -> 11008 at M = 4096: about
-// 500, 590 and 620 ns at BN = 128, 192 and 224).  A wider tile does more work
-// per k-block but may leave the last round of pairs half idle.
-int t2_sparse_bn(int row_tiles, int M, const int pairs[3]) {
-  static const int bns[3] = {128, 192, 224};
-  int best = 128;
+// Token tile of the pair GEMM: the fewest (rounds of the pairs) x (time of one
+// tile).  A wider tile does more work per k-block but may leave the last round
+// of pairs half idle.  A tile's time is modelled as a + b x (K / 256) ns: a =
+// 3.5 ns per token (epilogue and pipeline fill), b fitted to measured GEMM
+// times of 2048 -> 11008 and 11008 -> 2048 at M = 4096 on 148 SMs.  Dense b
+// grows with the tile (the codes in shared memory are read by every MMA, and
+// BN = 128 keeps them in TMEM instead); 2:4 b barely does.
+constexpr int kT2Bn[4] = {128, 160, 192, 224};
+constexpr int kT2B[2][4] = {{418, 577, 600, 633}, {456, 511, 511, 514}};  // [dense, 2:4][BN]: ns per 256 k
+
+int t2_pick_bn(int nm, int row_tiles, int M, int K, const int pairs[4]) {
+  int best = 0;
   int64_t best_cost = -1;
-  for (int v = 0; v < 3; ++v) {
+  for (int v = 0; v < 4; ++v) {
     if (pairs[v] < 1) continue;
-    const int64_t units = static_cast<int64_t>(row_tiles) * ((M + bns[v] - 1) / bns[v]);
-    const int64_t cost = (units + pairs[v] - 1) / pairs[v] * (272 + bns[v]);
+    const int64_t units = static_cast<int64_t>(row_tiles) * ((M + kT2Bn[v] - 1) / kT2Bn[v]);
+    const int64_t tile_ns = (7 * kT2Bn[v]) / 2 + static_cast<int64_t>(kT2B[nm == 0 ? 0 : 1][v]) * K / 256;
+    const int64_t cost = (units + pairs[v] - 1) / pairs[v] * tile_ns;
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
-      best = bns[v];
+      best = kT2Bn[v];
     }
   }
-  return best_cost < 0 ? 0 : best;
+  return best;
 }
 
 // The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
@@ -580,18 +585,14 @@ int t2_sparse_bn(int row_tiles, int M, const int pairs[3]) {
 template <int NM>
 bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
                           cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
-  if constexpr (NM == 0) {
-    const int pairs = t2_active_pairs<0, 128>(dev);
-    if (pairs < 1) return BITLINEAR_ERR_DEVICE;
-    return tc2_launch<0, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs);
-  } else {
-    const int pairs[3] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 192>(dev), t2_active_pairs<NM, 224>(dev)};
-    switch (t2_sparse_bn((w->N + kT2Rows - 1) / kT2Rows, M, pairs)) {
-      case 128: return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs[0]);
-      case 192: return tc2_launch<NM, 192>(w, M, qw, y, acc, s, dev, qb, plan, pairs[1]);
-      case 224: return tc2_launch<NM, 224>(w, M, qw, y, acc, s, dev, qb, plan, pairs[2]);
-      default: return BITLINEAR_ERR_DEVICE;
-    }
+  const int pairs[4] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 160>(dev), t2_active_pairs<NM, 192>(dev),
+                        t2_active_pairs<NM, 224>(dev)};
+  switch (t2_pick_bn(NM, (w->N + kT2Rows - 1) / kT2Rows, M, w->K, pairs)) {
+    case 128: return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs[0]);
+    case 160: return tc2_launch<NM, 160>(w, M, qw, y, acc, s, dev, qb, plan, pairs[1]);
+    case 192: return tc2_launch<NM, 192>(w, M, qw, y, acc, s, dev, qb, plan, pairs[2]);
+    case 224: return tc2_launch<NM, 224>(w, M, qw, y, acc, s, dev, qb, plan, pairs[3]);
+    default: return BITLINEAR_ERR_DEVICE;
   }
 }
 

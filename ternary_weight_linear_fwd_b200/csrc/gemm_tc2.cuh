@@ -13,13 +13,15 @@
 //   D[256 rows, BN tokens] += A[256 rows, K] * B[BN tokens, K]^T
 //   CTA r of the pair: rows 128 r .. 128 r + 127 of A and D (its own TMEM),
 //                      tokens BN/2 r .. BN/2 r + BN/2 - 1 of B (its own shared memory).
-// Dense weights run BN = 128 (narrower tiles did less work per k-block in
-// nearly the same time: the k-block's cost is mostly per MMA instruction and
-// per hand-off; wider ones leave TMEM too few operand slots).  2:4 weights
-// read their operand from shared memory, where every MMA reads the 128 rows'
-// kept values again: a wider token tile spreads that read over more tokens,
-// so the host picks BN = 128, 192 or 224 by how many rounds of pairs a shape
-// takes.
+// Token tiles: BN = 128, 192 or 224, picked on the host by how many rounds of
+// pairs a shape takes.  Narrower tiles did less work per k-block in nearly the
+// same time (the k-block's cost is mostly per MMA instruction and per
+// hand-off).  Dense weights at BN = 128 keep their expanded codes in TMEM
+// (the MMA's A from TMEM, 512-k stages); wider tiles leave TMEM no room for
+// operand slots beside two accumulators, so there the codes go to shared
+// memory like the 2:4 kept values (A from shared memory, 256-k stages).  An
+// A operand in shared memory is read again by every MMA; a wider token tile
+// spreads that read over more tokens.
 //
 // Two rings: S copy stages in shared memory (the CTA's half of the activation
 // tile and its packed weights) and R operand slots (expanded codes in TMEM, or
@@ -49,26 +51,30 @@ namespace bl {
 
 constexpr int kT2Rows = 256;     // weight rows of a pair tile (the MMA's M)
 
-// Dense: 512-k stages, 4 copy stages of 48 KB, 2 operand slots of 128 TMEM
-// columns beside two 128-column accumulators.  2:4: 256-k stages, 4 to 6 copy
-// stages (by BN) and 4 slots of 16 KB compressed operand (+ 8 metadata columns each).
+// Dense at BN = 128: 512-k stages, 4 copy stages of 48 KB, 2 operand slots of
+// 128 TMEM columns beside two 128-column accumulators.  Dense, wider: 256-k
+// stages, 4 copy stages, 2 slots of 32 KB expanded codes in shared memory.
+// 2:4: 256-k stages, 4 to 6 copy stages (by BN) and 4 slots of 16 KB
+// compressed operand (+ 8 metadata columns each).
 // BN: tokens of a pair tile (the MMA's N, a multiple of 32), BN / 2 per CTA.
 template <int NM, int BN>
 struct T2 {
   static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 224, "pair token tile");
   static constexpr bool SP = NM == 3;
-  static constexpr int KSUB = SP ? 2 : 4;  // k-block: 512 k dense (16 MMAs per hand-off), 256 k for 2:4
+  static constexpr bool OPS = SP || BN > 128;  // A operand in shared memory
+  static constexpr int KSUB = OPS ? 2 : 4;     // k-block: 512 k with A in TMEM (16 MMAs per hand-off), else 256 k
   static constexpr int HALF = BN / 2;
   static constexpr int B_SUB = HALF * 128;  // a whole number of 8-row swizzle atoms
   static constexpr int B_STAGE = B_SUB * KSUB;
   static constexpr int A_VAL = kTcRows * (SP ? 16 : 32) * KSUB;      // TMA bytes of values ...
   static constexpr int A_META = SP ? kTcRows * 16 * KSUB : 0;        // ... and metadata per stage
   static constexpr int STAGE = B_STAGE + A_VAL + A_META;             // one copy stage
-  static constexpr int OPA = SP ? kTcRows * 128 : 0;                 // compressed operand in shared memory
-  static constexpr int SLOT = (SP ? 4 : 32) * KSUB;                  // TMEM columns per operand slot
+  // operand slot in shared memory: 2:4 compressed (128 B a row), dense codes (256 B a row: two swizzle columns)
+  static constexpr int OPA = SP ? kTcRows * 128 : OPS ? kTcRows * 256 : 0;
+  static constexpr int SLOT = SP ? 8 : OPS ? 0 : 32 * KSUB;          // TMEM columns per operand slot
   static constexpr int DCOLS = BN > 128 ? 256 : BN;  // accumulator 1's first column (256 for wide tiles)
-  static constexpr int R = SP ? 4 : (512 - 2 * BN) / SLOT;           // operand slots (dense: as TMEM holds)
+  static constexpr int R = SP ? 4 : OPS ? 2 : (512 - 2 * BN) / SLOT;  // operand slots (TMEM: as it holds)
   // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
   static constexpr int FIXED = 2 * BN * 8 + 256;
   static constexpr int S = tc_min3(kTcMaxStages, (kTcSmemMax - FIXED - R * OPA) / STAGE, 64) & ~1;  // even
@@ -236,6 +242,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                    bdesc + static_cast<uint64_t>((kk & 1) * 4), tmem + C::A_COL0 + j * C::SLOT + kk * 2,
                                    C::IDESC, (kb | kk) != 0 ? 1u : 0u);
             }
+          } else if (C::OPS) {
+#pragma unroll
+            for (int kk = 0; kk < 4 * KSUB; ++kk) {  // A: 128-byte swizzle columns of 128 k, like B
+              const uint64_t adesc = smem_desc_sw128_kmajor(smem_u32(sOp + j * C::OPA + (kk >> 2) * (kTcRows * 128)));
+              const uint64_t bdesc = smem_desc_sw128_kmajor(smem_u32(sB + (kk >> 2) * C::B_SUB));
+              tc_mma_i8_ss_pair(dcol, adesc + static_cast<uint64_t>((kk & 3) * 2),
+                                bdesc + static_cast<uint64_t>((kk & 3) * 2), C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
           } else {
 #pragma unroll
             for (int kk = 0; kk < 4 * KSUB; ++kk) {
@@ -291,10 +305,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_st_32x32b_x8(tmem + lane_base + C::A_COL0 + j * C::SLOT, mw);
         fence_proxy_async_smem();
+      } else if (C::OPS) {
+        // the packed row (64 bytes) landed 64-byte-swizzled: its 16-byte chunk c sits at chunk c ^ ((r / 2) % 4),
+        // so the 8 rows a quarter-warp reads at once fall in 8 different bank groups; the codes of 128 k
+        // go to one 128-byte-swizzled row of the operand (chunk g at g ^ (r % 8))
+        const uint8_t* arow = st + r * 64;
+        uint8_t* orow = sOp + j * C::OPA + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int sub = 0; sub < KSUB; ++sub) {
+          const uint4 lo = *reinterpret_cast<const uint4*>(arow + (((2 * sub) ^ ((r >> 1) & 3)) << 4));
+          const uint4 hi = *reinterpret_cast<const uint4*>(arow + (((2 * sub + 1) ^ ((r >> 1) & 3)) << 4));
+          const uint32_t dw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+          for (int gi = 0; gi < 8; ++gi) {
+            uint32_t o[4];
+            codes_word_natural(dw[gi], o);
+            *reinterpret_cast<uint4*>(orow + sub * (kTcRows * 128) + ((gi ^ (r & 7)) << 4)) =
+                make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+        fence_proxy_async_smem();
       } else {
         // the packed row (128 bytes) landed 128-byte-swizzled: its 16-byte chunk c sits at chunk c ^ (r % 8),
         // so the 8 rows a quarter-warp reads at once fall in 8 different bank groups
-        static_assert(SP || 32 * KSUB == 128, "one swizzle row of packed codes per weight row");
+        static_assert(SP || C::OPS || 32 * KSUB == 128, "one swizzle row of packed codes per weight row");
         const uint8_t* arow = st + r * 128;
 #pragma unroll
         for (int sub = 0; sub < KSUB; ++sub) {

@@ -451,35 +451,43 @@ def test_forward_group_all_nm24_uses_sparse_mma():
 
 # ---------------------------------------------------------------- pairs of SMs (cta_group::2)
 
+def _check_pair_kernel(prefix, bn):
+    """The pair GEMM ran, with the token tile the host picks on a 148-SM B200."""
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert bl.last_kernel() == f"{prefix}_bn{bn}", bl.last_kernel()
+    else:
+        assert bl.last_kernel().startswith(prefix), bl.last_kernel()
+
+
 # Shapes whose plan is 128-token tiles without a K split (at least 75 tiles of 128 x 128), so the GEMM
 # runs on CTA pairs sharing one M = 256 MMA: ragged M (a last tile of 1 or 44 tokens), ragged N (the
 # last pair tile's second CTA partly or wholly past N), K not a multiple of the 256-k stage.
-@pytest.mark.parametrize("M,K,N", [(1000, 2560, 2000), (4096, 1032, 640), (300, 2048, 11008), (129, 6912, 9000),
-                                   (4736, 512, 256), (2048, 2560, 2560)])
-def test_forward_pair_gemm_dense(M, K, N):
+# The token tile (128 to 224 tokens a pair) follows the rounds of pairs a shape takes on 148 SMs: codes in
+# TMEM at 128 tokens, in shared memory for the wider tiles.
+@pytest.mark.parametrize("M,K,N,bn", [(1000, 2560, 2000, 128), (4096, 1032, 640, 192), (300, 2048, 11008, 128),
+                                      (129, 6912, 9000, 128), (4736, 512, 256, 128), (2048, 2560, 2560, 160),
+                                      (4000, 1032, 11000, 224)])
+def test_forward_pair_gemm_dense(M, K, N, bn):
     x, Wt, a, w = _dense_case(M, K, N, seed=M + K + N)
     y, acc = bl.forward(w, to_dev_bf16(x), want_acc=True)
-    assert bl.last_kernel() == "tc2_gemm_dense", bl.last_kernel()
+    _check_pair_kernel("tc2_gemm_dense", bn)
+    edges = [0, bn // 2 - 1, bn // 2, bn - 1, bn, M - 1]  # each CTA's token half
     rows = np.arange(M) if M * N <= 3_000_000 else np.unique(np.concatenate(
-        [[0, 63, 64, 127, 128, M - 1], synth.splitmix64(M, 7, 18) % M])).astype(np.int64)
+        [[t for t in edges if t < M], synth.splitmix64(M, 7, 18) % M])).astype(np.int64)
     _check_rows(x, Wt, a, y, acc, rows)
 
 
-# The token tile (128, 192 or 224 tokens a pair) follows the rounds of pairs a shape takes on 148 SMs;
-# the wide tiles run here with a ragged last token tile, ragged N and K off the 256-k stage.
+# The wide tiles run here with a ragged last token tile, ragged N and K off the 256-k stage.
 @pytest.mark.parametrize("M,K,N,bn", [(1000, 2048, 2000, 128), (129, 4096, 9000, 128), (2048, 11008, 2048, 128),
-                                      (4736, 512, 256, 128), (3001, 1544, 2050, 192), (4000, 1032, 11000, 224),
-                                      (4096, 2048, 11008, 224)])
+                                      (4736, 512, 256, 128), (2048, 2560, 2560, 160), (3001, 1544, 2050, 192),
+                                      (4000, 1032, 11000, 224), (4096, 2048, 11008, 224)])
 def test_forward_pair_gemm_sparse24(M, K, N, bn):
     """2:4 weights on the pair's structured-sparse MMA, against the expanded one-CTA kernel (bit for bit)
     and the oracle (sampled tokens)."""
     x, Wt, a, w = _nm_case(M, K, N, 2, 4, seed=M + K)
     xd = to_dev_bf16(x)
     y, acc = bl.forward_nm(w, xd, want_acc=True)
-    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
-        assert bl.last_kernel() == f"tc2_gemm_sp24_bn{bn}", bl.last_kernel()
-    else:
-        assert bl.last_kernel().startswith("tc2_gemm_sp24"), bl.last_kernel()
+    _check_pair_kernel("tc2_gemm_sp24", bn)
     ye, acce = bl.forward_nm(w, xd, want_acc=True, flags=bl.FLAG_NM24_EXPAND)
     assert torch.equal(acc, acce) and torch.equal(y.view(torch.int16), ye.view(torch.int16))
     edges = [t for t in (0, bn // 2 - 1, bn // 2, bn - 1, bn, M - 1) if t < M]  # each CTA's token half
