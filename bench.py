@@ -927,6 +927,23 @@ def _case_pair_gemm_m2048(dev):
         bl.forward_q8(w, q, g, rs)
 
 
+def _case_pair_gemm_wide_m2048(dev):
+    """bitlinear_forward_q8 at M = 2048 on the 2B4T down projection 6912 -> 2560: the pair GEMM with a
+    160-token tile (expanded codes in shared memory, A of the MMA from shared memory)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+    W = torch.from_numpy(synth.latent_weights(2560, 6912, seed=3)).to(dev)
+    w = bl.pack_weights(W)
+    del W
+    x = torch.from_numpy(synth.activations(2048, 6912, seed=3).view(np.int16)).to(dev).view(torch.bfloat16)
+    q, g, rs = bl.quant_act(x)
+    for _ in range(3):
+        bl.forward_q8(w, q, g, rs)
+
+
 def _case_prefill_forward_m2048(dev):
     """bitlinear_forward (quantisation launch + GEMM) at M = 2048 on the 2B4T gate projection 2560 -> 6912."""
     import numpy as np
@@ -943,7 +960,8 @@ def _case_prefill_forward_m2048(dev):
 
 
 PROFILE_CASES = {"few_token_m16": _case_few_token, "hbit_m1": _case_hbit_m1, "sparse24_m2048": _case_sparse24_m2048,
-                 "pair_gemm_m2048": _case_pair_gemm_m2048, "prefill_forward_m2048": _case_prefill_forward_m2048}
+                 "pair_gemm_m2048": _case_pair_gemm_m2048, "pair_gemm_wide_m2048": _case_pair_gemm_wide_m2048,
+                 "prefill_forward_m2048": _case_prefill_forward_m2048}
 
 
 def run_profile_case(name: str):
