@@ -53,7 +53,7 @@ struct DeviceState {
   int sm_count = 0;
   int32_t* status = nullptr;
   int sk_clusters[kSkMaxCluster + 1] = {};  // clusters of each size the few-token kernel fits at once (0: not asked)
-  int t2_pairs[2][4] = {};  // CTA pairs of the pair GEMM resident at once ([dense, 2:4][BN 128 .. 224]; 0: not asked)
+  int t2_pairs[3][4] = {};  // CTA pairs of the pair GEMM resident at once ([dense, 2:4, n:8][BN 128 .. 224]; 0: not asked)
 };
 
 std::mutex g_mu;
@@ -311,7 +311,7 @@ bitlinear_status launch_tc(int bn, const CUtensorMap& mB, const CUtensorMap& mA,
 // CTA pairs of the pair GEMM resident at once (one CTA per SM), asked once per device and variant.
 template <int NM, int BN>
 int t2_active_pairs(DeviceState* dev) {
-  int& slot = dev->t2_pairs[NM == 0 ? 0 : 1][(BN - 128) / 32];
+  int& slot = dev->t2_pairs[NM == 0 ? 0 : NM == 3 ? 1 : 2][(BN - 128) / 32];
   std::lock_guard<std::mutex> lk(g_mu);
   if (slot == 0) {
     int n = -1;
@@ -521,8 +521,12 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
     int64_t ldv = 0, ldm = 0;
     if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
       return BITLINEAR_ERR_PATTERN;
-    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, 16 * C::KSUB, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
-    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, 16 * C::KSUB, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
+    // n:8: the kept codes of 512 k (16 n bytes) and their 64 mask bytes per row and stage
+    const uint32_t vbox = NM == 2 ? static_cast<uint32_t>(16 * w->nm_n) : static_cast<uint32_t>(16 * C::KSUB);
+    const uint32_t mbox = NM == 2 ? 64u : static_cast<uint32_t>(16 * C::KSUB);
+    if (ldv < vbox || ldm < mbox) return BITLINEAR_ERR_DEVICE;  // rows shorter than one stage's box
+    if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
+    if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, mbox, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
   }
   TcArgs ta;
   std::memset(&ta, 0, sizeof ta);
@@ -537,6 +541,7 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
   ta.gamma = qw.gamma;
   ta.alpha = w->alpha;
   ta.rowsum = NM == 3 ? nullptr : qw.rowsum;
+  ta.nm_n = w->nm_n;
   ta.y = y;
   ta.acc = acc;
   ta.qb = qb;
@@ -545,10 +550,11 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
   pairs = std::min(pairs, ta.row_tiles * ta.tok_tiles);
   const bitlinear_status st =
       launch_ex(tc2_gemm_kernel<NM, BN>, dim3(2 * pairs), dim3(kTcThreads), C::SMEM, s, true, 2, mB, mA, mMeta, ta);
-  static const char* names[2][4] = {
+  static const char* names[3][4] = {
       {"tc2_gemm_dense_bn128", "tc2_gemm_dense_bn160", "tc2_gemm_dense_bn192", "tc2_gemm_dense_bn224"},
-      {"tc2_gemm_sp24_bn128", "tc2_gemm_sp24_bn160", "tc2_gemm_sp24_bn192", "tc2_gemm_sp24_bn224"}};
-  if (st == BITLINEAR_OK) t_last_kernel = names[NM == 0 ? 0 : 1][(BN - 128) / 32];
+      {"tc2_gemm_sp24_bn128", "tc2_gemm_sp24_bn160", "tc2_gemm_sp24_bn192", "tc2_gemm_sp24_bn224"},
+      {"tc2_gemm_n8_bn128", "", "", ""}};
+  if (st == BITLINEAR_OK) t_last_kernel = names[NM == 0 ? 0 : NM == 3 ? 1 : 2][(BN - 128) / 32];
   return st;
 }
 
@@ -585,14 +591,20 @@ int t2_pick_bn(int nm, int row_tiles, int M, int K, const int pairs[4]) {
 template <int NM>
 bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
                           cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
-  const int pairs[4] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 160>(dev), t2_active_pairs<NM, 192>(dev),
-                        t2_active_pairs<NM, 224>(dev)};
-  switch (t2_pick_bn(NM, (w->N + kT2Rows - 1) / kT2Rows, M, w->K, pairs)) {
-    case 128: return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs[0]);
-    case 160: return tc2_launch<NM, 160>(w, M, qw, y, acc, s, dev, qb, plan, pairs[1]);
-    case 192: return tc2_launch<NM, 192>(w, M, qw, y, acc, s, dev, qb, plan, pairs[2]);
-    case 224: return tc2_launch<NM, 224>(w, M, qw, y, acc, s, dev, qb, plan, pairs[3]);
-    default: return BITLINEAR_ERR_DEVICE;
+  if constexpr (NM == 2) {  // n:8: 128-token tiles only
+    const int pairs = t2_active_pairs<2, 128>(dev);
+    if (pairs < 1) return BITLINEAR_ERR_DEVICE;
+    return tc2_launch<2, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs);
+  } else {
+    const int pairs[4] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 160>(dev),
+                          t2_active_pairs<NM, 192>(dev), t2_active_pairs<NM, 224>(dev)};
+    switch (t2_pick_bn(NM, (w->N + kT2Rows - 1) / kT2Rows, M, w->K, pairs)) {
+      case 128: return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs[0]);
+      case 160: return tc2_launch<NM, 160>(w, M, qw, y, acc, s, dev, qb, plan, pairs[1]);
+      case 192: return tc2_launch<NM, 192>(w, M, qw, y, acc, s, dev, qb, plan, pairs[2]);
+      case 224: return tc2_launch<NM, 224>(w, M, qw, y, acc, s, dev, qb, plan, pairs[3]);
+      default: return BITLINEAR_ERR_DEVICE;
+    }
   }
 }
 
@@ -602,9 +614,10 @@ bitlinear_status tc_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, u
   const int N = w->N, K = w->K;
   const int nm = (w->nm_m == 0) ? 0 : (w->nm_m == 4 ? (sparse24 ? 3 : 1) : 2);
   const TcPlan plan = tc_plan(M, N, K, nm, dev->sm_count);
-  if ((nm == 0 || nm == 3) && plan.bn == 128 && plan.ksplit == 1) {
-    const bitlinear_status st = nm == 0 ? tc2_gemm<0>(w, M, qw, y, acc, s, dev, qb, plan)
-                                        : tc2_gemm<3>(w, M, qw, y, acc, s, dev, qb, plan);
+  if ((nm == 0 || nm == 2 || nm == 3) && plan.bn == 128 && plan.ksplit == 1) {
+    const bitlinear_status st = nm == 0   ? tc2_gemm<0>(w, M, qw, y, acc, s, dev, qb, plan)
+                                : nm == 3 ? tc2_gemm<3>(w, M, qw, y, acc, s, dev, qb, plan)
+                                          : tc2_gemm<2>(w, M, qw, y, acc, s, dev, qb, plan);
     if (st != BITLINEAR_ERR_DEVICE) return st;  // DEVICE: no pair fits at once, take the one-CTA kernel
   }
   const int bn = plan.bn;

@@ -51,24 +51,94 @@ namespace bl {
 
 constexpr int kT2Rows = 256;     // weight rows of a pair tile (the MMA's M)
 
+// n:8 expansion.  Selectors of the two byte permutes that turn the spread
+// kept codes of one 8-block (bytes 0 .. n-1: kept codes in k order, byte 7:
+// code 1) into its eight codes: output byte p takes kept code j when p is the
+// j-th set bit of the mask, byte 7 (code 1, weight 0) when p is pruned.
+// Low 16 bits: positions 0..3; high 16 bits: positions 4..7.
+__device__ __forceinline__ uint32_t n8_perm_selectors(uint32_t mask) {
+  uint32_t sel = 0u, j = 0u;
+  for (int p = 0; p < 8; ++p) {
+    uint32_t nib = 7u;
+    if ((mask >> p) & 1u) nib = j < 7u ? j++ : 7u;
+    sel |= nib << (4 * p);
+  }
+  return sel;
+}
+
+// One weight row's 512 k of an n:8 stage into its TMEM operand slot (u8
+// codes, natural k order, four stores of 128 k): the row's kept codes (16 n
+// bytes, 2 n bits per 8-block, blocks in k order) are read with 16-byte loads
+// into registers, the masks (64 bytes, one per 8-block) 16 bytes per 128 k.
+// n is a compile-time constant, so every block's bit offset is one too.
+template <int NK>
+__device__ __forceinline__ void n8_unpack_row(const uint8_t* vals, const uint8_t* masks, int r, const uint32_t* s_sel,
+                                              uint32_t taddr);
+
+// The eight codes of one 8-block (natural k order, one byte each) from its
+// kept codes (2 bits each, k order from bit 0, at most 7) and its selectors.
+__device__ __forceinline__ void n8_block_codes(uint32_t kept, uint32_t sel, uint32_t& lo_out, uint32_t& hi_out) {
+  uint32_t lo = kept & 0xFFu, hi = (kept >> 8) & 0xFFu;
+  lo = (lo | (lo << 12)) & 0x000F000Fu;  // codes 0, 1 | codes 2, 3 sixteen bits up
+  lo = (lo | (lo << 6)) & 0x03030303u;   // one code per byte
+  hi = (hi | (hi << 12)) & 0x000F000Fu;
+  hi = ((hi | (hi << 6)) & 0x03030303u) | 0x01000000u;  // byte 7: code 1 (n <= 7, so no kept code there)
+  lo_out = __byte_perm(lo, hi, sel & 0xFFFFu);
+  hi_out = __byte_perm(lo, hi, sel >> 16);
+}
+
+template <int NK>
+__device__ __forceinline__ void n8_unpack_row(const uint8_t* vals, const uint8_t* masks, int r, const uint32_t* s_sel,
+                                              uint32_t taddr) {
+  uint32_t v[4 * NK];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    const uint4 t = reinterpret_cast<const uint4*>(vals + r * 16 * NK)[i];
+    v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+  }
+  constexpr uint32_t fmask = (1u << (2 * NK)) - 1u;
+#pragma unroll
+  for (int sub = 0; sub < 4; ++sub) {
+    const uint4 mq = reinterpret_cast<const uint4*>(masks + r * 64)[sub];
+    const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
+    uint32_t outw[32];
+#pragma unroll
+    for (int jb = 0; jb < 16; ++jb) {
+      constexpr int kBits = 2 * NK;
+      const int bit = (sub * 16 + jb) * kBits;  // compile-time after unrolling
+      const int wi = bit >> 5, sh = bit & 31;
+      uint32_t kv = v[wi] >> sh;
+      if (sh + kBits > 32) kv |= v[wi + 1] << (32 - sh);
+      const uint32_t sel = s_sel[(mw[jb >> 2] >> (8 * (jb & 3))) & 0xFFu];
+      n8_block_codes(kv & fmask, sel, outw[2 * jb], outw[2 * jb + 1]);
+    }
+    tc_st_32x32b_x32(taddr + sub * 32, outw);
+  }
+}
+
 // Dense at BN = 128: 512-k stages, 4 copy stages of 48 KB, 2 operand slots of
 // 128 TMEM columns beside two 128-column accumulators.  Dense, wider: 256-k
 // stages, 4 copy stages, 2 slots of 32 KB expanded codes in shared memory.
 // 2:4: 256-k stages, 4 to 6 copy stages (by BN) and 4 slots of 16 KB
-// compressed operand (+ 8 metadata columns each).
+// compressed operand (+ 8 metadata columns each).  n:8 (NM = 2): as dense at
+// BN = 128, the stage holding the kept codes (16 n bytes a row) and the masks
+// (64 bytes a row) of 512 k instead of the packed codes.
 // BN: tokens of a pair tile (the MMA's N, a multiple of 32), BN / 2 per CTA.
 template <int NM, int BN>
 struct T2 {
-  static_assert(NM == 0 || NM == 3, "pair GEMM: dense or 2:4 on the sparse MMA");
+  static_assert(NM == 0 || NM == 2 || NM == 3, "pair GEMM: dense, n:8 expanded, or 2:4 on the sparse MMA");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 224, "pair token tile");
+  static_assert(NM != 2 || BN == 128, "n:8 weights: 128-token tiles (expanded codes in TMEM)");
   static constexpr bool SP = NM == 3;
+  static constexpr bool N8 = NM == 2;
   static constexpr bool OPS = SP || BN > 128;  // A operand in shared memory
   static constexpr int KSUB = OPS ? 2 : 4;     // k-block: 512 k with A in TMEM (16 MMAs per hand-off), else 256 k
   static constexpr int HALF = BN / 2;
   static constexpr int B_SUB = HALF * 128;  // a whole number of 8-row swizzle atoms
   static constexpr int B_STAGE = B_SUB * KSUB;
-  static constexpr int A_VAL = kTcRows * (SP ? 16 : 32) * KSUB;      // TMA bytes of values ...
-  static constexpr int A_META = SP ? kTcRows * 16 * KSUB : 0;        // ... and metadata per stage
+  // TMA bytes of values and of metadata per stage (n:8: room for n = 7, 2 n bits per 8 k)
+  static constexpr int A_VAL = N8 ? kTcRows * 112 : kTcRows * (SP ? 16 : 32) * KSUB;
+  static constexpr int A_META = SP ? kTcRows * 16 * KSUB : N8 ? kTcRows * 64 : 0;
   static constexpr int STAGE = B_STAGE + A_VAL + A_META;             // one copy stage
   // operand slot in shared memory: 2:4 compressed (128 B a row), dense codes (256 B a row: two swizzle columns)
   static constexpr int OPA = SP ? kTcRows * 128 : OPS ? kTcRows * 256 : 0;
@@ -76,7 +146,7 @@ struct T2 {
   static constexpr int DCOLS = BN > 128 ? 256 : BN;  // accumulator 1's first column (256 for wide tiles)
   static constexpr int R = SP ? 4 : OPS ? 2 : (512 - 2 * BN) / SLOT;  // operand slots (TMEM: as it holds)
   // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
-  static constexpr int FIXED = 2 * BN * 8 + 256;
+  static constexpr int FIXED = 2 * BN * 8 + 256 + (N8 ? 1024 : 0);  // scales, code sums, barriers (n:8: selectors)
   static constexpr int S = tc_min3(kTcMaxStages, (kTcSmemMax - FIXED - R * OPA) / STAGE, 64) & ~1;  // even
   static constexpr int SMEM = FIXED + S * STAGE + R * OPA;
   static constexpr int A_COL0 = DCOLS + BN;         // operand slots after accumulator 1
@@ -115,6 +185,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* accempty = accfull + 2; // [2] rank 0's: both CTAs' epilogue warps
   uint64_t* drain = accempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  // n:8: byte-permute selectors of the 256 masks, after the 256 bytes of barriers
+  uint32_t* s_sel = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(s_rowsum + 2 * BN) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -123,7 +195,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int nunits = a.row_tiles * a.tok_tiles;
   const int my_tiles = pair < nunits ? (nunits - 1 - pair) / npairs + 1 : 0;
   const int total_kb = my_tiles * KB;
-  const uint32_t tx_bytes = static_cast<uint32_t>(C::B_STAGE + C::A_VAL + C::A_META);
+  const uint32_t tx_bytes = static_cast<uint32_t>(C::B_STAGE + (C::N8 ? kTcRows * (16 * a.nm_n + 64) : C::A_VAL + C::A_META));
   auto unit_of = [&](int t, int& rt, int& tt) {  // token tile fastest: neighbouring pairs share weight rows
     const int g = pair + t * npairs;
     rt = g / a.tok_tiles;
@@ -151,6 +223,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc_pair(tmem_slot, 512);
     tmem_relinquish_pair();
   }
+  if (C::N8)
+    for (int m = threadIdx.x; m < 256; m += blockDim.x) s_sel[m] = n8_perm_selectors(static_cast<uint32_t>(m));
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrive or multicast commit
   tc_fence_after();
@@ -167,6 +241,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (SP) {
           tma_load_2d(dst, &mapA, kb * 16 * KSUB, row0, &full[s]);
           tma_load_2d(dst + C::A_VAL, &mapMeta, kb * 16 * KSUB, row0, &full[s]);
+        } else if (C::N8) {
+          tma_load_2d(dst, &mapA, kb * 16 * a.nm_n, row0, &full[s]);  // kept codes: 2 n bits per 8 k
+          tma_load_2d(dst + C::A_VAL, &mapMeta, kb * 64, row0, &full[s]);  // masks: one byte per 8 k
         } else {
           tma_load_2d(dst, &mapA, kb * 32 * KSUB, row0, &full[s]);
         }
@@ -325,10 +402,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         fence_proxy_async_smem();
+      } else if (C::N8) {
+        switch (a.nm_n) {
+          case 1: n8_unpack_row<1>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+          case 2: n8_unpack_row<2>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+          case 3: n8_unpack_row<3>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+          case 4: n8_unpack_row<4>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+          case 5: n8_unpack_row<5>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+          case 6: n8_unpack_row<6>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+          default: n8_unpack_row<7>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+        }
       } else {
         // the packed row (128 bytes) landed 128-byte-swizzled: its 16-byte chunk c sits at chunk c ^ (r % 8),
         // so the 8 rows a quarter-warp reads at once fall in 8 different bank groups
-        static_assert(SP || C::OPS || 32 * KSUB == 128, "one swizzle row of packed codes per weight row");
+        static_assert(SP || C::OPS || C::N8 || 32 * KSUB == 128, "one swizzle row of packed codes per weight row");
         const uint8_t* arow = st + r * 128;
 #pragma unroll
         for (int sub = 0; sub < KSUB; ++sub) {

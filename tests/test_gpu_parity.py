@@ -495,6 +495,23 @@ def test_forward_pair_gemm_sparse24(M, K, N, bn):
     _check_rows(x, Wt, a, y, acc, rows)
 
 
+# n:8 weights on the pair GEMM: kept codes and masks expanded to dense codes in TMEM (128-token tiles),
+# checked bit for bit against the same pruned ternary matrix packed dense, and against the oracle.
+@pytest.mark.parametrize("M,K,N,n", [(1000, 2048, 2000, 6), (1000, 2048, 2000, 1), (1000, 2048, 2000, 3),
+                                     (1000, 2048, 2000, 7), (4096, 1032, 640, 6), (300, 2048, 11008, 6),
+                                     (2048, 2560, 2560, 5)])
+def test_forward_pair_gemm_n8(M, K, N, n):
+    x, Wt, a, w = _nm_case(M, K, N, n, 8, seed=M + K + n)
+    xd = to_dev_bf16(x)
+    y, acc = bl.forward_nm(w, xd, want_acc=True)
+    assert bl.last_kernel() == "tc2_gemm_n8_bn128", bl.last_kernel()
+    wd = bl.pack_ternary(torch.from_numpy(np.ascontiguousarray(Wt, dtype=np.int8)).to(DEV), float(w.alpha.item()))
+    yd, accd = bl.forward(wd, xd, want_acc=True)
+    assert torch.equal(acc, accd) and torch.equal(y.view(torch.int16), yd.view(torch.int16))
+    rows = np.unique(np.concatenate([[0, 63, 64, 127, 128, M - 1], synth.splitmix64(M, 9, 12) % M])).astype(np.int64)
+    _check_rows(x, Wt, a, y, acc, rows)
+
+
 # ---------------------------------------------------------------- codes-in entry (the GEMM alone)
 
 @pytest.mark.parametrize("n,m", [(0, 0), (2, 4), (6, 8)])
