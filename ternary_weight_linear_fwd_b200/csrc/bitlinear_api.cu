@@ -521,9 +521,10 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
     int64_t ldv = 0, ldm = 0;
     if (bitlinear_packed_layout(N, K, w->nm_n, w->nm_m, &ldv, &ldm, nullptr, nullptr) != BITLINEAR_OK)
       return BITLINEAR_ERR_PATTERN;
-    // n:8: the kept codes of 512 k (16 n bytes) and their 64 mask bytes per row and stage
-    const uint32_t vbox = NM == 2 ? static_cast<uint32_t>(16 * w->nm_n) : static_cast<uint32_t>(16 * C::KSUB);
-    const uint32_t mbox = NM == 2 ? 64u : static_cast<uint32_t>(16 * C::KSUB);
+    // n:8: the kept codes (4 n bytes per 128 k) and the masks (16 bytes per 128 k) of a stage per row
+    const uint32_t vbox = static_cast<uint32_t>(NM == 2 ? 4 * C::KSUB * w->nm_n : 16 * C::KSUB);
+    const uint32_t mbox = static_cast<uint32_t>(16 * C::KSUB);
+    if (NM == 2 && vbox % 16 != 0) return BITLINEAR_ERR_DEVICE;  // odd n runs 512-k stages only
     if (ldv < vbox || ldm < mbox) return BITLINEAR_ERR_DEVICE;  // rows shorter than one stage's box
     if (!make_map_u8(&mA, w->codes, ldv, N, ldv, vbox, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
     if (!make_map_u8(&mMeta, w->meta, ldm, N, ldm, mbox, kTcRows, 0)) return BITLINEAR_ERR_CUDA;
@@ -553,7 +554,7 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
   static const char* names[3][4] = {
       {"tc2_gemm_dense_bn128", "tc2_gemm_dense_bn160", "tc2_gemm_dense_bn192", "tc2_gemm_dense_bn224"},
       {"tc2_gemm_sp24_bn128", "tc2_gemm_sp24_bn160", "tc2_gemm_sp24_bn192", "tc2_gemm_sp24_bn224"},
-      {"tc2_gemm_n8_bn128", "", "", ""}};
+      {"tc2_gemm_n8_bn128", "tc2_gemm_n8_bn160", "tc2_gemm_n8_bn192", "tc2_gemm_n8_bn224"}};
   if (st == BITLINEAR_OK) t_last_kernel = names[NM == 0 ? 0 : NM == 3 ? 1 : 2][(BN - 128) / 32];
   return st;
 }
@@ -564,9 +565,11 @@ bitlinear_status tc2_launch(const bitlinear_weights* w, int M, const QuantWs& qw
 // 3.5 ns per token (epilogue and pipeline fill), b fitted to measured GEMM
 // times of 2048 -> 11008 and 11008 -> 2048 at M = 4096 on 148 SMs.  Dense b
 // grows with the tile (the codes in shared memory are read by every MMA, and
-// BN = 128 keeps them in TMEM instead); 2:4 b barely does.
+// BN = 128 keeps them in TMEM instead); 2:4 b barely does; n:8 b is set by
+// the expansion of kept codes and masks.
 constexpr int kT2Bn[4] = {128, 160, 192, 224};
-constexpr int kT2B[2][4] = {{418, 577, 600, 633}, {456, 511, 511, 514}};  // [dense, 2:4][BN]: ns per 256 k
+// [dense, 2:4, n:8][BN]: ns per 256 k (n:8 measured on 6:8)
+constexpr int kT2B[3][4] = {{418, 577, 600, 633}, {456, 511, 511, 514}, {793, 833, 832, 860}};
 
 int t2_pick_bn(int nm, int row_tiles, int M, int K, const int pairs[4]) {
   int best = 0;
@@ -574,7 +577,7 @@ int t2_pick_bn(int nm, int row_tiles, int M, int K, const int pairs[4]) {
   for (int v = 0; v < 4; ++v) {
     if (pairs[v] < 1) continue;
     const int64_t units = static_cast<int64_t>(row_tiles) * ((M + kT2Bn[v] - 1) / kT2Bn[v]);
-    const int64_t tile_ns = (7 * kT2Bn[v]) / 2 + static_cast<int64_t>(kT2B[nm == 0 ? 0 : 1][v]) * K / 256;
+    const int64_t tile_ns = (7 * kT2Bn[v]) / 2 + static_cast<int64_t>(kT2B[nm == 0 ? 0 : nm == 3 ? 1 : 2][v]) * K / 256;
     const int64_t cost = (units + pairs[v] - 1) / pairs[v] * tile_ns;
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
@@ -591,10 +594,10 @@ int t2_pick_bn(int nm, int row_tiles, int M, int K, const int pairs[4]) {
 template <int NM>
 bitlinear_status tc2_gemm(const bitlinear_weights* w, int M, const QuantWs& qw, uint16_t* y, int32_t* acc,
                           cudaStream_t s, DeviceState* dev, float qb, const TcPlan& plan) {
-  if constexpr (NM == 2) {  // n:8: 128-token tiles only
-    const int pairs = t2_active_pairs<2, 128>(dev);
+  if (NM == 2 && (w->nm_n & 1)) {  // odd n: 128-token tiles (512-k stages keep the kept codes 16-byte aligned)
+    const int pairs = t2_active_pairs<NM, 128>(dev);
     if (pairs < 1) return BITLINEAR_ERR_DEVICE;
-    return tc2_launch<2, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs);
+    return tc2_launch<NM, 128>(w, M, qw, y, acc, s, dev, qb, plan, pairs);
   } else {
     const int pairs[4] = {t2_active_pairs<NM, 128>(dev), t2_active_pairs<NM, 160>(dev),
                           t2_active_pairs<NM, 192>(dev), t2_active_pairs<NM, 224>(dev)};

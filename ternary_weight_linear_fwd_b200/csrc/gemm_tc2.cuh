@@ -66,14 +66,16 @@ __device__ __forceinline__ uint32_t n8_perm_selectors(uint32_t mask) {
   return sel;
 }
 
-// One weight row's 512 k of an n:8 stage into its TMEM operand slot (u8
-// codes, natural k order, four stores of 128 k): the row's kept codes (16 n
-// bytes, 2 n bits per 8-block, blocks in k order) are read with 16-byte loads
-// into registers, the masks (64 bytes, one per 8-block) 16 bytes per 128 k.
-// n is a compile-time constant, so every block's bit offset is one too.
-template <int NK>
+// One weight row of an n:8 stage (SUBS x 128 k) into its operand slot: u8
+// codes in natural k order, either to TMEM (four stores of 128 k) or to the
+// 128-byte-swizzled shared-memory operand (orow: the row's line in the first
+// 128-k column; chunk g of a column at g ^ (r % 8)).  The row's kept codes
+// (4 SUBS n bytes, 2 n bits per 8-block, blocks in k order) are read with
+// 16-byte loads into registers, the masks (one byte per 8-block) 16 bytes per
+// 128 k.  n is a compile-time constant, so every block's bit offset is one.
+template <int NK, int SUBS, bool SMEM>
 __device__ __forceinline__ void n8_unpack_row(const uint8_t* vals, const uint8_t* masks, int r, const uint32_t* s_sel,
-                                              uint32_t taddr);
+                                              uint32_t taddr, uint8_t* orow);
 
 // The eight codes of one 8-block (natural k order, one byte each) from its
 // kept codes (2 bits each, k order from bit 0, at most 7) and its selectors.
@@ -87,32 +89,44 @@ __device__ __forceinline__ void n8_block_codes(uint32_t kept, uint32_t sel, uint
   hi_out = __byte_perm(lo, hi, sel >> 16);
 }
 
-template <int NK>
+template <int NK, int SUBS, bool SMEM>
 __device__ __forceinline__ void n8_unpack_row(const uint8_t* vals, const uint8_t* masks, int r, const uint32_t* s_sel,
-                                              uint32_t taddr) {
-  uint32_t v[4 * NK];
+                                              uint32_t taddr, uint8_t* orow) {
+  constexpr int VW = SUBS * NK;  // 32-bit words of kept codes in the row's stage
+  if constexpr (VW % 4 != 0) {   // rows not 16-byte aligned: never launched (the host keeps odd n at 512 k)
+    return;
+  } else {
+    uint32_t v[VW];
 #pragma unroll
-  for (int i = 0; i < NK; ++i) {
-    const uint4 t = reinterpret_cast<const uint4*>(vals + r * 16 * NK)[i];
-    v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
-  }
-  constexpr uint32_t fmask = (1u << (2 * NK)) - 1u;
-#pragma unroll
-  for (int sub = 0; sub < 4; ++sub) {
-    const uint4 mq = reinterpret_cast<const uint4*>(masks + r * 64)[sub];
-    const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
-    uint32_t outw[32];
-#pragma unroll
-    for (int jb = 0; jb < 16; ++jb) {
-      constexpr int kBits = 2 * NK;
-      const int bit = (sub * 16 + jb) * kBits;  // compile-time after unrolling
-      const int wi = bit >> 5, sh = bit & 31;
-      uint32_t kv = v[wi] >> sh;
-      if (sh + kBits > 32) kv |= v[wi + 1] << (32 - sh);
-      const uint32_t sel = s_sel[(mw[jb >> 2] >> (8 * (jb & 3))) & 0xFFu];
-      n8_block_codes(kv & fmask, sel, outw[2 * jb], outw[2 * jb + 1]);
+    for (int i = 0; i < VW / 4; ++i) {
+      const uint4 t = reinterpret_cast<const uint4*>(vals + r * 4 * VW)[i];
+      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
     }
-    tc_st_32x32b_x32(taddr + sub * 32, outw);
+    constexpr uint32_t fmask = (1u << (2 * NK)) - 1u;
+#pragma unroll
+    for (int sub = 0; sub < SUBS; ++sub) {
+      const uint4 mq = reinterpret_cast<const uint4*>(masks + r * 16 * SUBS)[sub];
+      const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
+      uint32_t outw[32];
+#pragma unroll
+      for (int jb = 0; jb < 16; ++jb) {
+        constexpr int kBits = 2 * NK;
+        const int bit = (sub * 16 + jb) * kBits;  // compile-time after unrolling
+        const int wi = bit >> 5, sh = bit & 31;
+        uint32_t kv = v[wi] >> sh;
+        if (sh + kBits > 32) kv |= v[wi + 1] << (32 - sh);
+        const uint32_t sel = s_sel[(mw[jb >> 2] >> (8 * (jb & 3))) & 0xFFu];
+        n8_block_codes(kv & fmask, sel, outw[2 * jb], outw[2 * jb + 1]);
+      }
+      if constexpr (SMEM) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<uint4*>(orow + sub * (kTcRows * 128) + ((g ^ (r & 7)) << 4)) =
+              make_uint4(outw[4 * g], outw[4 * g + 1], outw[4 * g + 2], outw[4 * g + 3]);
+      } else {
+        tc_st_32x32b_x32(taddr + sub * 32, outw);
+      }
+    }
   }
 }
 
@@ -120,15 +134,15 @@ __device__ __forceinline__ void n8_unpack_row(const uint8_t* vals, const uint8_t
 // 128 TMEM columns beside two 128-column accumulators.  Dense, wider: 256-k
 // stages, 4 copy stages, 2 slots of 32 KB expanded codes in shared memory.
 // 2:4: 256-k stages, 4 to 6 copy stages (by BN) and 4 slots of 16 KB
-// compressed operand (+ 8 metadata columns each).  n:8 (NM = 2): as dense at
-// BN = 128, the stage holding the kept codes (16 n bytes a row) and the masks
-// (64 bytes a row) of 512 k instead of the packed codes.
+// compressed operand (+ 8 metadata columns each).  n:8 (NM = 2): as dense,
+// the stage holding the kept codes (2 n bits per 8 k) and the masks (one byte
+// per 8 k) instead of the packed codes; wider tiles than 128 only for even n
+// (a 256-k stage's 8 n bytes of kept codes must start 16-byte aligned).
 // BN: tokens of a pair tile (the MMA's N, a multiple of 32), BN / 2 per CTA.
 template <int NM, int BN>
 struct T2 {
   static_assert(NM == 0 || NM == 2 || NM == 3, "pair GEMM: dense, n:8 expanded, or 2:4 on the sparse MMA");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 224, "pair token tile");
-  static_assert(NM != 2 || BN == 128, "n:8 weights: 128-token tiles (expanded codes in TMEM)");
   static constexpr bool SP = NM == 3;
   static constexpr bool N8 = NM == 2;
   static constexpr bool OPS = SP || BN > 128;  // A operand in shared memory
@@ -136,9 +150,9 @@ struct T2 {
   static constexpr int HALF = BN / 2;
   static constexpr int B_SUB = HALF * 128;  // a whole number of 8-row swizzle atoms
   static constexpr int B_STAGE = B_SUB * KSUB;
-  // TMA bytes of values and of metadata per stage (n:8: room for n = 7, 2 n bits per 8 k)
-  static constexpr int A_VAL = N8 ? kTcRows * 112 : kTcRows * (SP ? 16 : 32) * KSUB;
-  static constexpr int A_META = SP ? kTcRows * 16 * KSUB : N8 ? kTcRows * 64 : 0;
+  // TMA bytes of values and of metadata per stage (n:8: room for n = 7, 2 n bits and one mask bit per 8 k)
+  static constexpr int A_VAL = N8 ? kTcRows * 28 * KSUB : kTcRows * (SP ? 16 : 32) * KSUB;
+  static constexpr int A_META = SP || N8 ? kTcRows * 16 * KSUB : 0;
   static constexpr int STAGE = B_STAGE + A_VAL + A_META;             // one copy stage
   // operand slot in shared memory: 2:4 compressed (128 B a row), dense codes (256 B a row: two swizzle columns)
   static constexpr int OPA = SP ? kTcRows * 128 : OPS ? kTcRows * 256 : 0;
@@ -195,7 +209,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int nunits = a.row_tiles * a.tok_tiles;
   const int my_tiles = pair < nunits ? (nunits - 1 - pair) / npairs + 1 : 0;
   const int total_kb = my_tiles * KB;
-  const uint32_t tx_bytes = static_cast<uint32_t>(C::B_STAGE + (C::N8 ? kTcRows * (16 * a.nm_n + 64) : C::A_VAL + C::A_META));
+  const uint32_t tx_bytes =
+      static_cast<uint32_t>(C::B_STAGE + (C::N8 ? kTcRows * (4 * KSUB * a.nm_n + 16 * KSUB) : C::A_VAL + C::A_META));
   auto unit_of = [&](int t, int& rt, int& tt) {  // token tile fastest: neighbouring pairs share weight rows
     const int g = pair + t * npairs;
     rt = g / a.tok_tiles;
@@ -242,8 +257,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tma_load_2d(dst, &mapA, kb * 16 * KSUB, row0, &full[s]);
           tma_load_2d(dst + C::A_VAL, &mapMeta, kb * 16 * KSUB, row0, &full[s]);
         } else if (C::N8) {
-          tma_load_2d(dst, &mapA, kb * 16 * a.nm_n, row0, &full[s]);  // kept codes: 2 n bits per 8 k
-          tma_load_2d(dst + C::A_VAL, &mapMeta, kb * 64, row0, &full[s]);  // masks: one byte per 8 k
+          tma_load_2d(dst, &mapA, kb * 4 * KSUB * a.nm_n, row0, &full[s]);  // kept codes: 2 n bits per 8 k
+          tma_load_2d(dst + C::A_VAL, &mapMeta, kb * 16 * KSUB, row0, &full[s]);  // masks: one byte per 8 k
         } else {
           tma_load_2d(dst, &mapA, kb * 32 * KSUB, row0, &full[s]);
         }
@@ -382,7 +397,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_st_32x32b_x8(tmem + lane_base + C::A_COL0 + j * C::SLOT, mw);
         fence_proxy_async_smem();
-      } else if (C::OPS) {
+      } else if (C::OPS && !C::N8) {
         // the packed row (64 bytes) landed 64-byte-swizzled: its 16-byte chunk c sits at chunk c ^ ((r / 2) % 4),
         // so the 8 rows a quarter-warp reads at once fall in 8 different bank groups; the codes of 128 k
         // go to one 128-byte-swizzled row of the operand (chunk g at g ^ (r % 8))
@@ -403,15 +418,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         fence_proxy_async_smem();
       } else if (C::N8) {
-        switch (a.nm_n) {
-          case 1: n8_unpack_row<1>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
-          case 2: n8_unpack_row<2>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
-          case 3: n8_unpack_row<3>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
-          case 4: n8_unpack_row<4>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
-          case 5: n8_unpack_row<5>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
-          case 6: n8_unpack_row<6>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
-          default: n8_unpack_row<7>(st, st + C::A_VAL, r, s_sel, tmem + lane_base + C::A_COL0 + j * C::SLOT); break;
+        const uint32_t taddr = tmem + lane_base + C::A_COL0 + j * C::SLOT;
+        uint8_t* orow = sOp + j * C::OPA + (r >> 3) * 1024 + (r & 7) * 128;
+        switch (a.nm_n) {  // odd n never runs wide tiles (the host keeps them at 128 tokens)
+          case 2: n8_unpack_row<2, KSUB, C::OPS>(st, st + C::A_VAL, r, s_sel, taddr, orow); break;
+          case 4: n8_unpack_row<4, KSUB, C::OPS>(st, st + C::A_VAL, r, s_sel, taddr, orow); break;
+          case 6: n8_unpack_row<6, KSUB, C::OPS>(st, st + C::A_VAL, r, s_sel, taddr, orow); break;
+          case 1: n8_unpack_row<1, KSUB, C::OPS>(st, st + C::A_VAL, r, s_sel, taddr, orow); break;
+          case 3: n8_unpack_row<3, KSUB, C::OPS>(st, st + C::A_VAL, r, s_sel, taddr, orow); break;
+          case 5: n8_unpack_row<5, KSUB, C::OPS>(st, st + C::A_VAL, r, s_sel, taddr, orow); break;
+          default: n8_unpack_row<7, KSUB, C::OPS>(st, st + C::A_VAL, r, s_sel, taddr, orow); break;
         }
+        if (C::OPS) fence_proxy_async_smem();
       } else {
         // the packed row (128 bytes) landed 128-byte-swizzled: its 16-byte chunk c sits at chunk c ^ (r % 8),
         // so the 8 rows a quarter-warp reads at once fall in 8 different bank groups

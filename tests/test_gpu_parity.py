@@ -495,20 +495,25 @@ def test_forward_pair_gemm_sparse24(M, K, N, bn):
     _check_rows(x, Wt, a, y, acc, rows)
 
 
-# n:8 weights on the pair GEMM: kept codes and masks expanded to dense codes in TMEM (128-token tiles),
-# checked bit for bit against the same pruned ternary matrix packed dense, and against the oracle.
-@pytest.mark.parametrize("M,K,N,n", [(1000, 2048, 2000, 6), (1000, 2048, 2000, 1), (1000, 2048, 2000, 3),
-                                     (1000, 2048, 2000, 7), (4096, 1032, 640, 6), (300, 2048, 11008, 6),
-                                     (2048, 2560, 2560, 5)])
-def test_forward_pair_gemm_n8(M, K, N, n):
+# n:8 weights on the pair GEMM: kept codes and masks expanded to dense codes (in TMEM at 128-token tiles,
+# in shared memory at wider ones, even n only), checked bit for bit against the same pruned ternary matrix
+# packed dense, and against the oracle.
+@pytest.mark.parametrize("M,K,N,n,bn", [(1000, 2048, 2000, 6, 128), (1000, 2048, 2000, 1, 128),
+                                        (1000, 2048, 2000, 3, 128), (1000, 2048, 2000, 7, 128),
+                                        (4096, 1032, 640, 6, 192), (300, 2048, 11008, 6, 128),
+                                        (2048, 2560, 2560, 5, 128), (4000, 1032, 11000, 6, 224),
+                                        (2048, 6912, 2560, 6, 160), (3001, 1544, 2050, 2, 192),
+                                        (2048, 2560, 6912, 4, 224)])
+def test_forward_pair_gemm_n8(M, K, N, n, bn):
     x, Wt, a, w = _nm_case(M, K, N, n, 8, seed=M + K + n)
     xd = to_dev_bf16(x)
     y, acc = bl.forward_nm(w, xd, want_acc=True)
-    assert bl.last_kernel() == "tc2_gemm_n8_bn128", bl.last_kernel()
+    _check_pair_kernel("tc2_gemm_n8", bn)
     wd = bl.pack_ternary(torch.from_numpy(np.ascontiguousarray(Wt, dtype=np.int8)).to(DEV), float(w.alpha.item()))
     yd, accd = bl.forward(wd, xd, want_acc=True)
     assert torch.equal(acc, accd) and torch.equal(y.view(torch.int16), yd.view(torch.int16))
-    rows = np.unique(np.concatenate([[0, 63, 64, 127, 128, M - 1], synth.splitmix64(M, 9, 12) % M])).astype(np.int64)
+    edges = [0, bn // 2 - 1, bn // 2, bn - 1, bn, M - 1]  # each CTA's token half
+    rows = np.unique(np.concatenate([[t for t in edges if t < M], synth.splitmix64(M, 9, 12) % M])).astype(np.int64)
     _check_rows(x, Wt, a, y, acc, rows)
 
 
