@@ -944,6 +944,23 @@ def _case_pair_gemm_wide_m2048(dev):
         bl.forward_q8(w, q, g, rs)
 
 
+def _case_n8_gemm_m2048(dev):
+    """bitlinear_forward_q8 at M = 2048 on the 2B4T gate projection 2560 -> 6912 pruned 6:8: the pair GEMM
+    expanding kept codes and masks to dense codes (224-token tiles)."""
+    import numpy as np
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+    from ternary_weight_linear_fwd_b200 import synth
+    W = torch.from_numpy(synth.latent_weights(6912, 2560, seed=3)).to(dev)
+    w = bl.pack_weights(W, 6, 8)
+    del W
+    x = torch.from_numpy(synth.activations(2048, 2560, seed=3).view(np.int16)).to(dev).view(torch.bfloat16)
+    q, g, rs = bl.quant_act(x)
+    for _ in range(3):
+        bl.forward_q8(w, q, g, rs)
+
+
 def _case_prefill_forward_m2048(dev):
     """bitlinear_forward (quantisation launch + GEMM) at M = 2048 on the 2B4T gate projection 2560 -> 6912."""
     import numpy as np
@@ -961,6 +978,7 @@ def _case_prefill_forward_m2048(dev):
 
 PROFILE_CASES = {"few_token_m16": _case_few_token, "hbit_m1": _case_hbit_m1, "sparse24_m2048": _case_sparse24_m2048,
                  "pair_gemm_m2048": _case_pair_gemm_m2048, "pair_gemm_wide_m2048": _case_pair_gemm_wide_m2048,
+                 "n8_gemm_m2048": _case_n8_gemm_m2048,
                  "prefill_forward_m2048": _case_prefill_forward_m2048}
 
 
