@@ -70,6 +70,7 @@ def _load():
             "orc_hadamard_rows": (None, [P, i32, i32, i32, P]),
             "orc_quant_act4": (None, [P, i32, i32, P, P, P]),
             "orc_forward_hbit": (i32, [P, i32, i32, P, i32, f32, P, P, P, P]),
+            "orc_relu2_glu": (None, [P, P, i64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -252,6 +253,17 @@ def dequant(acc: np.ndarray, gamma: np.ndarray, alpha, Qb: int = QB) -> np.ndarr
 
 def bf16_from_f64(v: float) -> int:
     return int(_load().orc_bf16_from_f64(float(v)))
+
+
+def relu2_glu(g_bf16: np.ndarray, u_bf16: np.ndarray) -> np.ndarray:
+    """h = RN_bf16(RN_bf16(max(g, 0)^2) * u) elementwise on bf16 bits (the 2B4T FFN's squared ReLU on
+    the gate, times the up projection)."""
+    g = np.ascontiguousarray(g_bf16, dtype=np.uint16)
+    u = np.ascontiguousarray(u_bf16, dtype=np.uint16)
+    assert g.shape == u.shape
+    h = np.empty(g.shape, dtype=np.uint16)
+    _load().orc_relu2_glu(_ptr(g), _ptr(u), g.size, _ptr(h))
+    return h
 
 
 def forward(x_bf16: np.ndarray, Wt: np.ndarray, alpha, Qb: int = QB, threads: int = 1):

@@ -449,6 +449,23 @@ void orc_dequant(const int32_t* acc, const float* gamma, float alpha, int M, int
         }
 }
 
+/* Squared-ReLU gate of the FFN pair.  BitNet b1.58 2B4T technical report
+ * summary (greeksharifa.github.io page), section 2 "Architecture": the FFN
+ * sublayer uses squared ReLU, the rectified activation squared.  With the
+ * block's gate and up projections (both BitLinears of the same x, outputs g
+ * and u in bf16), the reading taken here is h = ReLU(g)^2 * u elementwise,
+ * every bf16 operation rounded once: sq = RN_bf16(max(g, 0)^2), then
+ * h = RN_bf16(sq * u).  Both products are exact in double (8-bit significands),
+ * so each line rounds exactly once. */
+void orc_relu2_glu(const uint16_t* g, const uint16_t* u, int64_t count, uint16_t* h) {
+    for (int64_t i = 0; i < count; ++i) {
+        double gv = (double)orc_bf16_to_f32(g[i]);
+        double r = gv > 0.0 ? gv : 0.0;
+        uint16_t sq = orc_bf16_from_f64(r * r);
+        h[i] = orc_bf16_from_f64((double)orc_bf16_to_f32(sq) * (double)orc_bf16_to_f32(u[i]));
+    }
+}
+
 /* Whole forward for a dense ternary matrix: quantise activations, contract,
  * dequantise.  q_out/acc_out/gamma_out may be NULL.  Returns 0 or -1. */
 int orc_forward(const uint16_t* x, int M, int K, const int8_t* Wt, int N, float alpha, int Qb,

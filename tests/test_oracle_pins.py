@@ -448,3 +448,58 @@ def test_threaded_contraction_equals_plain_loop():
     for th in (2, 3, 8, 400):
         np.testing.assert_array_equal(oracle.matmul_i32_threads(q, T, th), a1)
     np.testing.assert_array_equal(a1, (q.astype(np.float64) @ T.astype(np.float64).T).astype(np.int64))
+
+
+# ---------------------------------------------------------------- squared-ReLU gate/up (FFN of the 2B4T model)
+
+def _f32_of_bf16(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32)
+
+
+def test_relu2_glu_nonpositive_gate_is_signed_zero():
+    """ReLU of a non-positive gate is 0, so h is a zero carrying the sign of u (IEEE 0 * u)."""
+    g = _bf16([-2.5, -0.0, 0.0, -1e-3, -300.0])
+    u = _bf16([3.0, 1.5, -7.0, -2.0, 0.25])
+    h = oracle.relu2_glu(g, u)
+    assert [int(v) for v in h] == [0x0000, 0x0000, 0x8000, 0x8000, 0x0000]
+
+
+def test_relu2_glu_powers_of_two_exact():
+    """g = 2^a > 0, u = +-2^b: h = +-2^(2a + b) exactly (no rounding anywhere)."""
+    rng = np.random.default_rng(3)
+    a = rng.integers(-20, 20, 64)
+    b = rng.integers(-20, 20, 64)
+    s = rng.choice([-1.0, 1.0], 64)
+    g = _bf16([2.0 ** int(v) for v in a])
+    u = _bf16([float(sv) * 2.0 ** int(v) for sv, v in zip(s, b)])
+    h = _f32_of_bf16(oracle.relu2_glu(g, u))
+    assert np.array_equal(h, (s * 2.0 ** (2 * a + b)).astype(np.float32))
+
+
+def test_relu2_glu_hand_rounding():
+    """Worked by hand.  g = 1 + 2^-7 squares to 1 + 2^-6 + 2^-14, which bf16 (8 significant bits,
+    spacing 2^-7 on [1, 2)) rounds to 1 + 2^-6 = 1.015625.  Times u = 3: 3.046875 = 1.5234375 * 2,
+    exact in bf16 (0x4043).  Times u = 1.25: 1.26953125, exactly half-way between 1.265625 and
+    1.2734375, so ties-to-even gives 1.265625 (0x3FA2) -- whereas rounding g^2 u only once
+    (1.26960754...) would give 1.2734375 (0x3FA3): the squared gate is rounded first.
+    g = 1.5, u = 2: 2.25 * 2 = 4.5 (0x4090)."""
+    g = _bf16([1.0 + 2.0 ** -7, 1.0 + 2.0 ** -7, 1.5])
+    u = _bf16([3.0, 1.25, 2.0])
+    assert [int(v) for v in oracle.relu2_glu(g, u)] == [0x4043, 0x3FA2, 0x4090]
+
+
+def test_relu2_glu_odd_in_u_and_within_two_roundings():
+    """h(g, -u) = -h(g, u); and |h - max(g, 0)^2 u| <= (2^-8 + 2^-8 + 2^-16) |max(g, 0)^2 u| for
+    normal results (two roundings to 8 significant bits)."""
+    rng = np.random.default_rng(11)
+    gv = rng.normal(0, 3, 4096)
+    uv = rng.normal(0, 3, 4096)
+    g, u = _bf16(gv), _bf16(uv)
+    h = oracle.relu2_glu(g, u)
+    hn = oracle.relu2_glu(g, _bf16(-_f32_of_bf16(u).astype(np.float64)))
+    assert np.array_equal(_f32_of_bf16(hn), -_f32_of_bf16(h))
+    ex = np.maximum(_f32_of_bf16(g).astype(np.float64), 0.0) ** 2 * _f32_of_bf16(u).astype(np.float64)
+    hv = _f32_of_bf16(h).astype(np.float64)
+    big = np.abs(ex) > 1e-30
+    assert np.all(np.abs(hv[big] - ex[big]) <= (2.0 ** -7 + 2.0 ** -16) * np.abs(ex[big]))
+    assert np.all(hv[~big] == 0.0)
