@@ -326,6 +326,34 @@ bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t cou
                                          uint16_t* const* y, int32_t* const* acc, void* workspace,
                                          size_t workspace_bytes, uint32_t flags, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * FFN gate/up pair with squared ReLU.
+ *
+ * Source: BitNet b1.58 2B4T technical report summary (greeksharifa.github.io
+ * page), section 2 "Architecture": the FFN sublayer uses squared ReLU, the
+ * rectified activation squared.  With the block's gate and up projections
+ * (two BitLinears of the same x) the result is taken as, elementwise,
+ *     h = RN_bf16( RN_bf16( max(g, 0)^2 ) * u ),
+ * g = BitLinear_gate(x) and u = BitLinear_up(x) in bf16 exactly as
+ * bitlinear_forward returns them, each bf16 operation rounded once.
+ *
+ * w_gate, w_up: packed weights of the same N and K (dense or N:M), device.
+ * x: bf16 bits [M, K], device, 16-byte aligned.  h: bf16 bits [M, N], device.
+ * workspace: device scratch of at least
+ * bitlinear_forward_relu2_glu_workspace_bytes(M, N, K, flags) bytes, 16-byte
+ * aligned (g and u for M > 1, then the forward's own workspace); may be NULL
+ * when M = 1, both matrices are dense and BITLINEAR_FLAG_PATH_TC is not set:
+ * then one launch computes both BitLinears and h.  Otherwise the pair runs as
+ * bitlinear_forward_group into the workspace and h is formed by one more
+ * launch.  flags: as bitlinear_forward (BITLINEAR_FLAG_DECODE_LUT rejected).
+ * Errors: NULL, SHAPE (N or K differ, M out of range), ALIGN, FLAGS,
+ * WORKSPACE, PATTERN, DEVICE, CUDA; h is then unspecified.
+ * ------------------------------------------------------------------------- */
+size_t bitlinear_forward_relu2_glu_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags);
+bitlinear_status bitlinear_forward_relu2_glu(const bitlinear_weights* w_gate, const bitlinear_weights* w_up,
+                                             const uint16_t* x, int32_t M, uint16_t* h, void* workspace,
+                                             size_t workspace_bytes, uint32_t flags, void* stream);
+
 /* Largest scratch, in bytes, that bitlinear_forward_noalloc can use. */
 #define BITLINEAR_NOALLOC_SCRATCH_BYTES (8u << 20)
 

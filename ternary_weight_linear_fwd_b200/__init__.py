@@ -16,7 +16,8 @@ __all__ = [
     "BitLinearError", "PackedWeights", "lib", "packed_layout", "pack_weights", "pack_ternary",
     "quant_act", "rmsnorm_quant_act", "forward", "forward_nm", "forward_group", "forward_norm",
     "forward_workspace_bytes", "device_status", "last_kernel", "layout_version", "hadamard_quant_act4",
-    "forward_hbit", "HBIT_MAX_K", "forward_q8", "forward_q8_workspace_bytes",
+    "forward_hbit", "HBIT_MAX_K", "forward_q8", "forward_q8_workspace_bytes", "forward_relu2_glu",
+    "forward_relu2_glu_workspace_bytes",
     "FLAG_PDL", "FLAG_PATH_GEMV", "FLAG_PATH_TC", "FLAG_DECODE_LUT", "FLAG_PATH_PERSISTENT", "FLAG_NM24_EXPAND",
 ]
 
@@ -75,6 +76,9 @@ def lib() -> ctypes.CDLL:
             "bitlinear_forward_hbit": (st, [ctypes.POINTER(_Weights), P, i32, P, P, P, sz, u32, P]),
             "bitlinear_forward_q8": (st, [ctypes.POINTER(_Weights), P, i32, P, P, i32, P, P, P, sz, u32, P]),
             "bitlinear_forward_q8_workspace_bytes": (sz, [i32, i32, i32]),
+            "bitlinear_forward_relu2_glu": (st, [ctypes.POINTER(_Weights), ctypes.POINTER(_Weights), P, i32, P, P, sz,
+                                                 u32, P]),
+            "bitlinear_forward_relu2_glu_workspace_bytes": (sz, [i32, i32, i32, u32]),
             "bitlinear_device_status": (st, [P, ctypes.POINTER(i32), i32]),
             "bitlinear_last_kernel": (ctypes.c_char_p, []),
             "bitlinear_layout_version": (i32, []),
@@ -336,6 +340,32 @@ def forward_group(ws, x, want_acc: bool = False, flags: int = 0, workspace=None,
     _check(lib().bitlinear_forward_group(arr, count, _ptr(x), M, yp, ap, _ptr(workspace), ws_n, flags,
                                          _stream(stream)), "forward_group")
     return list(zip(ys, accs)) if want_acc else ys
+
+
+def forward_relu2_glu_workspace_bytes(M: int, N: int, K: int, flags: int = 0) -> int:
+    return int(lib().bitlinear_forward_relu2_glu_workspace_bytes(M, N, K, flags))
+
+
+def forward_relu2_glu(w_gate: PackedWeights, w_up: PackedWeights, x, flags: int = 0, workspace=None, out=None,
+                      stream=None):
+    """h = RN(RN(max(g, 0)^2) * u) with g, u the BitLinear outputs of the FFN's gate and up projections
+    on x (same N and K): the 2B4T FFN's squared ReLU on the gate, times the up projection."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 2 and x.shape[1] == w_gate.K
+    if (w_up.N, w_up.K) != (w_gate.N, w_gate.K):
+        raise ValueError("forward_relu2_glu: gate and up must have the same N and K")
+    M = x.shape[0]
+    _check_out(out, (M, w_gate.N), torch.bfloat16, x.device, "out")
+    _check_workspace(workspace, x.device)
+    h = out if out is not None else torch.empty((M, w_gate.N), dtype=torch.bfloat16, device=x.device)
+    need = forward_relu2_glu_workspace_bytes(M, w_gate.N, w_gate.K, flags)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    wg, wu = w_gate.c_struct(), w_up.c_struct()
+    _check(lib().bitlinear_forward_relu2_glu(ctypes.byref(wg), ctypes.byref(wu), _ptr(x), M, _ptr(h),
+                                             _ptr(workspace), ws_n, flags, _stream(stream)), "forward_relu2_glu")
+    return h
 
 
 def forward_norm(w: PackedWeights, x, g, eps: float, want_acc: bool = False, flags: int = 0, workspace=None,

@@ -829,6 +829,25 @@ bitlinear_status gemv_dense_launch(const bitlinear_weights* const* w, uint16_t* 
   return st;
 }
 
+// Rows per CTA of the fused one-token kernel: about one CTA per SM, doubled
+// until both matrices' rows fit the shared-memory budget and a box of at most
+// 128 rows (a multiple of 8).  False: no such split (very long K).
+bool glu_split(int N, int64_t ld, int C, int sm_count, int* ctas, int* rows_box) {
+  int c = std::max(1, std::min(N, sm_count));
+  for (;;) {
+    const int rows = (N + c - 1) / c;
+    const int box = (rows + 7) / 8 * 8;
+    if (box <= 128 && gemv_glu_smem_bytes(box, ld, C) <= static_cast<size_t>(kGemvWeightSmem) + 16 * 1024) {
+      *ctas = c;
+      *rows_box = box;
+      return true;
+    }
+    if (c >= N) return false;
+    c = std::min(N, 2 * c);
+  }
+}
+
+
 // The lookup-table variant of the dense decode GEMV (one matrix).
 bitlinear_status gemv_lut_launch(const bitlinear_weights* w, uint16_t* y, int32_t* acc, const uint16_t* x, bool pdl,
                                  cudaStream_t s, DeviceState* dev) {
@@ -1292,6 +1311,78 @@ size_t bitlinear_forward_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32
   // enough for dense and for N:M weights (their k-blocks differ, and with them the K split)
   const int sm = plan_sm_count();
   return std::max({tc_workspace(M, N, K, 0, sm), tc_workspace(M, N, K, 1, sm), tc_workspace(M, N, K, 2, sm)});
+}
+
+// ---------------------------------------------------------------- FFN gate/up with squared ReLU
+
+size_t bitlinear_forward_relu2_glu_workspace_bytes(int32_t M, int32_t N, int32_t K, uint32_t flags) {
+  if (M < 1 || K < 1 || N < 1) return 0;
+  // the two BitLinear outputs, then the forward's own workspace (none for the fused one-token kernel)
+  return 2 * align256(static_cast<size_t>(M) * N * 2) + bitlinear_forward_workspace_bytes(M, N, K, flags);
+}
+
+bitlinear_status bitlinear_forward_relu2_glu(const bitlinear_weights* w_gate, const bitlinear_weights* w_up,
+                                             const uint16_t* x, int32_t M, uint16_t* h, void* workspace,
+                                             size_t workspace_bytes, uint32_t flags, void* stream) {
+  if (!w_gate || !w_up || !x || !h) return BITLINEAR_ERR_NULL;
+  bitlinear_status st = check_matrix(w_gate, h, nullptr);
+  if (st != BITLINEAR_OK) return st;
+  st = check_matrix(w_up, h, nullptr);
+  if (st != BITLINEAR_OK) return st;
+  if (w_gate->N != w_up->N || w_gate->K != w_up->K) return BITLINEAR_ERR_SHAPE;
+  if (M < 1 || M > BITLINEAR_MAX_M) return BITLINEAR_ERR_SHAPE;
+  if (!aligned16(x)) return BITLINEAR_ERR_ALIGN;
+  st = check_flags(flags, M);
+  if (st != BITLINEAR_OK) return st;
+  if (flags & BITLINEAR_FLAG_DECODE_LUT) return BITLINEAR_ERR_FLAGS;
+  DeviceState* dev = nullptr;
+  st = current_device(&dev);
+  if (st != BITLINEAR_OK) return st;
+  const bool pdl = (flags & BITLINEAR_FLAG_PDL) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int N = w_gate->N, K = w_gate->K;
+  // one token, dense weights: both BitLinears and h in one launch
+  if (M == 1 && !(flags & BITLINEAR_FLAG_PATH_TC) && w_gate->nm_m == 0 && w_up->nm_m == 0) {
+    GemvGlu g;
+    std::memset(&g, 0, sizeof g);
+    g.ld = dense_ld(K);
+    g.C = static_cast<int>(g.ld / 16);
+    g.K = K;
+    g.x = x;
+    g.h = h;
+    g.alpha_g = w_gate->alpha;
+    g.alpha_u = w_up->alpha;
+    g.status = dev->status;
+    int ctas = 0;
+    if (glu_split(N, g.ld, g.C, dev->sm_count, &ctas, &g.rows_box)) {
+      g.rows_base = N / ctas;
+      g.rows_rem = N % ctas;
+      CUtensorMap mg, mu;
+      if (!make_map_u8(&mg, w_gate->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N),
+                       static_cast<uint64_t>(g.ld), 128, static_cast<uint32_t>(g.rows_box), 128) ||
+          !make_map_u8(&mu, w_up->codes, static_cast<uint64_t>(g.ld), static_cast<uint64_t>(N),
+                       static_cast<uint64_t>(g.ld), 128, static_cast<uint32_t>(g.rows_box), 128))
+        return BITLINEAR_ERR_CUDA;
+      st = launch(gemv_glu_kernel, dim3(ctas), dim3(kGemvThreads), gemv_glu_smem_bytes(g.rows_box, g.ld, g.C), s, pdl,
+                  mg, mu, g);
+      if (st == BITLINEAR_OK) t_last_kernel = "gemv_m1_relu2_glu";
+      return st;
+    }
+  }
+  // otherwise: the two BitLinears as one grouped call into the workspace, then h elementwise
+  const size_t yb = align256(static_cast<size_t>(M) * N * 2);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < 2 * yb) return BITLINEAR_ERR_WORKSPACE;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  uint16_t* ys[2] = {reinterpret_cast<uint16_t*>(wsb), reinterpret_cast<uint16_t*>(wsb + yb)};
+  const bitlinear_weights pair[2] = {*w_gate, *w_up};
+  st = forward_group(pair, 2, x, M, ys, nullptr, wsb + 2 * yb, workspace_bytes - 2 * yb, flags, stream);
+  if (st != BITLINEAR_OK) return st;
+  const size_t count = static_cast<size_t>(M) * N;
+  const bool vec = aligned16(h);  // the workspace halves are 256-byte aligned
+  const int blocks = static_cast<int>(std::min<size_t>(static_cast<size_t>(4 * dev->sm_count), (count / 8 + 255) / 256 + 1));
+  st = launch(relu2_glu_kernel, dim3(blocks), dim3(256), 0, s, true, ys[0], ys[1], h, count, vec);
+  if (st == BITLINEAR_OK) t_last_kernel = "relu2_glu";
+  return st;
 }
 
 size_t bitlinear_forward_q8_workspace_bytes(int32_t M, int32_t N, int32_t K) {

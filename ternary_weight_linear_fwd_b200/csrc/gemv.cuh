@@ -396,6 +396,151 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr] - qsum, s);
 }
 
+// ------------------------------------------------------------------ FFN gate/up with squared ReLU, M = 1
+// The FFN of BitNet b1.58 2B4T uses squared ReLU (2B4T report summary,
+// section 2, Architecture).  With the block's gate and up projections (two
+// BitLinears of one x, outputs g and u in bf16) the result is taken as
+//     h = RN_bf16(RN_bf16(max(g, 0)^2) * u)
+// elementwise; both products are exact in fp32 (8-bit significands), so each
+// step rounds once, as the bf16 operations would.
+__device__ __forceinline__ uint16_t relu2_glu_bf16(uint16_t gb, uint16_t ub) {
+  const float gv = __uint_as_float(static_cast<uint32_t>(gb) << 16);
+  const float r = gv > 0.0f ? gv : 0.0f;
+  const __nv_bfloat16 sq = __float2bfloat16_rn(__fmul_rn(r, r));
+  const __nv_bfloat16 h = __float2bfloat16_rn(
+      __fmul_rn(__bfloat162float(sq), __uint_as_float(static_cast<uint32_t>(ub) << 16)));
+  return *reinterpret_cast<const uint16_t*>(&h);
+}
+
+// One token: each CTA owns the same rows of both matrices.  Its stripes hold
+// the gate rows at lines 0.. and the up rows at lines rows_box.. (rows_box a
+// multiple of 8, so both boxes keep the 128-byte swizzle phase), and thread
+// (segment, p) contracts gate row p and up row p over its segment; the store
+// forms y_gate and y_up as the single-matrix GEMV would and writes h only.
+struct GemvGlu {
+  const float* alpha_g;
+  const float* alpha_u;
+  uint16_t* h;        // [N]
+  const uint16_t* x;  // one bf16 row [K]
+  int32_t* status;
+  int64_t ld;
+  int K, C, rows_box, rows_base, rows_rem;
+};
+
+__host__ __device__ __forceinline__ size_t gemv_glu_smem_bytes(int rows_box, int64_t ld, int C) {
+  return 1024 + static_cast<size_t>(gemv_stripes(ld)) * gemv_stripe_bytes(2 * rows_box) +
+         static_cast<size_t>(C) * 4 * 16 + 16 + static_cast<size_t>(2 * rows_box) * 4;
+}
+
+__global__ void __launch_bounds__(kGemvThreads) gemv_glu_kernel(const __grid_constant__ CUtensorMap map_g,
+                                                                const __grid_constant__ CUtensorMap map_u,
+                                                                const GemvGlu g) {
+  extern __shared__ uint8_t s_raw[];
+  __shared__ uint64_t s_bar;
+  __shared__ float s_red[32];
+  const int b = blockIdx.x;
+  const int r0 = b * g.rows_base + min(b, g.rows_rem);
+  const int nrows = g.rows_base + (b < g.rows_rem ? 1 : 0);
+  const int C = g.C;
+  const int rows_box = g.rows_box;
+  const int stripes = gemv_stripes(g.ld);
+  const int stripe_bytes = gemv_stripe_bytes(2 * rows_box);
+  uint8_t* s_w = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
+  uint4* s_act = reinterpret_cast<uint4*>(s_w + static_cast<size_t>(stripes) * stripe_bytes);
+  int32_t* s_qsum = reinterpret_cast<int32_t*>(s_act + 4 * C);
+  int32_t* s_acc = s_qsum + 4;  // [2 * rows_box]: gate rows, then up rows
+
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&map_g);
+    tma_prefetch_desc(&map_u);
+    mbar_arrive_expect_tx(&s_bar,
+                          static_cast<uint32_t>(stripes) * 256u * static_cast<uint32_t>(rows_box) + test_extra_tx());
+    const uint64_t pol = l2_policy_evict_first();
+    for (int st = 0; st < stripes; ++st) {
+      tma_load_2d_hint(s_w + st * stripe_bytes, &map_g, st * 128, r0, &s_bar, pol);
+      tma_load_2d_hint(s_w + st * stripe_bytes + rows_box * 128, &map_u, st * 128, r0, &s_bar, pol);
+    }
+  }
+  const float alpha_g = *g.alpha_g, alpha_u = *g.alpha_u;
+  for (int r = threadIdx.x; r < 2 * rows_box; r += blockDim.x) s_acc[r] = 0;
+  if (threadIdx.x == 0) *s_qsum = 0;
+  __syncthreads();
+
+  pdl_wait_primary();  // x may come from the preceding kernel
+  const float gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qsum, s_red);
+  pdl_launch_dependents();
+  const float sg = __fdiv_rn(__fmul_rn(alpha_g, gamma), kQb);
+  const float su = __fdiv_rn(__fmul_rn(alpha_u, gamma), kQb);
+  const bool landed = mbar_wait(&s_bar, 0);
+
+  if (landed && nrows > 0) {
+    // as gemv_dense_kernel, with the pair (gate row p, up row p): consecutive threads take consecutive
+    // rows of one segment, so a warp reads one activation chunk (broadcast) and conflict-free weight slots
+    const int nseg = blockDim.x / nrows;  // rows_box <= 128: at least 4 segments
+    const int seg = threadIdx.x / nrows, p = threadIdx.x - seg * nrows;
+    if (seg < nseg) {
+      const int c_beg = seg * C / nseg, c_end = (seg + 1) * C / nseg;
+      int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
+      for (int ch = c_beg; ch < c_end; ++ch) {
+        const uint4 wa = gemv_wchunk(s_w, stripe_bytes, p, ch);
+        const uint4 wb = gemv_wchunk(s_w, stripe_bytes, rows_box + p, ch);
+        const uint4 q0 = s_act[ch], q1 = s_act[C + ch], q2 = s_act[2 * C + ch], q3 = s_act[3 * C + ch];
+        dot_word(wa.x, q0.x, q0.y, q0.z, q0.w, a0, a1, a2, a3);
+        dot_word(wb.x, q0.x, q0.y, q0.z, q0.w, b0, b1, b2, b3);
+        dot_word(wa.y, q1.x, q1.y, q1.z, q1.w, a0, a1, a2, a3);
+        dot_word(wb.y, q1.x, q1.y, q1.z, q1.w, b0, b1, b2, b3);
+        dot_word(wa.z, q2.x, q2.y, q2.z, q2.w, a0, a1, a2, a3);
+        dot_word(wb.z, q2.x, q2.y, q2.z, q2.w, b0, b1, b2, b3);
+        dot_word(wa.w, q3.x, q3.y, q3.z, q3.w, a0, a1, a2, a3);
+        dot_word(wb.w, q3.x, q3.y, q3.z, q3.w, b0, b1, b2, b3);
+      }
+      if (c_end > c_beg) {
+        atomicAdd(&s_acc[p], a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6));
+        atomicAdd(&s_acc[rows_box + p], b0 + (b1 >> 2) + (b2 >> 4) + (b3 >> 6));
+      }
+    }
+  }
+  if (gemv_gave_up(landed, &s_bar, g.status)) return;
+  const int32_t qsum = *s_qsum;
+  for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) {
+    const __nv_bfloat16 yg = __float2bfloat16_rn(__fmul_rn(static_cast<float>(s_acc[rr] - qsum), sg));
+    const __nv_bfloat16 yu = __float2bfloat16_rn(__fmul_rn(static_cast<float>(s_acc[rows_box + rr] - qsum), su));
+    g.h[r0 + rr] = relu2_glu_bf16(*reinterpret_cast<const uint16_t*>(&yg), *reinterpret_cast<const uint16_t*>(&yu));
+  }
+}
+
+// Many tokens: h from the two BitLinear outputs (bf16 bits), 8 per thread and
+// step when the three arrays are 16-byte aligned.
+__global__ void __launch_bounds__(256) relu2_glu_kernel(const uint16_t* __restrict__ yg,
+                                                        const uint16_t* __restrict__ yu, uint16_t* __restrict__ h,
+                                                        size_t count, bool vec) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (vec) {
+    for (; 8 * i + 8 <= count; i += stride) {
+      const uint4 a = reinterpret_cast<const uint4*>(yg)[i], b = reinterpret_cast<const uint4*>(yu)[i];
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        o[j] = relu2_glu_bf16(static_cast<uint16_t>(aw[j]), static_cast<uint16_t>(bw[j])) |
+               (static_cast<uint32_t>(relu2_glu_bf16(static_cast<uint16_t>(aw[j] >> 16),
+                                                     static_cast<uint16_t>(bw[j] >> 16))) << 16);
+      reinterpret_cast<uint4*>(h)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    // the tail (count % 8 elements) by the first threads
+    const size_t tail0 = count / 8 * 8;
+    const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (tail0 + t < count) h[tail0 + t] = relu2_glu_bf16(yg[tail0 + t], yu[tail0 + t]);
+  } else {
+    for (; i < count; i += stride) h[i] = relu2_glu_bf16(yg[i], yu[i]);
+  }
+}
+
 // ------------------------------------------------------------------ dense M = 1, lookup tables
 // The TL2 lookup idea of bitnet.cpp ("BitNet 1-Bit LLM" blog, section "I2_S
 // kernel internals"): two consecutive ternary weights index a table of the

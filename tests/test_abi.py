@@ -254,3 +254,34 @@ def test_forward_q8_host_checks(L):
     assert f(ctypes.byref(w), q, 264, g, rs, 0, y, None, None, 0, 0, None) == 2   # M = 0
     assert f(ctypes.byref(w), q + 8, 256, g, rs, 4, y, None, None, 0, 0, None) == 3
     assert f(ctypes.byref(w), q, 256, g, rs, 4, y, None, None, 0, 0x2, None) == 8  # no GEMV path
+
+
+def test_relu2_glu_host_checks(L):
+    """Gate/up with squared ReLU: argument errors come back before any device work (fake addresses)."""
+    f = L.bitlinear_forward_relu2_glu
+    f.restype = ctypes.c_int
+    x, h = 0x30000, 0x40000
+    wg, wu = _w(L), _w(L)
+    assert f(None, ctypes.byref(wu), x, 1, h, None, 0, 0, None) == 1
+    assert f(ctypes.byref(wg), None, x, 1, h, None, 0, 0, None) == 1
+    assert f(ctypes.byref(wg), ctypes.byref(wu), None, 1, h, None, 0, 0, None) == 1
+    assert f(ctypes.byref(wg), ctypes.byref(wu), x, 1, None, None, 0, 0, None) == 1
+    other_n = _w(L, N=96)
+    assert f(ctypes.byref(wg), ctypes.byref(other_n), x, 1, h, None, 0, 0, None) == 2   # N differs
+    other_k = _w(L, K=512)
+    assert f(ctypes.byref(wg), ctypes.byref(other_k), x, 1, h, None, 0, 0, None) == 2   # K differs
+    assert f(ctypes.byref(wg), ctypes.byref(wu), x, 0, h, None, 0, 0, None) == 2        # M = 0
+    assert f(ctypes.byref(wg), ctypes.byref(wu), x + 8, 1, h, None, 0, 0, None) == 3    # x not 16-byte aligned
+    bad_p = _w(L, n=3, m=4, meta=0x50000)
+    assert f(ctypes.byref(wg), ctypes.byref(bad_p), x, 1, h, None, 0, 0, None) == 4
+    assert f(ctypes.byref(wg), ctypes.byref(wu), x, 1, h, None, 0, 0x100, None) == 8    # unknown flag
+    assert f(ctypes.byref(wg), ctypes.byref(wu), x, 1, h, None, 0, 0x8, None) == 8      # no lookup-table path
+
+
+def test_relu2_glu_workspace_bytes(L):
+    q = L.bitlinear_forward_relu2_glu_workspace_bytes
+    q.restype = ctypes.c_size_t
+    q.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_uint32]
+    assert q(0, 64, 256, 0) == 0
+    for M, N, K in ((1, 6912, 2560), (2048, 6912, 2560), (300, 2000, 1032)):
+        assert q(M, N, K, 0) >= 2 * M * N * 2 + L.bitlinear_forward_workspace_bytes(M, N, K, 0)

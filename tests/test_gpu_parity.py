@@ -703,3 +703,53 @@ def test_forward_norm(n, m, M, K, N):
 def test_status_word_clean():
     torch.cuda.synchronize()
     assert bl.device_status(clear=False) == 0
+
+
+# ---------------------------------------------------------------- FFN gate/up with squared ReLU
+
+def _check_relu2_glu(x, cases, wg, wu, xd, h, rows):
+    """h against the oracle: exactly the oracle's squared-ReLU product of the device's own g and u (each
+    the BitLinear output, identical to bitlinear_forward), and exactly the oracle's h wherever the device's
+    g and u equal the oracle's (elsewhere they differ by the documented bf16 ulp of the rescale)."""
+    (Wg, ag), (Wu, au) = cases
+    fwd = lambda w: bl.forward_nm(w, xd) if w.nm_m else bl.forward(w, xd)  # noqa: E731
+    yg, yu = bf16_bits(fwd(wg))[rows], bf16_bits(fwd(wu))[rows]
+    hb = bf16_bits(h)[rows]
+    np.testing.assert_array_equal(hb, oracle.relu2_glu(yg, yu))
+    ygo, yuo = oracle.forward(x[rows], Wg, ag)[0], oracle.forward(x[rows], Wu, au)[0]
+    assert_bf16_close(yg, ygo)
+    assert_bf16_close(yu, yuo)
+    same = (yg == ygo) & (yu == yuo)
+    np.testing.assert_array_equal(hb[same], oracle.relu2_glu(ygo, yuo)[same])
+
+
+@pytest.mark.parametrize("M,K,N,flags,kernel", [
+    (1, 2560, 6912, 0, "gemv_m1_relu2_glu"), (1, 6912, 2560, 0, "gemv_m1_relu2_glu"),
+    (1, 1032, 37, 0, "gemv_m1_relu2_glu"), (1, 200, 333, 0, "gemv_m1_relu2_glu"),
+    (1, 2560, 6912, 0x4, "relu2_glu"), (5, 1032, 300, 0, "relu2_glu"), (70, 2560, 640, 0, "relu2_glu"),
+    (300, 2048, 2000, 0, "relu2_glu")])
+def test_forward_relu2_glu(M, K, N, flags, kernel):
+    x, Wg, ag, wg = _dense_case(M, K, N, seed=M + K + N)
+    _, Wu, au, wu = _dense_case(M, K, N, seed=M + K + N + 1)
+    xd = to_dev_bf16(x)
+    h = bl.forward_relu2_glu(wg, wu, xd, flags=flags)
+    assert bl.last_kernel() == kernel, bl.last_kernel()
+    assert torch.equal(h.view(torch.int16), bl.forward_relu2_glu(wg, wu, xd, flags=flags).view(torch.int16))
+    _check_relu2_glu(x, [(Wg, ag), (Wu, au)], wg, wu, xd, h, np.arange(M))
+
+
+def test_forward_relu2_glu_nm_and_prefill_sampled():
+    """6:8 weights at one token (grouped N:M GEMVs, then h), and the 2B4T gate/up at M = 2048 on sampled
+    tokens (pair GEMMs, then h)."""
+    x, Wg, ag, wg = _nm_case(1, 2048, 1000, 6, 8, seed=21)
+    _, Wu, au, wu = _nm_case(1, 2048, 1000, 6, 8, seed=22)
+    xd = to_dev_bf16(x)
+    h = bl.forward_relu2_glu(wg, wu, xd)
+    _check_relu2_glu(x, [(Wg, ag), (Wu, au)], wg, wu, xd, h, np.arange(1))
+    M, K, N = 2048, 2560, 6912
+    x, Wg, ag, wg = _dense_case(M, K, N, seed=31, ternary=True)
+    _, Wu, au, wu = _dense_case(M, K, N, seed=32, ternary=True)
+    xd = to_dev_bf16(x)
+    h = bl.forward_relu2_glu(wg, wu, xd)
+    rows = np.unique(np.concatenate([[0, 127, 128, M - 1], synth.splitmix64(M, 5, 10) % M])).astype(np.int64)
+    _check_relu2_glu(x, [(Wg, ag), (Wu, au)], wg, wu, xd, h, rows)
