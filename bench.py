@@ -372,6 +372,29 @@ def run_decode(dev, steps, warmup, layers, clock_index):
             "e2e_eager_gbps": decode_step_bytes(layers) * eager_steps / eager_secs / 1e9}
 
 
+def run_ffn_glu(dev, layers: int, steps: int = 200, warmup: int = 5):
+    """The decode FFN stack with its own dataflow: per layer h = ReLU(gate x)^2 * (up x) in one launch
+    (bitlinear_forward_relu2_glu at M = 1), then down(h) reading that h; one CUDA graph with PDL edges.
+    Same weight bytes per step as the headline decode step."""
+    import torch
+
+    import ternary_weight_linear_fwd_b200 as bl
+
+    layers_w, x_in, h_in, y_gate, y_up, y_down = build_decode(dev, layers)
+    h = torch.empty((layers, 6912), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        for l, w in enumerate(layers_w):
+            bl.forward_relu2_glu(w["gate"], w["up"], x_in[l:l + 1], out=h[l:l + 1], flags=bl.FLAG_PDL)
+            bl.forward(w["down"], h[l:l + 1], out=y_down[l:l + 1], flags=bl.FLAG_PDL)
+
+    secs = time_chain_graph(dev, [step], warmup, steps)
+    kern = bl.last_kernel()
+    step_bytes = decode_step_bytes(layers) - layers * 6912 * 2  # one FFN intermediate instead of two outputs
+    return {"us_per_step": secs * 1e6, "GBps": step_bytes / secs / 1e9, "launches_per_step": 2 * layers,
+            "kernels": ["gemv_m1_relu2_glu", kern]}
+
+
 def run_prefill(dev, iters: int, warmup: int):
     """Per shape: forward at M = 2048, timed on the device two ways: over rotating copies of x and of
     the weights (working set > 2 x L2; the reported figure), and with an L2 flush (256 MB write)
@@ -1082,8 +1105,9 @@ def main():
 
     pre = run_prefill(dev, args.prefill_iters, 3)
     iso = run_isolated(dev)
-    sweep = nm = norm = lut = hbit = None
+    sweep = nm = norm = lut = hbit = ffn = None
     if not args.no_sweep:
+        ffn = run_ffn_glu(dev, args.layers)
         sweep = run_sweep(dev)
         nm = run_nm(dev)
         norm = run_norm(dev)
@@ -1163,6 +1187,10 @@ def main():
                                   "M=4096: 16 calls); "
                                   "bytes = packed values + metadata + 4 + 2MK + 2MN; TOPS counts dense-equivalent "
                                   "2MNK", "cases": nm}
+        line["ffn_glu"] = {"workload": f"decode FFN stack with its dataflow, {args.layers} layers at M=1: "
+                                       "h = ReLU(gate x)^2 * (up x) in one launch (bitlinear_forward_relu2_glu), "
+                                       "then down(h); one CUDA graph with PDL edges; bytes = the decode step's "
+                                       "weights + x + h + y", **ffn}
         line["norm"] = {"workload": "RMSNorm (fp32 weight, eps 1e-5) fused into the activation quantisation, "
                                     "2B4T gate 2560->6912, ternary P(0)=0.42; PDL-chained graphs of 16 calls; "
                                     "rmsnorm_quant_act bytes = 2MK (x) + MK (q) + 4K (g) + 8M; forward_norm vs "
