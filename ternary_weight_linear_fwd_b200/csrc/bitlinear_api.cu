@@ -587,7 +587,8 @@ int t2_pick_bn(int nm, int row_tiles, int M, int K, const int pairs[4]) {
   return best;
 }
 
-// The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split.
+// The pair GEMM (gemm_tc2.cuh) for a plan of 128-token tiles without a K split
+// (the pair kernel then picks its own token tile, 128 to 224).
 // DEVICE: no pair fits at once.  (Dense token tiles of 96 and 64 were measured
 // too: a k-block's cost is mostly per instruction and per hand-off, so a
 // narrower tile did less work in nearly the same time.)

@@ -6,14 +6,15 @@
 // kernel that skipped both the MMAs and the unpacking still took four fifths
 // of the full kernel's time (2048 -> 11008 at M = 4096).  Here two CTAs of a
 // cluster share one MMA of M = 256 weight rows: each CTA holds its own 128
-// weight rows (expanded codes in its TMEM for dense weights, the compressed
-// kept values in its shared memory for 2:4 weights) and HALF of the BN
-// tokens' activation tile, so the activation bytes per MAC halve.
+// weight rows (expanded codes in its TMEM or shared memory for dense and n:8
+// weights, the compressed kept values in its shared memory for 2:4 weights)
+// and HALF of the BN tokens' activation tile, so the activation bytes per MAC
+// halve.
 //
 //   D[256 rows, BN tokens] += A[256 rows, K] * B[BN tokens, K]^T
 //   CTA r of the pair: rows 128 r .. 128 r + 127 of A and D (its own TMEM),
 //                      tokens BN/2 r .. BN/2 r + BN/2 - 1 of B (its own shared memory).
-// Token tiles: BN = 128, 192 or 224, picked on the host by how many rounds of
+// Token tiles: BN = 128, 160, 192 or 224, picked on the host by how many rounds of
 // pairs a shape takes.  Narrower tiles did less work per k-block in nearly the
 // same time (the k-block's cost is mostly per MMA instruction and per
 // hand-off).  Dense weights at BN = 128 keep their expanded codes in TMEM
