@@ -207,6 +207,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int KB = a.kbs;
+  // dense codes into TMEM (A from TMEM): both unpack groups take every k-block, group g the half of its
+  // 512 k in subs 2g, 2g + 1, so a slot is refilled in half the time after its release
+  constexpr bool kSplit = !SP && !C::OPS && !C::N8;
   const int nunits = a.row_tiles * a.tok_tiles;
   const int my_tiles = pair < nunits ? (nunits - 1 - pair) / npairs + 1 : 0;
   const int total_kb = my_tiles * KB;
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int j = 0; j < R; ++j) mbar_init(&aready[j], 8);
+    for (int j = 0; j < R; ++j) mbar_init(&aready[j], kSplit ? 16 : 8);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 8);
@@ -363,15 +366,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp >= 4 && warp < kTcEpiWarp0) {
     // -------------------------------------------------------------- unpack (both CTAs)
-    // group g takes the k-blocks of parity g: with S and R even, every use of
-    // its copy stages and operand slots, so no parity wait skips a phase.  The
-    // operand slot of k-block i is free once the MMAs of k-block i - R have
-    // completed: the commit that frees copy stage (i - R) % S says so.
+    // Group g takes the k-blocks of parity g (with kSplit: every k-block, its
+    // half of the k): with S and R even it sees every use of its copy stages
+    // and operand slots, so no parity wait skips a phase.  The operand slot of
+    // k-block i is free once the MMAs of k-block i - R have completed: the
+    // commit that frees copy stage (i - R) % S says so.
     const int grp = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    for (int i = grp; i < total_kb; i += 2) {
+    for (int i = kSplit ? 0 : grp; i < total_kb; i += kSplit ? 1 : 2) {
       const int s = i % S, j = i % R;
       if (!mbar_wait(&full[s], (i / S) & 1) || (i >= R && !mbar_wait(&empty[(i - R) % S], ((i - R) / S) & 1))) {
         *a.status = kDevTimeoutUnpack;
@@ -437,7 +441,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         static_assert(SP || C::OPS || C::N8 || 32 * KSUB == 128, "one swizzle row of packed codes per weight row");
         const uint8_t* arow = st + r * 128;
 #pragma unroll
-        for (int sub = 0; sub < KSUB; ++sub) {
+        for (int hs = 0; hs < (kSplit ? KSUB / 2 : KSUB); ++hs) {
+          const int sub = kSplit ? grp * (KSUB / 2) + hs : hs;
           const uint4 lo = *reinterpret_cast<const uint4*>(arow + (((2 * sub) ^ (r & 7)) << 4));
           const uint4 hi = *reinterpret_cast<const uint4*>(arow + (((2 * sub + 1) ^ (r & 7)) << 4));
           const uint32_t dw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
