@@ -1513,4 +1513,17 @@ extern "C" bitlinear_status bitlinear_test_set_wait_fault(uint64_t wait_limit_ns
     return BITLINEAR_ERR_CUDA;
   return cudaDeviceSynchronize() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
+
+extern "C" int32_t bitlinear_test_timeline(uint64_t* records, int32_t max_records) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  uint32_t seq = 0;
+  if (cudaMemcpyFromSymbol(&seq, g_timeline_seq, sizeof seq) != cudaSuccess) return -1;
+  const int32_t n = static_cast<int32_t>(std::min<uint32_t>(seq, static_cast<uint32_t>(kTlSlots)));
+  if (records && max_records > 0 &&
+      cudaMemcpyFromSymbol(records, g_timeline, sizeof(uint64_t) * kTlWords * std::min(n, max_records)) != cudaSuccess)
+    return -1;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_timeline_seq, &zero, sizeof zero) != cudaSuccess) return -1;
+  return static_cast<int32_t>(seq);
+}
 #endif

@@ -161,7 +161,8 @@ struct T2 {
   static constexpr int DCOLS = BN > 128 ? 256 : BN;  // accumulator 1's first column (256 for wide tiles)
   static constexpr int R = SP ? 4 : OPS ? 2 : (512 - 2 * BN) / SLOT;  // operand slots (TMEM: as it holds)
   // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
-  static constexpr int FIXED = 2 * BN * 8 + 256 + (N8 ? 1024 : 0);  // scales, code sums, barriers (n:8: selectors)
+  // scales, code sums, barriers (n:8: selectors; test builds: the phase stamps)
+  static constexpr int FIXED = 2 * BN * 8 + 256 + (N8 ? 1024 : 0) + (kTimeline ? 64 : 0);
   static constexpr int S = tc_min3(kTcMaxStages, (kTcSmemMax - FIXED - R * OPA) / STAGE, 64) & ~1;  // even
   static constexpr int SMEM = FIXED + S * STAGE + R * OPA;
   static constexpr int A_COL0 = DCOLS + BN;         // operand slots after accumulator 1
@@ -182,6 +183,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int KSUB = C::KSUB;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint64_t t_entry = tl_now();
   // both CTAs see the same offset, so both leave here together (before any cluster barrier)
   if ((smem_u32(smem_raw) & 1023u) != 0u) {
     if (threadIdx.x == 0) *a.status = kDevBadSmemAlign;
@@ -202,6 +204,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   // n:8: byte-permute selectors of the 256 masks, after the 256 bytes of barriers
   uint32_t* s_sel = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(s_rowsum + 2 * BN) + 256);
+  // test builds: phase stamps (0 entry, 1 set-up done, 2 producer past the dependency wait, 3 first stage
+  // landed, 4 first tile's MMAs issued, 5 first accumulator ready, 6 last epilogue done, 7 end)
+  uint64_t* s_tl = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(s_rowsum + 2 * BN) + 256 +
+                                               (C::N8 ? 1024 : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -244,9 +250,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   if (C::N8)
     for (int m = threadIdx.x; m < 256; m += blockDim.x) s_sel[m] = n8_perm_selectors(static_cast<uint32_t>(m));
+  if (kTimeline && threadIdx.x < 8) s_tl[threadIdx.x] = threadIdx.x == 0 ? t_entry : 0ull;
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrive or multicast commit
   tc_fence_after();
+  if (kTimeline && threadIdx.x == 0) s_tl[1] = tl_now();
   const uint32_t tmem = *tmem_slot;
   const uint32_t aready0 = mapa_shared(smem_u32(aready), 0);
   const uint32_t accempty0 = mapa_shared(smem_u32(accempty), 0);
@@ -280,6 +288,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         load_a(rt, i % KB, i);
       }
       pdl_wait_primary();
+      if (kTimeline) s_tl[2] = tl_now();
       for (int i = 0; i < pre; ++i) {
         int rt, tt;
         unit_of(i / KB, rt, tt);
@@ -358,6 +367,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           issued = true;
         }
         if (ok) tc_commit_pair_mc(&accfull[buf], 0x3);
+        if (kTimeline && t == 0) s_tl[4] = tl_now();
       }
       if (!ok && issued) {
         tc_commit_pair(drain);
@@ -381,6 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *a.status = kDevTimeoutUnpack;
         break;
       }
+      if (kTimeline && i == 0 && warp == 4 && lane == 0) s_tl[3] = tl_now();
       const uint8_t* st = sStage + s * C::STAGE + C::B_STAGE;
       if (SP) {
         const uint4* vp = reinterpret_cast<const uint4*>(st + r * 32);
@@ -481,6 +492,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *a.status = kDevTimeoutEpilogue;
         break;
       }
+      if (kTimeline && t == 0 && q == 0 && lane == 0) s_tl[5] = tl_now();
       tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -492,10 +504,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote_cta(accempty0 + static_cast<uint32_t>(buf * 8));
+      if (kTimeline && q == 0 && lane == 0) s_tl[6] = tl_now();
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (kTimeline && threadIdx.x == 0) {
+    uint64_t t8[8];
+    for (int i = 0; i < 7; ++i) t8[i] = s_tl[i];
+    t8[7] = tl_now();
+    tl_commit(2, (static_cast<uint64_t>(a.M) << 32) | (static_cast<uint64_t>(blockIdx.x) << 16) | gridDim.x, t8);
+  }
   cluster_sync_all();  // no remote arrive or multicast commit is left in flight towards either CTA
   if (warp == 2) {
     tc_fence_after();

@@ -304,6 +304,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   extern __shared__ uint8_t s_raw[];
   __shared__ uint64_t s_bar;
   __shared__ float s_red[32];
+  // test builds: phase stamps of thread 0 (0 entry, 1 past the dependency wait, 2 x quantised, 3 weights
+  // landed, 4 contracted, 5 stored)
+  uint64_t tl[8] = {tl_now(), 0ull, 0ull, 0ull, 0ull, 0ull, 0ull, 0ull};
   int mi = 0;
 #pragma unroll
   for (int i = 1; i < kGemvGroup; ++i)
@@ -347,16 +350,19 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   __syncthreads();
 
   pdl_wait_primary();  // x may come from the preceding kernel
+  if (kTimeline) tl[1] = tl_now();
   float gamma;
   if (kNorm)
     gamma = quantise_row_smem_norm(g.x, g.K, 4 * C, s_act, s_qsum, s_red, s_redd, s_g, g.eps);
   else
     gamma = quantise_row_smem(g.x, g.K, 4 * C, s_act, s_qsum, s_red);
+  if (kTimeline) tl[2] = tl_now();
   // The next kernel may start now: its weight copies then stream while this
   // one contracts, and no longer delay this kernel's read of x.
   pdl_launch_dependents();
   const float s = __fdiv_rn(__fmul_rn(alpha, gamma), kQb);
   const bool landed = mbar_wait(&s_bar, 0);
+  if (kTimeline) tl[3] = tl_now();
 
   if (landed) {
     // Thread (seg, p) takes row pair p (rows p and p + half) over the chunks of
@@ -392,8 +398,13 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
     }
   }
   if (gemv_gave_up(landed, &s_bar, g.status)) return;
+  if (kTimeline) tl[4] = tl_now();
   const int32_t qsum = *s_qsum;
   for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr] - qsum, s);
+  if (kTimeline && threadIdx.x == 0) {
+    tl[5] = tl_now();
+    tl_commit(1, (static_cast<uint64_t>(g.K) << 32) | (static_cast<uint64_t>(blockIdx.x) << 16) | gridDim.x, tl);
+  }
 }
 
 // ------------------------------------------------------------------ FFN gate/up with squared ReLU, M = 1

@@ -45,6 +45,32 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Phase timeline (test builds only): a CTA stamps %globaltimer at the borders
+// of its phases into a local array and appends one record of kTlWords words
+// (kind, a word of launch facts, then the stamps) to a ring in global memory
+// at its end; the host reads the ring.  In the product library every stamp
+// and the record compile to nothing.
+constexpr int kTlWords = 10;
+constexpr int kTlSlots = 1 << 17;
+#ifdef BITLINEAR_TEST_HOOKS
+constexpr bool kTimeline = true;
+__device__ uint64_t g_timeline[kTlSlots * kTlWords];
+__device__ uint32_t g_timeline_seq;
+__device__ __forceinline__ uint64_t tl_now() { return globaltimer_ns(); }
+__device__ __forceinline__ void tl_commit(uint64_t kind, uint64_t facts, const uint64_t (&t)[8]) {
+  const uint32_t slot = atomicAdd(&g_timeline_seq, 1u) & static_cast<uint32_t>(kTlSlots - 1);
+  uint64_t* o = g_timeline + static_cast<size_t>(slot) * kTlWords;
+  o[0] = kind;
+  o[1] = facts;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[2 + i] = t[i];
+}
+#else
+constexpr bool kTimeline = false;
+__device__ __forceinline__ uint64_t tl_now() { return 0ull; }
+__device__ __forceinline__ void tl_commit(uint64_t, uint64_t, const uint64_t (&)[8]) {}
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

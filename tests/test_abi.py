@@ -46,7 +46,7 @@ def test_headers_cover_every_header_file():
 def test_test_hooks_only_in_the_test_build(L):
     """The test build exports the product ABI plus the hooks; the product library has no hook."""
     hooks = _declared(HOOKS_HEADER)
-    assert hooks == ["bitlinear_test_set_wait_fault"]
+    assert hooks == ["bitlinear_test_set_wait_fault", "bitlinear_test_timeline"]
     T = ctypes.CDLL(blbuild.build_test_hooks())
     for n in _declared() + hooks:
         assert hasattr(T, n), n
