@@ -5,7 +5,7 @@
  * export them.  The pages have no counterpart: the first serves the
  * failure-handling convention of bitlinear.h (a kernel that gives up on a
  * bounded wait writes a code to the device status word instead of trapping),
- * the second reads the phase stamps this build's kernels record
+ * the second reads the phase stamps the test build's kernels record
  * (python -m ternary_weight_linear_fwd_b200.timeline prints them).
  */
 #ifndef BITLINEAR_TEST_HOOKS_H_

@@ -13,7 +13,7 @@ Builds ``libbitlinear_testhooks.so`` (the product sources with
 
 reads every CTA's record and prints one JSON object: per launch kind, the
 median over launches of each phase (ns).  The stamps, the ring writes and
-the extra registers make this build a little slower than the product one; the
+the extra registers make the test build a little slower than the product one; the
 phase split, not the absolute time, is what it is for.
 """
 from __future__ import annotations
