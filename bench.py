@@ -182,14 +182,20 @@ GEMV_DEFS = ("gemv_dense_kernel", "quantise_row_smem", "quantise_row_smem_norm",
              "gemv_row_totals")
 
 
+# Lines of the test build's phase stamps: compiled out of the product library, so not part of the
+# fingerprint of the code the measured kernel runs.
+TIMELINE_MARKS = ("tl_now", "tl_commit", "kTimeline")
+
+
 def gemv_source_hash() -> str:
     """Fingerprint of the text of the definitions in GEMV_DEFS: a top-level definition runs from
-    its first line to the next line that is a lone closing brace."""
+    its first line to the next line that is a lone closing brace (lines of the test build's phase
+    stamps left out)."""
     import re
     h = hashlib.sha256()
     for n in GEMV_SOURCES:
         with open(os.path.join(ROOT, "ternary_weight_linear_fwd_b200", "csrc", n)) as f:
-            lines = f.read().split("\n")
+            lines = [ln for ln in f.read().split("\n") if not any(m in ln for m in TIMELINE_MARKS)]
         i = 0
         while i < len(lines):
             line = lines[i]

@@ -304,9 +304,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   extern __shared__ uint8_t s_raw[];
   __shared__ uint64_t s_bar;
   __shared__ float s_red[32];
-  // test builds: phase stamps of thread 0 (0 entry, 1 past the dependency wait, 2 x quantised, 3 weights
-  // landed, 4 contracted, 5 stored)
-  uint64_t tl[8] = {tl_now(), 0ull, 0ull, 0ull, 0ull, 0ull, 0ull, 0ull};
+  uint64_t tl[8] = {tl_now(), 0ull, 0ull, 0ull, 0ull, 0ull, 0ull, 0ull};  // test-build phase stamps (tl_now)
   int mi = 0;
 #pragma unroll
   for (int i = 1; i < kGemvGroup; ++i)
@@ -401,10 +399,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_dense_kernel(const __grid_c
   if (kTimeline) tl[4] = tl_now();
   const int32_t qsum = *s_qsum;
   for (int rr = threadIdx.x; rr < nrows; rr += blockDim.x) gemv_store(mt.y, mt.acc, r0 + rr, s_acc[rr] - qsum, s);
-  if (kTimeline && threadIdx.x == 0) {
-    tl[5] = tl_now();
-    tl_commit(1, (static_cast<uint64_t>(g.K) << 32) | (static_cast<uint64_t>(blockIdx.x) << 16) | gridDim.x, tl);
-  }
+  if (kTimeline && threadIdx.x == 0) tl_commit_now(1, (static_cast<uint64_t>(g.K) << 32) | (blockIdx.x << 16) | gridDim.x, tl, 5);
 }
 
 // ------------------------------------------------------------------ FFN gate/up with squared ReLU, M = 1

@@ -70,6 +70,11 @@ constexpr bool kTimeline = false;
 __device__ __forceinline__ uint64_t tl_now() { return 0ull; }
 __device__ __forceinline__ void tl_commit(uint64_t, uint64_t, const uint64_t (&)[8]) {}
 #endif
+// tl_commit after stamping t[i] with the present time (the last phase of a CTA).
+__device__ __forceinline__ void tl_commit_now(uint64_t kind, uint64_t facts, uint64_t (&t)[8], int i) {
+  t[i] = tl_now();
+  tl_commit(kind, facts, t);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
