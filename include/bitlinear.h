@@ -342,8 +342,9 @@ bitlinear_status bitlinear_forward_group(const bitlinear_weights* w, int32_t cou
  * workspace: device scratch of at least
  * bitlinear_forward_relu2_glu_workspace_bytes(M, N, K, flags) bytes, 16-byte
  * aligned (g and u for M > 1, then the forward's own workspace); may be NULL
- * when M = 1, both matrices are dense and BITLINEAR_FLAG_PATH_TC is not set:
- * then one launch computes both BitLinears and h.  Otherwise the pair runs as
+ * when M = 1, both matrices are dense, K <= 22528 (the rows of both matrices
+ * fit one CTA's shared memory) and BITLINEAR_FLAG_PATH_TC is not set: then one
+ * launch computes both BitLinears and h.  Otherwise the pair runs as
  * bitlinear_forward_group into the workspace and h is formed by one more
  * launch.  flags: as bitlinear_forward (BITLINEAR_FLAG_DECODE_LUT rejected).
  * Errors: NULL, SHAPE (N or K differ, M out of range), ALIGN, FLAGS,
