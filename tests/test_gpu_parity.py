@@ -726,7 +726,8 @@ def _check_relu2_glu(x, cases, wg, wu, xd, h, rows):
 @pytest.mark.parametrize("M,K,N,flags,kernel", [
     (1, 2560, 6912, 0, "gemv_m1_relu2_glu"), (1, 6912, 2560, 0, "gemv_m1_relu2_glu"),
     (1, 1032, 37, 0, "gemv_m1_relu2_glu"), (1, 200, 333, 0, "gemv_m1_relu2_glu"),
-    (1, 2560, 6912, 0x4, "relu2_glu"), (5, 1032, 300, 0, "relu2_glu"), (70, 2560, 640, 0, "relu2_glu"),
+    (1, 2560, 6912, 0x4, "relu2_glu"), (1, 24576, 130, 0, "relu2_glu"),  # K past the one-launch kernel
+    (5, 1032, 300, 0, "relu2_glu"), (70, 2560, 640, 0, "relu2_glu"),
     (300, 2048, 2000, 0, "relu2_glu")])
 def test_forward_relu2_glu(M, K, N, flags, kernel):
     x, Wg, ag, wg = _dense_case(M, K, N, seed=M + K + N)
